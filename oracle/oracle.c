@@ -1,0 +1,430 @@
+/*
+ * oracle.c -- plain CPU float64 oracle of the windowed atom attention block.
+ *
+ * TEST INFRASTRUCTURE: see oracle.h. Straight loops in the order the pages state
+ * the steps; no blocking, fusion or reordering. Every step cites its passage:
+ *   [WAA n] = "Local atom attention, encoder pooling and decoder skip/readout",
+ *             Required behavior, bullet n;
+ *   [AF3 RB] / [ESM RB] = "AlphaFold 3 / ESMFold 2 Atom Attention Encoder",
+ *             Required behavior.
+ */
+#include "oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* sigmoid(z) = 1 / (1 + e^-z); SiLU(z) = z * sigmoid(z)  [ESM RB, last-but-one item].
+ * For z < 0 the same value is formed as e^z / (1 + e^z), so that a representable
+ * subnormal tail is kept rather than flushed through an overflowing e^-z  [WAA 23] */
+double orc_sigmoid(double z) {
+  if (z >= 0.0) return 1.0 / (1.0 + exp(-z));
+  double e = exp(z);
+  return e / (1.0 + e);
+}
+double orc_silu(double z) { return z * orc_sigmoid(z); }
+
+/* Population LayerNorm without affine, eps inside the root  [WAA 7] */
+void orc_layer_norm(const double *v, int64_t n, double eps, double *out) {
+  double mean = 0.0, var = 0.0;
+  for (int64_t i = 0; i < n; ++i) mean += v[i];
+  mean /= (double)n;
+  for (int64_t i = 0; i < n; ++i) var += (v[i] - mean) * (v[i] - mean);
+  var /= (double)n;
+  double inv = 1.0 / sqrt(var + eps);
+  for (int64_t i = 0; i < n; ++i) out[i] = (v[i] - mean) * inv;
+}
+
+/* RMS(z) = z / sqrt(mean(z^2) + eps), no affine  [WAA 12] */
+void orc_rms_norm(const double *v, int64_t n, double eps, double *out) {
+  double ms = 0.0;
+  for (int64_t i = 0; i < n; ++i) ms += v[i] * v[i];
+  ms /= (double)n;
+  double inv = 1.0 / sqrt(ms + eps);
+  for (int64_t i = 0; i < n; ++i) out[i] = v[i] * inv;
+}
+
+/* q * cos + rotate_half(q) * sin, rotate_half([q1, q2]) = [-q2, q1]  [WAA 13] */
+void orc_rope_half_split(const double *q, const double *cosv, const double *sinv,
+                         int64_t D, double *out) {
+  int64_t h = D / 2;
+  for (int64_t d = 0; d < D; ++d) {
+    double rot = (d < h) ? -q[d + h] : q[d - h];
+    out[d] = q[d] * cosv[d] + rot * sinv[d];
+  }
+}
+
+/* Stabilised masked softmax; a row with no permitted entry is all zero  [WAA 15] */
+void orc_masked_softmax(const double *logits, const uint8_t *permitted, int64_t K,
+                        double *out) {
+  int any = 0;
+  double mx = 0.0;
+  for (int64_t k = 0; k < K; ++k) {
+    if (!permitted[k]) continue;
+    if (!any || logits[k] > mx) mx = logits[k];
+    any = 1;
+  }
+  double sum = 0.0;
+  for (int64_t k = 0; k < K; ++k) {
+    out[k] = permitted[k] ? exp(logits[k] - mx) : 0.0;
+    sum += out[k];
+  }
+  if (any)
+    for (int64_t k = 0; k < K; ++k) out[k] /= sum;
+}
+
+/* usable iff valid, 0 <= atom_to_token < T, and the mapped token is valid  [WAA 2] */
+void orc_usable(const orc_dims *d, const orc_inputs *in, uint8_t *usable) {
+  for (int64_t b = 0; b < d->B; ++b)
+    for (int64_t a = 0; a < d->A; ++a) {
+      int64_t i = b * d->A + a;
+      int64_t t = in->atom_to_token[i];
+      usable[i] = in->valid[i] && t >= 0 && t < d->T && in->token_valid[b * d->T + t];
+    }
+}
+
+/* A slot is permitted iff 0 <= key id < A, query and key usable, window_mask,
+ * and |key - query| <= radius when radius >= 0; ids are within one batch
+ * element  [WAA 4, WAA 5] */
+void orc_permitted(const orc_dims *d, const orc_inputs *in, const uint8_t *usable,
+                   int64_t radius, uint8_t *permitted) {
+  for (int64_t b = 0; b < d->B; ++b)
+    for (int64_t a = 0; a < d->A; ++a)
+      for (int64_t k = 0; k < d->K; ++k) {
+        int64_t s = (b * d->A + a) * d->K + k;
+        int64_t j = in->key_index[s];
+        int ok = j >= 0 && j < d->A;
+        ok = ok && usable[b * d->A + a] && usable[b * d->A + j];
+        ok = ok && in->window_mask[s];
+        if (ok && radius >= 0) {
+          int64_t diff = j - a;
+          if (diff < 0) diff = -diff;
+          ok = diff <= radius;
+        }
+        permitted[s] = (uint8_t)ok;
+      }
+}
+
+/* y[n_out] = x[n_in] @ W[n_in, n_out] (+ bias if given) */
+static void vecmat(const double *x, const double *W, const double *bias, int64_t n_in,
+                   int64_t n_out, double *y) {
+  for (int64_t o = 0; o < n_out; ++o) y[o] = bias ? bias[o] : 0.0;
+  for (int64_t i = 0; i < n_in; ++i) {
+    double xi = x[i];
+    const double *row = W + i * n_out;
+    for (int64_t o = 0; o < n_out; ++o) y[o] += xi * row[o];
+  }
+}
+
+typedef struct {
+  double *buf[16];
+  int n;
+} arena;
+
+static double *grab(arena *ar, int64_t n) {
+  double *p = (double *)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+  if (p) ar->buf[ar->n++] = p;
+  return p;
+}
+
+static void arena_free(arena *ar) {
+  for (int i = 0; i < ar->n; ++i) free(ar->buf[i]);
+  ar->n = 0;
+}
+
+int orc_forward(int style, int stage, const orc_dims *d, const orc_inputs *in,
+                const orc_params *p, double eps, int64_t radius,
+                const uint8_t *query_select, orc_outputs *out) {
+  if (style != ORC_STYLE_AF3 && style != ORC_STYLE_ESMFOLD2) return ORC_ERR_ARG;
+  if (stage != ORC_STAGE_DECODER && stage != ORC_STAGE_ENCODER) return ORC_ERR_ARG;
+  const int af3 = style == ORC_STYLE_AF3, enc = stage == ORC_STAGE_ENCODER;
+  const int64_t B = d->B, A = d->A, T = d->T, K = d->K, C = d->C, S = d->S, H = d->H,
+                D = d->D, P = d->P, M = d->M, U = d->U, V = d->V, HD = H * D;
+  /* dims >= 1, D even for ESMFold2, eps > 0, radius >= -1  [WAA 1, WAA 2, WAA 12] */
+  if (B < 1 || A < 1 || T < 1 || K < 1 || C < 1 || S < 1 || H < 1 || D < 1 || M < 1)
+    return ORC_ERR_DIM;
+  if (enc && U < 1) return ORC_ERR_DIM;
+  if (!enc && V < 1) return ORC_ERR_DIM;
+  if (af3 && P < 1) return ORC_ERR_DIM;
+  if (!af3 && (D % 2) != 0) return ORC_ERR_DIM;
+  if (!(eps > 0.0) || !isfinite(eps)) return ORC_ERR_EPS;
+  if (radius < -1) return ORC_ERR_RADIUS;
+  if (!in->atom || !in->condition || !in->valid || !in->token_valid || !in->window_mask ||
+      !in->key_index || !in->atom_to_token || !out->hidden || !out->attention)
+    return ORC_ERR_ARG;
+  if (af3 && (!in->pair || !p->cond_scale || !p->w_scale || !p->b_scale || !p->w_shift ||
+              !p->w_residual_gate || !p->b_residual_gate || !p->b_q || !p->pair_scale ||
+              !p->w_pair))
+    return ORC_ERR_ARG;
+  if (!af3 && (!p->w_mod || !in->rope_cos || !in->rope_sin)) return ORC_ERR_ARG;
+  if (!p->w_q || !p->w_k || !p->w_v || !p->w_value_gate || !p->w_attention_out ||
+      !p->w_ff_gate || !p->w_ff_up || !p->w_ff_out)
+    return ORC_ERR_ARG;
+  if (enc && (!p->w_pool || !out->token_output)) return ORC_ERR_ARG;
+  if (!enc && (!in->token || !p->w_token || !p->readout_scale || !p->w_readout ||
+               !out->position_update || (!af3 && !p->readout_bias)))
+    return ORC_ERR_ARG;
+
+  const double inv_sqrt_d = 1.0 / sqrt((double)D);
+  const int64_t GW = p->value_gate_per_head ? H : HD; /* value-gate logit width */
+
+  uint8_t *usable = (uint8_t *)malloc((size_t)(B * A));
+  uint8_t *perm = (uint8_t *)malloc((size_t)(B * A * K));
+  uint8_t *need = (uint8_t *)malloc((size_t)A);
+  if (!usable || !perm || !need) {
+    free(usable); free(perm); free(need);
+    return ORC_ERR_NOMEM;
+  }
+  orc_usable(d, in, usable);
+  orc_permitted(d, in, usable, radius, perm);
+
+  arena ar = {{0}, 0};
+  double *x = grab(&ar, A * C);        /* residual state per atom */
+  double *Q = grab(&ar, A * HD), *Kf = grab(&ar, A * HD), *Vf = grab(&ar, A * HD);
+  double *G = grab(&ar, A * GW);
+  double *g0 = grab(&ar, A * C), *g1 = grab(&ar, A * C);    /* residual gates */
+  double *tsc = grab(&ar, A * C), *tsh = grab(&ar, A * C);  /* transition scale/shift */
+  double *tmp = grab(&ar, 8 * (C + S + HD + M + U + V + P + K) + 64);
+  double *pooled = enc ? grab(&ar, T * U) : NULL;
+  int64_t *count = enc ? (int64_t *)malloc((size_t)T * sizeof(int64_t)) : NULL;
+  uint8_t *tok_ok = enc ? (uint8_t *)malloc((size_t)T) : NULL;
+  int fail = (ar.n != 10 + (enc ? 1 : 0)) || (enc && (!count || !tok_ok));
+  for (int i = 0; i < ar.n && !fail; ++i) fail = ar.buf[i] == NULL;
+  if (fail) {
+    arena_free(&ar); free(usable); free(perm); free(need); free(count); free(tok_ok);
+    return ORC_ERR_NOMEM;
+  }
+
+  /* scratch rows carved from tmp */
+  double *r_c = tmp;              /* clean condition [S] */
+  double *r_ln = r_c + S;         /* LN(c) or SiLU(c) [S] */
+  double *r_cj = r_ln + S;        /* LN(c) * cond_scale[j] [S] */
+  double *r_x = r_cj + S;         /* normalised x [C] */
+  double *r_sc = r_x + C;         /* scale logits [C] */
+  double *r_sh = r_sc + C;        /* shift [C] */
+  double *r_f0 = r_sh + C;        /* query features / shared attention input [C] */
+  double *r_f1 = r_f0 + C;        /* key/value features [C] */
+  double *r_m = r_f1 + C;         /* ESMFold2 six vectors [6C] */
+  double *r_q = r_m + 6 * C;      /* projection before head norm [HD] */
+  double *r_h = r_q + HD;         /* one head [D] */
+  double *r_o = r_h + D;          /* attention output [HD] */
+  double *r_u = r_o + HD;         /* out-projection [C] */
+  double *r_z = r_u + C;          /* transition input [C] */
+  double *r_a = r_z + C;          /* z @ w_ff_gate [M] */
+  double *r_b = r_a + M;          /* z @ w_ff_up [M] */
+  double *r_ff = r_b + M;         /* transition update [C] */
+  double *r_pool = r_ff + C;      /* hidden @ w_pool [U] */
+  double *r_lg = r_pool + U;      /* logits of one row [K] */
+  double *r_w = r_lg + K;         /* weights of one row [K] */
+  double *r_pr = r_w + K;         /* LN(pair) [P] */
+  double *r_tk = r_pr + P;        /* token @ w_token [C] */
+
+  for (int64_t b = 0; b < B; ++b) {
+    const uint8_t *use = usable + b * A;
+    const uint8_t *sel = query_select ? query_select + b * A : NULL;
+    const uint8_t *pm = perm + b * A * K;
+    const int64_t *kid = in->key_index + b * A * K;
+    const int64_t *att = in->atom_to_token + b * A;
+
+    /* atoms whose features are needed: selected queries and their permitted keys */
+    for (int64_t a = 0; a < A; ++a) need[a] = 0;
+    for (int64_t a = 0; a < A; ++a) {
+      if (sel && !sel[a]) continue;
+      need[a] = 1;
+      for (int64_t k = 0; k < K; ++k)
+        if (pm[a * K + k]) need[kid[a * K + k]] = 1;
+    }
+
+    /* ---- residual start and conditioning for every needed usable atom ---- */
+    for (int64_t a = 0; a < A; ++a) {
+      if (!need[a] || !use[a]) continue;
+      const int64_t ia = b * A + a;
+      /* sanitised payloads: an unusable atom is never reached here, so the
+       * select below is the usable branch  [WAA 3] */
+      const double *atom_row = in->atom + ia * C;
+      double *xa = x + a * C;
+      if (enc) {
+        for (int64_t c = 0; c < C; ++c) xa[c] = atom_row[c];          /* x = atom */
+      } else {
+        /* x = skip + gather(token @ w_token, atom_to_token), bias free  [WAA 3] */
+        vecmat(in->token + (b * T + att[a]) * V, p->w_token, NULL, V, C, r_tk);
+        for (int64_t c = 0; c < C; ++c) xa[c] = atom_row[c] + r_tk[c];
+      }
+      for (int64_t s = 0; s < S; ++s) r_c[s] = in->condition[ia * S + s];
+
+      if (af3) {
+        /* A_j(z, c) = LN(z) * sigmoid(c_j @ w_scale[j] + b_scale[j]) + c_j @ w_shift[j],
+         * c_j = LN(c) * cond_scale[j]; j = 0 query, 1 key/value, 2 transition  [WAA 7] */
+        orc_layer_norm(r_c, S, eps, r_ln);
+        orc_layer_norm(xa, C, eps, r_x);
+        for (int j = 0; j < 3; ++j) {
+          for (int64_t s = 0; s < S; ++s) r_cj[s] = r_ln[s] * p->cond_scale[j * S + s];
+          vecmat(r_cj, p->w_scale + j * S * C, p->b_scale + j * C, S, C, r_sc);
+          vecmat(r_cj, p->w_shift + j * S * C, NULL, S, C, r_sh);
+          if (j < 2) {
+            double *f = j == 0 ? r_f0 : r_f1;
+            for (int64_t c = 0; c < C; ++c) f[c] = r_x[c] * orc_sigmoid(r_sc[c]) + r_sh[c];
+          } else {
+            /* transition stage: kept as scale logits / shift, applied to x' later */
+            for (int64_t c = 0; c < C; ++c) {
+              tsc[a * C + c] = r_sc[c];
+              tsh[a * C + c] = r_sh[c];
+            }
+          }
+        }
+        /* residual gates sigmoid(raw condition @ w_residual_gate[j] + b[j])  [WAA 9] */
+        vecmat(r_c, p->w_residual_gate, p->b_residual_gate, S, C, g0 + a * C);
+        vecmat(r_c, p->w_residual_gate + S * C, p->b_residual_gate + C, S, C, g1 + a * C);
+        for (int64_t c = 0; c < C; ++c) {
+          g0[a * C + c] = orc_sigmoid(g0[a * C + c]);
+          g1[a * C + c] = orc_sigmoid(g1[a * C + c]);
+        }
+        /* Q from query features with b_q; K, V from key features, no bias; value
+         * gate from query features  [WAA 8, WAA 16] */
+        vecmat(r_f0, p->w_q, p->b_q, C, HD, Q + a * HD);
+        vecmat(r_f1, p->w_k, NULL, C, HD, Kf + a * HD);
+        vecmat(r_f1, p->w_v, NULL, C, HD, Vf + a * HD);
+        vecmat(r_f0, p->w_value_gate, NULL, C, GW, G + a * GW);
+      } else {
+        /* six vectors SiLU(condition) @ w_mod[S,6,C], in the order attention shift,
+         * scale, gate; transition shift, scale, gate  [WAA 10] */
+        for (int64_t s = 0; s < S; ++s) r_ln[s] = orc_silu(r_c[s]);
+        vecmat(r_ln, p->w_mod, NULL, S, 6 * C, r_m);
+        const double *a_shift = r_m, *a_scale = r_m + C, *a_gate = r_m + 2 * C;
+        const double *t_shift = r_m + 3 * C, *t_scale = r_m + 4 * C, *t_gate = r_m + 5 * C;
+        /* attention input RMS(x) * (1 + attention_scale) + attention_shift  [WAA 11] */
+        orc_rms_norm(xa, C, eps, r_x);
+        for (int64_t c = 0; c < C; ++c) r_f0[c] = r_x[c] * (1.0 + a_scale[c]) + a_shift[c];
+        /* raw gates, no sigmoid  [WAA 14] */
+        for (int64_t c = 0; c < C; ++c) {
+          g0[a * C + c] = a_gate[c];
+          g1[a * C + c] = t_gate[c];
+          tsc[a * C + c] = t_scale[c];
+          tsh[a * C + c] = t_shift[c];
+        }
+        /* bias-free Q/K/V and value gate from the shared input  [ESM RB, WAA 11] */
+        vecmat(r_f0, p->w_q, NULL, C, HD, Q + a * HD);
+        vecmat(r_f0, p->w_k, NULL, C, HD, Kf + a * HD);
+        vecmat(r_f0, p->w_v, NULL, C, HD, Vf + a * HD);
+        vecmat(r_f0, p->w_value_gate, NULL, C, GW, G + a * GW);
+        /* per-head RMS on Q and K, then half-split rotary before gathering
+         * [WAA 12, WAA 13] */
+        const double *cs = in->rope_cos + ia * D, *sn = in->rope_sin + ia * D;
+        double *mats[2] = {Q + a * HD, Kf + a * HD};
+        for (int m = 0; m < 2; ++m)
+          for (int64_t h = 0; h < H; ++h) {
+            double *vh = mats[m] + h * D;
+            orc_rms_norm(vh, D, eps, r_h);
+            orc_rope_half_split(r_h, cs, sn, D, vh);
+          }
+      }
+    }
+
+    /* ---- attention, residual, transition per selected query ---- */
+    for (int64_t a = 0; a < A; ++a) {
+      if (sel && !sel[a]) continue;
+      const int64_t ia = b * A + a;
+      for (int64_t h = 0; h < H; ++h) {
+        double *arow = out->attention + ((b * H + h) * A + a) * K;
+        for (int64_t k = 0; k < K; ++k) {
+          r_lg[k] = 0.0;
+          if (!pm[a * K + k]) continue;
+          int64_t j = kid[a * K + k];
+          /* dot(Q_query, K_key) / sqrt(D)  [WAA 15] */
+          double dot = 0.0;
+          for (int64_t e = 0; e < D; ++e) dot += Q[a * HD + h * D + e] * Kf[j * HD + h * D + e];
+          double lg = dot * inv_sqrt_d;
+          if (af3) {
+            /* + (LN(pair) * pair_scale) @ w_pair, one value per head  [WAA 8] */
+            orc_layer_norm(in->pair + (ia * K + k) * P, P, eps, r_pr);
+            double beta = 0.0;
+            for (int64_t q = 0; q < P; ++q) beta += r_pr[q] * p->pair_scale[q] * p->w_pair[q * H + h];
+            lg += beta;
+          }
+          r_lg[k] = lg;
+        }
+        orc_masked_softmax(r_lg, pm + a * K, K, arow);
+        /* weighted values; repeated slots are separate terms  [WAA 5, WAA 16] */
+        for (int64_t e = 0; e < D; ++e) r_o[h * D + e] = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+          if (!pm[a * K + k]) continue;
+          int64_t j = kid[a * K + k];
+          for (int64_t e = 0; e < D; ++e) r_o[h * D + e] += arow[k] * Vf[j * HD + h * D + e];
+        }
+      }
+      double *hid = out->hidden + ia * C;
+      if (!use[a]) {
+        /* hidden is masked to zero  [WAA 18] */
+        for (int64_t c = 0; c < C; ++c) hid[c] = 0.0;
+        if (!enc) for (int c = 0; c < 3; ++c) out->position_update[ia * 3 + c] = 0.0;
+        continue;
+      }
+      /* value gate sigmoid(query features @ w_value_gate), flattened head-major
+       * (index h*D + e), then w_attention_out without bias  [WAA 16] */
+      for (int64_t h = 0; h < H; ++h)
+        for (int64_t e = 0; e < D; ++e) {
+          double gl = p->value_gate_per_head ? G[a * GW + h] : G[a * GW + h * D + e];
+          r_o[h * D + e] *= orc_sigmoid(gl);
+        }
+      vecmat(r_o, p->w_attention_out, NULL, HD, C, r_u);
+      double *xa = x + a * C;
+      for (int64_t c = 0; c < C; ++c) hid[c] = xa[c] + g0[a * C + c] * r_u[c];   /* x' */
+
+      /* transition norm on the NEW x: AF3 A_2(x', c); ESMFold2
+       * RMS(x') * (1 + transition_scale) + transition_shift  [WAA 17] */
+      if (af3) {
+        orc_layer_norm(hid, C, eps, r_x);
+        for (int64_t c = 0; c < C; ++c)
+          r_z[c] = r_x[c] * orc_sigmoid(tsc[a * C + c]) + tsh[a * C + c];
+      } else {
+        orc_rms_norm(hid, C, eps, r_x);
+        for (int64_t c = 0; c < C; ++c)
+          r_z[c] = r_x[c] * (1.0 + tsc[a * C + c]) + tsh[a * C + c];
+      }
+      /* SiLU(z @ w_ff_gate) * (z @ w_ff_up), then w_ff_out, then gated residual  [WAA 17] */
+      vecmat(r_z, p->w_ff_gate, NULL, C, M, r_a);
+      vecmat(r_z, p->w_ff_up, NULL, C, M, r_b);
+      for (int64_t m = 0; m < M; ++m) r_a[m] = orc_silu(r_a[m]) * r_b[m];
+      vecmat(r_a, p->w_ff_out, NULL, M, C, r_ff);
+      for (int64_t c = 0; c < C; ++c) hid[c] += g1[a * C + c] * r_ff[c];   /* hidden */
+
+      if (!enc) {
+        /* position_update = (LN(hidden) * readout_scale [+ readout_bias]) @ w_readout,
+         * masked; an update, not coordinates  [WAA 18, WAA 19, WAA 20] */
+        orc_layer_norm(hid, C, eps, r_x);
+        for (int64_t c = 0; c < C; ++c)
+          r_x[c] = r_x[c] * p->readout_scale[c] + (af3 ? 0.0 : p->readout_bias[c]);
+        vecmat(r_x, p->w_readout, NULL, C, 3, out->position_update + ia * 3);
+      }
+    }
+
+    /* ---- encoder pooling: exact per-token mean of ReLU(hidden @ w_pool) over the
+     * usable atoms assigned to it; tokens without atoms give zero  [WAA 19] ---- */
+    if (enc) {
+      for (int64_t t = 0; t < T; ++t) {
+        count[t] = 0;
+        tok_ok[t] = 1;
+        for (int64_t u = 0; u < U; ++u) pooled[t * U + u] = 0.0;
+      }
+      for (int64_t a = 0; a < A; ++a) {   /* ascending atom order */
+        if (!use[a]) continue;
+        int64_t t = att[a];
+        if (sel && !sel[a]) { tok_ok[t] = 0; continue; }
+        vecmat(out->hidden + (b * A + a) * C, p->w_pool, NULL, C, U, r_pool);
+        for (int64_t u = 0; u < U; ++u)
+          pooled[t * U + u] += r_pool[u] > 0.0 ? r_pool[u] : 0.0;
+        count[t] += 1;
+      }
+      for (int64_t t = 0; t < T; ++t) {
+        if (!tok_ok[t]) continue;
+        double *orow = out->token_output + (b * T + t) * U;
+        for (int64_t u = 0; u < U; ++u)
+          orow[u] = count[t] > 0 ? pooled[t * U + u] / (double)count[t] : 0.0;
+      }
+    }
+  }
+
+  arena_free(&ar);
+  free(usable); free(perm); free(need); free(count); free(tok_ok);
+  return ORC_OK;
+}
