@@ -1,0 +1,426 @@
+#!/usr/bin/env python3
+"""Benchmark of the windowed atom attention forward pass on B200.
+
+One step = one forward pass of the whole block (usability + conditioning, projections,
+slot-gathered attention, transition, encoder pooling / decoder readout) over one
+synthetic batch, through the C ABI. Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the float64 CPU oracle on the host cores
+
+Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own seeded batch
+(independent problems, no collective on the data path: weak scaling); timing is the
+max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_windowed_atom_b200 import workloads  # noqa: E402
+
+DEFAULT_WORKLOAD = "esm_encoder_fp32_a4096"
+METRIC = "atom-encoder atoms/s and attention entries/s (A·H·K); % of HBM roofline"
+FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["atomenc", "reference"], default="atomenc")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=workloads.WORKLOAD_ORDER)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="host seconds for the oracle baseline sample")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def attention_bytes(spec: workloads.WorkloadSpec) -> int:
+    """Algorithmic HBM bytes of one slot-attention launch: key_index (int64), window_mask,
+    pair rows (AF3, storage type) and the usable flags read once; Q, K, V and value-gate
+    logits read once and the gated output written once (float32 workspace); the attention
+    weights written once (storage type)."""
+    s = 2 if spec.dtype == "bfloat16" else 4
+    slots = spec.B * spec.A * spec.K
+    hd = spec.H * spec.D
+    b = slots * (8 + 1)
+    if spec.style == "af3":
+        b += slots * spec.P * s
+    b += spec.B * spec.A * (1 + 5 * hd * 4)
+    b += spec.B * spec.H * spec.A * spec.K * s
+    return b
+
+
+def config_of(spec, world):
+    return {
+        "workload": spec.name, "description": spec.description, "style": spec.style,
+        "stage": spec.stage, "storage": "bf16" if spec.dtype == "bfloat16" else "fp32",
+        "B": spec.B, "A": spec.A, "T": spec.T, "K": spec.K, "C": spec.C, "S": spec.S,
+        "H": spec.H, "D": spec.D, "P": spec.P, "M": spec.M, "U": spec.U, "V": spec.V,
+        "radius": spec.radius, "atoms_per_step": spec.atoms * world,
+        "entries_per_step": spec.entries * world,
+        "l2": f"flushed before every timed step ({FLUSH_BYTES >> 20} MiB write)",
+        "parallelism": f"replicas x{world} (independent batches per GPU)",
+    }
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, STREAM-style copy)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s earlier measurement on this pool)"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for name in ("attention.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "sparse_windowed_atom_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per attention launch from a committed ncu summary, if it was taken on
+    the current kernel source for this workload; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic_k_slot_attention.txt")
+    if not os.path.exists(path):
+        return None
+    sha = kernel_source_sha()
+    with open(path) as f:
+        for line in f:
+            if line.startswith("#") or "=" not in line:
+                continue
+            kv = dict(x.split("=", 1) for x in line.split())
+            if kv.get("workload") == workload and kv.get("source_sha") == sha:
+                return int(kv["dram_bytes_per_launch"])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, device_uuid: str | None):
+        self.samples = []
+        self.t0 = self.t1 = None
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if device_uuid:
+            cmd[1:1] = ["-i", device_uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 8:
+                self.samples.append((time.monotonic(), parts))
+
+    def start(self):
+        self.t0 = time.monotonic()
+
+    def stop(self):
+        self.t1 = time.monotonic()
+        time.sleep(0.25)
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        inside = [p for t, p in self.samples if self.t0 - 0.15 <= t <= self.t1 + 0.15]
+        note = "timed region"
+        if not inside:
+            # a timed region shorter than the sampling period: take the nearest samples
+            inside = [p for t, p in sorted(self.samples, key=lambda s: abs(s[0] - self.t1))[:3]]
+            note = "nearest samples (timed region shorter than the 100 ms sampling period)"
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[0]) for p in inside if num(p[0]) is not None]
+        mx = [num(p[1]) for p in inside if num(p[1]) is not None]
+        reasons = set()
+        for p in inside:
+            for name, val in zip(self.NAMES, p[4:8]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(inside), "window": note}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_rate(spec, budget_s: float, seed: int = 0):
+    """Time the float64 oracle (as it stands, one host thread) on a bounded sample of the
+    workload: batch element 0, the first n query atoms (n doubled until the budget is
+    used), repeated until budget_s. Returns (atoms/s, sample description, seconds)."""
+    import oracle
+    w = workloads.make_inputs(spec.replace(B=1), seed=seed)
+    f64 = lambda d: {k: v.astype(np.float64) for k, v in d.items()}
+    act, prm = f64(w["activations"]), f64(w["parameters"])
+    n = min(spec.A, 1024)
+    done, spent, passes = 0, 0.0, 0
+    while spent < budget_s:
+        sel = np.zeros((1, spec.A), bool)
+        sel[0, :n] = True
+        t = time.perf_counter()
+        oracle.windowed_atom_attention(act, prm, w["masks"], w["structure"], eps=spec.eps,
+                                       style=spec.style, stage=spec.stage, radius=spec.radius,
+                                       query_select=None if n == spec.A else sel)
+        dt = time.perf_counter() - t
+        spent += dt
+        done += n
+        passes += 1
+        if dt < budget_s / 6 and n < spec.A:
+            n = min(spec.A, n * 2)
+    sample = (f"batch element 0 of {spec.name}: {passes} oracle passes over the first "
+              f"<= {n} of {spec.A} query atoms ({done} atoms total)")
+    return done / spent, sample, spent
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    spec = workloads.WORKLOADS[args.workload]
+    steps, warm = args.steps, args.warmup
+    per_step = max(0.5, min(8.0, 150.0 / max(1, steps + warm)))
+    for _ in range(warm):
+        oracle_rate(spec, per_step / 4)
+    total_atoms, total_s, sample = 0.0, 0.0, ""
+    for _ in range(steps):
+        r, sample, s = oracle_rate(spec, per_step)
+        total_atoms += r * s
+        total_s += s
+    rate = total_atoms / total_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": "atoms/s",
+        "n_gpus": args.gpus, "steps": steps, "warmup": warm, "ms_per_step": 1e3 * total_s / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "config": config_of(spec, 1),
+        "entries_per_s": rate * spec.H * spec.K,
+        "cpu_baseline": {"value": rate, "unit": "atoms/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: {sample}"},
+        "e2e": {"value": rate, "unit": "atoms/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_atomenc(args):
+    import torch
+    import torch.distributed as dist
+
+    from sparse_windowed_atom_b200 import atomenc
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU path exists)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    spec = workloads.WORKLOADS[args.workload]
+    w = workloads.make_inputs(spec, seed=rank)
+    fdt = torch.bfloat16 if spec.dtype == "bfloat16" else torch.float32
+    host = {}
+    for grp in ("activations", "parameters"):
+        for k, v in w[grp].items():
+            host[k] = torch.from_numpy(np.ascontiguousarray(v)).to(fdt)
+    for grp in ("masks", "structure"):
+        for k, v in w[grp].items():
+            host[k] = torch.from_numpy(np.ascontiguousarray(v))
+    pnames = set(w["parameters"])
+    devt = {k: v.to(dev) for k, v in host.items()}
+    inputs = {k: v for k, v in devt.items() if k not in pnames}
+    params = {k: v for k, v in devt.items() if k in pnames}
+    outs = {k: torch.empty(s, dtype=fdt, device=dev)
+            for k, s in atomenc.output_shapes(spec.style, spec.stage, inputs, params).items()}
+    ws = torch.empty(atomenc.atomenc_workspace_size(spec.style, spec.stage, inputs, params, outs),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    nph = atomenc.NUM_PHASES + 1
+    K, W = args.steps, args.warmup
+
+    def make_events(n):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nph)] for _ in range(n)]
+        for row in evs:
+            for e in row:
+                e.record(stream)
+        return evs
+
+    def fwd(evrow):
+        return atomenc.atomenc_forward_profiled(spec.style, spec.stage, inputs, params, spec.eps,
+                                                spec.radius, outs, ws, evrow, stream)
+
+    warm_ev = make_events(1)[0]
+    for _ in range(W):
+        flush.zero_()
+        fwd(warm_ev)
+    evs = make_events(K)
+    torch.cuda.synchronize(dev)
+    status = atomenc.atomenc_get_status(ws, stream)
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    launches = 0
+    for i in range(K):
+        flush.zero_()
+        launches += fwd(evs[i])
+    torch.cuda.synchronize(dev)
+    barrier()
+    sampler.stop()
+
+    step_ms = [evs[i][0].elapsed_time(evs[i][nph - 1]) for i in range(K)]
+    phase_ms = [statistics.fmean(evs[i][p].elapsed_time(evs[i][p + 1]) for i in range(K))
+                for p in range(atomenc.NUM_PHASES)]
+    total_ms = max_over_ranks(sum(step_ms))
+    ms_per_step = total_ms / K
+    atoms = spec.atoms * world
+    value = atoms / (ms_per_step / 1e3)
+
+    # ---- roofline of the slot-attention kernel (timed live, phase 3 = that kernel alone)
+    attn_ms = max_over_ranks(phase_ms[3])
+    peak, peak_src = load_peaks()
+    abytes = attention_bytes(spec)
+    achieved = abytes / (attn_ms / 1e3) / 1e9
+    dominant = max(range(atomenc.NUM_PHASES), key=lambda p: phase_ms[p])
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": recorded_traffic(spec.name),
+                "kernel": "k_slot_attention", "bytes_per_launch": abytes,
+                "avg_launch_ms": attn_ms, "peak_source": peak_src,
+                "frac_of_8TBs": achieved / 8000.0}
+
+    # ---- end to end: pinned host inputs -> device, forward, outputs -> pinned host
+    e2e = None
+    if not args.no_e2e:
+        hpin = {k: v.pin_memory() for k, v in host.items()}
+        hout = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outs.items()}
+        h2d = sum(v.numel() * v.element_size() for v in hpin.values())
+        d2h = sum(v.numel() * v.element_size() for v in hout.values())
+        ke = max(3, min(K, 20))
+
+        def e2e_step():
+            for k, v in hpin.items():
+                devt[k].copy_(v, non_blocking=True)
+            atomenc.atomenc_forward(spec.style, spec.stage, inputs, params, spec.eps, spec.radius,
+                                    outs, ws, stream)
+            for k, v in outs.items():
+                hout[k].copy_(v, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_ms = max_over_ranks(e0.elapsed_time(e1)) / ke
+        e2e = {"value": atoms / (e_ms / 1e3), "unit": "atoms/s", "h2d_bytes_per_step": h2d * world,
+               "d2h_bytes_per_step": d2h * world, "ms_per_step": e_ms, "steps": ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, sample, spent = oracle_rate(spec, args.cpu_seconds)
+        cpu = {"value": rate, "unit": "atoms/s", "cores": 1, "kind": "oracle", "sample": sample,
+               "seconds": spent}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "atoms/s", "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded workload generator; no dataset)",
+            "config": config_of(spec, world),
+            "entries_per_s": spec.entries * world / (ms_per_step / 1e3),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": sampler.summary(),
+            "phase_ms": dict(zip(atomenc.PHASES, phase_ms)),
+            "dominant_phase": atomenc.PHASES[dominant],
+            "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_atomenc(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

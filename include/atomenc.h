@@ -1,0 +1,195 @@
+/*
+ * atomenc.h -- C ABI of the B200 (sm_100a) windowed atom attention library.
+ *
+ * One call runs the forward pass of one learned local atom block in AlphaFold3 or
+ * ESMFold2 style, with its encoder (per-token pooled output) or decoder (coordinate
+ * update) boundary, as defined on the page "Local atom attention, encoder pooling
+ * and decoder skip/readout" (windowed_atom_attention), Required behavior; the two
+ * encoder pages ("AlphaFold 3 Atom Attention Encoder", "ESMFold 2 Atom Attention
+ * Encoder") are its encoder specialisations.
+ *
+ * Conventions
+ *  - Every tensor is described by an atomenc_tensor: a DEVICE pointer, an element
+ *    type, a rank and a shape. Strides are in elements; the library accepts only
+ *    dense row-major tensors (stride[i] == product of shape[i+1..]) and returns
+ *    ATOMENC_ERR_STRIDE otherwise.
+ *  - All floating tensors of one call (activations, parameters, outputs) share one
+ *    element type, ATOMENC_F32 or ATOMENC_BF16; arithmetic is float32 inside the
+ *    kernels (bf16 values are widened exactly). Indices are ATOMENC_I64, masks
+ *    ATOMENC_BOOL (one byte, 0 or 1).
+ *  - A tensor that the chosen style/stage does not use may be left empty
+ *    (data == NULL, ndim == 0); it is not read.
+ *  - Ownership: the caller owns every buffer, including the workspace. The library
+ *    never allocates device or pinned memory and never writes to an input.
+ *  - Streams: atomenc_forward only enqueues work on `stream` and returns; it does
+ *    not synchronise. All errors are decided on the host before the first launch,
+ *    so a non-zero return means nothing was enqueued. Launch failures reported by
+ *    the CUDA runtime are returned as ATOMENC_ERR_CUDA.
+ *  - Inputs must not alias outputs or the workspace. Calls that share a workspace
+ *    must be ordered on one stream.
+ *
+ * Shapes (B batch, A atoms, T tokens, K key slots, C atom width, S condition width,
+ * H heads, D head width, P pair channels, M transition width, U pooled width,
+ * V token width). Every weight is applied as x @ W with W stored [in, out]; the
+ * pages print no shape table, so these shapes are the reading the formulas give.
+ */
+#ifndef ATOMENC_H
+#define ATOMENC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *atomenc_stream_t; /* a cudaStream_t; NULL = legacy default */
+
+enum atomenc_dtype { ATOMENC_F32 = 0, ATOMENC_BF16 = 1, ATOMENC_I64 = 2, ATOMENC_BOOL = 3 };
+
+/* style: "af3" (default on the windowed page) or "esmfold2" */
+enum atomenc_style { ATOMENC_AF3 = 0, ATOMENC_ESMFOLD2 = 1 };
+/* stage: "decoder" (default on the windowed page) or "encoder" */
+enum atomenc_stage { ATOMENC_DECODER = 0, ATOMENC_ENCODER = 1 };
+
+enum atomenc_status {
+  ATOMENC_OK = 0,
+  ATOMENC_ERR_NULL = -1,        /* a required tensor, pointer or struct is missing */
+  ATOMENC_ERR_STYLE = -2,       /* unknown style or stage */
+  ATOMENC_ERR_DTYPE = -3,       /* float types differ, index not int64, mask not bool */
+  ATOMENC_ERR_SHAPE = -4,       /* ranks or sizes disagree, a dimension < 1 */
+  ATOMENC_ERR_STRIDE = -5,      /* a tensor is not dense row-major */
+  ATOMENC_ERR_EPS = -6,         /* eps not finite or not > 0 in the float type */
+  ATOMENC_ERR_RADIUS = -7,      /* radius < -1 */
+  ATOMENC_ERR_ODD_HEAD = -8,    /* ESMFold2 style with odd D (half-split rotary) */
+  ATOMENC_ERR_UNSUPPORTED = -9, /* a size outside what the kernels are built for */
+  ATOMENC_ERR_WORKSPACE = -10,  /* workspace NULL, too small or not 256-byte aligned */
+  ATOMENC_ERR_CUDA = -11        /* the CUDA runtime rejected a launch */
+};
+
+typedef struct {
+  void *data;         /* device pointer */
+  int32_t dtype;      /* enum atomenc_dtype */
+  int32_t ndim;       /* 0 = empty / not supplied */
+  int64_t shape[5];
+  int64_t stride[5];  /* elements */
+} atomenc_tensor;
+
+/* "activations", "masks" and "structure" dictionaries of the page signatures. */
+typedef struct {
+  atomenc_tensor atom;          /* [B,A,C] encoder input x / decoder skip */
+  atomenc_tensor condition;     /* [B,A,S] per-atom condition */
+  atomenc_tensor pair;          /* [B,A,K,P] pair descriptor per query slot (AF3) */
+  atomenc_tensor token;         /* [B,T,V] token features (decoder) */
+  atomenc_tensor rope_cos;      /* [B,A,D] full-width rotary cos (ESMFold2), shared by heads */
+  atomenc_tensor rope_sin;      /* [B,A,D] */
+  atomenc_tensor valid;         /* [B,A] bool */
+  atomenc_tensor token_valid;   /* [B,T] bool */
+  atomenc_tensor window_mask;   /* [B,A,K] bool, True permits the slot */
+  atomenc_tensor key_index;     /* [B,A,K] int64 atom ids within the batch element;
+                                   ids outside [0,A) are missing slots */
+  atomenc_tensor atom_to_token; /* [B,A] int64, any order; out of range = unusable */
+} atomenc_inputs;
+
+/* "parameters" dictionary (names follow the page formulas). */
+typedef struct {
+  atomenc_tensor cond_scale;       /* [3,S]   AF3 */
+  atomenc_tensor w_scale;          /* [3,S,C] AF3 */
+  atomenc_tensor b_scale;          /* [3,C]   AF3 */
+  atomenc_tensor w_shift;          /* [3,S,C] AF3 */
+  atomenc_tensor w_residual_gate;  /* [2,S,C] AF3 */
+  atomenc_tensor b_residual_gate;  /* [2,C]   AF3 */
+  atomenc_tensor w_mod;            /* [S,6,C] ESMFold2 */
+  atomenc_tensor w_q;              /* [C,H*D] */
+  atomenc_tensor b_q;              /* [H*D]   AF3 */
+  atomenc_tensor w_k;              /* [C,H*D] */
+  atomenc_tensor w_v;              /* [C,H*D] */
+  atomenc_tensor w_value_gate;     /* [C,H*D] */
+  atomenc_tensor pair_scale;       /* [P]     AF3 */
+  atomenc_tensor w_pair;           /* [P,H]   AF3 (gives H) */
+  atomenc_tensor w_attention_out;  /* [H*D,C] */
+  atomenc_tensor w_ff_gate;        /* [C,M] */
+  atomenc_tensor w_ff_up;          /* [C,M] */
+  atomenc_tensor w_ff_out;         /* [M,C] */
+  atomenc_tensor w_pool;           /* [C,U]   encoder */
+  atomenc_tensor w_token;          /* [V,C]   decoder */
+  atomenc_tensor readout_scale;    /* [C]     decoder */
+  atomenc_tensor readout_bias;     /* [C]     decoder, ESMFold2 */
+  atomenc_tensor w_readout;        /* [C,3]   decoder */
+} atomenc_params;
+
+typedef struct {
+  atomenc_tensor hidden;           /* [B,A,C]   always */
+  atomenc_tensor attention;        /* [B,H,A,K] always; 0 on slots that are not permitted */
+  atomenc_tensor token_output;     /* [B,T,U]   encoder only */
+  atomenc_tensor position_update;  /* [B,A,3]   decoder only */
+} atomenc_outputs;
+
+/*
+ * Bytes of device workspace atomenc_forward needs for these shapes (0 on a
+ * validation error; the same checks as atomenc_forward, minus eps/radius).
+ * The heads count H is taken from w_pair (AF3) or rope_cos's last dim D (ESMFold2).
+ */
+size_t atomenc_workspace_size(int style, int stage, const atomenc_inputs *in,
+                              const atomenc_params *params, const atomenc_outputs *out);
+
+/*
+ * Enqueue the forward pass on `stream`.
+ *   style, stage  enum atomenc_style / atomenc_stage
+ *   eps           > 0; the one stabiliser added inside the square root of every
+ *                 LayerNorm and RMS normalisation of the block (windowed page,
+ *                 Required behavior, eps bullet)
+ *   radius        -1 (no index window) or >= 0: a slot also needs |key - query| <= radius
+ *   workspace     device buffer of at least atomenc_workspace_size() bytes, 256-byte
+ *                 aligned; contents need not be initialised and are overwritten.
+ * Writes every element of out->hidden and out->attention, and of out->token_output
+ * (encoder) or out->position_update (decoder). Returns enum atomenc_status.
+ */
+int atomenc_forward(int style, int stage, const atomenc_inputs *in,
+                    const atomenc_params *params, double eps, int64_t radius,
+                    const atomenc_outputs *out, void *workspace, size_t workspace_bytes,
+                    atomenc_stream_t stream);
+
+/* Phases of one forward pass, in launch order (for atomenc_forward_profiled). */
+enum atomenc_phase {
+  ATOMENC_PHASE_INPUTS = 0,        /* weight panels, usability, sanitisation, residual start */
+  ATOMENC_PHASE_CONDITIONING = 1,  /* AF3 adaptive-norm / gate projections; ESMFold2 w_mod */
+  ATOMENC_PHASE_PROJECTIONS = 2,   /* attention inputs, Q/K/V/value gate (+ head RMS, rotary) */
+  ATOMENC_PHASE_ATTENTION = 3,     /* the slot-gathered attention kernel alone */
+  ATOMENC_PHASE_TRANSITION = 4,    /* out-projection, residual, transition, hidden */
+  ATOMENC_PHASE_BOUNDARY = 5,      /* encoder pooling / decoder readout */
+  ATOMENC_NUM_PHASES = 6
+};
+
+/*
+ * atomenc_forward with timing hooks: `events` holds n_events == ATOMENC_NUM_PHASES + 1
+ * cudaEvent_t handles created by the caller; events[0] is recorded on `stream` before
+ * the first launch and events[i + 1] after phase i, so cudaEventElapsedTime(events[i],
+ * events[i + 1]) is the device time of phase i. *n_launches (if not NULL) receives the
+ * number of kernels the call launched. Same results and errors as atomenc_forward.
+ */
+int atomenc_forward_profiled(int style, int stage, const atomenc_inputs *in,
+                             const atomenc_params *params, double eps, int64_t radius,
+                             const atomenc_outputs *out, void *workspace, size_t workspace_bytes,
+                             atomenc_stream_t stream, void *const *events, int n_events,
+                             int *n_launches);
+
+/*
+ * Read the device status word that the last forward pass using `workspace` left
+ * (waits for `stream`). Bits: 1 = some query tile's keys spanned more rows than the
+ * shared-memory stage holds and were gathered from L2 instead (slower, same result);
+ * 2 = atom_to_token was not grouped by token, so pooling scanned wider atom ranges
+ * (slower, same result). Never an error; returns enum atomenc_status.
+ */
+int atomenc_get_status(const void *workspace, int *device_status, atomenc_stream_t stream);
+
+/* Static English text for an atomenc_status code. */
+const char *atomenc_strerror(int code);
+
+/* Library version, for the Python binding's load check. */
+int atomenc_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ATOMENC_H */

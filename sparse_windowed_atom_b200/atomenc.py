@@ -1,0 +1,210 @@
+"""Thin Python binding of the atomenc C ABI (include/atomenc.h).
+
+Argument marshalling only: every step of the block runs in the CUDA library
+libatomenc.so. torch supplies device memory and streams. There is no CPU path: if
+the library is missing or no CUDA device is present, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libatomenc.so")
+
+ATOMENC_F32, ATOMENC_BF16, ATOMENC_I64, ATOMENC_BOOL = 0, 1, 2, 3
+STYLES = {"af3": 0, "esmfold2": 1}
+STAGES = {"decoder": 0, "encoder": 1}
+_DTYPES = {torch.float32: ATOMENC_F32, torch.bfloat16: ATOMENC_BF16,
+           torch.int64: ATOMENC_I64, torch.bool: ATOMENC_BOOL}
+
+
+class AtomencTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 5), ("stride", ctypes.c_int64 * 5)]
+
+
+INPUT_FIELDS = ["atom", "condition", "pair", "token", "rope_cos", "rope_sin", "valid",
+                "token_valid", "window_mask", "key_index", "atom_to_token"]
+PARAM_FIELDS = ["cond_scale", "w_scale", "b_scale", "w_shift", "w_residual_gate",
+                "b_residual_gate", "w_mod", "w_q", "b_q", "w_k", "w_v", "w_value_gate",
+                "pair_scale", "w_pair", "w_attention_out", "w_ff_gate", "w_ff_up", "w_ff_out",
+                "w_pool", "w_token", "readout_scale", "readout_bias", "w_readout"]
+OUTPUT_FIELDS = ["hidden", "attention", "token_output", "position_update"]
+
+
+class AtomencInputs(ctypes.Structure):
+    _fields_ = [(n, AtomencTensor) for n in INPUT_FIELDS]
+
+
+class AtomencParams(ctypes.Structure):
+    _fields_ = [(n, AtomencTensor) for n in PARAM_FIELDS]
+
+
+class AtomencOutputs(ctypes.Structure):
+    _fields_ = [(n, AtomencTensor) for n in OUTPUT_FIELDS]
+
+
+class AtomencError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: atomenc error {code}: {atomenc_strerror(code)}")
+        self.code = code
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libatomenc.so; raise if it has not been built (no fallback exists)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m sparse_windowed_atom_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER
+        lib.atomenc_workspace_size.restype = ctypes.c_size_t
+        lib.atomenc_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, P(AtomencInputs),
+                                               P(AtomencParams), P(AtomencOutputs)]
+        lib.atomenc_forward.restype = ctypes.c_int
+        lib.atomenc_forward.argtypes = [ctypes.c_int, ctypes.c_int, P(AtomencInputs),
+                                        P(AtomencParams), ctypes.c_double, ctypes.c_int64,
+                                        P(AtomencOutputs), ctypes.c_void_p, ctypes.c_size_t,
+                                        ctypes.c_void_p]
+        lib.atomenc_forward_profiled.restype = ctypes.c_int
+        lib.atomenc_forward_profiled.argtypes = lib.atomenc_forward.argtypes + [
+            P(ctypes.c_void_p), ctypes.c_int, P(ctypes.c_int)]
+        lib.atomenc_get_status.restype = ctypes.c_int
+        lib.atomenc_get_status.argtypes = [ctypes.c_void_p, P(ctypes.c_int), ctypes.c_void_p]
+        lib.atomenc_strerror.restype = ctypes.c_char_p
+        lib.atomenc_strerror.argtypes = [ctypes.c_int]
+        lib.atomenc_version.restype = ctypes.c_int
+        lib.atomenc_version.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def describe(t) -> AtomencTensor:
+    """atomenc_tensor for a torch tensor (or an empty descriptor for None)."""
+    d = AtomencTensor()
+    if t is None:
+        return d
+    if t.dim() > 5:
+        raise ValueError("atomenc tensors have at most 5 dims")
+    d.data = t.data_ptr()
+    d.dtype = _DTYPES.get(t.dtype, 99)      # the library rejects unknown codes
+    d.ndim = t.dim()
+    for i, (s, st) in enumerate(zip(t.shape, t.stride())):
+        d.shape[i] = s
+        d.stride[i] = st
+    return d
+
+
+def _structs(inputs: dict, params: dict, outputs: dict):
+    ins = AtomencInputs(**{n: describe(inputs.get(n)) for n in INPUT_FIELDS})
+    prm = AtomencParams(**{n: describe(params.get(n)) for n in PARAM_FIELDS})
+    outs = AtomencOutputs(**{n: describe(outputs.get(n)) for n in OUTPUT_FIELDS})
+    return ins, prm, outs
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def atomenc_strerror(code: int) -> str:
+    return load_library().atomenc_strerror(int(code)).decode()
+
+
+def atomenc_version() -> int:
+    return load_library().atomenc_version()
+
+
+def atomenc_workspace_size(style: str, stage: str, inputs: dict, params: dict,
+                           outputs: dict) -> int:
+    ins, prm, outs = _structs(inputs, params, outputs)
+    n = load_library().atomenc_workspace_size(STYLES[style], STAGES[stage], ctypes.byref(ins),
+                                              ctypes.byref(prm), ctypes.byref(outs))
+    if n == 0:
+        raise ValueError("atomenc_workspace_size: the arguments do not validate")
+    return int(n)
+
+
+def atomenc_forward(style: str, stage: str, inputs: dict, params: dict, eps: float,
+                    radius: int, outputs: dict, workspace: torch.Tensor, stream=None) -> None:
+    ins, prm, outs = _structs(inputs, params, outputs)
+    rc = load_library().atomenc_forward(STYLES[style], STAGES[stage], ctypes.byref(ins),
+                                        ctypes.byref(prm), float(eps), int(radius),
+                                        ctypes.byref(outs), workspace.data_ptr(),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream_ptr(stream))
+    if rc != 0:
+        raise AtomencError(rc, "atomenc_forward")
+
+
+NUM_PHASES = 6
+PHASES = ["inputs", "conditioning", "projections", "attention", "transition", "boundary"]
+
+
+def atomenc_forward_profiled(style: str, stage: str, inputs: dict, params: dict, eps: float,
+                             radius: int, outputs: dict, workspace: torch.Tensor, events,
+                             stream=None) -> int:
+    """atomenc_forward that records events[0] before the first launch and events[i+1]
+    after phase i (torch.cuda.Event objects, already recorded once so that they
+    exist). Returns the number of kernels launched."""
+    ins, prm, outs = _structs(inputs, params, outputs)
+    handles = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
+    n = ctypes.c_int(0)
+    rc = load_library().atomenc_forward_profiled(
+        STYLES[style], STAGES[stage], ctypes.byref(ins), ctypes.byref(prm), float(eps),
+        int(radius), ctypes.byref(outs), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream_ptr(stream), handles,
+        len(events), ctypes.byref(n))
+    if rc != 0:
+        raise AtomencError(rc, "atomenc_forward_profiled")
+    return n.value
+
+
+def atomenc_get_status(workspace: torch.Tensor, stream=None) -> int:
+    v = ctypes.c_int(0)
+    rc = load_library().atomenc_get_status(workspace.data_ptr(), ctypes.byref(v),
+                                           _stream_ptr(stream))
+    if rc != 0:
+        raise AtomencError(rc, "atomenc_get_status")
+    return v.value
+
+
+def output_shapes(style: str, stage: str, inputs: dict, params: dict) -> dict:
+    B, A, C = inputs["atom"].shape
+    K = inputs["key_index"].shape[-1]
+    T = inputs["token_valid"].shape[-1]
+    HD = params["w_q"].shape[-1]
+    H = params["w_pair"].shape[-1] if style == "af3" else HD // inputs["rope_cos"].shape[-1]
+    shapes = {"hidden": (B, A, C), "attention": (B, H, A, K)}
+    if stage == "encoder":
+        shapes["token_output"] = (B, T, params["w_pool"].shape[-1])
+    else:
+        shapes["position_update"] = (B, A, 3)
+    return shapes
+
+
+def windowed_atom_attention(activations: dict, parameters: dict, masks: dict, structure: dict,
+                            eps: float = 1e-5, style: str = "af3", stage: str = "decoder",
+                            radius: int = -1, workspace: torch.Tensor | None = None,
+                            stream=None) -> dict:
+    """Forward pass with the page's signature: dicts of CUDA tensors in, a dict out
+    (hidden, attention, and token_output for the encoder or position_update for the
+    decoder). Allocates the outputs (and the workspace unless one is given) with torch."""
+    inputs = {**activations, **masks, **structure}
+    dev = activations["atom"].device
+    fdt = activations["atom"].dtype
+    outputs = {k: torch.empty(s, dtype=fdt, device=dev)
+               for k, s in output_shapes(style, stage, inputs, parameters).items()}
+    need = atomenc_workspace_size(style, stage, inputs, parameters, outputs)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    atomenc_forward(style, stage, inputs, parameters, eps, radius, outputs, workspace, stream)
+    return outputs

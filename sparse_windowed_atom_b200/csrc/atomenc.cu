@@ -1,0 +1,559 @@
+// atomenc.cu -- host side of the C ABI declared in include/atomenc.h: argument checks,
+// workspace plan and the launch sequence of the windowed atom attention block.
+//
+// Order of the steps (page "Local atom attention, encoder pooling and decoder
+// skip/readout", Required behavior): usability + sanitisation + residual start
+// (bullets 2-3), conditioning (AF3 bullets 7, 9; ESMFold2 bullet 10), attention inputs and
+// Q/K/V/value-gate projections (bullets 8, 11-13), slot-gathered attention (bullets 4-6,
+// 15-16), out-projection and gated residual (bullet 16), transition (bullet 17), hidden
+// (bullet 18), encoder pooling or decoder readout (bullets 18-20).
+#include <climits>
+#include <cmath>
+#include <cstring>
+
+#include "../../include/atomenc.h"
+#include "attention.cuh"
+#include "common.cuh"
+#include "gemm_simt.cuh"
+#include "rows.cuh"
+
+using namespace atomenc;
+
+namespace {
+
+constexpr int kVersion = 1;
+constexpr int kMaxD = 64;
+constexpr size_t kAttnSmemBudget = 110 * 1024;
+
+struct Dims {
+  int64_t B = 0, A = 0, T = 0, K = 0, C = 0, S = 0, H = 0, D = 0, P = 0, M = 0, U = 0, V = 0;
+};
+
+bool present(const atomenc_tensor &t) { return t.data != nullptr && t.ndim > 0; }
+
+int check_tensor(const atomenc_tensor &t, int dtype, int ndim, const int64_t *shape) {
+  if (!present(t)) return ATOMENC_ERR_NULL;
+  if (t.dtype != dtype) return ATOMENC_ERR_DTYPE;
+  if (t.ndim != ndim) return ATOMENC_ERR_SHAPE;
+  for (int i = 0; i < ndim; ++i)
+    if (t.shape[i] != shape[i] || shape[i] < 1) return ATOMENC_ERR_SHAPE;
+  int64_t st = 1;
+  for (int i = ndim - 1; i >= 0; --i) {
+    if (t.shape[i] > 1 && t.stride[i] != st) return ATOMENC_ERR_STRIDE;
+    st *= t.shape[i];
+  }
+  return ATOMENC_OK;
+}
+
+#define CHECK(expr)                 \
+  do {                              \
+    int _rc = (expr);               \
+    if (_rc != ATOMENC_OK) return _rc; \
+  } while (0)
+
+float bf16_round_host(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  u = (u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+struct Plan {
+  int style = 0, stage = 0, fdt = 0;
+  bool af3 = false, enc = false;
+  Dims d;
+  // workspace layout (byte offsets)
+  size_t o_status, o_usable, o_first, o_last, o_tp, o_x, o_opc, o_rawc, o_cond, o_gate, o_feat,
+      o_q, o_k, o_v, o_g, o_o, o_xp, o_z, o_h, o_hid, o_pool;
+  size_t o_wcond, o_wgate, o_wqkv, o_wout, o_wff1, o_wff2, o_wpool, o_wtok, o_wread, o_bscale,
+      o_brg, o_bq, o_wpair, o_rscale, o_rbias;
+  size_t bytes = 0;
+  // attention launch
+  int QT = 0, cap = 0, DP = 0;
+  size_t attn_smem = 0;
+};
+
+size_t take(size_t &cur, size_t bytes) {
+  size_t o = cur;
+  cur += (bytes + 255) & ~size_t(255);
+  return o;
+}
+
+int validate(int style, int stage, const atomenc_inputs *in, const atomenc_params *p,
+             const atomenc_outputs *out, Plan &pl) {
+  if (!in || !p || !out) return ATOMENC_ERR_NULL;
+  if (style != ATOMENC_AF3 && style != ATOMENC_ESMFOLD2) return ATOMENC_ERR_STYLE;
+  if (stage != ATOMENC_DECODER && stage != ATOMENC_ENCODER) return ATOMENC_ERR_STYLE;
+  pl.style = style;
+  pl.stage = stage;
+  pl.af3 = style == ATOMENC_AF3;
+  pl.enc = stage == ATOMENC_ENCODER;
+  Dims &d = pl.d;
+  if (!present(in->atom) || !present(in->condition) || !present(in->key_index) ||
+      !present(in->token_valid))
+    return ATOMENC_ERR_NULL;
+  if (in->atom.ndim != 3 || in->condition.ndim != 3 || in->key_index.ndim != 3 ||
+      in->token_valid.ndim != 2)
+    return ATOMENC_ERR_SHAPE;
+  const int fdt = in->atom.dtype;
+  if (fdt != ATOMENC_F32 && fdt != ATOMENC_BF16) return ATOMENC_ERR_DTYPE;
+  pl.fdt = fdt;
+  d.B = in->atom.shape[0];
+  d.A = in->atom.shape[1];
+  d.C = in->atom.shape[2];
+  d.S = in->condition.shape[2];
+  d.K = in->key_index.shape[2];
+  d.T = in->token_valid.shape[1];
+  if (!present(p->w_q) || p->w_q.ndim != 2) return ATOMENC_ERR_NULL;
+  const int64_t HD = p->w_q.shape[1];
+  if (pl.af3) {
+    if (!present(p->w_pair) || p->w_pair.ndim != 2 || !present(in->pair) || in->pair.ndim != 4)
+      return ATOMENC_ERR_NULL;
+    d.H = p->w_pair.shape[1];
+    d.P = p->w_pair.shape[0];
+    if (d.H < 1 || HD % d.H != 0) return ATOMENC_ERR_SHAPE;
+    d.D = HD / d.H;
+  } else {
+    if (!present(in->rope_cos) || in->rope_cos.ndim != 3) return ATOMENC_ERR_NULL;
+    d.D = in->rope_cos.shape[2];
+    if (d.D < 1 || HD % d.D != 0) return ATOMENC_ERR_SHAPE;
+    d.H = HD / d.D;
+    if (d.D % 2 != 0) return ATOMENC_ERR_ODD_HEAD;
+  }
+  if (!present(p->w_ff_gate) || p->w_ff_gate.ndim != 2) return ATOMENC_ERR_NULL;
+  d.M = p->w_ff_gate.shape[1];
+  if (pl.enc) {
+    if (!present(p->w_pool) || p->w_pool.ndim != 2) return ATOMENC_ERR_NULL;
+    d.U = p->w_pool.shape[1];
+  } else {
+    if (!present(in->token) || in->token.ndim != 3) return ATOMENC_ERR_NULL;
+    d.V = in->token.shape[2];
+  }
+  const int64_t B = d.B, A = d.A, T = d.T, K = d.K, C = d.C, S = d.S, H = d.H, D = d.D,
+                P = d.P, M = d.M, U = d.U, V = d.V;
+  {
+    const int64_t s3[] = {B, A, C}, sc[] = {B, A, S}, sk[] = {B, A, K}, sa[] = {B, A},
+                  st[] = {B, T};
+    CHECK(check_tensor(in->atom, fdt, 3, s3));
+    CHECK(check_tensor(in->condition, fdt, 3, sc));
+    CHECK(check_tensor(in->key_index, ATOMENC_I64, 3, sk));
+    CHECK(check_tensor(in->window_mask, ATOMENC_BOOL, 3, sk));
+    CHECK(check_tensor(in->valid, ATOMENC_BOOL, 2, sa));
+    CHECK(check_tensor(in->atom_to_token, ATOMENC_I64, 2, sa));
+    CHECK(check_tensor(in->token_valid, ATOMENC_BOOL, 2, st));
+  }
+  {
+    const int64_t cq[] = {C, HD}, oc[] = {HD, C}, cm[] = {C, M}, mc[] = {M, C};
+    CHECK(check_tensor(p->w_q, fdt, 2, cq));
+    CHECK(check_tensor(p->w_k, fdt, 2, cq));
+    CHECK(check_tensor(p->w_v, fdt, 2, cq));
+    CHECK(check_tensor(p->w_value_gate, fdt, 2, cq));
+    CHECK(check_tensor(p->w_attention_out, fdt, 2, oc));
+    CHECK(check_tensor(p->w_ff_gate, fdt, 2, cm));
+    CHECK(check_tensor(p->w_ff_up, fdt, 2, cm));
+    CHECK(check_tensor(p->w_ff_out, fdt, 2, mc));
+  }
+  if (pl.af3) {
+    const int64_t pr[] = {B, A, K, P}, s3s[] = {3, S}, w3[] = {3, S, C}, b3[] = {3, C},
+                  w2[] = {2, S, C}, b2[] = {2, C}, bq[] = {HD}, ps[] = {P}, wp[] = {P, H};
+    CHECK(check_tensor(in->pair, fdt, 4, pr));
+    CHECK(check_tensor(p->cond_scale, fdt, 2, s3s));
+    CHECK(check_tensor(p->w_scale, fdt, 3, w3));
+    CHECK(check_tensor(p->b_scale, fdt, 2, b3));
+    CHECK(check_tensor(p->w_shift, fdt, 3, w3));
+    CHECK(check_tensor(p->w_residual_gate, fdt, 3, w2));
+    CHECK(check_tensor(p->b_residual_gate, fdt, 2, b2));
+    CHECK(check_tensor(p->b_q, fdt, 1, bq));
+    CHECK(check_tensor(p->pair_scale, fdt, 1, ps));
+    CHECK(check_tensor(p->w_pair, fdt, 2, wp));
+    if (P > kPairMax) return ATOMENC_ERR_UNSUPPORTED;
+  } else {
+    const int64_t rp[] = {B, A, D}, wm[] = {S, 6, C};
+    CHECK(check_tensor(in->rope_cos, fdt, 3, rp));
+    CHECK(check_tensor(in->rope_sin, fdt, 3, rp));
+    CHECK(check_tensor(p->w_mod, fdt, 3, wm));
+  }
+  if (pl.enc) {
+    const int64_t cu[] = {C, U}, tu[] = {B, T, U};
+    CHECK(check_tensor(p->w_pool, fdt, 2, cu));
+    CHECK(check_tensor(out->token_output, fdt, 3, tu));
+  } else {
+    const int64_t tv[] = {B, T, V}, vc[] = {V, C}, c1[] = {C}, c3[] = {C, 3}, a3[] = {B, A, 3};
+    CHECK(check_tensor(in->token, fdt, 3, tv));
+    CHECK(check_tensor(p->w_token, fdt, 2, vc));
+    CHECK(check_tensor(p->readout_scale, fdt, 1, c1));
+    if (!pl.af3) CHECK(check_tensor(p->readout_bias, fdt, 1, c1));
+    CHECK(check_tensor(p->w_readout, fdt, 2, c3));
+    CHECK(check_tensor(out->position_update, fdt, 3, a3));
+  }
+  {
+    const int64_t hc[] = {B, A, C}, at[] = {B, H, A, K};
+    CHECK(check_tensor(out->hidden, fdt, 3, hc));
+    CHECK(check_tensor(out->attention, fdt, 4, at));
+  }
+  if (D > kMaxD || A >= INT_MAX || K >= INT_MAX / 64) return ATOMENC_ERR_UNSUPPORTED;
+
+  // ---- workspace plan
+  const int64_t R = B * A;
+  size_t cur = 0;
+  pl.o_status = take(cur, 256);
+  pl.o_usable = take(cur, R);
+  pl.o_first = take(cur, pl.enc ? B * T * 4 : 0);
+  pl.o_last = take(cur, pl.enc ? B * T * 4 : 0);
+  pl.o_tp = take(cur, pl.enc ? 0 : B * T * C * 4);
+  pl.o_x = take(cur, R * C * 4);
+  pl.o_opc = take(cur, R * S * 4);
+  pl.o_rawc = take(cur, pl.af3 ? R * S * 4 : 0);
+  pl.o_cond = take(cur, R * 6 * C * 4);
+  pl.o_gate = take(cur, pl.af3 ? R * 2 * C * 4 : 0);
+  pl.o_feat = take(cur, R * (pl.af3 ? 2 : 1) * C * 4);
+  pl.o_q = take(cur, R * HD * 4);
+  pl.o_k = take(cur, R * HD * 4);
+  pl.o_v = take(cur, R * HD * 4);
+  pl.o_g = take(cur, R * HD * 4);
+  pl.o_o = take(cur, R * HD * 4);
+  pl.o_xp = take(cur, R * C * 4);
+  pl.o_z = take(cur, R * C * 4);
+  pl.o_h = take(cur, R * M * 4);
+  pl.o_hid = take(cur, R * C * 4);
+  pl.o_pool = take(cur, pl.enc ? R * U * 4 : 0);
+  pl.o_wcond = take(cur, S * 6 * C * 4);
+  pl.o_wgate = take(cur, pl.af3 ? S * 2 * C * 4 : 0);
+  pl.o_wqkv = take(cur, C * 4 * HD * 4);
+  pl.o_wout = take(cur, HD * C * 4);
+  pl.o_wff1 = take(cur, C * 2 * M * 4);
+  pl.o_wff2 = take(cur, M * C * 4);
+  pl.o_wpool = take(cur, pl.enc ? C * U * 4 : 0);
+  pl.o_wtok = take(cur, pl.enc ? 0 : V * C * 4);
+  pl.o_wread = take(cur, pl.enc ? 0 : C * 3 * 4);
+  pl.o_bscale = take(cur, pl.af3 ? 3 * C * 4 : 0);
+  pl.o_brg = take(cur, pl.af3 ? 2 * C * 4 : 0);
+  pl.o_bq = take(cur, pl.af3 ? HD * 4 : 0);
+  pl.o_wpair = take(cur, pl.af3 ? P * H * 4 : 0);
+  pl.o_rscale = take(cur, pl.enc ? 0 : C * 4);
+  pl.o_rbias = take(cur, pl.enc ? 0 : C * 4);
+  pl.bytes = cur;
+
+  // ---- attention tile: QT queries per CTA; stage as many K/V rows as fit
+  int dp = (int)((D + 3) / 4 * 4);
+  if ((dp / 4) % 2 == 0) dp += 4;  // odd number of 16-byte chunks per row: no bank conflicts
+  pl.DP = dp;
+  int qt = pl.af3 ? 16 : 32;
+  for (;;) {
+    size_t fixed = (size_t)qt * K * 4 + (pl.af3 ? (size_t)qt * K * H * 4 : 0) +
+                   (size_t)kAttnWarps * K * 4 + 64;
+    long cap = fixed < kAttnSmemBudget ? (long)((kAttnSmemBudget - fixed) / (2 * 4 * (size_t)dp)) : 0;
+    if (cap >= 64 || qt == 1) {
+      if (fixed > 200 * 1024) return ATOMENC_ERR_UNSUPPORTED;
+      pl.QT = qt;
+      pl.cap = (int)(cap < 0 ? 0 : cap);
+      pl.attn_smem = fixed + (size_t)pl.cap * 2 * 4 * dp;
+      break;
+    }
+    qt /= 2;
+  }
+  return ATOMENC_OK;
+}
+
+struct Hooks {
+  cudaEvent_t const *ev = nullptr;  // ATOMENC_NUM_PHASES + 1 events, or null
+  int launches = 0;
+  void mark(int i, cudaStream_t st) const {
+    if (ev) cudaEventRecord(ev[i], st);
+  }
+};
+
+template <typename Elt>
+int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p,
+               float eps, int64_t radius, const atomenc_outputs *out, unsigned char *ws,
+               cudaStream_t st, Hooks &hk) {
+  const Dims &d = pl.d;
+  const int64_t B = d.B, A = d.A, T = d.T, K = d.K, C = d.C, S = d.S, H = d.H, D = d.D,
+                P = d.P, M = d.M, U = d.U, V = d.V, HD = H * D, R = B * A;
+  auto F = [&](size_t off) { return reinterpret_cast<float *>(ws + off); };
+  unsigned *status = reinterpret_cast<unsigned *>(ws + pl.o_status);
+  uint8_t *usable = ws + pl.o_usable;
+  int *first = reinterpret_cast<int *>(ws + pl.o_first);
+  int *last = reinterpret_cast<int *>(ws + pl.o_last);
+
+  hk.mark(0, st);
+  cudaMemsetAsync(status, 0, 4, st);
+  if (pl.enc) {
+    cudaMemsetAsync(first, 0x7F, B * T * 4, st);
+    cudaMemsetAsync(last, 0xFF, B * T * 4, st);
+  }
+
+  // ---- weights into float32 panels
+  CopyJobs jobs;
+  std::memset(&jobs, 0, sizeof(jobs));
+  auto job = [&](const atomenc_tensor &src, size_t src_off_elems, int64_t rows, int64_t cols,
+                 size_t dst_off, int64_t dst_ld, int64_t col0, int64_t cstride,
+                 const atomenc_tensor *rowscale, size_t rs_off) {
+    CopyJob &j = jobs.job[jobs.n++];
+    const size_t es = sizeof(Elt);
+    j.src = static_cast<const unsigned char *>(src.data) + src_off_elems * es;
+    j.rowscale = rowscale ? static_cast<const unsigned char *>(rowscale->data) + rs_off * es : nullptr;
+    j.dst = F(dst_off);
+    j.rows = (int32_t)rows;
+    j.cols = (int32_t)cols;
+    j.dst_ld = (int32_t)dst_ld;
+    j.dst_col0 = (int32_t)col0;
+    j.dst_cstride = (int32_t)cstride;
+  };
+  if (pl.af3) {
+    for (int jj = 0; jj < 3; ++jj) {
+      job(p->w_scale, (size_t)jj * S * C, S, C, pl.o_wcond, 6 * C, 2 * jj * C, 1, &p->cond_scale, (size_t)jj * S);
+      job(p->w_shift, (size_t)jj * S * C, S, C, pl.o_wcond, 6 * C, 2 * jj * C + C, 1, &p->cond_scale, (size_t)jj * S);
+    }
+    job(p->w_residual_gate, 0, S, C, pl.o_wgate, 2 * C, 0, 1, nullptr, 0);
+    job(p->w_residual_gate, (size_t)S * C, S, C, pl.o_wgate, 2 * C, C, 1, nullptr, 0);
+    job(p->w_q, 0, C, HD, pl.o_wqkv, 2 * HD, 0, 1, nullptr, 0);
+    job(p->w_value_gate, 0, C, HD, pl.o_wqkv, 2 * HD, HD, 1, nullptr, 0);
+    job(p->w_k, 0, C, HD, pl.o_wqkv + (size_t)C * 2 * HD * 4, 2 * HD, 0, 1, nullptr, 0);
+    job(p->w_v, 0, C, HD, pl.o_wqkv + (size_t)C * 2 * HD * 4, 2 * HD, HD, 1, nullptr, 0);
+    job(p->b_scale, 0, 1, 3 * C, pl.o_bscale, 3 * C, 0, 1, nullptr, 0);
+    job(p->b_residual_gate, 0, 1, 2 * C, pl.o_brg, 2 * C, 0, 1, nullptr, 0);
+    job(p->b_q, 0, 1, HD, pl.o_bq, HD, 0, 1, nullptr, 0);
+    job(p->w_pair, 0, P, H, pl.o_wpair, H, 0, 1, &p->pair_scale, 0);
+  } else {
+    job(p->w_mod, 0, S, 6 * C, pl.o_wcond, 6 * C, 0, 1, nullptr, 0);
+    job(p->w_q, 0, C, HD, pl.o_wqkv, 4 * HD, 0, 1, nullptr, 0);
+    job(p->w_k, 0, C, HD, pl.o_wqkv, 4 * HD, HD, 1, nullptr, 0);
+    job(p->w_v, 0, C, HD, pl.o_wqkv, 4 * HD, 2 * HD, 1, nullptr, 0);
+    job(p->w_value_gate, 0, C, HD, pl.o_wqkv, 4 * HD, 3 * HD, 1, nullptr, 0);
+  }
+  job(p->w_attention_out, 0, HD, C, pl.o_wout, C, 0, 1, nullptr, 0);
+  job(p->w_ff_gate, 0, C, M, pl.o_wff1, 2 * M, 0, 2, nullptr, 0);
+  job(p->w_ff_up, 0, C, M, pl.o_wff1, 2 * M, 1, 2, nullptr, 0);
+  job(p->w_ff_out, 0, M, C, pl.o_wff2, C, 0, 1, nullptr, 0);
+  if (pl.enc) {
+    job(p->w_pool, 0, C, U, pl.o_wpool, U, 0, 1, nullptr, 0);
+  } else {
+    job(p->w_token, 0, V, C, pl.o_wtok, C, 0, 1, nullptr, 0);
+    job(p->readout_scale, 0, 1, C, pl.o_rscale, C, 0, 1, nullptr, 0);
+    if (!pl.af3) job(p->readout_bias, 0, 1, C, pl.o_rbias, C, 0, 1, nullptr, 0);
+    job(p->w_readout, 0, C, 3, pl.o_wread, 3, 0, 1, nullptr, 0);
+  }
+  k_prep_weights<Elt><<<dim3(64, jobs.n), 256, 0, st>>>(jobs);
+  ++hk.launches;
+
+  auto gemm = [&](auto *A_, int64_t lda, const float *W, int64_t ldw, int64_t Mr, int64_t N,
+                  int64_t Kd, auto epi) {
+    dim3 grid((unsigned)((N + kGemmBN - 1) / kGemmBN), (unsigned)((Mr + kGemmBM - 1) / kGemmBM));
+    k_gemm_simt<<<grid, kGemmThreads, 0, st>>>(A_, lda, W, ldw, Mr, N, Kd, epi);
+    ++hk.launches;
+  };
+  const int rows_per_block = 8;  // warps per 256-thread block for warp-per-row kernels
+  const unsigned row_blocks = (unsigned)((R + rows_per_block - 1) / rows_per_block);
+
+  // ---- decoder: token @ w_token, gathered per atom in the row pass
+  if (!pl.enc)
+    gemm(static_cast<const Elt *>(in->token.data), V, F(pl.o_wtok), C, B * T, C, V,
+         Quad<EpiStore>{{F(pl.o_tp), C}});
+
+  // ---- usable, sanitised residual start, normalised condition
+  RowsArgs ra;
+  ra.B = B; ra.A = A; ra.T = T; ra.C = C; ra.S = S; ra.eps = eps;
+  ra.af3 = pl.af3; ra.decoder = !pl.enc; ra.encoder = pl.enc;
+  ra.atom = in->atom.data; ra.condition = in->condition.data;
+  ra.valid = static_cast<const uint8_t *>(in->valid.data);
+  ra.token_valid = static_cast<const uint8_t *>(in->token_valid.data);
+  ra.att = static_cast<const int64_t *>(in->atom_to_token.data);
+  ra.token_proj = F(pl.o_tp);
+  ra.usable = usable; ra.x = F(pl.o_x); ra.opc = F(pl.o_opc); ra.rawc = F(pl.o_rawc);
+  ra.tok_first = first; ra.tok_last = last;
+  k_rows_prep<Elt><<<row_blocks, 256, 0, st>>>(ra);
+  ++hk.launches;
+  hk.mark(1, st);
+
+  // ---- conditioning
+  if (pl.af3) {
+    gemm(F(pl.o_opc), S, F(pl.o_wcond), 6 * C, R, 6 * C, S,
+         Quad<EpiCondAF3>{{F(pl.o_cond), F(pl.o_bscale), C}});
+    gemm(F(pl.o_rawc), S, F(pl.o_wgate), 2 * C, R, 2 * C, S,
+         Quad<EpiGateAF3>{{F(pl.o_gate), F(pl.o_brg), C}});
+  } else {
+    gemm(F(pl.o_opc), S, F(pl.o_wcond), 6 * C, R, 6 * C, S, Quad<EpiStore>{{F(pl.o_cond), 6 * C}});
+  }
+  hk.mark(2, st);
+  FeatArgs fa{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_x), F(pl.o_cond), F(pl.o_feat)};
+  k_features<<<row_blocks, 256, 0, st>>>(fa);
+  ++hk.launches;
+
+  // ---- projections
+  if (pl.af3) {
+    EpiSplit e0{{F(pl.o_q), F(pl.o_g), nullptr, nullptr}, {F(pl.o_bq), nullptr, nullptr, nullptr}, HD};
+    gemm(F(pl.o_feat), 2 * C, F(pl.o_wqkv), 2 * HD, R, 2 * HD, C, Quad<EpiSplit>{e0});
+    EpiSplit e1{{F(pl.o_k), F(pl.o_v), nullptr, nullptr}, {nullptr, nullptr, nullptr, nullptr}, HD};
+    gemm(F(pl.o_feat) + C, 2 * C, F(pl.o_wqkv + (size_t)C * 2 * HD * 4), 2 * HD, R, 2 * HD, C,
+         Quad<EpiSplit>{e1});
+  } else {
+    EpiSplit e{{F(pl.o_q), F(pl.o_k), F(pl.o_v), F(pl.o_g)}, {nullptr, nullptr, nullptr, nullptr}, HD};
+    gemm(F(pl.o_feat), C, F(pl.o_wqkv), 4 * HD, R, 4 * HD, C, Quad<EpiSplit>{e});
+    RopeArgs rp{R, H, D, eps, usable, in->rope_cos.data, in->rope_sin.data, F(pl.o_q), F(pl.o_k)};
+    const int64_t n = R * H * 2;
+    k_qk_rope<Elt><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(rp);
+    ++hk.launches;
+  }
+  hk.mark(3, st);
+
+  // ---- slot-gathered attention
+  AttnArgs ag;
+  ag.B = B; ag.A = A; ag.K = K; ag.H = H; ag.D = D; ag.P = P; ag.radius = radius;
+  ag.inv_sqrt_d = (float)(1.0 / std::sqrt((double)D));
+  ag.eps = eps;
+  ag.QT = pl.QT; ag.cap_rows = pl.cap; ag.DP = pl.DP;
+  ag.Q = F(pl.o_q); ag.Kf = F(pl.o_k); ag.Vf = F(pl.o_v); ag.G = F(pl.o_g);
+  ag.key_index = static_cast<const int64_t *>(in->key_index.data);
+  ag.window = static_cast<const uint8_t *>(in->window_mask.data);
+  ag.usable = usable;
+  ag.pair = pl.af3 ? in->pair.data : nullptr;
+  ag.w_pair = F(pl.o_wpair);
+  ag.attention = out->attention.data;
+  ag.O = F(pl.o_o);
+  ag.status = status;
+  {
+    dim3 grid((unsigned)((A + pl.QT - 1) / pl.QT), (unsigned)B);
+    auto go = [&](auto kern) {
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.attn_smem);
+      kern<<<grid, kAttnThreads, pl.attn_smem, st>>>(ag);
+      ++hk.launches;
+    };
+    const int dm = D <= 8 ? 8 : D <= 16 ? 16 : D <= 32 ? 32 : 64;
+    if (pl.af3) {
+      if (dm == 8) go(k_slot_attention<Elt, 8, true>);
+      else if (dm == 16) go(k_slot_attention<Elt, 16, true>);
+      else if (dm == 32) go(k_slot_attention<Elt, 32, true>);
+      else go(k_slot_attention<Elt, 64, true>);
+    } else {
+      if (dm == 8) go(k_slot_attention<Elt, 8, false>);
+      else if (dm == 16) go(k_slot_attention<Elt, 16, false>);
+      else if (dm == 32) go(k_slot_attention<Elt, 32, false>);
+      else go(k_slot_attention<Elt, 64, false>);
+    }
+  }
+
+  hk.mark(4, st);
+
+  // ---- out-projection + gated residual: x' = x + g_attn * (o @ w_attention_out)
+  const float *gbuf = pl.af3 ? F(pl.o_gate) : F(pl.o_cond);
+  const int64_t gld = pl.af3 ? 2 * C : 6 * C;
+  const int64_t g0off = pl.af3 ? 0 : 2 * C, g1off = pl.af3 ? C : 5 * C;
+  gemm(F(pl.o_o), HD, F(pl.o_wout), C, R, C, HD,
+       Quad<EpiResidual>{{F(pl.o_x), gbuf, gld, g0off, C, F(pl.o_xp)}});
+
+  // ---- transition on the new state
+  TNormArgs ta{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_xp), F(pl.o_cond), F(pl.o_z)};
+  k_transition_norm<<<row_blocks, 256, 0, st>>>(ta);
+  ++hk.launches;
+  gemm(F(pl.o_z), C, F(pl.o_wff1), 2 * M, R, 2 * M, C, EpiSwiGLU{F(pl.o_h), M});
+  gemm(F(pl.o_h), M, F(pl.o_wff2), C, R, C, M,
+       Quad<EpiHidden<Elt>>{{F(pl.o_xp), gbuf, gld, g1off, C, usable, F(pl.o_hid),
+                           static_cast<Elt *>(out->hidden.data)}});
+
+  hk.mark(5, st);
+
+  // ---- boundary
+  if (pl.enc) {
+    gemm(F(pl.o_hid), C, F(pl.o_wpool), U, R, U, C, Quad<EpiRelu>{{F(pl.o_pool), U}});
+    PoolArgs pa{B, A, T, U, usable, static_cast<const int64_t *>(in->atom_to_token.data), first,
+                last, F(pl.o_pool), out->token_output.data};
+    k_token_mean<Elt><<<(unsigned)(B * T), 128, 0, st>>>(pa);
+    ++hk.launches;
+  } else {
+    ReadoutArgs rd{R, C, eps, pl.af3 ? 0 : 1, usable, F(pl.o_hid), F(pl.o_rscale), F(pl.o_rbias),
+                   F(pl.o_wread), out->position_update.data};
+    k_readout<Elt><<<row_blocks, 256, 0, st>>>(rd);
+    ++hk.launches;
+  }
+  hk.mark(6, st);
+  return cudaGetLastError() == cudaSuccess ? ATOMENC_OK : ATOMENC_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t atomenc_workspace_size(int style, int stage, const atomenc_inputs *in,
+                              const atomenc_params *params, const atomenc_outputs *out) {
+  Plan pl;
+  if (validate(style, stage, in, params, out, pl) != ATOMENC_OK) return 0;
+  return pl.bytes;
+}
+
+static int forward_impl(int style, int stage, const atomenc_inputs *in,
+                        const atomenc_params *params, double eps, int64_t radius,
+                        const atomenc_outputs *out, void *workspace, size_t workspace_bytes,
+                        atomenc_stream_t stream, Hooks &hk) {
+  Plan pl;
+  CHECK(validate(style, stage, in, params, out, pl));
+  if (!std::isfinite(eps) || !(eps > 0.0)) return ATOMENC_ERR_EPS;
+  float feps = (float)eps;
+  if (!(feps > 0.f) || !std::isfinite(feps)) return ATOMENC_ERR_EPS;
+  if (pl.fdt == ATOMENC_BF16 && !(bf16_round_host(feps) > 0.f)) return ATOMENC_ERR_EPS;
+  if (radius < -1) return ATOMENC_ERR_RADIUS;
+  if (!workspace || workspace_bytes < pl.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return ATOMENC_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char *ws = static_cast<unsigned char *>(workspace);
+  if (pl.fdt == ATOMENC_F32) return launch_all<float>(pl, in, params, feps, radius, out, ws, st, hk);
+  return launch_all<__nv_bfloat16>(pl, in, params, feps, radius, out, ws, st, hk);
+}
+
+int atomenc_forward(int style, int stage, const atomenc_inputs *in, const atomenc_params *params,
+                    double eps, int64_t radius, const atomenc_outputs *out, void *workspace,
+                    size_t workspace_bytes, atomenc_stream_t stream) {
+  Hooks hk;
+  return forward_impl(style, stage, in, params, eps, radius, out, workspace, workspace_bytes,
+                      stream, hk);
+}
+
+int atomenc_forward_profiled(int style, int stage, const atomenc_inputs *in,
+                             const atomenc_params *params, double eps, int64_t radius,
+                             const atomenc_outputs *out, void *workspace, size_t workspace_bytes,
+                             atomenc_stream_t stream, void *const *events, int n_events,
+                             int *n_launches) {
+  if (!events || n_events != ATOMENC_NUM_PHASES + 1) return ATOMENC_ERR_NULL;
+  for (int i = 0; i < n_events; ++i)
+    if (!events[i]) return ATOMENC_ERR_NULL;
+  Hooks hk;
+  hk.ev = reinterpret_cast<cudaEvent_t const *>(events);
+  int rc = forward_impl(style, stage, in, params, eps, radius, out, workspace, workspace_bytes,
+                        stream, hk);
+  if (n_launches) *n_launches = hk.launches;
+  return rc;
+}
+
+int atomenc_get_status(const void *workspace, int *device_status, atomenc_stream_t stream) {
+  if (!workspace || !device_status) return ATOMENC_ERR_NULL;
+  unsigned v = 0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return ATOMENC_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ATOMENC_ERR_CUDA;
+  *device_status = (int)v;
+  return ATOMENC_OK;
+}
+
+const char *atomenc_strerror(int code) {
+  switch (code) {
+    case ATOMENC_OK: return "ok";
+    case ATOMENC_ERR_NULL: return "a required tensor, pointer or struct is missing";
+    case ATOMENC_ERR_STYLE: return "unknown style or stage";
+    case ATOMENC_ERR_DTYPE: return "element types disagree (floats must match; int64 indices; bool masks)";
+    case ATOMENC_ERR_SHAPE: return "tensor ranks or sizes disagree, or a dimension is < 1";
+    case ATOMENC_ERR_STRIDE: return "a tensor is not dense row-major";
+    case ATOMENC_ERR_EPS: return "eps must be finite and > 0 in the float type";
+    case ATOMENC_ERR_RADIUS: return "radius must be -1 or >= 0";
+    case ATOMENC_ERR_ODD_HEAD: return "ESMFold2 style needs an even head width D";
+    case ATOMENC_ERR_UNSUPPORTED: return "a size is outside what the kernels are built for";
+    case ATOMENC_ERR_WORKSPACE: return "workspace is NULL, too small or not 256-byte aligned";
+    case ATOMENC_ERR_CUDA: return "the CUDA runtime rejected a launch";
+    default: return "unknown atomenc status";
+  }
+}
+
+int atomenc_version(void) { return kVersion; }
+
+}  // extern "C"

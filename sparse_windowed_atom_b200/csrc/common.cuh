@@ -1,0 +1,53 @@
+// common.cuh -- device helpers shared by the atomenc kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace atomenc {
+
+constexpr int kWarp = 32;
+
+// ---- element access: every float tensor is float32 or bf16 in memory, float32 in math
+__device__ __forceinline__ float ldf(const float *p, int64_t i) { return p[i]; }
+__device__ __forceinline__ float ldf(const __nv_bfloat16 *p, int64_t i) {
+  return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void stf(float *p, int64_t i, float v) { p[i] = v; }
+__device__ __forceinline__ void stf(__nv_bfloat16 *p, int64_t i, float v) {
+  p[i] = __float2bfloat16_rn(v);
+}
+
+// ---- activations (no fast-math: IEEE division, expf, subnormals kept)
+// sigmoid(z) = 1 / (1 + e^-z); for z < 0 the same value as e^z / (1 + e^z) so that a
+// representable subnormal tail is not flushed by an overflowing e^-z.
+__device__ __forceinline__ float sigmoidf_(float z) {
+  if (z >= 0.f) return 1.f / (1.f + expf(-z));
+  float e = expf(z);
+  return e / (1.f + e);
+}
+__device__ __forceinline__ float siluf_(float z) { return z * sigmoidf_(z); }
+
+// ---- warp reductions
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// usable iff valid, 0 <= atom_to_token < T and the mapped token is valid
+__device__ __forceinline__ bool atom_usable(const uint8_t *valid, const int64_t *att,
+                                            const uint8_t *token_valid, int64_t b,
+                                            int64_t a, int64_t A, int64_t T) {
+  int64_t i = b * A + a;
+  int64_t t = att[i];
+  return valid[i] != 0 && t >= 0 && t < T && token_valid[b * T + t] != 0;
+}
+
+}  // namespace atomenc

@@ -1,0 +1,302 @@
+// rows.cuh -- per-row (atom / token) kernels: masking, sanitisation, normalisation,
+// rotary, pooling and readout. Each kernel cites the passage of the page "Local atom
+// attention, encoder pooling and decoder skip/readout" (Required behavior) it follows.
+#pragma once
+
+#include "common.cuh"
+
+namespace atomenc {
+
+// ------------------------------------------------------------------ weight preparation
+// The block's weights are re-laid out once per call into float32 panels that the
+// projection kernels read: the AF3 cond_scale[j] is folded into w_scale[j] / w_shift[j]
+// (c_j @ W = LN(c) @ (diag(cond_scale[j]) W)), projections that share an input are
+// concatenated along N, and the SwiGLU gate/up weights are interleaved column-wise.
+struct CopyJob {
+  const void *src;       // [rows, cols] dense
+  const void *rowscale;  // optional [rows], same element type as src
+  float *dst;
+  int32_t rows, cols;
+  int32_t dst_ld, dst_col0, dst_cstride;
+  int32_t pad;
+};
+constexpr int kMaxCopyJobs = 28;
+struct CopyJobs {
+  CopyJob job[kMaxCopyJobs];
+  int n;
+};
+
+template <typename T>
+__global__ void k_prep_weights(CopyJobs jobs) {
+  const CopyJob &j = jobs.job[blockIdx.y];
+  const int64_t total = (int64_t)j.rows * j.cols;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    int64_t r = i / j.cols, c = i % j.cols;
+    float v = ldf((const T *)j.src, i);
+    if (j.rowscale) v *= ldf((const T *)j.rowscale, r);
+    j.dst[r * j.dst_ld + j.dst_col0 + c * j.dst_cstride] = v;
+  }
+}
+
+// ------------------------------------------------------------------ row preparation
+struct RowsArgs {
+  int64_t B, A, T, C, S;
+  float eps;
+  int af3, decoder, encoder;
+  const void *atom, *condition;
+  const uint8_t *valid, *token_valid;
+  const int64_t *att;
+  const float *token_proj;  // [B*T, C] decoder: token @ w_token
+  uint8_t *usable;          // [B*A]
+  float *x;                 // [B*A, C] residual state start
+  float *opc;               // [B*A, S] AF3: LN(c); ESMFold2: SiLU(c)
+  float *rawc;              // [B*A, S] AF3: sanitised raw condition
+  int *tok_first, *tok_last;  // [B*T] encoder pooling ranges
+};
+
+// One warp per atom. usable = valid & 0 <= atom_to_token < T & token_valid  (bullet 2);
+// payloads of unusable atoms are replaced by zero with a select before any arithmetic
+// (bullet 3); encoder x = atom, decoder x = skip + gather(token @ w_token) (bullet 3).
+template <typename T>
+__global__ void k_rows_prep(RowsArgs r) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= r.B * r.A) return;
+  const int64_t b = row / r.A, a = row % r.A;
+  const bool use = atom_usable(r.valid, r.att, r.token_valid, b, a, r.A, r.T);
+  const int64_t t = use ? r.att[row] : 0;
+  if (lane == 0) {
+    r.usable[row] = use ? 1 : 0;
+    if (use && r.encoder) {
+      atomicMin(r.tok_first + b * r.T + t, (int)a);
+      atomicMax(r.tok_last + b * r.T + t, (int)a);
+    }
+  }
+  const T *atom = (const T *)r.atom + row * r.C;
+  for (int64_t c = lane; c < r.C; c += kWarp) {
+    float v = 0.f;
+    if (use) {
+      v = ldf(atom, c);
+      if (r.decoder) v += r.token_proj[(b * r.T + t) * r.C + c];
+    }
+    r.x[row * r.C + c] = v;
+  }
+  const T *cond = (const T *)r.condition + row * r.S;
+  if (r.af3) {
+    // population LayerNorm of the condition, eps inside the root (bullet 7)
+    float s = 0.f;
+    for (int64_t k = lane; k < r.S; k += kWarp) s += use ? ldf(cond, k) : 0.f;
+    const float mean = warp_sum(s) / (float)r.S;
+    float q = 0.f;
+    for (int64_t k = lane; k < r.S; k += kWarp) {
+      float d = (use ? ldf(cond, k) : 0.f) - mean;
+      q += d * d;
+    }
+    const float rstd = 1.f / sqrtf(warp_sum(q) / (float)r.S + r.eps);
+    for (int64_t k = lane; k < r.S; k += kWarp) {
+      float v = use ? ldf(cond, k) : 0.f;
+      r.rawc[row * r.S + k] = v;
+      r.opc[row * r.S + k] = (v - mean) * rstd;
+    }
+  } else {
+    // SiLU(condition) feeds w_mod (bullet 10)
+    for (int64_t k = lane; k < r.S; k += kWarp) {
+      float v = use ? ldf(cond, k) : 0.f;
+      r.opc[row * r.S + k] = siluf_(v);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ attention inputs
+struct FeatArgs {
+  int64_t rows, C;
+  float eps;
+  int af3;
+  const float *x;     // [rows, C]
+  const float *cond;  // AF3 [rows, 6C] = (sig(scale_j + b), shift_j) j=0..2; ESM [rows, 6C] raw
+  float *feat;        // AF3 [rows, 2C] = (A_0(x), A_1(x)); ESM [rows, C] attention input
+};
+
+// AF3: A_j(x) = LN(x) * sigmoid(c_j @ w_scale[j] + b_scale[j]) + c_j @ w_shift[j]  (bullet 7)
+// ESM: attention input = RMS(x) * (1 + attention_scale) + attention_shift  (bullet 11)
+__global__ void k_features(FeatArgs f) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= f.rows) return;
+  const float *x = f.x + row * f.C;
+  const float *cd = f.cond + row * 6 * f.C;
+  if (f.af3) {
+    float s = 0.f;
+    for (int64_t c = lane; c < f.C; c += kWarp) s += x[c];
+    const float mean = warp_sum(s) / (float)f.C;
+    float q = 0.f;
+    for (int64_t c = lane; c < f.C; c += kWarp) q += (x[c] - mean) * (x[c] - mean);
+    const float rstd = 1.f / sqrtf(warp_sum(q) / (float)f.C + f.eps);
+    for (int64_t c = lane; c < f.C; c += kWarp) {
+      float ln = (x[c] - mean) * rstd;
+      f.feat[row * 2 * f.C + c] = ln * cd[c] + cd[f.C + c];
+      f.feat[row * 2 * f.C + f.C + c] = ln * cd[2 * f.C + c] + cd[3 * f.C + c];
+    }
+  } else {
+    float q = 0.f;
+    for (int64_t c = lane; c < f.C; c += kWarp) q += x[c] * x[c];
+    const float rstd = 1.f / sqrtf(warp_sum(q) / (float)f.C + f.eps);
+    for (int64_t c = lane; c < f.C; c += kWarp)
+      f.feat[row * f.C + c] = x[c] * rstd * (1.f + cd[f.C + c]) + cd[c];
+  }
+}
+
+// ------------------------------------------------------------------ ESMFold2 Q/K head norm + rotary
+struct RopeArgs {
+  int64_t rows, H, D;
+  float eps;
+  const uint8_t *usable;
+  const void *cos, *sin;  // [rows, D]
+  float *Q, *K;           // [rows, H*D], rewritten in place
+};
+
+// Per-head RMS of Q and K over D, then q * cos + rotate_half(q) * sin with
+// rotate_half([q1, q2]) = [-q2, q1], before keys are gathered (bullets 12, 13).
+// One thread per (atom, head, Q-or-K); D <= 128.
+template <typename T>
+__global__ void k_qk_rope(RopeArgs r) {
+  const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= r.rows * r.H * 2) return;
+  const int which = (int)(id & 1);
+  const int64_t rh = id >> 1;
+  const int64_t row = rh / r.H, h = rh % r.H;
+  float *v = (which ? r.K : r.Q) + row * r.H * r.D + h * r.D;
+  const bool use = r.usable[row] != 0;
+  float buf[128];
+  float ss = 0.f;
+  for (int d = 0; d < r.D; ++d) {
+    buf[d] = v[d];
+    ss += buf[d] * buf[d];
+  }
+  const float rstd = 1.f / sqrtf(ss / (float)r.D + r.eps);
+  const T *cs = (const T *)r.cos + row * r.D;
+  const T *sn = (const T *)r.sin + row * r.D;
+  const int half = (int)(r.D / 2);
+  for (int d = 0; d < r.D; ++d) {
+    float qd = buf[d] * rstd;
+    float rot = d < half ? -buf[d + half] * rstd : buf[d - half] * rstd;
+    float c = use ? ldf(cs, d) : 0.f, s = use ? ldf(sn, d) : 0.f;
+    v[d] = use ? qd * c + rot * s : 0.f;
+  }
+}
+
+// ------------------------------------------------------------------ transition norm
+struct TNormArgs {
+  int64_t rows, C;
+  float eps;
+  int af3;
+  const float *xp;    // [rows, C] x' after the attention residual
+  const float *cond;  // [rows, 6C] as in FeatArgs
+  float *z;           // [rows, C]
+};
+
+// Normalise the NEW residual state: AF3 A_2(x'); ESMFold2
+// RMS(x') * (1 + transition_scale) + transition_shift  (bullet 17)
+__global__ void k_transition_norm(TNormArgs f) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= f.rows) return;
+  const float *x = f.xp + row * f.C;
+  const float *cd = f.cond + row * 6 * f.C;
+  if (f.af3) {
+    float s = 0.f;
+    for (int64_t c = lane; c < f.C; c += kWarp) s += x[c];
+    const float mean = warp_sum(s) / (float)f.C;
+    float q = 0.f;
+    for (int64_t c = lane; c < f.C; c += kWarp) q += (x[c] - mean) * (x[c] - mean);
+    const float rstd = 1.f / sqrtf(warp_sum(q) / (float)f.C + f.eps);
+    for (int64_t c = lane; c < f.C; c += kWarp)
+      f.z[row * f.C + c] = (x[c] - mean) * rstd * cd[4 * f.C + c] + cd[5 * f.C + c];
+  } else {
+    float q = 0.f;
+    for (int64_t c = lane; c < f.C; c += kWarp) q += x[c] * x[c];
+    const float rstd = 1.f / sqrtf(warp_sum(q) / (float)f.C + f.eps);
+    for (int64_t c = lane; c < f.C; c += kWarp)
+      f.z[row * f.C + c] = x[c] * rstd * (1.f + cd[4 * f.C + c]) + cd[3 * f.C + c];
+  }
+}
+
+// ------------------------------------------------------------------ encoder pooling
+struct PoolArgs {
+  int64_t B, A, T, U;
+  const uint8_t *usable;
+  const int64_t *att;
+  const int *tok_first, *tok_last;
+  const float *pooled;  // [B*A, U] ReLU(hidden @ w_pool)
+  void *out;            // [B, T, U]
+};
+
+// token_output[t] = exact mean of ReLU(hidden @ w_pool) over the usable atoms mapped
+// to t, summed in ascending atom order (deterministic); 0 for a token with none
+// (bullet 19). One block per token, one thread per output channel.
+template <typename T>
+__global__ void k_token_mean(PoolArgs p) {
+  const int64_t bt = blockIdx.x;
+  const int64_t b = bt / p.T, t = bt % p.T;
+  const int first = p.tok_first[bt], last = p.tok_last[bt];
+  for (int64_t u = threadIdx.x; u < p.U; u += blockDim.x) {
+    float acc = 0.f;
+    int n = 0;
+    for (int a = first; a <= last; ++a) {
+      const int64_t row = b * p.A + a;
+      if (p.usable[row] && p.att[row] == t) {
+        acc += p.pooled[row * p.U + u];
+        ++n;
+      }
+    }
+    stf((T *)p.out, bt * p.U + u, n > 0 ? acc / (float)n : 0.f);
+  }
+}
+
+// ------------------------------------------------------------------ decoder readout
+struct ReadoutArgs {
+  int64_t rows, C;
+  float eps;
+  int has_bias;
+  const uint8_t *usable;
+  const float *hid;        // [rows, C]
+  const float *scale;      // [C]
+  const float *bias;       // [C] ESMFold2
+  const float *w_readout;  // [C, 3]
+  void *out;               // [rows, 3]
+};
+
+// position_update = (LN(hidden) * readout_scale [+ readout_bias]) @ w_readout, masked
+// to zero; an update, not coordinates (bullets 18-20). One warp per atom.
+template <typename T>
+__global__ void k_readout(ReadoutArgs r) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= r.rows) return;
+  const float *x = r.hid + row * r.C;
+  float s = 0.f;
+  for (int64_t c = lane; c < r.C; c += kWarp) s += x[c];
+  const float mean = warp_sum(s) / (float)r.C;
+  float q = 0.f;
+  for (int64_t c = lane; c < r.C; c += kWarp) q += (x[c] - mean) * (x[c] - mean);
+  const float rstd = 1.f / sqrtf(warp_sum(q) / (float)r.C + r.eps);
+  float o0 = 0.f, o1 = 0.f, o2 = 0.f;
+  for (int64_t c = lane; c < r.C; c += kWarp) {
+    float y = (x[c] - mean) * rstd * r.scale[c] + (r.has_bias ? r.bias[c] : 0.f);
+    o0 += y * r.w_readout[c * 3 + 0];
+    o1 += y * r.w_readout[c * 3 + 1];
+    o2 += y * r.w_readout[c * 3 + 2];
+  }
+  o0 = warp_sum(o0);
+  o1 = warp_sum(o1);
+  o2 = warp_sum(o2);
+  if (lane == 0) {
+    const bool use = r.usable[row] != 0;
+    stf((T *)r.out, row * 3 + 0, use ? o0 : 0.f);
+    stf((T *)r.out, row * 3 + 1, use ? o1 : 0.f);
+    stf((T *)r.out, row * 3 + 2, use ? o2 : 0.f);
+  }
+}
+
+}  // namespace atomenc
