@@ -10,11 +10,13 @@
 #include <climits>
 #include <cmath>
 #include <cstring>
+#include <type_traits>
 
 #include "../../include/atomenc.h"
 #include "attention.cuh"
 #include "common.cuh"
-#include "gemm_simt.cuh"
+#include "epilogues.cuh"
+#include "gemm_umma.cuh"
 #include "rows.cuh"
 
 using namespace atomenc;
@@ -23,7 +25,7 @@ namespace {
 
 constexpr int kVersion = 1;
 constexpr int kMaxD = 64;
-constexpr size_t kAttnSmemBudget = 110 * 1024;
+constexpr size_t kAttnSmemBudget = 104 * 1024;  // two CTAs per SM
 
 struct Dims {
   int64_t B = 0, A = 0, T = 0, K = 0, C = 0, S = 0, H = 0, D = 0, P = 0, M = 0, U = 0, V = 0;
@@ -68,9 +70,11 @@ struct Plan {
       o_q, o_k, o_v, o_g, o_o, o_xp, o_z, o_h, o_hid, o_pool;
   size_t o_wcond, o_wgate, o_wqkv, o_wout, o_wff1, o_wff2, o_wpool, o_wtok, o_wread, o_bscale,
       o_brg, o_bq, o_wpair, o_rscale, o_rbias;
+  // tensor-core images of the weight panels (bf16, hi[/lo])
+  size_t k_cond, k_gate, k_qkv0, k_qkv1, k_out, k_ff1, k_ff2, k_pool, k_tok;
   size_t bytes = 0;
   // attention launch
-  int QT = 0, cap = 0, DP = 0;
+  int QT = 0, DP = 0, kv_floats = 0;
   size_t attn_smem = 0;
 };
 
@@ -167,7 +171,7 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
     CHECK(check_tensor(p->b_q, fdt, 1, bq));
     CHECK(check_tensor(p->pair_scale, fdt, 1, ps));
     CHECK(check_tensor(p->w_pair, fdt, 2, wp));
-    if (P > kPairMax) return ATOMENC_ERR_UNSUPPORTED;
+    if (P > kPairMax || H > kAttnHeadsMax) return ATOMENC_ERR_UNSUPPORTED;
   } else {
     const int64_t rp[] = {B, A, D}, wm[] = {S, 6, C};
     CHECK(check_tensor(in->rope_cos, fdt, 3, rp));
@@ -233,26 +237,30 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   pl.o_wpair = take(cur, pl.af3 ? P * H * 4 : 0);
   pl.o_rscale = take(cur, pl.enc ? 0 : C * 4);
   pl.o_rbias = take(cur, pl.enc ? 0 : C * 4);
+  const bool split = fdt == ATOMENC_F32;
+  pl.k_cond = take(cur, packed_bytes(S, 6 * C, split));
+  pl.k_gate = take(cur, pl.af3 ? packed_bytes(S, 2 * C, split) : 0);
+  pl.k_qkv0 = take(cur, packed_bytes(C, (pl.af3 ? 2 : 4) * HD, split));
+  pl.k_qkv1 = take(cur, pl.af3 ? packed_bytes(C, 2 * HD, split) : 0);
+  pl.k_out = take(cur, packed_bytes(HD, C, split));
+  pl.k_ff1 = take(cur, packed_bytes(C, 2 * M, split));
+  pl.k_ff2 = take(cur, packed_bytes(M, C, split));
+  pl.k_pool = take(cur, pl.enc ? packed_bytes(C, U, split) : 0);
+  pl.k_tok = take(cur, pl.enc ? 0 : packed_bytes(V, C, split));
   pl.bytes = cur;
 
-  // ---- attention tile: QT queries per CTA; stage as many K/V rows as fit
-  int dp = (int)((D + 3) / 4 * 4);
-  if ((dp / 4) % 2 == 0) dp += 4;  // odd number of 16-byte chunks per row: no bank conflicts
-  pl.DP = dp;
-  int qt = pl.af3 ? 16 : 32;
-  for (;;) {
-    size_t fixed = (size_t)qt * K * 4 + (pl.af3 ? (size_t)qt * K * H * 4 : 0) +
-                   (size_t)kAttnWarps * K * 4 + 64;
-    long cap = fixed < kAttnSmemBudget ? (long)((kAttnSmemBudget - fixed) / (2 * 4 * (size_t)dp)) : 0;
-    if (cap >= 64 || qt == 1) {
-      if (fixed > 200 * 1024) return ATOMENC_ERR_UNSUPPORTED;
-      pl.QT = qt;
-      pl.cap = (int)(cap < 0 ? 0 : cap);
-      pl.attn_smem = fixed + (size_t)pl.cap * 2 * 4 * dp;
-      break;
-    }
+  // ---- attention tile: QT queries per CTA (small enough that the grid covers the
+  // GPU twice over), a slot plan of QT*K ints and a K/V stage in the rest of the budget
+  const int dmax = D <= 8 ? 8 : D <= 16 ? 16 : D <= 32 ? 32 : 64;
+  pl.DP = dmax + 4;  // odd number of 16-byte chunks per staged row: no bank conflicts
+  int qt = 32;
+  while (qt > 1 && ((int64_t)B * ((A + qt - 1) / qt) < 2 * 148 || (int64_t)qt * K * 4 > 32768))
     qt /= 2;
-  }
+  pl.QT = qt;
+  const size_t plan_bytes = (((size_t)qt * K + 3) & ~size_t(3)) * 4;
+  if (plan_bytes + 16 * 1024 > kAttnSmemBudget) return ATOMENC_ERR_UNSUPPORTED;
+  pl.kv_floats = (int)((kAttnSmemBudget - plan_bytes) / 4);
+  pl.attn_smem = plan_bytes + (size_t)pl.kv_floats * 4;
   return ATOMENC_OK;
 }
 
@@ -338,10 +346,64 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   k_prep_weights<Elt><<<dim3(64, jobs.n), 256, 0, st>>>(jobs);
   ++hk.launches;
 
-  auto gemm = [&](auto *A_, int64_t lda, const float *W, int64_t ldw, int64_t Mr, int64_t N,
-                  int64_t Kd, auto epi) {
-    dim3 grid((unsigned)((N + kGemmBN - 1) / kGemmBN), (unsigned)((Mr + kGemmBM - 1) / kGemmBM));
-    k_gemm_simt<<<grid, kGemmThreads, 0, st>>>(A_, lda, W, ldw, Mr, N, Kd, epi);
+  // ---- tensor-core images of the panels
+  const bool split = pl.fdt == ATOMENC_F32;
+  PackJobs pj;
+  std::memset(&pj, 0, sizeof(pj));
+  auto pack = [&](size_t panel, int64_t Kd, int64_t N, int64_t ld, size_t dst) {
+    PackJob &j = pj.job[pj.n++];
+    j.src = F(panel);
+    j.dst = ws + dst;
+    j.K = (int32_t)Kd;
+    j.N = (int32_t)N;
+    j.ld = (int32_t)ld;
+    j.split = split ? 1 : 0;
+  };
+  pack(pl.o_wcond, S, 6 * C, 6 * C, pl.k_cond);
+  if (pl.af3) {
+    pack(pl.o_wgate, S, 2 * C, 2 * C, pl.k_gate);
+    pack(pl.o_wqkv, C, 2 * HD, 2 * HD, pl.k_qkv0);
+    pack(pl.o_wqkv + (size_t)C * 2 * HD * 4, C, 2 * HD, 2 * HD, pl.k_qkv1);
+  } else {
+    pack(pl.o_wqkv, C, 4 * HD, 4 * HD, pl.k_qkv0);
+  }
+  pack(pl.o_wout, HD, C, C, pl.k_out);
+  pack(pl.o_wff1, C, 2 * M, 2 * M, pl.k_ff1);
+  pack(pl.o_wff2, M, C, C, pl.k_ff2);
+  if (pl.enc) pack(pl.o_wpool, C, U, U, pl.k_pool);
+  else pack(pl.o_wtok, V, C, C, pl.k_tok);
+  k_pack_weights<<<dim3(64, pj.n), 256, 0, st>>>(pj);
+  ++hk.launches;
+
+  // out = epi(A @ W) on the tensor cores; W given by its packed image. K <= 256: the
+  // row-block kernel (A resident, weights streamed); larger K: the streaming kernel.
+  auto gemm = [&](auto *A_, int64_t lda, size_t wpk, int64_t Mr, int64_t N, int64_t Kd, auto epi) {
+    using TA = std::remove_cv_t<std::remove_pointer_t<decltype(A_)>>;
+    using E = decltype(epi);
+    const int64_t mt = (Mr + kUmmaBM - 1) / kUmmaBM, nt = (N + kUmmaBN - 1) / kUmmaBN;
+    if (Kd <= kRowsKMax) {
+      const int64_t want = (148 + mt - 1) / mt;           // CTAs per row block to fill the GPU
+      const int per = (int)((nt + (want < nt ? want : nt) - 1) / (want < nt ? want : nt));
+      dim3 grid((unsigned)((nt + per - 1) / per), (unsigned)mt);
+      const size_t smem = rows_smem_bytes(Kd, split);
+      if (split) {
+        cudaFuncSetAttribute(k_gemm_rows<TA, true, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k_gemm_rows<TA, true, E><<<grid, kRowsThreads, smem, st>>>(A_, lda, ws + wpk, Mr, N, Kd, per, epi, status);
+      } else {
+        cudaFuncSetAttribute(k_gemm_rows<TA, false, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k_gemm_rows<TA, false, E><<<grid, kRowsThreads, smem, st>>>(A_, lda, ws + wpk, Mr, N, Kd, per, epi, status);
+      }
+    } else {
+      dim3 grid((unsigned)nt, (unsigned)mt);
+      const size_t smem = umma_smem_bytes(split);
+      if (split) {
+        cudaFuncSetAttribute(k_gemm_umma<TA, true, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k_gemm_umma<TA, true, E><<<grid, kUmmaThreads, smem, st>>>(A_, lda, ws + wpk, Mr, N, Kd, epi, status);
+      } else {
+        cudaFuncSetAttribute(k_gemm_umma<TA, false, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k_gemm_umma<TA, false, E><<<grid, kUmmaThreads, smem, st>>>(A_, lda, ws + wpk, Mr, N, Kd, epi, status);
+      }
+    }
     ++hk.launches;
   };
   const int rows_per_block = 8;  // warps per 256-thread block for warp-per-row kernels
@@ -349,7 +411,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
 
   // ---- decoder: token @ w_token, gathered per atom in the row pass
   if (!pl.enc)
-    gemm(static_cast<const Elt *>(in->token.data), V, F(pl.o_wtok), C, B * T, C, V,
+    gemm(static_cast<const Elt *>(in->token.data), V, pl.k_tok, B * T, C, V,
          Quad<EpiStore>{{F(pl.o_tp), C}});
 
   // ---- usable, sanitised residual start, normalised condition
@@ -369,12 +431,12 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
 
   // ---- conditioning
   if (pl.af3) {
-    gemm(F(pl.o_opc), S, F(pl.o_wcond), 6 * C, R, 6 * C, S,
-         Quad<EpiCondAF3>{{F(pl.o_cond), F(pl.o_bscale), C}});
-    gemm(F(pl.o_rawc), S, F(pl.o_wgate), 2 * C, R, 2 * C, S,
-         Quad<EpiGateAF3>{{F(pl.o_gate), F(pl.o_brg), C}});
+    gemm(F(pl.o_opc), S, pl.k_cond, R, 6 * C, S,
+         EpiCondAF3{F(pl.o_cond), F(pl.o_bscale), C});
+    gemm(F(pl.o_rawc), S, pl.k_gate, R, 2 * C, S,
+         EpiGateAF3{F(pl.o_gate), F(pl.o_brg), C});
   } else {
-    gemm(F(pl.o_opc), S, F(pl.o_wcond), 6 * C, R, 6 * C, S, Quad<EpiStore>{{F(pl.o_cond), 6 * C}});
+    gemm(F(pl.o_opc), S, pl.k_cond, R, 6 * C, S, Quad<EpiStore>{{F(pl.o_cond), 6 * C}});
   }
   hk.mark(2, st);
   FeatArgs fa{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_x), F(pl.o_cond), F(pl.o_feat)};
@@ -384,13 +446,13 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   // ---- projections
   if (pl.af3) {
     EpiSplit e0{{F(pl.o_q), F(pl.o_g), nullptr, nullptr}, {F(pl.o_bq), nullptr, nullptr, nullptr}, HD};
-    gemm(F(pl.o_feat), 2 * C, F(pl.o_wqkv), 2 * HD, R, 2 * HD, C, Quad<EpiSplit>{e0});
+    gemm(F(pl.o_feat), 2 * C, pl.k_qkv0, R, 2 * HD, C, e0);
     EpiSplit e1{{F(pl.o_k), F(pl.o_v), nullptr, nullptr}, {nullptr, nullptr, nullptr, nullptr}, HD};
-    gemm(F(pl.o_feat) + C, 2 * C, F(pl.o_wqkv + (size_t)C * 2 * HD * 4), 2 * HD, R, 2 * HD, C,
-         Quad<EpiSplit>{e1});
+    gemm(F(pl.o_feat) + C, 2 * C, pl.k_qkv1, R, 2 * HD, C,
+         e1);
   } else {
     EpiSplit e{{F(pl.o_q), F(pl.o_k), F(pl.o_v), F(pl.o_g)}, {nullptr, nullptr, nullptr, nullptr}, HD};
-    gemm(F(pl.o_feat), C, F(pl.o_wqkv), 4 * HD, R, 4 * HD, C, Quad<EpiSplit>{e});
+    gemm(F(pl.o_feat), C, pl.k_qkv0, R, 4 * HD, C, e);
     RopeArgs rp{R, H, D, eps, usable, in->rope_cos.data, in->rope_sin.data, F(pl.o_q), F(pl.o_k)};
     const int64_t n = R * H * 2;
     k_qk_rope<Elt><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(rp);
@@ -403,7 +465,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   ag.B = B; ag.A = A; ag.K = K; ag.H = H; ag.D = D; ag.P = P; ag.radius = radius;
   ag.inv_sqrt_d = (float)(1.0 / std::sqrt((double)D));
   ag.eps = eps;
-  ag.QT = pl.QT; ag.cap_rows = pl.cap; ag.DP = pl.DP;
+  ag.QT = pl.QT; ag.DP = pl.DP; ag.kv_floats = pl.kv_floats;
   ag.Q = F(pl.o_q); ag.Kf = F(pl.o_k); ag.Vf = F(pl.o_v); ag.G = F(pl.o_g);
   ag.key_index = static_cast<const int64_t *>(in->key_index.data);
   ag.window = static_cast<const uint8_t *>(in->window_mask.data);
@@ -421,17 +483,18 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
       ++hk.launches;
     };
     const int dm = D <= 8 ? 8 : D <= 16 ? 16 : D <= 32 ? 32 : 64;
-    if (pl.af3) {
-      if (dm == 8) go(k_slot_attention<Elt, 8, true>);
-      else if (dm == 16) go(k_slot_attention<Elt, 16, true>);
-      else if (dm == 32) go(k_slot_attention<Elt, 32, true>);
-      else go(k_slot_attention<Elt, 64, true>);
-    } else {
-      if (dm == 8) go(k_slot_attention<Elt, 8, false>);
-      else if (dm == 16) go(k_slot_attention<Elt, 16, false>);
-      else if (dm == 32) go(k_slot_attention<Elt, 32, false>);
-      else go(k_slot_attention<Elt, 64, false>);
-    }
+    const bool multi = K > kChunk;
+#define ATTN_D(DM)                                                          \
+  if (dm == DM) {                                                           \
+    if (pl.af3)                                                             \
+      multi ? go(k_slot_attention<Elt, DM, true, true>)                     \
+            : go(k_slot_attention<Elt, DM, true, false>);                   \
+    else                                                                    \
+      multi ? go(k_slot_attention<Elt, DM, false, true>)                    \
+            : go(k_slot_attention<Elt, DM, false, false>);                  \
+  }
+    ATTN_D(8) ATTN_D(16) ATTN_D(32) ATTN_D(64)
+#undef ATTN_D
   }
 
   hk.mark(4, st);
@@ -440,15 +503,15 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   const float *gbuf = pl.af3 ? F(pl.o_gate) : F(pl.o_cond);
   const int64_t gld = pl.af3 ? 2 * C : 6 * C;
   const int64_t g0off = pl.af3 ? 0 : 2 * C, g1off = pl.af3 ? C : 5 * C;
-  gemm(F(pl.o_o), HD, F(pl.o_wout), C, R, C, HD,
+  gemm(F(pl.o_o), HD, pl.k_out, R, C, HD,
        Quad<EpiResidual>{{F(pl.o_x), gbuf, gld, g0off, C, F(pl.o_xp)}});
 
   // ---- transition on the new state
   TNormArgs ta{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_xp), F(pl.o_cond), F(pl.o_z)};
   k_transition_norm<<<row_blocks, 256, 0, st>>>(ta);
   ++hk.launches;
-  gemm(F(pl.o_z), C, F(pl.o_wff1), 2 * M, R, 2 * M, C, EpiSwiGLU{F(pl.o_h), M});
-  gemm(F(pl.o_h), M, F(pl.o_wff2), C, R, C, M,
+  gemm(F(pl.o_z), C, pl.k_ff1, R, 2 * M, C, EpiSwiGLU{F(pl.o_h), M});
+  gemm(F(pl.o_h), M, pl.k_ff2, R, C, M,
        Quad<EpiHidden<Elt>>{{F(pl.o_xp), gbuf, gld, g1off, C, usable, F(pl.o_hid),
                            static_cast<Elt *>(out->hidden.data)}});
 
@@ -456,7 +519,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
 
   // ---- boundary
   if (pl.enc) {
-    gemm(F(pl.o_hid), C, F(pl.o_wpool), U, R, U, C, Quad<EpiRelu>{{F(pl.o_pool), U}});
+    gemm(F(pl.o_hid), C, pl.k_pool, R, U, C, Quad<EpiRelu>{{F(pl.o_pool), U}});
     PoolArgs pa{B, A, T, U, usable, static_cast<const int64_t *>(in->atom_to_token.data), first,
                 last, F(pl.o_pool), out->token_output.data};
     k_token_mean<Elt><<<(unsigned)(B * T), 128, 0, st>>>(pa);

@@ -1,53 +1,10 @@
-// gemm_simt.cuh -- CUDA-core float32 GEMM with fused epilogues: out = epi(A @ W).
-// A [M, K] (float32 or the storage type), W [K, N] float32, both row-major.
-// 64x64 tile, 16-deep k step, 256 threads, 4x4 outputs per thread.
+// epilogues.cuh -- per-element epilogues of the projection GEMMs. Each functor ends one
+// step of the block; the GEMM hands it four consecutive columns of one output row.
 #pragma once
 
 #include "common.cuh"
 
 namespace atomenc {
-
-constexpr int kGemmBM = 64, kGemmBN = 64, kGemmBK = 16, kGemmThreads = 256;
-
-template <typename TA, class Epi>
-__global__ void __launch_bounds__(kGemmThreads)
-    k_gemm_simt(const TA *__restrict__ A, int64_t lda, const float *__restrict__ W,
-                int64_t ldw, int64_t M, int64_t N, int64_t K, Epi epi) {
-  __shared__ __align__(16) float As[kGemmBK][kGemmBM + 4];
-  __shared__ __align__(16) float Ws[kGemmBK][kGemmBN + 4];
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  const int64_t m0 = (int64_t)blockIdx.y * kGemmBM, n0 = (int64_t)blockIdx.x * kGemmBN;
-  float acc[4][4] = {};
-  for (int64_t k0 = 0; k0 < K; k0 += kGemmBK) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int idx = tid + e * kGemmThreads;
-      const int m = idx >> 4, k = idx & 15;
-      const int64_t gm = m0 + m, gk = k0 + k;
-      As[k][m] = (gm < M && gk < K) ? ldf(A, gm * lda + gk) : 0.f;
-      const int kk = idx >> 6, n = idx & 63;
-      const int64_t wk = k0 + kk, wn = n0 + n;
-      Ws[kk][n] = (wk < K && wn < N) ? W[wk * ldw + wn] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < kGemmBK; ++k) {
-      const float4 a = *reinterpret_cast<const float4 *>(&As[k][ty * 4]);
-      const float4 w = *reinterpret_cast<const float4 *>(&Ws[k][tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], wv[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t row = m0 + ty * 4 + i;
-    if (row < M && n0 + tx * 4 < N) epi.quad(row, n0 + tx * 4, acc[i], N);
-  }
-}
 
 // Per-element epilogues get the four consecutive columns of one thread through this.
 template <class E>
@@ -70,13 +27,33 @@ struct EpiStore {  // plain float32 store
 
 // AF3 conditioning: columns (scale_0, shift_0, scale_1, shift_1, scale_2, shift_2), C each;
 // scale columns become sigmoid(c_j @ w_scale[j] + b_scale[j])  (bullet 7)
+// Index math is done once per four columns, in 32 bits (C is a multiple of 4).
 struct EpiCondAF3 {
   float *out;  // [M, 6C]
   const float *b_scale;  // [3, C]
   int64_t C;
-  __device__ void operator()(int64_t r, int64_t c, float v) const {
-    const int64_t j = c / (2 * C), part = (c / C) & 1, ch = c % C;
-    out[r * 6 * C + c] = part == 0 ? sigmoidf_(v + b_scale[j * C + ch]) : v;
+  __device__ void quad(int64_t r, int64_t c0, const float (&v)[4], int64_t N) const {
+    const int c = (int)c0, Ci = (int)C;
+    if (Ci & 3) {  // a quad may straddle two blocks
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int ce = c + e;
+        if (ce >= N) break;
+        const int be = ce / Ci, he = ce - be * Ci;
+        out[r * 6 * C + ce] = (be & 1) ? v[e] : sigmoidf_(v[e] + b_scale[(be >> 1) * Ci + he]);
+      }
+      return;
+    }
+    const int blk = c / Ci, ch = c - blk * Ci;
+    float4 o = make_float4(v[0], v[1], v[2], v[3]);
+    if ((blk & 1) == 0) {  // scale block j = blk / 2
+      const float *bs = b_scale + (blk >> 1) * Ci + ch;
+      o.x = sigmoidf_(v[0] + bs[0]);
+      o.y = sigmoidf_(v[1] + bs[1]);
+      o.z = sigmoidf_(v[2] + bs[2]);
+      o.w = sigmoidf_(v[3] + bs[3]);
+    }
+    *reinterpret_cast<float4 *>(out + r * 6 * C + c0) = o;
   }
 };
 
@@ -85,8 +62,17 @@ struct EpiGateAF3 {
   float *out;  // [M, 2C]
   const float *b_rg;  // [2, C]
   int64_t C;
-  __device__ void operator()(int64_t r, int64_t c, float v) const {
-    out[r * 2 * C + c] = sigmoidf_(v + b_rg[c]);
+  __device__ void quad(int64_t r, int64_t c0, const float (&v)[4], int64_t N) const {
+    const float *b = b_rg + c0;
+    if (C & 1) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (c0 + e < N) out[r * 2 * C + c0 + e] = sigmoidf_(v[e] + b[e]);
+      return;
+    }
+    *reinterpret_cast<float4 *>(out + r * 2 * C + c0) =
+        make_float4(sigmoidf_(v[0] + b[0]), sigmoidf_(v[1] + b[1]), sigmoidf_(v[2] + b[2]),
+                    sigmoidf_(v[3] + b[3]));
   }
 };
 
@@ -96,10 +82,28 @@ struct EpiSplit {
   float *dst[4];
   const float *bias[4];
   int64_t HD;
-  __device__ void operator()(int64_t r, int64_t c, float v) const {
-    const int64_t part = c / HD, ch = c % HD;
-    if (bias[part]) v += bias[part][ch];
-    dst[part][r * HD + ch] = v;
+  __device__ void quad(int64_t r, int64_t c0, const float (&v)[4], int64_t N) const {
+    const int HDi = (int)HD, c = (int)c0, part = c / HDi, ch = c - part * HDi;
+    float o[4] = {v[0], v[1], v[2], v[3]};
+    const float *b = bias[part];
+    if (b) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[e] += b[ch + e];
+    }
+    float *d = dst[part] + r * HD + ch;
+    if ((HDi & 3) == 0) {
+      *reinterpret_cast<float4 *>(d) = make_float4(o[0], o[1], o[2], o[3]);
+    } else {  // a quad may straddle two parts when HD is not a multiple of 4
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int ce = c + e;
+        if (ce >= N) break;
+        const int pe = ce / HDi, he = ce - pe * HDi;
+        float x = v[e];
+        if (bias[pe]) x += bias[pe][he];
+        dst[pe][r * HD + he] = x;
+      }
+    }
   }
 };
 

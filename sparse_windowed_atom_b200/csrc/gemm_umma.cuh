@@ -1,0 +1,407 @@
+// gemm_umma.cuh -- tcgen05 (5th-generation tensor core) GEMM with fused epilogues:
+//   out = epi(A @ W),  A [M, K] float32 or bf16 in global memory, W [K, N] prepacked.
+//
+// One CTA computes a 128 x 128 output tile; 128 threads (4 warps).
+//  * W is prepacked (k_pack_weights) as bf16 blocks of 128 output columns x 64 k in the
+//    exact 128B-swizzled shared-memory image, so a block arrives with one bulk async
+//    copy (mbarrier transaction count).
+//  * The CTA's threads convert their A chunk (128 rows x 64 k) to bf16 and store it
+//    swizzled; with SPLIT (float32 workloads) A and W are each split into bf16 high and
+//    low parts and the product is hi*hi + hi*lo + lo*hi (three MMAs per k step), which
+//    carries about 16 significant bits per operand into the float32 accumulator.
+//  * Two shared-memory stages: the conversion of chunk c+1 overlaps the MMAs of chunk c.
+//  * One thread issues tcgen05.mma (M=128, N=128, K=16) into a 128-column TMEM
+//    accumulator and commits to mbarriers; every wait is bounded (status bit 4 on
+//    timeout, never a hang).
+//  * Epilogue: warp w reads TMEM lanes 32w..32w+31 (one output row per thread) with
+//    tcgen05.ld and hands four consecutive columns at a time to the epilogue functor.
+#pragma once
+
+#include "common.cuh"
+#include "umma.cuh"
+
+namespace atomenc {
+
+constexpr int kUmmaBM = 128, kUmmaBN = 128, kUmmaBK = 64, kUmmaThreads = 128, kUmmaStages = 2;
+constexpr uint32_t kUmmaBlockBytes = kUmmaBN * kUmmaBK * 2;   // one bf16 [128 x 64] block
+constexpr unsigned kStatusMmaTimeout = 4u;
+
+__host__ __device__ constexpr size_t umma_smem_bytes(bool split) {
+  // per stage: A (hi[, lo]) + B (hi[, lo]); + 1 KB for alignment and barriers
+  return (size_t)kUmmaStages * (split ? 4 : 2) * kUmmaBlockBytes + 2048;
+}
+
+// Bytes of the packed image of a [K, N] weight.
+__host__ __device__ inline size_t packed_bytes(int64_t K, int64_t N, bool split) {
+  return (size_t)((N + kUmmaBN - 1) / kUmmaBN) * ((K + kUmmaBK - 1) / kUmmaBK) *
+         kUmmaBlockBytes * (split ? 2 : 1);
+}
+
+struct PackJob {
+  const float *src;   // [K, N] float32 panel, row stride ld
+  uint8_t *dst;
+  int32_t K, N, ld, split;
+};
+constexpr int kMaxPackJobs = 12;
+struct PackJobs {
+  PackJob job[kMaxPackJobs];
+  int n;
+};
+
+// Pack W [K, N] into blocks (n-tile t, k-chunk c) of [128 n x 64 k] bf16, swizzled K-major,
+// hi block then (split) lo block; zero outside [K, N].
+__global__ void k_pack_weights(PackJobs jobs) {
+  const PackJob &j = jobs.job[blockIdx.y];
+  const int64_t nt = (j.N + kUmmaBN - 1) / kUmmaBN, kc = (j.K + kUmmaBK - 1) / kUmmaBK;
+  const int64_t total = nt * kUmmaBN * kc * kUmmaBK;
+  const int nparts = j.split ? 2 : 1;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t k = i % (kc * kUmmaBK), n = i / (kc * kUmmaBK);
+    const float w = (k < j.K && n < j.N) ? j.src[k * j.ld + n] : 0.f;
+    const int64_t t = n / kUmmaBN, c = k / kUmmaBK;
+    const int nl = (int)(n % kUmmaBN), kl = (int)(k % kUmmaBK);
+    uint8_t *blk = j.dst + (t * kc + c) * nparts * kUmmaBlockBytes;
+    const uint16_t hi = umma::bf16_bits(w);
+    const uint32_t off = umma::swz_offset(nl, kl, kUmmaBN);
+    *reinterpret_cast<uint16_t *>(blk + off) = hi;
+    if (j.split)
+      *reinterpret_cast<uint16_t *>(blk + kUmmaBlockBytes + off) =
+          umma::bf16_bits(w - umma::bf16_val(hi));
+  }
+}
+
+template <typename TA>
+__device__ __forceinline__ void load8(const TA *A, int64_t lda, int64_t M, int64_t K, int64_t r,
+                                      int64_t k, float (&v)[8]);
+
+template <>
+__device__ __forceinline__ void load8<float>(const float *A, int64_t lda, int64_t M, int64_t K,
+                                             int64_t r, int64_t k, float (&v)[8]) {
+  if (r < M && k + 8 <= K && ((lda | k) & 3) == 0) {
+    const float4 x = *reinterpret_cast<const float4 *>(A + r * lda + k);
+    const float4 y = *reinterpret_cast<const float4 *>(A + r * lda + k + 4);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = (r < M && k + e < K) ? A[r * lda + k + e] : 0.f;
+  }
+}
+
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *A, int64_t lda,
+                                                     int64_t M, int64_t K, int64_t r, int64_t k,
+                                                     float (&v)[8]) {
+  if (r < M && k + 8 <= K && ((lda | k) & 7) == 0) {
+    const uint4 x = *reinterpret_cast<const uint4 *>(A + r * lda + k);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[2 * e] = __uint_as_float(w[e] << 16);
+      v[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = (r < M && k + e < K) ? ldf(A, r * lda + k + e) : 0.f;
+  }
+}
+
+template <typename TA, bool SPLIT, class Epi>
+__global__ void __launch_bounds__(kUmmaThreads)
+    k_gemm_umma(const TA *__restrict__ A, int64_t lda, const uint8_t *__restrict__ Wpk, int64_t M,
+                int64_t N, int64_t K, Epi epi, unsigned *status) {
+  extern __shared__ __align__(1024) uint8_t smem_dyn[];
+  // 1024-byte alignment of the operand blocks (swizzle atoms)
+  uint8_t *sm = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  constexpr int PARTS = SPLIT ? 2 : 1;
+  uint8_t *sA = sm;                                                  // [stage][part] blocks
+  uint8_t *sB = sm + kUmmaStages * PARTS * kUmmaBlockBytes;          // [stage][part] blocks
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sB + kUmmaStages * PARTS * kUmmaBlockBytes);
+  uint64_t *bar_b = bar, *bar_mma = bar + kUmmaStages, *bar_done = bar + 2 * kUmmaStages;
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 2 * kUmmaStages + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t n_tile = blockIdx.x, m0 = (int64_t)blockIdx.y * kUmmaBM, n0 = n_tile * kUmmaBN;
+  const int nkc = (int)((K + kUmmaBK - 1) / kUmmaBK);
+  constexpr uint32_t idesc = umma::idesc_bf16(kUmmaBM, kUmmaBN);
+
+  if (tid == 0) {
+    for (int s = 0; s < kUmmaStages; ++s) {
+      umma::mbar_init(bar_b + s, 1);
+      umma::mbar_init(bar_mma + s, 1);
+    }
+    umma::mbar_init(bar_done, 1);
+    umma::fence_mbar_init();
+  }
+  if (warp == 0) umma::tmem_alloc(tslot, kUmmaBN);
+  umma::tc_fence_before();
+  __syncthreads();
+  umma::tc_fence_after();
+  const uint32_t tmem = *tslot;
+  bool ok = true;
+
+  for (int c = 0; c < nkc; ++c) {
+    const int s = c % kUmmaStages;
+    if (c >= kUmmaStages && ok)  // the MMAs that read this stage two chunks ago are done
+      ok = umma::mbar_wait(bar_mma + s, ((c - kUmmaStages) / kUmmaStages) & 1);
+    uint8_t *a_s = sA + s * PARTS * kUmmaBlockBytes;
+    uint8_t *b_s = sB + s * PARTS * kUmmaBlockBytes;
+    if (tid == 0) {
+      umma::mbar_arrive_expect_tx(bar_b + s, PARTS * kUmmaBlockBytes);
+      umma::bulk_g2s(b_s, Wpk + ((n_tile * nkc + c) * PARTS) * (size_t)kUmmaBlockBytes,
+                     PARTS * kUmmaBlockBytes, bar_b + s);
+    }
+    // A chunk: warp w converts rows 32w..32w+31; 8 lanes per row, 8 k each
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int r = warp * 32 + it * 4 + (lane >> 3), seg = lane & 7;
+      float v[8];
+      load8<TA>(A, lda, M, K, m0 + r, (int64_t)c * kUmmaBK + seg * 8, v);
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint16_t h0 = umma::bf16_bits(v[2 * e]), h1 = umma::bf16_bits(v[2 * e + 1]);
+        hi[e] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+        if (SPLIT) {
+          const uint16_t l0 = umma::bf16_bits(v[2 * e] - umma::bf16_val(h0));
+          const uint16_t l1 = umma::bf16_bits(v[2 * e + 1] - umma::bf16_val(h1));
+          lo[e] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+        }
+      }
+      const uint32_t off = umma::swz_offset(r, seg * 8, kUmmaBM);
+      *reinterpret_cast<uint4 *>(a_s + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      if (SPLIT)
+        *reinterpret_cast<uint4 *>(a_s + kUmmaBlockBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+    umma::fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      if (ok) ok = umma::mbar_wait(bar_b + s, (c / kUmmaStages) & 1);
+      umma::tc_fence_after();
+      const uint32_t a0 = umma::smem_u32(a_s), b0 = umma::smem_u32(b_s);
+#pragma unroll
+      for (int kk = 0; kk < kUmmaBK / 16; ++kk) {
+        const uint64_t da = umma::sw128_desc(a0 + kk * 32), db = umma::sw128_desc(b0 + kk * 32);
+        umma::mma_bf16(tmem, da, db, idesc, (c | kk) != 0);
+        if (SPLIT) {
+          umma::mma_bf16(tmem, da, umma::sw128_desc(b0 + kUmmaBlockBytes + kk * 32), idesc, 1);
+          umma::mma_bf16(tmem, umma::sw128_desc(a0 + kUmmaBlockBytes + kk * 32), db, idesc, 1);
+        }
+      }
+      umma::mma_commit(bar_mma + s);
+    }
+  }
+  if (tid == 0) umma::mma_commit(bar_done);
+  if (ok) ok = umma::mbar_wait(bar_done, 0);
+  if (!ok && lane == 0) atomicOr(status, kStatusMmaTimeout);
+  umma::tc_fence_after();
+
+  // epilogue: thread (warp w, lane l) owns output row m0 + 32w + l
+  const int64_t row = m0 + warp * 32 + lane;
+  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll 1
+  for (int c0 = 0; c0 < kUmmaBN; c0 += 32) {
+    if (n0 + c0 >= N) break;
+    float v[32];
+    umma::tmem_ld32(trow + c0, v);
+    if (row < M && ok) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        if (n0 + c0 + j < N) {
+          const float q[4] = {v[j], v[j + 1], v[j + 2], v[j + 3]};
+          epi.quad(row, n0 + c0 + j, q, N);
+        }
+    }
+  }
+  umma::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) umma::tmem_dealloc(tmem, kUmmaBN);
+}
+
+// ----------------------------------------------------------------------------------
+// Row-block GEMM: one CTA owns 128 rows of A (all of K resident in shared memory,
+// converted once) and a contiguous range of 128-column output tiles. Warp roles:
+//   warps 0-3  convert A, then run the epilogue of each tile (warp w owns TMEM lanes
+//              32w..32w+31); the accumulator chunk is transposed through a per-warp
+//              shared tile so that the epilogue functor sees 8 lanes per 128-byte row
+//              segment (coalesced global reads and writes);
+//   warp 4     lane 0 issues the MMAs: two 128-column TMEM accumulators, so the MMAs of
+//              tile t+1 run while the epilogue drains tile t;
+//   warp 5     lane 0 streams the packed weight blocks through a ring of NSLOT shared
+//              buffers with bulk async copies.
+// Requires K <= kRowsKMax; every wait is bounded (status bit 4 on timeout).
+constexpr int kRowsThreads = 192;
+constexpr int kRowsKMax = 256;
+
+__host__ __device__ constexpr int rows_slots(bool split) { return split ? 2 : 3; }
+__host__ __device__ inline size_t rows_smem_bytes(int64_t K, bool split) {
+  const int parts = split ? 2 : 1;
+  const size_t nkc = (size_t)((K + kUmmaBK - 1) / kUmmaBK);
+  return 1024 + (nkc + rows_slots(split)) * parts * kUmmaBlockBytes + 4 * 32 * 33 * 4 + 256;
+}
+
+template <typename TA, bool SPLIT, class Epi>
+__global__ void __launch_bounds__(kRowsThreads, 1)
+    k_gemm_rows(const TA *__restrict__ A, int64_t lda, const uint8_t *__restrict__ Wpk, int64_t M,
+                int64_t N, int64_t K, int tiles_per_cta, Epi epi, unsigned *status) {
+  extern __shared__ __align__(1024) uint8_t smem_dyn[];
+  constexpr int PARTS = SPLIT ? 2 : 1, NSLOT = rows_slots(SPLIT);
+  constexpr uint32_t BLK = kUmmaBlockBytes;
+  constexpr uint32_t idesc = umma::idesc_bf16(kUmmaBM, kUmmaBN);
+  uint8_t *sm = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  const int nkc = (int)((K + kUmmaBK - 1) / kUmmaBK);
+  uint8_t *sA = sm;                                       // [nkc][PARTS] blocks
+  uint8_t *sR = sA + (size_t)nkc * PARTS * BLK;           // [NSLOT][PARTS] blocks
+  float *sT = reinterpret_cast<float *>(sR + (size_t)NSLOT * PARTS * BLK);   // [4][32][33]
+  uint64_t *full = reinterpret_cast<uint64_t *>(sT + 4 * 32 * 33);
+  uint64_t *empty = full + NSLOT, *accf = empty + NSLOT, *acce = accf + 2, *aready = acce + 2;
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(aready + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nt = (int)((N + kUmmaBN - 1) / kUmmaBN);
+  const int t_begin = blockIdx.x * tiles_per_cta;
+  const int ntl = min(nt, t_begin + tiles_per_cta) - t_begin;
+  if (ntl <= 0) return;  // uniform over the CTA
+  const int64_t m0 = (int64_t)blockIdx.y * kUmmaBM;
+
+  if (tid == 0) {
+    for (int s = 0; s < NSLOT; ++s) {
+      umma::mbar_init(full + s, 1);
+      umma::mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      umma::mbar_init(accf + b, 1);
+      umma::mbar_init(acce + b, 128);
+    }
+    umma::mbar_init(aready, 128);
+    *abort_flag = 0;
+    umma::fence_mbar_init();
+  }
+  if (warp == 0) umma::tmem_alloc(tslot, 2 * kUmmaBN);
+  umma::tc_fence_before();
+  __syncthreads();
+  umma::tc_fence_after();
+  const uint32_t tmem = *tslot;
+  bool ok = true;
+
+  if (warp < 4) {
+    // ---- A: rows 32w..32w+31 of the tile, every k chunk, bf16 (hi[, lo]) swizzled
+    for (int c = 0; c < nkc; ++c) {
+      uint8_t *a_c = sA + (size_t)c * PARTS * BLK;
+#pragma unroll 2
+      for (int it = 0; it < 8; ++it) {
+        const int r = warp * 32 + it * 4 + (lane >> 3), seg = lane & 7;
+        float v[8];
+        load8<TA>(A, lda, M, K, m0 + r, (int64_t)c * kUmmaBK + seg * 8, v);
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint16_t h0 = umma::bf16_bits(v[2 * e]), h1 = umma::bf16_bits(v[2 * e + 1]);
+          hi[e] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+          if (SPLIT) {
+            const uint16_t l0 = umma::bf16_bits(v[2 * e] - umma::bf16_val(h0));
+            const uint16_t l1 = umma::bf16_bits(v[2 * e + 1] - umma::bf16_val(h1));
+            lo[e] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+          }
+        }
+        const uint32_t off = umma::swz_offset(r, seg * 8, kUmmaBM);
+        *reinterpret_cast<uint4 *>(a_c + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        if (SPLIT)
+          *reinterpret_cast<uint4 *>(a_c + BLK + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+    }
+    umma::fence_async_smem();
+    umma::mbar_arrive(aready);
+
+    // ---- epilogue of each output tile
+    float *T = sT + warp * 32 * 33;
+    const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
+    for (int tl = 0; tl < ntl; ++tl) {
+      const int buf = tl & 1;
+      if (ok) ok = umma::mbar_wait(accf + buf, (tl >> 1) & 1, abort_flag);
+      umma::tc_fence_after();
+      const int64_t n0 = (int64_t)(t_begin + tl) * kUmmaBN;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kUmmaBN; c0 += 32) {
+        if (n0 + c0 >= N) break;
+        float v[32];
+        umma::tmem_ld32(tlane + buf * kUmmaBN + c0, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) T[lane * 33 + j] = v[j];
+        __syncwarp();
+#pragma unroll 2
+        for (int i = 0; i < 8; ++i) {
+          const int rl = i * 4 + (lane >> 3), q = lane & 7;
+          const int64_t row = m0 + warp * 32 + rl, col = n0 + c0 + 4 * q;
+          if (ok && row < M && col < N) {
+            const float x[4] = {T[rl * 33 + 4 * q], T[rl * 33 + 4 * q + 1], T[rl * 33 + 4 * q + 2],
+                                T[rl * 33 + 4 * q + 3]};
+            epi.quad(row, col, x, N);
+          }
+        }
+        __syncwarp();
+      }
+      umma::tc_fence_before();
+      umma::mbar_arrive(acce + buf);
+    }
+  } else if (warp == 4) {
+    if (lane == 0) {
+      // ---- MMA issue
+      ok = umma::mbar_wait(aready, 0, abort_flag);
+      umma::tc_fence_after();
+      for (int tl = 0; tl < ntl && ok; ++tl) {
+        const int buf = tl & 1;
+        if (tl >= 2) {
+          ok = umma::mbar_wait(acce + buf, ((tl - 2) >> 1) & 1, abort_flag);
+          umma::tc_fence_after();
+        }
+        const uint32_t dtm = tmem + buf * kUmmaBN;
+        for (int c = 0; c < nkc && ok; ++c) {
+          const int i = tl * nkc + c, slot = i % NSLOT;
+          ok = umma::mbar_wait(full + slot, (i / NSLOT) & 1, abort_flag);
+          umma::tc_fence_after();
+          const uint32_t a0 = umma::smem_u32(sA + (size_t)c * PARTS * BLK);
+          const uint32_t b0 = umma::smem_u32(sR + (size_t)slot * PARTS * BLK);
+#pragma unroll
+          for (int kk = 0; kk < kUmmaBK / 16; ++kk) {
+            const uint64_t da = umma::sw128_desc(a0 + kk * 32), db = umma::sw128_desc(b0 + kk * 32);
+            umma::mma_bf16(dtm, da, db, idesc, (c | kk) != 0);
+            if (SPLIT) {
+              umma::mma_bf16(dtm, da, umma::sw128_desc(b0 + BLK + kk * 32), idesc, 1);
+              umma::mma_bf16(dtm, umma::sw128_desc(a0 + BLK + kk * 32), db, idesc, 1);
+            }
+          }
+          umma::mma_commit(empty + slot);
+        }
+        umma::mma_commit(accf + buf);
+      }
+    }
+  } else {
+    if (lane == 0) {
+      // ---- weight blocks, ring of NSLOT buffers
+      const int total = ntl * nkc;
+      for (int i = 0; i < total && ok; ++i) {
+        const int slot = i % NSLOT;
+        if (i >= NSLOT) ok = umma::mbar_wait(empty + slot, ((i - NSLOT) / NSLOT) & 1, abort_flag);
+        const int tl = i / nkc, c = i - tl * nkc;
+        umma::mbar_arrive_expect_tx(full + slot, PARTS * BLK);
+        umma::bulk_g2s(sR + (size_t)slot * PARTS * BLK,
+                       Wpk + ((size_t)(t_begin + tl) * nkc + c) * PARTS * BLK, PARTS * BLK,
+                       full + slot);
+      }
+    }
+  }
+  if (!ok) {
+    *abort_flag = 1;
+    atomicOr(status, kStatusMmaTimeout);
+  }
+  umma::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) umma::tmem_dealloc(tmem, 2 * kUmmaBN);
+}
+
+}  // namespace atomenc
