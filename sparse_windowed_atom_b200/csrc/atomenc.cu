@@ -25,7 +25,7 @@ namespace {
 
 constexpr int kVersion = 1;
 constexpr int kMaxD = 64;
-constexpr size_t kAttnSmemBudget = 104 * 1024;  // two CTAs per SM
+constexpr size_t kAttnSmemBudget = 104 * 1024;  // two CTAs per SM (dynamic part)
 
 struct Dims {
   int64_t B = 0, A = 0, T = 0, K = 0, C = 0, S = 0, H = 0, D = 0, P = 0, M = 0, U = 0, V = 0;
@@ -249,18 +249,20 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   pl.k_tok = take(cur, pl.enc ? 0 : packed_bytes(V, C, split));
   pl.bytes = cur;
 
-  // ---- attention tile: QT queries per CTA (small enough that the grid covers the
-  // GPU twice over), a slot plan of QT*K ints and a K/V stage in the rest of the budget
+  // ---- attention tile: QT queries per CTA (the grid should cover 2 CTAs x 148 SMs), a
+  // slot plan, (AF3) the pair-bias table and the Q rows; the K/V stage gets the rest
   const int dmax = D <= 8 ? 8 : D <= 16 ? 16 : D <= 32 ? 32 : 64;
   pl.DP = dmax + 4;  // odd number of 16-byte chunks per staged row: no bank conflicts
-  int qt = 32;
-  while (qt > 1 && ((int64_t)B * ((A + qt - 1) / qt) < 2 * 148 || (int64_t)qt * K * 4 > 32768))
+  int qt = pl.af3 ? 16 : 32;
+  const int64_t fill = (B * A + 2 * 148 - 1) / (2 * 148);
+  if (fill < qt) qt = (int)(fill < 1 ? 1 : fill);
+  while (qt > 1 && attn_fixed_smem(qt, (int)K, (int)H, (int)(H * D), pl.af3) > kAttnSmemBudget / 2)
     qt /= 2;
+  const size_t fixed = attn_fixed_smem(qt, (int)K, (int)H, (int)(H * D), pl.af3);
+  if (fixed + 8 * 1024 > kAttnSmemBudget) return ATOMENC_ERR_UNSUPPORTED;
   pl.QT = qt;
-  const size_t plan_bytes = (((size_t)qt * K + 3) & ~size_t(3)) * 4;
-  if (plan_bytes + 16 * 1024 > kAttnSmemBudget) return ATOMENC_ERR_UNSUPPORTED;
-  pl.kv_floats = (int)((kAttnSmemBudget - plan_bytes) / 4);
-  pl.attn_smem = plan_bytes + (size_t)pl.kv_floats * 4;
+  pl.kv_floats = (int)((kAttnSmemBudget - fixed) / 4);
+  pl.attn_smem = fixed + (size_t)pl.kv_floats * 4;
   return ATOMENC_OK;
 }
 
@@ -462,8 +464,9 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
 
   // ---- slot-gathered attention
   AttnArgs ag;
-  ag.B = B; ag.A = A; ag.K = K; ag.H = H; ag.D = D; ag.P = P; ag.radius = radius;
-  ag.inv_sqrt_d = (float)(1.0 / std::sqrt((double)D));
+  ag.B = (int)B; ag.A = (int)A; ag.K = (int)K; ag.H = (int)H; ag.D = (int)D; ag.P = (int)P;
+  ag.radius = radius < 0 ? -1 : (radius > INT_MAX ? INT_MAX : (int)radius);
+  ag.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   ag.eps = eps;
   ag.QT = pl.QT; ag.DP = pl.DP; ag.kv_floats = pl.kv_floats;
   ag.Q = F(pl.o_q); ag.Kf = F(pl.o_k); ag.Vf = F(pl.o_v); ag.G = F(pl.o_g);

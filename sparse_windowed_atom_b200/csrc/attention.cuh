@@ -9,19 +9,21 @@
 // entries (bullets 5, 6, 15); the weighted values are multiplied by sigmoid of the value
 // gate logits and stored head-major (bullet 16).
 //
-// One CTA owns QT consecutive queries of one batch element.
-//  Phase 1 reads key_index and window_mask once and writes the tile's slot plan (key id
-//  or -1) to shared memory, with the span [klo, khi] of the permitted key ids.
-//  Phase 2 walks the heads in groups: as many heads as the shared-memory stage holds for
-//  this span are staged (K and V rows of the span, float32), then each warp takes one
-//  query at a time with its 32 lanes over the slots (4 slots per lane per 128-slot
-//  chunk): logits, masked softmax (max / sum by warp shuffles), attention weights
-//  written once, the weighted value sum kept per lane and folded across lanes by a
-//  butterfly reduce-scatter (lane l ends with channel l), value gate, store.
-//  AF3: the pair bias of the lane's slots is computed from the pair rows (read once per
-//  head group, LayerNorm over P in registers) for every head of the group.
-//  When even one head of the span does not fit, the tile reads K/V rows straight from
-//  global memory (L2) instead and sets status bit 1; the results are the same.
+// One CTA (256 threads, two per SM) owns QT consecutive queries of one batch element.
+//  Phase 0  the tile's Q rows are copied to shared memory with cp.async.
+//  Phase 1  each thread reads 8 consecutive slots of the tile's key_index / window_mask
+//           (16-byte loads), decides eligibility and writes the slot plan (key id or -1)
+//           and the span [klo, khi] of the permitted ids; AF3: the pair bias of every
+//           permitted (slot, head) is computed from its pair row (LayerNorm over P,
+//           one pass) and kept in shared memory as float32 [head][slot].
+//  Phase 2  head groups: the K and V rows of the span for as many heads as fit are staged
+//           (float32, cp.async); each warp takes one query at a time, lanes over the slots
+//           (4 per lane per 128-slot chunk): logits, max, one exp2 per entry, sum, weights
+//           written once (bf16 rounded with integer ops), the weighted value sum per lane
+//           with packed f32x2 FMAs, folded across lanes by a butterfly reduce-scatter,
+//           value gate, store.
+// A tile whose span does not fit even one head reads K/V rows from global memory (L2)
+// instead and sets status bit 1; the results are the same.
 #pragma once
 
 #include <climits>
@@ -35,13 +37,14 @@ constexpr int kAttnWarps = kAttnThreads / kWarp;
 constexpr int kPairMax = 32;
 constexpr int kSlotsPerLane = 4;                       // one chunk = 128 slots
 constexpr int kChunk = kWarp * kSlotsPerLane;
-constexpr int kAf3HeadsMax = 4;   // pair-bias heads held in registers per stage
-constexpr int kAttnHeadsMax = 64;  // AF3 w_pair columns kept in shared memory
+constexpr int kAttnHeadsMax = 32;                      // AF3 w_pair columns in shared memory
+constexpr int kPlanSlots = 8;                          // slots per thread in phase 1
 
 struct AttnArgs {
-  int64_t B, A, K, H, D, P;
-  int64_t radius;
-  float inv_sqrt_d, eps;
+  int B, A, K, H, D, P;
+  int radius;                     // -1 = no index window
+  float scale_log2;               // log2(e) / sqrt(D)
+  float eps;
   int QT, DP, kv_floats;          // queries per CTA, padded row width, K/V stage size
   const float *Q, *Kf, *Vf, *G;   // [B*A, H*D]
   const int64_t *key_index;       // [B, A, K]
@@ -53,6 +56,44 @@ struct AttnArgs {
   float *O;                       // [B*A, H*D] gated attention output
   unsigned *status;
 };
+
+// float counts of the shared regions, each rounded to 4 floats (16-byte aligned regions)
+__host__ __device__ inline size_t ru4(size_t n) { return (n + 3) & ~size_t(3); }
+__host__ __device__ inline size_t attn_fixed_smem(int QT, int K, int H, int HD, bool af3) {
+  const size_t slots = (size_t)QT * K;
+  return 4 * (ru4(slots) + (af3 ? ru4((size_t)H * slots) : 0) + ru4((size_t)QT * HD));
+}
+
+// d0,d1 += a * b elementwise on a pair of floats (one packed f32x2 FMA on sm_100)
+__device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%0, %1};\n\t"
+      "fma.rn.f32x2 rc, ra, rb, rc;\n\tmov.b64 {%0, %1}, rc;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// 2^x on the special-function unit (the exponent of the softmax is always <= 0 here)
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// float -> bf16 bits, round to nearest even, by integer arithmetic (finite inputs)
+__device__ __forceinline__ uint16_t bf16_rne(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (uint16_t)((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
+}
+
+template <typename T>
+__device__ __forceinline__ void store_weight(T *p, int64_t i, float w);
+template <>
+__device__ __forceinline__ void store_weight<float>(float *p, int64_t i, float w) { p[i] = w; }
+template <>
+__device__ __forceinline__ void store_weight<__nv_bfloat16>(__nv_bfloat16 *p, int64_t i, float w) {
+  reinterpret_cast<uint16_t *>(p)[i] = bf16_rne(w);
+}
 
 // Butterfly reduce-scatter of v[0..W) summed over the 32 lanes: afterwards v[0] holds
 // the full sum of channel (lane & (W-1)). W is a power of two <= 32.
@@ -73,83 +114,95 @@ __device__ __forceinline__ float reduce_scatter(float (&v)[W], int lane) {
   return v[0];
 }
 
+// pair row of one slot -> bias for every head: rstd * (sum_p y_p W'[p,h] - m * sum_p W'[p,h]),
+// y = pair - pair_0 (shift for a well-conditioned one-pass variance), m = mean(y)
+template <typename T>
+__device__ __forceinline__ void slot_pair_bias(const T *pr, int P, int H, float eps,
+                                               const float *wp, const float *wsum, float *out,
+                                               int out_stride) {
+  float y[kPairMax];
+  const float x0 = ldf(pr, 0);
+  float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+  for (int p = 0; p < kPairMax; ++p)
+    if (p < P) {
+      y[p] = ldf(pr, p) - x0;
+      s1 += y[p];
+      s2 = fmaf(y[p], y[p], s2);
+    }
+  const float invP = 1.f / (float)P;
+  const float m = s1 * invP;
+  const float var = fmaxf(s2 * invP - m * m, 0.f);
+  const float rstd = rsqrtf(var + eps);
+  for (int h = 0; h < H; ++h) {
+    float d = 0.f;
+#pragma unroll
+    for (int p = 0; p < kPairMax; ++p)
+      if (p < P) d = fmaf(y[p], wp[p * H + h], d);
+    out[h * out_stride] = rstd * (d - m * wsum[h]);
+  }
+}
+
 template <int DMAX>
-__device__ __forceinline__ float dot_row(const float (&q)[DMAX], const float *r) {
-  // r is 16-byte aligned and zero-padded to DMAX in shared memory
+__device__ __forceinline__ float dot_row(const float *q, const float *r) {
+  // q, r: 16-byte aligned, zero-padded to DMAX in shared memory
   float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
   for (int d = 0; d < DMAX; d += 4) {
+    const float4 a = *reinterpret_cast<const float4 *>(q + d);
     const float4 k = *reinterpret_cast<const float4 *>(r + d);
-    s0 = fmaf(q[d], k.x, s0);
-    s1 = fmaf(q[d + 1], k.y, s1);
-    s2 = fmaf(q[d + 2], k.z, s2);
-    s3 = fmaf(q[d + 3], k.w, s3);
+    fma2(s0, s1, a.x, a.y, k.x, k.y);
+    fma2(s2, s3, a.z, a.w, k.z, k.w);
   }
   return (s0 + s1) + (s2 + s3);
 }
 
 template <int DMAX>
-__device__ __forceinline__ float dot_global(const float (&q)[DMAX], const float *r, int64_t D) {
-  float s0 = 0.f, s1 = 0.f;
+__device__ __forceinline__ float dot_plain(const float (&q)[DMAX], const float *r, int D) {
+  float s = 0.f;
 #pragma unroll
-  for (int d = 0; d < DMAX; d += 2) {
-    if (d < D) s0 = fmaf(q[d], r[d], s0);
-    if (d + 1 < D) s1 = fmaf(q[d + 1], r[d + 1], s1);
-  }
-  return s0 + s1;
+  for (int d = 0; d < DMAX; ++d)
+    if (d < D) s = fmaf(q[d], r[d], s);
+  return s;
 }
 
-// Pair bias of one slot for heads h0 .. h0+NB-1 (those < hg):
-//   beta_h = sum_p LN(pair)_p * pair_scale_p * w_pair[p, h]
-//          = rstd * (sum_p y_p W'[p, h] - m * sum_p W'[p, h]),
-// with y_p = pair_p - pair_0 (a shift that keeps the one-pass variance well conditioned),
-// m = mean(y), rstd = 1 / sqrt(mean(y^2) - m^2 + eps) (population variance, eps inside
-// the root). W' = pair_scale * w_pair and its column sums live in shared memory.
-template <typename T, int NB>
-__device__ __forceinline__ void pair_bias(const T *pr, int P, float eps, const float *wp,
-                                          const float *wsum, int H, int h0, int hg,
-                                          float (&beta)[NB]) {
-  const float x0 = ldf(pr, 0);
-  float s1 = 0.f, s2 = 0.f, dot[NB];
-#pragma unroll
-  for (int x = 0; x < NB; ++x) dot[x] = 0.f;
-  for (int p = 0; p < P; ++p) {
-    const float y = ldf(pr, p) - x0;
-    s1 += y;
-    s2 = fmaf(y, y, s2);
-#pragma unroll
-    for (int x = 0; x < NB; ++x)
-      if (x < hg) dot[x] = fmaf(y, wp[p * H + h0 + x], dot[x]);
-  }
-  const float m = s1 / (float)P;
-  const float var = fmaxf(s2 / (float)P - m * m, 0.f);
-  const float rstd = 1.f / sqrtf(var + eps);
-#pragma unroll
-  for (int x = 0; x < NB; ++x) beta[x] = x < hg ? rstd * (dot[x] - m * wsum[h0 + x]) : 0.f;
-}
-
-// MULTI = false: K <= 128, one chunk, logits kept in registers.
+// MULTI = false: K <= 128, one chunk, logits and exponentials kept in registers.
 // MULTI = true:  any K; pass 1 finds the max and the sum chunk by chunk, pass 2
 //                recomputes the logits to write the weights and accumulate the values.
 template <typename T, int DMAX, bool AF3, bool MULTI>
 __global__ void __launch_bounds__(kAttnThreads, 2) k_slot_attention(AttnArgs g) {
   extern __shared__ __align__(16) float smem[];
   constexpr int DW = DMAX < 32 ? DMAX : 32;            // channels per reduce-scatter
-  constexpr int NB = AF3 ? kAf3HeadsMax : 1;            // pair-bias heads kept per slot
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t b = blockIdx.y, a0 = (int64_t)blockIdx.x * g.QT;
-  const int QT = g.QT;
-  const int64_t K = g.K, A = g.A;
-  const int H = (int)g.H, D = (int)g.D, HD = H * D;
-  const int DP = g.DP, P = (int)g.P;
+  const int b = blockIdx.y, a0 = blockIdx.x * g.QT;
+  const int QT = g.QT, K = g.K, H = g.H, D = g.D, A = g.A, HD = H * D, DP = g.DP, P = g.P;
+  const int nq = min(QT, A - a0);                      // queries of this tile
+  const int slots = QT * K;
+  const bool vecD = (D & 3) == 0;                      // 16-byte rows of Q, K, V
+  const bool fullD = D == DMAX;                        // shared Q rows cover DMAX exactly
 
-  int *plan = reinterpret_cast<int *>(smem);                           // [QT*K]
-  float *kv = smem + (((int64_t)QT * K + 3) & ~int64_t(3));            // [kv_floats]
+  int *plan = reinterpret_cast<int *>(smem);                          // [QT*K]
+  float *beta = smem + ru4(slots);                                    // [H][QT*K] (AF3)
+  float *qs = beta + (AF3 ? ru4((size_t)H * slots) : 0);              // [QT][HD]
+  float *kv = qs + ru4((size_t)QT * HD);                              // [kv_floats]
   __shared__ int s_lo, s_hi;
-  __shared__ float s_wp[kPairMax * kAttnHeadsMax], s_wsum[kAttnHeadsMax];
+  __shared__ float s_wp[AF3 ? kPairMax * kAttnHeadsMax : 1], s_wsum[AF3 ? kAttnHeadsMax : 1];
   if (tid == 0) {
     s_lo = INT_MAX;
     s_hi = -1;
+  }
+
+  // ---------------- phase 0: the tile's Q rows -> shared (async), pair weights
+  const int64_t qbase = ((int64_t)b * A + a0) * HD;
+  if (vecD) {
+    for (int i = tid; i < nq * HD / 4; i += kAttnThreads) {
+      const uint32_t dst = (uint32_t)__cvta_generic_to_shared(qs + 4 * i);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(g.Q + qbase + 4 * i)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  } else {
+    for (int i = tid; i < nq * HD; i += kAttnThreads) qs[i] = g.Q[qbase + i];
   }
   if (AF3) {
     for (int i = tid; i < P * H; i += kAttnThreads) s_wp[i] = g.w_pair[i];
@@ -161,170 +214,201 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_slot_attention(AttnArgs g) 
   }
   __syncthreads();
 
-  // ---------------- phase 1: slot plan, one pass over the tile's key_index / window_mask
+  // ---------------- phase 1: slot plan (8 consecutive slots per thread) [+ pair bias]
   int lo = INT_MAX, hi = -1;
-  for (int q = warp; q < QT; q += kAttnWarps) {
-    const int64_t a = a0 + q;
-    const bool qok = a < A && g.usable[b * A + a] != 0;
-    for (int k = lane; k < (int)K; k += kWarp) {
-      int jj = -1;
-      if (qok) {
-        const int64_t s = (b * A + a) * K + k;
-        const int64_t j = g.key_index[s];
-        bool ok = j >= 0 && j < A && g.window[s] != 0;
-        ok = ok && g.usable[b * A + j] != 0;
-        if (ok && g.radius >= 0) ok = (j > a ? j - a : a - j) <= g.radius;
-        if (ok) {
-          jj = (int)j;
-          lo = min(lo, jj);
-          hi = max(hi, jj);
-        }
+  const int64_t sbase = ((int64_t)b * A + a0) * K;     // first slot of the tile
+  const int vslots = nq * K;
+  for (int s0 = tid * kPlanSlots; s0 < slots; s0 += kAttnThreads * kPlanSlots) {
+    int64_t kid[kPlanSlots];
+    uint8_t win[kPlanSlots];
+    const bool full = s0 + kPlanSlots <= vslots && ((sbase + s0) & 1) == 0;
+    if (full) {
+#pragma unroll
+      for (int e = 0; e < kPlanSlots; e += 2) {
+        const longlong2 v = *reinterpret_cast<const longlong2 *>(g.key_index + sbase + s0 + e);
+        kid[e] = v.x;
+        kid[e + 1] = v.y;
       }
-      plan[q * (int)K + k] = jj;
+      if (((sbase + s0) & 7) == 0) {
+        const uint2 w = *reinterpret_cast<const uint2 *>(g.window + sbase + s0);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          win[e] = (w.x >> (8 * e)) & 0xFF;
+          win[e + 4] = (w.y >> (8 * e)) & 0xFF;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < kPlanSlots; ++e) win[e] = g.window[sbase + s0 + e];
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < kPlanSlots; ++e) {
+        const bool in = s0 + e < vslots;
+        kid[e] = in ? g.key_index[sbase + s0 + e] : -1;
+        win[e] = in ? g.window[sbase + s0 + e] : 0;
+      }
+    }
+    int q = s0 / K, k = s0 - q * K;
+    bool quse = q < nq && g.usable[(int64_t)b * A + a0 + q] != 0;
+    int jj[kPlanSlots];
+#pragma unroll
+    for (int e = 0; e < kPlanSlots; ++e) {
+      if (k == K) {  // next query
+        k = 0;
+        ++q;
+        quse = q < nq && g.usable[(int64_t)b * A + a0 + q] != 0;
+      }
+      const int64_t j = kid[e];
+      const int a = a0 + q;
+      bool ok = quse && win[e] != 0 && j >= 0 && j < A;
+      if (ok && g.radius >= 0) ok = (j > a ? j - a : a - j) <= g.radius;
+      jj[e] = ok ? (int)j : -1;
+      ++k;
+    }
+#pragma unroll
+    for (int e = 0; e < kPlanSlots; ++e) {
+      if (jj[e] >= 0 && g.usable[(int64_t)b * A + jj[e]] == 0) jj[e] = -1;
+      if (s0 + e < slots) plan[s0 + e] = jj[e];
+      if (jj[e] >= 0) {
+        lo = min(lo, jj[e]);
+        hi = max(hi, jj[e]);
+      }
+    }
+    if (AF3) {
+#pragma unroll 1
+      for (int e = 0; e < kPlanSlots; ++e)
+        if (jj[e] >= 0)
+          slot_pair_bias<T>((const T *)g.pair + (sbase + s0 + e) * P, P, H, g.eps, s_wp, s_wsum,
+                            beta + s0 + e, slots);
     }
   }
-  if (lo <= hi) {
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  if (lane == 0 && lo <= hi) {
     atomicMin(&s_lo, lo);
     atomicMax(&s_hi, hi);
   }
+  if (vecD) asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
   const int klo = s_lo, khi = s_hi;
   const int span = khi >= klo ? khi - klo + 1 : 0;
   int HG = H;
   if (span > 0) {
-    const int64_t fit = g.kv_floats / (2 * (int64_t)span * DP);
-    HG = (int)(fit < H ? fit : H);
+    const int fit = g.kv_floats / (2 * span * DP);
+    HG = fit < H ? fit : H;
   }
   const bool staged = span > 0 && HG >= 1;
   if (!staged) HG = H;
-  if (AF3) HG = min(HG, kAf3HeadsMax);
   if (span > 0 && !staged && tid == 0) atomicOr(g.status, 1u);
-  const int nchunks = MULTI ? (int)((K + kChunk - 1) / kChunk) : 1;
-  const float log2e = 1.4426950408889634f;
+  const int nchunks = MULTI ? (K + kChunk - 1) / kChunk : 1;
 
   // ---------------- phase 2: head groups
   for (int h0 = 0; h0 < H; h0 += HG) {
     const int hg = H - h0 < HG ? H - h0 : HG;
-    float *ks = kv, *vs = kv + (int64_t)hg * span * DP;
+    float *ks = kv, *vs = kv + hg * span * DP;
     if (staged) {
-      // one float4 chunk of one staged row per lane: rows_per_pass rows per warp pass
       const int CH = DP / 4, rpp = kWarp / CH, rsub = lane / CH, c4 = (lane - rsub * CH) * 4;
-      const bool vec = (D & 3) == 0;
       for (int hl = 0; hl < hg; ++hl) {
-        const int64_t col = (int64_t)(h0 + hl) * D + c4;
+        const int col = (h0 + hl) * D + c4;
         for (int r0 = warp * rpp; r0 < span; r0 += kAttnWarps * rpp) {
           const int rr = r0 + rsub;
           if (rsub >= rpp || rr >= span) continue;
-          float4 kx = make_float4(0.f, 0.f, 0.f, 0.f), vx = kx;
-          const int64_t src = (b * A + klo + rr) * HD + col;
-          if (vec) {
-            if (c4 < D) {
-              kx = *reinterpret_cast<const float4 *>(g.Kf + src);
-              vx = *reinterpret_cast<const float4 *>(g.Vf + src);
-            }
+          const int64_t src = ((int64_t)b * A + klo + rr) * HD + col;
+          float *kd = ks + (hl * span + rr) * DP + c4, *vd = vs + (hl * span + rr) * DP + c4;
+          if (vecD && c4 < D) {
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                             (uint32_t)__cvta_generic_to_shared(kd)),
+                         "l"(g.Kf + src)
+                         : "memory");
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                             (uint32_t)__cvta_generic_to_shared(vd)),
+                         "l"(g.Vf + src)
+                         : "memory");
           } else {
-            float kk[4] = {0.f, 0.f, 0.f, 0.f}, vv[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int e = 0; e < 4; ++e)
-              if (c4 + e < D) {
-                kk[e] = g.Kf[src + e];
-                vv[e] = g.Vf[src + e];
-              }
-            kx = make_float4(kk[0], kk[1], kk[2], kk[3]);
-            vx = make_float4(vv[0], vv[1], vv[2], vv[3]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              kd[e] = c4 + e < D ? g.Kf[src + e] : 0.f;
+              vd[e] = c4 + e < D ? g.Vf[src + e] : 0.f;
+            }
           }
-          const int64_t dst = ((int64_t)hl * span + rr) * DP + c4;
-          *reinterpret_cast<float4 *>(ks + dst) = kx;
-          *reinterpret_cast<float4 *>(vs + dst) = vx;
         }
       }
+      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
     }
     __syncthreads();
 
-    for (int q = warp; q < QT; q += kAttnWarps) {
-      const int64_t a = a0 + q;
-      if (a >= A) break;
-      const int64_t arow = b * A + a;
-      const T *prow = AF3 ? (const T *)g.pair + arow * K * P : nullptr;
-
+    for (int q = warp; q < nq; q += kAttnWarps) {
+      const int a = a0 + q;
+      const int64_t arow = (int64_t)b * A + a;
       int jr[kSlotsPerLane];
-      float beta[kSlotsPerLane][NB];
       if (!MULTI) {
 #pragma unroll
         for (int i = 0; i < kSlotsPerLane; ++i) {
           const int k = i * kWarp + lane;
           jr[i] = k < K ? plan[q * K + k] : -1;
-          if (AF3) {
-            if (jr[i] >= 0)
-              pair_bias<T, NB>(prow + (int64_t)k * P, P, g.eps, s_wp, s_wsum, H, h0, hg, beta[i]);
-            else
-#pragma unroll
-              for (int x = 0; x < NB; ++x) beta[i][x] = 0.f;
-          }
         }
       }
-
       for (int hl = 0; hl < hg; ++hl) {
         const int h = h0 + hl;
-        float qv[DMAX];
-        const float *qsrc = g.Q + arow * HD + h * D;
-        if ((D & 3) == 0) {
+        const float *qv = qs + q * HD + h * D;
+        const float *kbase = staged ? ks + (hl * span - klo) * DP : nullptr;
+        const float *vbase = staged ? vs + (hl * span - klo) * DP : nullptr;
+        const float *bh = AF3 ? beta + h * slots + q * K : nullptr;
+        float qreg[DMAX];
+        if (!fullD || !staged) {
 #pragma unroll
-          for (int d = 0; d < DMAX; d += 4) {
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (d < D) x = *reinterpret_cast<const float4 *>(qsrc + d);
-            qv[d] = x.x;
-            qv[d + 1] = x.y;
-            qv[d + 2] = x.z;
-            qv[d + 3] = x.w;
-          }
-        } else {
-#pragma unroll
-          for (int d = 0; d < DMAX; ++d) qv[d] = d < D ? qsrc[d] : 0.f;
+          for (int d = 0; d < DMAX; ++d) qreg[d] = d < D ? qv[d] : 0.f;
         }
-        const float *kbase = staged ? ks + (int64_t)hl * span * DP : nullptr;
-        const float *vbase = staged ? vs + (int64_t)hl * span * DP : nullptr;
 
-        // logit in log2 units (exp2 of a difference of them = e^difference)
-        auto logit = [&](int64_t k, int i, int j) -> float {
-          float dot = staged ? dot_row<DMAX>(qv, kbase + (int64_t)(j - klo) * DP)
-                             : dot_global<DMAX>(qv, g.Kf + (b * A + j) * HD + h * D, D);
-          float l = dot * g.inv_sqrt_d;
-          if (AF3) {
-            if (!MULTI) {
-              float bsel = 0.f;
-#pragma unroll
-              for (int x = 0; x < NB; ++x)
-                if (x == hl) bsel = beta[i][x];
-              l += bsel;
-            } else {
-              float b1[1];
-              pair_bias<T, 1>(prow + k * P, P, g.eps, s_wp, s_wsum, H, h, 1, b1);
-              l += b1[0];
-            }
-          }
-          return l * log2e;
+        // logit of slot k (key j) in log2 units
+        auto logit = [&](int k, int j) -> float {
+          float dot;
+          if (staged && fullD)
+            dot = dot_row<DMAX>(qv, kbase + j * DP);
+          else if (staged)
+            dot = dot_plain<DMAX>(qreg, kbase + j * DP, D);
+          else
+            dot = dot_plain<DMAX>(qreg, g.Kf + ((int64_t)b * A + j) * HD + h * D, D);
+          float l = dot * g.scale_log2;
+          if (AF3) l = fmaf(bh[k], 1.4426950408889634f, l);
+          return l;
         };
 
         float mx = -INFINITY, sum = 0.f;
-        float l2[kSlotsPerLane];
-        for (int c = 0; c < nchunks; ++c) {
-          float cmx = -INFINITY;
+        float ev[kSlotsPerLane];
+        if (!MULTI) {
 #pragma unroll
           for (int i = 0; i < kSlotsPerLane; ++i) {
-            const int64_t k = (int64_t)c * kChunk + i * kWarp + lane;
-            if (MULTI) jr[i] = k < K ? plan[q * K + k] : -1;
-            l2[i] = jr[i] >= 0 ? logit(k, i, jr[i]) : -INFINITY;
-            cmx = fmaxf(cmx, l2[i]);
+            ev[i] = jr[i] >= 0 ? logit(i * kWarp + lane, jr[i]) : -INFINITY;
+            mx = fmaxf(mx, ev[i]);
           }
-          cmx = warp_max(cmx);
-          if (cmx > -INFINITY) {
-            const float nm = fmaxf(mx, cmx);
-            float cs = 0.f;
+          mx = warp_max(mx);
 #pragma unroll
-            for (int i = 0; i < kSlotsPerLane; ++i)
-              if (jr[i] >= 0) cs += exp2f(l2[i] - nm);
-            sum = sum * exp2f(mx - nm) + warp_sum(cs);
-            mx = nm;
+          for (int i = 0; i < kSlotsPerLane; ++i) {
+            ev[i] = jr[i] >= 0 ? exp2_approx(ev[i] - mx) : 0.f;
+            sum += ev[i];
+          }
+          sum = warp_sum(sum);
+        } else {
+          for (int c = 0; c < nchunks; ++c) {
+            float cmx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < kSlotsPerLane; ++i) {
+              const int k = c * kChunk + i * kWarp + lane;
+              jr[i] = k < K ? plan[q * K + k] : -1;
+              ev[i] = jr[i] >= 0 ? logit(k, jr[i]) : -INFINITY;
+              cmx = fmaxf(cmx, ev[i]);
+            }
+            cmx = warp_max(cmx);
+            if (cmx > -INFINITY) {
+              const float nm = fmaxf(mx, cmx);
+              float cs = 0.f;
+#pragma unroll
+              for (int i = 0; i < kSlotsPerLane; ++i)
+                if (jr[i] >= 0) cs += exp2_approx(ev[i] - nm);
+              sum = sum * exp2_approx(mx - nm) + warp_sum(cs);
+              mx = nm;
+            }
           }
         }
         const float inv = sum > 0.f ? 1.f / sum : 0.f;
@@ -332,30 +416,30 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_slot_attention(AttnArgs g) 
         float acc[DMAX];
 #pragma unroll
         for (int d = 0; d < DMAX; ++d) acc[d] = 0.f;
+        T *arow_out = (T *)g.attention + (((int64_t)b * H + h) * A + a) * K;
         for (int c = 0; c < nchunks; ++c) {
 #pragma unroll
           for (int i = 0; i < kSlotsPerLane; ++i) {
-            const int64_t k = (int64_t)c * kChunk + i * kWarp + lane;
+            const int k = c * kChunk + i * kWarp + lane;
             if (MULTI) {
               jr[i] = k < K ? plan[q * K + k] : -1;
-              l2[i] = jr[i] >= 0 ? logit(k, i, jr[i]) : -INFINITY;
+              ev[i] = jr[i] >= 0 ? exp2_approx(logit(k, jr[i]) - mx) : 0.f;
             }
             const int j = jr[i];
-            const float wgt = j >= 0 ? exp2f(l2[i] - mx) * inv : 0.f;
-            if (k < K) stf((T *)g.attention, ((b * H + h) * A + a) * K + k, wgt);
+            const float wgt = ev[i] * inv;
+            if (k < K) store_weight<T>(arow_out, k, wgt);
             if (j >= 0) {
-              if (staged) {
-                const float *vr = vbase + (int64_t)(j - klo) * DP;
+              if (staged && vecD) {
+                const float *vr = vbase + j * DP;
 #pragma unroll
                 for (int d = 0; d < DMAX; d += 4) {
                   const float4 v = *reinterpret_cast<const float4 *>(vr + d);
-                  acc[d] = fmaf(wgt, v.x, acc[d]);
-                  acc[d + 1] = fmaf(wgt, v.y, acc[d + 1]);
-                  acc[d + 2] = fmaf(wgt, v.z, acc[d + 2]);
-                  acc[d + 3] = fmaf(wgt, v.w, acc[d + 3]);
+                  fma2(acc[d], acc[d + 1], wgt, wgt, v.x, v.y);
+                  fma2(acc[d + 2], acc[d + 3], wgt, wgt, v.z, v.w);
                 }
               } else {
-                const float *vr = g.Vf + (b * A + j) * HD + h * D;
+                const float *vr =
+                    staged ? vbase + j * DP : g.Vf + ((int64_t)b * A + j) * HD + h * D;
 #pragma unroll
                 for (int d = 0; d < DMAX; ++d)
                   if (d < D) acc[d] = fmaf(wgt, vr[d], acc[d]);
