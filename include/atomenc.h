@@ -64,7 +64,9 @@ enum atomenc_status {
   ATOMENC_ERR_ODD_HEAD = -8,    /* ESMFold2 style with odd D (half-split rotary) */
   ATOMENC_ERR_UNSUPPORTED = -9, /* a size outside what the kernels are built for */
   ATOMENC_ERR_WORKSPACE = -10,  /* workspace NULL, too small or not 256-byte aligned */
-  ATOMENC_ERR_CUDA = -11        /* the CUDA runtime rejected a launch */
+  ATOMENC_ERR_CUDA = -11,       /* the CUDA runtime rejected a launch */
+  ATOMENC_ERR_TOO_LARGE = -12   /* atomenc_forward_noalloc: the shapes need more scratch
+                                   than its fixed device array holds */
 };
 
 typedef struct {
@@ -182,6 +184,33 @@ int atomenc_forward_profiled(int style, int stage, const atomenc_inputs *in,
  * (slower, same result). Never an error; returns enum atomenc_status.
  */
 int atomenc_get_status(const void *workspace, int *device_status, atomenc_stream_t stream);
+
+/*
+ * Forward pass that allocates nothing and takes no workspace argument.
+ *
+ * For callers that cannot call cudaMalloc (or have the library do it): code running
+ * inside a CUDA stream capture of another framework, where allocation calls are not
+ * allowed; hosts whose memory pool owns all device memory and must not see memory
+ * taken behind its back; latency-critical loops that cannot afford the implicit
+ * synchronisation an allocation may bring. They pass inputs and outputs as for
+ * atomenc_forward; the scratch the pass needs lives in one file-scope device array
+ * of ATOMENC_NOALLOC_SCRATCH_BYTES (64 MiB) inside this library, which every GPU that
+ * loads the library keeps until the process exits.
+ *  - The first call on a device (with that device current) looks up the array's
+ *    device address once (cudaGetSymbolAddress); make that first call before any
+ *    stream capture. Later calls only enqueue work on `stream`.
+ *  - Shapes whose atomenc_workspace_size() exceeds the array are rejected with
+ *    ATOMENC_ERR_TOO_LARGE before anything is enqueued.
+ *  - All calls share the one array and it keeps the last call's contents; each call
+ *    clears what it needs zeroed itself. Two calls whose GPU work overlaps (different
+ *    streams without ordering, or different host threads) race on the array: order
+ *    them on one stream.
+ * No counterpart on the pages; results and other errors are those of atomenc_forward.
+ */
+#define ATOMENC_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+int atomenc_forward_noalloc(int style, int stage, const atomenc_inputs *in,
+                            const atomenc_params *params, double eps, int64_t radius,
+                            const atomenc_outputs *out, atomenc_stream_t stream);
 
 /* Static English text for an atomenc_status code. */
 const char *atomenc_strerror(int code);

@@ -76,6 +76,10 @@ def load_library() -> ctypes.CDLL:
         lib.atomenc_forward_profiled.restype = ctypes.c_int
         lib.atomenc_forward_profiled.argtypes = lib.atomenc_forward.argtypes + [
             P(ctypes.c_void_p), ctypes.c_int, P(ctypes.c_int)]
+        lib.atomenc_forward_noalloc.restype = ctypes.c_int
+        lib.atomenc_forward_noalloc.argtypes = [ctypes.c_int, ctypes.c_int, P(AtomencInputs),
+                                                P(AtomencParams), ctypes.c_double, ctypes.c_int64,
+                                                P(AtomencOutputs), ctypes.c_void_p]
         lib.atomenc_get_status.restype = ctypes.c_int
         lib.atomenc_get_status.argtypes = [ctypes.c_void_p, P(ctypes.c_int), ctypes.c_void_p]
         lib.atomenc_strerror.restype = ctypes.c_char_p
@@ -143,6 +147,25 @@ def atomenc_forward(style: str, stage: str, inputs: dict, params: dict, eps: flo
                                         _stream_ptr(stream))
     if rc != 0:
         raise AtomencError(rc, "atomenc_forward")
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def atomenc_forward_noalloc(style: str, stage: str, inputs: dict, params: dict, eps: float,
+                            radius: int, outputs: dict, stream=None) -> None:
+    """Forward pass that allocates nothing: the library's own fixed 64 MiB device
+    array is its scratch, so no workspace is passed. For callers that may not allocate
+    device memory (inside another framework's stream capture, under a host allocator
+    that owns all memory, in latency-critical loops). The first call on a device sets
+    the array's address up and should come before any stream capture; calls whose GPU
+    work overlaps share the array and race, so order them on one stream."""
+    ins, prm, outs = _structs(inputs, params, outputs)
+    rc = load_library().atomenc_forward_noalloc(STYLES[style], STAGES[stage], ctypes.byref(ins),
+                                                ctypes.byref(prm), float(eps), int(radius),
+                                                ctypes.byref(outs), _stream_ptr(stream))
+    if rc != 0:
+        raise AtomencError(rc, "atomenc_forward_noalloc")
 
 
 NUM_PHASES = 6

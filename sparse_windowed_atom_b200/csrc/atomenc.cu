@@ -10,6 +10,7 @@
 #include <climits>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <type_traits>
 
 #include "../../include/atomenc.h"
@@ -591,6 +592,40 @@ int atomenc_forward_profiled(int style, int stage, const atomenc_inputs *in,
   return rc;
 }
 
+// ---- no-allocation variant: scratch in a file-scope device array, address looked up
+// once per device with that device current
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATOMENC_NOALLOC_SCRATCH_BYTES];
+constexpr int kMaxDevices = 64;
+static void *g_noalloc_addr[kMaxDevices];
+static std::mutex g_noalloc_mutex;
+
+static int noalloc_scratch(void **ptr) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATOMENC_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATOMENC_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ATOMENC_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *ptr = g_noalloc_addr[dev];
+  return ATOMENC_OK;
+}
+
+int atomenc_forward_noalloc(int style, int stage, const atomenc_inputs *in,
+                            const atomenc_params *params, double eps, int64_t radius,
+                            const atomenc_outputs *out, atomenc_stream_t stream) {
+  Plan pl;
+  CHECK(validate(style, stage, in, params, out, pl));
+  if (pl.bytes > ATOMENC_NOALLOC_SCRATCH_BYTES) return ATOMENC_ERR_TOO_LARGE;
+  void *scratch = nullptr;
+  CHECK(noalloc_scratch(&scratch));
+  Hooks hk;
+  return forward_impl(style, stage, in, params, eps, radius, out, scratch,
+                      ATOMENC_NOALLOC_SCRATCH_BYTES, stream, hk);
+}
+
 int atomenc_get_status(const void *workspace, int *device_status, atomenc_stream_t stream) {
   if (!workspace || !device_status) return ATOMENC_ERR_NULL;
   unsigned v = 0;
@@ -616,6 +651,8 @@ const char *atomenc_strerror(int code) {
     case ATOMENC_ERR_UNSUPPORTED: return "a size is outside what the kernels are built for";
     case ATOMENC_ERR_WORKSPACE: return "workspace is NULL, too small or not 256-byte aligned";
     case ATOMENC_ERR_CUDA: return "the CUDA runtime rejected a launch";
+    case ATOMENC_ERR_TOO_LARGE:
+      return "the shapes need more scratch than the no-allocation entry point's fixed 64 MiB array";
     default: return "unknown atomenc status";
   }
 }
