@@ -197,7 +197,7 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
     CHECK(check_tensor(out->hidden, fdt, 3, hc));
     CHECK(check_tensor(out->attention, fdt, 4, at));
   }
-  if (D > kMaxD || A >= INT_MAX || K >= INT_MAX / 64) return ATOMENC_ERR_UNSUPPORTED;
+  if (D > kMaxD || A >= INT_MAX || K > 8192) return ATOMENC_ERR_UNSUPPORTED;
 
   // ---- workspace plan
   const int64_t R = B * A;
@@ -470,6 +470,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   ag.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   ag.eps = eps;
   ag.QT = pl.QT; ag.DP = pl.DP; ag.kv_floats = pl.kv_floats;
+  ag.kmagic = K > 1 ? (uint32_t)(((uint64_t)1 << 32) / (uint64_t)K + (((uint64_t)1 << 32) % (uint64_t)K != 0)) : 0u;
   ag.Q = F(pl.o_q); ag.Kf = F(pl.o_k); ag.Vf = F(pl.o_v); ag.G = F(pl.o_g);
   ag.key_index = static_cast<const int64_t *>(in->key_index.data);
   ag.window = static_cast<const uint8_t *>(in->window_mask.data);

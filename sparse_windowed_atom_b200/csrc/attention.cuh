@@ -11,11 +11,12 @@
 //
 // One CTA (256 threads, two per SM) owns QT consecutive queries of one batch element.
 //  Phase 0  the tile's Q rows are copied to shared memory with cp.async.
-//  Phase 1  each thread reads 8 consecutive slots of the tile's key_index / window_mask
-//           (16-byte loads), decides eligibility and writes the slot plan (key id or -1)
-//           and the span [klo, khi] of the permitted ids; AF3: the pair bias of every
-//           permitted (slot, head) is computed from its pair row (LayerNorm over P,
-//           one pass) and kept in shared memory as float32 [head][slot].
+//  Phase 1  one slot per thread per round (four rounds in flight): key_index and
+//           window_mask are read once (coalesced), eligibility decided and the slot plan
+//           (key id or -1) written with the span [klo, khi] of the permitted ids; AF3:
+//           the pair bias of every permitted (slot, head) is computed from its pair row
+//           (16-byte loads, LayerNorm over P in one shifted pass) and kept in shared
+//           memory as float32 [head][slot].
 //  Phase 2  head groups: the K and V rows of the span for as many heads as fit are staged
 //           (float32, cp.async); each warp takes one query at a time, lanes over the slots
 //           (4 per lane per 128-slot chunk): logits, max, one exp2 per entry, sum, weights
@@ -38,7 +39,6 @@ constexpr int kPairMax = 32;
 constexpr int kSlotsPerLane = 4;                       // one chunk = 128 slots
 constexpr int kChunk = kWarp * kSlotsPerLane;
 constexpr int kAttnHeadsMax = 32;                      // AF3 w_pair columns in shared memory
-constexpr int kPlanSlots = 8;                          // slots per thread in phase 1
 
 struct AttnArgs {
   int B, A, K, H, D, P;
@@ -46,6 +46,7 @@ struct AttnArgs {
   float scale_log2;               // log2(e) / sqrt(D)
   float eps;
   int QT, DP, kv_floats;          // queries per CTA, padded row width, K/V stage size
+  uint32_t kmagic;                // ceil(2^32 / K) for K > 1: s / K == umulhi(s, kmagic), s < QT*K
   const float *Q, *Kf, *Vf, *G;   // [B*A, H*D]
   const int64_t *key_index;       // [B, A, K]
   const uint8_t *window;          // [B, A, K]
@@ -114,31 +115,94 @@ __device__ __forceinline__ float reduce_scatter(float (&v)[W], int lane) {
   return v[0];
 }
 
-// pair row of one slot -> bias for every head: rstd * (sum_p y_p W'[p,h] - m * sum_p W'[p,h]),
-// y = pair - pair_0 (shift for a well-conditioned one-pass variance), m = mean(y)
-template <typename T>
-__device__ __forceinline__ void slot_pair_bias(const T *pr, int P, int H, float eps,
+// Pair bias of one slot for every head:
+//   beta_h = sum_p LN(pair)_p * pair_scale_p * w_pair[p, h]
+//          = rstd * (sum_p y_p W'[p, h] - m * sum_p W'[p, h]),
+// y_p = pair_p - pair_0 (a shift that keeps the one-pass variance well conditioned),
+// m = mean(y), rstd = 1 / sqrt(mean(y^2) - m^2 + eps); W' = pair_scale * w_pair and its
+// column sums are in shared memory ([P][H] and [H]).
+template <int NP>
+__device__ __forceinline__ void pair_bias_from(const float (&x)[NP], int P, int H, float eps,
                                                const float *wp, const float *wsum, float *out,
                                                int out_stride) {
-  float y[kPairMax];
-  const float x0 = ldf(pr, 0);
+  float y[NP];
   float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-  for (int p = 0; p < kPairMax; ++p)
-    if (p < P) {
-      y[p] = ldf(pr, p) - x0;
-      s1 += y[p];
-      s2 = fmaf(y[p], y[p], s2);
-    }
-  const float invP = 1.f / (float)P;
+  for (int p = 0; p < NP; ++p) {
+    y[p] = x[p] - x[0];
+    s1 += y[p];
+    s2 = fmaf(y[p], y[p], s2);
+  }
+  const float invP = 1.f / (float)NP;
   const float m = s1 * invP;
   const float var = fmaxf(s2 * invP - m * m, 0.f);
   const float rstd = rsqrtf(var + eps);
-  for (int h = 0; h < H; ++h) {
+  int h = 0;
+  if ((H & 3) == 0) {
+    for (; h < H; h += 4) {
+      float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        const float4 w = *reinterpret_cast<const float4 *>(wp + p * H + h);
+        d0 = fmaf(y[p], w.x, d0);
+        d1 = fmaf(y[p], w.y, d1);
+        d2 = fmaf(y[p], w.z, d2);
+        d3 = fmaf(y[p], w.w, d3);
+      }
+      out[(h + 0) * out_stride] = rstd * (d0 - m * wsum[h + 0]);
+      out[(h + 1) * out_stride] = rstd * (d1 - m * wsum[h + 1]);
+      out[(h + 2) * out_stride] = rstd * (d2 - m * wsum[h + 2]);
+      out[(h + 3) * out_stride] = rstd * (d3 - m * wsum[h + 3]);
+    }
+  }
+  for (; h < H; ++h) {
     float d = 0.f;
 #pragma unroll
-    for (int p = 0; p < kPairMax; ++p)
-      if (p < P) d = fmaf(y[p], wp[p * H + h], d);
+    for (int p = 0; p < NP; ++p) d = fmaf(y[p], wp[p * H + h], d);
+    out[h * out_stride] = rstd * (d - m * wsum[h]);
+  }
+}
+
+// 16 channels of a pair row by 16-byte loads (bf16: 2 loads, float32: 4 loads)
+__device__ __forceinline__ void load_pair16(const __nv_bfloat16 *pr, float (&x)[16]) {
+  const uint4 a = *reinterpret_cast<const uint4 *>(pr);
+  const uint4 b = *reinterpret_cast<const uint4 *>(pr + 8);
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void load_pair16(const float *pr, float (&x)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 v = *reinterpret_cast<const float4 *>(pr + 4 * i);
+    x[4 * i] = v.x;
+    x[4 * i + 1] = v.y;
+    x[4 * i + 2] = v.z;
+    x[4 * i + 3] = v.w;
+  }
+}
+
+// generic P (any width up to kPairMax): scalar loads
+template <typename T>
+__device__ __forceinline__ void pair_bias_generic(const T *pr, int P, int H, float eps,
+                                                  const float *wp, const float *wsum, float *out,
+                                                  int out_stride) {
+  const float x0 = ldf(pr, 0);
+  float s1 = 0.f, s2 = 0.f;
+  for (int p = 0; p < P; ++p) {
+    const float y = ldf(pr, p) - x0;
+    s1 += y;
+    s2 = fmaf(y, y, s2);
+  }
+  const float m = s1 / (float)P;
+  const float var = fmaxf(s2 / (float)P - m * m, 0.f);
+  const float rstd = rsqrtf(var + eps);
+  for (int h = 0; h < H; ++h) {
+    float d = 0.f;
+    for (int p = 0; p < P; ++p) d = fmaf(ldf(pr, p) - x0, wp[p * H + h], d);
     out[h * out_stride] = rstd * (d - m * wsum[h]);
   }
 }
@@ -186,7 +250,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_slot_attention(AttnArgs g) 
   float *qs = beta + (AF3 ? ru4((size_t)H * slots) : 0);              // [QT][HD]
   float *kv = qs + ru4((size_t)QT * HD);                              // [kv_floats]
   __shared__ int s_lo, s_hi;
-  __shared__ float s_wp[AF3 ? kPairMax * kAttnHeadsMax : 1], s_wsum[AF3 ? kAttnHeadsMax : 1];
+  __shared__ __align__(16) float s_wp[AF3 ? kPairMax * kAttnHeadsMax : 4];  // float4 rows
+  __shared__ __align__(16) float s_wsum[AF3 ? kAttnHeadsMax : 4];
   if (tid == 0) {
     s_lo = INT_MAX;
     s_hi = -1;
@@ -214,72 +279,44 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_slot_attention(AttnArgs g) 
   }
   __syncthreads();
 
-  // ---------------- phase 1: slot plan (8 consecutive slots per thread) [+ pair bias]
+  // ---------------- phase 1a: slot plan, one slot per thread per round (coalesced
+  // 8-byte key_index loads, consecutive shared stores), four rounds in flight
   int lo = INT_MAX, hi = -1;
   const int64_t sbase = ((int64_t)b * A + a0) * K;     // first slot of the tile
   const int vslots = nq * K;
-  for (int s0 = tid * kPlanSlots; s0 < slots; s0 += kAttnThreads * kPlanSlots) {
-    int64_t kid[kPlanSlots];
-    uint8_t win[kPlanSlots];
-    const bool full = s0 + kPlanSlots <= vslots && ((sbase + s0) & 1) == 0;
-    if (full) {
+  constexpr int R = 4;
+  for (int s0 = tid; s0 < slots; s0 += kAttnThreads * R) {
+    int64_t kid[R];
+    uint8_t win[R];
 #pragma unroll
-      for (int e = 0; e < kPlanSlots; e += 2) {
-        const longlong2 v = *reinterpret_cast<const longlong2 *>(g.key_index + sbase + s0 + e);
-        kid[e] = v.x;
-        kid[e + 1] = v.y;
-      }
-      if (((sbase + s0) & 7) == 0) {
-        const uint2 w = *reinterpret_cast<const uint2 *>(g.window + sbase + s0);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          win[e] = (w.x >> (8 * e)) & 0xFF;
-          win[e + 4] = (w.y >> (8 * e)) & 0xFF;
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < kPlanSlots; ++e) win[e] = g.window[sbase + s0 + e];
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < kPlanSlots; ++e) {
-        const bool in = s0 + e < vslots;
-        kid[e] = in ? g.key_index[sbase + s0 + e] : -1;
-        win[e] = in ? g.window[sbase + s0 + e] : 0;
-      }
+    for (int u = 0; u < R; ++u) {
+      const int s = s0 + u * kAttnThreads;
+      const bool in = s < vslots;
+      kid[u] = in ? g.key_index[sbase + s] : -1;
+      win[u] = in ? g.window[sbase + s] : 0;
     }
-    int q = s0 / K, k = s0 - q * K;
-    bool quse = q < nq && g.usable[(int64_t)b * A + a0 + q] != 0;
-    int jj[kPlanSlots];
+    int jj[R];
+    bool qu[R];
 #pragma unroll
-    for (int e = 0; e < kPlanSlots; ++e) {
-      if (k == K) {  // next query
-        k = 0;
-        ++q;
-        quse = q < nq && g.usable[(int64_t)b * A + a0 + q] != 0;
-      }
-      const int64_t j = kid[e];
+    for (int u = 0; u < R; ++u) {
+      const int s = s0 + u * kAttnThreads;
+      const int q = K == 1 ? s : (int)__umulhi((uint32_t)s, g.kmagic);
       const int a = a0 + q;
-      bool ok = quse && win[e] != 0 && j >= 0 && j < A;
+      const int64_t j = kid[u];
+      bool ok = s < vslots && win[u] != 0 && j >= 0 && j < A;
       if (ok && g.radius >= 0) ok = (j > a ? j - a : a - j) <= g.radius;
-      jj[e] = ok ? (int)j : -1;
-      ++k;
+      jj[u] = ok ? (int)j : -1;
+      qu[u] = s < vslots && g.usable[(int64_t)b * A + a] != 0;
     }
 #pragma unroll
-    for (int e = 0; e < kPlanSlots; ++e) {
-      if (jj[e] >= 0 && g.usable[(int64_t)b * A + jj[e]] == 0) jj[e] = -1;
-      if (s0 + e < slots) plan[s0 + e] = jj[e];
-      if (jj[e] >= 0) {
-        lo = min(lo, jj[e]);
-        hi = max(hi, jj[e]);
+    for (int u = 0; u < R; ++u) {
+      const int s = s0 + u * kAttnThreads;
+      if (jj[u] >= 0 && (!qu[u] || g.usable[(int64_t)b * A + jj[u]] == 0)) jj[u] = -1;
+      if (s < slots) plan[s] = jj[u];
+      if (jj[u] >= 0) {
+        lo = min(lo, jj[u]);
+        hi = max(hi, jj[u]);
       }
-    }
-    if (AF3) {
-#pragma unroll 1
-      for (int e = 0; e < kPlanSlots; ++e)
-        if (jj[e] >= 0)
-          slot_pair_bias<T>((const T *)g.pair + (sbase + s0 + e) * P, P, H, g.eps, s_wp, s_wsum,
-                            beta + s0 + e, slots);
     }
   }
   lo = __reduce_min_sync(0xffffffffu, lo);
@@ -287,6 +324,27 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_slot_attention(AttnArgs g) 
   if (lane == 0 && lo <= hi) {
     atomicMin(&s_lo, lo);
     atomicMax(&s_hi, hi);
+  }
+  // ---------------- phase 1b (AF3): pair bias of every permitted (slot, head), one slot
+  // per thread per round, rows read with 16-byte loads, two rows in flight
+  if (AF3) {
+    __syncthreads();
+    const T *pbase = (const T *)g.pair + sbase * P;
+    const bool p16 = P == 16;
+    for (int s0 = tid; s0 < vslots; s0 += 2 * kAttnThreads) {
+      const int s1 = s0 + kAttnThreads;
+      const bool on0 = plan[s0] >= 0, on1 = s1 < vslots && plan[s1] >= 0;
+      if (p16) {
+        float x0[16], x1[16];
+        if (on0) load_pair16(pbase + (int64_t)s0 * 16, x0);
+        if (on1) load_pair16(pbase + (int64_t)s1 * 16, x1);
+        if (on0) pair_bias_from<16>(x0, P, H, g.eps, s_wp, s_wsum, beta + s0, slots);
+        if (on1) pair_bias_from<16>(x1, P, H, g.eps, s_wp, s_wsum, beta + s1, slots);
+      } else {
+        if (on0) pair_bias_generic<T>(pbase + (int64_t)s0 * P, P, H, g.eps, s_wp, s_wsum, beta + s0, slots);
+        if (on1) pair_bias_generic<T>(pbase + (int64_t)s1 * P, P, H, g.eps, s_wp, s_wsum, beta + s1, slots);
+      }
+    }
   }
   if (vecD) asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
@@ -459,7 +517,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_slot_attention(AttnArgs g) 
           const int d = part + (lane & (DW - 1));
           if (lane < DW && d < D) {
             const int64_t oi = arow * HD + h * D + d;
-            g.O[oi] = has ? o * sigmoidf_(g.G[oi]) : 0.f;
+            g.O[oi] = has ? o * sigmoid_fast(g.G[oi]) : 0.f;
           }
         }
       }

@@ -40,7 +40,7 @@ struct EpiCondAF3 {
         const int ce = c + e;
         if (ce >= N) break;
         const int be = ce / Ci, he = ce - be * Ci;
-        out[r * 6 * C + ce] = (be & 1) ? v[e] : sigmoidf_(v[e] + b_scale[(be >> 1) * Ci + he]);
+        out[r * 6 * C + ce] = (be & 1) ? v[e] : sigmoid_fast(v[e] + b_scale[(be >> 1) * Ci + he]);
       }
       return;
     }
@@ -48,10 +48,10 @@ struct EpiCondAF3 {
     float4 o = make_float4(v[0], v[1], v[2], v[3]);
     if ((blk & 1) == 0) {  // scale block j = blk / 2
       const float *bs = b_scale + (blk >> 1) * Ci + ch;
-      o.x = sigmoidf_(v[0] + bs[0]);
-      o.y = sigmoidf_(v[1] + bs[1]);
-      o.z = sigmoidf_(v[2] + bs[2]);
-      o.w = sigmoidf_(v[3] + bs[3]);
+      o.x = sigmoid_fast(v[0] + bs[0]);
+      o.y = sigmoid_fast(v[1] + bs[1]);
+      o.z = sigmoid_fast(v[2] + bs[2]);
+      o.w = sigmoid_fast(v[3] + bs[3]);
     }
     *reinterpret_cast<float4 *>(out + r * 6 * C + c0) = o;
   }
@@ -67,12 +67,12 @@ struct EpiGateAF3 {
     if (C & 1) {
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        if (c0 + e < N) out[r * 2 * C + c0 + e] = sigmoidf_(v[e] + b[e]);
+        if (c0 + e < N) out[r * 2 * C + c0 + e] = sigmoid_fast(v[e] + b[e]);
       return;
     }
     *reinterpret_cast<float4 *>(out + r * 2 * C + c0) =
-        make_float4(sigmoidf_(v[0] + b[0]), sigmoidf_(v[1] + b[1]), sigmoidf_(v[2] + b[2]),
-                    sigmoidf_(v[3] + b[3]));
+        make_float4(sigmoid_fast(v[0] + b[0]), sigmoid_fast(v[1] + b[1]), sigmoid_fast(v[2] + b[2]),
+                    sigmoid_fast(v[3] + b[3]));
   }
 };
 
@@ -127,7 +127,7 @@ struct EpiSwiGLU {
   __device__ void quad(int64_t r, int64_t c0, const float (&v)[4], int64_t N) const {
 #pragma unroll
     for (int p = 0; p < 2; ++p)
-      if (c0 + 2 * p + 1 < N) h[r * Mh + c0 / 2 + p] = siluf_(v[2 * p]) * v[2 * p + 1];
+      if (c0 + 2 * p + 1 < N) h[r * Mh + c0 / 2 + p] = silu_fast(v[2 * p]) * v[2 * p + 1];
   }
 };
 

@@ -289,22 +289,26 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
   bool ok = true;
 
   if (warp < 4) {
-    // ---- A: rows 32w..32w+31 of the tile, every k chunk, bf16 (hi[, lo]) swizzled
+    // ---- A: rows 32w..32w+31 of the tile, every k chunk, bf16 (hi[, lo]) swizzled;
+    // the 8 row-segments of a chunk are loaded before any is converted (8 loads in flight)
     for (int c = 0; c < nkc; ++c) {
       uint8_t *a_c = sA + (size_t)c * PARTS * BLK;
-#pragma unroll 2
+      float v[8][8];
+#pragma unroll
+      for (int it = 0; it < 8; ++it)
+        load8<TA>(A, lda, M, K, m0 + warp * 32 + it * 4 + (lane >> 3),
+                  (int64_t)c * kUmmaBK + (lane & 7) * 8, v[it]);
+#pragma unroll
       for (int it = 0; it < 8; ++it) {
         const int r = warp * 32 + it * 4 + (lane >> 3), seg = lane & 7;
-        float v[8];
-        load8<TA>(A, lda, M, K, m0 + r, (int64_t)c * kUmmaBK + seg * 8, v);
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const uint16_t h0 = umma::bf16_bits(v[2 * e]), h1 = umma::bf16_bits(v[2 * e + 1]);
+          const uint16_t h0 = umma::bf16_bits(v[it][2 * e]), h1 = umma::bf16_bits(v[it][2 * e + 1]);
           hi[e] = (uint32_t)h0 | ((uint32_t)h1 << 16);
           if (SPLIT) {
-            const uint16_t l0 = umma::bf16_bits(v[2 * e] - umma::bf16_val(h0));
-            const uint16_t l1 = umma::bf16_bits(v[2 * e + 1] - umma::bf16_val(h1));
+            const uint16_t l0 = umma::bf16_bits(v[it][2 * e] - umma::bf16_val(h0));
+            const uint16_t l1 = umma::bf16_bits(v[it][2 * e + 1] - umma::bf16_val(h1));
             lo[e] = (uint32_t)l0 | ((uint32_t)l1 << 16);
           }
         }
