@@ -247,37 +247,68 @@ def run_reference(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- ranks
+
+class Ranks:
+    """One process per GPU (torchrun env: RANK, LOCAL_RANK, WORLD_SIZE, MASTER_*).
+    Every rank runs its own replica of the workload on its own seeded batch; the only
+    collectives are the barrier around the timed region and the max over ranks of the
+    device time (no collective on the data path)."""
+
+    def __init__(self, backend: str = "nccl", device=None, timeout_s: int = 120):
+        import torch
+        import torch.distributed as dist
+        self.dist, self.torch = dist, torch
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.device = device if device is not None else torch.device("cpu")
+        if self.world > 1:
+            kw = {"device_id": self.device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+
+    def seed(self) -> int:
+        return self.rank
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max(self, x: float) -> float:
+        if self.world == 1:
+            return x
+        t = self.torch.tensor([x], dtype=self.torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def job_rate(self, units_per_rank: float, ms_per_step: float) -> float:
+        """Whole-job throughput: the units every rank processed per step over the
+        slowest rank's time per step."""
+        return units_per_rank * self.world / (ms_per_step / 1e3)
+
+    def close(self):
+        if self.world > 1:
+            self.dist.destroy_process_group()
+
+
 # ----------------------------------------------------------------------------- GPU arm
 
 def run_atomenc(args):
     import torch
-    import torch.distributed as dist
 
     from sparse_windowed_atom_b200 import atomenc
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (no CPU path exists)")
+    local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     spec = workloads.WORKLOADS[args.workload]
-    w = workloads.make_inputs(spec, seed=rank)
+    w = workloads.make_inputs(spec, seed=ranks.seed())
     fdt = torch.bfloat16 if spec.dtype == "bfloat16" else torch.float32
     host = {}
     for grp in ("activations", "parameters"):
@@ -342,7 +373,7 @@ def run_atomenc(args):
     total_ms = max_over_ranks(sum(step_ms))
     ms_per_step = total_ms / K
     atoms = spec.atoms * world
-    value = atoms / (ms_per_step / 1e3)
+    value = ranks.job_rate(spec.atoms, ms_per_step)
 
     # ---- roofline of the slot-attention kernel (timed live, phase 3 = that kernel alone)
     attn_ms = max_over_ranks(phase_ms[3])
@@ -385,7 +416,7 @@ def run_atomenc(args):
         torch.cuda.synchronize(dev)
         barrier()
         e_ms = max_over_ranks(e0.elapsed_time(e1)) / ke
-        e2e = {"value": atoms / (e_ms / 1e3), "unit": "atoms/s", "h2d_bytes_per_step": h2d * world,
+        e2e = {"value": ranks.job_rate(spec.atoms, e_ms), "unit": "atoms/s", "h2d_bytes_per_step": h2d * world,
                "d2h_bytes_per_step": d2h * world, "ms_per_step": e_ms, "steps": ke}
 
     cpu = None
@@ -401,7 +432,7 @@ def run_atomenc(args):
             "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded workload generator; no dataset)",
             "config": config_of(spec, world),
-            "entries_per_s": spec.entries * world / (ms_per_step / 1e3),
+            "entries_per_s": ranks.job_rate(spec.entries, ms_per_step),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches,
             "clocks": sampler.summary(),
@@ -410,8 +441,7 @@ def run_atomenc(args):
             "device_status": status,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    ranks.close()
     return 0
 
 
