@@ -67,7 +67,7 @@ struct Plan {
   bool af3 = false, enc = false;
   Dims d;
   // workspace layout (byte offsets)
-  size_t o_status, o_usable, o_first, o_last, o_tp, o_x, o_opc, o_rawc, o_cond, o_gate, o_feat,
+  size_t o_status, o_usable, o_xstats, o_first, o_last, o_tp, o_x, o_opc, o_rawc, o_cond, o_gate, o_feat,
       o_q, o_k, o_v, o_g, o_o, o_xp, o_z, o_h, o_hid, o_pool;
   size_t o_wcond, o_wgate, o_wqkv, o_wout, o_wff1, o_wff2, o_wpool, o_wtok, o_wread, o_bscale,
       o_brg, o_bq, o_wpair, o_rscale, o_rbias;
@@ -204,6 +204,7 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   size_t cur = 0;
   pl.o_status = take(cur, 256);
   pl.o_usable = take(cur, R);
+  pl.o_xstats = take(cur, R * 2 * 4);
   pl.o_first = take(cur, pl.enc ? B * T * 4 : 0);
   pl.o_last = take(cur, pl.enc ? B * T * 4 : 0);
   pl.o_tp = take(cur, pl.enc ? 0 : B * T * C * 4);
@@ -212,7 +213,8 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   pl.o_rawc = take(cur, pl.af3 ? R * S * 4 : 0);
   pl.o_cond = take(cur, R * 6 * C * 4);
   pl.o_gate = take(cur, pl.af3 ? R * 2 * C * 4 : 0);
-  pl.o_feat = take(cur, R * (pl.af3 ? 2 : 1) * C * 4);
+  const bool fused = C <= kRowsKMax;
+  pl.o_feat = take(cur, fused ? 0 : R * (pl.af3 ? 2 : 1) * C * 4);
   pl.o_q = take(cur, R * HD * 4);
   pl.o_k = take(cur, R * HD * 4);
   pl.o_v = take(cur, R * HD * 4);
@@ -378,36 +380,50 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   k_pack_weights<<<dim3(64, pj.n), 256, 0, st>>>(pj);
   ++hk.launches;
 
-  // out = epi(A @ W) on the tensor cores; W given by its packed image. K <= 256: the
-  // row-block kernel (A resident, weights streamed); larger K: the streaming kernel.
+  // out = epi(A' @ W) on the tensor cores, W given by its packed image and A' produced by
+  // `prod` (A itself, or a row normalisation fused into the operand); K <= 256
+  auto gemm_rows = [&](auto prod, size_t wpk, int64_t Mr, int64_t N, int64_t Kd, auto epi) {
+    using P = decltype(prod);
+    using E = decltype(epi);
+    const int64_t mt = (Mr + kUmmaBM - 1) / kUmmaBM, nt = (N + kUmmaBN - 1) / kUmmaBN;
+    const int64_t want = (148 + mt - 1) / mt;             // CTAs per row block to fill the GPU
+    const int64_t sp = want < nt ? want : nt;
+    const int per = (int)((nt + sp - 1) / sp);
+    dim3 grid((unsigned)((nt + per - 1) / per), (unsigned)mt);
+    const size_t smem = rows_smem_bytes(Kd, split);
+    if (split) {
+      cudaFuncSetAttribute(k_gemm_rows<P, true, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      k_gemm_rows<P, true, E><<<grid, kRowsThreads, smem, st>>>(prod, ws + wpk, Mr, N, Kd, per, epi, status);
+    } else {
+      cudaFuncSetAttribute(k_gemm_rows<P, false, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      k_gemm_rows<P, false, E><<<grid, kRowsThreads, smem, st>>>(prod, ws + wpk, Mr, N, Kd, per, epi, status);
+    }
+    ++hk.launches;
+  };
+  // out = epi(A @ W): the row-block kernel for K <= 256, else the streaming kernel
   auto gemm = [&](auto *A_, int64_t lda, size_t wpk, int64_t Mr, int64_t N, int64_t Kd, auto epi) {
     using TA = std::remove_cv_t<std::remove_pointer_t<decltype(A_)>>;
     using E = decltype(epi);
-    const int64_t mt = (Mr + kUmmaBM - 1) / kUmmaBM, nt = (N + kUmmaBN - 1) / kUmmaBN;
     if (Kd <= kRowsKMax) {
-      const int64_t want = (148 + mt - 1) / mt;           // CTAs per row block to fill the GPU
-      const int per = (int)((nt + (want < nt ? want : nt) - 1) / (want < nt ? want : nt));
-      dim3 grid((unsigned)((nt + per - 1) / per), (unsigned)mt);
-      const size_t smem = rows_smem_bytes(Kd, split);
-      if (split) {
-        cudaFuncSetAttribute(k_gemm_rows<TA, true, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_gemm_rows<TA, true, E><<<grid, kRowsThreads, smem, st>>>(A_, lda, ws + wpk, Mr, N, Kd, per, epi, status);
-      } else {
-        cudaFuncSetAttribute(k_gemm_rows<TA, false, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_gemm_rows<TA, false, E><<<grid, kRowsThreads, smem, st>>>(A_, lda, ws + wpk, Mr, N, Kd, per, epi, status);
-      }
+      gemm_rows(ProdPlain<TA>{A_, lda, Mr, Kd}, wpk, Mr, N, Kd, epi);
+      return;
+    }
+    dim3 grid((unsigned)((N + kUmmaBN - 1) / kUmmaBN), (unsigned)((Mr + kUmmaBM - 1) / kUmmaBM));
+    const size_t smem = umma_smem_bytes(split);
+    if (split) {
+      cudaFuncSetAttribute(k_gemm_umma<TA, true, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      k_gemm_umma<TA, true, E><<<grid, kUmmaThreads, smem, st>>>(A_, lda, ws + wpk, Mr, N, Kd, epi, status);
     } else {
-      dim3 grid((unsigned)nt, (unsigned)mt);
-      const size_t smem = umma_smem_bytes(split);
-      if (split) {
-        cudaFuncSetAttribute(k_gemm_umma<TA, true, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_gemm_umma<TA, true, E><<<grid, kUmmaThreads, smem, st>>>(A_, lda, ws + wpk, Mr, N, Kd, epi, status);
-      } else {
-        cudaFuncSetAttribute(k_gemm_umma<TA, false, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_gemm_umma<TA, false, E><<<grid, kUmmaThreads, smem, st>>>(A_, lda, ws + wpk, Mr, N, Kd, epi, status);
-      }
+      cudaFuncSetAttribute(k_gemm_umma<TA, false, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      k_gemm_umma<TA, false, E><<<grid, kUmmaThreads, smem, st>>>(A_, lda, ws + wpk, Mr, N, Kd, epi, status);
     }
     ++hk.launches;
+  };
+  // the conditioning-modulated row norm of x (or x') fused into a projection's operand
+  const bool fuse_norm = C <= kRowsKMax;
+  auto norm_prod = [&](int64_t sc_off, int64_t sh_off, bool plus1) {
+    return ProdNorm{F(pl.o_x), F(pl.o_xstats), F(pl.o_cond), R, C, 6 * C, sc_off, sh_off,
+                    plus1 ? 1 : 0};
   };
   const int rows_per_block = 8;  // warps per 256-thread block for warp-per-row kernels
   const unsigned row_blocks = (unsigned)((R + rows_per_block - 1) / rows_per_block);
@@ -426,7 +442,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   ra.token_valid = static_cast<const uint8_t *>(in->token_valid.data);
   ra.att = static_cast<const int64_t *>(in->atom_to_token.data);
   ra.token_proj = F(pl.o_tp);
-  ra.usable = usable; ra.x = F(pl.o_x); ra.opc = F(pl.o_opc); ra.rawc = F(pl.o_rawc);
+  ra.usable = usable; ra.x = F(pl.o_x); ra.xstats = F(pl.o_xstats); ra.opc = F(pl.o_opc); ra.rawc = F(pl.o_rawc);
   ra.tok_first = first; ra.tok_last = last;
   k_rows_prep<Elt><<<row_blocks, 256, 0, st>>>(ra);
   ++hk.launches;
@@ -442,23 +458,37 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     gemm(F(pl.o_opc), S, pl.k_cond, R, 6 * C, S, Quad<EpiStore>{{F(pl.o_cond), 6 * C}});
   }
   hk.mark(2, st);
-  FeatArgs fa{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_x), F(pl.o_cond), F(pl.o_feat)};
-  k_features<<<row_blocks, 256, 0, st>>>(fa);
-  ++hk.launches;
+  if (!fuse_norm) {
+    FeatArgs fa{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_x), F(pl.o_cond), F(pl.o_feat)};
+    k_features<<<row_blocks, 256, 0, st>>>(fa);
+    ++hk.launches;
+  }
 
-  // ---- projections
+  // ---- projections (attention inputs fused into the operand when C <= 256)
   if (pl.af3) {
     EpiSplit e0{{F(pl.o_q), F(pl.o_g), nullptr, nullptr}, {F(pl.o_bq), nullptr, nullptr, nullptr}, HD};
-    gemm(F(pl.o_feat), 2 * C, pl.k_qkv0, R, 2 * HD, C, e0);
     EpiSplit e1{{F(pl.o_k), F(pl.o_v), nullptr, nullptr}, {nullptr, nullptr, nullptr, nullptr}, HD};
-    gemm(F(pl.o_feat) + C, 2 * C, pl.k_qkv1, R, 2 * HD, C,
-         e1);
+    if (fuse_norm) {
+      gemm_rows(norm_prod(0, C, false), pl.k_qkv0, R, 2 * HD, C, e0);
+      gemm_rows(norm_prod(2 * C, 3 * C, false), pl.k_qkv1, R, 2 * HD, C, e1);
+    } else {
+      gemm(F(pl.o_feat), 2 * C, pl.k_qkv0, R, 2 * HD, C, e0);
+      gemm(F(pl.o_feat) + C, 2 * C, pl.k_qkv1, R, 2 * HD, C, e1);
+    }
   } else {
     EpiSplit e{{F(pl.o_q), F(pl.o_k), F(pl.o_v), F(pl.o_g)}, {nullptr, nullptr, nullptr, nullptr}, HD};
-    gemm(F(pl.o_feat), C, pl.k_qkv0, R, 4 * HD, C, e);
+    if (fuse_norm)
+      gemm_rows(norm_prod(C, 0, true), pl.k_qkv0, R, 4 * HD, C, e);
+    else
+      gemm(F(pl.o_feat), C, pl.k_qkv0, R, 4 * HD, C, e);
     RopeArgs rp{R, H, D, eps, usable, in->rope_cos.data, in->rope_sin.data, F(pl.o_q), F(pl.o_k)};
-    const int64_t n = R * H * 2;
-    k_qk_rope<Elt><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(rp);
+    if (D >= 8 && D <= 128 && (D & (D - 1)) == 0) {
+      const int64_t warps = R * 2;
+      k_qk_rope_warp<Elt><<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(rp);
+    } else {
+      const int64_t n = R * H * 2;
+      k_qk_rope<Elt><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(rp);
+    }
     ++hk.launches;
   }
   hk.mark(3, st);

@@ -65,13 +65,22 @@ __host__ __device__ inline size_t attn_fixed_smem(int QT, int K, int H, int HD, 
   return 4 * (ru4(slots) + (af3 ? ru4((size_t)H * slots) : 0) + ru4((size_t)QT * HD));
 }
 
-// d0,d1 += a * b elementwise on a pair of floats (one packed f32x2 FMA on sm_100)
-__device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%0, %1};\n\t"
-      "fma.rn.f32x2 rc, ra, rb, rc;\n\tmov.b64 {%0, %1}, rc;\n\t}"
-      : "+f"(d0), "+f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+// Two floats packed in one 64-bit register, and the sm_100 packed FMA on them.
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 ffma2(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f32x2 pack2(float x, float y) {
+  f32x2 d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(x), "f"(y));
+  return d;
+}
+__device__ __forceinline__ float2 unpack2(f32x2 v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
 }
 
 // 2^x on the special-function unit (the exponent of the softmax is always <= 0 here)
@@ -207,27 +216,30 @@ __device__ __forceinline__ void pair_bias_generic(const T *pr, int P, int H, flo
   }
 }
 
+// q . r with the query already packed in registers (zero beyond D) and the key row in
+// shared memory (16-byte aligned, zero-padded to DMAX)
 template <int DMAX>
-__device__ __forceinline__ float dot_row(const float *q, const float *r) {
-  // q, r: 16-byte aligned, zero-padded to DMAX in shared memory
-  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+__device__ __forceinline__ float dot_q2(const f32x2 (&q2)[DMAX / 2], const float *r) {
+  f32x2 s0 = 0ull, s1 = 0ull;
 #pragma unroll
   for (int d = 0; d < DMAX; d += 4) {
-    const float4 a = *reinterpret_cast<const float4 *>(q + d);
-    const float4 k = *reinterpret_cast<const float4 *>(r + d);
-    fma2(s0, s1, a.x, a.y, k.x, k.y);
-    fma2(s2, s3, a.z, a.w, k.z, k.w);
+    const ulonglong2 k = *reinterpret_cast<const ulonglong2 *>(r + d);
+    s0 = ffma2(q2[d / 2], k.x, s0);
+    s1 = ffma2(q2[d / 2 + 1], k.y, s1);
   }
-  return (s0 + s1) + (s2 + s3);
+  const float2 x = unpack2(s0), y = unpack2(s1);
+  return (x.x + x.y) + (y.x + y.y);
 }
-
+// the same with the key row read from global memory (D floats, any alignment)
 template <int DMAX>
-__device__ __forceinline__ float dot_plain(const float (&q)[DMAX], const float *r, int D) {
-  float s = 0.f;
+__device__ __forceinline__ float dot_q2_global(const f32x2 (&q2)[DMAX / 2], const float *r, int D) {
+  f32x2 s = 0ull;
 #pragma unroll
-  for (int d = 0; d < DMAX; ++d)
-    if (d < D) s = fmaf(q[d], r[d], s);
-  return s;
+  for (int d = 0; d < DMAX; d += 2) {
+    if (d < D) s = ffma2(q2[d / 2], pack2(r[d], d + 1 < D ? r[d + 1] : 0.f), s);
+  }
+  const float2 x = unpack2(s);
+  return x.x + x.y;
 }
 
 // MULTI = false: K <= 128, one chunk, logits and exponentials kept in registers.
@@ -412,32 +424,40 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_slot_attention(AttnArgs g) 
         const float *kbase = staged ? ks + (hl * span - klo) * DP : nullptr;
         const float *vbase = staged ? vs + (hl * span - klo) * DP : nullptr;
         const float *bh = AF3 ? beta + h * slots + q * K : nullptr;
-        float qreg[DMAX];
-        if (!fullD || !staged) {
+        // the query, packed once per (query, head), zero beyond D
+        f32x2 q2[DMAX / 2];
+        if (fullD) {
 #pragma unroll
-          for (int d = 0; d < DMAX; ++d) qreg[d] = d < D ? qv[d] : 0.f;
+          for (int d = 0; d < DMAX; d += 4) {
+            const ulonglong2 x = *reinterpret_cast<const ulonglong2 *>(qv + d);
+            q2[d / 2] = x.x;
+            q2[d / 2 + 1] = x.y;
+          }
+        } else {
+#pragma unroll
+          for (int d = 0; d < DMAX; d += 2)
+            q2[d / 2] = pack2(d < D ? qv[d] : 0.f, d + 1 < D ? qv[d + 1] : 0.f);
         }
 
-        // logit of slot k (key j) in log2 units
+        // logit of slot k (key j, clamped to a readable row when the slot is not
+        // permitted; the caller masks that value) in log2 units
         auto logit = [&](int k, int j) -> float {
-          float dot;
-          if (staged && fullD)
-            dot = dot_row<DMAX>(qv, kbase + j * DP);
-          else if (staged)
-            dot = dot_plain<DMAX>(qreg, kbase + j * DP, D);
-          else
-            dot = dot_plain<DMAX>(qreg, g.Kf + ((int64_t)b * A + j) * HD + h * D, D);
+          const float dot = staged ? dot_q2<DMAX>(q2, kbase + j * DP)
+                                   : dot_q2_global<DMAX>(q2, g.Kf + ((int64_t)b * A + j) * HD + h * D, D);
           float l = dot * g.scale_log2;
           if (AF3) l = fmaf(bh[k], 1.4426950408889634f, l);
           return l;
         };
+        const int jsafe = staged ? klo : 0;
 
         float mx = -INFINITY, sum = 0.f;
         float ev[kSlotsPerLane];
         if (!MULTI) {
 #pragma unroll
           for (int i = 0; i < kSlotsPerLane; ++i) {
-            ev[i] = jr[i] >= 0 ? logit(i * kWarp + lane, jr[i]) : -INFINITY;
+            const int k = i * kWarp + lane;
+            const float l = logit(k < K ? k : 0, jr[i] >= 0 ? jr[i] : jsafe);
+            ev[i] = jr[i] >= 0 ? l : -INFINITY;
             mx = fmaxf(mx, ev[i]);
           }
           mx = warp_max(mx);
@@ -469,11 +489,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_slot_attention(AttnArgs g) 
             }
           }
         }
-        const float inv = sum > 0.f ? 1.f / sum : 0.f;
+        float inv = 0.f;
+        if (sum > 0.f) asm("rcp.approx.f32 %0, %1;" : "=f"(inv) : "f"(sum));
 
-        float acc[DMAX];
+        f32x2 acc2[DMAX / 2];
 #pragma unroll
-        for (int d = 0; d < DMAX; ++d) acc[d] = 0.f;
+        for (int d = 0; d < DMAX / 2; ++d) acc2[d] = 0ull;
         T *arow_out = (T *)g.attention + (((int64_t)b * H + h) * A + a) * K;
         for (int c = 0; c < nchunks; ++c) {
 #pragma unroll
@@ -483,24 +504,27 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_slot_attention(AttnArgs g) 
               jr[i] = k < K ? plan[q * K + k] : -1;
               ev[i] = jr[i] >= 0 ? exp2_approx(logit(k, jr[i]) - mx) : 0.f;
             }
-            const int j = jr[i];
+            const int j = jr[i] >= 0 ? jr[i] : jsafe;   // weight 0 on a readable row
             const float wgt = ev[i] * inv;
             if (k < K) store_weight<T>(arow_out, k, wgt);
-            if (j >= 0) {
-              if (staged && vecD) {
+            if (sum > 0.f) {
+              if (staged) {
                 const float *vr = vbase + j * DP;
+                const f32x2 w2 = pack2(wgt, wgt);
 #pragma unroll
                 for (int d = 0; d < DMAX; d += 4) {
-                  const float4 v = *reinterpret_cast<const float4 *>(vr + d);
-                  fma2(acc[d], acc[d + 1], wgt, wgt, v.x, v.y);
-                  fma2(acc[d + 2], acc[d + 3], wgt, wgt, v.z, v.w);
+                  const ulonglong2 v = *reinterpret_cast<const ulonglong2 *>(vr + d);
+                  acc2[d / 2] = ffma2(w2, v.x, acc2[d / 2]);
+                  acc2[d / 2 + 1] = ffma2(w2, v.y, acc2[d / 2 + 1]);
                 }
               } else {
                 const float *vr =
                     staged ? vbase + j * DP : g.Vf + ((int64_t)b * A + j) * HD + h * D;
 #pragma unroll
-                for (int d = 0; d < DMAX; ++d)
-                  if (d < D) acc[d] = fmaf(wgt, vr[d], acc[d]);
+                for (int d = 0; d < DMAX; d += 2) {
+                  const float v0 = d < D ? vr[d] : 0.f, v1 = d + 1 < D ? vr[d + 1] : 0.f;
+                  acc2[d / 2] = ffma2(pack2(wgt, wgt), pack2(v0, v1), acc2[d / 2]);
+                }
               }
             }
           }
@@ -508,6 +532,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_slot_attention(AttnArgs g) 
 
         // fold the lanes' partial outputs: lane l ends with channel l (and l + 32)
         const bool has = sum > 0.f;
+        float acc[DMAX];
+#pragma unroll
+        for (int d = 0; d < DMAX; d += 2) {
+          const float2 p = unpack2(acc2[d / 2]);
+          acc[d] = p.x;
+          acc[d + 1] = p.y;
+        }
 #pragma unroll
         for (int part = 0; part < DMAX; part += DW) {
           float v[DW];

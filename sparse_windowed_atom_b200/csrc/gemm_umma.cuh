@@ -72,11 +72,11 @@ __global__ void k_pack_weights(PackJobs jobs) {
 }
 
 template <typename TA>
-__device__ __forceinline__ void load8(const TA *A, int64_t lda, int64_t M, int64_t K, int64_t r,
-                                      int64_t k, float (&v)[8]);
+__device__ __forceinline__ void load8_t(const TA *A, int64_t lda, int64_t M, int64_t K, int64_t r,
+                                        int64_t k, float (&v)[8]);
 
 template <>
-__device__ __forceinline__ void load8<float>(const float *A, int64_t lda, int64_t M, int64_t K,
+__device__ __forceinline__ void load8_t<float>(const float *A, int64_t lda, int64_t M, int64_t K,
                                              int64_t r, int64_t k, float (&v)[8]) {
   if (r < M && k + 8 <= K && ((lda | k) & 3) == 0) {
     const float4 x = *reinterpret_cast<const float4 *>(A + r * lda + k);
@@ -90,7 +90,7 @@ __device__ __forceinline__ void load8<float>(const float *A, int64_t lda, int64_
 }
 
 template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *A, int64_t lda,
+__device__ __forceinline__ void load8_t<__nv_bfloat16>(const __nv_bfloat16 *A, int64_t lda,
                                                      int64_t M, int64_t K, int64_t r, int64_t k,
                                                      float (&v)[8]) {
   if (r < M && k + 8 <= K && ((lda | k) & 7) == 0) {
@@ -106,6 +106,46 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *A, int
     for (int e = 0; e < 8; ++e) v[e] = (r < M && k + e < K) ? ldf(A, r * lda + k + e) : 0.f;
   }
 }
+
+// ---- A producers of the row-block GEMM: what the CTA converts into its A operand.
+// ProdPlain: A itself. ProdNorm: a row normalisation fused into the operand,
+//   (x - mean) * rstd * scale + shift      (AF3 adaptive LN; the scale column already
+//                                           holds sigmoid(...))
+//   x * rstd * (1 + scale) + shift         (ESMFold2 modulation; mean = 0 for RMS)
+// with the per-row mean/rstd computed where x is produced and scale/shift read from the
+// conditioning rows.
+template <typename TA>
+struct ProdPlain {
+  static constexpr bool kStats = false;
+  const TA *A;
+  int64_t lda, M, K;
+  __device__ void row_stats(int64_t, int, float *) const {}
+  __device__ void load8(int64_t r, int, int64_t k, const float *, float (&v)[8]) const {
+    load8_t(A, lda, M, K, r, k, v);
+  }
+};
+
+struct ProdNorm {
+  static constexpr bool kStats = false;
+  const float *x;        // [M, K]
+  const float *stats;    // [M, 2]: mean (0 for RMS) and rstd of each row of x
+  const float *cond;     // rows of cond_ld floats
+  int64_t M, K, cond_ld, sc_off, sh_off;
+  int plus1;
+  __device__ void row_stats(int64_t, int, float *) const {}
+  __device__ void load8(int64_t r, int, int64_t k, const float *, float (&v)[8]) const {
+    float xv[8], sc[8], sh[8];
+    load8_t(x, K, M, K, r, k, xv);
+    load8_t(cond + sc_off, cond_ld, M, K, r, k, sc);
+    load8_t(cond + sh_off, cond_ld, M, K, r, k, sh);
+    const float2 ms = r < M ? *reinterpret_cast<const float2 *>(stats + 2 * r) : make_float2(0.f, 0.f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float s = plus1 ? 1.f + sc[e] : sc[e];
+      v[e] = (r < M && k + e < K) ? fmaf((xv[e] - ms.x) * ms.y, s, sh[e]) : 0.f;
+    }
+  }
+};
 
 template <typename TA, bool SPLIT, class Epi>
 __global__ void __launch_bounds__(kUmmaThreads)
@@ -158,7 +198,7 @@ __global__ void __launch_bounds__(kUmmaThreads)
     for (int it = 0; it < 8; ++it) {
       const int r = warp * 32 + it * 4 + (lane >> 3), seg = lane & 7;
       float v[8];
-      load8<TA>(A, lda, M, K, m0 + r, (int64_t)c * kUmmaBK + seg * 8, v);
+      load8_t<TA>(A, lda, M, K, m0 + r, (int64_t)c * kUmmaBK + seg * 8, v);
       uint32_t hi[4], lo[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -239,13 +279,14 @@ __host__ __device__ constexpr int rows_slots(bool split) { return split ? 2 : 3;
 __host__ __device__ inline size_t rows_smem_bytes(int64_t K, bool split) {
   const int parts = split ? 2 : 1;
   const size_t nkc = (size_t)((K + kUmmaBK - 1) / kUmmaBK);
-  return 1024 + (nkc + rows_slots(split)) * parts * kUmmaBlockBytes + 4 * 32 * 33 * 4 + 256;
+  return 1024 + (nkc + rows_slots(split)) * parts * kUmmaBlockBytes + 4 * 32 * 33 * 4 + 256 +
+         128 * 2 * 4;
 }
 
-template <typename TA, bool SPLIT, class Epi>
+template <class Prod, bool SPLIT, class Epi>
 __global__ void __launch_bounds__(kRowsThreads, 1)
-    k_gemm_rows(const TA *__restrict__ A, int64_t lda, const uint8_t *__restrict__ Wpk, int64_t M,
-                int64_t N, int64_t K, int tiles_per_cta, Epi epi, unsigned *status) {
+    k_gemm_rows(Prod prod, const uint8_t *__restrict__ Wpk, int64_t M, int64_t N, int64_t K,
+                int tiles_per_cta, Epi epi, unsigned *status) {
   extern __shared__ __align__(1024) uint8_t smem_dyn[];
   constexpr int PARTS = SPLIT ? 2 : 1, NSLOT = rows_slots(SPLIT);
   constexpr uint32_t BLK = kUmmaBlockBytes;
@@ -260,6 +301,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
   uint64_t *empty = full + NSLOT, *accf = empty + NSLOT, *acce = accf + 2, *aready = acce + 2;
   uint32_t *tslot = reinterpret_cast<uint32_t *>(aready + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
+  float *sStats = reinterpret_cast<float *>(tslot + 4);                   // [128][2]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nt = (int)((N + kUmmaBN - 1) / kUmmaBN);
@@ -291,13 +333,18 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
   if (warp < 4) {
     // ---- A: rows 32w..32w+31 of the tile, every k chunk, bf16 (hi[, lo]) swizzled;
     // the 8 row-segments of a chunk are loaded before any is converted (8 loads in flight)
+    if (Prod::kStats) {
+      prod.row_stats(m0 + warp * 32, lane, sStats + warp * 64);
+      __syncwarp();
+    }
     for (int c = 0; c < nkc; ++c) {
       uint8_t *a_c = sA + (size_t)c * PARTS * BLK;
       float v[8][8];
 #pragma unroll
-      for (int it = 0; it < 8; ++it)
-        load8<TA>(A, lda, M, K, m0 + warp * 32 + it * 4 + (lane >> 3),
-                  (int64_t)c * kUmmaBK + (lane & 7) * 8, v[it]);
+      for (int it = 0; it < 8; ++it) {
+        const int rl = warp * 32 + it * 4 + (lane >> 3);
+        prod.load8(m0 + rl, rl, (int64_t)c * kUmmaBK + (lane & 7) * 8, sStats, v[it]);
+      }
 #pragma unroll
       for (int it = 0; it < 8; ++it) {
         const int r = warp * 32 + it * 4 + (lane >> 3), seg = lane & 7;

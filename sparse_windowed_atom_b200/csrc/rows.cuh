@@ -50,6 +50,7 @@ struct RowsArgs {
   const float *token_proj;  // [B*T, C] decoder: token @ w_token
   uint8_t *usable;          // [B*A]
   float *x;                 // [B*A, C] residual state start
+  float *xstats;            // [B*A, 2] AF3: mean, 1/sqrt(var+eps); ESM: 0, 1/sqrt(mean sq+eps)
   float *opc;               // [B*A, S] AF3: LN(c); ESMFold2: SiLU(c)
   float *rawc;              // [B*A, S] AF3: sanitised raw condition
   int *tok_first, *tok_last;  // [B*T] encoder pooling ranges
@@ -74,6 +75,7 @@ __global__ void k_rows_prep(RowsArgs r) {
     }
   }
   const T *atom = (const T *)r.atom + row * r.C;
+  float s1 = 0.f;
   for (int64_t c = lane; c < r.C; c += kWarp) {
     float v = 0.f;
     if (use) {
@@ -81,6 +83,21 @@ __global__ void k_rows_prep(RowsArgs r) {
       if (r.decoder) v += r.token_proj[(b * r.T + t) * r.C + c];
     }
     r.x[row * r.C + c] = v;
+    s1 += v;
+  }
+  // row statistics of x for the attention inputs: AF3 population LayerNorm (bullet 7),
+  // ESMFold2 RMS (bullet 11); the second pass re-reads the row just written
+  __syncwarp();
+  const float mean = r.af3 ? warp_sum(s1) / (float)r.C : 0.f;
+  float s2 = 0.f;
+  for (int64_t c = lane; c < r.C; c += kWarp) {
+    const float d = r.x[row * r.C + c] - mean;
+    s2 = fmaf(d, d, s2);
+  }
+  s2 = warp_sum(s2);
+  if (lane == 0) {
+    r.xstats[2 * row] = mean;
+    r.xstats[2 * row + 1] = 1.f / sqrtf(s2 / (float)r.C + r.eps);
   }
   const T *cond = (const T *)r.condition + row * r.S;
   if (r.af3) {
@@ -183,6 +200,50 @@ __global__ void k_qk_rope(RopeArgs r) {
     float rot = d < half ? -buf[d + half] * rstd : buf[d - half] * rstd;
     float c = use ? ldf(cs, d) : 0.f, s = use ? ldf(sn, d) : 0.f;
     v[d] = use ? qd * c + rot * s : 0.f;
+  }
+}
+
+// Warp per (atom, Q-or-K) for head widths D in {8, 16, 32, 64, 128}: lane l holds four
+// consecutive channels of each 128-channel chunk, the D/4 lanes of one head reduce the
+// sum of squares with xor-shuffles, and the half-split partner of channel d (d +- D/2)
+// sits D/8 lanes away in the same head group.
+template <typename T>
+__global__ void k_qk_rope_warp(RopeArgs r) {
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (wid >= r.rows * 2) return;
+  const int64_t row = wid >> 1;
+  const int D = (int)r.D, HD = (int)(r.H * r.D), glanes = D / 4, half = D / 2;
+  float *v = ((wid & 1) ? r.K : r.Q) + row * HD;
+  const bool use = r.usable[row] != 0;
+  const T *cs = (const T *)r.cos + row * D;
+  const T *sn = (const T *)r.sin + row * D;
+  for (int c0 = 0; c0 < HD; c0 += 128) {
+    const int c = c0 + lane * 4;
+    const bool in = c < HD;
+    float4 x = in ? *reinterpret_cast<const float4 *>(v + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float ss = x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+    for (int o = 1; o < glanes; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rstd = 1.f / sqrtf(ss / (float)D + r.eps);
+    x.x *= rstd; x.y *= rstd; x.z *= rstd; x.w *= rstd;
+    const int po = D / 8;  // lanes between channel d and d +- D/2
+    float4 p;
+    p.x = __shfl_xor_sync(0xffffffffu, x.x, po);
+    p.y = __shfl_xor_sync(0xffffffffu, x.y, po);
+    p.z = __shfl_xor_sync(0xffffffffu, x.z, po);
+    p.w = __shfl_xor_sync(0xffffffffu, x.w, po);
+    const int d = c % D;
+    const float sg = d < half ? -1.f : 1.f;   // rotate_half: [-q2, q1]
+    if (in) {
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (use) {
+        o.x = x.x * ldf(cs, d) + sg * p.x * ldf(sn, d);
+        o.y = x.y * ldf(cs, d + 1) + sg * p.y * ldf(sn, d + 1);
+        o.z = x.z * ldf(cs, d + 2) + sg * p.z * ldf(sn, d + 2);
+        o.w = x.w * ldf(cs, d + 3) + sg * p.w * ldf(sn, d + 3);
+      }
+      *reinterpret_cast<float4 *>(v + c) = o;
+    }
   }
 }
 
