@@ -83,6 +83,18 @@ __device__ __forceinline__ float2 unpack2(f32x2 v) {
   return r;
 }
 
+// 16-byte / 4-byte shared-memory loads by 32-bit shared address
+__device__ __forceinline__ ulonglong2 lds128(uint32_t addr) {
+  ulonglong2 v;
+  asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float lds32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
 // 2^x on the special-function unit (the exponent of the softmax is always <= 0 here)
 __device__ __forceinline__ float exp2_approx(float x) {
   float y;
@@ -377,12 +389,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_slot_attention(AttnArgs g) 
     const int hg = H - h0 < HG ? H - h0 : HG;
     float *ks = kv, *vs = kv + hg * span * DP;
     if (staged) {
-      const int CH = DP / 4, rpp = kWarp / CH, rsub = lane / CH, c4 = (lane - rsub * CH) * 4;
+      // one 16-byte chunk of one staged row per lane; only the DMAX columns that are read
+      // (zero-filled beyond D when D < DMAX), so every lane of a pass does the same work
+      constexpr int CH = DMAX / 4, rpp = kWarp / CH;
+      const int rsub = lane / CH, c4 = (lane - rsub * CH) * 4;
       for (int hl = 0; hl < hg; ++hl) {
         const int col = (h0 + hl) * D + c4;
         for (int r0 = warp * rpp; r0 < span; r0 += kAttnWarps * rpp) {
           const int rr = r0 + rsub;
-          if (rsub >= rpp || rr >= span) continue;
+          if (rr >= span) continue;
           const int64_t src = ((int64_t)b * A + klo + rr) * HD + col;
           float *kd = ks + (hl * span + rr) * DP + c4, *vd = vs + (hl * span + rr) * DP + c4;
           if (vecD && c4 < D) {
@@ -417,6 +432,98 @@ __global__ void __launch_bounds__(kAttnThreads, 2) k_slot_attention(AttnArgs g) 
           const int k = i * kWarp + lane;
           jr[i] = k < K ? plan[q * K + k] : -1;
         }
+      }
+      if (!MULTI && staged && K == kChunk) {
+        // ---- fast path: 128 slots, staged K/V, 32-bit shared addresses, no slot guards
+        const uint32_t rowb = (uint32_t)DP * 4u;
+        for (int hl = 0; hl < hg; ++hl) {
+          const int h = h0 + hl;
+          const uint32_t kb = (uint32_t)__cvta_generic_to_shared(ks) + (uint32_t)(hl * span - klo) * rowb;
+          const uint32_t vb = (uint32_t)__cvta_generic_to_shared(vs) + (uint32_t)(hl * span - klo) * rowb;
+          const uint32_t qa = (uint32_t)__cvta_generic_to_shared(qs) + (uint32_t)(q * HD + h * D) * 4u;
+          f32x2 q2[DMAX / 2];
+          if (fullD) {
+#pragma unroll
+            for (int d = 0; d < DMAX; d += 4) {
+              const ulonglong2 x = lds128(qa + 4u * d);
+              q2[d / 2] = x.x;
+              q2[d / 2 + 1] = x.y;
+            }
+          } else {
+#pragma unroll
+            for (int d = 0; d < DMAX; d += 2)
+              q2[d / 2] = pack2(d < D ? lds32(qa + 4u * d) : 0.f, d + 1 < D ? lds32(qa + 4u * d + 4u) : 0.f);
+          }
+          const uint32_t ba = AF3 ? (uint32_t)__cvta_generic_to_shared(beta) +
+                                        (uint32_t)(h * slots + q * K + lane) * 4u
+                                  : 0u;
+          float ev[kSlotsPerLane];
+          uint32_t ja[kSlotsPerLane];
+          float mx = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < kSlotsPerLane; ++i) {
+            ja[i] = (uint32_t)(jr[i] >= 0 ? jr[i] : klo) * rowb;
+            f32x2 s0 = 0ull, s1 = 0ull;
+#pragma unroll
+            for (int d = 0; d < DMAX; d += 4) {
+              const ulonglong2 k = lds128(kb + ja[i] + 4u * d);
+              s0 = ffma2(q2[d / 2], k.x, s0);
+              s1 = ffma2(q2[d / 2 + 1], k.y, s1);
+            }
+            const float2 x = unpack2(s0), y = unpack2(s1);
+            float l = ((x.x + x.y) + (y.x + y.y)) * g.scale_log2;
+            if (AF3) l = fmaf(lds32(ba + 128u * i), 1.4426950408889634f, l);
+            ev[i] = jr[i] >= 0 ? l : -INFINITY;
+            mx = fmaxf(mx, ev[i]);
+          }
+          mx = warp_max(mx);
+          float sum = 0.f;
+#pragma unroll
+          for (int i = 0; i < kSlotsPerLane; ++i) {
+            ev[i] = jr[i] >= 0 ? exp2_approx(ev[i] - mx) : 0.f;
+            sum += ev[i];
+          }
+          sum = warp_sum(sum);
+          float inv = 0.f;
+          if (sum > 0.f) asm("rcp.approx.f32 %0, %1;" : "=f"(inv) : "f"(sum));
+          T *wout = (T *)g.attention + (((int64_t)b * H + h) * A + a) * K + lane;
+          f32x2 acc2[DMAX / 2];
+#pragma unroll
+          for (int d = 0; d < DMAX / 2; ++d) acc2[d] = 0ull;
+#pragma unroll
+          for (int i = 0; i < kSlotsPerLane; ++i) {
+            const float wgt = ev[i] * inv;
+            store_weight<T>(wout, i * kWarp, wgt);
+            const f32x2 w2 = pack2(wgt, wgt);
+#pragma unroll
+            for (int d = 0; d < DMAX; d += 4) {
+              const ulonglong2 v = lds128(vb + ja[i] + 4u * d);
+              acc2[d / 2] = ffma2(w2, v.x, acc2[d / 2]);
+              acc2[d / 2 + 1] = ffma2(w2, v.y, acc2[d / 2 + 1]);
+            }
+          }
+          const bool has = sum > 0.f;
+          float acc[DMAX];
+#pragma unroll
+          for (int d = 0; d < DMAX; d += 2) {
+            const float2 p2 = unpack2(acc2[d / 2]);
+            acc[d] = p2.x;
+            acc[d + 1] = p2.y;
+          }
+#pragma unroll
+          for (int part = 0; part < DMAX; part += DW) {
+            float v[DW];
+#pragma unroll
+            for (int i = 0; i < DW; ++i) v[i] = acc[part + i];
+            const float o = reduce_scatter<DW>(v, lane);
+            const int d = part + (lane & (DW - 1));
+            if (lane < DW && d < D) {
+              const int64_t oi = arow * HD + h * D + d;
+              g.O[oi] = has ? o * sigmoid_fast(g.G[oi]) : 0.f;
+            }
+          }
+        }
+        continue;
       }
       for (int hl = 0; hl < hg; ++hl) {
         const int h = h0 + hl;
