@@ -19,6 +19,7 @@
 #include "epilogues.cuh"
 #include "gemm_umma.cuh"
 #include "rows.cuh"
+#include "transition.cuh"
 
 using namespace atomenc;
 
@@ -64,7 +65,7 @@ float bf16_round_host(float f) {
 
 struct Plan {
   int style = 0, stage = 0, fdt = 0;
-  bool af3 = false, enc = false;
+  bool af3 = false, enc = false, fuse_tail = false;
   Dims d;
   // workspace layout (byte offsets)
   size_t o_status, o_usable, o_xstats, o_first, o_last, o_tp, o_x, o_opc, o_rawc, o_cond, o_gate, o_feat,
@@ -220,9 +221,12 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   pl.o_v = take(cur, R * HD * 4);
   pl.o_g = take(cur, R * HD * 4);
   pl.o_o = take(cur, R * HD * 4);
-  pl.o_xp = take(cur, R * C * 4);
-  pl.o_z = take(cur, R * C * 4);
-  pl.o_h = take(cur, R * M * 4);
+  // the fused tail (out-projection .. hidden in one kernel) keeps x', z and the SwiGLU
+  // intermediate on chip
+  pl.fuse_tail = C == 128 && (HD == 64 || HD == 128) && M % 128 == 0;
+  pl.o_xp = take(cur, pl.fuse_tail ? 0 : R * C * 4);
+  pl.o_z = take(cur, pl.fuse_tail ? 0 : R * C * 4);
+  pl.o_h = take(cur, pl.fuse_tail ? 0 : R * M * 4);
   pl.o_hid = take(cur, R * C * 4);
   pl.o_pool = take(cur, pl.enc ? R * U * 4 : 0);
   pl.o_wcond = take(cur, S * 6 * C * 4);
@@ -534,21 +538,41 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
 
   hk.mark(4, st);
 
-  // ---- out-projection + gated residual: x' = x + g_attn * (o @ w_attention_out)
+  // ---- out-projection + gated residual, transition norm, SwiGLU, gated residual + mask
   const float *gbuf = pl.af3 ? F(pl.o_gate) : F(pl.o_cond);
   const int64_t gld = pl.af3 ? 2 * C : 6 * C;
   const int64_t g0off = pl.af3 ? 0 : 2 * C, g1off = pl.af3 ? C : 5 * C;
-  gemm(F(pl.o_o), HD, pl.k_out, R, C, HD,
-       Quad<EpiResidual>{{F(pl.o_x), gbuf, gld, g0off, C, F(pl.o_xp)}});
-
-  // ---- transition on the new state
-  TNormArgs ta{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_xp), F(pl.o_cond), F(pl.o_z)};
-  k_transition_norm<<<row_blocks, 256, 0, st>>>(ta);
-  ++hk.launches;
-  gemm(F(pl.o_z), C, pl.k_ff1, R, 2 * M, C, EpiSwiGLU{F(pl.o_h), M});
-  gemm(F(pl.o_h), M, pl.k_ff2, R, C, M,
-       Quad<EpiHidden<Elt>>{{F(pl.o_xp), gbuf, gld, g1off, C, usable, F(pl.o_hid),
-                           static_cast<Elt *>(out->hidden.data)}});
+  if (pl.fuse_tail) {
+    TransArgs ta;
+    ta.R = R; ta.HD = (int)HD; ta.M = (int)M;
+    ta.O = F(pl.o_o); ta.x = F(pl.o_x);
+    ta.g0 = gbuf + g0off; ta.g1 = gbuf + g1off; ta.g_ld = gld;
+    ta.sc = F(pl.o_cond) + 4 * C; ta.sh = F(pl.o_cond) + (pl.af3 ? 5 : 3) * C; ta.cond_ld = 6 * C;
+    ta.rms = pl.af3 ? 0 : 1; ta.plus1 = pl.af3 ? 0 : 1; ta.eps = eps;
+    ta.usable = usable;
+    ta.w_out = ws + pl.k_out; ta.w_ff1 = ws + pl.k_ff1; ta.w_ff2 = ws + pl.k_ff2;
+    ta.hid32 = F(pl.o_hid); ta.hidden = out->hidden.data; ta.status = status;
+    const size_t smem = trans_smem_bytes(split);
+    const dim3 grid((unsigned)((R + kUmmaBM - 1) / kUmmaBM));
+    if (split) {
+      cudaFuncSetAttribute(k_transition<true, Elt>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      k_transition<true, Elt><<<grid, kTransThreads, smem, st>>>(ta);
+    } else {
+      cudaFuncSetAttribute(k_transition<false, Elt>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      k_transition<false, Elt><<<grid, kTransThreads, smem, st>>>(ta);
+    }
+    ++hk.launches;
+  } else {
+    gemm(F(pl.o_o), HD, pl.k_out, R, C, HD,
+         Quad<EpiResidual>{{F(pl.o_x), gbuf, gld, g0off, C, F(pl.o_xp)}});
+    TNormArgs tn{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_xp), F(pl.o_cond), F(pl.o_z)};
+    k_transition_norm<<<row_blocks, 256, 0, st>>>(tn);
+    ++hk.launches;
+    gemm(F(pl.o_z), C, pl.k_ff1, R, 2 * M, C, EpiSwiGLU{F(pl.o_h), M});
+    gemm(F(pl.o_h), M, pl.k_ff2, R, C, M,
+         Quad<EpiHidden<Elt>>{{F(pl.o_xp), gbuf, gld, g1off, C, usable, F(pl.o_hid),
+                               static_cast<Elt *>(out->hidden.data)}});
+  }
 
   hk.mark(5, st);
 

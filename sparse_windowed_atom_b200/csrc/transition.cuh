@@ -1,0 +1,330 @@
+// transition.cuh -- one kernel for the tail of the block, per 128-row block:
+//   x'     = x + g_attn * (o @ w_attention_out)                           (bullet 16)
+//   z      = AF3: LN(x') * sigmoid(scale_2) + shift_2;
+//            ESMFold2: RMS(x') * (1 + transition_scale) + transition_shift (bullet 17)
+//   hidden = usable * (x' + g_trans * ((SiLU(z @ w_ff_gate) * (z @ w_ff_up)) @ w_ff_out))
+//                                                                          (bullets 17, 18)
+// (page "Local atom attention, encoder pooling and decoder skip/readout", Required
+// behavior). The three products run on tcgen05 with their operands chained through
+// shared memory and three TMEM accumulators: out-projection (128 columns), one 128-wide
+// chunk of the SwiGLU hidden width at a time (256 interleaved gate/up columns) and
+// w_ff_out (128 columns), 512 TMEM columns in all; x', z and the SwiGLU intermediate
+// never go to HBM.
+//
+// Warp roles: warps 0-3 convert the o rows into the first operand, then work one output
+// row per thread (TMEM lanes 32w..32w+31): residual, row statistics and z (written as the
+// next operand), SiLU(gate) * up per chunk (written as the last operand), and the final
+// gated residual; warp 4 lane 0 issues the MMAs; warp 5 lane 0 streams the packed weight
+// blocks through a ring of bulk async copies in the order the MMAs consume them. Every
+// wait is bounded (status bit 4 on timeout). Needs C == 128, H*D in {64, 128}, M a
+// multiple of 128.
+#pragma once
+
+#include "common.cuh"
+#include "gemm_umma.cuh"
+#include "umma.cuh"
+
+namespace atomenc {
+
+constexpr int kTransThreads = 192;
+
+struct TransArgs {
+  int64_t R;
+  int HD, M;                   // C is 128
+  const float *O;              // [R, HD] gated attention output
+  const float *x;              // [R, 128] residual state start
+  const float *g0, *g1;        // attention / transition residual gates (row stride g_ld)
+  int64_t g_ld;
+  const float *sc, *sh;        // transition norm scale / shift (row stride cond_ld)
+  int64_t cond_ld;
+  int rms, plus1;
+  float eps;
+  const uint8_t *usable;
+  const uint8_t *w_out, *w_ff1, *w_ff2;   // packed tensor-core images
+  float *hid32;                // [R, 128] float32 hidden
+  void *hidden;                // [R, 128] output
+  unsigned *status;
+};
+
+__host__ __device__ inline size_t trans_smem_bytes(bool split) {
+  const size_t parts = split ? 2 : 1, slots = split ? 2 : 3;
+  return 1024 + (2 + 2 + slots) * parts * kUmmaBlockBytes + 256;
+}
+
+template <typename T>
+__device__ __forceinline__ void store4(T *p, int64_t i, float4 v);
+template <>
+__device__ __forceinline__ void store4<float>(float *p, int64_t i, float4 v) {
+  *reinterpret_cast<float4 *>(p + i) = v;
+}
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *p, int64_t i, float4 v) {
+  const uint32_t lo = (uint32_t)umma::bf16_bits(v.x) | ((uint32_t)umma::bf16_bits(v.y) << 16);
+  const uint32_t hi = (uint32_t)umma::bf16_bits(v.z) | ((uint32_t)umma::bf16_bits(v.w) << 16);
+  *reinterpret_cast<uint2 *>(p + i) = make_uint2(lo, hi);
+}
+
+// eight floats of one row into an operand block pair (hi, and lo when split) at column k
+template <bool SPLIT>
+__device__ __forceinline__ void put8(uint8_t *blk, int r, int k, const float (&v)[8]) {
+  uint32_t hi[4], lo[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const uint16_t h0 = umma::bf16_bits(v[2 * e]), h1 = umma::bf16_bits(v[2 * e + 1]);
+    hi[e] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+    if (SPLIT) {
+      const uint16_t l0 = umma::bf16_bits(v[2 * e] - umma::bf16_val(h0));
+      const uint16_t l1 = umma::bf16_bits(v[2 * e + 1] - umma::bf16_val(h1));
+      lo[e] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+    }
+  }
+  const uint32_t off = umma::swz_offset(r, k, kUmmaBM);
+  *reinterpret_cast<uint4 *>(blk + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  if (SPLIT)
+    *reinterpret_cast<uint4 *>(blk + kUmmaBlockBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+}
+
+// 32 consecutive floats of row r from global memory (zeros when r is out of range)
+__device__ __forceinline__ void row32(const float *p, int64_t ld, int64_t r, bool ok, int c0,
+                                      float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (ok) x = *reinterpret_cast<const float4 *>(p + r * ld + c0 + i);
+    v[i] = x.x;
+    v[i + 1] = x.y;
+    v[i + 2] = x.z;
+    v[i + 3] = x.w;
+  }
+}
+
+template <bool SPLIT, typename TOut>
+__global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
+  extern __shared__ __align__(1024) uint8_t smem_dyn[];
+  constexpr int P = SPLIT ? 2 : 1, NSLOT = SPLIT ? 2 : 3, C = 128;
+  constexpr uint32_t BLK = kUmmaBlockBytes;
+  constexpr uint32_t idesc = umma::idesc_bf16(kUmmaBM, kUmmaBN);
+  uint8_t *sm = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  uint8_t *sA = sm;                        // [2][P]: o operand, later z
+  uint8_t *sH = sA + 2 * P * BLK;          // [2][P]: SwiGLU chunk
+  uint8_t *sR = sH + 2 * P * BLK;          // weight ring [NSLOT][P]
+  uint64_t *full = reinterpret_cast<uint64_t *>(sR + NSLOT * P * BLK);
+  uint64_t *empty = full + NSLOT, *a_ready = empty + NSLOT, *acc0_done = a_ready + 1,
+           *z_ready = acc0_done + 1, *acc1_done = z_ready + 1, *h_ready = acc1_done + 1,
+           *h_free = h_ready + 1, *acc2_done = h_free + 1;
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(acc2_done + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t m0 = (int64_t)blockIdx.x * kUmmaBM;
+  const int nkc_out = t.HD / kUmmaBK, nM = t.M / 128;
+
+  if (tid == 0) {
+    for (int s = 0; s < NSLOT; ++s) {
+      umma::mbar_init(full + s, 1);
+      umma::mbar_init(empty + s, 1);
+    }
+    umma::mbar_init(a_ready, 128);
+    umma::mbar_init(acc0_done, 1);
+    umma::mbar_init(z_ready, 128);
+    umma::mbar_init(acc1_done, 1);
+    umma::mbar_init(h_ready, 128);
+    umma::mbar_init(h_free, 1);
+    umma::mbar_init(acc2_done, 1);
+    *abort_flag = 0;
+    umma::fence_mbar_init();
+  }
+  if (warp == 0) umma::tmem_alloc(tslot, 512);
+  umma::tc_fence_before();
+  __syncthreads();
+  umma::tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const uint32_t acc0 = tmem, acc1 = tmem + 128, acc2 = tmem + 384;
+  bool ok = true;
+
+  if (warp < 4) {
+    const int rl = warp * 32 + lane;
+    const int64_t r = m0 + rl;
+    const bool rok = r < t.R;
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+
+    // ---- o rows -> first operand (8 lanes per row segment, coalesced)
+    for (int kc = 0; kc < nkc_out; ++kc) {
+      float v[8][8];
+#pragma unroll
+      for (int it = 0; it < 8; ++it)
+        load8_t(t.O, t.HD, t.R, t.HD, m0 + warp * 32 + it * 4 + (lane >> 3),
+                (int64_t)kc * kUmmaBK + (lane & 7) * 8, v[it]);
+#pragma unroll
+      for (int it = 0; it < 8; ++it)
+        put8<SPLIT>(sA + kc * P * BLK, warp * 32 + it * 4 + (lane >> 3), (lane & 7) * 8, v[it]);
+    }
+    umma::fence_async_smem();
+    umma::mbar_arrive(a_ready);
+
+    // ---- x' = x + g0 * acc0; statistics of x' (one shifted pass), then z -> operand
+    if (ok) ok = umma::mbar_wait(acc0_done, 0, abort_flag);
+    umma::tc_fence_after();
+    float shift = 0.f, s1 = 0.f, s2 = 0.f;
+#pragma unroll 1
+    for (int c0 = 0; c0 < C; c0 += 32) {
+      float a[32], xv[32], gv[32];
+      umma::tmem_ld32(tl + c0, a);
+      row32(t.x, C, r, rok, c0, xv);
+      row32(t.g0, t.g_ld, r, rok, c0, gv);
+      if (c0 == 0) shift = t.rms ? 0.f : fmaf(gv[0], a[0], xv[0]);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float d = fmaf(gv[i], a[i], xv[i]) - shift;
+        s1 += d;
+        s2 = fmaf(d, d, s2);
+      }
+    }
+    const float m = s1 / (float)C;
+    const float mean = t.rms ? 0.f : shift + m;
+    const float var = t.rms ? s2 / (float)C : fmaxf(s2 / (float)C - m * m, 0.f);
+    const float rstd = 1.f / sqrtf(var + t.eps);
+#pragma unroll 1
+    for (int c0 = 0; c0 < C; c0 += 32) {
+      float a[32], xv[32], gv[32], sv[32], hv[32];
+      umma::tmem_ld32(tl + c0, a);
+      row32(t.x, C, r, rok, c0, xv);
+      row32(t.g0, t.g_ld, r, rok, c0, gv);
+      row32(t.sc, t.cond_ld, r, rok, c0, sv);
+      row32(t.sh, t.cond_ld, r, rok, c0, hv);
+#pragma unroll
+      for (int s8 = 0; s8 < 4; ++s8) {
+        float z[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int i = s8 * 8 + e;
+          const float xp = fmaf(gv[i], a[i], xv[i]);
+          const float sc = t.plus1 ? 1.f + sv[i] : sv[i];
+          z[e] = rok ? fmaf((xp - mean) * rstd, sc, hv[i]) : 0.f;
+        }
+        const int k = c0 + s8 * 8;
+        put8<SPLIT>(sA + (k / kUmmaBK) * P * BLK, rl, k % kUmmaBK, z);
+      }
+    }
+    umma::tc_fence_before();
+    umma::fence_async_smem();
+    umma::mbar_arrive(z_ready);
+
+    // ---- SwiGLU, one 128-wide chunk of the hidden width at a time -> last operand
+    for (int mc = 0; mc < nM; ++mc) {
+      if (ok) ok = umma::mbar_wait(acc1_done, mc & 1, abort_flag);
+      if (mc > 0 && ok) ok = umma::mbar_wait(h_free, (mc - 1) & 1, abort_flag);
+      umma::tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 0; c0 < 256; c0 += 32) {
+        float a[32];
+        umma::tmem_ld32(tl + 128 + c0, a);
+#pragma unroll
+        for (int s8 = 0; s8 < 2; ++s8) {
+          float h[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int i = s8 * 16 + 2 * e;
+            h[e] = silu_fast(a[i]) * a[i + 1];
+          }
+          const int k = c0 / 2 + s8 * 8;
+          put8<SPLIT>(sH + (k / kUmmaBK) * P * BLK, rl, k % kUmmaBK, h);
+        }
+      }
+      umma::tc_fence_before();
+      umma::fence_async_smem();
+      umma::mbar_arrive(h_ready);
+    }
+
+    // ---- hidden = usable * (x' + g1 * acc2)
+    if (ok) ok = umma::mbar_wait(acc2_done, 0, abort_flag);
+    umma::tc_fence_after();
+    const bool use = rok && t.usable[r] != 0;
+#pragma unroll 1
+    for (int c0 = 0; c0 < C; c0 += 32) {
+      float a[32], f[32], xv[32], gv[32], g1v[32];
+      umma::tmem_ld32(tl + c0, a);
+      umma::tmem_ld32(tl + 384 + c0, f);
+      row32(t.x, C, r, rok, c0, xv);
+      row32(t.g0, t.g_ld, r, rok, c0, gv);
+      row32(t.g1, t.g_ld, r, rok, c0, g1v);
+      if (rok && ok) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          float o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            o[e] = use ? fmaf(g1v[i + e], f[i + e], fmaf(gv[i + e], a[i + e], xv[i + e])) : 0.f;
+          const float4 o4 = make_float4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<float4 *>(t.hid32 + r * C + c0 + i) = o4;
+          store4<TOut>((TOut *)t.hidden, r * C + c0 + i, o4);
+        }
+      }
+    }
+  } else if (warp == 4) {
+    if (lane == 0) {
+      int i = 0;
+      auto mma_block = [&](uint32_t dtm, const uint8_t *a_blk, bool first) {
+        const int slot = i % NSLOT;
+        if (ok) ok = umma::mbar_wait(full + slot, (i / NSLOT) & 1, abort_flag);
+        umma::tc_fence_after();
+        const uint32_t a0 = umma::smem_u32(a_blk), b0 = umma::smem_u32(sR + slot * P * BLK);
+#pragma unroll
+        for (int kk = 0; kk < kUmmaBK / 16; ++kk) {
+          const uint64_t da = umma::sw128_desc(a0 + kk * 32), db = umma::sw128_desc(b0 + kk * 32);
+          umma::mma_bf16(dtm, da, db, idesc, (!first || kk > 0) ? 1u : 0u);
+          if (SPLIT) {
+            umma::mma_bf16(dtm, da, umma::sw128_desc(b0 + BLK + kk * 32), idesc, 1);
+            umma::mma_bf16(dtm, umma::sw128_desc(a0 + BLK + kk * 32), db, idesc, 1);
+          }
+        }
+        umma::mma_commit(empty + slot);
+        ++i;
+      };
+      if (ok) ok = umma::mbar_wait(a_ready, 0, abort_flag);
+      umma::tc_fence_after();
+      for (int kc = 0; kc < nkc_out; ++kc) mma_block(acc0, sA + kc * P * BLK, kc == 0);
+      umma::mma_commit(acc0_done);
+      if (ok) ok = umma::mbar_wait(z_ready, 0, abort_flag);
+      umma::tc_fence_after();
+      for (int mc = 0; mc < nM && ok; ++mc) {
+        for (int nt = 0; nt < 2; ++nt)
+          for (int kc = 0; kc < 2; ++kc) mma_block(acc1 + nt * 128, sA + kc * P * BLK, kc == 0);
+        umma::mma_commit(acc1_done);
+        if (ok) ok = umma::mbar_wait(h_ready, mc & 1, abort_flag);
+        umma::tc_fence_after();
+        for (int kc = 0; kc < 2; ++kc) mma_block(acc2, sH + kc * P * BLK, mc == 0 && kc == 0);
+        umma::mma_commit(h_free);
+      }
+      umma::mma_commit(acc2_done);
+    }
+  } else {
+    if (lane == 0) {
+      int i = 0;
+      auto put = [&](const uint8_t *W, int nkcW, int tile, int kc) {
+        const int slot = i % NSLOT;
+        if (i >= NSLOT && ok) ok = umma::mbar_wait(empty + slot, ((i - NSLOT) / NSLOT) & 1, abort_flag);
+        umma::mbar_arrive_expect_tx(full + slot, P * BLK);
+        umma::bulk_g2s(sR + slot * P * BLK, W + ((size_t)tile * nkcW + kc) * P * BLK, P * BLK,
+                       full + slot);
+        ++i;
+      };
+      for (int kc = 0; kc < nkc_out && ok; ++kc) put(t.w_out, nkc_out, 0, kc);
+      for (int mc = 0; mc < nM && ok; ++mc) {
+        for (int nt = 2 * mc; nt < 2 * mc + 2; ++nt)
+          for (int kc = 0; kc < 2; ++kc) put(t.w_ff1, 2, nt, kc);
+        for (int kc = 2 * mc; kc < 2 * mc + 2; ++kc) put(t.w_ff2, 2 * nM, 0, kc);
+      }
+    }
+  }
+  if (!ok) {
+    *abort_flag = 1;
+    atomicOr(t.status, kStatusMmaTimeout);
+  }
+  umma::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) umma::tmem_dealloc(tmem, 512);
+}
+
+}  // namespace atomenc
