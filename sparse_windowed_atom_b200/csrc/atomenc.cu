@@ -27,7 +27,7 @@ namespace {
 
 constexpr int kVersion = 1;
 constexpr int kMaxD = 64;
-constexpr size_t kAttnSmemBudget = 104 * 1024;  // two CTAs per SM (dynamic part)
+constexpr size_t kAttnSmemBudget = 210 * 1024;  // one CTA per SM (dynamic part)
 
 struct Dims {
   int64_t B = 0, A = 0, T = 0, K = 0, C = 0, S = 0, H = 0, D = 0, P = 0, M = 0, U = 0, V = 0;
@@ -256,12 +256,12 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   pl.k_tok = take(cur, pl.enc ? 0 : packed_bytes(V, C, split));
   pl.bytes = cur;
 
-  // ---- attention tile: QT queries per CTA (the grid should cover 2 CTAs x 148 SMs), a
-  // slot plan, (AF3) the pair-bias table and the Q rows; the K/V stage gets the rest
+  // ---- attention tile: QT queries per CTA (the grid should cover the 148 SMs), a slot
+  // plan, (AF3) the pair-bias table and the Q rows; the K/V stage gets the rest
   const int dmax = D <= 8 ? 8 : D <= 16 ? 16 : D <= 32 ? 32 : 64;
   pl.DP = dmax + 4;  // odd number of 16-byte chunks per staged row: no bank conflicts
-  int qt = pl.af3 ? 16 : 32;
-  const int64_t fill = (B * A + 2 * 148 - 1) / (2 * 148);
+  int qt = pl.af3 ? 32 : 64;
+  const int64_t fill = (B * A + 148 - 1) / 148;
   if (fill < qt) qt = (int)(fill < 1 ? 1 : fill);
   while (qt > 1 && attn_fixed_smem(qt, (int)K, (int)H, (int)(H * D), pl.af3) > kAttnSmemBudget / 2)
     qt /= 2;

@@ -9,7 +9,7 @@
 // entries (bullets 5, 6, 15); the weighted values are multiplied by sigmoid of the value
 // gate logits and stored head-major (bullet 16).
 //
-// One CTA (256 threads, two per SM) owns QT consecutive queries of one batch element.
+// One CTA (512 threads, one per SM) owns QT consecutive queries of one batch element.
 //  Phase 0  the tile's Q rows are copied to shared memory with cp.async.
 //  Phase 1  one slot per thread per round (four rounds in flight): key_index and
 //           window_mask are read once (coalesced), eligibility decided and the slot plan
@@ -33,7 +33,7 @@
 
 namespace atomenc {
 
-constexpr int kAttnThreads = 256;
+constexpr int kAttnThreads = 512;
 constexpr int kAttnWarps = kAttnThreads / kWarp;
 constexpr int kPairMax = 32;
 constexpr int kSlotsPerLane = 4;                       // one chunk = 128 slots
@@ -258,7 +258,7 @@ __device__ __forceinline__ float dot_q2_global(const f32x2 (&q2)[DMAX / 2], cons
 // MULTI = true:  any K; pass 1 finds the max and the sum chunk by chunk, pass 2
 //                recomputes the logits to write the weights and accumulate the values.
 template <typename T, int DMAX, bool AF3, bool MULTI>
-__global__ void __launch_bounds__(kAttnThreads, 2) k_slot_attention(AttnArgs g) {
+__global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) {
   extern __shared__ __align__(16) float smem[];
   constexpr int DW = DMAX < 32 ? DMAX : 32;            // channels per reduce-scatter
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
