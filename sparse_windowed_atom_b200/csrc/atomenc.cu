@@ -20,6 +20,7 @@
 #include "gemm_umma.cuh"
 #include "rows.cuh"
 #include "transition.cuh"
+#include "weights.cuh"
 
 using namespace atomenc;
 
@@ -70,8 +71,7 @@ struct Plan {
   // workspace layout (byte offsets)
   size_t o_status, o_usable, o_xstats, o_first, o_last, o_tp, o_x, o_opc, o_rawc, o_cond, o_gate, o_feat,
       o_q, o_k, o_v, o_g, o_o, o_xp, o_z, o_h, o_hid, o_pool;
-  size_t o_wcond, o_wgate, o_wqkv, o_wout, o_wff1, o_wff2, o_wpool, o_wtok, o_wread, o_bscale,
-      o_brg, o_bq, o_wpair, o_rscale, o_rbias;
+  size_t o_wread, o_bscale, o_brg, o_bq, o_wpair, o_rscale, o_rbias;
   // tensor-core images of the weight panels (bf16, hi[/lo])
   size_t k_cond, k_gate, k_qkv0, k_qkv1, k_out, k_ff1, k_ff2, k_pool, k_tok;
   size_t bytes = 0;
@@ -198,7 +198,7 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
     CHECK(check_tensor(out->hidden, fdt, 3, hc));
     CHECK(check_tensor(out->attention, fdt, 4, at));
   }
-  if (D > kMaxD || A >= INT_MAX || K > 8192) return ATOMENC_ERR_UNSUPPORTED;
+  if (D > kMaxD || A > INT_MAX - 4096 || K > 8192) return ATOMENC_ERR_UNSUPPORTED;
 
   // ---- workspace plan
   const int64_t R = B * A;
@@ -229,14 +229,6 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   pl.o_h = take(cur, pl.fuse_tail ? 0 : R * M * 4);
   pl.o_hid = take(cur, R * C * 4);
   pl.o_pool = take(cur, pl.enc ? R * U * 4 : 0);
-  pl.o_wcond = take(cur, S * 6 * C * 4);
-  pl.o_wgate = take(cur, pl.af3 ? S * 2 * C * 4 : 0);
-  pl.o_wqkv = take(cur, C * 4 * HD * 4);
-  pl.o_wout = take(cur, HD * C * 4);
-  pl.o_wff1 = take(cur, C * 2 * M * 4);
-  pl.o_wff2 = take(cur, M * C * 4);
-  pl.o_wpool = take(cur, pl.enc ? C * U * 4 : 0);
-  pl.o_wtok = take(cur, pl.enc ? 0 : V * C * 4);
   pl.o_wread = take(cur, pl.enc ? 0 : C * 3 * 4);
   pl.o_bscale = take(cur, pl.af3 ? 3 * C * 4 : 0);
   pl.o_brg = take(cur, pl.af3 ? 2 * C * 4 : 0);
@@ -295,93 +287,91 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   int *last = reinterpret_cast<int *>(ws + pl.o_last);
 
   hk.mark(0, st);
-  cudaMemsetAsync(status, 0, 4, st);
-  if (pl.enc) {
-    cudaMemsetAsync(first, 0x7F, B * T * 4, st);
-    cudaMemsetAsync(last, 0xFF, B * T * 4, st);
-  }
 
-  // ---- weights into float32 panels
-  CopyJobs jobs;
-  std::memset(&jobs, 0, sizeof(jobs));
-  auto job = [&](const atomenc_tensor &src, size_t src_off_elems, int64_t rows, int64_t cols,
-                 size_t dst_off, int64_t dst_ld, int64_t col0, int64_t cstride,
-                 const atomenc_tensor *rowscale, size_t rs_off) {
-    CopyJob &j = jobs.job[jobs.n++];
-    const size_t es = sizeof(Elt);
-    j.src = static_cast<const unsigned char *>(src.data) + src_off_elems * es;
-    j.rowscale = rowscale ? static_cast<const unsigned char *>(rowscale->data) + rs_off * es : nullptr;
+  // ---- one launch: tensor-core images of the projection weights (built from the
+  // caller's tensors), small float32 panels, status and token-range resets
+  WeightJobs wj;
+  std::memset(&wj, 0, sizeof(wj));
+  const size_t es = sizeof(Elt);
+  auto elt = [&](const atomenc_tensor &t, size_t off) -> const void * {
+    return t.data ? static_cast<const unsigned char *>(t.data) + off * es : nullptr;
+  };
+  auto copy = [&](const atomenc_tensor &src, size_t src_off, int64_t rows, int64_t cols, size_t dst_off,
+                  int64_t dst_ld, int64_t col0, const atomenc_tensor *rowscale, size_t rs_off) {
+    CopyJob &j = wj.copy[wj.ncopy++];
+    j.src = elt(src, src_off);
+    j.rowscale = rowscale ? elt(*rowscale, rs_off) : nullptr;
     j.dst = F(dst_off);
     j.rows = (int32_t)rows;
     j.cols = (int32_t)cols;
     j.dst_ld = (int32_t)dst_ld;
     j.dst_col0 = (int32_t)col0;
-    j.dst_cstride = (int32_t)cstride;
+    j.dst_cstride = 1;
   };
-  if (pl.af3) {
-    for (int jj = 0; jj < 3; ++jj) {
-      job(p->w_scale, (size_t)jj * S * C, S, C, pl.o_wcond, 6 * C, 2 * jj * C, 1, &p->cond_scale, (size_t)jj * S);
-      job(p->w_shift, (size_t)jj * S * C, S, C, pl.o_wcond, 6 * C, 2 * jj * C + C, 1, &p->cond_scale, (size_t)jj * S);
-    }
-    job(p->w_residual_gate, 0, S, C, pl.o_wgate, 2 * C, 0, 1, nullptr, 0);
-    job(p->w_residual_gate, (size_t)S * C, S, C, pl.o_wgate, 2 * C, C, 1, nullptr, 0);
-    job(p->w_q, 0, C, HD, pl.o_wqkv, 2 * HD, 0, 1, nullptr, 0);
-    job(p->w_value_gate, 0, C, HD, pl.o_wqkv, 2 * HD, HD, 1, nullptr, 0);
-    job(p->w_k, 0, C, HD, pl.o_wqkv + (size_t)C * 2 * HD * 4, 2 * HD, 0, 1, nullptr, 0);
-    job(p->w_v, 0, C, HD, pl.o_wqkv + (size_t)C * 2 * HD * 4, 2 * HD, HD, 1, nullptr, 0);
-    job(p->b_scale, 0, 1, 3 * C, pl.o_bscale, 3 * C, 0, 1, nullptr, 0);
-    job(p->b_residual_gate, 0, 1, 2 * C, pl.o_brg, 2 * C, 0, 1, nullptr, 0);
-    job(p->b_q, 0, 1, HD, pl.o_bq, HD, 0, 1, nullptr, 0);
-    job(p->w_pair, 0, P, H, pl.o_wpair, H, 0, 1, &p->pair_scale, 0);
-  } else {
-    job(p->w_mod, 0, S, 6 * C, pl.o_wcond, 6 * C, 0, 1, nullptr, 0);
-    job(p->w_q, 0, C, HD, pl.o_wqkv, 4 * HD, 0, 1, nullptr, 0);
-    job(p->w_k, 0, C, HD, pl.o_wqkv, 4 * HD, HD, 1, nullptr, 0);
-    job(p->w_v, 0, C, HD, pl.o_wqkv, 4 * HD, 2 * HD, 1, nullptr, 0);
-    job(p->w_value_gate, 0, C, HD, pl.o_wqkv, 4 * HD, 3 * HD, 1, nullptr, 0);
-  }
-  job(p->w_attention_out, 0, HD, C, pl.o_wout, C, 0, 1, nullptr, 0);
-  job(p->w_ff_gate, 0, C, M, pl.o_wff1, 2 * M, 0, 2, nullptr, 0);
-  job(p->w_ff_up, 0, C, M, pl.o_wff1, 2 * M, 1, 2, nullptr, 0);
-  job(p->w_ff_out, 0, M, C, pl.o_wff2, C, 0, 1, nullptr, 0);
-  if (pl.enc) {
-    job(p->w_pool, 0, C, U, pl.o_wpool, U, 0, 1, nullptr, 0);
-  } else {
-    job(p->w_token, 0, V, C, pl.o_wtok, C, 0, 1, nullptr, 0);
-    job(p->readout_scale, 0, 1, C, pl.o_rscale, C, 0, 1, nullptr, 0);
-    if (!pl.af3) job(p->readout_bias, 0, 1, C, pl.o_rbias, C, 0, 1, nullptr, 0);
-    job(p->w_readout, 0, C, 3, pl.o_wread, 3, 0, 1, nullptr, 0);
-  }
-  k_prep_weights<Elt><<<dim3(64, jobs.n), 256, 0, st>>>(jobs);
-  ++hk.launches;
-
-  // ---- tensor-core images of the panels
   const bool split = pl.fdt == ATOMENC_F32;
-  PackJobs pj;
-  std::memset(&pj, 0, sizeof(pj));
-  auto pack = [&](size_t panel, int64_t Kd, int64_t N, int64_t ld, size_t dst) {
-    PackJob &j = pj.job[pj.n++];
-    j.src = F(panel);
+  auto pack = [&](size_t dst, int64_t Kd, int64_t N) -> PackJob & {
+    PackJob &j = wj.pack[wj.npack++];
     j.dst = ws + dst;
     j.K = (int32_t)Kd;
     j.N = (int32_t)N;
-    j.ld = (int32_t)ld;
     j.split = split ? 1 : 0;
+    return j;
   };
-  pack(pl.o_wcond, S, 6 * C, 6 * C, pl.k_cond);
+  auto seg = [&](PackJob &j, const atomenc_tensor &src, size_t src_off, int64_t cols, int64_t col0,
+                 int cshift, const atomenc_tensor *rowscale, size_t rs_off) {
+    PackSeg &g = j.seg[j.nseg++];
+    g.src = elt(src, src_off);
+    g.rowscale = rowscale ? elt(*rowscale, rs_off) : nullptr;
+    g.cols = (int32_t)cols;
+    g.col0 = (int32_t)col0;
+    g.cshift = cshift;
+  };
   if (pl.af3) {
-    pack(pl.o_wgate, S, 2 * C, 2 * C, pl.k_gate);
-    pack(pl.o_wqkv, C, 2 * HD, 2 * HD, pl.k_qkv0);
-    pack(pl.o_wqkv + (size_t)C * 2 * HD * 4, C, 2 * HD, 2 * HD, pl.k_qkv1);
+    PackJob &jc = pack(pl.k_cond, S, 6 * C);
+    for (int jj = 0; jj < 3; ++jj) {
+      seg(jc, p->w_scale, (size_t)jj * S * C, C, 2 * jj * C, 0, &p->cond_scale, (size_t)jj * S);
+      seg(jc, p->w_shift, (size_t)jj * S * C, C, 2 * jj * C + C, 0, &p->cond_scale, (size_t)jj * S);
+    }
+    PackJob &jg = pack(pl.k_gate, S, 2 * C);
+    seg(jg, p->w_residual_gate, 0, C, 0, 0, nullptr, 0);
+    seg(jg, p->w_residual_gate, (size_t)S * C, C, C, 0, nullptr, 0);
+    PackJob &j0 = pack(pl.k_qkv0, C, 2 * HD);
+    seg(j0, p->w_q, 0, HD, 0, 0, nullptr, 0);
+    seg(j0, p->w_value_gate, 0, HD, HD, 0, nullptr, 0);
+    PackJob &j1 = pack(pl.k_qkv1, C, 2 * HD);
+    seg(j1, p->w_k, 0, HD, 0, 0, nullptr, 0);
+    seg(j1, p->w_v, 0, HD, HD, 0, nullptr, 0);
+    copy(p->b_scale, 0, 1, 3 * C, pl.o_bscale, 3 * C, 0, nullptr, 0);
+    copy(p->b_residual_gate, 0, 1, 2 * C, pl.o_brg, 2 * C, 0, nullptr, 0);
+    copy(p->b_q, 0, 1, HD, pl.o_bq, HD, 0, nullptr, 0);
+    copy(p->w_pair, 0, P, H, pl.o_wpair, H, 0, &p->pair_scale, 0);
   } else {
-    pack(pl.o_wqkv, C, 4 * HD, 4 * HD, pl.k_qkv0);
+    seg(pack(pl.k_cond, S, 6 * C), p->w_mod, 0, 6 * C, 0, 0, nullptr, 0);
+    PackJob &j0 = pack(pl.k_qkv0, C, 4 * HD);
+    seg(j0, p->w_q, 0, HD, 0, 0, nullptr, 0);
+    seg(j0, p->w_k, 0, HD, HD, 0, nullptr, 0);
+    seg(j0, p->w_v, 0, HD, 2 * HD, 0, nullptr, 0);
+    seg(j0, p->w_value_gate, 0, HD, 3 * HD, 0, nullptr, 0);
   }
-  pack(pl.o_wout, HD, C, C, pl.k_out);
-  pack(pl.o_wff1, C, 2 * M, 2 * M, pl.k_ff1);
-  pack(pl.o_wff2, M, C, C, pl.k_ff2);
-  if (pl.enc) pack(pl.o_wpool, C, U, U, pl.k_pool);
-  else pack(pl.o_wtok, V, C, C, pl.k_tok);
-  k_pack_weights<<<dim3(64, pj.n), 256, 0, st>>>(pj);
+  seg(pack(pl.k_out, HD, C), p->w_attention_out, 0, C, 0, 0, nullptr, 0);
+  PackJob &jf = pack(pl.k_ff1, C, 2 * M);
+  seg(jf, p->w_ff_gate, 0, M, 0, 1, nullptr, 0);
+  seg(jf, p->w_ff_up, 0, M, 1, 1, nullptr, 0);
+  seg(pack(pl.k_ff2, M, C), p->w_ff_out, 0, C, 0, 0, nullptr, 0);
+  if (pl.enc) {
+    seg(pack(pl.k_pool, C, U), p->w_pool, 0, U, 0, 0, nullptr, 0);
+  } else {
+    seg(pack(pl.k_tok, V, C), p->w_token, 0, C, 0, 0, nullptr, 0);
+    copy(p->readout_scale, 0, 1, C, pl.o_rscale, C, 0, nullptr, 0);
+    if (!pl.af3) copy(p->readout_bias, 0, 1, C, pl.o_rbias, C, 0, nullptr, 0);
+    copy(p->w_readout, 0, C, 3, pl.o_wread, 3, 0, nullptr, 0);
+  }
+  wj.fill[wj.nfill++] = FillJob{reinterpret_cast<int *>(status), 1, 0, 0};
+  if (pl.enc) {
+    wj.fill[wj.nfill++] = FillJob{first, B * T, INT_MAX, 0};
+    wj.fill[wj.nfill++] = FillJob{last, B * T, -1, 0};
+  }
+  k_prep_weights<Elt><<<dim3(64, wj.ncopy + wj.npack + wj.nfill), 256, 0, st>>>(wj);
   ++hk.launches;
 
   // out = epi(A' @ W) on the tensor cores, W given by its packed image and A' produced by
@@ -581,7 +571,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     gemm(F(pl.o_hid), C, pl.k_pool, R, U, C, Quad<EpiRelu>{{F(pl.o_pool), U}});
     PoolArgs pa{B, A, T, U, usable, static_cast<const int64_t *>(in->atom_to_token.data), first,
                 last, F(pl.o_pool), out->token_output.data};
-    k_token_mean<Elt><<<(unsigned)(B * T), 128, 0, st>>>(pa);
+    k_token_mean<Elt><<<(unsigned)(B * T), kPoolThreads, 0, st>>>(pa);
     ++hk.launches;
   } else {
     ReadoutArgs rd{R, C, eps, pl.af3 ? 0 : 1, usable, F(pl.o_hid), F(pl.o_rscale), F(pl.o_rbias),

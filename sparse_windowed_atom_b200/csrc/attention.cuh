@@ -11,7 +11,7 @@
 //
 // One CTA (512 threads, one per SM) owns QT consecutive queries of one batch element.
 //  Phase 0  the tile's Q rows are copied to shared memory with cp.async.
-//  Phase 1  one slot per thread per round (four rounds in flight): key_index and
+//  Phase 1  one slot per thread per round (eight rounds in flight): key_index and
 //           window_mask are read once (coalesced), eligibility decided and the slot plan
 //           (key id or -1) written with the span [klo, khi] of the permitted ids; AF3:
 //           the pair bias of every permitted (slot, head) is computed from its pair row
@@ -304,11 +304,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) 
   __syncthreads();
 
   // ---------------- phase 1a: slot plan, one slot per thread per round (coalesced
-  // 8-byte key_index loads, consecutive shared stores), four rounds in flight
+  // 8-byte key_index loads, consecutive shared stores), eight rounds in flight
   int lo = INT_MAX, hi = -1;
   const int64_t sbase = ((int64_t)b * A + a0) * K;     // first slot of the tile
   const int vslots = nq * K;
-  constexpr int R = 4;
+  constexpr int R = 8;
   for (int s0 = tid; s0 < slots; s0 += kAttnThreads * R) {
     int64_t kid[R];
     uint8_t win[R];
@@ -422,93 +422,241 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) 
     }
     __syncthreads();
 
-    for (int q = warp; q < nq; q += kAttnWarps) {
-      const int a = a0 + q;
-      const int64_t arow = (int64_t)b * A + a;
-      int jr[kSlotsPerLane];
-      if (!MULTI) {
+    if (!MULTI && staged && K == kChunk) {
+      // ---- fast path: 128 slots, staged K/V, 32-bit shared addresses, no slot guards;
+      // the warps share the tile's (query, head) pairs evenly
+      const uint32_t rowb = (uint32_t)DP * 4u;
+      const uint32_t hmagic = hg > 1 ? (uint32_t)(0xFFFFFFFFu / (uint32_t)hg + 1u) : 0u;  // ceil(2^32/hg)
+      for (int pr = warp; pr < nq * hg; pr += kAttnWarps) {
+        const int q = hg > 1 ? (int)__umulhi((uint32_t)pr, hmagic) : pr;
+        const int hl = pr - q * hg, h = h0 + hl;
+        const int a = a0 + q;
+        const int64_t arow = (int64_t)b * A + a;
+        // the value-gate logits of this (query, head), fetched early
+        float gv[DMAX / DW];
+#pragma unroll
+        for (int part = 0; part < DMAX; part += DW) {
+          const int d = part + (lane & (DW - 1));
+          gv[part / DW] = lane < DW && d < D ? g.G[arow * HD + h * D + d] : 0.f;
+        }
+        int jr[kSlotsPerLane];
+#pragma unroll
+        for (int i = 0; i < kSlotsPerLane; ++i) jr[i] = plan[q * K + i * kWarp + lane];
+        const uint32_t kb = (uint32_t)__cvta_generic_to_shared(ks) + (uint32_t)(hl * span - klo) * rowb;
+        const uint32_t vb = (uint32_t)__cvta_generic_to_shared(vs) + (uint32_t)(hl * span - klo) * rowb;
+        const uint32_t qa = (uint32_t)__cvta_generic_to_shared(qs) + (uint32_t)(q * HD + h * D) * 4u;
+        f32x2 q2[DMAX / 2];
+        if (fullD) {
+#pragma unroll
+          for (int d = 0; d < DMAX; d += 4) {
+            const ulonglong2 x = lds128(qa + 4u * d);
+            q2[d / 2] = x.x;
+            q2[d / 2 + 1] = x.y;
+          }
+        } else {
+#pragma unroll
+          for (int d = 0; d < DMAX; d += 2)
+            q2[d / 2] = pack2(d < D ? lds32(qa + 4u * d) : 0.f, d + 1 < D ? lds32(qa + 4u * d + 4u) : 0.f);
+        }
+        const uint32_t ba = AF3 ? (uint32_t)__cvta_generic_to_shared(beta) +
+                                      (uint32_t)(h * slots + q * K + lane) * 4u
+                                : 0u;
+        float ev[kSlotsPerLane];
+        uint32_t ja[kSlotsPerLane];
+        float mx = -INFINITY;
 #pragma unroll
         for (int i = 0; i < kSlotsPerLane; ++i) {
-          const int k = i * kWarp + lane;
-          jr[i] = k < K ? plan[q * K + k] : -1;
+          ja[i] = (uint32_t)(jr[i] >= 0 ? jr[i] : klo) * rowb;
+          f32x2 s0 = 0ull, s1 = 0ull;
+#pragma unroll
+          for (int d = 0; d < DMAX; d += 4) {
+            const ulonglong2 k = lds128(kb + ja[i] + 4u * d);
+            s0 = ffma2(q2[d / 2], k.x, s0);
+            s1 = ffma2(q2[d / 2 + 1], k.y, s1);
+          }
+          const float2 x = unpack2(s0), y = unpack2(s1);
+          float l = ((x.x + x.y) + (y.x + y.y)) * g.scale_log2;
+          if (AF3) l = fmaf(lds32(ba + 128u * i), 1.4426950408889634f, l);
+          ev[i] = jr[i] >= 0 ? l : -INFINITY;
+          mx = fmaxf(mx, ev[i]);
+        }
+        mx = warp_max(mx);
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < kSlotsPerLane; ++i) {
+          ev[i] = jr[i] >= 0 ? exp2_approx(ev[i] - mx) : 0.f;
+          sum += ev[i];
+        }
+        sum = warp_sum(sum);
+        float inv = 0.f;
+        if (sum > 0.f) asm("rcp.approx.f32 %0, %1;" : "=f"(inv) : "f"(sum));
+        T *wout = (T *)g.attention + (((int64_t)b * H + h) * A + a) * K + lane;
+        f32x2 acc2[DMAX / 2];
+#pragma unroll
+        for (int d = 0; d < DMAX / 2; ++d) acc2[d] = 0ull;
+#pragma unroll
+        for (int i = 0; i < kSlotsPerLane; ++i) {
+          const float wgt = ev[i] * inv;
+          store_weight<T>(wout, i * kWarp, wgt);
+          const f32x2 w2 = pack2(wgt, wgt);
+#pragma unroll
+          for (int d = 0; d < DMAX; d += 4) {
+            const ulonglong2 v = lds128(vb + ja[i] + 4u * d);
+            acc2[d / 2] = ffma2(w2, v.x, acc2[d / 2]);
+            acc2[d / 2 + 1] = ffma2(w2, v.y, acc2[d / 2 + 1]);
+          }
+        }
+        const bool has = sum > 0.f;
+        float acc[DMAX];
+#pragma unroll
+        for (int d = 0; d < DMAX; d += 2) {
+          const float2 p2 = unpack2(acc2[d / 2]);
+          acc[d] = p2.x;
+          acc[d + 1] = p2.y;
+        }
+#pragma unroll
+        for (int part = 0; part < DMAX; part += DW) {
+          float v[DW];
+#pragma unroll
+          for (int i = 0; i < DW; ++i) v[i] = acc[part + i];
+          const float o = reduce_scatter<DW>(v, lane);
+          const int d = part + (lane & (DW - 1));
+          if (lane < DW && d < D)
+            g.O[arow * HD + h * D + d] = has ? o * sigmoid_fast(gv[part / DW]) : 0.f;
         }
       }
-      if (!MULTI && staged && K == kChunk) {
-        // ---- fast path: 128 slots, staged K/V, 32-bit shared addresses, no slot guards
-        const uint32_t rowb = (uint32_t)DP * 4u;
+    } else {
+      for (int q = warp; q < nq; q += kAttnWarps) {
+        const int a = a0 + q;
+        const int64_t arow = (int64_t)b * A + a;
+        int jr[kSlotsPerLane];
+        if (!MULTI) {
+#pragma unroll
+          for (int i = 0; i < kSlotsPerLane; ++i) {
+            const int k = i * kWarp + lane;
+            jr[i] = k < K ? plan[q * K + k] : -1;
+          }
+        }
         for (int hl = 0; hl < hg; ++hl) {
           const int h = h0 + hl;
-          const uint32_t kb = (uint32_t)__cvta_generic_to_shared(ks) + (uint32_t)(hl * span - klo) * rowb;
-          const uint32_t vb = (uint32_t)__cvta_generic_to_shared(vs) + (uint32_t)(hl * span - klo) * rowb;
-          const uint32_t qa = (uint32_t)__cvta_generic_to_shared(qs) + (uint32_t)(q * HD + h * D) * 4u;
+          const float *qv = qs + q * HD + h * D;
+          const float *kbase = staged ? ks + (hl * span - klo) * DP : nullptr;
+          const float *vbase = staged ? vs + (hl * span - klo) * DP : nullptr;
+          const float *bh = AF3 ? beta + h * slots + q * K : nullptr;
+          // the query, packed once per (query, head), zero beyond D
           f32x2 q2[DMAX / 2];
           if (fullD) {
 #pragma unroll
             for (int d = 0; d < DMAX; d += 4) {
-              const ulonglong2 x = lds128(qa + 4u * d);
+              const ulonglong2 x = *reinterpret_cast<const ulonglong2 *>(qv + d);
               q2[d / 2] = x.x;
               q2[d / 2 + 1] = x.y;
             }
           } else {
 #pragma unroll
             for (int d = 0; d < DMAX; d += 2)
-              q2[d / 2] = pack2(d < D ? lds32(qa + 4u * d) : 0.f, d + 1 < D ? lds32(qa + 4u * d + 4u) : 0.f);
+              q2[d / 2] = pack2(d < D ? qv[d] : 0.f, d + 1 < D ? qv[d + 1] : 0.f);
           }
-          const uint32_t ba = AF3 ? (uint32_t)__cvta_generic_to_shared(beta) +
-                                        (uint32_t)(h * slots + q * K + lane) * 4u
-                                  : 0u;
+
+          // logit of slot k (key j, clamped to a readable row when the slot is not
+          // permitted; the caller masks that value) in log2 units
+          auto logit = [&](int k, int j) -> float {
+            const float dot = staged ? dot_q2<DMAX>(q2, kbase + j * DP)
+                                     : dot_q2_global<DMAX>(q2, g.Kf + ((int64_t)b * A + j) * HD + h * D, D);
+            float l = dot * g.scale_log2;
+            if (AF3) l = fmaf(bh[k], 1.4426950408889634f, l);
+            return l;
+          };
+          const int jsafe = staged ? klo : 0;
+
+          float mx = -INFINITY, sum = 0.f;
           float ev[kSlotsPerLane];
-          uint32_t ja[kSlotsPerLane];
-          float mx = -INFINITY;
+          if (!MULTI) {
 #pragma unroll
-          for (int i = 0; i < kSlotsPerLane; ++i) {
-            ja[i] = (uint32_t)(jr[i] >= 0 ? jr[i] : klo) * rowb;
-            f32x2 s0 = 0ull, s1 = 0ull;
-#pragma unroll
-            for (int d = 0; d < DMAX; d += 4) {
-              const ulonglong2 k = lds128(kb + ja[i] + 4u * d);
-              s0 = ffma2(q2[d / 2], k.x, s0);
-              s1 = ffma2(q2[d / 2 + 1], k.y, s1);
+            for (int i = 0; i < kSlotsPerLane; ++i) {
+              const int k = i * kWarp + lane;
+              const float l = logit(k < K ? k : 0, jr[i] >= 0 ? jr[i] : jsafe);
+              ev[i] = jr[i] >= 0 ? l : -INFINITY;
+              mx = fmaxf(mx, ev[i]);
             }
-            const float2 x = unpack2(s0), y = unpack2(s1);
-            float l = ((x.x + x.y) + (y.x + y.y)) * g.scale_log2;
-            if (AF3) l = fmaf(lds32(ba + 128u * i), 1.4426950408889634f, l);
-            ev[i] = jr[i] >= 0 ? l : -INFINITY;
-            mx = fmaxf(mx, ev[i]);
-          }
-          mx = warp_max(mx);
-          float sum = 0.f;
+            mx = warp_max(mx);
 #pragma unroll
-          for (int i = 0; i < kSlotsPerLane; ++i) {
-            ev[i] = jr[i] >= 0 ? exp2_approx(ev[i] - mx) : 0.f;
-            sum += ev[i];
+            for (int i = 0; i < kSlotsPerLane; ++i) {
+              ev[i] = jr[i] >= 0 ? exp2_approx(ev[i] - mx) : 0.f;
+              sum += ev[i];
+            }
+            sum = warp_sum(sum);
+          } else {
+            for (int c = 0; c < nchunks; ++c) {
+              float cmx = -INFINITY;
+#pragma unroll
+              for (int i = 0; i < kSlotsPerLane; ++i) {
+                const int k = c * kChunk + i * kWarp + lane;
+                jr[i] = k < K ? plan[q * K + k] : -1;
+                ev[i] = jr[i] >= 0 ? logit(k, jr[i]) : -INFINITY;
+                cmx = fmaxf(cmx, ev[i]);
+              }
+              cmx = warp_max(cmx);
+              if (cmx > -INFINITY) {
+                const float nm = fmaxf(mx, cmx);
+                float cs = 0.f;
+#pragma unroll
+                for (int i = 0; i < kSlotsPerLane; ++i)
+                  if (jr[i] >= 0) cs += exp2_approx(ev[i] - nm);
+                sum = sum * exp2_approx(mx - nm) + warp_sum(cs);
+                mx = nm;
+              }
+            }
           }
-          sum = warp_sum(sum);
           float inv = 0.f;
           if (sum > 0.f) asm("rcp.approx.f32 %0, %1;" : "=f"(inv) : "f"(sum));
-          T *wout = (T *)g.attention + (((int64_t)b * H + h) * A + a) * K + lane;
+
           f32x2 acc2[DMAX / 2];
 #pragma unroll
           for (int d = 0; d < DMAX / 2; ++d) acc2[d] = 0ull;
+          T *arow_out = (T *)g.attention + (((int64_t)b * H + h) * A + a) * K;
+          for (int c = 0; c < nchunks; ++c) {
 #pragma unroll
-          for (int i = 0; i < kSlotsPerLane; ++i) {
-            const float wgt = ev[i] * inv;
-            store_weight<T>(wout, i * kWarp, wgt);
-            const f32x2 w2 = pack2(wgt, wgt);
+            for (int i = 0; i < kSlotsPerLane; ++i) {
+              const int k = c * kChunk + i * kWarp + lane;
+              if (MULTI) {
+                jr[i] = k < K ? plan[q * K + k] : -1;
+                ev[i] = jr[i] >= 0 ? exp2_approx(logit(k, jr[i]) - mx) : 0.f;
+              }
+              const int j = jr[i] >= 0 ? jr[i] : jsafe;   // weight 0 on a readable row
+              const float wgt = ev[i] * inv;
+              if (k < K) store_weight<T>(arow_out, k, wgt);
+              if (sum > 0.f) {
+                if (staged) {
+                  const float *vr = vbase + j * DP;
+                  const f32x2 w2 = pack2(wgt, wgt);
 #pragma unroll
-            for (int d = 0; d < DMAX; d += 4) {
-              const ulonglong2 v = lds128(vb + ja[i] + 4u * d);
-              acc2[d / 2] = ffma2(w2, v.x, acc2[d / 2]);
-              acc2[d / 2 + 1] = ffma2(w2, v.y, acc2[d / 2 + 1]);
+                  for (int d = 0; d < DMAX; d += 4) {
+                    const ulonglong2 v = *reinterpret_cast<const ulonglong2 *>(vr + d);
+                    acc2[d / 2] = ffma2(w2, v.x, acc2[d / 2]);
+                    acc2[d / 2 + 1] = ffma2(w2, v.y, acc2[d / 2 + 1]);
+                  }
+                } else {
+                  const float *vr =
+                      staged ? vbase + j * DP : g.Vf + ((int64_t)b * A + j) * HD + h * D;
+#pragma unroll
+                  for (int d = 0; d < DMAX; d += 2) {
+                    const float v0 = d < D ? vr[d] : 0.f, v1 = d + 1 < D ? vr[d + 1] : 0.f;
+                    acc2[d / 2] = ffma2(pack2(wgt, wgt), pack2(v0, v1), acc2[d / 2]);
+                  }
+                }
+              }
             }
           }
+
+          // fold the lanes' partial outputs: lane l ends with channel l (and l + 32)
           const bool has = sum > 0.f;
           float acc[DMAX];
 #pragma unroll
           for (int d = 0; d < DMAX; d += 2) {
-            const float2 p2 = unpack2(acc2[d / 2]);
-            acc[d] = p2.x;
-            acc[d + 1] = p2.y;
+            const float2 p = unpack2(acc2[d / 2]);
+            acc[d] = p.x;
+            acc[d + 1] = p.y;
           }
 #pragma unroll
           for (int part = 0; part < DMAX; part += DW) {
@@ -521,141 +669,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) 
               const int64_t oi = arow * HD + h * D + d;
               g.O[oi] = has ? o * sigmoid_fast(g.G[oi]) : 0.f;
             }
-          }
-        }
-        continue;
-      }
-      for (int hl = 0; hl < hg; ++hl) {
-        const int h = h0 + hl;
-        const float *qv = qs + q * HD + h * D;
-        const float *kbase = staged ? ks + (hl * span - klo) * DP : nullptr;
-        const float *vbase = staged ? vs + (hl * span - klo) * DP : nullptr;
-        const float *bh = AF3 ? beta + h * slots + q * K : nullptr;
-        // the query, packed once per (query, head), zero beyond D
-        f32x2 q2[DMAX / 2];
-        if (fullD) {
-#pragma unroll
-          for (int d = 0; d < DMAX; d += 4) {
-            const ulonglong2 x = *reinterpret_cast<const ulonglong2 *>(qv + d);
-            q2[d / 2] = x.x;
-            q2[d / 2 + 1] = x.y;
-          }
-        } else {
-#pragma unroll
-          for (int d = 0; d < DMAX; d += 2)
-            q2[d / 2] = pack2(d < D ? qv[d] : 0.f, d + 1 < D ? qv[d + 1] : 0.f);
-        }
-
-        // logit of slot k (key j, clamped to a readable row when the slot is not
-        // permitted; the caller masks that value) in log2 units
-        auto logit = [&](int k, int j) -> float {
-          const float dot = staged ? dot_q2<DMAX>(q2, kbase + j * DP)
-                                   : dot_q2_global<DMAX>(q2, g.Kf + ((int64_t)b * A + j) * HD + h * D, D);
-          float l = dot * g.scale_log2;
-          if (AF3) l = fmaf(bh[k], 1.4426950408889634f, l);
-          return l;
-        };
-        const int jsafe = staged ? klo : 0;
-
-        float mx = -INFINITY, sum = 0.f;
-        float ev[kSlotsPerLane];
-        if (!MULTI) {
-#pragma unroll
-          for (int i = 0; i < kSlotsPerLane; ++i) {
-            const int k = i * kWarp + lane;
-            const float l = logit(k < K ? k : 0, jr[i] >= 0 ? jr[i] : jsafe);
-            ev[i] = jr[i] >= 0 ? l : -INFINITY;
-            mx = fmaxf(mx, ev[i]);
-          }
-          mx = warp_max(mx);
-#pragma unroll
-          for (int i = 0; i < kSlotsPerLane; ++i) {
-            ev[i] = jr[i] >= 0 ? exp2_approx(ev[i] - mx) : 0.f;
-            sum += ev[i];
-          }
-          sum = warp_sum(sum);
-        } else {
-          for (int c = 0; c < nchunks; ++c) {
-            float cmx = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < kSlotsPerLane; ++i) {
-              const int k = c * kChunk + i * kWarp + lane;
-              jr[i] = k < K ? plan[q * K + k] : -1;
-              ev[i] = jr[i] >= 0 ? logit(k, jr[i]) : -INFINITY;
-              cmx = fmaxf(cmx, ev[i]);
-            }
-            cmx = warp_max(cmx);
-            if (cmx > -INFINITY) {
-              const float nm = fmaxf(mx, cmx);
-              float cs = 0.f;
-#pragma unroll
-              for (int i = 0; i < kSlotsPerLane; ++i)
-                if (jr[i] >= 0) cs += exp2_approx(ev[i] - nm);
-              sum = sum * exp2_approx(mx - nm) + warp_sum(cs);
-              mx = nm;
-            }
-          }
-        }
-        float inv = 0.f;
-        if (sum > 0.f) asm("rcp.approx.f32 %0, %1;" : "=f"(inv) : "f"(sum));
-
-        f32x2 acc2[DMAX / 2];
-#pragma unroll
-        for (int d = 0; d < DMAX / 2; ++d) acc2[d] = 0ull;
-        T *arow_out = (T *)g.attention + (((int64_t)b * H + h) * A + a) * K;
-        for (int c = 0; c < nchunks; ++c) {
-#pragma unroll
-          for (int i = 0; i < kSlotsPerLane; ++i) {
-            const int k = c * kChunk + i * kWarp + lane;
-            if (MULTI) {
-              jr[i] = k < K ? plan[q * K + k] : -1;
-              ev[i] = jr[i] >= 0 ? exp2_approx(logit(k, jr[i]) - mx) : 0.f;
-            }
-            const int j = jr[i] >= 0 ? jr[i] : jsafe;   // weight 0 on a readable row
-            const float wgt = ev[i] * inv;
-            if (k < K) store_weight<T>(arow_out, k, wgt);
-            if (sum > 0.f) {
-              if (staged) {
-                const float *vr = vbase + j * DP;
-                const f32x2 w2 = pack2(wgt, wgt);
-#pragma unroll
-                for (int d = 0; d < DMAX; d += 4) {
-                  const ulonglong2 v = *reinterpret_cast<const ulonglong2 *>(vr + d);
-                  acc2[d / 2] = ffma2(w2, v.x, acc2[d / 2]);
-                  acc2[d / 2 + 1] = ffma2(w2, v.y, acc2[d / 2 + 1]);
-                }
-              } else {
-                const float *vr =
-                    staged ? vbase + j * DP : g.Vf + ((int64_t)b * A + j) * HD + h * D;
-#pragma unroll
-                for (int d = 0; d < DMAX; d += 2) {
-                  const float v0 = d < D ? vr[d] : 0.f, v1 = d + 1 < D ? vr[d + 1] : 0.f;
-                  acc2[d / 2] = ffma2(pack2(wgt, wgt), pack2(v0, v1), acc2[d / 2]);
-                }
-              }
-            }
-          }
-        }
-
-        // fold the lanes' partial outputs: lane l ends with channel l (and l + 32)
-        const bool has = sum > 0.f;
-        float acc[DMAX];
-#pragma unroll
-        for (int d = 0; d < DMAX; d += 2) {
-          const float2 p = unpack2(acc2[d / 2]);
-          acc[d] = p.x;
-          acc[d + 1] = p.y;
-        }
-#pragma unroll
-        for (int part = 0; part < DMAX; part += DW) {
-          float v[DW];
-#pragma unroll
-          for (int i = 0; i < DW; ++i) v[i] = acc[part + i];
-          const float o = reduce_scatter<DW>(v, lane);
-          const int d = part + (lane & (DW - 1));
-          if (lane < DW && d < D) {
-            const int64_t oi = arow * HD + h * D + d;
-            g.O[oi] = has ? o * sigmoid_fast(g.G[oi]) : 0.f;
           }
         }
       }

@@ -2,7 +2,7 @@
 //   out = epi(A @ W),  A [M, K] float32 or bf16 in global memory, W [K, N] prepacked.
 //
 // One CTA computes a 128 x 128 output tile; 128 threads (4 warps).
-//  * W is prepacked (k_pack_weights) as bf16 blocks of 128 output columns x 64 k in the
+//  * W is prepacked (k_prep_weights) as bf16 blocks of 128 output columns x 64 k in the
 //    exact 128B-swizzled shared-memory image, so a block arrives with one bulk async
 //    copy (mbarrier transaction count).
 //  * The CTA's threads convert their A chunk (128 rows x 64 k) to bf16 and store it
@@ -35,40 +35,6 @@ __host__ __device__ constexpr size_t umma_smem_bytes(bool split) {
 __host__ __device__ inline size_t packed_bytes(int64_t K, int64_t N, bool split) {
   return (size_t)((N + kUmmaBN - 1) / kUmmaBN) * ((K + kUmmaBK - 1) / kUmmaBK) *
          kUmmaBlockBytes * (split ? 2 : 1);
-}
-
-struct PackJob {
-  const float *src;   // [K, N] float32 panel, row stride ld
-  uint8_t *dst;
-  int32_t K, N, ld, split;
-};
-constexpr int kMaxPackJobs = 12;
-struct PackJobs {
-  PackJob job[kMaxPackJobs];
-  int n;
-};
-
-// Pack W [K, N] into blocks (n-tile t, k-chunk c) of [128 n x 64 k] bf16, swizzled K-major,
-// hi block then (split) lo block; zero outside [K, N].
-__global__ void k_pack_weights(PackJobs jobs) {
-  const PackJob &j = jobs.job[blockIdx.y];
-  const int64_t nt = (j.N + kUmmaBN - 1) / kUmmaBN, kc = (j.K + kUmmaBK - 1) / kUmmaBK;
-  const int64_t total = nt * kUmmaBN * kc * kUmmaBK;
-  const int nparts = j.split ? 2 : 1;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t k = i % (kc * kUmmaBK), n = i / (kc * kUmmaBK);
-    const float w = (k < j.K && n < j.N) ? j.src[k * j.ld + n] : 0.f;
-    const int64_t t = n / kUmmaBN, c = k / kUmmaBK;
-    const int nl = (int)(n % kUmmaBN), kl = (int)(k % kUmmaBK);
-    uint8_t *blk = j.dst + (t * kc + c) * nparts * kUmmaBlockBytes;
-    const uint16_t hi = umma::bf16_bits(w);
-    const uint32_t off = umma::swz_offset(nl, kl, kUmmaBN);
-    *reinterpret_cast<uint16_t *>(blk + off) = hi;
-    if (j.split)
-      *reinterpret_cast<uint16_t *>(blk + kUmmaBlockBytes + off) =
-          umma::bf16_bits(w - umma::bf16_val(hi));
-  }
 }
 
 template <typename TA>

@@ -7,38 +7,6 @@
 
 namespace atomenc {
 
-// ------------------------------------------------------------------ weight preparation
-// The block's weights are re-laid out once per call into float32 panels that the
-// projection kernels read: the AF3 cond_scale[j] is folded into w_scale[j] / w_shift[j]
-// (c_j @ W = LN(c) @ (diag(cond_scale[j]) W)), projections that share an input are
-// concatenated along N, and the SwiGLU gate/up weights are interleaved column-wise.
-struct CopyJob {
-  const void *src;       // [rows, cols] dense
-  const void *rowscale;  // optional [rows], same element type as src
-  float *dst;
-  int32_t rows, cols;
-  int32_t dst_ld, dst_col0, dst_cstride;
-  int32_t pad;
-};
-constexpr int kMaxCopyJobs = 28;
-struct CopyJobs {
-  CopyJob job[kMaxCopyJobs];
-  int n;
-};
-
-template <typename T>
-__global__ void k_prep_weights(CopyJobs jobs) {
-  const CopyJob &j = jobs.job[blockIdx.y];
-  const int64_t total = (int64_t)j.rows * j.cols;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    int64_t r = i / j.cols, c = i % j.cols;
-    float v = ldf((const T *)j.src, i);
-    if (j.rowscale) v *= ldf((const T *)j.rowscale, r);
-    j.dst[r * j.dst_ld + j.dst_col0 + c * j.dst_cstride] = v;
-  }
-}
-
 // ------------------------------------------------------------------ row preparation
 struct RowsArgs {
   int64_t B, A, T, C, S;
@@ -295,23 +263,54 @@ struct PoolArgs {
 
 // token_output[t] = exact mean of ReLU(hidden @ w_pool) over the usable atoms mapped
 // to t, summed in ascending atom order (deterministic); 0 for a token with none
-// (bullet 19). One block per token, one thread per output channel.
+// (bullet 19). One block of kPoolThreads per token: the atoms of the token's range are
+// tested 128 at a time into a shared flag row, then each thread sums three output
+// channels over the flagged rows with four rows' loads in flight.
+constexpr int kPoolThreads = 128;
 template <typename T>
-__global__ void k_token_mean(PoolArgs p) {
+__global__ void __launch_bounds__(kPoolThreads) k_token_mean(PoolArgs p) {
+  __shared__ uint8_t s_flag[kPoolThreads + 4];
+  const int tid = threadIdx.x;
   const int64_t bt = blockIdx.x;
   const int64_t b = bt / p.T, t = bt % p.T;
   const int first = p.tok_first[bt], last = p.tok_last[bt];
-  for (int64_t u = threadIdx.x; u < p.U; u += blockDim.x) {
-    float acc = 0.f;
+  const int64_t U = p.U;
+  for (int64_t u0 = 0; u0 < U; u0 += 3 * kPoolThreads) {
+    float acc[3] = {0.f, 0.f, 0.f};
     int n = 0;
-    for (int a = first; a <= last; ++a) {
-      const int64_t row = b * p.A + a;
-      if (p.usable[row] && p.att[row] == t) {
-        acc += p.pooled[row * p.U + u];
-        ++n;
+    for (int base = first; base <= last; base += kPoolThreads) {
+      const int a = base + tid;
+      bool f = false;
+      if (a <= last) {
+        const int64_t row = b * p.A + a;
+        f = p.usable[row] != 0 && p.att[row] == t;
       }
+      s_flag[tid] = f ? 1 : 0;
+      if (tid < 4) s_flag[kPoolThreads + tid] = 0;
+      n += __syncthreads_count(f);
+      const int cnt = min(kPoolThreads, last - base + 1);
+      const float *rows = p.pooled + (b * p.A + base) * U + u0 + tid;
+      for (int i = 0; i < cnt; i += 4) {
+        float x[4][3];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+#pragma unroll
+          for (int c = 0; c < 3; ++c)
+            x[e][c] = s_flag[i + e] && u0 + tid + c * kPoolThreads < U
+                          ? rows[(int64_t)(i + e) * U + c * kPoolThreads]
+                          : 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+#pragma unroll
+          for (int c = 0; c < 3; ++c) acc[c] += x[e][c];
+      }
+      __syncthreads();
     }
-    stf((T *)p.out, bt * p.U + u, n > 0 ? acc / (float)n : 0.f);
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      const int64_t u = u0 + tid + c * kPoolThreads;
+      if (u < U) stf((T *)p.out, bt * U + u, n > 0 ? acc[c] / (float)n : 0.f);
+    }
   }
 }
 

@@ -1,0 +1,139 @@
+// weights.cuh -- once-per-call weight preparation, one launch for the whole block:
+//  * tensor-core images: every projection weight W [K, N] (input dim K, output columns N)
+//    is written as bf16 blocks of 128 output columns x 64 k in the exact 128B-swizzled
+//    shared-memory layout the tcgen05 kernels read (hi block, then lo = bf16(w - hi)
+//    for float32 workloads), straight from the caller's tensors. A destination may
+//    gather its columns from several source tensors (projections that share an input
+//    are concatenated along N; the SwiGLU gate/up columns are interleaved), and a
+//    per-input-row scale may be folded in (AF3: c_j @ W = LN(c) @ (diag(cond_scale[j]) W)).
+//  * small float32 panels (biases, the folded pair weights, the readout weights);
+//  * the status word and the per-token atom ranges are reset.
+// Page "Local atom attention, encoder pooling and decoder skip/readout", Required
+// behavior bullets 7-10 and 16-20 name the weights; the layouts are this library's.
+#pragma once
+
+#include "common.cuh"
+#include "gemm_umma.cuh"
+#include "umma.cuh"
+
+namespace atomenc {
+
+// float32 panel: dst[r * dst_ld + dst_col0 + c * dst_cstride] = src[r, c] (* rowscale[r])
+struct CopyJob {
+  const void *src;       // [rows, cols] dense
+  const void *rowscale;  // optional [rows], same element type as src
+  float *dst;
+  int32_t rows, cols;
+  int32_t dst_ld, dst_col0, dst_cstride;
+  int32_t pad;
+};
+
+// destination columns col0 + (c << cshift), c < cols, come from src [K, cols]
+struct PackSeg {
+  const void *src;
+  const void *rowscale;  // optional [K]
+  int32_t cols, col0, cshift, pad;
+};
+constexpr int kMaxPackSegs = 6;
+struct PackJob {
+  PackSeg seg[kMaxPackSegs];
+  uint8_t *dst;
+  int32_t K, N, nseg, split;
+};
+
+struct FillJob {
+  int *dst;
+  int64_t n;
+  int value;
+  int pad;
+};
+
+constexpr int kMaxCopyJobs = 12, kMaxPackJobs = 10, kMaxFillJobs = 3;
+struct WeightJobs {
+  CopyJob copy[kMaxCopyJobs];
+  PackJob pack[kMaxPackJobs];
+  FillJob fill[kMaxFillJobs];
+  int ncopy, npack, nfill, pad;
+};
+
+// One 16-byte chunk of the image per thread: output column n, eight consecutive k
+// (lanes take consecutive n, so each of the eight source rows is read coalesced).
+template <typename T>
+__device__ __forceinline__ void pack_chunk(const PackJob &j, int64_t i, int64_t Npad, int64_t kc) {
+  const int n = (int)(i % Npad), k0 = (int)(i / Npad) * 8;
+  int s_hit = -1, c = 0;
+  for (int s = 0; s < j.nseg; ++s) {
+    const int rel = n - j.seg[s].col0;
+    if (rel >= 0 && (rel & ((1 << j.seg[s].cshift) - 1)) == 0 && (rel >> j.seg[s].cshift) < j.seg[s].cols) {
+      s_hit = s;
+      c = rel >> j.seg[s].cshift;
+    }
+  }
+  float v[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) v[e] = 0.f;
+  if (s_hit >= 0 && n < j.N) {
+    const PackSeg &sg = j.seg[s_hit];
+    const T *src = static_cast<const T *>(sg.src);
+    const T *rs = static_cast<const T *>(sg.rowscale);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int k = k0 + e;
+      if (k < j.K) {
+        v[e] = ldf(src, (int64_t)k * sg.cols + c);
+        if (rs) v[e] *= ldf(rs, k);
+      }
+    }
+  }
+  uint32_t hi[4], lo[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const uint16_t h0 = umma::bf16_bits(v[2 * w]), h1 = umma::bf16_bits(v[2 * w + 1]);
+    hi[w] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+    const uint16_t l0 = umma::bf16_bits(v[2 * w] - umma::bf16_val(h0));
+    const uint16_t l1 = umma::bf16_bits(v[2 * w + 1] - umma::bf16_val(h1));
+    lo[w] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+  }
+  const int64_t t = n / kUmmaBN, cb = k0 / kUmmaBK;
+  const int nparts = j.split ? 2 : 1;
+  uint8_t *blk = j.dst + (t * kc + cb) * nparts * kUmmaBlockBytes;
+  const uint32_t off = umma::swz_offset(n % kUmmaBN, k0 % kUmmaBK, kUmmaBN);
+  *reinterpret_cast<uint4 *>(blk + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  if (j.split)
+    *reinterpret_cast<uint4 *>(blk + kUmmaBlockBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+}
+
+// grid.y = ncopy + npack + nfill jobs; grid.x strides over each job's elements
+template <typename T>
+__global__ void k_prep_weights(WeightJobs w) {
+  int y = blockIdx.y;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (y < w.ncopy) {
+    const CopyJob &j = w.copy[y];
+    const int64_t total = (int64_t)j.rows * j.cols;
+    for (int64_t i = i0; i < total; i += stride) {
+      const int64_t r = i / j.cols, c = i % j.cols;
+      float v = ldf((const T *)j.src, i);
+      if (j.rowscale) v *= ldf((const T *)j.rowscale, r);
+      j.dst[r * j.dst_ld + j.dst_col0 + c * j.dst_cstride] = v;
+    }
+    return;
+  }
+  y -= w.ncopy;
+  if (y < w.npack) {
+    const PackJob &j = w.pack[y];
+    const int64_t Npad = (j.N + kUmmaBN - 1) / kUmmaBN * kUmmaBN;
+    const int64_t kc = (j.K + kUmmaBK - 1) / kUmmaBK;
+    const int64_t total = Npad * kc * (kUmmaBK / 8);
+    for (int64_t i = i0; i < total; i += stride) pack_chunk<T>(j, i, Npad, kc);
+    return;
+  }
+  y -= w.npack;
+  if (y < w.nfill) {
+    const FillJob &f = w.fill[y];
+    for (int64_t i = i0; i < f.n; i += stride) f.dst[i] = f.value;
+  }
+}
+
+}  // namespace atomenc
