@@ -341,11 +341,18 @@ def run_atomenc(args):
         return atomenc.atomenc_forward_profiled(spec.style, spec.stage, inputs, params, spec.eps,
                                                 spec.radius, outs, ws, evrow, stream)
 
+    def fwd_plain():
+        atomenc.atomenc_forward(spec.style, spec.stage, inputs, params, spec.eps, spec.radius,
+                                outs, ws, stream)
+
     warm_ev = make_events(1)[0]
+    per_step_launches = 0
     for _ in range(W):
         flush.zero_()
-        fwd(warm_ev)
+        per_step_launches = fwd(warm_ev)
     evs = make_events(K)
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
     torch.cuda.synchronize(dev)
     status = atomenc.atomenc_get_status(ws, stream)
 
@@ -356,20 +363,35 @@ def run_atomenc(args):
         pass
     sampler = ClockSampler(uuid)
     time.sleep(0.3)
+    # ---- the timed steps: one forward per step through the C ABI, events only around it
+    # (kernels of a step follow each other with programmatic dependent launch)
     barrier()
     torch.cuda.synchronize(dev)
     sampler.start()
-    launches = 0
     for i in range(K):
         flush.zero_()
-        launches += fwd(evs[i])
+        step_ev[i][0].record(stream)
+        fwd_plain()
+        step_ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     sampler.stop()
+    launches = per_step_launches * K
 
-    step_ms = [evs[i][0].elapsed_time(evs[i][nph - 1]) for i in range(K)]
+    # ---- phase pass: the same steps again with an event at every phase boundary (these
+    # events serialise the phases); gives the breakdown and the attention kernel's time
+    barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        flush.zero_()
+        fwd(evs[i])
+    torch.cuda.synchronize(dev)
+    barrier()
+
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
     phase_ms = [statistics.fmean(evs[i][p].elapsed_time(evs[i][p + 1]) for i in range(K))
                 for p in range(atomenc.NUM_PHASES)]
+    phased_step_ms = statistics.fmean(evs[i][0].elapsed_time(evs[i][nph - 1]) for i in range(K))
     total_ms = max_over_ranks(sum(step_ms))
     ms_per_step = total_ms / K
     atoms = spec.atoms * world
@@ -437,6 +459,7 @@ def run_atomenc(args):
             "gpu_launches": launches,
             "clocks": sampler.summary(),
             "phase_ms": dict(zip(atomenc.PHASES, phase_ms)),
+            "phase_pass_ms_per_step": phased_step_ms,
             "dominant_phase": atomenc.PHASES[dominant],
             "device_status": status,
         }

@@ -12,6 +12,7 @@
 #include <cstring>
 #include <mutex>
 #include <type_traits>
+#include <utility>
 
 #include "../../include/atomenc.h"
 #include "attention.cuh"
@@ -227,7 +228,7 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   pl.o_xp = take(cur, pl.fuse_tail ? 0 : R * C * 4);
   pl.o_z = take(cur, pl.fuse_tail ? 0 : R * C * 4);
   pl.o_h = take(cur, pl.fuse_tail ? 0 : R * M * 4);
-  pl.o_hid = take(cur, R * C * 4);
+  pl.o_hid = take(cur, pl.fuse_tail && fdt == ATOMENC_F32 ? 0 : R * C * 4);  // float32 hidden copy
   pl.o_pool = take(cur, pl.enc ? R * U * 4 : 0);
   pl.o_wread = take(cur, pl.enc ? 0 : C * 3 * 4);
   pl.o_bscale = take(cur, pl.af3 ? 3 * C * 4 : 0);
@@ -268,8 +269,28 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
 struct Hooks {
   cudaEvent_t const *ev = nullptr;  // ATOMENC_NUM_PHASES + 1 events, or null
   int launches = 0;
+  cudaError_t err = cudaSuccess;    // first launch failure
   void mark(int i, cudaStream_t st) const {
     if (ev) cudaEventRecord(ev[i], st);
+  }
+  // Every kernel is launched here, with programmatic stream serialization: it may be
+  // scheduled while its predecessor finishes and waits for it in pdl_enter().
+  template <typename... KP, typename... Args>
+  void launch(void (*kern)(KP...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+              Args &&...args) {
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    if (e != cudaSuccess && err == cudaSuccess) err = e;
+    ++launches;
   }
 };
 
@@ -371,8 +392,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     wj.fill[wj.nfill++] = FillJob{first, B * T, INT_MAX, 0};
     wj.fill[wj.nfill++] = FillJob{last, B * T, -1, 0};
   }
-  k_prep_weights<Elt><<<dim3(64, wj.ncopy + wj.npack + wj.nfill), 256, 0, st>>>(wj);
-  ++hk.launches;
+  hk.launch((k_prep_weights<Elt>), dim3(64, wj.ncopy + wj.npack + wj.nfill), 256, 0, st, wj);
 
   // out = epi(A' @ W) on the tensor cores, W given by its packed image and A' produced by
   // `prod` (A itself, or a row normalisation fused into the operand); K <= 256
@@ -387,12 +407,11 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     const size_t smem = rows_smem_bytes(Kd, split);
     if (split) {
       cudaFuncSetAttribute(k_gemm_rows<P, true, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      k_gemm_rows<P, true, E><<<grid, kRowsThreads, smem, st>>>(prod, ws + wpk, Mr, N, Kd, per, epi, status);
+      hk.launch((k_gemm_rows<P, true, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, epi, status);
     } else {
       cudaFuncSetAttribute(k_gemm_rows<P, false, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      k_gemm_rows<P, false, E><<<grid, kRowsThreads, smem, st>>>(prod, ws + wpk, Mr, N, Kd, per, epi, status);
+      hk.launch((k_gemm_rows<P, false, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, epi, status);
     }
-    ++hk.launches;
   };
   // out = epi(A @ W): the row-block kernel for K <= 256, else the streaming kernel
   auto gemm = [&](auto *A_, int64_t lda, size_t wpk, int64_t Mr, int64_t N, int64_t Kd, auto epi) {
@@ -406,12 +425,11 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     const size_t smem = umma_smem_bytes(split);
     if (split) {
       cudaFuncSetAttribute(k_gemm_umma<TA, true, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      k_gemm_umma<TA, true, E><<<grid, kUmmaThreads, smem, st>>>(A_, lda, ws + wpk, Mr, N, Kd, epi, status);
+      hk.launch((k_gemm_umma<TA, true, E>), grid, kUmmaThreads, smem, st, A_, lda, ws + wpk, Mr, N, Kd, epi, status);
     } else {
       cudaFuncSetAttribute(k_gemm_umma<TA, false, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      k_gemm_umma<TA, false, E><<<grid, kUmmaThreads, smem, st>>>(A_, lda, ws + wpk, Mr, N, Kd, epi, status);
+      hk.launch((k_gemm_umma<TA, false, E>), grid, kUmmaThreads, smem, st, A_, lda, ws + wpk, Mr, N, Kd, epi, status);
     }
-    ++hk.launches;
   };
   // the conditioning-modulated row norm of x (or x') fused into a projection's operand
   const bool fuse_norm = C <= kRowsKMax;
@@ -438,8 +456,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   ra.token_proj = F(pl.o_tp);
   ra.usable = usable; ra.x = F(pl.o_x); ra.xstats = F(pl.o_xstats); ra.opc = F(pl.o_opc); ra.rawc = F(pl.o_rawc);
   ra.tok_first = first; ra.tok_last = last;
-  k_rows_prep<Elt><<<row_blocks, 256, 0, st>>>(ra);
-  ++hk.launches;
+  hk.launch((k_rows_prep<Elt>), row_blocks, 256, 0, st, ra);
   hk.mark(1, st);
 
   // ---- conditioning
@@ -454,8 +471,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   hk.mark(2, st);
   if (!fuse_norm) {
     FeatArgs fa{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_x), F(pl.o_cond), F(pl.o_feat)};
-    k_features<<<row_blocks, 256, 0, st>>>(fa);
-    ++hk.launches;
+    hk.launch(k_features, row_blocks, 256, 0, st, fa);
   }
 
   // ---- projections (attention inputs fused into the operand when C <= 256)
@@ -478,12 +494,11 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     RopeArgs rp{R, H, D, eps, usable, in->rope_cos.data, in->rope_sin.data, F(pl.o_q), F(pl.o_k)};
     if (D >= 8 && D <= 128 && (D & (D - 1)) == 0) {
       const int64_t warps = R * 2;
-      k_qk_rope_warp<Elt><<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(rp);
+      hk.launch((k_qk_rope_warp<Elt>), (unsigned)((warps + 7) / 8), 256, 0, st, rp);
     } else {
       const int64_t n = R * H * 2;
-      k_qk_rope<Elt><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(rp);
+      hk.launch((k_qk_rope<Elt>), (unsigned)((n + 255) / 256), 256, 0, st, rp);
     }
-    ++hk.launches;
   }
   hk.mark(3, st);
 
@@ -508,8 +523,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     dim3 grid((unsigned)((A + pl.QT - 1) / pl.QT), (unsigned)B);
     auto go = [&](auto kern) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.attn_smem);
-      kern<<<grid, kAttnThreads, pl.attn_smem, st>>>(ag);
-      ++hk.launches;
+      hk.launch(kern, grid, kAttnThreads, pl.attn_smem, st, ag);
     };
     const int dm = D <= 8 ? 8 : D <= 16 ? 16 : D <= 32 ? 32 : 64;
     const bool multi = K > kChunk;
@@ -541,23 +555,21 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     ta.rms = pl.af3 ? 0 : 1; ta.plus1 = pl.af3 ? 0 : 1; ta.eps = eps;
     ta.usable = usable;
     ta.w_out = ws + pl.k_out; ta.w_ff1 = ws + pl.k_ff1; ta.w_ff2 = ws + pl.k_ff2;
-    ta.hid32 = F(pl.o_hid); ta.hidden = out->hidden.data; ta.status = status;
+    ta.hid32 = split ? nullptr : F(pl.o_hid); ta.hidden = out->hidden.data; ta.status = status;
     const size_t smem = trans_smem_bytes(split);
     const dim3 grid((unsigned)((R + kUmmaBM - 1) / kUmmaBM));
     if (split) {
       cudaFuncSetAttribute(k_transition<true, Elt>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      k_transition<true, Elt><<<grid, kTransThreads, smem, st>>>(ta);
+      hk.launch((k_transition<true, Elt>), grid, kTransThreads, smem, st, ta);
     } else {
       cudaFuncSetAttribute(k_transition<false, Elt>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      k_transition<false, Elt><<<grid, kTransThreads, smem, st>>>(ta);
+      hk.launch((k_transition<false, Elt>), grid, kTransThreads, smem, st, ta);
     }
-    ++hk.launches;
   } else {
     gemm(F(pl.o_o), HD, pl.k_out, R, C, HD,
          Quad<EpiResidual>{{F(pl.o_x), gbuf, gld, g0off, C, F(pl.o_xp)}});
     TNormArgs tn{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_xp), F(pl.o_cond), F(pl.o_z)};
-    k_transition_norm<<<row_blocks, 256, 0, st>>>(tn);
-    ++hk.launches;
+    hk.launch(k_transition_norm, row_blocks, 256, 0, st, tn);
     gemm(F(pl.o_z), C, pl.k_ff1, R, 2 * M, C, EpiSwiGLU{F(pl.o_h), M});
     gemm(F(pl.o_h), M, pl.k_ff2, R, C, M,
          Quad<EpiHidden<Elt>>{{F(pl.o_xp), gbuf, gld, g1off, C, usable, F(pl.o_hid),
@@ -566,20 +578,20 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
 
   hk.mark(5, st);
 
-  // ---- boundary
+  // ---- boundary (float32 hidden: the output itself when it is float32 and fused)
+  const float *hid = pl.fuse_tail && split ? static_cast<const float *>(out->hidden.data) : F(pl.o_hid);
   if (pl.enc) {
-    gemm(F(pl.o_hid), C, pl.k_pool, R, U, C, Quad<EpiRelu>{{F(pl.o_pool), U}});
+    gemm(hid, C, pl.k_pool, R, U, C, Quad<EpiRelu>{{F(pl.o_pool), U}});
     PoolArgs pa{B, A, T, U, usable, static_cast<const int64_t *>(in->atom_to_token.data), first,
                 last, F(pl.o_pool), out->token_output.data};
-    k_token_mean<Elt><<<(unsigned)(B * T), kPoolThreads, 0, st>>>(pa);
-    ++hk.launches;
+    hk.launch((k_token_mean<Elt>), (unsigned)(B * T), kPoolThreads, 0, st, pa);
   } else {
-    ReadoutArgs rd{R, C, eps, pl.af3 ? 0 : 1, usable, F(pl.o_hid), F(pl.o_rscale), F(pl.o_rbias),
+    ReadoutArgs rd{R, C, eps, pl.af3 ? 0 : 1, usable, hid, F(pl.o_rscale), F(pl.o_rbias),
                    F(pl.o_wread), out->position_update.data};
-    k_readout<Elt><<<row_blocks, 256, 0, st>>>(rd);
-    ++hk.launches;
+    hk.launch((k_readout<Elt>), row_blocks, 256, 0, st, rd);
   }
   hk.mark(6, st);
+  if (hk.err != cudaSuccess) return ATOMENC_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ATOMENC_OK : ATOMENC_ERR_CUDA;
 }
 

@@ -259,6 +259,7 @@ __device__ __forceinline__ float dot_q2_global(const f32x2 (&q2)[DMAX / 2], cons
 //                recomputes the logits to write the weights and accumulate the values.
 template <typename T, int DMAX, bool AF3, bool MULTI>
 __global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) {
+  pdl_enter();
   extern __shared__ __align__(16) float smem[];
   constexpr int DW = DMAX < 32 ? DMAX : 32;            // channels per reduce-scatter
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;

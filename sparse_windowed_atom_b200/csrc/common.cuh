@@ -10,6 +10,16 @@ namespace atomenc {
 constexpr int kWarp = 32;
 
 // ---- element access: every float tensor is float32 or bf16 in memory, float32 in math
+// Programmatic dependent launch. Every kernel of a forward pass is launched so that it
+// may be scheduled while its predecessor in the stream is still running. Its first act
+// is to wait until that predecessor grid has completed and its writes are visible
+// (before any global or tensor memory is touched, so chains of such kernels stay in
+// stream order); then it lets its own successor begin launching.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ float ldf(const float *p, int64_t i) { return p[i]; }
 __device__ __forceinline__ float ldf(const __nv_bfloat16 *p, int64_t i) {
   return __bfloat162float(p[i]);

@@ -117,6 +117,7 @@ template <typename TA, bool SPLIT, class Epi>
 __global__ void __launch_bounds__(kUmmaThreads)
     k_gemm_umma(const TA *__restrict__ A, int64_t lda, const uint8_t *__restrict__ Wpk, int64_t M,
                 int64_t N, int64_t K, Epi epi, unsigned *status) {
+  pdl_enter();
   extern __shared__ __align__(1024) uint8_t smem_dyn[];
   // 1024-byte alignment of the operand blocks (swizzle atoms)
   uint8_t *sm = reinterpret_cast<uint8_t *>(
@@ -253,6 +254,7 @@ template <class Prod, bool SPLIT, class Epi>
 __global__ void __launch_bounds__(kRowsThreads, 1)
     k_gemm_rows(Prod prod, const uint8_t *__restrict__ Wpk, int64_t M, int64_t N, int64_t K,
                 int tiles_per_cta, Epi epi, unsigned *status) {
+  pdl_enter();
   extern __shared__ __align__(1024) uint8_t smem_dyn[];
   constexpr int PARTS = SPLIT ? 2 : 1, NSLOT = rows_slots(SPLIT);
   constexpr uint32_t BLK = kUmmaBlockBytes;

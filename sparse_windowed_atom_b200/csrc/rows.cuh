@@ -29,6 +29,7 @@ struct RowsArgs {
 // (bullet 3); encoder x = atom, decoder x = skip + gather(token @ w_token) (bullet 3).
 template <typename T>
 __global__ void k_rows_prep(RowsArgs r) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= r.B * r.A) return;
@@ -106,6 +107,7 @@ struct FeatArgs {
 // AF3: A_j(x) = LN(x) * sigmoid(c_j @ w_scale[j] + b_scale[j]) + c_j @ w_shift[j]  (bullet 7)
 // ESM: attention input = RMS(x) * (1 + attention_scale) + attention_shift  (bullet 11)
 __global__ void k_features(FeatArgs f) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= f.rows) return;
@@ -146,6 +148,7 @@ struct RopeArgs {
 // One thread per (atom, head, Q-or-K); D <= 128.
 template <typename T>
 __global__ void k_qk_rope(RopeArgs r) {
+  pdl_enter();
   const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (id >= r.rows * r.H * 2) return;
   const int which = (int)(id & 1);
@@ -177,6 +180,7 @@ __global__ void k_qk_rope(RopeArgs r) {
 // sits D/8 lanes away in the same head group.
 template <typename T>
 __global__ void k_qk_rope_warp(RopeArgs r) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (wid >= r.rows * 2) return;
@@ -228,6 +232,7 @@ struct TNormArgs {
 // Normalise the NEW residual state: AF3 A_2(x'); ESMFold2
 // RMS(x') * (1 + transition_scale) + transition_shift  (bullet 17)
 __global__ void k_transition_norm(TNormArgs f) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= f.rows) return;
@@ -269,6 +274,7 @@ struct PoolArgs {
 constexpr int kPoolThreads = 128;
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads) k_token_mean(PoolArgs p) {
+  pdl_enter();
   __shared__ uint8_t s_flag[kPoolThreads + 4];
   const int tid = threadIdx.x;
   const int64_t bt = blockIdx.x;
@@ -331,6 +337,7 @@ struct ReadoutArgs {
 // to zero; an update, not coordinates (bullets 18-20). One warp per atom.
 template <typename T>
 __global__ void k_readout(ReadoutArgs r) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= r.rows) return;

@@ -12,9 +12,9 @@
 // never go to HBM.
 //
 // Warp roles: warps 0-3 convert the o rows into the first operand, then work one output
-// row per thread (TMEM lanes 32w..32w+31): residual, row statistics and z (written as the
-// next operand), SiLU(gate) * up per chunk (written as the last operand), and the final
-// gated residual; warp 4 lane 0 issues the MMAs; warp 5 lane 0 streams the packed weight
+// row per thread (TMEM lanes 32w..32w+31): residual x' (stored back into TMEM over the
+// out-projection accumulator), row statistics and z (written as the next operand),
+// SiLU(gate) * up per chunk (written as the last operand), and the final gated residual; warp 4 lane 0 issues the MMAs; warp 5 lane 0 streams the packed weight
 // blocks through a ring of bulk async copies in the order the MMAs consume them. Every
 // wait is bounded (status bit 4 on timeout). Needs C == 128, H*D in {64, 128}, M a
 // multiple of 128.
@@ -41,7 +41,7 @@ struct TransArgs {
   float eps;
   const uint8_t *usable;
   const uint8_t *w_out, *w_ff1, *w_ff2;   // packed tensor-core images
-  float *hid32;                // [R, 128] float32 hidden
+  float *hid32;                // [R, 128] float32 copy of hidden (null: not needed)
   void *hidden;                // [R, 128] output
   unsigned *status;
 };
@@ -49,19 +49,6 @@ struct TransArgs {
 __host__ __device__ inline size_t trans_smem_bytes(bool split) {
   const size_t parts = split ? 2 : 1, slots = split ? 2 : 3;
   return 1024 + (2 + 2 + slots) * parts * kUmmaBlockBytes + 256;
-}
-
-template <typename T>
-__device__ __forceinline__ void store4(T *p, int64_t i, float4 v);
-template <>
-__device__ __forceinline__ void store4<float>(float *p, int64_t i, float4 v) {
-  *reinterpret_cast<float4 *>(p + i) = v;
-}
-template <>
-__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *p, int64_t i, float4 v) {
-  const uint32_t lo = (uint32_t)umma::bf16_bits(v.x) | ((uint32_t)umma::bf16_bits(v.y) << 16);
-  const uint32_t hi = (uint32_t)umma::bf16_bits(v.z) | ((uint32_t)umma::bf16_bits(v.w) << 16);
-  *reinterpret_cast<uint2 *>(p + i) = make_uint2(lo, hi);
 }
 
 // eight floats of one row into an operand block pair (hi, and lo when split) at column k
@@ -98,8 +85,22 @@ __device__ __forceinline__ void row32(const float *p, int64_t ld, int64_t r, boo
   }
 }
 
+template <typename T>
+__device__ __forceinline__ void store4(T *p, int64_t i, float4 v);
+template <>
+__device__ __forceinline__ void store4<float>(float *p, int64_t i, float4 v) {
+  *reinterpret_cast<float4 *>(p + i) = v;
+}
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *p, int64_t i, float4 v) {
+  const uint32_t lo = (uint32_t)umma::bf16_bits(v.x) | ((uint32_t)umma::bf16_bits(v.y) << 16);
+  const uint32_t hi = (uint32_t)umma::bf16_bits(v.z) | ((uint32_t)umma::bf16_bits(v.w) << 16);
+  *reinterpret_cast<uint2 *>(p + i) = make_uint2(lo, hi);
+}
+
 template <bool SPLIT, typename TOut>
 __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
+  pdl_enter();
   extern __shared__ __align__(1024) uint8_t smem_dyn[];
   constexpr int P = SPLIT ? 2 : 1, NSLOT = SPLIT ? 2 : 3, C = 128;
   constexpr uint32_t BLK = kUmmaBlockBytes;
@@ -163,45 +164,47 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
     umma::fence_async_smem();
     umma::mbar_arrive(a_ready);
 
-    // ---- x' = x + g0 * acc0; statistics of x' (one shifted pass), then z -> operand
+    // ---- x' = x + g0 * acc0, kept in TMEM in place of acc0; statistics of x' (one
+    // shifted pass); then z -> operand
     if (ok) ok = umma::mbar_wait(acc0_done, 0, abort_flag);
     umma::tc_fence_after();
     float shift = 0.f, s1 = 0.f, s2 = 0.f;
 #pragma unroll 1
     for (int c0 = 0; c0 < C; c0 += 32) {
       float a[32], xv[32], gv[32];
-      umma::tmem_ld32(tl + c0, a);
       row32(t.x, C, r, rok, c0, xv);
       row32(t.g0, t.g_ld, r, rok, c0, gv);
-      if (c0 == 0) shift = t.rms ? 0.f : fmaf(gv[0], a[0], xv[0]);
+      umma::tmem_ld32(tl + c0, a);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) a[i] = fmaf(gv[i], a[i], xv[i]);
+      if (c0 == 0) shift = t.rms ? 0.f : a[0];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float d = fmaf(gv[i], a[i], xv[i]) - shift;
+        const float d = a[i] - shift;
         s1 += d;
         s2 = fmaf(d, d, s2);
       }
+      umma::tmem_st32(tl + c0, a);
     }
+    umma::tmem_wait_st();
     const float m = s1 / (float)C;
     const float mean = t.rms ? 0.f : shift + m;
     const float var = t.rms ? s2 / (float)C : fmaxf(s2 / (float)C - m * m, 0.f);
     const float rstd = 1.f / sqrtf(var + t.eps);
 #pragma unroll 1
     for (int c0 = 0; c0 < C; c0 += 32) {
-      float a[32], xv[32], gv[32], sv[32], hv[32];
-      umma::tmem_ld32(tl + c0, a);
-      row32(t.x, C, r, rok, c0, xv);
-      row32(t.g0, t.g_ld, r, rok, c0, gv);
+      float a[32], sv[32], hv[32];
       row32(t.sc, t.cond_ld, r, rok, c0, sv);
       row32(t.sh, t.cond_ld, r, rok, c0, hv);
+      umma::tmem_ld32(tl + c0, a);
 #pragma unroll
       for (int s8 = 0; s8 < 4; ++s8) {
         float z[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int i = s8 * 8 + e;
-          const float xp = fmaf(gv[i], a[i], xv[i]);
           const float sc = t.plus1 ? 1.f + sv[i] : sv[i];
-          z[e] = rok ? fmaf((xp - mean) * rstd, sc, hv[i]) : 0.f;
+          z[e] = rok ? fmaf((a[i] - mean) * rstd, sc, hv[i]) : 0.f;
         }
         const int k = c0 + s8 * 8;
         put8<SPLIT>(sA + (k / kUmmaBK) * P * BLK, rl, k % kUmmaBK, z);
@@ -240,24 +243,21 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
     // ---- hidden = usable * (x' + g1 * acc2)
     if (ok) ok = umma::mbar_wait(acc2_done, 0, abort_flag);
     umma::tc_fence_after();
-    const bool use = rok && t.usable[r] != 0;
+    const bool use = ok && rok && t.usable[r] != 0;
 #pragma unroll 1
     for (int c0 = 0; c0 < C; c0 += 32) {
-      float a[32], f[32], xv[32], gv[32], g1v[32];
+      float a[32], f[32], g1v[32];
+      row32(t.g1, t.g_ld, r, rok, c0, g1v);
       umma::tmem_ld32(tl + c0, a);
       umma::tmem_ld32(tl + 384 + c0, f);
-      row32(t.x, C, r, rok, c0, xv);
-      row32(t.g0, t.g_ld, r, rok, c0, gv);
-      row32(t.g1, t.g_ld, r, rok, c0, g1v);
-      if (rok && ok) {
+      if (rok) {
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
           float o[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            o[e] = use ? fmaf(g1v[i + e], f[i + e], fmaf(gv[i + e], a[i + e], xv[i + e])) : 0.f;
+          for (int e = 0; e < 4; ++e) o[e] = use ? fmaf(g1v[i + e], f[i + e], a[i + e]) : 0.f;
           const float4 o4 = make_float4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<float4 *>(t.hid32 + r * C + c0 + i) = o4;
+          if (t.hid32) *reinterpret_cast<float4 *>(t.hid32 + r * C + c0 + i) = o4;
           store4<TOut>((TOut *)t.hidden, r * C + c0 + i, o4);
         }
       }

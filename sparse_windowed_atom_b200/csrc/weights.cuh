@@ -106,6 +106,7 @@ __device__ __forceinline__ void pack_chunk(const PackJob &j, int64_t i, int64_t 
 // grid.y = ncopy + npack + nfill jobs; grid.x strides over each job's elements
 template <typename T>
 __global__ void k_prep_weights(WeightJobs w) {
+  pdl_enter();
   int y = blockIdx.y;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
