@@ -6,8 +6,9 @@
 //                                                                          (bullets 17, 18)
 // (page "Local atom attention, encoder pooling and decoder skip/readout", Required
 // behavior). The three products run on tcgen05 with their operands chained through
-// shared memory and three TMEM accumulators: out-projection (128 columns), one 128-wide
-// chunk of the SwiGLU hidden width at a time (256 interleaved gate/up columns) and
+// shared memory and TMEM accumulators: out-projection (128 columns), the SwiGLU hidden
+// width in 64-wide chunks (128 interleaved gate/up columns each, two TMEM buffers and two
+// shared operand buffers, so the products of chunk i+1 overlap the SiLU of chunk i) and
 // w_ff_out (128 columns), 512 TMEM columns in all; x', z and the SwiGLU intermediate
 // never go to HBM.
 //
@@ -46,8 +47,9 @@ struct TransArgs {
   unsigned *status;
 };
 
+constexpr int kTransSlotsSplit = 3, kTransSlotsPlain = 6;   // weight ring depth
 __host__ __device__ inline size_t trans_smem_bytes(bool split) {
-  const size_t parts = split ? 2 : 1, slots = split ? 2 : 3;
+  const size_t parts = split ? 2 : 1, slots = split ? kTransSlotsSplit : kTransSlotsPlain;
   return 1024 + (2 + 2 + slots) * parts * kUmmaBlockBytes + 256;
 }
 
@@ -102,7 +104,7 @@ template <bool SPLIT, typename TOut>
 __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
   pdl_enter();
   extern __shared__ __align__(1024) uint8_t smem_dyn[];
-  constexpr int P = SPLIT ? 2 : 1, NSLOT = SPLIT ? 2 : 3, C = 128;
+  constexpr int P = SPLIT ? 2 : 1, NSLOT = SPLIT ? kTransSlotsSplit : kTransSlotsPlain, C = 128;
   constexpr uint32_t BLK = kUmmaBlockBytes;
   constexpr uint32_t idesc = umma::idesc_bf16(kUmmaBM, kUmmaBN);
   uint8_t *sm = reinterpret_cast<uint8_t *>(
@@ -112,14 +114,14 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
   uint8_t *sR = sH + 2 * P * BLK;          // weight ring [NSLOT][P]
   uint64_t *full = reinterpret_cast<uint64_t *>(sR + NSLOT * P * BLK);
   uint64_t *empty = full + NSLOT, *a_ready = empty + NSLOT, *acc0_done = a_ready + 1,
-           *z_ready = acc0_done + 1, *acc1_done = z_ready + 1, *h_ready = acc1_done + 1,
-           *h_free = h_ready + 1, *acc2_done = h_free + 1;
+           *z_ready = acc0_done + 1, *acc1_full = z_ready + 1, *h_ready = acc1_full + 2,
+           *h_free = h_ready + 2, *acc2_done = h_free + 2;                 // [2] = per buffer
   uint32_t *tslot = reinterpret_cast<uint32_t *>(acc2_done + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t m0 = (int64_t)blockIdx.x * kUmmaBM;
-  const int nkc_out = t.HD / kUmmaBK, nM = t.M / 128;
+  const int nkc_out = t.HD / kUmmaBK, nC = t.M / 64;   // 64-wide hidden chunks
 
   if (tid == 0) {
     for (int s = 0; s < NSLOT; ++s) {
@@ -129,9 +131,11 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
     umma::mbar_init(a_ready, 128);
     umma::mbar_init(acc0_done, 1);
     umma::mbar_init(z_ready, 128);
-    umma::mbar_init(acc1_done, 1);
-    umma::mbar_init(h_ready, 128);
-    umma::mbar_init(h_free, 1);
+    for (int b = 0; b < 2; ++b) {
+      umma::mbar_init(acc1_full + b, 1);
+      umma::mbar_init(h_ready + b, 128);
+      umma::mbar_init(h_free + b, 1);
+    }
     umma::mbar_init(acc2_done, 1);
     *abort_flag = 0;
     umma::fence_mbar_init();
@@ -141,7 +145,7 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
   __syncthreads();
   umma::tc_fence_after();
   const uint32_t tmem = *tslot;
-  const uint32_t acc0 = tmem, acc1 = tmem + 128, acc2 = tmem + 384;
+  const uint32_t acc0 = tmem, acc1 = tmem + 128, acc2 = tmem + 384;   // acc1: two 128-col buffers
   bool ok = true;
 
   if (warp < 4) {
@@ -166,14 +170,19 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
 
     // ---- x' = x + g0 * acc0, kept in TMEM in place of acc0; statistics of x' (one
     // shifted pass); then z -> operand
+    float xv[32], gv[32];                       // chunk 0 fetched before the wait
+    row32(t.x, C, r, rok, 0, xv);
+    row32(t.g0, t.g_ld, r, rok, 0, gv);
     if (ok) ok = umma::mbar_wait(acc0_done, 0, abort_flag);
     umma::tc_fence_after();
     float shift = 0.f, s1 = 0.f, s2 = 0.f;
 #pragma unroll 1
     for (int c0 = 0; c0 < C; c0 += 32) {
-      float a[32], xv[32], gv[32];
-      row32(t.x, C, r, rok, c0, xv);
-      row32(t.g0, t.g_ld, r, rok, c0, gv);
+      float a[32];
+      if (c0 > 0) {
+        row32(t.x, C, r, rok, c0, xv);
+        row32(t.g0, t.g_ld, r, rok, c0, gv);
+      }
       umma::tmem_ld32(tl + c0, a);
 #pragma unroll
       for (int i = 0; i < 32; ++i) a[i] = fmaf(gv[i], a[i], xv[i]);
@@ -214,40 +223,44 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
     umma::fence_async_smem();
     umma::mbar_arrive(z_ready);
 
-    // ---- SwiGLU, one 128-wide chunk of the hidden width at a time -> last operand
-    for (int mc = 0; mc < nM; ++mc) {
-      if (ok) ok = umma::mbar_wait(acc1_done, mc & 1, abort_flag);
-      if (mc > 0 && ok) ok = umma::mbar_wait(h_free, (mc - 1) & 1, abort_flag);
+    // ---- SwiGLU, one 64-wide chunk i of the hidden width at a time: TMEM buffer i % 2
+    // (128 interleaved gate/up columns) -> shared operand buffer i % 2
+    for (int ch = 0; ch < nC; ++ch) {
+      const int bf = ch & 1;
+      if (ok) ok = umma::mbar_wait(acc1_full + bf, (ch >> 1) & 1, abort_flag);
+      if (ch >= 2 && ok) ok = umma::mbar_wait(h_free + bf, ((ch - 2) >> 1) & 1, abort_flag);
       umma::tc_fence_after();
 #pragma unroll 1
-      for (int c0 = 0; c0 < 256; c0 += 32) {
+      for (int c0 = 0; c0 < 128; c0 += 32) {
         float a[32];
-        umma::tmem_ld32(tl + 128 + c0, a);
+        umma::tmem_ld32(tl + 128 + bf * 128 + c0, a);
 #pragma unroll
         for (int s8 = 0; s8 < 2; ++s8) {
           float h[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const int i = s8 * 16 + 2 * e;
-            h[e] = silu_fast(a[i]) * a[i + 1];
+            const int j = s8 * 16 + 2 * e;
+            h[e] = silu_fast(a[j]) * a[j + 1];
           }
-          const int k = c0 / 2 + s8 * 8;
-          put8<SPLIT>(sH + (k / kUmmaBK) * P * BLK, rl, k % kUmmaBK, h);
+          put8<SPLIT>(sH + bf * P * BLK, rl, c0 / 2 + s8 * 8, h);
         }
       }
       umma::tc_fence_before();
       umma::fence_async_smem();
-      umma::mbar_arrive(h_ready);
+      umma::mbar_arrive(h_ready + bf);
     }
 
     // ---- hidden = usable * (x' + g1 * acc2)
+    float g1v[32];                              // chunk 0 fetched before the wait
+    row32(t.g1, t.g_ld, r, rok, 0, g1v);
+    const bool use_row = rok && t.usable[r] != 0;
     if (ok) ok = umma::mbar_wait(acc2_done, 0, abort_flag);
     umma::tc_fence_after();
-    const bool use = ok && rok && t.usable[r] != 0;
+    const bool use = ok && use_row;
 #pragma unroll 1
     for (int c0 = 0; c0 < C; c0 += 32) {
-      float a[32], f[32], g1v[32];
-      row32(t.g1, t.g_ld, r, rok, c0, g1v);
+      float a[32], f[32];
+      if (c0 > 0) row32(t.g1, t.g_ld, r, rok, c0, g1v);
       umma::tmem_ld32(tl + c0, a);
       umma::tmem_ld32(tl + 384 + c0, f);
       if (rok) {
@@ -288,14 +301,18 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
       umma::mma_commit(acc0_done);
       if (ok) ok = umma::mbar_wait(z_ready, 0, abort_flag);
       umma::tc_fence_after();
-      for (int mc = 0; mc < nM && ok; ++mc) {
-        for (int nt = 0; nt < 2; ++nt)
-          for (int kc = 0; kc < 2; ++kc) mma_block(acc1 + nt * 128, sA + kc * P * BLK, kc == 0);
-        umma::mma_commit(acc1_done);
-        if (ok) ok = umma::mbar_wait(h_ready, mc & 1, abort_flag);
+      auto ff1 = [&](int ch) {   // hidden chunk ch (n-tile ch of w_ff1) -> acc1 buffer ch % 2
+        for (int kc = 0; kc < 2; ++kc) mma_block(acc1 + (ch & 1) * 128, sA + kc * P * BLK, kc == 0);
+        umma::mma_commit(acc1_full + (ch & 1));
+      };
+      ff1(0);
+      if (nC > 1) ff1(1);
+      for (int ch = 0; ch < nC && ok; ++ch) {
+        if (ok) ok = umma::mbar_wait(h_ready + (ch & 1), (ch >> 1) & 1, abort_flag);
         umma::tc_fence_after();
-        for (int kc = 0; kc < 2; ++kc) mma_block(acc2, sH + kc * P * BLK, mc == 0 && kc == 0);
-        umma::mma_commit(h_free);
+        mma_block(acc2, sH + (ch & 1) * P * BLK, ch == 0);
+        umma::mma_commit(h_free + (ch & 1));
+        if (ch + 2 < nC) ff1(ch + 2);
       }
       umma::mma_commit(acc2_done);
     }
@@ -311,10 +328,15 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
         ++i;
       };
       for (int kc = 0; kc < nkc_out && ok; ++kc) put(t.w_out, nkc_out, 0, kc);
-      for (int mc = 0; mc < nM && ok; ++mc) {
-        for (int nt = 2 * mc; nt < 2 * mc + 2; ++nt)
-          for (int kc = 0; kc < 2; ++kc) put(t.w_ff1, 2, nt, kc);
-        for (int kc = 2 * mc; kc < 2 * mc + 2; ++kc) put(t.w_ff2, 2 * nM, 0, kc);
+      // same order as the MMAs consume them
+      auto ld_ff1 = [&](int ch) {
+        for (int kc = 0; kc < 2; ++kc) put(t.w_ff1, 2, ch, kc);
+      };
+      ld_ff1(0);
+      if (nC > 1) ld_ff1(1);
+      for (int ch = 0; ch < nC && ok; ++ch) {
+        put(t.w_ff2, nC, 0, ch);
+        if (ch + 2 < nC) ld_ff1(ch + 2);
       }
     }
   }
