@@ -341,8 +341,7 @@ def run_atomenc(args):
         return atomenc.atomenc_forward_profiled(spec.style, spec.stage, inputs, params, spec.eps,
                                                 spec.radius, outs, ws, evrow, stream)
 
-    def fwd_plain():
-        atomenc.atomenc_forward(spec.style, spec.stage, inputs, params, spec.eps, spec.radius,
+    fwd_plain = atomenc.Forward(spec.style, spec.stage, inputs, params, spec.eps, spec.radius,
                                 outs, ws, stream)
 
     warm_ev = make_events(1)[0]
@@ -368,10 +367,13 @@ def run_atomenc(args):
     barrier()
     torch.cuda.synchronize(dev)
     sampler.start()
+    host_s = 0.0
     for i in range(K):
         flush.zero_()
         step_ev[i][0].record(stream)
+        h0 = time.perf_counter()
         fwd_plain()
+        host_s += time.perf_counter() - h0
         step_ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -460,6 +462,7 @@ def run_atomenc(args):
             "clocks": sampler.summary(),
             "phase_ms": dict(zip(atomenc.PHASES, phase_ms)),
             "phase_pass_ms_per_step": phased_step_ms,
+            "host_us_per_call": 1e6 * host_s / K,
             "dominant_phase": atomenc.PHASES[dominant],
             "device_status": status,
         }

@@ -149,6 +149,29 @@ def atomenc_forward(style: str, stage: str, inputs: dict, params: dict, eps: flo
         raise AtomencError(rc, "atomenc_forward")
 
 
+class Forward:
+    """atomenc_forward prepared once for a fixed set of tensors: the descriptors are
+    built at construction, so each call is a single C call (no per-call marshalling).
+    The tensors must stay alive, in place and unchanged in shape while it is used."""
+
+    def __init__(self, style: str, stage: str, inputs: dict, params: dict, eps: float,
+                 radius: int, outputs: dict, workspace: torch.Tensor, stream=None):
+        self._ins, self._prm, self._outs = _structs(inputs, params, outputs)
+        self._keep = (inputs, params, outputs, workspace)
+        self._fn = load_library().atomenc_forward
+        self._args = (STYLES[style], STAGES[stage], ctypes.byref(self._ins),
+                      ctypes.byref(self._prm), float(eps), int(radius), ctypes.byref(self._outs),
+                      workspace.data_ptr(), workspace.numel() * workspace.element_size())
+        self._stream = None if stream is None else _stream_ptr(stream)
+
+    def __call__(self, stream=None) -> None:
+        sp = _stream_ptr(stream) if stream is not None else (
+            self._stream if self._stream is not None else _stream_ptr(None))
+        rc = self._fn(*self._args, sp)
+        if rc != 0:
+            raise AtomencError(rc, "atomenc_forward")
+
+
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 

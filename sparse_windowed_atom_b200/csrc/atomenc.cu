@@ -10,6 +10,7 @@
 #include <climits>
 #include <cmath>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <type_traits>
 #include <utility>
@@ -266,6 +267,41 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   return ATOMENC_OK;
 }
 
+constexpr int kMaxDevices = 64;
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device), and again only
+// if a larger size is asked for: the attribute outlives the call, so repeating it on
+// every forward would only add host time.
+struct SmemLimit {
+  const void *fn;
+  int dev, bytes;
+};
+constexpr int kMaxSmemLimits = 512;
+SmemLimit g_smem_limits[kMaxSmemLimits];
+int g_num_smem_limits = 0;
+std::mutex g_smem_limits_mutex;
+
+template <typename... KP>
+cudaError_t smem_limit(void (*kern)(KP...), size_t bytes) {
+  const void *fn = reinterpret_cast<const void *>(kern);
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  std::lock_guard<std::mutex> lock(g_smem_limits_mutex);
+  int slot = -1;
+  for (int i = 0; i < g_num_smem_limits; ++i)
+    if (g_smem_limits[i].fn == fn && g_smem_limits[i].dev == dev) slot = i;
+  if (slot >= 0 && (int)bytes <= g_smem_limits[slot].bytes) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess || dev < 0) return e;
+  if (slot < 0 && g_num_smem_limits < kMaxSmemLimits) {
+    slot = g_num_smem_limits++;
+    g_smem_limits[slot].fn = fn;
+    g_smem_limits[slot].dev = dev;
+  }
+  if (slot >= 0) g_smem_limits[slot].bytes = (int)bytes;
+  return e;
+}
+
 struct Hooks {
   cudaEvent_t const *ev = nullptr;  // ATOMENC_NUM_PHASES + 1 events, or null
   int launches = 0;
@@ -406,10 +442,10 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     dim3 grid((unsigned)((nt + per - 1) / per), (unsigned)mt);
     const size_t smem = rows_smem_bytes(Kd, split);
     if (split) {
-      cudaFuncSetAttribute(k_gemm_rows<P, true, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      smem_limit(k_gemm_rows<P, true, E>, smem);
       hk.launch((k_gemm_rows<P, true, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, epi, status);
     } else {
-      cudaFuncSetAttribute(k_gemm_rows<P, false, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      smem_limit(k_gemm_rows<P, false, E>, smem);
       hk.launch((k_gemm_rows<P, false, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, epi, status);
     }
   };
@@ -424,10 +460,10 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     dim3 grid((unsigned)((N + kUmmaBN - 1) / kUmmaBN), (unsigned)((Mr + kUmmaBM - 1) / kUmmaBM));
     const size_t smem = umma_smem_bytes(split);
     if (split) {
-      cudaFuncSetAttribute(k_gemm_umma<TA, true, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      smem_limit(k_gemm_umma<TA, true, E>, smem);
       hk.launch((k_gemm_umma<TA, true, E>), grid, kUmmaThreads, smem, st, A_, lda, ws + wpk, Mr, N, Kd, epi, status);
     } else {
-      cudaFuncSetAttribute(k_gemm_umma<TA, false, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      smem_limit(k_gemm_umma<TA, false, E>, smem);
       hk.launch((k_gemm_umma<TA, false, E>), grid, kUmmaThreads, smem, st, A_, lda, ws + wpk, Mr, N, Kd, epi, status);
     }
   };
@@ -522,7 +558,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   {
     dim3 grid((unsigned)((A + pl.QT - 1) / pl.QT), (unsigned)B);
     auto go = [&](auto kern) {
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.attn_smem);
+      smem_limit(kern, pl.attn_smem);
       hk.launch(kern, grid, kAttnThreads, pl.attn_smem, st, ag);
     };
     const int dm = D <= 8 ? 8 : D <= 16 ? 16 : D <= 32 ? 32 : 64;
@@ -559,10 +595,10 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     const size_t smem = trans_smem_bytes(split);
     const dim3 grid((unsigned)((R + kUmmaBM - 1) / kUmmaBM));
     if (split) {
-      cudaFuncSetAttribute(k_transition<true, Elt>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      smem_limit(k_transition<true, Elt>, smem);
       hk.launch((k_transition<true, Elt>), grid, kTransThreads, smem, st, ta);
     } else {
-      cudaFuncSetAttribute(k_transition<false, Elt>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      smem_limit(k_transition<false, Elt>, smem);
       hk.launch((k_transition<false, Elt>), grid, kTransThreads, smem, st, ta);
     }
   } else {
@@ -652,7 +688,6 @@ int atomenc_forward_profiled(int style, int stage, const atomenc_inputs *in,
 // ---- no-allocation variant: scratch in a file-scope device array, address looked up
 // once per device with that device current
 static __device__ __align__(256) unsigned char g_noalloc_scratch[ATOMENC_NOALLOC_SCRATCH_BYTES];
-constexpr int kMaxDevices = 64;
 static void *g_noalloc_addr[kMaxDevices];
 static std::mutex g_noalloc_mutex;
 

@@ -285,9 +285,9 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       umma::mbar_init(accf + b, 1);
-      umma::mbar_init(acce + b, 128);
+      umma::mbar_init(acce + b, 4);        // one arrival per epilogue warp
     }
-    umma::mbar_init(aready, 128);
+    umma::mbar_init(aready, 4);
     *abort_flag = 0;
     umma::fence_mbar_init();
   }
@@ -334,14 +334,15 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
       }
     }
     umma::fence_async_smem();
-    umma::mbar_arrive(aready);
+    __syncwarp();
+    if (lane == 0) umma::mbar_arrive(aready);
 
     // ---- epilogue of each output tile
     float *T = sT + warp * 32 * 33;
     const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
     for (int tl = 0; tl < ntl; ++tl) {
       const int buf = tl & 1;
-      if (ok) ok = umma::mbar_wait(accf + buf, (tl >> 1) & 1, abort_flag);
+      if (ok) ok = umma::mbar_wait_warp(accf + buf, (tl >> 1) & 1, abort_flag, lane);
       umma::tc_fence_after();
       const int64_t n0 = (int64_t)(t_begin + tl) * kUmmaBN;
 #pragma unroll 1
@@ -365,7 +366,8 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         __syncwarp();
       }
       umma::tc_fence_before();
-      umma::mbar_arrive(acce + buf);
+      __syncwarp();
+      if (lane == 0) umma::mbar_arrive(acce + buf);
     }
   } else if (warp == 4) {
     if (lane == 0) {

@@ -128,12 +128,12 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
       umma::mbar_init(full + s, 1);
       umma::mbar_init(empty + s, 1);
     }
-    umma::mbar_init(a_ready, 128);
+    umma::mbar_init(a_ready, 4);          // one arrival per epilogue warp
     umma::mbar_init(acc0_done, 1);
-    umma::mbar_init(z_ready, 128);
+    umma::mbar_init(z_ready, 4);
     for (int b = 0; b < 2; ++b) {
       umma::mbar_init(acc1_full + b, 1);
-      umma::mbar_init(h_ready + b, 128);
+      umma::mbar_init(h_ready + b, 4);
       umma::mbar_init(h_free + b, 1);
     }
     umma::mbar_init(acc2_done, 1);
@@ -166,14 +166,15 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
         put8<SPLIT>(sA + kc * P * BLK, warp * 32 + it * 4 + (lane >> 3), (lane & 7) * 8, v[it]);
     }
     umma::fence_async_smem();
-    umma::mbar_arrive(a_ready);
+    __syncwarp();
+    if (lane == 0) umma::mbar_arrive(a_ready);
 
     // ---- x' = x + g0 * acc0, kept in TMEM in place of acc0; statistics of x' (one
     // shifted pass); then z -> operand
     float xv[32], gv[32];                       // chunk 0 fetched before the wait
     row32(t.x, C, r, rok, 0, xv);
     row32(t.g0, t.g_ld, r, rok, 0, gv);
-    if (ok) ok = umma::mbar_wait(acc0_done, 0, abort_flag);
+    if (ok) ok = umma::mbar_wait_warp(acc0_done, 0, abort_flag, lane);
     umma::tc_fence_after();
     float shift = 0.f, s1 = 0.f, s2 = 0.f;
 #pragma unroll 1
@@ -221,14 +222,15 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
     }
     umma::tc_fence_before();
     umma::fence_async_smem();
-    umma::mbar_arrive(z_ready);
+    __syncwarp();
+    if (lane == 0) umma::mbar_arrive(z_ready);
 
     // ---- SwiGLU, one 64-wide chunk i of the hidden width at a time: TMEM buffer i % 2
     // (128 interleaved gate/up columns) -> shared operand buffer i % 2
     for (int ch = 0; ch < nC; ++ch) {
       const int bf = ch & 1;
-      if (ok) ok = umma::mbar_wait(acc1_full + bf, (ch >> 1) & 1, abort_flag);
-      if (ch >= 2 && ok) ok = umma::mbar_wait(h_free + bf, ((ch - 2) >> 1) & 1, abort_flag);
+      if (ok) ok = umma::mbar_wait_warp(acc1_full + bf, (ch >> 1) & 1, abort_flag, lane);
+      if (ch >= 2 && ok) ok = umma::mbar_wait_warp(h_free + bf, ((ch - 2) >> 1) & 1, abort_flag, lane);
       umma::tc_fence_after();
 #pragma unroll 1
       for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -247,14 +249,15 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
       }
       umma::tc_fence_before();
       umma::fence_async_smem();
-      umma::mbar_arrive(h_ready + bf);
+      __syncwarp();
+      if (lane == 0) umma::mbar_arrive(h_ready + bf);
     }
 
     // ---- hidden = usable * (x' + g1 * acc2)
     float g1v[32];                              // chunk 0 fetched before the wait
     row32(t.g1, t.g_ld, r, rok, 0, g1v);
     const bool use_row = rok && t.usable[r] != 0;
-    if (ok) ok = umma::mbar_wait(acc2_done, 0, abort_flag);
+    if (ok) ok = umma::mbar_wait_warp(acc2_done, 0, abort_flag, lane);
     umma::tc_fence_after();
     const bool use = ok && use_row;
 #pragma unroll 1

@@ -41,7 +41,9 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                : "memory");
 }
 // Wait for the phase with the given parity to complete; false if the poll limit ran out
-// or (when `abort` is given) another thread of the CTA already gave up.
+// or (when `abort` is given) another thread of the CTA already gave up. Polls with the
+// non-blocking test_wait: a try_wait that suspends the thread was seen to notice a
+// completed phase microseconds late.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           volatile int *abort = nullptr) {
   const uint32_t a = smem_u32(bar);
@@ -50,7 +52,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
         : "r"(a), "r"(parity)
@@ -58,6 +60,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     if (done) return true;
   }
   return false;
+}
+
+// The same wait for a whole warp: lane 0 polls, the other lanes learn the outcome from it
+// (one poller per warp keeps the barrier word free for the arrivals). Warp-uniform call.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity,
+                                               volatile int *abort, int lane) {
+  int done = 1;
+  if (lane == 0) done = mbar_wait(bar, parity, abort) ? 1 : 0;
+  done = __shfl_sync(0xffffffffu, done, 0);
+  __syncwarp();
+  return done != 0;
 }
 
 // ---- bulk async copy global -> shared (16-byte aligned, size a multiple of 16)

@@ -146,6 +146,29 @@ def test_deterministic_and_inputs_untouched():
                 and torch.equal(torch.nan_to_num(v), torch.nan_to_num(before[k])), k
 
 
+@pytest.mark.parametrize("style", ["af3", "esmfold2"])
+def test_prepared_forward_matches_the_plain_call(style):
+    """atomenc.Forward (descriptors built once) gives bit-identical results to
+    atomenc_forward, call after call."""
+    w = workloads.make_inputs(workloads.tiny_spec(style, "encoder", A=500, T=64), seed=21)
+    act, prm, msk, st = to_torch(w)
+    spec = w["spec"]
+    ref = atomenc.windowed_atom_attention(act, prm, msk, st, style=style, stage="encoder",
+                                          eps=spec.eps, radius=spec.radius)
+    inputs = {**act, **msk, **st}
+    outs = {k: torch.empty_like(v) for k, v in ref.items()}
+    ws = torch.empty(atomenc.atomenc_workspace_size(style, "encoder", inputs, prm, outs),
+                     dtype=torch.uint8, device="cuda")
+    fwd = atomenc.Forward(style, "encoder", inputs, prm, spec.eps, spec.radius, outs, ws)
+    for _ in range(2):
+        for v in outs.values():
+            v.fill_(7.0)
+        fwd()
+        torch.cuda.synchronize()
+        for k in ref:
+            assert torch.equal(outs[k], ref[k]), k
+
+
 def test_argument_errors_are_reported():
     w = workloads.make_inputs(workloads.tiny_spec("esmfold2", "encoder"), seed=13)
     act, prm, msk, st = to_torch(w)
