@@ -39,6 +39,7 @@ constexpr int kPairMax = 32;
 constexpr int kSlotsPerLane = 4;                       // one chunk = 128 slots
 constexpr int kChunk = kWarp * kSlotsPerLane;
 constexpr int kAttnHeadsMax = 32;                      // AF3 w_pair columns in shared memory
+constexpr int kMaxQT = 64;                             // queries per CTA at most
 
 struct AttnArgs {
   int B, A, K, H, D, P;
@@ -262,6 +263,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) 
   pdl_enter();
   extern __shared__ __align__(16) float smem[];
   constexpr int DW = DMAX < 32 ? DMAX : 32;            // channels per reduce-scatter
+  // Query pairs sharing their key rows are processed jointly in the 128-slot path; built
+  // for the ESMFold2 style at 16 < D <= 32 only (with the AF3 pair-bias reads, or at
+  // D <= 16, the joint path's registers were measured to cost more than the halved row
+  // reads save).
+  constexpr bool kPairs = !MULTI && !AF3 && DMAX == 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b = blockIdx.y, a0 = blockIdx.x * g.QT;
   const int QT = g.QT, K = g.K, H = g.H, D = g.D, A = g.A, HD = H * D, DP = g.DP, P = g.P;
@@ -275,6 +281,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) 
   float *qs = beta + (AF3 ? ru4((size_t)H * slots) : 0);              // [QT][HD]
   float *kv = qs + ru4((size_t)QT * HD);                              // [kv_floats]
   __shared__ int s_lo, s_hi;
+  __shared__ int s_pairs_differ;                    // some pair (2p, 2p + 1) reads different rows
   __shared__ __align__(16) float s_wp[AF3 ? kPairMax * kAttnHeadsMax : 4];  // float4 rows
   __shared__ __align__(16) float s_wsum[AF3 ? kAttnHeadsMax : 4];
   if (tid == 0) {
@@ -320,7 +327,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) 
       kid[u] = in ? g.key_index[sbase + s] : -1;
       win[u] = in ? g.window[sbase + s] : 0;
     }
-    int jj[R];
+    int jj[R], raw[R];
     bool qu[R];
 #pragma unroll
     for (int u = 0; u < R; ++u) {
@@ -329,6 +336,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) 
       const int a = a0 + q;
       const int64_t j = kid[u];
       bool ok = s < vslots && win[u] != 0 && j >= 0 && j < A;
+      raw[u] = kPairs && s < vslots && j >= 0 && j < A ? (int)j : -1;
       if (ok && g.radius >= 0) ok = (j > a ? j - a : a - j) <= g.radius;
       jj[u] = ok ? (int)j : -1;
       qu[u] = s < vslots && g.usable[(int64_t)b * A + a] != 0;
@@ -337,7 +345,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) 
     for (int u = 0; u < R; ++u) {
       const int s = s0 + u * kAttnThreads;
       if (jj[u] >= 0 && (!qu[u] || g.usable[(int64_t)b * A + jj[u]] == 0)) jj[u] = -1;
-      if (s < slots) plan[s] = jj[u];
+      // plan: key id of a permitted slot; -2 - id for a slot that names a key in [0, A)
+      // but is not permitted (its row may still be read, with weight 0); -1 otherwise
+      if (s < slots) plan[s] = jj[u] >= 0 ? jj[u] : (kPairs && raw[u] >= 0 ? -2 - raw[u] : -1);
       if (jj[u] >= 0) {
         lo = min(lo, jj[u]);
         hi = max(hi, jj[u]);
@@ -385,6 +395,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) 
   if (span > 0 && !staged && tid == 0) atomicOr(g.status, 1u);
   const int nchunks = MULTI ? (K + kChunk - 1) / kChunk : 1;
 
+  // the staged row a slot reads: its key if permitted, else its named key when that is in
+  // the span, else the span's first row (weight 0 either way)
+  auto row_of = [&](int p) -> int {
+    const int r = p >= 0 ? p : -2 - p;
+    return p >= 0 || (p <= -2 && r >= klo && r <= khi) ? r : klo;
+  };
+  // 128-slot path: does every pair of queries (2p, 2p + 1) of the tile read the same row
+  // in every slot (blocked windows)? Then each pair is processed by one warp with every
+  // K/V row read once for both queries.
+  const bool fast = !MULTI && staged && K == kChunk;
+  if (kPairs && fast) {
+    if (tid == 0) s_pairs_differ = 0;
+    __syncthreads();
+    bool differ = false;
+    for (int q = 2 * warp; q + 1 < nq; q += 2 * kAttnWarps) {
+#pragma unroll
+      for (int i = 0; i < kSlotsPerLane; ++i) {
+        const int k = i * kWarp + lane;
+        differ = differ || row_of(plan[q * K + k]) != row_of(plan[(q + 1) * K + k]);
+      }
+    }
+    if (__any_sync(0xffffffffu, differ) && lane == 0) s_pairs_differ = 1;
+    __syncthreads();
+  }
+  const bool all_pairs = kPairs && fast && s_pairs_differ == 0;
+
   // ---------------- phase 2: head groups
   for (int h0 = 0; h0 < H; h0 += HG) {
     const int hg = H - h0 < HG ? H - h0 : HG;
@@ -423,107 +459,315 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) 
     }
     __syncthreads();
 
-    if (!MULTI && staged && K == kChunk) {
-      // ---- fast path: 128 slots, staged K/V, 32-bit shared addresses, no slot guards;
-      // the warps share the tile's (query, head) pairs evenly
-      const uint32_t rowb = (uint32_t)DP * 4u;
-      const uint32_t hmagic = hg > 1 ? (uint32_t)(0xFFFFFFFFu / (uint32_t)hg + 1u) : 0u;  // ceil(2^32/hg)
-      for (int pr = warp; pr < nq * hg; pr += kAttnWarps) {
-        const int q = hg > 1 ? (int)__umulhi((uint32_t)pr, hmagic) : pr;
-        const int hl = pr - q * hg, h = h0 + hl;
-        const int a = a0 + q;
-        const int64_t arow = (int64_t)b * A + a;
-        // the value-gate logits of this (query, head), fetched early
-        float gv[DMAX / DW];
-#pragma unroll
-        for (int part = 0; part < DMAX; part += DW) {
-          const int d = part + (lane & (DW - 1));
-          gv[part / DW] = lane < DW && d < D ? g.G[arow * HD + h * D + d] : 0.f;
-        }
-        int jr[kSlotsPerLane];
-#pragma unroll
-        for (int i = 0; i < kSlotsPerLane; ++i) jr[i] = plan[q * K + i * kWarp + lane];
-        const uint32_t kb = (uint32_t)__cvta_generic_to_shared(ks) + (uint32_t)(hl * span - klo) * rowb;
-        const uint32_t vb = (uint32_t)__cvta_generic_to_shared(vs) + (uint32_t)(hl * span - klo) * rowb;
-        const uint32_t qa = (uint32_t)__cvta_generic_to_shared(qs) + (uint32_t)(q * HD + h * D) * 4u;
-        f32x2 q2[DMAX / 2];
-        if (fullD) {
-#pragma unroll
-          for (int d = 0; d < DMAX; d += 4) {
-            const ulonglong2 x = lds128(qa + 4u * d);
-            q2[d / 2] = x.x;
-            q2[d / 2 + 1] = x.y;
+    if (fast) {
+      if constexpr (kPairs) {
+        // ---- fast path: 128 slots, staged K/V, 32-bit shared addresses, no slot guards.
+        // Work items are (query pair, head); a pair whose queries read the same rows is
+        // done jointly, otherwise its queries one after the other.
+        const uint32_t rowb = (uint32_t)DP * 4u;
+        const uint32_t kbase = (uint32_t)__cvta_generic_to_shared(ks);
+        const uint32_t vbase = (uint32_t)__cvta_generic_to_shared(vs);
+        const uint32_t qbase_s = (uint32_t)__cvta_generic_to_shared(qs);
+        const uint32_t bbase = AF3 ? (uint32_t)__cvta_generic_to_shared(beta) : 0u;
+
+        // q2 <- the query row (zero beyond D) from shared memory
+        auto load_q = [&](uint32_t qa, f32x2 (&q2)[DMAX / 2]) {
+          if (fullD) {
+  #pragma unroll
+            for (int d = 0; d < DMAX; d += 4) {
+              const ulonglong2 x = lds128(qa + 4u * d);
+              q2[d / 2] = x.x;
+              q2[d / 2 + 1] = x.y;
+            }
+          } else {
+  #pragma unroll
+            for (int d = 0; d < DMAX; d += 2)
+              q2[d / 2] = pack2(d < D ? lds32(qa + 4u * d) : 0.f, d + 1 < D ? lds32(qa + 4u * d + 4u) : 0.f);
           }
+        };
+        // ev <- exp2(l - max) of the permitted slots (0 elsewhere); returns 1/sum (0: none)
+        auto softmax = [&](float (&ev)[kSlotsPerLane], const int (&jr)[kSlotsPerLane]) -> float {
+          float mx = -INFINITY;
+  #pragma unroll
+          for (int i = 0; i < kSlotsPerLane; ++i) mx = fmaxf(mx, ev[i]);
+          mx = warp_max(mx);
+          float sum = 0.f;
+  #pragma unroll
+          for (int i = 0; i < kSlotsPerLane; ++i) {
+            ev[i] = jr[i] >= 0 ? exp2_approx(ev[i] - mx) : 0.f;
+            sum += ev[i];
+          }
+          sum = warp_sum(sum);
+          float inv = 0.f;
+          if (sum > 0.f) asm("rcp.approx.f32 %0, %1;" : "=f"(inv) : "f"(sum));
+          return inv;
+        };
+        // fold the lanes' partial outputs, gate, store (lane l ends with channel l)
+        auto finish = [&](f32x2 (&acc2)[DMAX / 2], const float (&gv)[DMAX / DW], bool has,
+                          int64_t obase) {
+          float acc[DMAX];
+  #pragma unroll
+          for (int d = 0; d < DMAX; d += 2) {
+            const float2 p2 = unpack2(acc2[d / 2]);
+            acc[d] = p2.x;
+            acc[d + 1] = p2.y;
+          }
+  #pragma unroll
+          for (int part = 0; part < DMAX; part += DW) {
+            float v[DW];
+  #pragma unroll
+            for (int i = 0; i < DW; ++i) v[i] = acc[part + i];
+            const float o = reduce_scatter<DW>(v, lane);
+            const int d = part + (lane & (DW - 1));
+            if (lane < DW && d < D) g.O[obase + d] = has ? o * sigmoid_fast(gv[part / DW]) : 0.f;
+          }
+        };
+        auto gates = [&](int64_t obase, float (&gv)[DMAX / DW]) {
+  #pragma unroll
+          for (int part = 0; part < DMAX; part += DW) {
+            const int d = part + (lane & (DW - 1));
+            gv[part / DW] = lane < DW && d < D ? g.G[obase + d] : 0.f;
+          }
+        };
+
+        // one query, one head
+        auto single = [&](int q, int hl) {
+          const int h = h0 + hl, a = a0 + q;
+          const int64_t obase = ((int64_t)b * A + a) * HD + h * D;
+          float gv[DMAX / DW];
+          gates(obase, gv);
+          int jr[kSlotsPerLane];
+          uint32_t ja[kSlotsPerLane];
+  #pragma unroll
+          for (int i = 0; i < kSlotsPerLane; ++i) {
+            jr[i] = plan[q * K + i * kWarp + lane];
+            ja[i] = (uint32_t)(jr[i] >= 0 ? jr[i] : klo) * rowb;
+          }
+          const uint32_t kb = kbase + (uint32_t)(hl * span - klo) * rowb;
+          const uint32_t vb = vbase + (uint32_t)(hl * span - klo) * rowb;
+          f32x2 q2[DMAX / 2];
+          load_q(qbase_s + (uint32_t)(q * HD + h * D) * 4u, q2);
+          const uint32_t ba = bbase + (uint32_t)(h * slots + q * K + lane) * 4u;
+          float ev[kSlotsPerLane];
+  #pragma unroll
+          for (int i = 0; i < kSlotsPerLane; ++i) {
+            f32x2 s0 = 0ull, s1 = 0ull;
+  #pragma unroll
+            for (int d = 0; d < DMAX; d += 4) {
+              const ulonglong2 k = lds128(kb + ja[i] + 4u * d);
+              s0 = ffma2(q2[d / 2], k.x, s0);
+              s1 = ffma2(q2[d / 2 + 1], k.y, s1);
+            }
+            const float2 x = unpack2(s0), y = unpack2(s1);
+            float l = ((x.x + x.y) + (y.x + y.y)) * g.scale_log2;
+            if (AF3) l = fmaf(lds32(ba + 128u * i), 1.4426950408889634f, l);
+            ev[i] = jr[i] >= 0 ? l : -INFINITY;
+          }
+          const float inv = softmax(ev, jr);
+          T *wout = (T *)g.attention + (((int64_t)b * H + h) * A + a) * K + lane;
+          f32x2 acc2[DMAX / 2];
+  #pragma unroll
+          for (int d = 0; d < DMAX / 2; ++d) acc2[d] = 0ull;
+  #pragma unroll
+          for (int i = 0; i < kSlotsPerLane; ++i) {
+            const float wgt = ev[i] * inv;
+            store_weight<T>(wout, i * kWarp, wgt);
+            const f32x2 w2 = pack2(wgt, wgt);
+  #pragma unroll
+            for (int d = 0; d < DMAX; d += 4) {
+              const ulonglong2 v = lds128(vb + ja[i] + 4u * d);
+              acc2[d / 2] = ffma2(w2, v.x, acc2[d / 2]);
+              acc2[d / 2 + 1] = ffma2(w2, v.y, acc2[d / 2 + 1]);
+            }
+          }
+          finish(acc2, gv, inv > 0.f, obase);
+        };
+
+        // queries q and q + 1, one head, every K/V row read once for both
+        auto joint = [&](int q, int hl) {
+          const int h = h0 + hl, a = a0 + q;
+          const int64_t obase = ((int64_t)b * A + a) * HD + h * D;
+          float gv0[DMAX / DW], gv1[DMAX / DW];
+          gates(obase, gv0);
+          gates(obase + HD, gv1);
+          int j0[kSlotsPerLane], j1[kSlotsPerLane];
+          uint32_t ja[kSlotsPerLane];
+  #pragma unroll
+          for (int i = 0; i < kSlotsPerLane; ++i) {
+            j0[i] = plan[q * K + i * kWarp + lane];
+            j1[i] = plan[(q + 1) * K + i * kWarp + lane];
+            ja[i] = (uint32_t)row_of(j0[i]) * rowb;
+          }
+          const uint32_t kb = kbase + (uint32_t)(hl * span - klo) * rowb;
+          const uint32_t vb = vbase + (uint32_t)(hl * span - klo) * rowb;
+          float e0[kSlotsPerLane], e1[kSlotsPerLane];
+          {
+            f32x2 qa[DMAX / 2], qb[DMAX / 2];
+            load_q(qbase_s + (uint32_t)(q * HD + h * D) * 4u, qa);
+            load_q(qbase_s + (uint32_t)((q + 1) * HD + h * D) * 4u, qb);
+            const uint32_t ba = bbase + (uint32_t)(h * slots + q * K + lane) * 4u;
+  #pragma unroll
+            for (int i = 0; i < kSlotsPerLane; ++i) {
+              f32x2 sa = 0ull, sb = 0ull, ta = 0ull, tb = 0ull;
+  #pragma unroll
+              for (int d = 0; d < DMAX; d += 4) {
+                const ulonglong2 k = lds128(kb + ja[i] + 4u * d);
+                sa = ffma2(qa[d / 2], k.x, sa);
+                ta = ffma2(qa[d / 2 + 1], k.y, ta);
+                sb = ffma2(qb[d / 2], k.x, sb);
+                tb = ffma2(qb[d / 2 + 1], k.y, tb);
+              }
+              const float2 xa = unpack2(sa), ya = unpack2(ta), xb = unpack2(sb), yb = unpack2(tb);
+              float la = ((xa.x + xa.y) + (ya.x + ya.y)) * g.scale_log2;
+              float lb = ((xb.x + xb.y) + (yb.x + yb.y)) * g.scale_log2;
+              if (AF3) {
+                la = fmaf(lds32(ba + 128u * i), 1.4426950408889634f, la);
+                lb = fmaf(lds32(ba + 128u * i + 4u * K), 1.4426950408889634f, lb);
+              }
+              e0[i] = j0[i] >= 0 ? la : -INFINITY;
+              e1[i] = j1[i] >= 0 ? lb : -INFINITY;
+            }
+          }
+          const float inv0 = softmax(e0, j0), inv1 = softmax(e1, j1);
+          T *w0 = (T *)g.attention + (((int64_t)b * H + h) * A + a) * K + lane;
+          f32x2 acca[DMAX / 2], accb[DMAX / 2];
+  #pragma unroll
+          for (int d = 0; d < DMAX / 2; ++d) acca[d] = accb[d] = 0ull;
+  #pragma unroll
+          for (int i = 0; i < kSlotsPerLane; ++i) {
+            const float wa = e0[i] * inv0, wb = e1[i] * inv1;
+            store_weight<T>(w0, i * kWarp, wa);
+            store_weight<T>(w0, K + i * kWarp, wb);
+            const f32x2 wa2 = pack2(wa, wa), wb2 = pack2(wb, wb);
+  #pragma unroll
+            for (int d = 0; d < DMAX; d += 4) {
+              const ulonglong2 v = lds128(vb + ja[i] + 4u * d);
+              acca[d / 2] = ffma2(wa2, v.x, acca[d / 2]);
+              acca[d / 2 + 1] = ffma2(wa2, v.y, acca[d / 2 + 1]);
+              accb[d / 2] = ffma2(wb2, v.x, accb[d / 2]);
+              accb[d / 2 + 1] = ffma2(wb2, v.y, accb[d / 2 + 1]);
+            }
+          }
+          finish(acca, gv0, inv0 > 0.f, obase);
+          finish(accb, gv1, inv1 > 0.f, obase + HD);
+        };
+
+        const uint32_t hmagic = hg > 1 ? (uint32_t)(0xFFFFFFFFu / (uint32_t)hg + 1u) : 0u;  // ceil(2^32/hg)
+        if (kPairs && all_pairs) {
+          for (int pr = warp; pr < (nq >> 1) * hg; pr += kAttnWarps) {
+            const int qp = hg > 1 ? (int)__umulhi((uint32_t)pr, hmagic) : pr;
+            joint(2 * qp, pr - qp * hg);
+          }
+          if (nq & 1)
+            for (int hl = warp; hl < hg; hl += kAttnWarps) single(nq - 1, hl);
         } else {
-#pragma unroll
-          for (int d = 0; d < DMAX; d += 2)
-            q2[d / 2] = pack2(d < D ? lds32(qa + 4u * d) : 0.f, d + 1 < D ? lds32(qa + 4u * d + 4u) : 0.f);
-        }
-        const uint32_t ba = AF3 ? (uint32_t)__cvta_generic_to_shared(beta) +
-                                      (uint32_t)(h * slots + q * K + lane) * 4u
-                                : 0u;
-        float ev[kSlotsPerLane];
-        uint32_t ja[kSlotsPerLane];
-        float mx = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < kSlotsPerLane; ++i) {
-          ja[i] = (uint32_t)(jr[i] >= 0 ? jr[i] : klo) * rowb;
-          f32x2 s0 = 0ull, s1 = 0ull;
-#pragma unroll
-          for (int d = 0; d < DMAX; d += 4) {
-            const ulonglong2 k = lds128(kb + ja[i] + 4u * d);
-            s0 = ffma2(q2[d / 2], k.x, s0);
-            s1 = ffma2(q2[d / 2 + 1], k.y, s1);
-          }
-          const float2 x = unpack2(s0), y = unpack2(s1);
-          float l = ((x.x + x.y) + (y.x + y.y)) * g.scale_log2;
-          if (AF3) l = fmaf(lds32(ba + 128u * i), 1.4426950408889634f, l);
-          ev[i] = jr[i] >= 0 ? l : -INFINITY;
-          mx = fmaxf(mx, ev[i]);
-        }
-        mx = warp_max(mx);
-        float sum = 0.f;
-#pragma unroll
-        for (int i = 0; i < kSlotsPerLane; ++i) {
-          ev[i] = jr[i] >= 0 ? exp2_approx(ev[i] - mx) : 0.f;
-          sum += ev[i];
-        }
-        sum = warp_sum(sum);
-        float inv = 0.f;
-        if (sum > 0.f) asm("rcp.approx.f32 %0, %1;" : "=f"(inv) : "f"(sum));
-        T *wout = (T *)g.attention + (((int64_t)b * H + h) * A + a) * K + lane;
-        f32x2 acc2[DMAX / 2];
-#pragma unroll
-        for (int d = 0; d < DMAX / 2; ++d) acc2[d] = 0ull;
-#pragma unroll
-        for (int i = 0; i < kSlotsPerLane; ++i) {
-          const float wgt = ev[i] * inv;
-          store_weight<T>(wout, i * kWarp, wgt);
-          const f32x2 w2 = pack2(wgt, wgt);
-#pragma unroll
-          for (int d = 0; d < DMAX; d += 4) {
-            const ulonglong2 v = lds128(vb + ja[i] + 4u * d);
-            acc2[d / 2] = ffma2(w2, v.x, acc2[d / 2]);
-            acc2[d / 2 + 1] = ffma2(w2, v.y, acc2[d / 2 + 1]);
+          for (int pr = warp; pr < nq * hg; pr += kAttnWarps) {
+            const int q = hg > 1 ? (int)__umulhi((uint32_t)pr, hmagic) : pr;
+            single(q, pr - q * hg);
           }
         }
-        const bool has = sum > 0.f;
-        float acc[DMAX];
-#pragma unroll
-        for (int d = 0; d < DMAX; d += 2) {
-          const float2 p2 = unpack2(acc2[d / 2]);
-          acc[d] = p2.x;
-          acc[d + 1] = p2.y;
-        }
-#pragma unroll
-        for (int part = 0; part < DMAX; part += DW) {
-          float v[DW];
-#pragma unroll
-          for (int i = 0; i < DW; ++i) v[i] = acc[part + i];
-          const float o = reduce_scatter<DW>(v, lane);
-          const int d = part + (lane & (DW - 1));
-          if (lane < DW && d < D)
-            g.O[arow * HD + h * D + d] = has ? o * sigmoid_fast(gv[part / DW]) : 0.f;
+      } else {
+        // ---- fast path: 128 slots, staged K/V, 32-bit shared addresses, no slot guards;
+        // the warps share the tile's (query, head) pairs evenly
+        const uint32_t rowb = (uint32_t)DP * 4u;
+        const uint32_t hmagic = hg > 1 ? (uint32_t)(0xFFFFFFFFu / (uint32_t)hg + 1u) : 0u;  // ceil(2^32/hg)
+        for (int pr = warp; pr < nq * hg; pr += kAttnWarps) {
+          const int q = hg > 1 ? (int)__umulhi((uint32_t)pr, hmagic) : pr;
+          const int hl = pr - q * hg, h = h0 + hl;
+          const int a = a0 + q;
+          const int64_t arow = (int64_t)b * A + a;
+          // the value-gate logits of this (query, head), fetched early
+          float gv[DMAX / DW];
+  #pragma unroll
+          for (int part = 0; part < DMAX; part += DW) {
+            const int d = part + (lane & (DW - 1));
+            gv[part / DW] = lane < DW && d < D ? g.G[arow * HD + h * D + d] : 0.f;
+          }
+          int jr[kSlotsPerLane];
+  #pragma unroll
+          for (int i = 0; i < kSlotsPerLane; ++i) jr[i] = plan[q * K + i * kWarp + lane];
+          const uint32_t kb = (uint32_t)__cvta_generic_to_shared(ks) + (uint32_t)(hl * span - klo) * rowb;
+          const uint32_t vb = (uint32_t)__cvta_generic_to_shared(vs) + (uint32_t)(hl * span - klo) * rowb;
+          const uint32_t qa = (uint32_t)__cvta_generic_to_shared(qs) + (uint32_t)(q * HD + h * D) * 4u;
+          f32x2 q2[DMAX / 2];
+          if (fullD) {
+  #pragma unroll
+            for (int d = 0; d < DMAX; d += 4) {
+              const ulonglong2 x = lds128(qa + 4u * d);
+              q2[d / 2] = x.x;
+              q2[d / 2 + 1] = x.y;
+            }
+          } else {
+  #pragma unroll
+            for (int d = 0; d < DMAX; d += 2)
+              q2[d / 2] = pack2(d < D ? lds32(qa + 4u * d) : 0.f, d + 1 < D ? lds32(qa + 4u * d + 4u) : 0.f);
+          }
+          const uint32_t ba = AF3 ? (uint32_t)__cvta_generic_to_shared(beta) +
+                                        (uint32_t)(h * slots + q * K + lane) * 4u
+                                  : 0u;
+          float ev[kSlotsPerLane];
+          uint32_t ja[kSlotsPerLane];
+          float mx = -INFINITY;
+  #pragma unroll
+          for (int i = 0; i < kSlotsPerLane; ++i) {
+            ja[i] = (uint32_t)(jr[i] >= 0 ? jr[i] : klo) * rowb;
+            f32x2 s0 = 0ull, s1 = 0ull;
+  #pragma unroll
+            for (int d = 0; d < DMAX; d += 4) {
+              const ulonglong2 k = lds128(kb + ja[i] + 4u * d);
+              s0 = ffma2(q2[d / 2], k.x, s0);
+              s1 = ffma2(q2[d / 2 + 1], k.y, s1);
+            }
+            const float2 x = unpack2(s0), y = unpack2(s1);
+            float l = ((x.x + x.y) + (y.x + y.y)) * g.scale_log2;
+            if (AF3) l = fmaf(lds32(ba + 128u * i), 1.4426950408889634f, l);
+            ev[i] = jr[i] >= 0 ? l : -INFINITY;
+            mx = fmaxf(mx, ev[i]);
+          }
+          mx = warp_max(mx);
+          float sum = 0.f;
+  #pragma unroll
+          for (int i = 0; i < kSlotsPerLane; ++i) {
+            ev[i] = jr[i] >= 0 ? exp2_approx(ev[i] - mx) : 0.f;
+            sum += ev[i];
+          }
+          sum = warp_sum(sum);
+          float inv = 0.f;
+          if (sum > 0.f) asm("rcp.approx.f32 %0, %1;" : "=f"(inv) : "f"(sum));
+          T *wout = (T *)g.attention + (((int64_t)b * H + h) * A + a) * K + lane;
+          f32x2 acc2[DMAX / 2];
+  #pragma unroll
+          for (int d = 0; d < DMAX / 2; ++d) acc2[d] = 0ull;
+  #pragma unroll
+          for (int i = 0; i < kSlotsPerLane; ++i) {
+            const float wgt = ev[i] * inv;
+            store_weight<T>(wout, i * kWarp, wgt);
+            const f32x2 w2 = pack2(wgt, wgt);
+  #pragma unroll
+            for (int d = 0; d < DMAX; d += 4) {
+              const ulonglong2 v = lds128(vb + ja[i] + 4u * d);
+              acc2[d / 2] = ffma2(w2, v.x, acc2[d / 2]);
+              acc2[d / 2 + 1] = ffma2(w2, v.y, acc2[d / 2 + 1]);
+            }
+          }
+          const bool has = sum > 0.f;
+          float acc[DMAX];
+  #pragma unroll
+          for (int d = 0; d < DMAX; d += 2) {
+            const float2 p2 = unpack2(acc2[d / 2]);
+            acc[d] = p2.x;
+            acc[d + 1] = p2.y;
+          }
+  #pragma unroll
+          for (int part = 0; part < DMAX; part += DW) {
+            float v[DW];
+  #pragma unroll
+            for (int i = 0; i < DW; ++i) v[i] = acc[part + i];
+            const float o = reduce_scatter<DW>(v, lane);
+            const int d = part + (lane & (DW - 1));
+            if (lane < DW && d < D)
+              g.O[arow * HD + h * D + d] = has ? o * sigmoid_fast(gv[part / DW]) : 0.f;
+          }
         }
       }
     } else {

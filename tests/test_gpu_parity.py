@@ -97,6 +97,18 @@ def test_esmfold2_head_widths(D, H):
     _check(workloads.make_inputs(spec, seed=10), f"D={D}")
 
 
+@pytest.mark.parametrize("dtype,A,radius,valid_p", [("float32", 900, 64, 1.0), ("float32", 700, 64, 0.9),
+                                                   ("bfloat16", 611, -1, 1.0)])
+def test_blocked_windows_with_shared_rows(dtype, A, radius, valid_p):
+    """128 slots in blocked windows: queries whose slots name the same key rows are
+    processed in pairs (each with its own mask), tiles whose pairs differ and odd tails
+    one query at a time."""
+    spec = workloads.tiny_spec("esmfold2", "encoder", dtype=dtype, A=A, T=120, K=128,
+                               keys=("blocked", 32, 48), radius=radius, dup_p=0.0, miss_p=0.0,
+                               window_p=1.0 if valid_p == 1.0 else 0.9, valid_p=valid_p)
+    _check(workloads.make_inputs(spec, seed=23), f"blocked A={A}")
+
+
 @pytest.mark.parametrize("eps", [1.0, 1e-3])
 def test_eps(eps):
     w = workloads.make_inputs(workloads.tiny_spec("af3", "decoder"), seed=11)
