@@ -492,7 +492,15 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   ra.token_proj = F(pl.o_tp);
   ra.usable = usable; ra.x = F(pl.o_x); ra.xstats = F(pl.o_xstats); ra.opc = F(pl.o_opc); ra.rawc = F(pl.o_rawc);
   ra.tok_first = first; ra.tok_last = last;
-  hk.launch((k_rows_prep<Elt>), row_blocks, 256, 0, st, ra);
+  {
+    const uintptr_t al = sizeof(Elt) == 4 ? 15 : 7;   // 4-element loads of atom / condition rows
+    const bool reg = C % 4 == 0 && S % 4 == 0 && C <= 256 && S <= 256 &&
+                     ((reinterpret_cast<uintptr_t>(in->atom.data) | reinterpret_cast<uintptr_t>(in->condition.data)) & al) == 0;
+    if (reg)
+      hk.launch((k_rows_prep_reg<Elt>), row_blocks, 256, 0, st, ra);
+    else
+      hk.launch((k_rows_prep<Elt>), row_blocks, 256, 0, st, ra);
+  }
   hk.mark(1, st);
 
   // ---- conditioning

@@ -10,19 +10,21 @@
 // gate logits and stored head-major (bullet 16).
 //
 // One CTA (512 threads, one per SM) owns QT consecutive queries of one batch element.
-//  Phase 0  the tile's Q rows are copied to shared memory with cp.async.
-//  Phase 1  one slot per thread per round (eight rounds in flight): key_index and
-//           window_mask are read once (coalesced), eligibility decided and the slot plan
-//           (key id or -1) written with the span [klo, khi] of the permitted ids; AF3:
-//           the pair bias of every permitted (slot, head) is computed from its pair row
-//           (16-byte loads, LayerNorm over P in one shifted pass) and kept in shared
-//           memory as float32 [head][slot].
+//  Phase 1  (may run while the projections finish) one slot per thread per round, eight
+//           rounds in flight: key_index and window_mask are read once (coalesced),
+//           eligibility decided and the slot plan written with the span [klo, khi] of
+//           the permitted ids; AF3: the pair bias of every permitted (slot, head) is
+//           computed from its pair row (16-byte loads, LayerNorm over P in one shifted
+//           pass) and kept in shared memory as float32 [head][slot].
+//  Phase 0  (after the wait for the projections) the tile's Q rows are copied to shared
+//           memory with cp.async.
 //  Phase 2  head groups: the K and V rows of the span for as many heads as fit are staged
-//           (float32, cp.async); each warp takes one query at a time, lanes over the slots
-//           (4 per lane per 128-slot chunk): logits, max, one exp2 per entry, sum, weights
-//           written once (bf16 rounded with integer ops), the weighted value sum per lane
-//           with packed f32x2 FMAs, folded across lanes by a butterfly reduce-scatter,
-//           value gate, store.
+//           (float32, cp.async); the warps share the (query, head) pairs, lanes over the
+//           slots (4 per lane per 128-slot chunk): logits, max, one exp2 per entry, sum,
+//           weights written once (bf16 rounded with integer ops), the weighted value sum
+//           per lane with packed f32x2 FMAs, folded across lanes by a butterfly
+//           reduce-scatter, value gate, store. Queries that read the same key rows may be
+//           processed two at a time (each row read once for both).
 // A tile whose span does not fit even one head reads K/V rows from global memory (L2)
 // instead and sets status bit 1; the results are the same.
 #pragma once
@@ -260,7 +262,10 @@ __device__ __forceinline__ float dot_q2_global(const f32x2 (&q2)[DMAX / 2], cons
 //                recomputes the logits to write the weights and accumulate the values.
 template <typename T, int DMAX, bool AF3, bool MULTI>
 __global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) {
-  pdl_enter();
+  // the slot plan and the pair bias read only the caller's inputs, the usable flags and
+  // the folded pair weights (all from kernels at least two places earlier), so they run
+  // before the wait for the projections; Q, K, V, G are read after it
+  pdl_launch_next();
   extern __shared__ __align__(16) float smem[];
   constexpr int DW = DMAX < 32 ? DMAX : 32;            // channels per reduce-scatter
   // Query pairs sharing their key rows are processed jointly in the 128-slot path; built
@@ -289,18 +294,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) 
     s_hi = -1;
   }
 
-  // ---------------- phase 0: the tile's Q rows -> shared (async), pair weights
-  const int64_t qbase = ((int64_t)b * A + a0) * HD;
-  if (vecD) {
-    for (int i = tid; i < nq * HD / 4; i += kAttnThreads) {
-      const uint32_t dst = (uint32_t)__cvta_generic_to_shared(qs + 4 * i);
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(g.Q + qbase + 4 * i)
-                   : "memory");
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  } else {
-    for (int i = tid; i < nq * HD; i += kAttnThreads) qs[i] = g.Q[qbase + i];
-  }
+  // ---------------- pair weights
   if (AF3) {
     for (int i = tid; i < P * H; i += kAttnThreads) s_wp[i] = g.w_pair[i];
     for (int h = tid; h < H; h += kAttnThreads) {
@@ -381,7 +375,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) 
       }
     }
   }
-  if (vecD) asm volatile("cp.async.wait_group 0;" ::: "memory");
+
+  // ---------------- phase 0 (after the wait for the projections): the tile's Q rows
+  pdl_wait();
+  const int64_t qbase = ((int64_t)b * A + a0) * HD;
+  if (vecD) {
+    for (int i = tid; i < nq * HD / 4; i += kAttnThreads) {
+      const uint32_t dst = (uint32_t)__cvta_generic_to_shared(qs + 4 * i);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(g.Q + qbase + 4 * i)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+  } else {
+    for (int i = tid; i < nq * HD; i += kAttnThreads) qs[i] = g.Q[qbase + i];
+  }
   __syncthreads();
   const int klo = s_lo, khi = s_hi;
   const int span = khi >= klo ? khi - klo + 1 : 0;

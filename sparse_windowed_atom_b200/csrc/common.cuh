@@ -15,10 +15,21 @@ constexpr int kWarp = 32;
 // is to wait until that predecessor grid has completed and its writes are visible
 // (before any global or tensor memory is touched, so chains of such kernels stay in
 // stream order); then it lets its own successor begin launching.
-__device__ __forceinline__ void pdl_enter() {
+__device__ __forceinline__ void pdl_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_launch_next() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+__device__ __forceinline__ void pdl_enter() {
+  pdl_wait();
+  pdl_launch_next();
+}
+// A kernel may read before pdl_wait() what the kernels two or more places earlier in the
+// stream wrote: its predecessor only launches it after passing its own pdl_wait(), so
+// those kernels have completed and their writes are visible. The caller's inputs count
+// as such (the first kernel of a pass waits for everything before it). Writes, and reads
+// of the immediate predecessor's results, come after pdl_wait().
 
 __device__ __forceinline__ float ldf(const float *p, int64_t i) { return p[i]; }
 __device__ __forceinline__ float ldf(const __nv_bfloat16 *p, int64_t i) {

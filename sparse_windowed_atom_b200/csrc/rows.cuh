@@ -94,6 +94,119 @@ __global__ void k_rows_prep(RowsArgs r) {
   }
 }
 
+// Four consecutive elements as floats (16-byte float32 / 8-byte bf16 loads).
+__device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p) {
+  const uint2 u = *reinterpret_cast<const uint2 *>(p);
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+}
+
+// k_rows_prep for C, S multiples of 4 up to 256 (aligned rows): the same arithmetic with
+// the row held in registers (lane l owns channels 4l..4l+3 and 128+4l..128+4l+3). Every
+// load of the caller's inputs is issued before the wait for the previous kernel, whose
+// results (the reset token ranges; the token projection in the decoder) are used after.
+template <typename T>
+__global__ void k_rows_prep_reg(RowsArgs r) {
+  pdl_launch_next();
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const bool live = row < r.B * r.A;
+  const int64_t b = live ? row / r.A : 0, a = live ? row % r.A : 0;
+  const bool use = live && atom_usable(r.valid, r.att, r.token_valid, b, a, r.A, r.T);
+  const int64_t t = use ? r.att[row] : 0;
+  const int C = (int)r.C, S = (int)r.S;
+  float xv[8], cv[8];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int c = h * 128 + 4 * lane;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
+    if (use && c < C) x = ld4((const T *)r.atom + row * C + c);
+    if (use && c < S) y = ld4((const T *)r.condition + row * S + c);
+    xv[4 * h] = x.x; xv[4 * h + 1] = x.y; xv[4 * h + 2] = x.z; xv[4 * h + 3] = x.w;
+    cv[4 * h] = y.x; cv[4 * h + 1] = y.y; cv[4 * h + 2] = y.z; cv[4 * h + 3] = y.w;
+  }
+  pdl_wait();
+  if (!live) return;
+  if (lane == 0) {
+    r.usable[row] = use ? 1 : 0;
+    if (use && r.encoder) {
+      atomicMin(r.tok_first + b * r.T + t, (int)a);
+      atomicMax(r.tok_last + b * r.T + t, (int)a);
+    }
+  }
+  // x = atom, or skip + gathered token projection (bullet 3); its row statistics
+  // (AF3 population LayerNorm, bullet 7; ESMFold2 RMS, bullet 11)
+  float s1 = 0.f;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int c = h * 128 + 4 * lane;
+    if (c < C) {
+      if (r.decoder && use) {
+        const float4 tp = ld4(r.token_proj + (b * r.T + t) * C + c);
+        xv[4 * h] += tp.x; xv[4 * h + 1] += tp.y; xv[4 * h + 2] += tp.z; xv[4 * h + 3] += tp.w;
+      }
+      *reinterpret_cast<float4 *>(r.x + row * C + c) =
+          make_float4(xv[4 * h], xv[4 * h + 1], xv[4 * h + 2], xv[4 * h + 3]);
+      s1 += (xv[4 * h] + xv[4 * h + 1]) + (xv[4 * h + 2] + xv[4 * h + 3]);
+    }
+  }
+  const float mean = r.af3 ? warp_sum(s1) / (float)C : 0.f;
+  float s2 = 0.f;
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+    if (h * 128 + 4 * lane < C)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float d = xv[4 * h + e] - mean;
+        s2 = fmaf(d, d, s2);
+      }
+  s2 = warp_sum(s2);
+  if (lane == 0) {
+    r.xstats[2 * row] = mean;
+    r.xstats[2 * row + 1] = 1.f / sqrtf(s2 / (float)C + r.eps);
+  }
+  if (r.af3) {
+    // population LayerNorm of the condition, eps inside the root (bullet 7)
+    float sc = 0.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      if (h * 128 + 4 * lane < S) sc += (cv[4 * h] + cv[4 * h + 1]) + (cv[4 * h + 2] + cv[4 * h + 3]);
+    const float cm = warp_sum(sc) / (float)S;
+    float q = 0.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      if (h * 128 + 4 * lane < S)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float d = cv[4 * h + e] - cm;
+          q = fmaf(d, d, q);
+        }
+    const float rstd = 1.f / sqrtf(warp_sum(q) / (float)S + r.eps);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = h * 128 + 4 * lane;
+      if (c < S) {
+        *reinterpret_cast<float4 *>(r.rawc + row * S + c) =
+            make_float4(cv[4 * h], cv[4 * h + 1], cv[4 * h + 2], cv[4 * h + 3]);
+        *reinterpret_cast<float4 *>(r.opc + row * S + c) =
+            make_float4((cv[4 * h] - cm) * rstd, (cv[4 * h + 1] - cm) * rstd,
+                        (cv[4 * h + 2] - cm) * rstd, (cv[4 * h + 3] - cm) * rstd);
+      }
+    }
+  } else {
+    // SiLU(condition) feeds w_mod (bullet 10)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = h * 128 + 4 * lane;
+      if (c < S)
+        *reinterpret_cast<float4 *>(r.opc + row * S + c) =
+            make_float4(siluf_(cv[4 * h]), siluf_(cv[4 * h + 1]), siluf_(cv[4 * h + 2]),
+                        siluf_(cv[4 * h + 3]));
+    }
+  }
+}
+
 // ------------------------------------------------------------------ attention inputs
 struct FeatArgs {
   int64_t rows, C;

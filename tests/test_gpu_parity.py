@@ -109,6 +109,29 @@ def test_blocked_windows_with_shared_rows(dtype, A, radius, valid_p):
     _check(workloads.make_inputs(spec, seed=23), f"blocked A={A}")
 
 
+@pytest.mark.parametrize("style,stage", [("af3", "encoder"), ("esmfold2", "decoder")])
+def test_unaligned_atom_and_condition_rows(style, stage):
+    """atom and condition views that start one element into their storage (dense, but not
+    16-byte aligned) take the general row-preparation kernel; same results."""
+    w = workloads.make_inputs(workloads.tiny_spec(style, stage), seed=29)
+    ref = run_oracle(w)
+    act, prm, msk, st = to_torch(w)
+    for k in ("atom", "condition"):
+        v = act[k]
+        buf = torch.empty(v.numel() + 1, dtype=v.dtype, device=v.device)
+        view = buf[1:].view(v.shape)
+        view.copy_(v)
+        assert view.data_ptr() % 16 != 0
+        act[k] = view
+    spec = w["spec"]
+    out = atomenc.windowed_atom_attention(act, prm, msk, st, eps=spec.eps, style=style,
+                                          stage=stage, radius=spec.radius)
+    torch.cuda.synchronize()
+    got = {k: v.float().cpu().numpy().astype(np.float64) for k, v in out.items()}
+    compare(got, ref, spec.dtype, "unaligned rows")
+    exact_zero_pattern(got, ref)
+
+
 @pytest.mark.parametrize("eps", [1.0, 1e-3])
 def test_eps(eps):
     w = workloads.make_inputs(workloads.tiny_spec("af3", "decoder"), seed=11)
