@@ -27,7 +27,8 @@
 
 namespace atomenc {
 
-constexpr int kTransThreads = 192;
+constexpr int kTransEpiWarps = 8;                       // two per TMEM lane quadrant
+constexpr int kTransThreads = (kTransEpiWarps + 2) * 32;   // + MMA issuer + weight loader
 
 struct TransArgs {
   int64_t R;
@@ -128,12 +129,12 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
       umma::mbar_init(full + s, 1);
       umma::mbar_init(empty + s, 1);
     }
-    umma::mbar_init(a_ready, 4);          // one arrival per epilogue warp
+    umma::mbar_init(a_ready, kTransEpiWarps);          // one arrival per epilogue warp
     umma::mbar_init(acc0_done, 1);
-    umma::mbar_init(z_ready, 4);
+    umma::mbar_init(z_ready, kTransEpiWarps);
     for (int b = 0; b < 2; ++b) {
       umma::mbar_init(acc1_full + b, 1);
-      umma::mbar_init(h_ready + b, 4);
+      umma::mbar_init(h_ready + b, kTransEpiWarps);
       umma::mbar_init(h_free + b, 1);
     }
     umma::mbar_init(acc2_done, 1);
@@ -148,46 +149,52 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
   const uint32_t acc0 = tmem, acc1 = tmem + 128, acc2 = tmem + 384;   // acc1: two 128-col buffers
   bool ok = true;
 
-  if (warp < 4) {
-    const int rl = warp * 32 + lane;
+  if (warp < kTransEpiWarps) {
+    // warp w: TMEM lane quadrant w % 4 (rows 32 (w % 4) ..), column half w / 4 of every
+    // 128-column matrix
+    const int qd = warp & 3, hf = warp >> 2, cb = hf * 64;
+    const int rl = qd * 32 + lane;
     const int64_t r = m0 + rl;
     const bool rok = r < t.R;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
+    auto epi_sync = []() { asm volatile("bar.sync 1, %0;" ::"n"(kTransEpiWarps * 32) : "memory"); };
 
-    // ---- o rows -> first operand (8 lanes per row segment, coalesced)
+    // ---- o rows -> first operand (warp w converts rows 16w..16w+15; 8 lanes per row
+    // segment, coalesced)
     for (int kc = 0; kc < nkc_out; ++kc) {
-      float v[8][8];
+      float v[4][8];
 #pragma unroll
-      for (int it = 0; it < 8; ++it)
-        load8_t(t.O, t.HD, t.R, t.HD, m0 + warp * 32 + it * 4 + (lane >> 3),
+      for (int it = 0; it < 4; ++it)
+        load8_t(t.O, t.HD, t.R, t.HD, m0 + warp * 16 + it * 4 + (lane >> 3),
                 (int64_t)kc * kUmmaBK + (lane & 7) * 8, v[it]);
 #pragma unroll
-      for (int it = 0; it < 8; ++it)
-        put8<SPLIT>(sA + kc * P * BLK, warp * 32 + it * 4 + (lane >> 3), (lane & 7) * 8, v[it]);
+      for (int it = 0; it < 4; ++it)
+        put8<SPLIT>(sA + kc * P * BLK, warp * 16 + it * 4 + (lane >> 3), (lane & 7) * 8, v[it]);
     }
     umma::fence_async_smem();
     __syncwarp();
     if (lane == 0) umma::mbar_arrive(a_ready);
 
-    // ---- x' = x + g0 * acc0, kept in TMEM in place of acc0; statistics of x' (one
-    // shifted pass); then z -> operand
+    // ---- x' = x + g0 * acc0 on this warp's 64 columns, kept in TMEM in place of acc0;
+    // partial statistics (shifted by the half's first x'), combined with the other half
+    // through shared memory; then z -> operand
     float xv[32], gv[32];                       // chunk 0 fetched before the wait
-    row32(t.x, C, r, rok, 0, xv);
-    row32(t.g0, t.g_ld, r, rok, 0, gv);
+    row32(t.x, C, r, rok, cb, xv);
+    row32(t.g0, t.g_ld, r, rok, cb, gv);
     if (ok) ok = umma::mbar_wait_warp(acc0_done, 0, abort_flag, lane);
     umma::tc_fence_after();
     float shift = 0.f, s1 = 0.f, s2 = 0.f;
 #pragma unroll 1
-    for (int c0 = 0; c0 < C; c0 += 32) {
+    for (int c0 = cb; c0 < cb + 64; c0 += 32) {
       float a[32];
-      if (c0 > 0) {
+      if (c0 > cb) {
         row32(t.x, C, r, rok, c0, xv);
         row32(t.g0, t.g_ld, r, rok, c0, gv);
       }
       umma::tmem_ld32(tl + c0, a);
 #pragma unroll
       for (int i = 0; i < 32; ++i) a[i] = fmaf(gv[i], a[i], xv[i]);
-      if (c0 == 0) shift = t.rms ? 0.f : a[0];
+      if (c0 == cb) shift = t.rms ? 0.f : a[0];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float d = a[i] - shift;
@@ -197,12 +204,26 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
       umma::tmem_st32(tl + c0, a);
     }
     umma::tmem_wait_st();
-    const float m = s1 / (float)C;
-    const float mean = t.rms ? 0.f : shift + m;
-    const float var = t.rms ? s2 / (float)C : fmaxf(s2 / (float)C - m * m, 0.f);
-    const float rstd = 1.f / sqrtf(var + t.eps);
+    // the SwiGLU operand buffer is free until the first SwiGLU chunk: partials go there
+    float *part = reinterpret_cast<float *>(sH);      // [2][128][3]
+    part[(hf * 128 + rl) * 3 + 0] = s1;
+    part[(hf * 128 + rl) * 3 + 1] = s2;
+    part[(hf * 128 + rl) * 3 + 2] = shift;
+    epi_sync();
+    float mean = 0.f, ssd = 0.f;                // sum of squared deviations from mean
+    {
+      const float* p0 = part + rl * 3, *p1 = part + (128 + rl) * 3;
+      if (t.rms) {
+        ssd = p0[1] + p1[1];
+      } else {
+        mean = ((p0[0] + 64.f * p0[2]) + (p1[0] + 64.f * p1[2])) / (float)C;
+        const float d0 = p0[2] - mean, d1 = p1[2] - mean;
+        ssd = (p0[1] + 2.f * d0 * p0[0] + 64.f * d0 * d0) + (p1[1] + 2.f * d1 * p1[0] + 64.f * d1 * d1);
+      }
+    }
+    const float rstd = 1.f / sqrtf(fmaxf(ssd, 0.f) / (float)C + t.eps);
 #pragma unroll 1
-    for (int c0 = 0; c0 < C; c0 += 32) {
+    for (int c0 = cb; c0 < cb + 64; c0 += 32) {
       float a[32], sv[32], hv[32];
       row32(t.sc, t.cond_ld, r, rok, c0, sv);
       row32(t.sh, t.cond_ld, r, rok, c0, hv);
@@ -226,14 +247,14 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
     if (lane == 0) umma::mbar_arrive(z_ready);
 
     // ---- SwiGLU, one 64-wide chunk i of the hidden width at a time: TMEM buffer i % 2
-    // (128 interleaved gate/up columns) -> shared operand buffer i % 2
+    // (128 interleaved gate/up columns, this warp's 64) -> shared operand buffer i % 2
     for (int ch = 0; ch < nC; ++ch) {
       const int bf = ch & 1;
       if (ok) ok = umma::mbar_wait_warp(acc1_full + bf, (ch >> 1) & 1, abort_flag, lane);
       if (ch >= 2 && ok) ok = umma::mbar_wait_warp(h_free + bf, ((ch - 2) >> 1) & 1, abort_flag, lane);
       umma::tc_fence_after();
 #pragma unroll 1
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int c0 = cb; c0 < cb + 64; c0 += 32) {
         float a[32];
         umma::tmem_ld32(tl + 128 + bf * 128 + c0, a);
 #pragma unroll
@@ -255,15 +276,15 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
 
     // ---- hidden = usable * (x' + g1 * acc2)
     float g1v[32];                              // chunk 0 fetched before the wait
-    row32(t.g1, t.g_ld, r, rok, 0, g1v);
+    row32(t.g1, t.g_ld, r, rok, cb, g1v);
     const bool use_row = rok && t.usable[r] != 0;
     if (ok) ok = umma::mbar_wait_warp(acc2_done, 0, abort_flag, lane);
     umma::tc_fence_after();
     const bool use = ok && use_row;
 #pragma unroll 1
-    for (int c0 = 0; c0 < C; c0 += 32) {
+    for (int c0 = cb; c0 < cb + 64; c0 += 32) {
       float a[32], f[32];
-      if (c0 > 0) row32(t.g1, t.g_ld, r, rok, c0, g1v);
+      if (c0 > cb) row32(t.g1, t.g_ld, r, rok, c0, g1v);
       umma::tmem_ld32(tl + c0, a);
       umma::tmem_ld32(tl + 384 + c0, f);
       if (rok) {
@@ -278,7 +299,7 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
         }
       }
     }
-  } else if (warp == 4) {
+  } else if (warp == kTransEpiWarps) {
     if (lane == 0) {
       int i = 0;
       auto mma_block = [&](uint32_t dtm, const uint8_t *a_blk, bool first) {
