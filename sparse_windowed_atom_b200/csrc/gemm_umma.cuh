@@ -82,24 +82,20 @@ __device__ __forceinline__ void load8_t<__nv_bfloat16>(const __nv_bfloat16 *A, i
 // conditioning rows.
 template <typename TA>
 struct ProdPlain {
-  static constexpr bool kStats = false;
   const TA *A;
   int64_t lda, M, K;
-  __device__ void row_stats(int64_t, int, float *) const {}
-  __device__ void load8(int64_t r, int, int64_t k, const float *, float (&v)[8]) const {
+  __device__ void load8(int64_t r, int64_t k, float (&v)[8]) const {
     load8_t(A, lda, M, K, r, k, v);
   }
 };
 
 struct ProdNorm {
-  static constexpr bool kStats = false;
   const float *x;        // [M, K]
   const float *stats;    // [M, 2]: mean (0 for RMS) and rstd of each row of x
   const float *cond;     // rows of cond_ld floats
   int64_t M, K, cond_ld, sc_off, sh_off;
   int plus1;
-  __device__ void row_stats(int64_t, int, float *) const {}
-  __device__ void load8(int64_t r, int, int64_t k, const float *, float (&v)[8]) const {
+  __device__ void load8(int64_t r, int64_t k, float (&v)[8]) const {
     float xv[8], sc[8], sh[8];
     load8_t(x, K, M, K, r, k, xv);
     load8_t(cond + sc_off, cond_ld, M, K, r, k, sc);
@@ -230,24 +226,26 @@ __global__ void __launch_bounds__(kUmmaThreads)
 // ----------------------------------------------------------------------------------
 // Row-block GEMM: one CTA owns 128 rows of A (all of K resident in shared memory,
 // converted once) and a contiguous range of 128-column output tiles. Warp roles:
-//   warps 0-3  convert A, then run the epilogue of each tile (warp w owns TMEM lanes
-//              32w..32w+31); the accumulator chunk is transposed through a per-warp
-//              shared tile so that the epilogue functor sees 8 lanes per 128-byte row
-//              segment (coalesced global reads and writes);
-//   warp 4     lane 0 issues the MMAs: two 128-column TMEM accumulators, so the MMAs of
+//   warps 0-7  convert A (warp w: rows 16w..16w+15), then run the epilogue of each tile
+//              (warp w: TMEM lanes 32 (w % 4).. and the column half w / 4); the
+//              accumulator chunk is transposed through a per-warp shared tile so that
+//              the epilogue functor sees 8 lanes per 128-byte row segment (coalesced
+//              global reads and writes);
+//   warp 8     lane 0 issues the MMAs: two 128-column TMEM accumulators, so the MMAs of
 //              tile t+1 run while the epilogue drains tile t;
-//   warp 5     lane 0 streams the packed weight blocks through a ring of NSLOT shared
+//   warp 9     lane 0 streams the packed weight blocks through a ring of NSLOT shared
 //              buffers with bulk async copies.
 // Requires K <= kRowsKMax; every wait is bounded (status bit 4 on timeout).
-constexpr int kRowsThreads = 192;
+constexpr int kRowsEpiWarps = 8;                        // two per TMEM lane quadrant
+constexpr int kRowsThreads = (kRowsEpiWarps + 2) * 32;  // + MMA issuer + weight loader
 constexpr int kRowsKMax = 256;
 
-__host__ __device__ constexpr int rows_slots(bool split) { return split ? 2 : 3; }
+__host__ __device__ constexpr int rows_slots(bool) { return 2; }   // keeps two bf16 CTAs per SM
 __host__ __device__ inline size_t rows_smem_bytes(int64_t K, bool split) {
   const int parts = split ? 2 : 1;
   const size_t nkc = (size_t)((K + kUmmaBK - 1) / kUmmaBK);
-  return 1024 + (nkc + rows_slots(split)) * parts * kUmmaBlockBytes + 4 * 32 * 33 * 4 + 256 +
-         128 * 2 * 4;
+  return 1024 + (nkc + rows_slots(split)) * parts * kUmmaBlockBytes +
+         (size_t)kRowsEpiWarps * 32 * 33 * 4 + 256;
 }
 
 template <class Prod, bool SPLIT, class Epi>
@@ -264,12 +262,11 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
   const int nkc = (int)((K + kUmmaBK - 1) / kUmmaBK);
   uint8_t *sA = sm;                                       // [nkc][PARTS] blocks
   uint8_t *sR = sA + (size_t)nkc * PARTS * BLK;           // [NSLOT][PARTS] blocks
-  float *sT = reinterpret_cast<float *>(sR + (size_t)NSLOT * PARTS * BLK);   // [4][32][33]
-  uint64_t *full = reinterpret_cast<uint64_t *>(sT + 4 * 32 * 33);
+  float *sT = reinterpret_cast<float *>(sR + (size_t)NSLOT * PARTS * BLK);   // [warps][32][33]
+  uint64_t *full = reinterpret_cast<uint64_t *>(sT + kRowsEpiWarps * 32 * 33);
   uint64_t *empty = full + NSLOT, *accf = empty + NSLOT, *acce = accf + 2, *aready = acce + 2;
   uint32_t *tslot = reinterpret_cast<uint32_t *>(aready + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
-  float *sStats = reinterpret_cast<float *>(tslot + 4);                   // [128][2]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nt = (int)((N + kUmmaBN - 1) / kUmmaBN);
@@ -285,9 +282,9 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       umma::mbar_init(accf + b, 1);
-      umma::mbar_init(acce + b, 4);        // one arrival per epilogue warp
+      umma::mbar_init(acce + b, kRowsEpiWarps);        // one arrival per epilogue warp
     }
-    umma::mbar_init(aready, 4);
+    umma::mbar_init(aready, kRowsEpiWarps);
     *abort_flag = 0;
     umma::fence_mbar_init();
   }
@@ -298,24 +295,20 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
   const uint32_t tmem = *tslot;
   bool ok = true;
 
-  if (warp < 4) {
-    // ---- A: rows 32w..32w+31 of the tile, every k chunk, bf16 (hi[, lo]) swizzled;
-    // the 8 row-segments of a chunk are loaded before any is converted (8 loads in flight)
-    if (Prod::kStats) {
-      prod.row_stats(m0 + warp * 32, lane, sStats + warp * 64);
-      __syncwarp();
-    }
+  if (warp < kRowsEpiWarps) {
+    // ---- A: rows 16w..16w+15 of the tile, every k chunk, bf16 (hi[, lo]) swizzled;
+    // the 4 row-segments of a chunk are loaded before any is converted
     for (int c = 0; c < nkc; ++c) {
       uint8_t *a_c = sA + (size_t)c * PARTS * BLK;
-      float v[8][8];
+      float v[4][8];
 #pragma unroll
-      for (int it = 0; it < 8; ++it) {
-        const int rl = warp * 32 + it * 4 + (lane >> 3);
-        prod.load8(m0 + rl, rl, (int64_t)c * kUmmaBK + (lane & 7) * 8, sStats, v[it]);
+      for (int it = 0; it < 4; ++it) {
+        const int rl = warp * 16 + it * 4 + (lane >> 3);
+        prod.load8(m0 + rl, (int64_t)c * kUmmaBK + (lane & 7) * 8, v[it]);
       }
 #pragma unroll
-      for (int it = 0; it < 8; ++it) {
-        const int r = warp * 32 + it * 4 + (lane >> 3), seg = lane & 7;
+      for (int it = 0; it < 4; ++it) {
+        const int r = warp * 16 + it * 4 + (lane >> 3), seg = lane & 7;
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -337,16 +330,18 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
     __syncwarp();
     if (lane == 0) umma::mbar_arrive(aready);
 
-    // ---- epilogue of each output tile
+    // ---- epilogue of each output tile: warp w reads TMEM lane quadrant w % 4 and the
+    // column half w / 4 of the tile
+    const int qd = warp & 3, cb = (warp >> 2) * (kUmmaBN / 2);
     float *T = sT + warp * 32 * 33;
-    const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t tlane = tmem + ((uint32_t)(qd * 32) << 16);
     for (int tl = 0; tl < ntl; ++tl) {
       const int buf = tl & 1;
       if (ok) ok = umma::mbar_wait_warp(accf + buf, (tl >> 1) & 1, abort_flag, lane);
       umma::tc_fence_after();
       const int64_t n0 = (int64_t)(t_begin + tl) * kUmmaBN;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kUmmaBN; c0 += 32) {
+      for (int c0 = cb; c0 < cb + kUmmaBN / 2; c0 += 32) {
         if (n0 + c0 >= N) break;
         float v[32];
         umma::tmem_ld32(tlane + buf * kUmmaBN + c0, v);
@@ -356,7 +351,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
 #pragma unroll 2
         for (int i = 0; i < 8; ++i) {
           const int rl = i * 4 + (lane >> 3), q = lane & 7;
-          const int64_t row = m0 + warp * 32 + rl, col = n0 + c0 + 4 * q;
+          const int64_t row = m0 + qd * 32 + rl, col = n0 + c0 + 4 * q;
           if (ok && row < M && col < N) {
             const float x[4] = {T[rl * 33 + 4 * q], T[rl * 33 + 4 * q + 1], T[rl * 33 + 4 * q + 2],
                                 T[rl * 33 + 4 * q + 3]};
@@ -369,7 +364,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
       __syncwarp();
       if (lane == 0) umma::mbar_arrive(acce + buf);
     }
-  } else if (warp == 4) {
+  } else if (warp == kRowsEpiWarps) {
     if (lane == 0) {
       // ---- MMA issue
       ok = umma::mbar_wait(aready, 0, abort_flag);

@@ -12,10 +12,13 @@
 // w_ff_out (128 columns), 512 TMEM columns in all; x', z and the SwiGLU intermediate
 // never go to HBM.
 //
-// Warp roles: warps 0-3 convert the o rows into the first operand, then work one output
-// row per thread (TMEM lanes 32w..32w+31): residual x' (stored back into TMEM over the
-// out-projection accumulator), row statistics and z (written as the next operand),
-// SiLU(gate) * up per chunk (written as the last operand), and the final gated residual; warp 4 lane 0 issues the MMAs; warp 5 lane 0 streams the packed weight
+// Warp roles: warps 0-7 convert the o rows into the first operand, then work one output
+// row per thread (warp w: TMEM lanes 32 (w % 4).. and the column half w / 4 of every
+// 128-column matrix): residual x' (stored back into TMEM over the out-projection
+// accumulator), row statistics (the two halves combined through shared memory) and z
+// (written as the next operand), SiLU(gate) * up per chunk (written as the last
+// operand), and the final gated residual; warp 8 lane 0 issues the MMAs; warp 9 lane 0
+// streams the packed weight
 // blocks through a ring of bulk async copies in the order the MMAs consume them. Every
 // wait is bounded (status bit 4 on timeout). Needs C == 128, H*D in {64, 128}, M a
 // multiple of 128.
