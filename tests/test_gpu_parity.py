@@ -91,7 +91,7 @@ def test_af3_head_widths(D, H):
     _check(workloads.make_inputs(spec, seed=9), f"D={D}")
 
 
-@pytest.mark.parametrize("D,H", [(2, 4), (16, 8), (64, 2)])
+@pytest.mark.parametrize("D,H", [(2, 4), (8, 4), (16, 8), (64, 2)])
 def test_esmfold2_head_widths(D, H):
     spec = workloads.tiny_spec("esmfold2", "decoder", D=D, H=H, K=150)
     _check(workloads.make_inputs(spec, seed=10), f"D={D}")
