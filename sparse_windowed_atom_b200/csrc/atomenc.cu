@@ -68,11 +68,11 @@ float bf16_round_host(float f) {
 
 struct Plan {
   int style = 0, stage = 0, fdt = 0;
-  bool af3 = false, enc = false, fuse_tail = false;
+  bool af3 = false, enc = false, fuse_tail = false, tail_pair = false;
   Dims d;
   // workspace layout (byte offsets)
   size_t o_status, o_usable, o_xstats, o_first, o_last, o_tp, o_x, o_opc, o_rawc, o_cond, o_gate, o_feat,
-      o_q, o_k, o_v, o_g, o_o, o_xp, o_z, o_h, o_hid, o_pool;
+      o_q, o_k, o_v, o_g, o_o, o_xp, o_z, o_h, o_hid, o_pool, o_xfer, o_xflag;
   size_t o_wread, o_bscale, o_brg, o_bq, o_wpair, o_rscale, o_rbias;
   // tensor-core images of the weight panels (bf16, hi[/lo])
   size_t k_cond, k_gate, k_qkv0, k_qkv1, k_out, k_ff1, k_ff2, k_pool, k_tok;
@@ -226,6 +226,12 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   // the fused tail (out-projection .. hidden in one kernel) keeps x', z and the SwiGLU
   // intermediate on chip
   pl.fuse_tail = C == 128 && (HD == 64 || HD == 128) && M % 128 == 0;
+  // few row blocks: two CTAs per row block, each on half of the SwiGLU width (all CTAs
+  // fit on the GPU at once, one per SM)
+  const int64_t nrb = (R + kUmmaBM - 1) / kUmmaBM;
+  pl.tail_pair = pl.fuse_tail && 2 * nrb <= 148;
+  pl.o_xfer = take(cur, pl.tail_pair ? nrb * 2 * 128 * 64 * 4 : 0);
+  pl.o_xflag = take(cur, pl.tail_pair ? nrb * 2 * 4 : 0);
   pl.o_xp = take(cur, pl.fuse_tail ? 0 : R * C * 4);
   pl.o_z = take(cur, pl.fuse_tail ? 0 : R * C * 4);
   pl.o_h = take(cur, pl.fuse_tail ? 0 : R * M * 4);
@@ -424,6 +430,8 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     copy(p->w_readout, 0, C, 3, pl.o_wread, 3, 0, nullptr, 0);
   }
   wj.fill[wj.nfill++] = FillJob{reinterpret_cast<int *>(status), 1, 0, 0};
+  if (pl.tail_pair)
+    wj.fill[wj.nfill++] = FillJob{reinterpret_cast<int *>(ws + pl.o_xflag), 2 * ((R + kUmmaBM - 1) / kUmmaBM), 0, 0};
   if (pl.enc) {
     wj.fill[wj.nfill++] = FillJob{first, B * T, INT_MAX, 0};
     wj.fill[wj.nfill++] = FillJob{last, B * T, -1, 0};
@@ -600,15 +608,17 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     ta.usable = usable;
     ta.w_out = ws + pl.k_out; ta.w_ff1 = ws + pl.k_ff1; ta.w_ff2 = ws + pl.k_ff2;
     ta.hid32 = split ? nullptr : F(pl.o_hid); ta.hidden = out->hidden.data; ta.status = status;
+    ta.xfer = F(pl.o_xfer); ta.xflag = reinterpret_cast<int *>(ws + pl.o_xflag);
     const size_t smem = trans_smem_bytes(split);
-    const dim3 grid((unsigned)((R + kUmmaBM - 1) / kUmmaBM));
-    if (split) {
-      smem_limit(k_transition<true, Elt>, smem);
-      hk.launch((k_transition<true, Elt>), grid, kTransThreads, smem, st, ta);
-    } else {
-      smem_limit(k_transition<false, Elt>, smem);
-      hk.launch((k_transition<false, Elt>), grid, kTransThreads, smem, st, ta);
-    }
+    const dim3 grid((unsigned)(((R + kUmmaBM - 1) / kUmmaBM) * (pl.tail_pair ? 2 : 1)));
+    auto go = [&](auto kern) {
+      smem_limit(kern, smem);
+      hk.launch(kern, grid, kTransThreads, smem, st, ta);
+    };
+    if (split)
+      pl.tail_pair ? go(k_transition<true, Elt, true>) : go(k_transition<true, Elt, false>);
+    else
+      pl.tail_pair ? go(k_transition<false, Elt, true>) : go(k_transition<false, Elt, false>);
   } else {
     gemm(F(pl.o_o), HD, pl.k_out, R, C, HD,
          Quad<EpiResidual>{{F(pl.o_x), gbuf, gld, g0off, C, F(pl.o_xp)}});

@@ -49,6 +49,10 @@ struct TransArgs {
   float *hid32;                // [R, 128] float32 copy of hidden (null: not needed)
   void *hidden;                // [R, 128] output
   unsigned *status;
+  // PAIR mode: two CTAs per row block, each on half of the SwiGLU width; w_ff_out partials
+  // of the half of the columns the other CTA finishes go through global scratch
+  float *xfer;                 // [row blocks][2][128][64] partial columns
+  int *xflag;                  // [row blocks][2], zero at entry
 };
 
 constexpr int kTransSlotsSplit = 3, kTransSlotsPlain = 6;   // weight ring depth
@@ -104,7 +108,16 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *p, int64_t 
   *reinterpret_cast<uint2 *>(p + i) = make_uint2(lo, hi);
 }
 
-template <bool SPLIT, typename TOut>
+// the CTA pair's flags (global memory, GPU scope); a poll gives up after kPeerSpinLimit
+// reads (status bit 4), so a missing peer cannot hang the kernel
+constexpr uint32_t kPeerSpinLimit = 1u << 22;
+__device__ __forceinline__ int ld_acquire(const int *p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+template <bool SPLIT, typename TOut, bool PAIR>
 __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
   pdl_enter();
   extern __shared__ __align__(1024) uint8_t smem_dyn[];
@@ -124,8 +137,12 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t m0 = (int64_t)blockIdx.x * kUmmaBM;
-  const int nkc_out = t.HD / kUmmaBK, nC = t.M / 64;   // 64-wide hidden chunks
+  // PAIR: CTAs 2p and 2p+1 share row block p; rank k runs SwiGLU chunks [k nL, (k+1) nL)
+  // and finishes output columns [64k, 64k + 64)
+  const int pb = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x, rank = PAIR ? (int)(blockIdx.x & 1) : 0;
+  const int64_t m0 = (int64_t)pb * kUmmaBM;
+  const int nkc_out = t.HD / kUmmaBK, nCall = t.M / 64;   // 64-wide hidden chunks
+  const int nC = PAIR ? nCall / 2 : nCall, ch0 = rank * nC;   // this CTA's chunks
 
   if (tid == 0) {
     for (int s = 0; s < NSLOT; ++s) {
@@ -278,27 +295,71 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
     }
 
     // ---- hidden = usable * (x' + g1 * acc2)
+    // PAIR: the warps of the column half the other CTA finishes send their w_ff_out
+    // partial through global scratch; the other warps add the peer's partial to theirs
+    const bool sender = PAIR && hf != rank;
+    const int64_t xrow = ((int64_t)pb * 2 + rank) * 128 + rl;        // this CTA's scratch row
+    const int64_t prow = ((int64_t)pb * 2 + (1 - rank)) * 128 + rl;  // the peer's
     float g1v[32];                              // chunk 0 fetched before the wait
-    row32(t.g1, t.g_ld, r, rok, cb, g1v);
+    if (!sender) row32(t.g1, t.g_ld, r, rok, cb, g1v);
     const bool use_row = rok && t.usable[r] != 0;
     if (ok) ok = umma::mbar_wait_warp(acc2_done, 0, abort_flag, lane);
     umma::tc_fence_after();
-    const bool use = ok && use_row;
+    if (PAIR) {
+      if (sender) {
 #pragma unroll 1
-    for (int c0 = cb; c0 < cb + 64; c0 += 32) {
-      float a[32], f[32];
-      if (c0 > cb) row32(t.g1, t.g_ld, r, rok, c0, g1v);
-      umma::tmem_ld32(tl + c0, a);
-      umma::tmem_ld32(tl + 384 + c0, f);
-      if (rok) {
+        for (int c0 = cb; c0 < cb + 64; c0 += 32) {
+          float f[32];
+          umma::tmem_ld32(tl + 384 + c0, f);
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          float o[4];
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4 *>(t.xfer + xrow * 64 + (c0 - cb) + i) =
+                make_float4(f[i], f[i + 1], f[i + 2], f[i + 3]);
+        }
+      }
+      epi_sync();
+      if (warp == 0 && lane == 0) {
+        __threadfence();
+        atomicExch(t.xflag + pb * 2 + rank, 1);
+      }
+      if (!sender) {   // wait (bounded) for the peer's partial
+        int got = 1;
+        if (lane == 0) {
+          got = 0;
+          for (uint32_t it = 0; it < kPeerSpinLimit && !got; ++it)
+            got = ld_acquire(t.xflag + pb * 2 + (1 - rank));
+        }
+        got = __shfl_sync(0xffffffffu, got, 0);
+        __syncwarp();
+        if (!got) ok = false;
+      }
+    }
+    const bool use = ok && use_row;
+    if (!sender) {
+#pragma unroll 1
+      for (int c0 = cb; c0 < cb + 64; c0 += 32) {
+        float a[32], f[32];
+        if (c0 > cb) row32(t.g1, t.g_ld, r, rok, c0, g1v);
+        umma::tmem_ld32(tl + c0, a);
+        umma::tmem_ld32(tl + 384 + c0, f);
+        if (PAIR) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) o[e] = use ? fmaf(g1v[i + e], f[i + e], a[i + e]) : 0.f;
-          const float4 o4 = make_float4(o[0], o[1], o[2], o[3]);
-          if (t.hid32) *reinterpret_cast<float4 *>(t.hid32 + r * C + c0 + i) = o4;
-          store4<TOut>((TOut *)t.hidden, r * C + c0 + i, o4);
+          for (int i = 0; i < 32; i += 4) {
+            const float4 q = ok ? __ldcg(reinterpret_cast<const float4 *>(t.xfer + prow * 64 + (c0 - cb) + i))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+            f[i] += q.x; f[i + 1] += q.y; f[i + 2] += q.z; f[i + 3] += q.w;
+          }
+        }
+        if (rok) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            float o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[e] = use ? fmaf(g1v[i + e], f[i + e], a[i + e]) : 0.f;
+            const float4 o4 = make_float4(o[0], o[1], o[2], o[3]);
+            if (t.hid32) *reinterpret_cast<float4 *>(t.hid32 + r * C + c0 + i) = o4;
+            store4<TOut>((TOut *)t.hidden, r * C + c0 + i, o4);
+          }
         }
       }
     }
@@ -357,12 +418,12 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
       for (int kc = 0; kc < nkc_out && ok; ++kc) put(t.w_out, nkc_out, 0, kc);
       // same order as the MMAs consume them
       auto ld_ff1 = [&](int ch) {
-        for (int kc = 0; kc < 2; ++kc) put(t.w_ff1, 2, ch, kc);
+        for (int kc = 0; kc < 2; ++kc) put(t.w_ff1, 2, ch0 + ch, kc);
       };
       ld_ff1(0);
       if (nC > 1) ld_ff1(1);
       for (int ch = 0; ch < nC && ok; ++ch) {
-        put(t.w_ff2, nC, 0, ch);
+        put(t.w_ff2, nCall, 0, ch0 + ch);
         if (ch + 2 < nC) ld_ff1(ch + 2);
       }
     }

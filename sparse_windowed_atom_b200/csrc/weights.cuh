@@ -48,7 +48,7 @@ struct FillJob {
   int pad;
 };
 
-constexpr int kMaxCopyJobs = 12, kMaxPackJobs = 10, kMaxFillJobs = 3;
+constexpr int kMaxCopyJobs = 12, kMaxPackJobs = 10, kMaxFillJobs = 4;
 struct WeightJobs {
   CopyJob copy[kMaxCopyJobs];
   PackJob pack[kMaxPackJobs];
