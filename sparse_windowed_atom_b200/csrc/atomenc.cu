@@ -30,7 +30,7 @@ namespace {
 
 constexpr int kVersion = 1;
 constexpr int kMaxD = 64;
-constexpr size_t kAttnSmemBudget = 210 * 1024;  // one CTA per SM (dynamic part)
+constexpr size_t kAttnSmemBudget = 210 * 1024;  // dynamic part: one CTA per SM, or per two (AF3) / 2 - 1 KB
 
 struct Dims {
   int64_t B = 0, A = 0, T = 0, K = 0, C = 0, S = 0, H = 0, D = 0, P = 0, M = 0, U = 0, V = 0;
@@ -260,15 +260,28 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   // plan, (AF3) the pair-bias table and the Q rows; the K/V stage gets the rest
   const int dmax = D <= 8 ? 8 : D <= 16 ? 16 : D <= 32 ? 32 : 64;
   pl.DP = dmax + 4;  // odd number of 16-byte chunks per staged row: no bank conflicts
-  int qt = pl.af3 ? 32 : 64;
-  const int64_t fill = (B * A + 148 - 1) / 148;
-  if (fill < qt) qt = (int)(fill < 1 ? 1 : fill);
-  while (qt > 1 && attn_fixed_smem(qt, (int)K, (int)H, (int)(H * D), pl.af3) > kAttnSmemBudget / 2)
-    qt /= 2;
+  // AF3 tiles share an SM two at a time when their tables fit half the budget
+  auto tile = [&](size_t budget, int per_sm) {
+    int q = pl.af3 ? 32 : 64;
+    const int64_t fill = (B * A + 148 * per_sm - 1) / (148 * per_sm);
+    if (fill < q) q = (int)(fill < 1 ? 1 : fill);
+    while (q > 1 && attn_fixed_smem(q, (int)K, (int)H, (int)(H * D), pl.af3) > budget / 2) q /= 2;
+    return q;
+  };
+  size_t budget = kAttnSmemBudget;
+  int qt = tile(budget, 1);
+  if (attn_ctas_per_sm(pl.af3) == 2) {
+    const size_t half = kAttnSmemBudget / 2 - 1024;
+    const int q2 = tile(half, 2);
+    if (attn_fixed_smem(q2, (int)K, (int)H, (int)(H * D), pl.af3) + 8 * 1024 <= half) {
+      budget = half;
+      qt = q2;
+    }
+  }
   const size_t fixed = attn_fixed_smem(qt, (int)K, (int)H, (int)(H * D), pl.af3);
-  if (fixed + 8 * 1024 > kAttnSmemBudget) return ATOMENC_ERR_UNSUPPORTED;
+  if (fixed + 8 * 1024 > budget) return ATOMENC_ERR_UNSUPPORTED;
   pl.QT = qt;
-  pl.kv_floats = (int)((kAttnSmemBudget - fixed) / 4);
+  pl.kv_floats = (int)((budget - fixed) / 4);
   pl.attn_smem = fixed + (size_t)pl.kv_floats * 4;
   return ATOMENC_OK;
 }
@@ -575,7 +588,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     dim3 grid((unsigned)((A + pl.QT - 1) / pl.QT), (unsigned)B);
     auto go = [&](auto kern) {
       smem_limit(kern, pl.attn_smem);
-      hk.launch(kern, grid, kAttnThreads, pl.attn_smem, st, ag);
+      hk.launch(kern, grid, attn_threads(pl.af3), pl.attn_smem, st, ag);
     };
     const int dm = D <= 8 ? 8 : D <= 16 ? 16 : D <= 32 ? 32 : 64;
     const bool multi = K > kChunk;

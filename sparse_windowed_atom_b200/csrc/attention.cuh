@@ -9,7 +9,8 @@
 // entries (bullets 5, 6, 15); the weighted values are multiplied by sigmoid of the value
 // gate logits and stored head-major (bullet 16).
 //
-// One CTA (512 threads, one per SM) owns QT consecutive queries of one batch element.
+// One CTA (512 threads, one per SM; AF3: 256 threads, two per SM) owns QT consecutive
+// queries of one batch element.
 //  Phase 1  (may run while the projections finish) one slot per thread per round, eight
 //           rounds in flight: key_index and window_mask are read once (coalesced),
 //           eligibility decided and the slot plan written with the span [klo, khi] of
@@ -35,8 +36,11 @@
 
 namespace atomenc {
 
-constexpr int kAttnThreads = 512;
-constexpr int kAttnWarps = kAttnThreads / kWarp;
+// block size: ESMFold2 one 512-thread CTA per SM; AF3 two 256-thread CTAs per SM, so that
+// one CTA's pair-bias phase (its pair rows are the largest input) overlaps the other's
+// attention
+__host__ __device__ constexpr int attn_threads(bool af3) { return af3 ? 256 : 512; }
+__host__ __device__ constexpr int attn_ctas_per_sm(bool af3) { return af3 ? 2 : 1; }
 constexpr int kPairMax = 32;
 constexpr int kSlotsPerLane = 4;                       // one chunk = 128 slots
 constexpr int kChunk = kWarp * kSlotsPerLane;
@@ -261,11 +265,12 @@ __device__ __forceinline__ float dot_q2_global(const f32x2 (&q2)[DMAX / 2], cons
 // MULTI = true:  any K; pass 1 finds the max and the sum chunk by chunk, pass 2
 //                recomputes the logits to write the weights and accumulate the values.
 template <typename T, int DMAX, bool AF3, bool MULTI>
-__global__ void __launch_bounds__(kAttnThreads, 1) k_slot_attention(AttnArgs g) {
+__global__ void __launch_bounds__(attn_threads(AF3), attn_ctas_per_sm(AF3)) k_slot_attention(AttnArgs g) {
   // the slot plan and the pair bias read only the caller's inputs, the usable flags and
   // the folded pair weights (all from kernels at least two places earlier), so they run
   // before the wait for the projections; Q, K, V, G are read after it
   pdl_launch_next();
+  constexpr int kAttnThreads = attn_threads(AF3), kAttnWarps = kAttnThreads / kWarp;
   extern __shared__ __align__(16) float smem[];
   constexpr int DW = DMAX < 32 ? DMAX : 32;            // channels per reduce-scatter
   // Query pairs sharing their key rows are processed jointly in the 128-slot path; built
