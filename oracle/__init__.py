@@ -99,6 +99,9 @@ def _load():
         lib.orc_forward.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(_Dims),
                                     ctypes.POINTER(_Inputs), ctypes.POINTER(_Params),
                                     ctypes.c_double, _i64, _pu8, ctypes.POINTER(_Outputs)]
+        lib.orc_single_to_pair.restype = ctypes.c_int
+        lib.orc_single_to_pair.argtypes = [_i64, _i64, _i64, _i64, _i64, _pd, _pu8] + [_pd] * 8 + [
+            ctypes.c_double, ctypes.c_int, _pd, _pd]
         _lib = lib
     return _lib
 
@@ -274,3 +277,35 @@ def permitted(activations, parameters, masks, structure, radius=-1, style="af3",
     _load().orc_permitted(ctypes.byref(dims), ctypes.byref(inputs), _ptr(use, _pu8),
                           int(radius), _ptr(out, _pu8))
     return out.astype(bool)
+
+
+# ---------------------------------------------------------------- single to pair
+
+def single_to_pair(activations, parameters, masks, eps=1e-5, output_norm=False):
+    """Page "ESMFold Single-to-Pair Features" (esmfold_single_to_pair), float64:
+    returns (pair_features [B,N,N,2H], output [B,N,N,D]). Keys as the page's worked
+    example prints them: x; mask; weight [C,2H], bias, norm_scale, norm_bias,
+    out_weight [2H,D], out_bias, and output_scale / output_bias for output_norm."""
+    x = _f64(activations["x"])
+    B, N, C = x.shape
+    mask = _u8(masks["mask"])
+    w = _f64(parameters["weight"])
+    H2 = w.shape[1]
+    if H2 % 2:
+        raise OracleError(-2, "weight has an odd number of columns")
+    ow = _f64(parameters["out_weight"])
+    Dp = ow.shape[1]
+    nsc, nbi = _f64(parameters["norm_scale"]), _f64(parameters["norm_bias"])
+    b, ob = _f64(parameters["bias"]), _f64(parameters["out_bias"])
+    osc = _f64(parameters["output_scale"]) if output_norm else None
+    obi = _f64(parameters["output_bias"]) if output_norm else None
+    pf = np.zeros((B, N, N, H2))
+    out = np.zeros((B, N, N, Dp))
+    rc = _load().orc_single_to_pair(B, N, C, H2 // 2, Dp, _ptr(x, _pd), _ptr(mask, _pu8),
+                                    _ptr(nsc, _pd), _ptr(nbi, _pd), _ptr(w, _pd), _ptr(b, _pd),
+                                    _ptr(ow, _pd), _ptr(ob, _pd), _ptr(osc, _pd), _ptr(obi, _pd),
+                                    float(eps), 1 if output_norm else 0, _ptr(pf, _pd),
+                                    _ptr(out, _pd))
+    if rc != 0:
+        raise OracleError(rc, "orc_single_to_pair")
+    return pf, out

@@ -428,3 +428,70 @@ int orc_forward(int style, int stage, const orc_dims *d, const orc_inputs *in,
   free(usable); free(perm); free(need); free(count); free(tok_ok);
   return ORC_OK;
 }
+
+/* ------------------------------------------------------------------ single to pair */
+
+/* [S2P] one call: every step in the order the Required behavior lists it. */
+int orc_single_to_pair(int64_t B, int64_t N, int64_t C, int64_t H, int64_t Dp,
+                       const double *x, const uint8_t *mask, const double *norm_scale,
+                       const double *norm_bias, const double *weight, const double *bias,
+                       const double *out_weight, const double *out_bias,
+                       const double *output_scale, const double *output_bias, double eps,
+                       int output_norm, double *pair_features, double *output) {
+  if (!x || !mask || !norm_scale || !norm_bias || !weight || !bias || !out_weight || !out_bias ||
+      !pair_features || !output || (output_norm && (!output_scale || !output_bias)))
+    return ORC_ERR_ARG;
+  if (B < 1 || N < 1 || C < 1 || H < 1 || Dp < 1) return ORC_ERR_DIM;
+  if (!(eps > 0.0) || !isfinite(eps)) return ORC_ERR_EPS;
+  const int64_t H2 = 2 * H;
+  double *qk = (double *)malloc(sizeof(double) * (size_t)(B * N * H2));
+  double *row = (double *)malloc(sizeof(double) * (size_t)C);
+  double *ln = (double *)malloc(sizeof(double) * (size_t)C);
+  double *f = (double *)malloc(sizeof(double) * (size_t)H2);
+  double *o = (double *)malloc(sizeof(double) * (size_t)Dp);
+  double *on = (double *)malloc(sizeof(double) * (size_t)Dp);
+  if (!qk || !row || !ln || !f || !o || !on) {
+    free(qk); free(row); free(ln); free(f); free(o); free(on);
+    return ORC_ERR_NOMEM;
+  }
+  for (int64_t bn = 0; bn < B * N; ++bn) {
+    /* bullet 1: features of absent tokens are replaced by zero before normalisation */
+    for (int64_t c = 0; c < C; ++c) row[c] = mask[bn] ? x[bn * C + c] : 0.0;
+    /* bullet 2: affine population LayerNorm, then the projection */
+    orc_layer_norm(row, C, eps, ln);
+    for (int64_t c = 0; c < C; ++c) ln[c] = ln[c] * norm_scale[c] + norm_bias[c];
+    for (int64_t e = 0; e < H2; ++e) {
+      double acc = bias[e];
+      for (int64_t c = 0; c < C; ++c) acc += ln[c] * weight[c * H2 + e];
+      qk[bn * H2 + e] = acc;
+    }
+  }
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t i = 0; i < N; ++i)
+      for (int64_t j = 0; j < N; ++j) {
+        const int64_t pij = (b * N + i) * N + j;
+        const double *qi = qk + (b * N + i) * H2, *qj = qk + (b * N + j) * H2;
+        const int both = mask[b * N + i] && mask[b * N + j];
+        /* bullet 3: q then k; pair(i, j) = [k_i * q_j, q_j - k_i] */
+        for (int64_t h = 0; h < H; ++h) {
+          f[h] = qi[H + h] * qj[h];
+          f[H + h] = qj[h] - qi[H + h];
+        }
+        /* bullet 4: the readout straight from the pair features */
+        for (int64_t e = 0; e < Dp; ++e) {
+          double acc = out_bias[e];
+          for (int64_t h = 0; h < H2; ++h) acc += f[h] * out_weight[h * Dp + e];
+          o[e] = acc;
+        }
+        /* bullet 5: optional affine LayerNorm of the output */
+        if (output_norm) {
+          orc_layer_norm(o, Dp, eps, on);
+          for (int64_t e = 0; e < Dp; ++e) o[e] = on[e] * output_scale[e] + output_bias[e];
+        }
+        /* bullet 1: both returned tensors are zero unless both endpoints are present */
+        for (int64_t h = 0; h < H2; ++h) pair_features[pij * H2 + h] = both ? f[h] : 0.0;
+        for (int64_t e = 0; e < Dp; ++e) output[pij * Dp + e] = both ? o[e] : 0.0;
+      }
+  free(qk); free(row); free(ln); free(f); free(o); free(on);
+  return ORC_OK;
+}

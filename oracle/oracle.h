@@ -13,6 +13,8 @@
  *            (bullets counted from 1 in the order printed).
  *   [AF3 ...] "AlphaFold 3 Atom Attention Encoder", Required behavior / Worked example.
  *   [ESM ...] "ESMFold 2 Atom Attention Encoder", Required behavior / Worked example.
+ *   [S2P n]  "ESMFold Single-to-Pair Features" (function esmfold_single_to_pair),
+ *            Required behavior, bullet n (counted from 1).
  *
  * Readings taken where the pages are silent (dictionary keys and weight shapes are
  * not printed on any page): every weight is applied as x @ W with W stored
@@ -130,6 +132,21 @@ void orc_permitted(const orc_dims *d, const orc_inputs *in, const uint8_t *usabl
 int orc_forward(int style, int stage, const orc_dims *d, const orc_inputs *in,
                 const orc_params *p, double eps, int64_t radius,
                 const uint8_t *query_select, orc_outputs *out);
+
+/*
+ * Single-to-pair features [S2P 1-6]. x [B,N,C], mask [B,N] (1 = present);
+ * norm_scale, norm_bias [C]; weight [C,2H], bias [2H] (columns 0..H-1 give q, H..2H-1
+ * give k); out_weight [2H,Dp], out_bias [Dp]; output_scale, output_bias [Dp] (read only
+ * when output_norm != 0). Writes pair_features [B,N,N,2H] = [k_i * q_j, q_j - k_i] and
+ * output [B,N,N,Dp] = pair_features @ out_weight + out_bias (then the affine LayerNorm
+ * when output_norm), both zero unless tokens i and j are present.
+ */
+int orc_single_to_pair(int64_t B, int64_t N, int64_t C, int64_t H, int64_t Dp,
+                       const double *x, const uint8_t *mask, const double *norm_scale,
+                       const double *norm_bias, const double *weight, const double *bias,
+                       const double *out_weight, const double *out_bias,
+                       const double *output_scale, const double *output_bias, double eps,
+                       int output_norm, double *pair_features, double *output);
 
 #ifdef __cplusplus
 }
