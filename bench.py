@@ -49,6 +49,9 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="host seconds for the oracle baseline sample")
+    p.add_argument("--op", choices=["block", "single_to_pair"], default="block",
+                   help="block: the atom attention block (default); single_to_pair: the pair "
+                        "feature pass, B=1 N=384 C=128 2H=64 D=128 with output_norm")
     return p.parse_args()
 
 
@@ -516,8 +519,56 @@ def run_atomenc(args):
     return 0
 
 
+def run_single_to_pair(args):
+    """Pair features of one N=384 chain (synthetic, seeded): pairs/s of device time, and the
+    pass's HBM roofline (x read once; pair_features and output written once)."""
+    import torch
+    from sparse_windowed_atom_b200 import atomenc
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU path exists)")
+    dev = torch.device("cuda", 0)
+    B, N, C, H, Dp = 1, 384, 128, 32, 128
+    rng = np.random.default_rng(0)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device=dev, dtype=torch.float32)
+    act = {"x": t(rng.normal(size=(B, N, C)))}
+    prm = {"weight": t(rng.normal(size=(C, 2 * H)) / np.sqrt(C)), "bias": t(0.1 * rng.normal(size=2 * H)),
+           "norm_scale": t(1 + 0.1 * rng.normal(size=C)), "norm_bias": t(0.1 * rng.normal(size=C)),
+           "out_weight": t(rng.normal(size=(2 * H, Dp)) / np.sqrt(2 * H)), "out_bias": t(0.1 * rng.normal(size=Dp)),
+           "output_scale": t(1 + 0.1 * rng.normal(size=Dp)), "output_bias": t(0.1 * rng.normal(size=Dp))}
+    msk = {"mask": torch.from_numpy(rng.random((B, N)) < 0.95).to(dev)}
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    ws = None
+    for _ in range(args.warmup):
+        flush.zero_()
+        pf, out = atomenc.single_to_pair(act, prm, msk, eps=1e-5, output_norm=True, workspace=ws)
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record()
+        atomenc.single_to_pair(act, prm, msk, eps=1e-5, output_norm=True, workspace=ws)
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    ms = statistics.fmean(a.elapsed_time(b) for a, b in evs)
+    nbytes = B * N * C * 4 + B * N * N * (2 * H + Dp) * 4
+    peak, src = load_peaks()
+    achieved = nbytes / (ms / 1e3) / 1e9
+    print(json.dumps({"op": "single_to_pair", "metric": "pair features: token pairs/s", "unit": "pairs/s",
+                      "value": B * N * N / (ms / 1e3), "ms_per_step": ms, "steps": args.steps,
+                      "warmup": args.warmup, "dtype": "f32", "data": "synthetic (seeded)",
+                      "config": {"B": B, "N": N, "C": C, "2H": 2 * H, "D": Dp, "output_norm": True,
+                                 "l2": f"flushed before every timed step ({FLUSH_BYTES >> 20} MiB write)"},
+                      "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                                   "frac": achieved / peak, "bytes_per_step": nbytes, "peak_source": src},
+                      "higher_is_better": True}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.op == "single_to_pair":
+        return run_single_to_pair(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_atomenc(args)

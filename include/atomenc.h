@@ -223,6 +223,49 @@ const char *atomenc_strerror(int code);
 /* Library version, for the Python binding's load check. */
 int atomenc_version(void);
 
+/* ---------------------------------------------------------------------------------
+ * Single-to-pair features: the page "ESMFold Single-to-Pair Features"
+ * (esmfold_single_to_pair), Required behavior. For every ordered token pair (i, j):
+ *   q, k = split(LN_affine(x_sanitised) @ weight + bias)          (q: first H columns)
+ *   pair_features[b,i,j] = [k_i * q_j, q_j - k_i]                 [2H]
+ *   output[b,i,j]        = pair_features[b,i,j] @ out_weight + out_bias, then (when
+ *                          output_norm != 0) an affine LayerNorm with output_scale/bias
+ * both zero unless mask[b,i] and mask[b,j]; rows of absent tokens are replaced by zero
+ * before the normalisation. Every LayerNorm is the population one with eps inside the
+ * square root. Shapes: x [B,N,C]; mask [B,N] bool; norm_scale, norm_bias [C];
+ * weight [C,2H], bias [2H]; out_weight [2H,Dp], out_bias [Dp]; output_scale,
+ * output_bias [Dp] (only read when output_norm != 0); pair_features [B,N,N,2H] and
+ * output [B,N,N,Dp]. Float tensors share one type (F32 or BF16). Limits: C <= 4096,
+ * 2H <= 256, Dp <= 256 and 2H * Dp <= 16384 (ATOMENC_ERR_UNSUPPORTED beyond).
+ * Errors are decided on the host before anything is enqueued, as for atomenc_forward.
+ */
+typedef struct {
+  atomenc_tensor x;     /* [B,N,C] single (per-token) features */
+  atomenc_tensor mask;  /* [B,N] bool, true = present */
+} atomenc_s2p_inputs;
+
+typedef struct {
+  atomenc_tensor norm_scale, norm_bias;      /* [C] */
+  atomenc_tensor weight, bias;               /* [C,2H], [2H] */
+  atomenc_tensor out_weight, out_bias;       /* [2H,Dp], [Dp] */
+  atomenc_tensor output_scale, output_bias;  /* [Dp], output_norm only */
+} atomenc_s2p_params;
+
+typedef struct {
+  atomenc_tensor pair_features;  /* [B,N,N,2H] */
+  atomenc_tensor output;         /* [B,N,N,Dp] */
+} atomenc_s2p_outputs;
+
+/* Workspace bytes (256-byte aligned) for atomenc_single_to_pair; 0 if the arguments do
+ * not validate. */
+size_t atomenc_s2p_workspace_size(const atomenc_s2p_inputs *in, const atomenc_s2p_params *params,
+                                  int output_norm, const atomenc_s2p_outputs *out);
+
+/* Enqueue the single-to-pair pass on `stream`; returns ATOMENC_OK or an error code. */
+int atomenc_single_to_pair(const atomenc_s2p_inputs *in, const atomenc_s2p_params *params,
+                           double eps, int output_norm, const atomenc_s2p_outputs *out,
+                           void *workspace, size_t workspace_bytes, atomenc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

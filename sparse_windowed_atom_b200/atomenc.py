@@ -47,6 +47,24 @@ class AtomencOutputs(ctypes.Structure):
     _fields_ = [(n, AtomencTensor) for n in OUTPUT_FIELDS]
 
 
+S2P_INPUT_FIELDS = ["x", "mask"]
+S2P_PARAM_FIELDS = ["norm_scale", "norm_bias", "weight", "bias", "out_weight", "out_bias",
+                    "output_scale", "output_bias"]
+S2P_OUTPUT_FIELDS = ["pair_features", "output"]
+
+
+class AtomencS2PInputs(ctypes.Structure):
+    _fields_ = [(n, AtomencTensor) for n in S2P_INPUT_FIELDS]
+
+
+class AtomencS2PParams(ctypes.Structure):
+    _fields_ = [(n, AtomencTensor) for n in S2P_PARAM_FIELDS]
+
+
+class AtomencS2POutputs(ctypes.Structure):
+    _fields_ = [(n, AtomencTensor) for n in S2P_OUTPUT_FIELDS]
+
+
 class AtomencError(RuntimeError):
     def __init__(self, code: int, what: str):
         super().__init__(f"{what}: atomenc error {code}: {atomenc_strerror(code)}")
@@ -86,6 +104,14 @@ def load_library() -> ctypes.CDLL:
         lib.atomenc_strerror.argtypes = [ctypes.c_int]
         lib.atomenc_version.restype = ctypes.c_int
         lib.atomenc_version.argtypes = []
+        lib.atomenc_s2p_workspace_size.restype = ctypes.c_size_t
+        lib.atomenc_s2p_workspace_size.argtypes = [P(AtomencS2PInputs), P(AtomencS2PParams),
+                                                   ctypes.c_int, P(AtomencS2POutputs)]
+        lib.atomenc_single_to_pair.restype = ctypes.c_int
+        lib.atomenc_single_to_pair.argtypes = [P(AtomencS2PInputs), P(AtomencS2PParams),
+                                               ctypes.c_double, ctypes.c_int,
+                                               P(AtomencS2POutputs), ctypes.c_void_p,
+                                               ctypes.c_size_t, ctypes.c_void_p]
         _lib = lib
     return _lib
 
@@ -254,3 +280,42 @@ def windowed_atom_attention(activations: dict, parameters: dict, masks: dict, st
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     atomenc_forward(style, stage, inputs, parameters, eps, radius, outputs, workspace, stream)
     return outputs
+
+
+# ---------------------------------------------------------------- single to pair
+
+def _s2p_structs(activations, parameters, masks, outputs):
+    ins = AtomencS2PInputs(x=describe(activations.get("x")), mask=describe(masks.get("mask")))
+    prm = AtomencS2PParams(**{n: describe(parameters.get(n)) for n in S2P_PARAM_FIELDS})
+    outs = AtomencS2POutputs(**{n: describe(outputs.get(n)) for n in S2P_OUTPUT_FIELDS})
+    return ins, prm, outs
+
+
+def single_to_pair(activations: dict, parameters: dict, masks: dict, eps: float = 1e-5,
+                   output_norm: bool = False, workspace: torch.Tensor | None = None,
+                   stream=None):
+    """Page "ESMFold Single-to-Pair Features" (esmfold_single_to_pair) on the GPU: dicts
+    of CUDA tensors in (x; mask; weight, bias, norm_scale, norm_bias, out_weight,
+    out_bias, output_scale/output_bias), (pair_features [B,N,N,2H], output [B,N,N,D])
+    out. Allocates the outputs (and the workspace unless one is given) with torch."""
+    x = activations["x"]
+    B, N, _ = x.shape
+    H2 = parameters["weight"].shape[1]
+    Dp = parameters["out_weight"].shape[1]
+    outputs = {"pair_features": torch.empty(B, N, N, H2, dtype=x.dtype, device=x.device),
+               "output": torch.empty(B, N, N, Dp, dtype=x.dtype, device=x.device)}
+    ins, prm, outs = _s2p_structs(activations, parameters, masks, outputs)
+    lib = load_library()
+    need = lib.atomenc_s2p_workspace_size(ctypes.byref(ins), ctypes.byref(prm),
+                                          1 if output_norm else 0, ctypes.byref(outs))
+    if need == 0:
+        raise ValueError("atomenc_s2p_workspace_size: the arguments do not validate")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    rc = lib.atomenc_single_to_pair(ctypes.byref(ins), ctypes.byref(prm), float(eps),
+                                    1 if output_norm else 0, ctypes.byref(outs),
+                                    workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                    _stream_ptr(stream))
+    if rc != 0:
+        raise AtomencError(rc, "atomenc_single_to_pair")
+    return outputs["pair_features"], outputs["output"]
