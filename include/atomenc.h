@@ -235,8 +235,9 @@ int atomenc_version(void);
  * square root. Shapes: x [B,N,C]; mask [B,N] bool; norm_scale, norm_bias [C];
  * weight [C,2H], bias [2H]; out_weight [2H,Dp], out_bias [Dp]; output_scale,
  * output_bias [Dp] (only read when output_norm != 0); pair_features [B,N,N,2H] and
- * output [B,N,N,Dp]. Float tensors share one type (F32 or BF16). Limits: C <= 4096,
- * 2H <= 256, Dp <= 256 and 2H * Dp <= 16384 (ATOMENC_ERR_UNSUPPORTED beyond).
+ * output [B,N,N,Dp]. Float tensors share one type (F32 or BF16). Limits: C <= 256,
+ * 2H <= 256, Dp <= 256, 2H * Dp <= 16384, C * 2H <= 49152
+ * (ATOMENC_ERR_UNSUPPORTED beyond).
  * Errors are decided on the host before anything is enqueued, as for atomenc_forward.
  */
 typedef struct {

@@ -1,9 +1,10 @@
 // s2p.cu -- single-to-pair features: page "ESMFold Single-to-Pair Features"
 // (esmfold_single_to_pair), Required behavior bullets 1-6.
 //
-//   k_s2p_qk     one warp per token: absent rows replaced by zero (bullet 1), affine
-//                population LayerNorm (bullet 2), projection x @ weight + bias into q
-//                then k (bullet 3); float32 [B*N, 2H] in the workspace.
+//   k_s2p_qk     one warp per token, the row held in registers and the weight staged in
+//                shared memory: absent rows replaced by zero (bullet 1), affine population
+//                LayerNorm (bullet 2), projection x @ weight + bias into q then k
+//                (bullet 3); float32 [B*N, 2H] in the workspace.
 //   k_s2p_pairs  one CTA per (b, i), warps over j: pair(i, j) = [k_i * q_j, q_j - k_i]
 //                (bullet 3), its readout with out_weight held in shared memory (bullet 4),
 //                the optional affine output LayerNorm (bullet 5); both returned tensors are
@@ -18,7 +19,7 @@
 namespace atomenc {
 namespace s2p {
 
-constexpr int kMaxH2 = 256, kMaxDp = 256, kMaxWeight = 16384, kMaxC = 4096;
+constexpr int kMaxH2 = 256, kMaxDp = 256, kMaxWeight = 16384, kMaxC = 256;
 constexpr int kPairThreads = 256;
 
 struct QKArgs {
@@ -31,38 +32,65 @@ struct QKArgs {
   float *qk;  // [rows, 2H]
 };
 
+// rows per CTA of the projection pass; its weight [C, 2H] is staged once per CTA
+constexpr int kQKRows = 16, kQKThreads = kQKRows * 32;
+
 template <typename T>
-__global__ void k_s2p_qk(QKArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+__global__ void __launch_bounds__(kQKThreads) k_s2p_qk(QKArgs a) {
+  extern __shared__ float sq[];  // weight [C][2H], then norm_scale [C], norm_bias [C]
+  const int tid = threadIdx.x, lane = tid & 31;
+  float *snsc = sq + a.C * a.H2, *snbi = snsc + a.C;
+  for (int k = tid; k < a.C * a.H2; k += kQKThreads) sq[k] = ldf((const T *)a.w, k);
+  for (int k = tid; k < a.C; k += kQKThreads) {
+    snsc[k] = ldf((const T *)a.nsc, k);
+    snbi[k] = ldf((const T *)a.nbi, k);
+  }
+  __syncthreads();
+  const int64_t row = (int64_t)blockIdx.x * kQKRows + (tid >> 5);
   if (row >= a.rows) return;
   const bool use = a.mask[row] != 0;
   const T *x = (const T *)a.x + row * a.C;
+  // the row in registers: lane holds channels lane + 32 u (C <= 32 * kMaxCU)
+  constexpr int kMaxCU = kMaxC / kWarp;
+  float v[kMaxCU];
   float s = 0.f;
-  for (int c = lane; c < a.C; c += kWarp) s += use ? ldf(x, c) : 0.f;
+#pragma unroll
+  for (int u = 0; u < kMaxCU; ++u) {
+    const int c = lane + u * kWarp;
+    v[u] = use && c < a.C ? ldf(x, c) : 0.f;
+    s += v[u];
+  }
   const float mean = warp_sum(s) / (float)a.C;
   float q = 0.f;
-  for (int c = lane; c < a.C; c += kWarp) {
-    const float d = (use ? ldf(x, c) : 0.f) - mean;
-    q = fmaf(d, d, q);
+#pragma unroll
+  for (int u = 0; u < kMaxCU; ++u) {
+    const int c = lane + u * kWarp;
+    if (c < a.C) q = fmaf(v[u] - mean, v[u] - mean, q);
   }
   const float rstd = 1.f / sqrtf(warp_sum(q) / (float)a.C + a.eps);
-  // lanes over the 2H output columns; the normalised value of channel c is formed by
-  // every lane (same-address loads)
+#pragma unroll
+  for (int u = 0; u < kMaxCU; ++u) {
+    const int c = lane + u * kWarp;
+    if (c < a.C) v[u] = (v[u] - mean) * rstd * snsc[c] + snbi[c];
+  }
   float acc[kMaxH2 / kWarp];
 #pragma unroll
   for (int t = 0; t < kMaxH2 / kWarp; ++t) {
     const int e = lane + t * kWarp;
     acc[t] = e < a.H2 ? ldf((const T *)a.bias, e) : 0.f;
   }
-  for (int c = 0; c < a.C; ++c) {
-    const float v = ((use ? ldf(x, c) : 0.f) - mean) * rstd * ldf((const T *)a.nsc, c) +
-                    ldf((const T *)a.nbi, c);
-    const T *wr = (const T *)a.w + (int64_t)c * a.H2;
 #pragma unroll
-    for (int t = 0; t < kMaxH2 / kWarp; ++t) {
-      const int e = lane + t * kWarp;
-      if (e < a.H2) acc[t] = fmaf(v, ldf(wr, e), acc[t]);
+  for (int u = 0; u < kMaxCU; ++u) {
+    if (u * kWarp >= a.C) break;
+    const int lim = a.C - u * kWarp < kWarp ? a.C - u * kWarp : kWarp;
+    for (int l = 0; l < lim; ++l) {
+      const float vc = __shfl_sync(0xffffffffu, v[u], l);
+      const float *wr = sq + (u * kWarp + l) * a.H2;
+#pragma unroll
+      for (int t = 0; t < kMaxH2 / kWarp; ++t) {
+        const int e = lane + t * kWarp;
+        if (e < a.H2) acc[t] = fmaf(vc, wr[e], acc[t]);
+      }
     }
   }
 #pragma unroll
@@ -119,47 +147,116 @@ __global__ void __launch_bounds__(kPairThreads) k_s2p_pairs(PairArgs a) {
       else if (h < H2) f[m] = qj[h - H] - ki[h - H];
       if (h < H2) stf(pf, h, f[m]);
     }
-    float o[kMaxDp / kWarp];
+    if ((Dp & 3) == 0) {
+      // readout: lane owns columns 4 lane + 128 t .. +3 (Dp a multiple of 4)
+      constexpr int kT = kMaxDp / 128;
+      float4 o[kT];
 #pragma unroll
-    for (int t = 0; t < kMaxDp / kWarp; ++t) {
-      const int e = lane + t * kWarp;
-      o[t] = e < Dp ? sb[e] : 0.f;
-    }
+      for (int t = 0; t < kT; ++t) {
+        const int e = 4 * lane + 128 * t;
+        o[t] = e < Dp ? *reinterpret_cast<const float4 *>(sb + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
 #pragma unroll
-    for (int m = 0; m < kMaxH2 / kWarp; ++m) {
-      if (m * kWarp >= H2) break;
-      const int lim = H2 - m * kWarp < kWarp ? H2 - m * kWarp : kWarp;
-      for (int l = 0; l < lim; ++l) {
-        const float fv = __shfl_sync(0xffffffffu, f[m], l);
-        const float *wr = sw + (m * kWarp + l) * Dp;
+      for (int m = 0; m < kMaxH2 / kWarp; ++m) {
+        if (m * kWarp >= H2) break;
+        const int lim = H2 - m * kWarp < kWarp ? H2 - m * kWarp : kWarp;
+        for (int l = 0; l < lim; ++l) {
+          const float fv = __shfl_sync(0xffffffffu, f[m], l);
+          const float *wr = sw + (m * kWarp + l) * Dp;
 #pragma unroll
-        for (int t = 0; t < kMaxDp / kWarp; ++t) {
-          const int e = lane + t * kWarp;
-          if (e < Dp) o[t] = fmaf(fv, wr[e], o[t]);
+          for (int t = 0; t < kT; ++t) {
+            const int e = 4 * lane + 128 * t;
+            if (e < Dp) {
+              const float4 w = *reinterpret_cast<const float4 *>(wr + e);
+              o[t].x = fmaf(fv, w.x, o[t].x);
+              o[t].y = fmaf(fv, w.y, o[t].y);
+              o[t].z = fmaf(fv, w.z, o[t].z);
+              o[t].w = fmaf(fv, w.w, o[t].w);
+            }
+          }
         }
       }
-    }
-    if (a.onorm) {
-      float s = 0.f;
+      if (a.onorm) {
+        float s = 0.f;
 #pragma unroll
-      for (int t = 0; t < kMaxDp / kWarp; ++t)
-        if (lane + t * kWarp < Dp) s += o[t];
-      const float mean = warp_sum(s) / (float)Dp;
-      float q = 0.f;
+        for (int t = 0; t < kT; ++t)
+          if (4 * lane + 128 * t < Dp) s += (o[t].x + o[t].y) + (o[t].z + o[t].w);
+        const float mean = warp_sum(s) / (float)Dp;
+        float q = 0.f;
 #pragma unroll
-      for (int t = 0; t < kMaxDp / kWarp; ++t)
-        if (lane + t * kWarp < Dp) q = fmaf(o[t] - mean, o[t] - mean, q);
-      const float rstd = 1.f / sqrtf(warp_sum(q) / (float)Dp + a.eps);
+        for (int t = 0; t < kT; ++t)
+          if (4 * lane + 128 * t < Dp) {
+            q = fmaf(o[t].x - mean, o[t].x - mean, q);
+            q = fmaf(o[t].y - mean, o[t].y - mean, q);
+            q = fmaf(o[t].z - mean, o[t].z - mean, q);
+            q = fmaf(o[t].w - mean, o[t].w - mean, q);
+          }
+        const float rstd = 1.f / sqrtf(warp_sum(q) / (float)Dp + a.eps);
+#pragma unroll
+        for (int t = 0; t < kT; ++t) {
+          const int e = 4 * lane + 128 * t;
+          if (e < Dp) {
+            o[t].x = fmaf((o[t].x - mean) * rstd, ssc[e], sbi[e]);
+            o[t].y = fmaf((o[t].y - mean) * rstd, ssc[e + 1], sbi[e + 1]);
+            o[t].z = fmaf((o[t].z - mean) * rstd, ssc[e + 2], sbi[e + 2]);
+            o[t].w = fmaf((o[t].w - mean) * rstd, ssc[e + 3], sbi[e + 3]);
+          }
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < kT; ++t) {
+        const int e = 4 * lane + 128 * t;
+        if (e < Dp) {
+          stf(out, e, o[t].x);
+          stf(out, e + 1, o[t].y);
+          stf(out, e + 2, o[t].z);
+          stf(out, e + 3, o[t].w);
+        }
+      }
+    } else {
+      // readout: lane owns columns lane + 32 t (any Dp)
+      float o[kMaxDp / kWarp];
 #pragma unroll
       for (int t = 0; t < kMaxDp / kWarp; ++t) {
         const int e = lane + t * kWarp;
-        if (e < Dp) o[t] = fmaf((o[t] - mean) * rstd, ssc[e], sbi[e]);
+        o[t] = e < Dp ? sb[e] : 0.f;
       }
-    }
 #pragma unroll
-    for (int t = 0; t < kMaxDp / kWarp; ++t) {
-      const int e = lane + t * kWarp;
-      if (e < Dp) stf(out, e, o[t]);
+      for (int m = 0; m < kMaxH2 / kWarp; ++m) {
+        if (m * kWarp >= H2) break;
+        const int lim = H2 - m * kWarp < kWarp ? H2 - m * kWarp : kWarp;
+        for (int l = 0; l < lim; ++l) {
+          const float fv = __shfl_sync(0xffffffffu, f[m], l);
+          const float *wr = sw + (m * kWarp + l) * Dp;
+#pragma unroll
+          for (int t = 0; t < kMaxDp / kWarp; ++t) {
+            const int e = lane + t * kWarp;
+            if (e < Dp) o[t] = fmaf(fv, wr[e], o[t]);
+          }
+        }
+      }
+      if (a.onorm) {
+        float s = 0.f;
+#pragma unroll
+        for (int t = 0; t < kMaxDp / kWarp; ++t)
+          if (lane + t * kWarp < Dp) s += o[t];
+        const float mean = warp_sum(s) / (float)Dp;
+        float q = 0.f;
+#pragma unroll
+        for (int t = 0; t < kMaxDp / kWarp; ++t)
+          if (lane + t * kWarp < Dp) q = fmaf(o[t] - mean, o[t] - mean, q);
+        const float rstd = 1.f / sqrtf(warp_sum(q) / (float)Dp + a.eps);
+#pragma unroll
+        for (int t = 0; t < kMaxDp / kWarp; ++t) {
+          const int e = lane + t * kWarp;
+          if (e < Dp) o[t] = fmaf((o[t] - mean) * rstd, ssc[e], sbi[e]);
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < kMaxDp / kWarp; ++t) {
+        const int e = lane + t * kWarp;
+        if (e < Dp) stf(out, e, o[t]);
+      }
     }
   }
 }
@@ -224,7 +321,8 @@ int validate(const atomenc_s2p_inputs *in, const atomenc_s2p_params *p, int onor
   }
   S2P_CHECK(check(out->pair_features, d.fdt, 4, spf));
   S2P_CHECK(check(out->output, d.fdt, 4, sout));
-  if (d.C > kMaxC || d.H2 > kMaxH2 || d.Dp > kMaxDp || d.H2 * d.Dp > kMaxWeight)
+  if (d.C > kMaxC || d.H2 > kMaxH2 || d.Dp > kMaxDp || d.H2 * d.Dp > kMaxWeight ||
+      d.C * d.H2 > 3 * kMaxWeight)
     return ATOMENC_ERR_UNSUPPORTED;
   if (d.B * d.N >= (int64_t)1 << 31) return ATOMENC_ERR_UNSUPPORTED;
   return ATOMENC_OK;
@@ -248,8 +346,11 @@ int launch(const Dims &d, const atomenc_s2p_inputs *in, const atomenc_s2p_params
   QKArgs qa{d.B * d.N, (int)d.C, (int)d.H2, eps, in->x.data,
             static_cast<const uint8_t *>(in->mask.data), p->norm_scale.data, p->norm_bias.data,
             p->weight.data, p->bias.data, qk};
-  const int64_t rows_per_block = 8;
-  k_s2p_qk<T><<<(unsigned)((d.B * d.N + rows_per_block - 1) / rows_per_block), 256, 0, st>>>(qa);
+  const size_t qsmem = (size_t)(d.C * d.H2 + 2 * d.C) * 4;
+  if (cudaFuncSetAttribute(k_s2p_qk<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qsmem) !=
+      cudaSuccess)
+    return ATOMENC_ERR_CUDA;
+  k_s2p_qk<T><<<(unsigned)((d.B * d.N + kQKRows - 1) / kQKRows), kQKThreads, qsmem, st>>>(qa);
   PairArgs pa{d.N, (int)(d.H2 / 2), (int)d.H2, (int)d.Dp, eps, onorm ? 1 : 0,
               static_cast<const uint8_t *>(in->mask.data), qk, p->out_weight.data,
               p->out_bias.data, onorm ? p->output_scale.data : nullptr,

@@ -93,7 +93,7 @@ def test_parity(dtype, output_norm):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("kw", [dict(B=1, N=1, C=5, H=1, Dp=1), dict(B=3, N=33, C=130, H=128, Dp=64),
+@pytest.mark.parametrize("kw", [dict(B=1, N=1, C=5, H=1, Dp=3), dict(B=3, N=33, C=130, H=128, Dp=64),
                                 dict(B=1, N=65, C=96, H=32, Dp=256), dict(B=2, N=20, p_present=0.0)])
 def test_shapes_and_edges(kw):
     _check(12, torch.float32, True, **kw)
