@@ -27,16 +27,26 @@ STYLES = {"af3": 0, "esmfold2": 1}
 STAGES = {"decoder": 0, "encoder": 1}
 
 
-def build(force: bool = False) -> str:
-    """Compile oracle.c into liboracle.so beside it (gcc, -O2, no fast-math)."""
-    stale = not os.path.exists(_LIB) or any(
-        os.path.getmtime(f) > os.path.getmtime(_LIB) for f in (_SRC, _HDR))
+_LIB_OMP = os.path.join(_HERE, "liboracle_omp.so")
+
+
+def _compile(lib: str, extra: list, force: bool) -> str:
+    stale = not os.path.exists(lib) or any(
+        os.path.getmtime(f) > os.path.getmtime(lib) for f in (_SRC, _HDR))
     if force or stale:
-        tmp = _LIB + f".tmp{os.getpid()}"
+        tmp = lib + f".tmp{os.getpid()}"
         subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared",
-                               "-fno-fast-math", "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB)
-    return _LIB
+                               "-fno-fast-math", *extra, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so beside it (gcc, -O2, no fast-math), and the
+    same source with -fopenmp into liboracle_omp.so (per-atom loops on all host cores,
+    each atom's arithmetic unchanged; used to time the oracle as a CPU baseline)."""
+    _compile(_LIB_OMP, ["-fopenmp"], force)
+    return _compile(_LIB, [], force)
 
 
 _i64 = ctypes.c_int64
@@ -72,13 +82,14 @@ class _Outputs(ctypes.Structure):
                 ("position_update", _pd)]
 
 
-_lib = None
+_libs = {}
 
 
-def _load():
-    global _lib
-    if _lib is None:
-        lib = ctypes.CDLL(build())
+def _load(threads: str = "one"):
+    """The oracle library: threads="one" (the checker) or "all" (OpenMP build)."""
+    if threads not in _libs:
+        build()
+        lib = ctypes.CDLL(_LIB if threads == "one" else _LIB_OMP)
         lib.orc_sigmoid.restype = ctypes.c_double
         lib.orc_sigmoid.argtypes = [ctypes.c_double]
         lib.orc_silu.restype = ctypes.c_double
@@ -102,8 +113,15 @@ def _load():
         lib.orc_single_to_pair.restype = ctypes.c_int
         lib.orc_single_to_pair.argtypes = [_i64, _i64, _i64, _i64, _i64, _pd, _pu8] + [_pd] * 8 + [
             ctypes.c_double, ctypes.c_int, _pd, _pd]
-        _lib = lib
-    return _lib
+        lib.orc_threads.restype = ctypes.c_int
+        lib.orc_threads.argtypes = []
+        _libs[threads] = lib
+    return _libs[threads]
+
+
+def threads_used(threads: str = "all") -> int:
+    """Host threads the per-atom loops of the chosen build run on."""
+    return int(_load(threads).orc_threads())
 
 
 def _f64(x):
@@ -195,15 +213,17 @@ class OracleError(RuntimeError):
 
 
 def windowed_atom_attention(activations, parameters, masks, structure, eps=1e-5,
-                            style="af3", stage="decoder", radius=-1, query_select=None):
+                            style="af3", stage="decoder", radius=-1, query_select=None,
+                            threads="one"):
     """Float64 forward pass; returns a dict of float64 numpy arrays.
 
     Returns hidden [B,A,C] and attention [B,H,A,K] plus token_output [B,T,U]
     (encoder) or position_update [B,A,3] (decoder). With ``query_select`` only the
     selected query atoms (and tokens all of whose usable atoms are selected) are
-    computed; everything else is NaN.
+    computed; everything else is NaN. ``threads="all"`` runs the OpenMP build of the
+    same source (identical per-atom arithmetic) on every host core.
     """
-    lib = _load()
+    lib = _load(threads)
     dm = infer_dims(style, stage, activations, parameters, masks, structure)
     dims = _Dims(**dm)
     keep = {}

@@ -14,6 +14,22 @@
 #include <stdlib.h>
 #include <string.h>
 
+/* Built twice: plain (one thread) and with -fopenmp, where the per-atom loops run on
+ * all host cores. Each atom's arithmetic is the same in both builds; every thread has
+ * its own scratch rows, and the pooled sums are still accumulated serially in
+ * ascending atom order. */
+#ifdef _OPENMP
+#include <omp.h>
+static int orc_nthreads(void) { return omp_get_max_threads(); }
+static int orc_tid(void) { return omp_get_thread_num(); }
+#else
+static int orc_nthreads(void) { return 1; }
+static int orc_tid(void) { return 0; }
+#endif
+
+/* threads the per-atom loops of orc_forward use */
+int orc_threads(void) { return orc_nthreads(); }
+
 /* sigmoid(z) = 1 / (1 + e^-z); SiLU(z) = z * sigmoid(z)  [ESM RB, last-but-one item].
  * For z < 0 the same value is formed as e^z / (1 + e^z), so that a representable
  * subnormal tail is kept rather than flushed through an overflowing e^-z  [WAA 23] */
@@ -132,6 +148,34 @@ static void arena_free(arena *ar) {
   ar->n = 0;
 }
 
+/* scratch rows of the calling thread, carved from its slice of tmp */
+#define ORC_SCRATCH_ROWS \
+  double *r_c = tmp + scratch * orc_tid();              /* clean condition [S] */ \
+  double *r_ln = r_c + S;         /* LN(c) or SiLU(c) [S] */ \
+  double *r_cj = r_ln + S;        /* LN(c) * cond_scale[j] [S] */ \
+  double *r_x = r_cj + S;         /* normalised x [C] */ \
+  double *r_sc = r_x + C;         /* scale logits [C] */ \
+  double *r_sh = r_sc + C;        /* shift [C] */ \
+  double *r_f0 = r_sh + C;        /* query features / shared attention input [C] */ \
+  double *r_f1 = r_f0 + C;        /* key/value features [C] */ \
+  double *r_m = r_f1 + C;         /* ESMFold2 six vectors [6C] */ \
+  double *r_q = r_m + 6 * C;      /* projection before head norm [HD] */ \
+  double *r_h = r_q + HD;         /* one head [D] */ \
+  double *r_o = r_h + D;          /* attention output [HD] */ \
+  double *r_u = r_o + HD;         /* out-projection [C] */ \
+  double *r_z = r_u + C;          /* transition input [C] */ \
+  double *r_a = r_z + C;          /* z @ w_ff_gate [M] */ \
+  double *r_b = r_a + M;          /* z @ w_ff_up [M] */ \
+  double *r_ff = r_b + M;         /* transition update [C] */ \
+  double *r_pool = r_ff + C;      /* hidden @ w_pool [U] */ \
+  double *r_lg = r_pool + U;      /* logits of one row [K] */ \
+  double *r_w = r_lg + K;         /* weights of one row [K] */ \
+  double *r_pr = r_w + K;         /* LN(pair) [P] */ \
+  double *r_tk = r_pr + P;        /* token @ w_token [C] */
+#define ORC_SCRATCH_USED (void)r_c; (void)r_ln; (void)r_cj; (void)r_x; (void)r_sc; (void)r_sh; \
+  (void)r_f0; (void)r_f1; (void)r_m; (void)r_q; (void)r_h; (void)r_o; (void)r_u; (void)r_z; \
+  (void)r_a; (void)r_b; (void)r_ff; (void)r_pool; (void)r_lg; (void)r_w; (void)r_pr; (void)r_tk
+
 int orc_forward(int style, int stage, const orc_dims *d, const orc_inputs *in,
                 const orc_params *p, double eps, int64_t radius,
                 const uint8_t *query_select, orc_outputs *out) {
@@ -184,7 +228,10 @@ int orc_forward(int style, int stage, const orc_dims *d, const orc_inputs *in,
   double *G = grab(&ar, A * GW);
   double *g0 = grab(&ar, A * C), *g1 = grab(&ar, A * C);    /* residual gates */
   double *tsc = grab(&ar, A * C), *tsh = grab(&ar, A * C);  /* transition scale/shift */
-  double *tmp = grab(&ar, 8 * (C + S + HD + M + U + V + P + K) + 64);
+  const int nthr = orc_nthreads();
+  /* per thread; covers every row carved below (3S + 15C + 2HD + D + 2M + U + 2K + P) */
+  const int64_t scratch = 16 * (C + S + HD + D + M + U + V + P + K) + 64;
+  double *tmp = grab(&ar, scratch * nthr);
   double *pooled = enc ? grab(&ar, T * U) : NULL;
   int64_t *count = enc ? (int64_t *)malloc((size_t)T * sizeof(int64_t)) : NULL;
   uint8_t *tok_ok = enc ? (uint8_t *)malloc((size_t)T) : NULL;
@@ -194,30 +241,6 @@ int orc_forward(int style, int stage, const orc_dims *d, const orc_inputs *in,
     arena_free(&ar); free(usable); free(perm); free(need); free(count); free(tok_ok);
     return ORC_ERR_NOMEM;
   }
-
-  /* scratch rows carved from tmp */
-  double *r_c = tmp;              /* clean condition [S] */
-  double *r_ln = r_c + S;         /* LN(c) or SiLU(c) [S] */
-  double *r_cj = r_ln + S;        /* LN(c) * cond_scale[j] [S] */
-  double *r_x = r_cj + S;         /* normalised x [C] */
-  double *r_sc = r_x + C;         /* scale logits [C] */
-  double *r_sh = r_sc + C;        /* shift [C] */
-  double *r_f0 = r_sh + C;        /* query features / shared attention input [C] */
-  double *r_f1 = r_f0 + C;        /* key/value features [C] */
-  double *r_m = r_f1 + C;         /* ESMFold2 six vectors [6C] */
-  double *r_q = r_m + 6 * C;      /* projection before head norm [HD] */
-  double *r_h = r_q + HD;         /* one head [D] */
-  double *r_o = r_h + D;          /* attention output [HD] */
-  double *r_u = r_o + HD;         /* out-projection [C] */
-  double *r_z = r_u + C;          /* transition input [C] */
-  double *r_a = r_z + C;          /* z @ w_ff_gate [M] */
-  double *r_b = r_a + M;          /* z @ w_ff_up [M] */
-  double *r_ff = r_b + M;         /* transition update [C] */
-  double *r_pool = r_ff + C;      /* hidden @ w_pool [U] */
-  double *r_lg = r_pool + U;      /* logits of one row [K] */
-  double *r_w = r_lg + K;         /* weights of one row [K] */
-  double *r_pr = r_w + K;         /* LN(pair) [P] */
-  double *r_tk = r_pr + P;        /* token @ w_token [C] */
 
   for (int64_t b = 0; b < B; ++b) {
     const uint8_t *use = usable + b * A;
@@ -236,7 +259,10 @@ int orc_forward(int style, int stage, const orc_dims *d, const orc_inputs *in,
     }
 
     /* ---- residual start and conditioning for every needed usable atom ---- */
+#pragma omp parallel for schedule(dynamic, 16)
     for (int64_t a = 0; a < A; ++a) {
+      ORC_SCRATCH_ROWS
+      ORC_SCRATCH_USED;
       if (!need[a] || !use[a]) continue;
       const int64_t ia = b * A + a;
       /* sanitised payloads: an unusable atom is never reached here, so the
@@ -321,7 +347,10 @@ int orc_forward(int style, int stage, const orc_dims *d, const orc_inputs *in,
     }
 
     /* ---- attention, residual, transition per selected query ---- */
+#pragma omp parallel for schedule(dynamic, 16)
     for (int64_t a = 0; a < A; ++a) {
+      ORC_SCRATCH_ROWS
+      ORC_SCRATCH_USED;
       if (sel && !sel[a]) continue;
       const int64_t ia = b * A + a;
       for (int64_t h = 0; h < H; ++h) {
@@ -401,6 +430,8 @@ int orc_forward(int style, int stage, const orc_dims *d, const orc_inputs *in,
     /* ---- encoder pooling: exact per-token mean of ReLU(hidden @ w_pool) over the
      * usable atoms assigned to it; tokens without atoms give zero  [WAA 19] ---- */
     if (enc) {
+      ORC_SCRATCH_ROWS
+      ORC_SCRATCH_USED;
       for (int64_t t = 0; t < T; ++t) {
         count[t] = 0;
         tok_ok[t] = 1;
