@@ -32,10 +32,12 @@ sys.path.insert(0, ROOT)
 
 from sparse_windowed_atom_b200 import workloads  # noqa: E402
 
-DEFAULT_WORKLOAD = "esm_encoder_fp32_a4096"
+DEFAULT_WORKLOAD = "esm_encoder_bf16_b2_a32768"
 METRIC = "atom-encoder atoms/s and attention entries/s (A·H·K); % of HBM roofline"
 FLUSH_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0            # burst
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0  # seconds-long loop under the power cap
 
 
 def parse_args():
@@ -58,19 +60,40 @@ def parse_args():
 # ----------------------------------------------------------------------------- helpers
 
 def attention_bytes(spec: workloads.WorkloadSpec) -> int:
-    """Algorithmic HBM bytes of one slot-attention launch: key_index (int64), window_mask,
-    pair rows (AF3, storage type) and the usable flags read once; Q, K, V and value-gate
-    logits read once and the gated output written once (float32 workspace); the attention
-    weights written once (storage type)."""
+    """Algorithmic HBM bytes of one slot-attention launch: key_index (int64) and
+    window_mask read once per slot, AF3 pair rows (storage type) once per slot, the
+    usable flag once per atom, Q, K, V and value-gate logits read once per atom and the
+    gated output written once per atom (storage type), the attention weights written
+    once (storage type)."""
     s = 2 if spec.dtype == "bfloat16" else 4
     slots = spec.B * spec.A * spec.K
     hd = spec.H * spec.D
     b = slots * (8 + 1)
     if spec.style == "af3":
         b += slots * spec.P * s
-    b += spec.B * spec.A * (1 + 5 * hd * 4)
+    b += spec.B * spec.A * (1 + 5 * hd * s)
     b += spec.B * spec.H * spec.A * spec.K * s
     return b
+
+
+def dense_flops(spec: workloads.WorkloadSpec) -> int:
+    """Algorithmic flops of the dense projections of one forward (2 per multiply-add):
+    conditioning (AF3: 3 scale + 3 shift + 2 gate blocks of C columns; ESMFold2: the six
+    w_mod blocks), Q/K/V/value gate, attention out-projection, SwiGLU gate/up and
+    w_ff_out, and the encoder's pooling projection or the decoder's token projection
+    (per token) and readout."""
+    C, S, HD, M, U, V = spec.C, spec.S, spec.H * spec.D, spec.M, spec.U, spec.V
+    per_atom = 2 * S * (8 * C if spec.style == "af3" else 6 * C)
+    per_atom += 2 * C * 4 * HD + 2 * HD * C + 2 * C * 2 * M + 2 * M * C
+    per_atom += 2 * C * U if spec.stage == "encoder" else 2 * C * 3
+    total = per_atom * spec.B * spec.A
+    if spec.stage == "decoder":
+        total += 2 * V * C * spec.B * spec.T
+    return total
+
+
+def storage_dtype(spec) -> str:
+    return "bf16" if spec.dtype == "bfloat16" else "f32"
 
 
 def config_of(spec, world):
@@ -87,13 +110,19 @@ def config_of(spec, world):
 
 
 def load_peaks():
+    """(hbm GB/s, bf16 TFLOP/s sustained, source) from MEASURED_PEAKS.json, else the
+    fallbacks measured earlier on this machine."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             pk = json.load(f)
-        return float(pk["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, STREAM-style copy)"
+        hbm = float(pk["hbm_gbs"])
+        tf = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+        tf = float(tf) if tf is not None else FALLBACK_BF16_TFLOPS_SUSTAINED
+        return hbm, tf, "measured (MEASURED_PEAKS.json: hbm_gbs STREAM-style copy, bf16_tflops_sustained cuBLAS loop)"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s earlier measurement on this pool)"
+        return (FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS_SUSTAINED,
+                "fallback (6.65 TB/s and 1.4 PFLOP/s sustained, earlier measurements on this pool)")
 
 
 def kernel_source_sha() -> str:
@@ -193,10 +222,12 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- CPU oracle
 
-def oracle_rate(spec, budget_s: float, seed: int = 0):
-    """Time the float64 oracle (as it stands, one host thread) on a bounded sample of the
-    workload: batch element 0, the first n query atoms (n doubled until the budget is
-    used), repeated until budget_s. Returns (atoms/s, sample description, seconds)."""
+def oracle_rate(spec, budget_s: float, seed: int = 0, threads: str = "all"):
+    """Time the float64 oracle (as it stands) on a bounded sample of the workload:
+    batch element 0, the first n query atoms (n doubled until the budget is used),
+    repeated until budget_s. threads="all" runs the OpenMP build of the same source on
+    every host core, "one" the one-thread build. Returns (atoms/s, sample, seconds,
+    threads used)."""
     import oracle
     w = workloads.make_inputs(spec.replace(B=1), seed=seed)
     f64 = lambda d: {k: v.astype(np.float64) for k, v in d.items()}
@@ -209,16 +240,18 @@ def oracle_rate(spec, budget_s: float, seed: int = 0):
         t = time.perf_counter()
         oracle.windowed_atom_attention(act, prm, w["masks"], w["structure"], eps=spec.eps,
                                        style=spec.style, stage=spec.stage, radius=spec.radius,
-                                       query_select=None if n == spec.A else sel)
+                                       query_select=None if n == spec.A else sel,
+                                       threads=threads)
         dt = time.perf_counter() - t
         spent += dt
         done += n
         passes += 1
         if dt < budget_s / 6 and n < spec.A:
             n = min(spec.A, n * 2)
+    cores = oracle.threads_used(threads)
     sample = (f"batch element 0 of {spec.name}: {passes} oracle passes over the first "
-              f"<= {n} of {spec.A} query atoms ({done} atoms total)")
-    return done / spent, sample, spent
+              f"<= {n} of {spec.A} query atoms ({done} atoms total), {cores} host thread(s)")
+    return done / spent, sample, spent, cores
 
 
 def run_reference(args):
@@ -230,9 +263,9 @@ def run_reference(args):
     per_step = max(0.5, min(8.0, 150.0 / max(1, steps + warm)))
     for _ in range(warm):
         oracle_rate(spec, per_step / 4)
-    total_atoms, total_s, sample = 0.0, 0.0, ""
+    total_atoms, total_s, sample, cores = 0.0, 0.0, "", 1
     for _ in range(steps):
-        r, sample, s = oracle_rate(spec, per_step)
+        r, sample, s, cores = oracle_rate(spec, per_step)
         total_atoms += r * s
         total_s += s
     rate = total_atoms / total_s
@@ -242,7 +275,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded)", "config": config_of(spec, 1),
         "entries_per_s": rate * spec.H * spec.K,
-        "cpu_baseline": {"value": rate, "unit": "atoms/s", "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": rate, "unit": "atoms/s", "cores": cores, "kind": "oracle",
                          "sample": f"each step: {sample}"},
         "e2e": {"value": rate, "unit": "atoms/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -393,6 +426,28 @@ def run_atomenc(args):
     torch.cuda.synchronize(dev)
     barrier()
 
+    # ---- traced pass: the same steps again with an event after every kernel (these
+    # events serialise the kernels); gives each kernel's own device time
+    nk = atomenc.MAX_LAUNCHES + 1
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk)] for _ in range(K)]
+    for row in kev:
+        for e in row:
+            e.record(stream)
+    barrier()
+    torch.cuda.synchronize(dev)
+    kinds = []
+    for i in range(K):
+        flush.zero_()
+        kinds = atomenc.atomenc_forward_traced(spec.style, spec.stage, inputs, params, spec.eps,
+                                               spec.radius, outs, ws, kev[i], stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    kernel_ms = [statistics.fmean(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(K))
+                 for j in range(len(kinds))]
+    by_kind = {}
+    for kd, t in zip(kinds, kernel_ms):
+        by_kind[kd] = by_kind.get(kd, 0.0) + t
+
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
     phase_ms = [statistics.fmean(evs[i][p].elapsed_time(evs[i][p + 1]) for i in range(K))
                 for p in range(atomenc.NUM_PHASES)]
@@ -402,17 +457,30 @@ def run_atomenc(args):
     atoms = spec.atoms * world
     value = ranks.job_rate(spec.atoms, ms_per_step)
 
-    # ---- roofline of the slot-attention kernel (timed live, phase 3 = that kernel alone)
-    attn_ms = max_over_ranks(phase_ms[3])
-    peak, peak_src = load_peaks()
+    # ---- roofline of the slot-attention kernel (its own device time, traced pass)
+    attn_ms = max_over_ranks(by_kind.get("attention", phase_ms[3]))
+    hbm_peak, tc_peak, peak_src = load_peaks()
     abytes = attention_bytes(spec)
     achieved = abytes / (attn_ms / 1e3) / 1e9
     dominant = max(range(atomenc.NUM_PHASES), key=lambda p: phase_ms[p])
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": recorded_traffic(spec.name),
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": recorded_traffic(spec.name),
                 "kernel": "k_slot_attention", "bytes_per_launch": abytes,
                 "avg_launch_ms": attn_ms, "peak_source": peak_src,
                 "frac_of_8TBs": achieved / 8000.0}
+    # ---- the dense projections on the tensor cores: algorithmic flops over the summed
+    # device time of the tcgen05 kernels (projection GEMMs and the fused tail)
+    tc_ms = max_over_ranks(by_kind.get("gemm", 0.0) + by_kind.get("transition", 0.0))
+    flops = dense_flops(spec)
+    tc_ach = flops / (tc_ms / 1e3) / 1e12 if tc_ms > 0 else 0.0
+    roofline_tc = {"bound": "tensor", "achieved": tc_ach, "peak": tc_peak, "unit": "TFLOP/s",
+                   "frac": tc_ach / tc_peak, "traffic": None,
+                   "kernels": "k_gemm_rows + k_transition (tcgen05)",
+                   "flops_per_step": flops, "ms_per_step": tc_ms, "peak_source": peak_src,
+                   "products": ("three bf16 tcgen05 products per float32 product (hi*hi + hi*lo "
+                                "+ lo*hi); the flops counted are the algorithmic ones"
+                                if spec.dtype == "float32" else
+                                "bf16 operands, float32 accumulation")}
 
     # ---- end to end: pinned host inputs -> device, forward, outputs -> pinned host, every
     # step through the public API. Two buffer sets and three streams: the host->device
@@ -493,19 +561,24 @@ def run_atomenc(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, sample, spent = oracle_rate(spec, args.cpu_seconds)
-        cpu = {"value": rate, "unit": "atoms/s", "cores": 1, "kind": "oracle", "sample": sample,
-               "seconds": spent}
+        rate, sample, spent, cores = oracle_rate(spec, args.cpu_seconds, threads="all")
+        rate1, sample1, spent1, _ = oracle_rate(spec, max(2.0, args.cpu_seconds / 3), threads="one")
+        cpu = {"value": rate, "unit": "atoms/s", "cores": cores, "kind": "oracle", "sample": sample,
+               "seconds": spent, "one_core": {"value": rate1, "cores": 1, "sample": sample1,
+                                              "seconds": spent1}}
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "atoms/s", "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32",
+            "vs_baseline": None, "dtype": storage_dtype(spec),
             "data": "synthetic (seeded workload generator; no dataset)",
             "config": config_of(spec, world),
             "entries_per_s": ranks.job_rate(spec.entries, ms_per_step),
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "roofline_projections": roofline_tc,
+            "cpu_baseline": cpu, "e2e": e2e,
+            "kernel_ms": {k: v for k, v in sorted(by_kind.items())},
+            "kernel_launches": kinds,
             "gpu_launches": launches,
             "clocks": sampler.summary(),
             "phase_ms": dict(zip(atomenc.PHASES, phase_ms)),
@@ -552,7 +625,7 @@ def run_single_to_pair(args):
     torch.cuda.synchronize()
     ms = statistics.fmean(a.elapsed_time(b) for a, b in evs)
     nbytes = B * N * C * 4 + B * N * N * (2 * H + Dp) * 4
-    peak, src = load_peaks()
+    peak, _, src = load_peaks()
     achieved = nbytes / (ms / 1e3) / 1e9
     print(json.dumps({"op": "single_to_pair", "metric": "pair features: token pairs/s", "unit": "pairs/s",
                       "value": B * N * N / (ms / 1e3), "ms_per_step": ms, "steps": args.steps,

@@ -182,13 +182,54 @@ int atomenc_forward_profiled(int style, int stage, const atomenc_inputs *in,
                              int *n_launches);
 
 /*
+ * Kinds of kernel one forward pass launches (for atomenc_forward_traced).
+ */
+enum atomenc_kernel_kind {
+  ATOMENC_KERNEL_PREP = 0,        /* weight images, panels, resets (CUDA cores) */
+  ATOMENC_KERNEL_GEMM = 1,        /* a tcgen05 projection GEMM with its fused epilogue */
+  ATOMENC_KERNEL_TRANSITION = 2,  /* the tcgen05 tail: out-projection .. hidden */
+  ATOMENC_KERNEL_ATTENTION = 3,   /* the slot-gathered attention */
+  ATOMENC_KERNEL_ROWS = 4,        /* a row kernel on CUDA cores (masking, norms, rotary, readout) */
+  ATOMENC_KERNEL_POOL = 5         /* the per-token mean */
+};
+
+/*
+ * atomenc_forward with an event per kernel: events[0] is recorded on `stream` before
+ * the first launch and events[i + 1] right after launch i (these records serialise
+ * the kernels: the pass is slightly slower than atomenc_forward); kinds[i] (if kinds
+ * is not NULL) receives the enum atomenc_kernel_kind of launch i and *n_launches the
+ * number of launches. n_events must exceed the number of launches (a pass launches at
+ * most 16 kernels); ATOMENC_ERR_NULL otherwise. Same results as atomenc_forward.
+ */
+int atomenc_forward_traced(int style, int stage, const atomenc_inputs *in,
+                           const atomenc_params *params, double eps, int64_t radius,
+                           const atomenc_outputs *out, void *workspace, size_t workspace_bytes,
+                           atomenc_stream_t stream, void *const *events, int n_events,
+                           int *kinds, int *n_launches);
+
+/*
  * Read the device status word that the last forward pass using `workspace` left
- * (waits for `stream`). Bits: 1 = some query tile's keys spanned more rows than the
- * shared-memory stage holds and were gathered from L2 instead (slower, same result);
- * 2 = atom_to_token was not grouped by token, so pooling scanned wider atom ranges
- * (slower, same result). Never an error; returns enum atomenc_status.
+ * (waits for `stream`). Bits:
+ *   1 = some query tile's keys spanned more rows than the shared-memory stage holds and
+ *       were gathered from L2 instead. Not an error: same results, slower.
+ *   4 = a bounded wait inside a kernel (a tensor-core completion, a bulk copy, or the
+ *       partner CTA of the paired transition) reached its poll limit and gave up. AN
+ *       ERROR: the kernel returned without finishing, and hidden, attention and the
+ *       pooled / readout outputs of this pass are invalid.
+ * Returns enum atomenc_status (of the read, not of the pass).
  */
 int atomenc_get_status(const void *workspace, int *device_status, atomenc_stream_t stream);
+
+/*
+ * Test hook of the bounded wait between the two CTAs of a row block in the paired
+ * transition kernel (used when row blocks are few): poll_limit = polls of the
+ * partner's flag before giving up (0 restores the default), withhold_flags != 0 makes
+ * every CTA skip raising its own flag, so that the partner's wait runs out and the pass
+ * sets status bit 4 instead of hanging. Process-wide; affects passes enqueued after
+ * the call. Leave it at (0, 0) outside tests. Returns ATOMENC_OK. No counterpart on
+ * the pages.
+ */
+int atomenc_debug_peer_wait(uint32_t poll_limit, int withhold_flags);
 
 /*
  * Forward pass that allocates nothing and takes no workspace argument.
@@ -210,12 +251,20 @@ int atomenc_get_status(const void *workspace, int *device_status, atomenc_stream
  *    clears what it needs zeroed itself. Two calls whose GPU work overlaps (different
  *    streams without ordering, or different host threads) race on the array: order
  *    them on one stream.
- * No counterpart on the pages; results and other errors are those of atomenc_forward.
+ * No counterpart on the pages; results and other errors are those of atomenc_forward,
+ * and atomenc_noalloc_get_status reads the pass's status word.
  */
 #define ATOMENC_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 int atomenc_forward_noalloc(int style, int stage, const atomenc_inputs *in,
                             const atomenc_params *params, double eps, int64_t radius,
                             const atomenc_outputs *out, atomenc_stream_t stream);
+
+/*
+ * The status word (bits as for atomenc_get_status) that the last atomenc_forward_noalloc
+ * pass on the current device left in the library's scratch array; waits for `stream`.
+ * Bit 4 means that pass's outputs are invalid. Returns enum atomenc_status.
+ */
+int atomenc_noalloc_get_status(int *device_status, atomenc_stream_t stream);
 
 /* Static English text for an atomenc_status code. */
 const char *atomenc_strerror(int code);

@@ -98,8 +98,15 @@ def load_library() -> ctypes.CDLL:
         lib.atomenc_forward_noalloc.argtypes = [ctypes.c_int, ctypes.c_int, P(AtomencInputs),
                                                 P(AtomencParams), ctypes.c_double, ctypes.c_int64,
                                                 P(AtomencOutputs), ctypes.c_void_p]
+        lib.atomenc_forward_traced.restype = ctypes.c_int
+        lib.atomenc_forward_traced.argtypes = lib.atomenc_forward.argtypes + [
+            P(ctypes.c_void_p), ctypes.c_int, P(ctypes.c_int), P(ctypes.c_int)]
         lib.atomenc_get_status.restype = ctypes.c_int
         lib.atomenc_get_status.argtypes = [ctypes.c_void_p, P(ctypes.c_int), ctypes.c_void_p]
+        lib.atomenc_noalloc_get_status.restype = ctypes.c_int
+        lib.atomenc_noalloc_get_status.argtypes = [P(ctypes.c_int), ctypes.c_void_p]
+        lib.atomenc_debug_peer_wait.restype = ctypes.c_int
+        lib.atomenc_debug_peer_wait.argtypes = [ctypes.c_uint32, ctypes.c_int]
         lib.atomenc_strerror.restype = ctypes.c_char_p
         lib.atomenc_strerror.argtypes = [ctypes.c_int]
         lib.atomenc_version.restype = ctypes.c_int
@@ -240,6 +247,57 @@ def atomenc_forward_profiled(style: str, stage: str, inputs: dict, params: dict,
     return n.value
 
 
+KERNEL_KINDS = ["prep", "gemm", "transition", "attention", "rows", "pool"]
+MAX_LAUNCHES = 16
+
+
+def atomenc_forward_traced(style: str, stage: str, inputs: dict, params: dict, eps: float,
+                           radius: int, outputs: dict, workspace: torch.Tensor, events,
+                           stream=None) -> list:
+    """atomenc_forward with an event after every kernel: events[0] is recorded before
+    the first launch and events[i+1] after launch i (torch.cuda.Event objects, already
+    recorded once; at least MAX_LAUNCHES + 1 of them). Returns the kernel kinds in
+    launch order (names from KERNEL_KINDS)."""
+    ins, prm, outs = _structs(inputs, params, outputs)
+    handles = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
+    kinds = (ctypes.c_int * len(events))()
+    n = ctypes.c_int(0)
+    rc = load_library().atomenc_forward_traced(
+        STYLES[style], STAGES[stage], ctypes.byref(ins), ctypes.byref(prm), float(eps),
+        int(radius), ctypes.byref(outs), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream_ptr(stream), handles,
+        len(events), kinds, ctypes.byref(n))
+    if rc != 0:
+        raise AtomencError(rc, "atomenc_forward_traced")
+    return [KERNEL_KINDS[kinds[i]] for i in range(n.value)]
+
+
+STATUS_L2_FALLBACK = 1     # keys gathered from L2 (same results)
+STATUS_WAIT_TIMEOUT = 4    # a bounded wait gave up: the pass's outputs are invalid
+
+
+class AtomencStatusError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: device status {status:#x}: a bounded wait inside a kernel "
+                         "reached its poll limit; the outputs of this pass are invalid")
+        self.status = status
+
+
+def atomenc_noalloc_get_status(stream=None) -> int:
+    """Status word of the last atomenc_forward_noalloc pass on the current device."""
+    v = ctypes.c_int(0)
+    rc = load_library().atomenc_noalloc_get_status(ctypes.byref(v), _stream_ptr(stream))
+    if rc != 0:
+        raise AtomencError(rc, "atomenc_noalloc_get_status")
+    return v.value
+
+
+def atomenc_debug_peer_wait(poll_limit: int = 0, withhold_flags: bool = False) -> None:
+    """Test hook of the paired transition kernel's bounded wait (0, False restores the
+    defaults)."""
+    load_library().atomenc_debug_peer_wait(int(poll_limit), 1 if withhold_flags else 0)
+
+
 def atomenc_get_status(workspace: torch.Tensor, stream=None) -> int:
     v = ctypes.c_int(0)
     rc = load_library().atomenc_get_status(workspace.data_ptr(), ctypes.byref(v),
@@ -266,10 +324,14 @@ def output_shapes(style: str, stage: str, inputs: dict, params: dict) -> dict:
 def windowed_atom_attention(activations: dict, parameters: dict, masks: dict, structure: dict,
                             eps: float = 1e-5, style: str = "af3", stage: str = "decoder",
                             radius: int = -1, workspace: torch.Tensor | None = None,
-                            stream=None) -> dict:
+                            stream=None, check_status: bool = True) -> dict:
     """Forward pass with the page's signature: dicts of CUDA tensors in, a dict out
     (hidden, attention, and token_output for the encoder or position_update for the
-    decoder). Allocates the outputs (and the workspace unless one is given) with torch."""
+    decoder). Allocates the outputs (and the workspace unless one is given) with torch.
+    With check_status (the default) it waits for the pass and raises
+    AtomencStatusError if a bounded wait inside a kernel gave up (status bit 4), so that
+    invalid outputs are never returned silently; check_status=False keeps the call
+    asynchronous (read atomenc_get_status yourself)."""
     inputs = {**activations, **masks, **structure}
     dev = activations["atom"].device
     fdt = activations["atom"].dtype
@@ -279,6 +341,10 @@ def windowed_atom_attention(activations: dict, parameters: dict, masks: dict, st
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     atomenc_forward(style, stage, inputs, parameters, eps, radius, outputs, workspace, stream)
+    if check_status:
+        st = atomenc_get_status(workspace, stream)
+        if st & STATUS_WAIT_TIMEOUT:
+            raise AtomencStatusError(st, "windowed_atom_attention")
     return outputs
 
 

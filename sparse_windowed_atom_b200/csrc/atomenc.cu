@@ -66,6 +66,24 @@ float bf16_round_host(float f) {
   return f;
 }
 
+constexpr int kMaxDevices = 64;
+
+// Multiprocessors of the current device, looked up once per device.
+int g_sm_count[kMaxDevices];
+std::mutex g_sm_mutex;
+int sm_count() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lock(g_sm_mutex);
+  if (g_sm_count[dev] <= 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_sm_count[dev] = n;
+  }
+  return g_sm_count[dev];
+}
+
 struct Plan {
   int style = 0, stage = 0, fdt = 0;
   bool af3 = false, enc = false, fuse_tail = false, tail_pair = false;
@@ -80,6 +98,7 @@ struct Plan {
   // attention launch
   int QT = 0, DP = 0, kv_floats = 0;
   size_t attn_smem = 0;
+  int sms = 148;                    // multiprocessors of the device the pass runs on
 };
 
 size_t take(size_t &cur, size_t bytes) {
@@ -229,7 +248,8 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   // few row blocks: two CTAs per row block, each on half of the SwiGLU width (all CTAs
   // fit on the GPU at once, one per SM)
   const int64_t nrb = (R + kUmmaBM - 1) / kUmmaBM;
-  pl.tail_pair = pl.fuse_tail && 2 * nrb <= 148;
+  pl.sms = sm_count();
+  pl.tail_pair = pl.fuse_tail && 2 * nrb <= pl.sms;
   pl.o_xfer = take(cur, pl.tail_pair ? nrb * 2 * 128 * 64 * 4 : 0);
   pl.o_xflag = take(cur, pl.tail_pair ? nrb * 2 * 4 : 0);
   pl.o_xp = take(cur, pl.fuse_tail ? 0 : R * C * 4);
@@ -256,14 +276,14 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   pl.k_tok = take(cur, pl.enc ? 0 : packed_bytes(V, C, split));
   pl.bytes = cur;
 
-  // ---- attention tile: QT queries per CTA (the grid should cover the 148 SMs), a slot
+  // ---- attention tile: QT queries per CTA (the grid should cover the SMs), a slot
   // plan, (AF3) the pair-bias table and the Q rows; the K/V stage gets the rest
   const int dmax = D <= 8 ? 8 : D <= 16 ? 16 : D <= 32 ? 32 : 64;
   pl.DP = dmax + 4;  // odd number of 16-byte chunks per staged row: no bank conflicts
   // AF3 tiles share an SM two at a time when their tables fit half the budget
   auto tile = [&](size_t budget, int per_sm) {
     int q = pl.af3 ? 32 : 64;
-    const int64_t fill = (B * A + 148 * per_sm - 1) / (148 * per_sm);
+    const int64_t fill = (B * A + (int64_t)pl.sms * per_sm - 1) / ((int64_t)pl.sms * per_sm);
     if (fill < q) q = (int)(fill < 1 ? 1 : fill);
     while (q > 1 && attn_fixed_smem(q, (int)K, (int)H, (int)(H * D), pl.af3) > budget / 2) q /= 2;
     return q;
@@ -285,8 +305,6 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   pl.attn_smem = fixed + (size_t)pl.kv_floats * 4;
   return ATOMENC_OK;
 }
-
-constexpr int kMaxDevices = 64;
 
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device), and again only
 // if a larger size is asked for: the attribute outlives the call, so repeating it on
@@ -323,31 +341,66 @@ cudaError_t smem_limit(void (*kern)(KP...), size_t bytes) {
 
 struct Hooks {
   cudaEvent_t const *ev = nullptr;  // ATOMENC_NUM_PHASES + 1 events, or null
+  cudaEvent_t const *kev = nullptr; // traced: one event before the pass and one per launch
+  int n_kev = 0;
+  int *kinds = nullptr;             // traced: enum atomenc_kernel_kind per launch
   int launches = 0;
   cudaError_t err = cudaSuccess;    // first launch failure
+  bool overflow = false;            // traced: more launches than events
   void mark(int i, cudaStream_t st) const {
     if (ev) cudaEventRecord(ev[i], st);
   }
+  void begin(cudaStream_t st) {
+    if (kev && n_kev > 0) cudaEventRecord(kev[0], st);
+  }
   // Every kernel is launched here, with programmatic stream serialization: it may be
-  // scheduled while its predecessor finishes and waits for it in pdl_enter().
+  // scheduled while its predecessor finishes and waits for it in pdl_enter(). A
+  // cluster size of 2 launches the grid as CTA pairs that the hardware schedules
+  // together.
   template <typename... KP, typename... Args>
-  void launch(void (*kern)(KP...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+  void launch(int kind, void (*kern)(KP...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
               Args &&...args) {
-    cudaLaunchAttribute at[1];
+    launch_cluster(kind, 1, kern, grid, block, smem, st, std::forward<Args>(args)...);
+  }
+  template <typename... KP, typename... Args>
+  void launch_cluster(int kind, int cluster, void (*kern)(KP...), dim3 grid, dim3 block,
+                      size_t smem, cudaStream_t st, Args &&...args) {
+    cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[0].val.programmaticStreamSerializationAllowed = 1;
+    int nat = 1;
+    if (cluster > 1) {
+      at[1].id = cudaLaunchAttributeClusterDimension;
+      at[1].val.clusterDim.x = (unsigned)cluster;
+      at[1].val.clusterDim.y = 1;
+      at[1].val.clusterDim.z = 1;
+      nat = 2;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = nat;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
     if (e != cudaSuccess && err == cudaSuccess) err = e;
+    if (kev) {
+      if (launches + 1 < n_kev) {
+        cudaEventRecord(kev[launches + 1], st);
+        if (kinds) kinds[launches] = kind;
+      } else {
+        overflow = true;
+      }
+    }
     ++launches;
   }
 };
+
+// Test hook for the bounded wait of the paired transition CTAs (see
+// atomenc_debug_peer_wait): poll limit, and whether the partials' flags are withheld.
+std::atomic<uint32_t> g_peer_spin_limit{kPeerSpinLimit};
+std::atomic<int> g_peer_withhold{0};
 
 template <typename Elt>
 int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p,
@@ -449,7 +502,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     wj.fill[wj.nfill++] = FillJob{first, B * T, INT_MAX, 0};
     wj.fill[wj.nfill++] = FillJob{last, B * T, -1, 0};
   }
-  hk.launch((k_prep_weights<Elt>), dim3(64, wj.ncopy + wj.npack + wj.nfill), 256, 0, st, wj);
+  hk.launch(ATOMENC_KERNEL_PREP, (k_prep_weights<Elt>), dim3(64, wj.ncopy + wj.npack + wj.nfill), 256, 0, st, wj);
 
   // out = epi(A' @ W) on the tensor cores, W given by its packed image and A' produced by
   // `prod` (A itself, or a row normalisation fused into the operand); K <= 256
@@ -457,17 +510,17 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     using P = decltype(prod);
     using E = decltype(epi);
     const int64_t mt = (Mr + kUmmaBM - 1) / kUmmaBM, nt = (N + kUmmaBN - 1) / kUmmaBN;
-    const int64_t want = (148 + mt - 1) / mt;             // CTAs per row block to fill the GPU
+    const int64_t want = (pl.sms + mt - 1) / mt;          // CTAs per row block to fill the GPU
     const int64_t sp = want < nt ? want : nt;
     const int per = (int)((nt + sp - 1) / sp);
     dim3 grid((unsigned)((nt + per - 1) / per), (unsigned)mt);
     const size_t smem = rows_smem_bytes(Kd, split);
     if (split) {
       smem_limit(k_gemm_rows<P, true, E>, smem);
-      hk.launch((k_gemm_rows<P, true, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, epi, status);
+      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_rows<P, true, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, epi, status);
     } else {
       smem_limit(k_gemm_rows<P, false, E>, smem);
-      hk.launch((k_gemm_rows<P, false, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, epi, status);
+      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_rows<P, false, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, epi, status);
     }
   };
   // out = epi(A @ W): the row-block kernel for K <= 256, else the streaming kernel
@@ -482,10 +535,10 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     const size_t smem = umma_smem_bytes(split);
     if (split) {
       smem_limit(k_gemm_umma<TA, true, E>, smem);
-      hk.launch((k_gemm_umma<TA, true, E>), grid, kUmmaThreads, smem, st, A_, lda, ws + wpk, Mr, N, Kd, epi, status);
+      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_umma<TA, true, E>), grid, kUmmaThreads, smem, st, A_, lda, ws + wpk, Mr, N, Kd, epi, status);
     } else {
       smem_limit(k_gemm_umma<TA, false, E>, smem);
-      hk.launch((k_gemm_umma<TA, false, E>), grid, kUmmaThreads, smem, st, A_, lda, ws + wpk, Mr, N, Kd, epi, status);
+      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_umma<TA, false, E>), grid, kUmmaThreads, smem, st, A_, lda, ws + wpk, Mr, N, Kd, epi, status);
     }
   };
   // the conditioning-modulated row norm of x (or x') fused into a projection's operand
@@ -518,9 +571,9 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     const bool reg = C % 4 == 0 && S % 4 == 0 && C <= 256 && S <= 256 &&
                      ((reinterpret_cast<uintptr_t>(in->atom.data) | reinterpret_cast<uintptr_t>(in->condition.data)) & al) == 0;
     if (reg)
-      hk.launch((k_rows_prep_reg<Elt>), row_blocks, 256, 0, st, ra);
+      hk.launch(ATOMENC_KERNEL_ROWS, (k_rows_prep_reg<Elt>), row_blocks, 256, 0, st, ra);
     else
-      hk.launch((k_rows_prep<Elt>), row_blocks, 256, 0, st, ra);
+      hk.launch(ATOMENC_KERNEL_ROWS, (k_rows_prep<Elt>), row_blocks, 256, 0, st, ra);
   }
   hk.mark(1, st);
 
@@ -536,7 +589,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   hk.mark(2, st);
   if (!fuse_norm) {
     FeatArgs fa{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_x), F(pl.o_cond), F(pl.o_feat)};
-    hk.launch(k_features, row_blocks, 256, 0, st, fa);
+    hk.launch(ATOMENC_KERNEL_ROWS, k_features, row_blocks, 256, 0, st, fa);
   }
 
   // ---- projections (attention inputs fused into the operand when C <= 256)
@@ -559,10 +612,10 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     RopeArgs rp{R, H, D, eps, usable, in->rope_cos.data, in->rope_sin.data, F(pl.o_q), F(pl.o_k)};
     if (D >= 8 && D <= 128 && (D & (D - 1)) == 0) {
       const int64_t warps = R * 2;
-      hk.launch((k_qk_rope_warp<Elt>), (unsigned)((warps + 7) / 8), 256, 0, st, rp);
+      hk.launch(ATOMENC_KERNEL_ROWS, (k_qk_rope_warp<Elt>), (unsigned)((warps + 7) / 8), 256, 0, st, rp);
     } else {
       const int64_t n = R * H * 2;
-      hk.launch((k_qk_rope<Elt>), (unsigned)((n + 255) / 256), 256, 0, st, rp);
+      hk.launch(ATOMENC_KERNEL_ROWS, (k_qk_rope<Elt>), (unsigned)((n + 255) / 256), 256, 0, st, rp);
     }
   }
   hk.mark(3, st);
@@ -588,7 +641,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     dim3 grid((unsigned)((A + pl.QT - 1) / pl.QT), (unsigned)B);
     auto go = [&](auto kern) {
       smem_limit(kern, pl.attn_smem);
-      hk.launch(kern, grid, attn_threads(pl.af3), pl.attn_smem, st, ag);
+      hk.launch(ATOMENC_KERNEL_ATTENTION, kern, grid, attn_threads(pl.af3), pl.attn_smem, st, ag);
     };
     const int dm = D <= 8 ? 8 : D <= 16 ? 16 : D <= 32 ? 32 : 64;
     const bool multi = K > kChunk;
@@ -622,11 +675,16 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     ta.w_out = ws + pl.k_out; ta.w_ff1 = ws + pl.k_ff1; ta.w_ff2 = ws + pl.k_ff2;
     ta.hid32 = split ? nullptr : F(pl.o_hid); ta.hidden = out->hidden.data; ta.status = status;
     ta.xfer = F(pl.o_xfer); ta.xflag = reinterpret_cast<int *>(ws + pl.o_xflag);
+    ta.peer_spin_limit = g_peer_spin_limit.load();
+    ta.withhold_flag = g_peer_withhold.load();
     const size_t smem = trans_smem_bytes(split);
     const dim3 grid((unsigned)(((R + kUmmaBM - 1) / kUmmaBM) * (pl.tail_pair ? 2 : 1)));
+    // the two CTAs of a row block exchange partials: launched as a 2-CTA cluster, so
+    // that they are always resident at the same time
     auto go = [&](auto kern) {
       smem_limit(kern, smem);
-      hk.launch(kern, grid, kTransThreads, smem, st, ta);
+      hk.launch_cluster(ATOMENC_KERNEL_TRANSITION, pl.tail_pair ? 2 : 1, kern, grid, kTransThreads,
+                        smem, st, ta);
     };
     if (split)
       pl.tail_pair ? go(k_transition<true, Elt, true>) : go(k_transition<true, Elt, false>);
@@ -636,7 +694,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     gemm(F(pl.o_o), HD, pl.k_out, R, C, HD,
          Quad<EpiResidual>{{F(pl.o_x), gbuf, gld, g0off, C, F(pl.o_xp)}});
     TNormArgs tn{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_xp), F(pl.o_cond), F(pl.o_z)};
-    hk.launch(k_transition_norm, row_blocks, 256, 0, st, tn);
+    hk.launch(ATOMENC_KERNEL_ROWS, k_transition_norm, row_blocks, 256, 0, st, tn);
     gemm(F(pl.o_z), C, pl.k_ff1, R, 2 * M, C, EpiSwiGLU{F(pl.o_h), M});
     gemm(F(pl.o_h), M, pl.k_ff2, R, C, M,
          Quad<EpiHidden<Elt>>{{F(pl.o_xp), gbuf, gld, g1off, C, usable, F(pl.o_hid),
@@ -651,11 +709,11 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     gemm(hid, C, pl.k_pool, R, U, C, Quad<EpiRelu>{{F(pl.o_pool), U}});
     PoolArgs pa{B, A, T, U, usable, static_cast<const int64_t *>(in->atom_to_token.data), first,
                 last, F(pl.o_pool), out->token_output.data};
-    hk.launch((k_token_mean<Elt>), (unsigned)(B * T), kPoolThreads, 0, st, pa);
+    hk.launch(ATOMENC_KERNEL_POOL, (k_token_mean<Elt>), (unsigned)(B * T), kPoolThreads, 0, st, pa);
   } else {
     ReadoutArgs rd{R, C, eps, pl.af3 ? 0 : 1, usable, hid, F(pl.o_rscale), F(pl.o_rbias),
                    F(pl.o_wread), out->position_update.data};
-    hk.launch((k_readout<Elt>), row_blocks, 256, 0, st, rd);
+    hk.launch(ATOMENC_KERNEL_ROWS, (k_readout<Elt>), row_blocks, 256, 0, st, rd);
   }
   hk.mark(6, st);
   if (hk.err != cudaSuccess) return ATOMENC_ERR_CUDA;
@@ -688,6 +746,7 @@ static int forward_impl(int style, int stage, const atomenc_inputs *in,
     return ATOMENC_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   unsigned char *ws = static_cast<unsigned char *>(workspace);
+  hk.begin(st);
   if (pl.fdt == ATOMENC_F32) return launch_all<float>(pl, in, params, feps, radius, out, ws, st, hk);
   return launch_all<__nv_bfloat16>(pl, in, params, feps, radius, out, ws, st, hk);
 }
@@ -714,6 +773,31 @@ int atomenc_forward_profiled(int style, int stage, const atomenc_inputs *in,
                         stream, hk);
   if (n_launches) *n_launches = hk.launches;
   return rc;
+}
+
+int atomenc_forward_traced(int style, int stage, const atomenc_inputs *in,
+                           const atomenc_params *params, double eps, int64_t radius,
+                           const atomenc_outputs *out, void *workspace, size_t workspace_bytes,
+                           atomenc_stream_t stream, void *const *events, int n_events,
+                           int *kinds, int *n_launches) {
+  if (!events || n_events < 2) return ATOMENC_ERR_NULL;
+  for (int i = 0; i < n_events; ++i)
+    if (!events[i]) return ATOMENC_ERR_NULL;
+  Hooks hk;
+  hk.kev = reinterpret_cast<cudaEvent_t const *>(events);
+  hk.n_kev = n_events;
+  hk.kinds = kinds;
+  int rc = forward_impl(style, stage, in, params, eps, radius, out, workspace, workspace_bytes,
+                        stream, hk);
+  if (n_launches) *n_launches = hk.launches;
+  if (rc == ATOMENC_OK && hk.overflow) return ATOMENC_ERR_NULL;
+  return rc;
+}
+
+int atomenc_debug_peer_wait(uint32_t poll_limit, int withhold_flags) {
+  g_peer_spin_limit.store(poll_limit == 0 ? kPeerSpinLimit : poll_limit);
+  g_peer_withhold.store(withhold_flags ? 1 : 0);
+  return ATOMENC_OK;
 }
 
 // ---- no-allocation variant: scratch in a file-scope device array, address looked up
@@ -747,6 +831,13 @@ int atomenc_forward_noalloc(int style, int stage, const atomenc_inputs *in,
   Hooks hk;
   return forward_impl(style, stage, in, params, eps, radius, out, scratch,
                       ATOMENC_NOALLOC_SCRATCH_BYTES, stream, hk);
+}
+
+int atomenc_noalloc_get_status(int *device_status, atomenc_stream_t stream) {
+  if (!device_status) return ATOMENC_ERR_NULL;
+  void *scratch = nullptr;
+  CHECK(noalloc_scratch(&scratch));
+  return atomenc_get_status(scratch, device_status, stream);
 }
 
 int atomenc_get_status(const void *workspace, int *device_status, atomenc_stream_t stream) {

@@ -53,6 +53,9 @@ struct TransArgs {
   // of the half of the columns the other CTA finishes go through global scratch
   float *xfer;                 // [row blocks][2][128][64] partial columns
   int *xflag;                  // [row blocks][2], zero at entry
+  uint32_t peer_spin_limit;    // polls of the peer's flag before giving up (status bit 4)
+  int withhold_flag;           // test hook: never raise this CTA's flag (the peer's wait
+                               // then runs out); 0 in normal use
 };
 
 constexpr int kTransSlotsSplit = 3, kTransSlotsPlain = 6;   // weight ring depth
@@ -108,8 +111,10 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *p, int64_t 
   *reinterpret_cast<uint2 *>(p + i) = make_uint2(lo, hi);
 }
 
-// the CTA pair's flags (global memory, GPU scope); a poll gives up after kPeerSpinLimit
-// reads (status bit 4), so a missing peer cannot hang the kernel
+// the CTA pair's flags (global memory, GPU scope); the pair is launched as a 2-CTA
+// cluster, so both CTAs are resident together, and a poll still gives up after
+// peer_spin_limit reads (default kPeerSpinLimit; status bit 4), so a missing peer cannot
+// hang the kernel
 constexpr uint32_t kPeerSpinLimit = 1u << 22;
 __device__ __forceinline__ int ld_acquire(const int *p) {
   int v;
@@ -318,7 +323,7 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
         }
       }
       epi_sync();
-      if (warp == 0 && lane == 0) {
+      if (warp == 0 && lane == 0 && !t.withhold_flag) {
         __threadfence();
         atomicExch(t.xflag + pb * 2 + rank, 1);
       }
@@ -326,7 +331,7 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
         int got = 1;
         if (lane == 0) {
           got = 0;
-          for (uint32_t it = 0; it < kPeerSpinLimit && !got; ++it)
+          for (uint32_t it = 0; it < t.peer_spin_limit && !got; ++it)
             got = ld_acquire(t.xflag + pb * 2 + (1 - rank));
         }
         got = __shfl_sync(0xffffffffu, got, 0);

@@ -23,7 +23,7 @@ def _tensor_bytes(spec):
     if spec.style == "af3":
         n += w["activations"]["pair"].size * s
     n += rows                                  # usable flags
-    n += 4 * rows * hd * 4 + rows * hd * 4     # Q, K, V, G read; gated output written
+    n += 4 * rows * hd * s + rows * hd * s     # Q, K, V, G read; gated output written
     n += spec.B * spec.H * spec.A * spec.K * s  # attention weights written
     return n
 
@@ -34,6 +34,26 @@ def test_attention_bytes_match_the_tensors():
         assert bench.attention_bytes(spec) == _tensor_bytes(spec)
     spec = workloads.tiny_spec("af3", "encoder", "bfloat16")
     assert bench.attention_bytes(spec) == _tensor_bytes(spec)
+
+
+def test_attention_bytes_of_the_headline_workload():
+    """The survey's per-launch figure for the ESMFold2 bf16 workload (B=2, A=32768, H=8,
+    K=128): 75.5 MB of key_index + window_mask, 134.2 MB of weights, 84.0 MB of Q/K/V/G/O
+    and usable flags."""
+    spec = workloads.WORKLOADS["esm_encoder_bf16_b2_a32768"]
+    assert bench.attention_bytes(spec) == 75_497_472 + 134_217_728 + 83_951_616
+
+
+def test_dense_flops_per_atom():
+    spec = workloads.WORKLOADS["esm_encoder_bf16_b2_a32768"]
+    assert bench.dense_flops(spec) == 851_968 * spec.B * spec.A
+    dec = workloads.WORKLOADS["af3_decoder_fp32_a24576"]
+    per_atom = 2 * 128 * 8 * 128 + 2 * 128 * 512 + 2 * 128 * 128 + 2 * 128 * 512 + 2 * 256 * 128 + 2 * 128 * 3
+    assert bench.dense_flops(dec) == per_atom * dec.A + 2 * 384 * 128 * dec.T
+
+
+def test_default_workload_is_the_largest():
+    assert bench.DEFAULT_WORKLOAD == max(workloads.WORKLOADS.values(), key=lambda w: w.entries).name
 
 
 def test_recorded_traffic_is_keyed_by_workload_and_source():
@@ -55,6 +75,7 @@ def test_reference_arm_prints_one_json_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "atoms/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert d["config"]["workload"] == "af3_encoder_fp32_a256"
     assert np.isfinite(d["ms_per_step"])

@@ -8,8 +8,8 @@ import pytest
 import torch
 
 from sparse_windowed_atom_b200 import atomenc, workloads
-from tests.cuda_harness import (TOL, compare, exact_zero_pattern, run_cuda, run_oracle,
-                                sample_queries, to_torch)
+from tests.cuda_harness import (TOL, assert_status_clean, compare, exact_zero_pattern, run_cuda,
+                                run_oracle, sample_queries, to_torch)
 from tests.oracle_cases import load_golden
 
 pytestmark = pytest.mark.gpu
@@ -73,6 +73,7 @@ def test_wide_random_keys_take_the_unstaged_path():
     atomenc.atomenc_forward("esmfold2", "encoder", {**act, **msk, **st}, prm, spec.eps,
                             spec.radius, outs, ws)
     assert atomenc.atomenc_get_status(ws) & 1
+    assert_status_clean(ws, "unstaged keys")
     _check(w, "unstaged keys")
 
 
@@ -200,6 +201,7 @@ def test_prepared_forward_matches_the_plain_call(style):
             v.fill_(7.0)
         fwd()
         torch.cuda.synchronize()
+        assert_status_clean(ws, "prepared forward")
         for k in ref:
             assert torch.equal(outs[k], ref[k]), k
 

@@ -46,11 +46,14 @@ def test_noalloc_matches_workspace_entry_point(style, stage, dtype):
     ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     atomenc.atomenc_forward(style, stage, inputs, params, spec.eps, spec.radius, ref, ws)
     torch.cuda.synchronize()
+    assert not atomenc.atomenc_get_status(ws) & atomenc.STATUS_WAIT_TIMEOUT
     tol = TOL[dtype]
     for call in range(2):   # two calls in a row share the library's scratch array
         out = {k: torch.full(s, float("nan"), dtype=fdt, device="cuda") for k, s in shapes.items()}
         atomenc.atomenc_forward_noalloc(style, stage, inputs, params, spec.eps, spec.radius, out)
         torch.cuda.synchronize()
+        st = atomenc.atomenc_noalloc_get_status()
+        assert not st & atomenc.STATUS_WAIT_TIMEOUT, f"call {call}: device status {st:#x}"
         for k in shapes:
             r, g = ref[k].double(), out[k].double()
             assert torch.isfinite(g).all(), (call, k)
