@@ -17,6 +17,7 @@
 
 #include "../../include/atomenc.h"
 #include "attention.cuh"
+#include "attn_rows.cuh"
 #include "common.cuh"
 #include "epilogues.cuh"
 #include "gemm_umma.cuh"
@@ -31,6 +32,7 @@ namespace {
 constexpr int kVersion = 1;
 constexpr int kMaxD = 64;
 constexpr size_t kAttnSmemBudget = 210 * 1024;  // dynamic part: one CTA per SM, or per two (AF3) / 2 - 1 KB
+constexpr size_t kRowAttnSmemBudget = 220 * 1024;  // dynamic part of the row-gather attention
 
 struct Dims {
   int64_t B = 0, A = 0, T = 0, K = 0, C = 0, S = 0, H = 0, D = 0, P = 0, M = 0, U = 0, V = 0;
@@ -99,6 +101,12 @@ struct Plan {
   int QT = 0, DP = 0, kv_floats = 0;
   size_t attn_smem = 0;
   int sms = 148;                    // multiprocessors of the device the pass runs on
+  // row-gather attention (k_attn_rows): H*D in {64, 128} ... see attn_rows.cuh; Q, K, V,
+  // value-gate logits and the gated output are then kept in the storage type
+  bool rg = false;
+  int rg_qt = 0, rg_stage_rows = 0;
+  size_t rg_smem = 0;
+  bool ws_bf16 = false;             // Q/K/V/G/O intermediates in bf16
 };
 
 size_t take(size_t &cur, size_t bytes) {
@@ -107,8 +115,10 @@ size_t take(size_t &cur, size_t bytes) {
   return o;
 }
 
+// radius_hint: the pass's radius, when known (it only steers the attention tile size;
+// the workspace size does not depend on it)
 int validate(int style, int stage, const atomenc_inputs *in, const atomenc_params *p,
-             const atomenc_outputs *out, Plan &pl) {
+             const atomenc_outputs *out, Plan &pl, int64_t radius_hint = -1) {
   if (!in || !p || !out) return ATOMENC_ERR_NULL;
   if (style != ATOMENC_AF3 && style != ATOMENC_ESMFOLD2) return ATOMENC_ERR_STYLE;
   if (stage != ATOMENC_DECODER && stage != ATOMENC_ENCODER) return ATOMENC_ERR_STYLE;
@@ -237,11 +247,20 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   pl.o_gate = take(cur, pl.af3 ? R * 2 * C * 4 : 0);
   const bool fused = C <= kRowsKMax;
   pl.o_feat = take(cur, fused ? 0 : R * (pl.af3 ? 2 : 1) * C * 4);
-  pl.o_q = take(cur, R * HD * 4);
-  pl.o_k = take(cur, R * HD * 4);
-  pl.o_v = take(cur, R * HD * 4);
-  pl.o_g = take(cur, R * HD * 4);
-  pl.o_o = take(cur, R * HD * 4);
+  // row-gather attention: whole rows of all heads per quarter-warp (H*D == 128, a head
+  // spans a whole number of lanes, at most 8 heads, K <= 128)
+  {
+    const int64_t lc = HD / 8;
+    pl.rg = HD == 128 && D >= lc && D % lc == 0 && HD / D <= kRowAttnHeadsMax &&
+            K <= kRowAttnKMax && (!pl.af3 || P <= kRowAttnPairMax);
+    pl.ws_bf16 = pl.rg && fdt == ATOMENC_BF16;
+  }
+  const int64_t wsz = pl.ws_bf16 ? 2 : 4;   // bytes per Q/K/V/G/O element
+  pl.o_q = take(cur, R * HD * wsz);
+  pl.o_k = take(cur, R * HD * wsz);
+  pl.o_v = take(cur, R * HD * wsz);
+  pl.o_g = take(cur, R * HD * wsz);
+  pl.o_o = take(cur, R * HD * wsz);
   // the fused tail (out-projection .. hidden in one kernel) keeps x', z and the SwiGLU
   // intermediate on chip
   pl.fuse_tail = C == 128 && (HD == 64 || HD == 128) && M % 128 == 0;
@@ -303,6 +322,28 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   pl.QT = qt;
   pl.kv_floats = (int)((budget - fixed) / 4);
   pl.attn_smem = fixed + (size_t)pl.kv_floats * 4;
+
+  if (pl.rg) {
+    // queries per CTA: the largest power of two (<= 64, and small enough that the grid
+    // covers the SMs) whose shared K/V stage holds the expected key span: the tile plus
+    // 2 radius + 1 rows with an index window, the tile plus K otherwise
+    const int es = (int)wsz, rb = (int)(HD * es);
+    const int64_t fill = (B * A + pl.sms - 1) / pl.sms;
+    int q = 64;
+    while (q > 1 && q > fill) q /= 2;
+    auto rows_cap = [&](int qq) -> int64_t {
+      const size_t fx = rowattn_fixed_smem(qq, (int)K, (int)H, es, pl.af3);
+      return fx >= kRowAttnSmemBudget ? 0 : (int64_t)((kRowAttnSmemBudget - fx) / (2 * (size_t)rb));
+    };
+    auto need = [&](int qq) -> int64_t {
+      return radius_hint >= 0 ? qq + 2 * radius_hint + 1 : qq + K;
+    };
+    while (q > 1 && rows_cap(q) < need(q)) q /= 2;
+    if (rows_cap(q) < 1) return ATOMENC_ERR_UNSUPPORTED;
+    pl.rg_qt = q;
+    pl.rg_stage_rows = (int)rows_cap(q);
+    pl.rg_smem = rowattn_fixed_smem(q, (int)K, (int)H, es, pl.af3) + 2 * (size_t)pl.rg_stage_rows * rb;
+  }
   return ATOMENC_OK;
 }
 
@@ -592,59 +633,101 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     hk.launch(ATOMENC_KERNEL_ROWS, k_features, row_blocks, 256, 0, st, fa);
   }
 
-  // ---- projections (attention inputs fused into the operand when C <= 256)
-  if (pl.af3) {
-    EpiSplit e0{{F(pl.o_q), F(pl.o_g), nullptr, nullptr}, {F(pl.o_bq), nullptr, nullptr, nullptr}, HD};
-    EpiSplit e1{{F(pl.o_k), F(pl.o_v), nullptr, nullptr}, {nullptr, nullptr, nullptr, nullptr}, HD};
-    if (fuse_norm) {
-      gemm_rows(norm_prod(0, C, false), pl.k_qkv0, R, 2 * HD, C, e0);
-      gemm_rows(norm_prod(2 * C, 3 * C, false), pl.k_qkv1, R, 2 * HD, C, e1);
+  // ---- projections .. transition; WT is the type of the Q/K/V/G/O intermediates
+  // (bf16 for bf16 workloads on the row-gather attention, float32 otherwise)
+  auto middle = [&](auto wt_tag) {
+    using WT = decltype(wt_tag);
+    WT *wq = reinterpret_cast<WT *>(ws + pl.o_q), *wk = reinterpret_cast<WT *>(ws + pl.o_k),
+       *wv = reinterpret_cast<WT *>(ws + pl.o_v), *wg = reinterpret_cast<WT *>(ws + pl.o_g),
+       *wo = reinterpret_cast<WT *>(ws + pl.o_o);
+    // ---- projections (attention inputs fused into the operand when C <= 256)
+    if (pl.af3) {
+      EpiSplitT<WT> e0{{wq, wg, nullptr, nullptr}, {F(pl.o_bq), nullptr, nullptr, nullptr}, HD};
+      EpiSplitT<WT> e1{{wk, wv, nullptr, nullptr}, {nullptr, nullptr, nullptr, nullptr}, HD};
+      if (fuse_norm) {
+        gemm_rows(norm_prod(0, C, false), pl.k_qkv0, R, 2 * HD, C, e0);
+        gemm_rows(norm_prod(2 * C, 3 * C, false), pl.k_qkv1, R, 2 * HD, C, e1);
+      } else {
+        gemm(F(pl.o_feat), 2 * C, pl.k_qkv0, R, 2 * HD, C, e0);
+        gemm(F(pl.o_feat) + C, 2 * C, pl.k_qkv1, R, 2 * HD, C, e1);
+      }
     } else {
-      gemm(F(pl.o_feat), 2 * C, pl.k_qkv0, R, 2 * HD, C, e0);
-      gemm(F(pl.o_feat) + C, 2 * C, pl.k_qkv1, R, 2 * HD, C, e1);
+      EpiSplitT<WT> e{{wq, wk, wv, wg}, {nullptr, nullptr, nullptr, nullptr}, HD};
+      if (fuse_norm)
+        gemm_rows(norm_prod(C, 0, true), pl.k_qkv0, R, 4 * HD, C, e);
+      else
+        gemm(F(pl.o_feat), C, pl.k_qkv0, R, 4 * HD, C, e);
+      RopeArgs rp{R, H, D, eps, usable, in->rope_cos.data, in->rope_sin.data, wq, wk};
+      if (D >= 8 && D <= 128 && (D & (D - 1)) == 0) {
+        const int64_t warps = R * 2;
+        hk.launch(ATOMENC_KERNEL_ROWS, (k_qk_rope_warp<Elt, WT>), (unsigned)((warps + 7) / 8), 256, 0, st, rp);
+      } else {
+        const int64_t n = R * H * 2;
+        hk.launch(ATOMENC_KERNEL_ROWS, (k_qk_rope<Elt>), (unsigned)((n + 255) / 256), 256, 0, st, rp);
+      }
     }
-  } else {
-    EpiSplit e{{F(pl.o_q), F(pl.o_k), F(pl.o_v), F(pl.o_g)}, {nullptr, nullptr, nullptr, nullptr}, HD};
-    if (fuse_norm)
-      gemm_rows(norm_prod(C, 0, true), pl.k_qkv0, R, 4 * HD, C, e);
-    else
-      gemm(F(pl.o_feat), C, pl.k_qkv0, R, 4 * HD, C, e);
-    RopeArgs rp{R, H, D, eps, usable, in->rope_cos.data, in->rope_sin.data, F(pl.o_q), F(pl.o_k)};
-    if (D >= 8 && D <= 128 && (D & (D - 1)) == 0) {
-      const int64_t warps = R * 2;
-      hk.launch(ATOMENC_KERNEL_ROWS, (k_qk_rope_warp<Elt>), (unsigned)((warps + 7) / 8), 256, 0, st, rp);
-    } else {
-      const int64_t n = R * H * 2;
-      hk.launch(ATOMENC_KERNEL_ROWS, (k_qk_rope<Elt>), (unsigned)((n + 255) / 256), 256, 0, st, rp);
-    }
-  }
-  hk.mark(3, st);
+    hk.mark(3, st);
 
-  // ---- slot-gathered attention
-  AttnArgs ag;
-  ag.B = (int)B; ag.A = (int)A; ag.K = (int)K; ag.H = (int)H; ag.D = (int)D; ag.P = (int)P;
-  ag.radius = radius < 0 ? -1 : (radius > INT_MAX ? INT_MAX : (int)radius);
-  ag.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-  ag.eps = eps;
-  ag.QT = pl.QT; ag.DP = pl.DP; ag.kv_floats = pl.kv_floats;
-  ag.kmagic = K > 1 ? (uint32_t)(((uint64_t)1 << 32) / (uint64_t)K + (((uint64_t)1 << 32) % (uint64_t)K != 0)) : 0u;
-  ag.Q = F(pl.o_q); ag.Kf = F(pl.o_k); ag.Vf = F(pl.o_v); ag.G = F(pl.o_g);
-  ag.key_index = static_cast<const int64_t *>(in->key_index.data);
-  ag.window = static_cast<const uint8_t *>(in->window_mask.data);
-  ag.usable = usable;
-  ag.pair = pl.af3 ? in->pair.data : nullptr;
-  ag.w_pair = F(pl.o_wpair);
-  ag.attention = out->attention.data;
-  ag.O = F(pl.o_o);
-  ag.status = status;
-  {
-    dim3 grid((unsigned)((A + pl.QT - 1) / pl.QT), (unsigned)B);
-    auto go = [&](auto kern) {
-      smem_limit(kern, pl.attn_smem);
-      hk.launch(ATOMENC_KERNEL_ATTENTION, kern, grid, attn_threads(pl.af3), pl.attn_smem, st, ag);
-    };
-    const int dm = D <= 8 ? 8 : D <= 16 ? 16 : D <= 32 ? 32 : 64;
-    const bool multi = K > kChunk;
+    // ---- slot-gathered attention
+    const int rad = radius < 0 ? -1 : (radius > INT_MAX ? INT_MAX : (int)radius);
+    if (pl.rg) {
+      RowAttnArgs ra2;
+      ra2.B = (int)B; ra2.A = (int)A; ra2.K = (int)K; ra2.H = (int)H; ra2.D = (int)D; ra2.P = (int)P;
+      ra2.radius = rad;
+      ra2.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+      ra2.eps = eps;
+      ra2.QT = pl.rg_qt;
+      ra2.stage_rows = pl.rg_stage_rows;
+      ra2.Q = wq; ra2.Kf = wk; ra2.Vf = wv; ra2.G = wg;
+      ra2.key_index = static_cast<const int64_t *>(in->key_index.data);
+      ra2.window = static_cast<const uint8_t *>(in->window_mask.data);
+      ra2.usable = usable;
+      ra2.pair = pl.af3 ? in->pair.data : nullptr;
+      ra2.w_pair = F(pl.o_wpair);
+      ra2.attention = out->attention.data;
+      ra2.O = wo;
+      ra2.status = status;
+      ra2.pair_vec = pl.af3 && P == 16 && (reinterpret_cast<uintptr_t>(in->pair.data) & 15) == 0;
+      ra2.att_vec = (reinterpret_cast<uintptr_t>(out->attention.data) & 15) == 0;
+      dim3 grid((unsigned)((A + pl.rg_qt - 1) / pl.rg_qt), (unsigned)B);
+      auto go = [&](auto kern) {
+        smem_limit(kern, pl.rg_smem);
+        hk.launch(ATOMENC_KERNEL_ATTENTION, kern, grid, kRowAttnThreads, pl.rg_smem, st, ra2);
+      };
+      // the attention weights are written in the storage type: WT == Elt here
+      if constexpr (std::is_same<WT, Elt>::value) {
+#define ROWATTN(DH)                                                 \
+  if (D == DH) {                                                    \
+    if (pl.af3) go(k_attn_rows<WT, 128, DH, true>);                 \
+    else go(k_attn_rows<WT, 128, DH, false>);                       \
+  }
+        ROWATTN(16) ROWATTN(32) ROWATTN(64)
+#undef ROWATTN
+      }
+    } else {
+      AttnArgs ag;
+      ag.B = (int)B; ag.A = (int)A; ag.K = (int)K; ag.H = (int)H; ag.D = (int)D; ag.P = (int)P;
+      ag.radius = rad;
+      ag.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+      ag.eps = eps;
+      ag.QT = pl.QT; ag.DP = pl.DP; ag.kv_floats = pl.kv_floats;
+      ag.kmagic = K > 1 ? (uint32_t)(((uint64_t)1 << 32) / (uint64_t)K + (((uint64_t)1 << 32) % (uint64_t)K != 0)) : 0u;
+      ag.Q = F(pl.o_q); ag.Kf = F(pl.o_k); ag.Vf = F(pl.o_v); ag.G = F(pl.o_g);
+      ag.key_index = static_cast<const int64_t *>(in->key_index.data);
+      ag.window = static_cast<const uint8_t *>(in->window_mask.data);
+      ag.usable = usable;
+      ag.pair = pl.af3 ? in->pair.data : nullptr;
+      ag.w_pair = F(pl.o_wpair);
+      ag.attention = out->attention.data;
+      ag.O = F(pl.o_o);
+      ag.status = status;
+      dim3 grid((unsigned)((A + pl.QT - 1) / pl.QT), (unsigned)B);
+      auto go = [&](auto kern) {
+        smem_limit(kern, pl.attn_smem);
+        hk.launch(ATOMENC_KERNEL_ATTENTION, kern, grid, attn_threads(pl.af3), pl.attn_smem, st, ag);
+      };
+      const int dm = D <= 8 ? 8 : D <= 16 ? 16 : D <= 32 ? 32 : 64;
+      const bool multi = K > kChunk;
 #define ATTN_D(DM)                                                          \
   if (dm == DM) {                                                           \
     if (pl.af3)                                                             \
@@ -654,51 +737,61 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
       multi ? go(k_slot_attention<Elt, DM, false, true>)                    \
             : go(k_slot_attention<Elt, DM, false, false>);                  \
   }
-    ATTN_D(8) ATTN_D(16) ATTN_D(32) ATTN_D(64)
+      ATTN_D(8) ATTN_D(16) ATTN_D(32) ATTN_D(64)
 #undef ATTN_D
-  }
+    }
 
-  hk.mark(4, st);
+    hk.mark(4, st);
 
-  // ---- out-projection + gated residual, transition norm, SwiGLU, gated residual + mask
-  const float *gbuf = pl.af3 ? F(pl.o_gate) : F(pl.o_cond);
-  const int64_t gld = pl.af3 ? 2 * C : 6 * C;
-  const int64_t g0off = pl.af3 ? 0 : 2 * C, g1off = pl.af3 ? C : 5 * C;
-  if (pl.fuse_tail) {
-    TransArgs ta;
-    ta.R = R; ta.HD = (int)HD; ta.M = (int)M;
-    ta.O = F(pl.o_o); ta.x = F(pl.o_x);
-    ta.g0 = gbuf + g0off; ta.g1 = gbuf + g1off; ta.g_ld = gld;
-    ta.sc = F(pl.o_cond) + 4 * C; ta.sh = F(pl.o_cond) + (pl.af3 ? 5 : 3) * C; ta.cond_ld = 6 * C;
-    ta.rms = pl.af3 ? 0 : 1; ta.plus1 = pl.af3 ? 0 : 1; ta.eps = eps;
-    ta.usable = usable;
-    ta.w_out = ws + pl.k_out; ta.w_ff1 = ws + pl.k_ff1; ta.w_ff2 = ws + pl.k_ff2;
-    ta.hid32 = split ? nullptr : F(pl.o_hid); ta.hidden = out->hidden.data; ta.status = status;
-    ta.xfer = F(pl.o_xfer); ta.xflag = reinterpret_cast<int *>(ws + pl.o_xflag);
-    ta.peer_spin_limit = g_peer_spin_limit.load();
-    ta.withhold_flag = g_peer_withhold.load();
-    const size_t smem = trans_smem_bytes(split);
-    const dim3 grid((unsigned)(((R + kUmmaBM - 1) / kUmmaBM) * (pl.tail_pair ? 2 : 1)));
-    // the two CTAs of a row block exchange partials: launched as a 2-CTA cluster, so
-    // that they are always resident at the same time
-    auto go = [&](auto kern) {
-      smem_limit(kern, smem);
-      hk.launch_cluster(ATOMENC_KERNEL_TRANSITION, pl.tail_pair ? 2 : 1, kern, grid, kTransThreads,
-                        smem, st, ta);
-    };
-    if (split)
-      pl.tail_pair ? go(k_transition<true, Elt, true>) : go(k_transition<true, Elt, false>);
+    // ---- out-projection + gated residual, transition norm, SwiGLU, gated residual + mask
+    const float *gbuf = pl.af3 ? F(pl.o_gate) : F(pl.o_cond);
+    const int64_t gld = pl.af3 ? 2 * C : 6 * C;
+    const int64_t g0off = pl.af3 ? 0 : 2 * C, g1off = pl.af3 ? C : 5 * C;
+    if (pl.fuse_tail) {
+      TransArgs ta;
+      ta.R = R; ta.HD = (int)HD; ta.M = (int)M;
+      ta.O = wo; ta.x = F(pl.o_x);
+      ta.g0 = gbuf + g0off; ta.g1 = gbuf + g1off; ta.g_ld = gld;
+      ta.sc = F(pl.o_cond) + 4 * C; ta.sh = F(pl.o_cond) + (pl.af3 ? 5 : 3) * C; ta.cond_ld = 6 * C;
+      ta.rms = pl.af3 ? 0 : 1; ta.plus1 = pl.af3 ? 0 : 1; ta.eps = eps;
+      ta.usable = usable;
+      ta.w_out = ws + pl.k_out; ta.w_ff1 = ws + pl.k_ff1; ta.w_ff2 = ws + pl.k_ff2;
+      ta.hid32 = split ? nullptr : F(pl.o_hid); ta.hidden = out->hidden.data; ta.status = status;
+      ta.xfer = F(pl.o_xfer); ta.xflag = reinterpret_cast<int *>(ws + pl.o_xflag);
+      ta.peer_spin_limit = g_peer_spin_limit.load();
+      ta.withhold_flag = g_peer_withhold.load();
+      const size_t smem = trans_smem_bytes(split);
+      const dim3 grid((unsigned)(((R + kUmmaBM - 1) / kUmmaBM) * (pl.tail_pair ? 2 : 1)));
+      // the two CTAs of a row block exchange partials: launched as a 2-CTA cluster, so
+      // that they are always resident at the same time
+      auto go = [&](auto kern) {
+        smem_limit(kern, smem);
+        hk.launch_cluster(ATOMENC_KERNEL_TRANSITION, pl.tail_pair ? 2 : 1, kern, grid, kTransThreads,
+                          smem, st, ta);
+      };
+      if constexpr (std::is_same<Elt, float>::value) {
+        pl.tail_pair ? go(k_transition<true, Elt, true, WT>) : go(k_transition<true, Elt, false, WT>);
+      } else {
+        pl.tail_pair ? go(k_transition<false, Elt, true, WT>) : go(k_transition<false, Elt, false, WT>);
+      }
+    } else {
+      gemm(static_cast<const WT *>(wo), HD, pl.k_out, R, C, HD,
+           Quad<EpiResidual>{{F(pl.o_x), gbuf, gld, g0off, C, F(pl.o_xp)}});
+      TNormArgs tn{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_xp), F(pl.o_cond), F(pl.o_z)};
+      hk.launch(ATOMENC_KERNEL_ROWS, k_transition_norm, row_blocks, 256, 0, st, tn);
+      gemm(F(pl.o_z), C, pl.k_ff1, R, 2 * M, C, EpiSwiGLU{F(pl.o_h), M});
+      gemm(F(pl.o_h), M, pl.k_ff2, R, C, M,
+           Quad<EpiHidden<Elt>>{{F(pl.o_xp), gbuf, gld, g1off, C, usable, F(pl.o_hid),
+                                 static_cast<Elt *>(out->hidden.data)}});
+    }
+  };
+  if constexpr (std::is_same<Elt, __nv_bfloat16>::value) {
+    if (pl.ws_bf16)
+      middle(__nv_bfloat16{});
     else
-      pl.tail_pair ? go(k_transition<false, Elt, true>) : go(k_transition<false, Elt, false>);
+      middle(float{});
   } else {
-    gemm(F(pl.o_o), HD, pl.k_out, R, C, HD,
-         Quad<EpiResidual>{{F(pl.o_x), gbuf, gld, g0off, C, F(pl.o_xp)}});
-    TNormArgs tn{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_xp), F(pl.o_cond), F(pl.o_z)};
-    hk.launch(ATOMENC_KERNEL_ROWS, k_transition_norm, row_blocks, 256, 0, st, tn);
-    gemm(F(pl.o_z), C, pl.k_ff1, R, 2 * M, C, EpiSwiGLU{F(pl.o_h), M});
-    gemm(F(pl.o_h), M, pl.k_ff2, R, C, M,
-         Quad<EpiHidden<Elt>>{{F(pl.o_xp), gbuf, gld, g1off, C, usable, F(pl.o_hid),
-                               static_cast<Elt *>(out->hidden.data)}});
+    middle(float{});
   }
 
   hk.mark(5, st);
@@ -736,7 +829,7 @@ static int forward_impl(int style, int stage, const atomenc_inputs *in,
                         const atomenc_outputs *out, void *workspace, size_t workspace_bytes,
                         atomenc_stream_t stream, Hooks &hk) {
   Plan pl;
-  CHECK(validate(style, stage, in, params, out, pl));
+  CHECK(validate(style, stage, in, params, out, pl, radius));
   if (!std::isfinite(eps) || !(eps > 0.0)) return ATOMENC_ERR_EPS;
   float feps = (float)eps;
   if (!(feps > 0.f) || !std::isfinite(feps)) return ATOMENC_ERR_EPS;

@@ -364,7 +364,7 @@ __global__ void __launch_bounds__(attn_threads(AF3), attn_ctas_per_sm(AF3)) k_sl
   if (AF3) {
     __syncthreads();
     const T *pbase = (const T *)g.pair + sbase * P;
-    const bool p16 = P == 16;
+    const bool p16 = P == 16 && (reinterpret_cast<uintptr_t>(g.pair) & 15) == 0;
     for (int s0 = tid; s0 < vslots; s0 += 2 * kAttnThreads) {
       const int s1 = s0 + kAttnThreads;
       const bool on0 = plan[s0] >= 0, on1 = s1 < vslots && plan[s1] >= 0;

@@ -1,0 +1,534 @@
+// attn_rows.cuh -- slot-gathered windowed attention, one warp per query over all heads.
+//
+// Page "Local atom attention, encoder pooling and decoder skip/readout", Required
+// behavior: a slot (query a, slot k) is permitted iff its key id j is in [0, A), both
+// atoms are usable, window_mask is set and, for radius >= 0, |j - a| <= radius (bullets
+// 4, 5); logits are Q_a . K_j / sqrt(D) plus, in AF3 style, the pair bias
+// (LN(pair) * pair_scale) @ w_pair (bullets 8, 15); a stabilised softmax runs over the
+// permitted slots only, a row without any gets exact zeros, repeated slots are separate
+// entries (bullets 5, 6, 15); the weighted values are multiplied by sigmoid of the value
+// gate logits and stored head-major (bullet 16).
+//
+// Layout and work split (H*D = HD in {64, 128}, D a multiple of HD / 8, K <= 128):
+//  * One CTA (512 threads, one per SM) owns QT consecutive queries of one batch element.
+//  * Before the wait for the projections (the inputs and the usable flags come from
+//    kernels at least two places earlier): warp w builds, for each of its queries, the
+//    compacted list of permitted slots (key id, slot index) with ballots, and the CTA's
+//    key span [klo, khi]; AF3: the pair bias of every listed slot for every head
+//    (LayerNorm over P in one shifted pass, folded pair_scale * w_pair) into a float32
+//    table in list order.
+//  * After the wait: the K and V rows of the span are staged in shared memory in the
+//    storage type, whole rows (all heads), each 16-byte chunk placed so that the eight
+//    lanes of a quarter-warp read one 128-byte segment of a row per load: lane i of
+//    every quarter-warp owns channels [HD/8 i, HD/8 (i + 1)) of the row (the same head
+//    for HD/8 / D of the lanes), so a gathered row never meets a bank conflict.
+//  * A warp takes one query: quarter-warp g takes list entries g, g + 4, ...; lane i
+//    forms the partial dot product of its channels, the lanes of a head combine theirs
+//    with xor-shuffles; logits stay in registers (log2 units), max and sum across the
+//    quarter-warps by shuffles, one exp2 per entry; weights go to a per-warp shared row
+//    buffer (zeros for slots that are not permitted) that is written out with 16-byte
+//    coalesced stores; the weighted value sum per lane, folded across the four
+//    quarter-warps by a reduce-scatter, is gated by sigmoid(value gate) and stored.
+// A span too wide for the shared stage is read from global memory (L2) instead with the
+// same lane mapping and sets status bit 1; the results are the same.
+#pragma once
+
+#include <climits>
+
+#include "common.cuh"
+
+namespace atomenc {
+
+constexpr int kRowAttnThreads = 512;
+constexpr int kRowAttnWarps = kRowAttnThreads / kWarp;
+constexpr int kRowAttnKMax = 128;                  // slots per query (list entries <= K)
+constexpr int kRowAttnIters = kRowAttnKMax / 4;     // list entries per quarter-warp
+constexpr int kRowAttnPairMax = 32;
+constexpr int kRowAttnHeadsMax = 8;
+
+struct RowAttnArgs {
+  int B, A, K, H, D, P;
+  int radius;                     // -1 = no index window
+  float scale_log2;               // log2(e) / sqrt(D)
+  float eps;
+  int QT;                         // queries per CTA
+  int stage_rows;                 // rows of K (and of V) the shared stage holds
+  const void *Q, *Kf, *Vf, *G;    // [B*A, HD] storage type
+  const int64_t *key_index;       // [B, A, K]
+  const uint8_t *window;          // [B, A, K]
+  const uint8_t *usable;          // [B*A]
+  const void *pair;               // [B, A, K, P] AF3
+  const float *w_pair;            // [P, H] = pair_scale[p] * w_pair[p, h]
+  void *attention;                // [B, H, A, K]
+  void *O;                        // [B*A, HD] gated attention output, storage type
+  unsigned *status;
+  int pair_vec;                   // pair rows may be read with 16-byte loads (P = 16, aligned)
+  int att_vec;                    // weight rows may be written with 16-byte stores (aligned)
+};
+
+// bytes of one per-warp weight row (K weights, 16-byte multiple, + 16 to spread banks)
+__host__ __device__ inline int rowattn_wrow_bytes(int K, int es) {
+  return ((K * es + 15) & ~15) + 16;
+}
+// shared bytes before the K/V stage: list keys, list slots, counts, (AF3) bias table,
+// per-warp weight rows; each region 128-byte aligned
+__host__ __device__ inline size_t rowattn_fixed_smem(int QT, int K, int H, int es, bool af3) {
+  auto r128 = [](size_t n) { return (n + 127) & ~size_t(127); };
+  size_t b = r128((size_t)QT * K * 4) + r128((size_t)QT * K) + r128((size_t)QT * 4);
+  if (af3) b += r128((size_t)QT * K * H * 4);
+  b += r128((size_t)kRowAttnWarps * H * rowattn_wrow_bytes(K, es));
+  return b;
+}
+
+namespace rowattn {
+
+// 16 bytes of a row -> floats (CH = 8 bf16 or 4 float32)
+__device__ __forceinline__ void unpack(const uint4 v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    f[2 * e] = __uint_as_float(w[e] << 16);
+    f[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void unpack(const uint4 v, float (&f)[4]) {
+  f[0] = __uint_as_float(v.x);
+  f[1] = __uint_as_float(v.y);
+  f[2] = __uint_as_float(v.z);
+  f[3] = __uint_as_float(v.w);
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <typename T>
+__device__ __forceinline__ void store_w(T *p, float w);
+template <>
+__device__ __forceinline__ void store_w<float>(float *p, float w) { *p = w; }
+template <>
+__device__ __forceinline__ void store_w<__nv_bfloat16>(__nv_bfloat16 *p, float w) {
+  const uint32_t u = __float_as_uint(w);
+  *reinterpret_cast<uint16_t *>(p) = (uint16_t)((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
+}
+
+// N consecutive channels of one row as floats, and the gated output store
+template <int N>
+__device__ __forceinline__ void ldn(const float *p, float (&v)[N]) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int c = 0; c < N; c += 4) {
+      const float4 x = *reinterpret_cast<const float4 *>(p + c);
+      v[c] = x.x; v[c + 1] = x.y; v[c + 2] = x.z; v[c + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < N; c += 2) {
+      const float2 x = *reinterpret_cast<const float2 *>(p + c);
+      v[c] = x.x; v[c + 1] = x.y;
+    }
+  }
+}
+template <int N>
+__device__ __forceinline__ void ldn(const __nv_bfloat16 *p, float (&v)[N]) {
+  static_assert(N % 2 == 0, "pairs");
+  if constexpr (N >= 8) {
+#pragma unroll
+    for (int c = 0; c < N; c += 8) {
+      float f[8];
+      unpack(*reinterpret_cast<const uint4 *>(p + c), f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[c + e] = f[e];
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < N; c += 2) {
+      const uint32_t u = *reinterpret_cast<const uint32_t *>(p + c);
+      v[c] = __uint_as_float(u << 16);
+      v[c + 1] = __uint_as_float(u & 0xFFFF0000u);
+    }
+  }
+}
+template <int N>
+__device__ __forceinline__ void stn(float *p, const float (&v)[N]) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int c = 0; c < N; c += 4) *reinterpret_cast<float4 *>(p + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+  } else {
+#pragma unroll
+    for (int c = 0; c < N; c += 2) *reinterpret_cast<float2 *>(p + c) = make_float2(v[c], v[c + 1]);
+  }
+}
+template <int N>
+__device__ __forceinline__ void stn(__nv_bfloat16 *p, const float (&v)[N]) {
+  uint32_t u[N / 2];
+#pragma unroll
+  for (int c = 0; c < N; c += 2) {
+    const uint32_t a = __float_as_uint(v[c]), b = __float_as_uint(v[c + 1]);
+    const uint32_t ha = (a + 0x7FFFu + ((a >> 16) & 1u)) >> 16;
+    const uint32_t hb = (b + 0x7FFFu + ((b >> 16) & 1u)) >> 16;
+    u[c / 2] = ha | (hb << 16);
+  }
+  if constexpr (N == 4) {
+    *reinterpret_cast<uint2 *>(p) = make_uint2(u[0], u[1]);
+  } else if constexpr (N == 2) {
+    *reinterpret_cast<uint32_t *>(p) = u[0];
+  } else {
+#pragma unroll
+    for (int c = 0; c < N / 2; c += 4) *reinterpret_cast<uint4 *>(p + 2 * c) = make_uint4(u[c], u[c + 1], u[c + 2], u[c + 3]);
+  }
+}
+
+// 16 pair channels of one slot by 16-byte loads (bf16: 2 loads, float32: 4 loads)
+__device__ __forceinline__ void ldpair16(const __nv_bfloat16 *pr, float (&x)[16]) {
+  float a[8], b[8];
+  unpack(*reinterpret_cast<const uint4 *>(pr), a);
+  unpack(*reinterpret_cast<const uint4 *>(pr + 8), b);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    x[e] = a[e];
+    x[8 + e] = b[e];
+  }
+}
+__device__ __forceinline__ void ldpair16(const float *pr, float (&x)[16]) { ldn<16>(pr, x); }
+
+// Pair bias of one slot for heads 0..H-1 (H <= 8):
+//   beta_h = sum_p LN(pair)_p * pair_scale_p * w_pair[p, h]
+//          = rstd * (sum_p y_p W'[p, h] - m * sum_p W'[p, h]),
+// y_p = pair_p - pair_0 (a shift that keeps the one-pass variance well conditioned),
+// m = mean(y), rstd = 1 / sqrt(mean(y^2) - m^2 + eps); W' = pair_scale * w_pair ([P][H]
+// in shared memory) and its column sums wsum.
+template <typename T, int H>
+__device__ __forceinline__ void pair_bias(const T *pr, int P, bool vec16, float eps,
+                                          const float *wp, const float *wsum, float *out) {
+  if (vec16) {
+    float x[16];
+    ldpair16(pr, x);
+    const float x0 = x[0];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      x[p] -= x0;
+      s1 += x[p];
+      s2 = fmaf(x[p], x[p], s2);
+    }
+    const float m = s1 * (1.f / 16.f);
+    const float rstd = rsqrtf(fmaxf(s2 * (1.f / 16.f) - m * m, 0.f) + eps);
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+      float d = 0.f;
+#pragma unroll
+      for (int p = 0; p < 16; ++p) d = fmaf(x[p], wp[p * H + h], d);
+      out[h] = rstd * (d - m * wsum[h]);
+    }
+    return;
+  }
+  // any P <= 32: statistics first, then the head sums with the channels read again
+  const float x0 = ldf(pr, 0);
+  float s1 = 0.f, s2 = 0.f;
+  for (int p = 0; p < P; ++p) {
+    const float y = ldf(pr, p) - x0;
+    s1 += y;
+    s2 = fmaf(y, y, s2);
+  }
+  const float m = s1 / (float)P;
+  const float rstd = rsqrtf(fmaxf(s2 / (float)P - m * m, 0.f) + eps);
+  float d[H];
+#pragma unroll
+  for (int h = 0; h < H; ++h) d[h] = 0.f;
+  for (int p = 0; p < P; ++p) {
+    const float y = ldf(pr, p) - x0;
+#pragma unroll
+    for (int h = 0; h < H; ++h) d[h] = fmaf(y, wp[p * H + h], d[h]);
+  }
+#pragma unroll
+  for (int h = 0; h < H; ++h) out[h] = rstd * (d[h] - m * wsum[h]);
+}
+
+}  // namespace rowattn
+
+template <typename T, int HD, int DH, bool AF3>
+__global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g) {
+  pdl_launch_next();
+  constexpr int ES = sizeof(T);
+  constexpr int LC = HD / 8;            // channels per lane; a quarter-warp covers a row
+  constexpr int CH = 16 / ES;           // channels per 16-byte chunk
+  constexpr int NSEG = LC / CH;         // 16-byte chunks per lane = 128-byte segments per row
+  constexpr int RB = HD * ES;           // bytes per staged row
+  constexpr int LPH = DH / LC;          // lanes of a quarter-warp per head
+  constexpr int H = HD / DH;
+  constexpr int OC = LC / 4;            // output channels per lane after the fold
+  static_assert(LC % CH == 0 && DH % LC == 0 && H <= kRowAttnHeadsMax, "row attention shape");
+  constexpr int NIT = kRowAttnIters;
+
+  extern __shared__ __align__(1024) uint8_t smem_dyn[];
+  __shared__ int s_lo, s_hi;
+  __shared__ __align__(16) float s_wp[AF3 ? kRowAttnPairMax * kRowAttnHeadsMax : 4];
+  __shared__ __align__(16) float s_wsum[AF3 ? kRowAttnHeadsMax : 4];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g4 = lane >> 3, li = lane & 7;            // quarter-warp, lane in it
+  const int b = blockIdx.y, a0 = blockIdx.x * g.QT;
+  const int QT = g.QT, K = g.K, A = g.A, P = g.P;
+  const int nq = min(QT, A - a0);
+
+  auto r128 = [](size_t n) { return (n + 127) & ~size_t(127); };
+  uint8_t *cur = smem_dyn;
+  int *ckey = reinterpret_cast<int *>(cur);           cur += r128((size_t)QT * K * 4);
+  uint8_t *cks = cur;                                  cur += r128((size_t)QT * K);
+  int *cnt = reinterpret_cast<int *>(cur);            cur += r128((size_t)QT * 4);
+  float *beta = reinterpret_cast<float *>(cur);       if (AF3) cur += r128((size_t)QT * K * H * 4);
+  const int WB = rowattn_wrow_bytes(K, ES);
+  uint8_t *wbuf_all = cur;                             cur += r128((size_t)kRowAttnWarps * H * WB);
+  uint8_t *kstage = cur;
+  uint8_t *vstage = cur + (size_t)g.stage_rows * RB;
+
+  if (tid == 0) {
+    s_lo = INT_MAX;
+    s_hi = -1;
+  }
+  if (AF3) {
+    for (int i = tid; i < P * H; i += kRowAttnThreads) s_wp[i] = g.w_pair[i];
+    for (int h = tid; h < H; h += kRowAttnThreads) {
+      float sw = 0.f;
+      for (int p = 0; p < P; ++p) sw += g.w_pair[p * H + h];
+      s_wsum[h] = sw;
+    }
+  }
+  __syncthreads();
+
+  // ---------------- list of permitted slots per query (before the wait)
+  const int64_t rbase = (int64_t)b * A;
+  int lo = INT_MAX, hi = -1;
+  for (int q = warp; q < QT; q += kRowAttnWarps) {
+    const int a = a0 + q;
+    const bool uq = q < nq && g.usable[rbase + a] != 0;
+    const int64_t sb = (rbase + a) * K;
+    int64_t kid[4];
+    uint8_t win[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int k = r * 32 + lane;
+      const bool in = uq && k < K;
+      kid[r] = in ? g.key_index[sb + k] : -1;
+      win[r] = in ? g.window[sb + k] : 0;
+    }
+    bool ok[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int64_t j = kid[r];
+      bool o = win[r] != 0 && j >= 0 && j < A;
+      if (o && g.radius >= 0) o = (j > a ? j - a : a - j) <= g.radius;
+      ok[r] = o;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+      if (ok[r]) ok[r] = g.usable[rbase + kid[r]] != 0;
+    int base = 0;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const unsigned bal = __ballot_sync(0xffffffffu, ok[r]);
+      if (ok[r]) {
+        const int pos = base + __popc(bal & ((1u << lane) - 1u));
+        ckey[q * K + pos] = (int)kid[r];
+        cks[q * K + pos] = (uint8_t)(r * 32 + lane);
+        lo = min(lo, (int)kid[r]);
+        hi = max(hi, (int)kid[r]);
+      }
+      base += __popc(bal);
+    }
+    if (lane == 0) cnt[q] = base;
+    if (AF3) {
+      // pair bias of every listed slot for every head, in list order
+      __syncwarp();
+      const T *prow = static_cast<const T *>(g.pair) + sb * P;
+      for (int e = lane; e < base; e += 32)
+        rowattn::pair_bias<T, H>(prow + (int64_t)cks[q * K + e] * P, P, g.pair_vec != 0, g.eps,
+                                 s_wp, s_wsum, beta + ((size_t)q * K + e) * H);
+    }
+  }
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  if (lane == 0 && lo <= hi) {
+    atomicMin(&s_lo, lo);
+    atomicMax(&s_hi, hi);
+  }
+
+  // ---------------- K/V stage (after the wait for the projections)
+  pdl_wait();
+  __syncthreads();
+  const int klo = s_lo, khi = s_hi;
+  const int span = khi >= klo ? khi - klo + 1 : 0;
+  const bool staged = span > 0 && span <= g.stage_rows;
+  if (span > 0 && !staged && tid == 0) atomicOr(g.status, 1u);
+  const uint8_t *Kg = static_cast<const uint8_t *>(g.Kf);
+  const uint8_t *Vg = static_cast<const uint8_t *>(g.Vf);
+  if (staged) {
+    // logical 16-byte chunk c of a row goes to position (c % NSEG) * 8 + c / NSEG
+    constexpr int CPR = RB / 16;                        // chunks per row
+    const int total = span * CPR;
+    const uint32_t ks = (uint32_t)__cvta_generic_to_shared(kstage);
+    const uint32_t vs = (uint32_t)__cvta_generic_to_shared(vstage);
+    for (int i = tid; i < total; i += kRowAttnThreads) {
+      const int r = i / CPR, c = i - r * CPR;
+      const int p = (c % NSEG) * 8 + c / NSEG;
+      const size_t src = (size_t)(rbase + klo + r) * RB + (size_t)c * 16;
+      const uint32_t dst = (uint32_t)(r * RB + p * 16);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ks + dst), "l"(Kg + src) : "memory");
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(vs + dst), "l"(Vg + src) : "memory");
+    }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+  }
+  __syncthreads();
+
+  // ---------------- one warp per query
+  const T *Qg = static_cast<const T *>(g.Q);
+  const T *Gg = static_cast<const T *>(g.G);
+  T *Og = static_cast<T *>(g.O);
+  T *Wg = static_cast<T *>(g.attention);
+  uint8_t *wbuf = wbuf_all + (size_t)warp * H * WB;
+  const int hd_lane = (li * LC) / DH;                 // this lane's head
+  const bool head_writer = (li % LPH) == 0;
+  const uint32_t kbase = (uint32_t)__cvta_generic_to_shared(kstage) + (uint32_t)li * 16u;
+  const uint32_t vbase = (uint32_t)__cvta_generic_to_shared(vstage) + (uint32_t)li * 16u;
+  const int oc0 = li * LC + OC * g4;                  // first output channel of this lane
+  const bool vecw = ((K * ES) & 15) == 0 && g.att_vec;
+
+  for (int q = warp; q < nq; q += kRowAttnWarps) {
+    const int a = a0 + q;
+    const int64_t arow = rbase + a;
+    const int n = cnt[q];
+    const int niter = (n + 3) >> 2;
+    // the query's channels and the value-gate logits of this lane's output channels
+    float qv[LC], gv[OC];
+    rowattn::ldn<LC>(Qg + arow * HD + li * LC, qv);
+    rowattn::ldn<OC>(Gg + arow * HD + oc0, gv);
+    // zero this warp's weight rows
+    for (int c = lane; c < H * WB / 16; c += 32)
+      *reinterpret_cast<uint4 *>(wbuf + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+
+    // ---- logits of the listed slots (log2 units)
+    float lt[NIT];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < NIT; ++t) {
+      lt[t] = -INFINITY;
+      if (t < niter) {
+        const int e = 4 * t + g4;
+        const bool live = e < n;
+        const int j = live ? ckey[q * K + e] : (staged ? klo : 0);
+        float part = 0.f;
+#pragma unroll
+        for (int s = 0; s < NSEG; ++s) {
+          uint4 raw;
+          if (staged)
+            raw = rowattn::lds128(kbase + (uint32_t)((j - klo) * RB + s * 128));
+          else
+            raw = *reinterpret_cast<const uint4 *>(Kg + (size_t)(rbase + j) * RB + (size_t)(NSEG * li + s) * 16);
+          float f[CH];
+          rowattn::unpack(raw, f);
+#pragma unroll
+          for (int c = 0; c < CH; ++c) part = fmaf(qv[s * CH + c], f[c], part);
+        }
+#pragma unroll
+        for (int w = 1; w < LPH; w <<= 1) part += __shfl_xor_sync(0xffffffffu, part, w);
+        float l = part * g.scale_log2;
+        if (AF3 && live) l = fmaf(beta[((size_t)q * K + e) * H + hd_lane], 1.4426950408889634f, l);
+        lt[t] = live ? l : -INFINITY;
+        mx = fmaxf(mx, lt[t]);
+      }
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    float sum = 0.f;
+#pragma unroll
+    for (int t = 0; t < NIT; ++t) {
+      if (t < niter) {
+        lt[t] = lt[t] > -INFINITY ? rowattn::ex2(lt[t] - mx) : 0.f;
+        sum += lt[t];
+      }
+    }
+    sum += __shfl_xor_sync(0xffffffffu, sum, 8);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 16);
+    float inv = 0.f;
+    if (sum > 0.f) asm("rcp.approx.f32 %0, %1;" : "=f"(inv) : "f"(sum));
+    __syncwarp();
+
+    // ---- weights out (per-warp rows), weighted values
+    float acc[LC];
+#pragma unroll
+    for (int c = 0; c < LC; ++c) acc[c] = 0.f;
+#pragma unroll
+    for (int t = 0; t < NIT; ++t) {
+      if (t < niter) {
+        const int e = 4 * t + g4;
+        const bool live = e < n;
+        const float w = lt[t] * inv;
+        if (live && head_writer)
+          rowattn::store_w<T>(reinterpret_cast<T *>(wbuf + hd_lane * WB) + cks[q * K + e], w);
+        const int j = live ? ckey[q * K + e] : (staged ? klo : 0);
+#pragma unroll
+        for (int s = 0; s < NSEG; ++s) {
+          uint4 raw;
+          if (staged)
+            raw = rowattn::lds128(vbase + (uint32_t)((j - klo) * RB + s * 128));
+          else
+            raw = *reinterpret_cast<const uint4 *>(Vg + (size_t)(rbase + j) * RB + (size_t)(NSEG * li + s) * 16);
+          float f[CH];
+          rowattn::unpack(raw, f);
+#pragma unroll
+          for (int c = 0; c < CH; ++c) acc[s * CH + c] = fmaf(w, f[c], acc[s * CH + c]);
+        }
+      }
+    }
+    // fold the four quarter-warps: lane (g4, li) ends with channels oc0 .. oc0 + OC
+#pragma unroll
+    for (int w = 16, h = LC / 2; w >= 8; w >>= 1, h >>= 1) {
+      const bool up = (lane & w) != 0;
+#pragma unroll
+      for (int c = 0; c < LC / 2; ++c) {
+        if (c < h) {
+          const float send = up ? acc[c] : acc[c + h];
+          const float keep = up ? acc[c + h] : acc[c];
+          acc[c] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+        }
+      }
+    }
+    float ov[OC];
+#pragma unroll
+    for (int c = 0; c < OC; ++c) ov[c] = sum > 0.f ? acc[c] * sigmoid_fast(gv[c]) : 0.f;
+    rowattn::stn<OC>(Og + arow * HD + oc0, ov);
+
+    // ---- the query's weight rows to attention[b, h, a, :]
+    __syncwarp();
+    if (vecw) {
+      const int cpr = K * ES / 16;
+      for (int c = lane; c < H * cpr; c += 32) {
+        const int h = c / cpr, cc = c - h * cpr;
+        const uint4 v = *reinterpret_cast<const uint4 *>(wbuf + h * WB + cc * 16);
+        *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(Wg + (((int64_t)b * H + h) * A + a) * K) + cc * 16) = v;
+      }
+    } else {
+      for (int c = lane; c < H * K; c += 32) {
+        const int h = c / K, k = c - h * K;
+        Wg[(((int64_t)b * H + h) * A + a) * K + k] = reinterpret_cast<const T *>(wbuf + h * WB)[k];
+      }
+    }
+    __syncwarp();
+  }
+
+  // queries of the tile past A: nothing; queries with no permitted slot were written
+  // as zero rows above (their list is empty)
+}
+
+}  // namespace atomenc

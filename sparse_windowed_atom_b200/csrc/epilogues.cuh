@@ -76,10 +76,24 @@ struct EpiGateAF3 {
   }
 };
 
+// four consecutive values of a [rows, HD] intermediate in its workspace type
+__device__ __forceinline__ void st4w(float *d, const float (&o)[4]) {
+  *reinterpret_cast<float4 *>(d) = make_float4(o[0], o[1], o[2], o[3]);
+}
+__device__ __forceinline__ void st4w(__nv_bfloat16 *d, const float (&o)[4]) {
+  const uint32_t a = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o[0])) |
+                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o[1])) << 16);
+  const uint32_t b = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o[2])) |
+                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o[3])) << 16);
+  *reinterpret_cast<uint2 *>(d) = make_uint2(a, b);
+}
+
 // Q/K/V/value-gate projections: the N columns are `nparts` blocks of HD written to
-// separate [M, HD] buffers; only Q takes a bias (AF3 b_q, bullet 8)
-struct EpiSplit {
-  float *dst[4];
+// separate [M, HD] buffers of type WT (float32, or bf16 for bf16 workloads whose
+// attention reads bf16 rows); only Q takes a bias (AF3 b_q, bullet 8)
+template <typename WT>
+struct EpiSplitT {
+  WT *dst[4];
   const float *bias[4];
   int64_t HD;
   __device__ void quad(int64_t r, int64_t c0, const float (&v)[4], int64_t N) const {
@@ -90,9 +104,9 @@ struct EpiSplit {
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[e] += b[ch + e];
     }
-    float *d = dst[part] + r * HD + ch;
+    WT *d = dst[part] + r * HD + ch;
     if ((HDi & 3) == 0) {
-      *reinterpret_cast<float4 *>(d) = make_float4(o[0], o[1], o[2], o[3]);
+      st4w(d, o);
     } else {  // a quad may straddle two parts when HD is not a multiple of 4
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -101,11 +115,12 @@ struct EpiSplit {
         const int pe = ce / HDi, he = ce - pe * HDi;
         float x = v[e];
         if (bias[pe]) x += bias[pe][he];
-        dst[pe][r * HD + he] = x;
+        stf(dst[pe], r * HD + he, x);
       }
     }
   }
 };
+using EpiSplit = EpiSplitT<float>;
 
 // x' = x + g_attn * (o @ w_attention_out)  (bullet 16)
 struct EpiResidual {

@@ -253,7 +253,8 @@ struct RopeArgs {
   float eps;
   const uint8_t *usable;
   const void *cos, *sin;  // [rows, D]
-  float *Q, *K;           // [rows, H*D], rewritten in place
+  void *Q, *K;            // [rows, H*D], rewritten in place (float32; k_qk_rope_warp:
+                          // its workspace type)
 };
 
 // Per-head RMS of Q and K over D, then q * cos + rotate_half(q) * sin with
@@ -267,7 +268,7 @@ __global__ void k_qk_rope(RopeArgs r) {
   const int which = (int)(id & 1);
   const int64_t rh = id >> 1;
   const int64_t row = rh / r.H, h = rh % r.H;
-  float *v = (which ? r.K : r.Q) + row * r.H * r.D + h * r.D;
+  float *v = static_cast<float *>(which ? r.K : r.Q) + row * r.H * r.D + h * r.D;
   const bool use = r.usable[row] != 0;
   float buf[128];
   float ss = 0.f;
@@ -287,11 +288,28 @@ __global__ void k_qk_rope(RopeArgs r) {
   }
 }
 
+// four consecutive values of a Q / K row, read and written in the workspace type
+__device__ __forceinline__ float4 ld4w(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 ld4w(const __nv_bfloat16 *p) {
+  const uint2 u = *reinterpret_cast<const uint2 *>(p);
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+}
+__device__ __forceinline__ void st4w(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+__device__ __forceinline__ void st4w(__nv_bfloat16 *p, float4 v) {
+  const uint32_t a = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.x)) |
+                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.y)) << 16);
+  const uint32_t b = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.z)) |
+                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.w)) << 16);
+  *reinterpret_cast<uint2 *>(p) = make_uint2(a, b);
+}
+
 // Warp per (atom, Q-or-K) for head widths D in {8, 16, 32, 64, 128}: lane l holds four
 // consecutive channels of each 128-channel chunk, the D/4 lanes of one head reduce the
 // sum of squares with xor-shuffles, and the half-split partner of channel d (d +- D/2)
-// sits D/8 lanes away in the same head group.
-template <typename T>
+// sits D/8 lanes away in the same head group. Q and K are of type WT (float32, or bf16
+// when the attention reads bf16 rows); the arithmetic is float32.
+template <typename T, typename WT>
 __global__ void k_qk_rope_warp(RopeArgs r) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
@@ -299,14 +317,14 @@ __global__ void k_qk_rope_warp(RopeArgs r) {
   if (wid >= r.rows * 2) return;
   const int64_t row = wid >> 1;
   const int D = (int)r.D, HD = (int)(r.H * r.D), glanes = D / 4, half = D / 2;
-  float *v = ((wid & 1) ? r.K : r.Q) + row * HD;
+  WT *v = static_cast<WT *>((wid & 1) ? r.K : r.Q) + row * HD;
   const bool use = r.usable[row] != 0;
   const T *cs = (const T *)r.cos + row * D;
   const T *sn = (const T *)r.sin + row * D;
   for (int c0 = 0; c0 < HD; c0 += 128) {
     const int c = c0 + lane * 4;
     const bool in = c < HD;
-    float4 x = in ? *reinterpret_cast<const float4 *>(v + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 x = in ? ld4w(v + c) : make_float4(0.f, 0.f, 0.f, 0.f);
     float ss = x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
     for (int o = 1; o < glanes; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float rstd = 1.f / sqrtf(ss / (float)D + r.eps);
@@ -327,7 +345,7 @@ __global__ void k_qk_rope_warp(RopeArgs r) {
         o.z = x.z * ldf(cs, d + 2) + sg * p.z * ldf(sn, d + 2);
         o.w = x.w * ldf(cs, d + 3) + sg * p.w * ldf(sn, d + 3);
       }
-      *reinterpret_cast<float4 *>(v + c) = o;
+      st4w(v + c, o);
     }
   }
 }

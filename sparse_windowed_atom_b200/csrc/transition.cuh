@@ -36,7 +36,8 @@ constexpr int kTransThreads = (kTransEpiWarps + 2) * 32;   // + MMA issuer + wei
 struct TransArgs {
   int64_t R;
   int HD, M;                   // C is 128
-  const float *O;              // [R, HD] gated attention output
+  const void *O;               // [R, HD] gated attention output (float32, or bf16 when
+                               // the attention wrote bf16 rows)
   const float *x;              // [R, 128] residual state start
   const float *g0, *g1;        // attention / transition residual gates (row stride g_ld)
   int64_t g_ld;
@@ -122,7 +123,7 @@ __device__ __forceinline__ int ld_acquire(const int *p) {
   return v;
 }
 
-template <bool SPLIT, typename TOut, bool PAIR>
+template <bool SPLIT, typename TOut, bool PAIR, typename TO = float>
 __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
   pdl_enter();
   extern __shared__ __align__(1024) uint8_t smem_dyn[];
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
       float v[4][8];
 #pragma unroll
       for (int it = 0; it < 4; ++it)
-        load8_t(t.O, t.HD, t.R, t.HD, m0 + warp * 16 + it * 4 + (lane >> 3),
+        load8_t(static_cast<const TO *>(t.O), t.HD, t.R, t.HD, m0 + warp * 16 + it * 4 + (lane >> 3),
                 (int64_t)kc * kUmmaBK + (lane & 7) * 8, v[it]);
 #pragma unroll
       for (int it = 0; it < 4; ++it)
