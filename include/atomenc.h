@@ -30,8 +30,8 @@
  *    waits for that work before reading or writing memory, so stream order holds.
  *  - Inputs must not alias outputs or the workspace. Calls that share a workspace
  *    must be ordered on one stream.
- *  - Size limits (ATOMENC_ERR_UNSUPPORTED beyond them): D <= 64; AF3 P <= 32 and
- *    H <= 32; K <= 8192; A <= 2^31 - 4097.
+ *  - Size limits (ATOMENC_ERR_UNSUPPORTED beyond them): D <= 64; S <= 256; AF3 P <= 32
+ *    and H <= 32; K <= 8192; A <= 2^31 - 4097.
  *
  * Shapes (B batch, A atoms, T tokens, K key slots, C atom width, S condition width,
  * H heads, D head width, P pair channels, M transition width, U pooled width,

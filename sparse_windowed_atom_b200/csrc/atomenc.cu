@@ -91,8 +91,8 @@ struct Plan {
   bool af3 = false, enc = false, fuse_tail = false, tail_pair = false;
   Dims d;
   // workspace layout (byte offsets)
-  size_t o_status, o_usable, o_xstats, o_first, o_last, o_tp, o_x, o_opc, o_rawc, o_cond, o_gate, o_feat,
-      o_q, o_k, o_v, o_g, o_o, o_xp, o_z, o_h, o_hid, o_pool, o_xfer, o_xflag;
+  size_t o_status, o_usable, o_xstats, o_cstats, o_first, o_last, o_tp, o_x, o_cond, o_gate, o_feat,
+      o_q, o_k, o_v, o_g, o_o, o_xp, o_z, o_h, o_pool, o_xfer, o_xflag;
   size_t o_wread, o_bscale, o_brg, o_bq, o_wpair, o_rscale, o_rbias;
   // tensor-core images of the weight panels (bf16, hi[/lo])
   size_t k_cond, k_gate, k_qkv0, k_qkv1, k_out, k_ff1, k_ff2, k_pool, k_tok;
@@ -229,22 +229,24 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
     CHECK(check_tensor(out->hidden, fdt, 3, hc));
     CHECK(check_tensor(out->attention, fdt, 4, at));
   }
-  if (D > kMaxD || A > INT_MAX - 4096 || K > 8192) return ATOMENC_ERR_UNSUPPORTED;
+  if (D > kMaxD || A > INT_MAX - 4096 || K > 8192 || S > kRowsKMax) return ATOMENC_ERR_UNSUPPORTED;
 
   // ---- workspace plan
   const int64_t R = B * A;
   size_t cur = 0;
   pl.o_status = take(cur, 256);
   pl.o_usable = take(cur, R);
+  // x, the conditioning vectors, the AF3 gates and the pooled rows are kept in the
+  // storage type (bf16 workloads: bf16)
+  const int64_t its = fdt == ATOMENC_BF16 ? 2 : 4;
   pl.o_xstats = take(cur, R * 2 * 4);
+  pl.o_cstats = take(cur, pl.af3 ? R * 2 * 4 : 0);
   pl.o_first = take(cur, pl.enc ? B * T * 4 : 0);
   pl.o_last = take(cur, pl.enc ? B * T * 4 : 0);
   pl.o_tp = take(cur, pl.enc ? 0 : B * T * C * 4);
-  pl.o_x = take(cur, R * C * 4);
-  pl.o_opc = take(cur, R * S * 4);
-  pl.o_rawc = take(cur, pl.af3 ? R * S * 4 : 0);
-  pl.o_cond = take(cur, R * 6 * C * 4);
-  pl.o_gate = take(cur, pl.af3 ? R * 2 * C * 4 : 0);
+  pl.o_x = take(cur, R * C * its);
+  pl.o_cond = take(cur, R * 6 * C * its);
+  pl.o_gate = take(cur, pl.af3 ? R * 2 * C * its : 0);
   const bool fused = C <= kRowsKMax;
   pl.o_feat = take(cur, fused ? 0 : R * (pl.af3 ? 2 : 1) * C * 4);
   // row-gather attention: whole rows of all heads per quarter-warp (H*D == 128, a head
@@ -274,8 +276,7 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   pl.o_xp = take(cur, pl.fuse_tail ? 0 : R * C * 4);
   pl.o_z = take(cur, pl.fuse_tail ? 0 : R * C * 4);
   pl.o_h = take(cur, pl.fuse_tail ? 0 : R * M * 4);
-  pl.o_hid = take(cur, pl.fuse_tail && fdt == ATOMENC_F32 ? 0 : R * C * 4);  // float32 hidden copy
-  pl.o_pool = take(cur, pl.enc ? R * U * 4 : 0);
+  pl.o_pool = take(cur, pl.enc ? R * U * its : 0);
   pl.o_wread = take(cur, pl.enc ? 0 : C * 3 * 4);
   pl.o_bscale = take(cur, pl.af3 ? 3 * C * 4 : 0);
   pl.o_brg = take(cur, pl.af3 ? 2 * C * 4 : 0);
@@ -584,9 +585,10 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   };
   // the conditioning-modulated row norm of x (or x') fused into a projection's operand
   const bool fuse_norm = C <= kRowsKMax;
+  Elt *xb = reinterpret_cast<Elt *>(ws + pl.o_x), *condb = reinterpret_cast<Elt *>(ws + pl.o_cond),
+      *gateb = reinterpret_cast<Elt *>(ws + pl.o_gate), *poolb = reinterpret_cast<Elt *>(ws + pl.o_pool);
   auto norm_prod = [&](int64_t sc_off, int64_t sh_off, bool plus1) {
-    return ProdNorm{F(pl.o_x), F(pl.o_xstats), F(pl.o_cond), R, C, 6 * C, sc_off, sh_off,
-                    plus1 ? 1 : 0};
+    return ProdNormT<Elt>{xb, F(pl.o_xstats), condb, R, C, 6 * C, sc_off, sh_off, plus1 ? 1 : 0};
   };
   const int rows_per_block = 8;  // warps per 256-thread block for warp-per-row kernels
   const unsigned row_blocks = (unsigned)((R + rows_per_block - 1) / rows_per_block);
@@ -605,7 +607,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   ra.token_valid = static_cast<const uint8_t *>(in->token_valid.data);
   ra.att = static_cast<const int64_t *>(in->atom_to_token.data);
   ra.token_proj = F(pl.o_tp);
-  ra.usable = usable; ra.x = F(pl.o_x); ra.xstats = F(pl.o_xstats); ra.opc = F(pl.o_opc); ra.rawc = F(pl.o_rawc);
+  ra.usable = usable; ra.x = xb; ra.xstats = F(pl.o_xstats); ra.cstats = F(pl.o_cstats);
   ra.tok_first = first; ra.tok_last = last;
   {
     const uintptr_t al = sizeof(Elt) == 4 ? 15 : 7;   // 4-element loads of atom / condition rows
@@ -618,19 +620,22 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   }
   hk.mark(1, st);
 
-  // ---- conditioning
+  // ---- conditioning: the operand (LN(c), raw c or SiLU(c) of the sanitised condition)
+  // is formed from the caller's condition rows inside the product
+  const Elt *cin = static_cast<const Elt *>(in->condition.data);
   if (pl.af3) {
-    gemm(F(pl.o_opc), S, pl.k_cond, R, 6 * C, S,
-         EpiCondAF3{F(pl.o_cond), F(pl.o_bscale), C});
-    gemm(F(pl.o_rawc), S, pl.k_gate, R, 2 * C, S,
-         EpiGateAF3{F(pl.o_gate), F(pl.o_brg), C});
+    gemm_rows(ProdCond<Elt, 2>{cin, usable, F(pl.o_cstats), R, S}, pl.k_cond, R, 6 * C, S,
+              EpiCondAF3<Elt>{condb, F(pl.o_bscale), C});
+    gemm_rows(ProdCond<Elt, 0>{cin, usable, nullptr, R, S}, pl.k_gate, R, 2 * C, S,
+              EpiGateAF3<Elt>{gateb, F(pl.o_brg), C});
   } else {
-    gemm(F(pl.o_opc), S, pl.k_cond, R, 6 * C, S, Quad<EpiStore>{{F(pl.o_cond), 6 * C}});
+    gemm_rows(ProdCond<Elt, 1>{cin, usable, nullptr, R, S}, pl.k_cond, R, 6 * C, S,
+              Quad<EpiStoreT<Elt>>{{condb, 6 * C}});
   }
   hk.mark(2, st);
   if (!fuse_norm) {
-    FeatArgs fa{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_x), F(pl.o_cond), F(pl.o_feat)};
-    hk.launch(ATOMENC_KERNEL_ROWS, k_features, row_blocks, 256, 0, st, fa);
+    FeatArgs fa{R, C, eps, pl.af3 ? 1 : 0, xb, condb, F(pl.o_feat)};
+    hk.launch(ATOMENC_KERNEL_ROWS, (k_features<Elt>), row_blocks, 256, 0, st, fa);
   }
 
   // ---- projections .. transition; WT is the type of the Q/K/V/G/O intermediates
@@ -744,19 +749,19 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     hk.mark(4, st);
 
     // ---- out-projection + gated residual, transition norm, SwiGLU, gated residual + mask
-    const float *gbuf = pl.af3 ? F(pl.o_gate) : F(pl.o_cond);
+    const Elt *gbuf = pl.af3 ? gateb : condb;
     const int64_t gld = pl.af3 ? 2 * C : 6 * C;
     const int64_t g0off = pl.af3 ? 0 : 2 * C, g1off = pl.af3 ? C : 5 * C;
     if (pl.fuse_tail) {
       TransArgs ta;
       ta.R = R; ta.HD = (int)HD; ta.M = (int)M;
-      ta.O = wo; ta.x = F(pl.o_x);
+      ta.O = wo; ta.x = xb;
       ta.g0 = gbuf + g0off; ta.g1 = gbuf + g1off; ta.g_ld = gld;
-      ta.sc = F(pl.o_cond) + 4 * C; ta.sh = F(pl.o_cond) + (pl.af3 ? 5 : 3) * C; ta.cond_ld = 6 * C;
+      ta.sc = condb + 4 * C; ta.sh = condb + (pl.af3 ? 5 : 3) * C; ta.cond_ld = 6 * C;
       ta.rms = pl.af3 ? 0 : 1; ta.plus1 = pl.af3 ? 0 : 1; ta.eps = eps;
       ta.usable = usable;
       ta.w_out = ws + pl.k_out; ta.w_ff1 = ws + pl.k_ff1; ta.w_ff2 = ws + pl.k_ff2;
-      ta.hid32 = split ? nullptr : F(pl.o_hid); ta.hidden = out->hidden.data; ta.status = status;
+      ta.hidden = out->hidden.data; ta.status = status;
       ta.xfer = F(pl.o_xfer); ta.xflag = reinterpret_cast<int *>(ws + pl.o_xflag);
       ta.peer_spin_limit = g_peer_spin_limit.load();
       ta.withhold_flag = g_peer_withhold.load();
@@ -776,12 +781,12 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
       }
     } else {
       gemm(static_cast<const WT *>(wo), HD, pl.k_out, R, C, HD,
-           Quad<EpiResidual>{{F(pl.o_x), gbuf, gld, g0off, C, F(pl.o_xp)}});
-      TNormArgs tn{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_xp), F(pl.o_cond), F(pl.o_z)};
-      hk.launch(ATOMENC_KERNEL_ROWS, k_transition_norm, row_blocks, 256, 0, st, tn);
+           Quad<EpiResidual<Elt>>{{xb, gbuf, gld, g0off, C, F(pl.o_xp)}});
+      TNormArgs tn{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_xp), condb, F(pl.o_z)};
+      hk.launch(ATOMENC_KERNEL_ROWS, (k_transition_norm<Elt>), row_blocks, 256, 0, st, tn);
       gemm(F(pl.o_z), C, pl.k_ff1, R, 2 * M, C, EpiSwiGLU{F(pl.o_h), M});
       gemm(F(pl.o_h), M, pl.k_ff2, R, C, M,
-           Quad<EpiHidden<Elt>>{{F(pl.o_xp), gbuf, gld, g1off, C, usable, F(pl.o_hid),
+           Quad<EpiHidden<Elt>>{{F(pl.o_xp), gbuf, gld, g1off, C, usable,
                                  static_cast<Elt *>(out->hidden.data)}});
     }
   };
@@ -796,12 +801,12 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
 
   hk.mark(5, st);
 
-  // ---- boundary (float32 hidden: the output itself when it is float32 and fused)
-  const float *hid = pl.fuse_tail && split ? static_cast<const float *>(out->hidden.data) : F(pl.o_hid);
+  // ---- boundary, read from the hidden output itself
+  const Elt *hid = static_cast<const Elt *>(out->hidden.data);
   if (pl.enc) {
-    gemm(hid, C, pl.k_pool, R, U, C, Quad<EpiRelu>{{F(pl.o_pool), U}});
+    gemm(hid, C, pl.k_pool, R, U, C, Quad<EpiRelu<Elt>>{{poolb, U}});
     PoolArgs pa{B, A, T, U, usable, static_cast<const int64_t *>(in->atom_to_token.data), first,
-                last, F(pl.o_pool), out->token_output.data};
+                last, poolb, out->token_output.data};
     hk.launch(ATOMENC_KERNEL_POOL, (k_token_mean<Elt>), (unsigned)(B * T), kPoolThreads, 0, st, pa);
   } else {
     ReadoutArgs rd{R, C, eps, pl.af3 ? 0 : 1, usable, hid, F(pl.o_rscale), F(pl.o_rbias),

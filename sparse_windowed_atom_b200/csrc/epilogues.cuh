@@ -19,17 +19,30 @@ struct Quad {
 
 // ---- epilogues (each a small functor; names say which step of the block they end)
 
-struct EpiStore {  // plain float32 store
-  float *out;
+template <typename IT>
+struct EpiStoreT {  // plain store in the intermediate type
+  IT *out;
   int64_t ld;
-  __device__ void operator()(int64_t r, int64_t c, float v) const { out[r * ld + c] = v; }
+  __device__ void operator()(int64_t r, int64_t c, float v) const { stf(out, r * ld + c, v); }
 };
+using EpiStore = EpiStoreT<float>;
+
+// four consecutive values in the intermediate type (16-byte float32 / 8-byte bf16)
+__device__ __forceinline__ void st4i(float *d, float4 o) { *reinterpret_cast<float4 *>(d) = o; }
+__device__ __forceinline__ void st4i(__nv_bfloat16 *d, float4 o) {
+  const uint32_t a = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o.x)) |
+                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o.y)) << 16);
+  const uint32_t b = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o.z)) |
+                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o.w)) << 16);
+  *reinterpret_cast<uint2 *>(d) = make_uint2(a, b);
+}
 
 // AF3 conditioning: columns (scale_0, shift_0, scale_1, shift_1, scale_2, shift_2), C each;
 // scale columns become sigmoid(c_j @ w_scale[j] + b_scale[j])  (bullet 7)
 // Index math is done once per four columns, in 32 bits (C is a multiple of 4).
+template <typename IT>
 struct EpiCondAF3 {
-  float *out;  // [M, 6C]
+  IT *out;     // [M, 6C]
   const float *b_scale;  // [3, C]
   int64_t C;
   __device__ void quad(int64_t r, int64_t c0, const float (&v)[4], int64_t N) const {
@@ -40,7 +53,7 @@ struct EpiCondAF3 {
         const int ce = c + e;
         if (ce >= N) break;
         const int be = ce / Ci, he = ce - be * Ci;
-        out[r * 6 * C + ce] = (be & 1) ? v[e] : sigmoid_fast(v[e] + b_scale[(be >> 1) * Ci + he]);
+        stf(out, r * 6 * C + ce, (be & 1) ? v[e] : sigmoid_fast(v[e] + b_scale[(be >> 1) * Ci + he]));
       }
       return;
     }
@@ -53,13 +66,14 @@ struct EpiCondAF3 {
       o.z = sigmoid_fast(v[2] + bs[2]);
       o.w = sigmoid_fast(v[3] + bs[3]);
     }
-    *reinterpret_cast<float4 *>(out + r * 6 * C + c0) = o;
+    st4i(out + r * 6 * C + c0, o);
   }
 };
 
 // AF3 residual gates sigmoid(raw condition @ w_residual_gate[j] + b_residual_gate[j])  (bullet 9)
+template <typename IT>
 struct EpiGateAF3 {
-  float *out;  // [M, 2C]
+  IT *out;     // [M, 2C]
   const float *b_rg;  // [2, C]
   int64_t C;
   __device__ void quad(int64_t r, int64_t c0, const float (&v)[4], int64_t N) const {
@@ -67,12 +81,12 @@ struct EpiGateAF3 {
     if (C & 1) {
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        if (c0 + e < N) out[r * 2 * C + c0 + e] = sigmoid_fast(v[e] + b[e]);
+        if (c0 + e < N) stf(out, r * 2 * C + c0 + e, sigmoid_fast(v[e] + b[e]));
       return;
     }
-    *reinterpret_cast<float4 *>(out + r * 2 * C + c0) =
-        make_float4(sigmoid_fast(v[0] + b[0]), sigmoid_fast(v[1] + b[1]), sigmoid_fast(v[2] + b[2]),
-                    sigmoid_fast(v[3] + b[3]));
+    st4i(out + r * 2 * C + c0,
+         make_float4(sigmoid_fast(v[0] + b[0]), sigmoid_fast(v[1] + b[1]), sigmoid_fast(v[2] + b[2]),
+                     sigmoid_fast(v[3] + b[3])));
   }
 };
 
@@ -122,14 +136,16 @@ struct EpiSplitT {
 };
 using EpiSplit = EpiSplitT<float>;
 
-// x' = x + g_attn * (o @ w_attention_out)  (bullet 16)
+// x' = x + g_attn * (o @ w_attention_out)  (bullet 16); x and the gates in the
+// intermediate type, x' in float32
+template <typename IT>
 struct EpiResidual {
-  const float *x;
-  const float *gate;  // gate[r * gate_ld + gate_off + c]
+  const IT *x;
+  const IT *gate;  // gate[r * gate_ld + gate_off + c]
   int64_t gate_ld, gate_off, C;
   float *out;
   __device__ void operator()(int64_t r, int64_t c, float v) const {
-    out[r * C + c] = x[r * C + c] + gate[r * gate_ld + gate_off + c] * v;
+    out[r * C + c] = ldf(x, r * C + c) + ldf(gate, r * gate_ld + gate_off + c) * v;
   }
 };
 
@@ -146,28 +162,28 @@ struct EpiSwiGLU {
   }
 };
 
-// hidden = usable * (x' + g_trans * ((...) @ w_ff_out))  (bullet 18)
+// hidden = usable * (x' + g_trans * ((...) @ w_ff_out))  (bullet 18); the gates in the
+// storage type T of the output
 template <typename T>
 struct EpiHidden {
   const float *xp;
-  const float *gate;
+  const T *gate;
   int64_t gate_ld, gate_off, C;
   const uint8_t *usable;
-  float *hid32;  // float32 copy for pooling / readout
   T *hid;        // output
   __device__ void operator()(int64_t r, int64_t c, float v) const {
-    const float h = usable[r] ? xp[r * C + c] + gate[r * gate_ld + gate_off + c] * v : 0.f;
-    hid32[r * C + c] = h;
+    const float h = usable[r] ? xp[r * C + c] + ldf(gate, r * gate_ld + gate_off + c) * v : 0.f;
     stf(hid, r * C + c, h);
   }
 };
 
-// ReLU(hidden @ w_pool) before the per-token mean (bullet 19)
+// ReLU(hidden @ w_pool) before the per-token mean (bullet 19), in the intermediate type
+template <typename IT>
 struct EpiRelu {
-  float *out;
+  IT *out;
   int64_t ld;
   __device__ void operator()(int64_t r, int64_t c, float v) const {
-    out[r * ld + c] = v > 0.f ? v : 0.f;
+    stf(out, r * ld + c, v > 0.f ? v : 0.f);
   }
 };
 

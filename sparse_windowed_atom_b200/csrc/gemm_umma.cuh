@@ -89,10 +89,11 @@ struct ProdPlain {
   }
 };
 
-struct ProdNorm {
-  const float *x;        // [M, K]
+template <typename IT>
+struct ProdNormT {
+  const IT *x;           // [M, K] residual state, storage type
   const float *stats;    // [M, 2]: mean (0 for RMS) and rstd of each row of x
-  const float *cond;     // rows of cond_ld floats
+  const IT *cond;        // rows of cond_ld values, storage type
   int64_t M, K, cond_ld, sc_off, sh_off;
   int plus1;
   __device__ void load8(int64_t r, int64_t k, float (&v)[8]) const {
@@ -105,6 +106,34 @@ struct ProdNorm {
     for (int e = 0; e < 8; ++e) {
       const float s = plus1 ? 1.f + sc[e] : sc[e];
       v[e] = (r < M && k + e < K) ? fmaf((xv[e] - ms.x) * ms.y, s, sh[e]) : 0.f;
+    }
+  }
+};
+using ProdNorm = ProdNormT<float>;
+
+// The condition operand of the conditioning products, formed from the caller's
+// condition rows: zero for an unusable atom (a select, so NaN / Inf payloads never
+// enter), else MODE 0 the raw value (AF3 residual gates, bullet 9), MODE 1 SiLU
+// (ESMFold2 w_mod, bullet 10), MODE 2 (c - mean) * rstd with the row's population
+// LayerNorm statistics (AF3 c_j, bullet 7; cond_scale[j] is folded into the weights).
+template <typename T, int MODE>
+struct ProdCond {
+  const T *c;            // [M, K] condition rows
+  const uint8_t *usable; // [M]
+  const float *stats;    // [M, 2] (MODE 2)
+  int64_t M, K;
+  __device__ void load8(int64_t r, int64_t k, float (&v)[8]) const {
+    const bool use = r < M && usable[r] != 0;
+    float cv[8];
+    load8_t(c, K, use ? M : 0, K, r, k, cv);   // rows of unusable atoms are not read
+    float2 ms = make_float2(0.f, 1.f);
+    if (MODE == 2 && use) ms = *reinterpret_cast<const float2 *>(stats + 2 * r);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float y = cv[e];
+      if (MODE == 1) y = silu_fast(y);
+      if (MODE == 2) y = (y - ms.x) * ms.y;
+      v[e] = (use && k + e < K) ? y : 0.f;
     }
   }
 };

@@ -17,12 +17,13 @@ struct RowsArgs {
   const int64_t *att;
   const float *token_proj;  // [B*T, C] decoder: token @ w_token
   uint8_t *usable;          // [B*A]
-  float *x;                 // [B*A, C] residual state start
+  void *x;                  // [B*A, C] residual state start, in the storage type
   float *xstats;            // [B*A, 2] AF3: mean, 1/sqrt(var+eps); ESM: 0, 1/sqrt(mean sq+eps)
-  float *opc;               // [B*A, S] AF3: LN(c); ESMFold2: SiLU(c)
-  float *rawc;              // [B*A, S] AF3: sanitised raw condition
+  float *cstats;            // [B*A, 2] AF3: mean, 1/sqrt(var+eps) of the sanitised condition
   int *tok_first, *tok_last;  // [B*T] encoder pooling ranges
 };
+// The conditioning products read the condition itself (sanitised, and SiLU'd or
+// normalised with cstats, while their operand is formed); no copy of it is written.
 
 // One warp per atom. usable = valid & 0 <= atom_to_token < T & token_valid  (bullet 2);
 // payloads of unusable atoms are replaced by zero with a select before any arithmetic
@@ -44,6 +45,7 @@ __global__ void k_rows_prep(RowsArgs r) {
     }
   }
   const T *atom = (const T *)r.atom + row * r.C;
+  T *xr = static_cast<T *>(r.x) + row * r.C;
   float s1 = 0.f;
   for (int64_t c = lane; c < r.C; c += kWarp) {
     float v = 0.f;
@@ -51,16 +53,16 @@ __global__ void k_rows_prep(RowsArgs r) {
       v = ldf(atom, c);
       if (r.decoder) v += r.token_proj[(b * r.T + t) * r.C + c];
     }
-    r.x[row * r.C + c] = v;
-    s1 += v;
+    stf(xr, c, v);
+    s1 += ldf(xr, c);
   }
-  // row statistics of x for the attention inputs: AF3 population LayerNorm (bullet 7),
-  // ESMFold2 RMS (bullet 11); the second pass re-reads the row just written
+  // row statistics of x (as stored) for the attention inputs: AF3 population LayerNorm
+  // (bullet 7), ESMFold2 RMS (bullet 11); the second pass re-reads the row just written
   __syncwarp();
   const float mean = r.af3 ? warp_sum(s1) / (float)r.C : 0.f;
   float s2 = 0.f;
   for (int64_t c = lane; c < r.C; c += kWarp) {
-    const float d = r.x[row * r.C + c] - mean;
+    const float d = ldf(xr, c) - mean;
     s2 = fmaf(d, d, s2);
   }
   s2 = warp_sum(s2);
@@ -68,38 +70,47 @@ __global__ void k_rows_prep(RowsArgs r) {
     r.xstats[2 * row] = mean;
     r.xstats[2 * row + 1] = 1.f / sqrtf(s2 / (float)r.C + r.eps);
   }
-  const T *cond = (const T *)r.condition + row * r.S;
   if (r.af3) {
-    // population LayerNorm of the condition, eps inside the root (bullet 7)
+    // population LayerNorm statistics of the condition, eps inside the root (bullet 7)
+    const T *cond = (const T *)r.condition + row * r.S;
     float s = 0.f;
     for (int64_t k = lane; k < r.S; k += kWarp) s += use ? ldf(cond, k) : 0.f;
-    const float mean = warp_sum(s) / (float)r.S;
+    const float cm = warp_sum(s) / (float)r.S;
     float q = 0.f;
     for (int64_t k = lane; k < r.S; k += kWarp) {
-      float d = (use ? ldf(cond, k) : 0.f) - mean;
+      float d = (use ? ldf(cond, k) : 0.f) - cm;
       q += d * d;
     }
     const float rstd = 1.f / sqrtf(warp_sum(q) / (float)r.S + r.eps);
-    for (int64_t k = lane; k < r.S; k += kWarp) {
-      float v = use ? ldf(cond, k) : 0.f;
-      r.rawc[row * r.S + k] = v;
-      r.opc[row * r.S + k] = (v - mean) * rstd;
-    }
-  } else {
-    // SiLU(condition) feeds w_mod (bullet 10)
-    for (int64_t k = lane; k < r.S; k += kWarp) {
-      float v = use ? ldf(cond, k) : 0.f;
-      r.opc[row * r.S + k] = siluf_(v);
+    if (lane == 0) {
+      r.cstats[2 * row] = cm;
+      r.cstats[2 * row + 1] = rstd;
     }
   }
 }
 
-// Four consecutive elements as floats (16-byte float32 / 8-byte bf16 loads).
+// Four consecutive elements as floats (16-byte float32 / 8-byte bf16 loads), and four
+// floats stored in the element type; the bf16 store rounds the values in place, so the
+// caller's copy equals what was stored.
 __device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 __device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p) {
   const uint2 u = *reinterpret_cast<const uint2 *>(p);
   return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
                      __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+}
+__device__ __forceinline__ void st4(float *p, float *v) {
+  *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void st4(__nv_bfloat16 *p, float *v) {
+  uint32_t u[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const __nv_bfloat16 a = __float2bfloat16_rn(v[2 * i]), b = __float2bfloat16_rn(v[2 * i + 1]);
+    v[2 * i] = __bfloat162float(a);
+    v[2 * i + 1] = __bfloat162float(b);
+    u[i] = (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
+  }
+  *reinterpret_cast<uint2 *>(p) = make_uint2(u[0], u[1]);
 }
 
 // k_rows_prep for C, S multiples of 4 up to 256 (aligned rows): the same arithmetic with
@@ -122,7 +133,7 @@ __global__ void k_rows_prep_reg(RowsArgs r) {
     const int c = h * 128 + 4 * lane;
     float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
     if (use && c < C) x = ld4((const T *)r.atom + row * C + c);
-    if (use && c < S) y = ld4((const T *)r.condition + row * S + c);
+    if (r.af3 && use && c < S) y = ld4((const T *)r.condition + row * S + c);
     xv[4 * h] = x.x; xv[4 * h + 1] = x.y; xv[4 * h + 2] = x.z; xv[4 * h + 3] = x.w;
     cv[4 * h] = y.x; cv[4 * h + 1] = y.y; cv[4 * h + 2] = y.z; cv[4 * h + 3] = y.w;
   }
@@ -135,8 +146,9 @@ __global__ void k_rows_prep_reg(RowsArgs r) {
       atomicMax(r.tok_last + b * r.T + t, (int)a);
     }
   }
-  // x = atom, or skip + gathered token projection (bullet 3); its row statistics
-  // (AF3 population LayerNorm, bullet 7; ESMFold2 RMS, bullet 11)
+  // x = atom, or skip + gathered token projection (bullet 3), stored in the storage type;
+  // the row statistics of the stored values (AF3 population LayerNorm, bullet 7;
+  // ESMFold2 RMS, bullet 11)
   float s1 = 0.f;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -146,8 +158,7 @@ __global__ void k_rows_prep_reg(RowsArgs r) {
         const float4 tp = ld4(r.token_proj + (b * r.T + t) * C + c);
         xv[4 * h] += tp.x; xv[4 * h + 1] += tp.y; xv[4 * h + 2] += tp.z; xv[4 * h + 3] += tp.w;
       }
-      *reinterpret_cast<float4 *>(r.x + row * C + c) =
-          make_float4(xv[4 * h], xv[4 * h + 1], xv[4 * h + 2], xv[4 * h + 3]);
+      st4(static_cast<T *>(r.x) + row * C + c, xv + 4 * h);
       s1 += (xv[4 * h] + xv[4 * h + 1]) + (xv[4 * h + 2] + xv[4 * h + 3]);
     }
   }
@@ -167,7 +178,7 @@ __global__ void k_rows_prep_reg(RowsArgs r) {
     r.xstats[2 * row + 1] = 1.f / sqrtf(s2 / (float)C + r.eps);
   }
   if (r.af3) {
-    // population LayerNorm of the condition, eps inside the root (bullet 7)
+    // population LayerNorm statistics of the condition, eps inside the root (bullet 7)
     float sc = 0.f;
 #pragma unroll
     for (int h = 0; h < 2; ++h)
@@ -183,26 +194,9 @@ __global__ void k_rows_prep_reg(RowsArgs r) {
           q = fmaf(d, d, q);
         }
     const float rstd = 1.f / sqrtf(warp_sum(q) / (float)S + r.eps);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int c = h * 128 + 4 * lane;
-      if (c < S) {
-        *reinterpret_cast<float4 *>(r.rawc + row * S + c) =
-            make_float4(cv[4 * h], cv[4 * h + 1], cv[4 * h + 2], cv[4 * h + 3]);
-        *reinterpret_cast<float4 *>(r.opc + row * S + c) =
-            make_float4((cv[4 * h] - cm) * rstd, (cv[4 * h + 1] - cm) * rstd,
-                        (cv[4 * h + 2] - cm) * rstd, (cv[4 * h + 3] - cm) * rstd);
-      }
-    }
-  } else {
-    // SiLU(condition) feeds w_mod (bullet 10)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int c = h * 128 + 4 * lane;
-      if (c < S)
-        *reinterpret_cast<float4 *>(r.opc + row * S + c) =
-            make_float4(siluf_(cv[4 * h]), siluf_(cv[4 * h + 1]), siluf_(cv[4 * h + 2]),
-                        siluf_(cv[4 * h + 3]));
+    if (lane == 0) {
+      r.cstats[2 * row] = cm;
+      r.cstats[2 * row + 1] = rstd;
     }
   }
 }
@@ -212,38 +206,39 @@ struct FeatArgs {
   int64_t rows, C;
   float eps;
   int af3;
-  const float *x;     // [rows, C]
-  const float *cond;  // AF3 [rows, 6C] = (sig(scale_j + b), shift_j) j=0..2; ESM [rows, 6C] raw
+  const void *x;      // [rows, C] storage type
+  const void *cond;   // storage type; AF3 [rows, 6C] = (sig(scale_j + b), shift_j) j=0..2; ESM [rows, 6C] raw
   float *feat;        // AF3 [rows, 2C] = (A_0(x), A_1(x)); ESM [rows, C] attention input
 };
 
 // AF3: A_j(x) = LN(x) * sigmoid(c_j @ w_scale[j] + b_scale[j]) + c_j @ w_shift[j]  (bullet 7)
 // ESM: attention input = RMS(x) * (1 + attention_scale) + attention_shift  (bullet 11)
+template <typename IT>
 __global__ void k_features(FeatArgs f) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= f.rows) return;
-  const float *x = f.x + row * f.C;
-  const float *cd = f.cond + row * 6 * f.C;
+  const IT *x = static_cast<const IT *>(f.x) + row * f.C;
+  const IT *cd = static_cast<const IT *>(f.cond) + row * 6 * f.C;
   if (f.af3) {
     float s = 0.f;
-    for (int64_t c = lane; c < f.C; c += kWarp) s += x[c];
+    for (int64_t c = lane; c < f.C; c += kWarp) s += ldf(x, c);
     const float mean = warp_sum(s) / (float)f.C;
     float q = 0.f;
-    for (int64_t c = lane; c < f.C; c += kWarp) q += (x[c] - mean) * (x[c] - mean);
+    for (int64_t c = lane; c < f.C; c += kWarp) q += (ldf(x, c) - mean) * (ldf(x, c) - mean);
     const float rstd = 1.f / sqrtf(warp_sum(q) / (float)f.C + f.eps);
     for (int64_t c = lane; c < f.C; c += kWarp) {
-      float ln = (x[c] - mean) * rstd;
-      f.feat[row * 2 * f.C + c] = ln * cd[c] + cd[f.C + c];
-      f.feat[row * 2 * f.C + f.C + c] = ln * cd[2 * f.C + c] + cd[3 * f.C + c];
+      float ln = (ldf(x, c) - mean) * rstd;
+      f.feat[row * 2 * f.C + c] = ln * ldf(cd, c) + ldf(cd, f.C + c);
+      f.feat[row * 2 * f.C + f.C + c] = ln * ldf(cd, 2 * f.C + c) + ldf(cd, 3 * f.C + c);
     }
   } else {
     float q = 0.f;
-    for (int64_t c = lane; c < f.C; c += kWarp) q += x[c] * x[c];
+    for (int64_t c = lane; c < f.C; c += kWarp) q += ldf(x, c) * ldf(x, c);
     const float rstd = 1.f / sqrtf(warp_sum(q) / (float)f.C + f.eps);
     for (int64_t c = lane; c < f.C; c += kWarp)
-      f.feat[row * f.C + c] = x[c] * rstd * (1.f + cd[f.C + c]) + cd[c];
+      f.feat[row * f.C + c] = ldf(x, c) * rstd * (1.f + ldf(cd, f.C + c)) + ldf(cd, c);
   }
 }
 
@@ -356,19 +351,20 @@ struct TNormArgs {
   float eps;
   int af3;
   const float *xp;    // [rows, C] x' after the attention residual
-  const float *cond;  // [rows, 6C] as in FeatArgs
+  const void *cond;   // [rows, 6C] as in FeatArgs, storage type
   float *z;           // [rows, C]
 };
 
 // Normalise the NEW residual state: AF3 A_2(x'); ESMFold2
 // RMS(x') * (1 + transition_scale) + transition_shift  (bullet 17)
+template <typename IT>
 __global__ void k_transition_norm(TNormArgs f) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= f.rows) return;
   const float *x = f.xp + row * f.C;
-  const float *cd = f.cond + row * 6 * f.C;
+  const IT *cd = static_cast<const IT *>(f.cond) + row * 6 * f.C;
   if (f.af3) {
     float s = 0.f;
     for (int64_t c = lane; c < f.C; c += kWarp) s += x[c];
@@ -377,13 +373,13 @@ __global__ void k_transition_norm(TNormArgs f) {
     for (int64_t c = lane; c < f.C; c += kWarp) q += (x[c] - mean) * (x[c] - mean);
     const float rstd = 1.f / sqrtf(warp_sum(q) / (float)f.C + f.eps);
     for (int64_t c = lane; c < f.C; c += kWarp)
-      f.z[row * f.C + c] = (x[c] - mean) * rstd * cd[4 * f.C + c] + cd[5 * f.C + c];
+      f.z[row * f.C + c] = (x[c] - mean) * rstd * ldf(cd, 4 * f.C + c) + ldf(cd, 5 * f.C + c);
   } else {
     float q = 0.f;
     for (int64_t c = lane; c < f.C; c += kWarp) q += x[c] * x[c];
     const float rstd = 1.f / sqrtf(warp_sum(q) / (float)f.C + f.eps);
     for (int64_t c = lane; c < f.C; c += kWarp)
-      f.z[row * f.C + c] = x[c] * rstd * (1.f + cd[4 * f.C + c]) + cd[3 * f.C + c];
+      f.z[row * f.C + c] = x[c] * rstd * (1.f + ldf(cd, 4 * f.C + c)) + ldf(cd, 3 * f.C + c);
   }
 }
 
@@ -393,7 +389,7 @@ struct PoolArgs {
   const uint8_t *usable;
   const int64_t *att;
   const int *tok_first, *tok_last;
-  const float *pooled;  // [B*A, U] ReLU(hidden @ w_pool)
+  const void *pooled;   // [B*A, U] ReLU(hidden @ w_pool), storage type
   void *out;            // [B, T, U]
 };
 
@@ -426,7 +422,7 @@ __global__ void __launch_bounds__(kPoolThreads) k_token_mean(PoolArgs p) {
       if (tid < 4) s_flag[kPoolThreads + tid] = 0;
       n += __syncthreads_count(f);
       const int cnt = min(kPoolThreads, last - base + 1);
-      const float *rows = p.pooled + (b * p.A + base) * U + u0 + tid;
+      const T *rows = static_cast<const T *>(p.pooled) + (b * p.A + base) * U + u0 + tid;
       for (int i = 0; i < cnt; i += 4) {
         float x[4][3];
 #pragma unroll
@@ -434,7 +430,7 @@ __global__ void __launch_bounds__(kPoolThreads) k_token_mean(PoolArgs p) {
 #pragma unroll
           for (int c = 0; c < 3; ++c)
             x[e][c] = s_flag[i + e] && u0 + tid + c * kPoolThreads < U
-                          ? rows[(int64_t)(i + e) * U + c * kPoolThreads]
+                          ? ldf(rows, (int64_t)(i + e) * U + c * kPoolThreads)
                           : 0.f;
 #pragma unroll
         for (int e = 0; e < 4; ++e)
@@ -457,7 +453,7 @@ struct ReadoutArgs {
   float eps;
   int has_bias;
   const uint8_t *usable;
-  const float *hid;        // [rows, C]
+  const void *hid;         // [rows, C] hidden (the output tensor, storage type)
   const float *scale;      // [C]
   const float *bias;       // [C] ESMFold2
   const float *w_readout;  // [C, 3]
@@ -472,16 +468,16 @@ __global__ void k_readout(ReadoutArgs r) {
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= r.rows) return;
-  const float *x = r.hid + row * r.C;
+  const T *x = static_cast<const T *>(r.hid) + row * r.C;
   float s = 0.f;
-  for (int64_t c = lane; c < r.C; c += kWarp) s += x[c];
+  for (int64_t c = lane; c < r.C; c += kWarp) s += ldf(x, c);
   const float mean = warp_sum(s) / (float)r.C;
   float q = 0.f;
-  for (int64_t c = lane; c < r.C; c += kWarp) q += (x[c] - mean) * (x[c] - mean);
+  for (int64_t c = lane; c < r.C; c += kWarp) q += (ldf(x, c) - mean) * (ldf(x, c) - mean);
   const float rstd = 1.f / sqrtf(warp_sum(q) / (float)r.C + r.eps);
   float o0 = 0.f, o1 = 0.f, o2 = 0.f;
   for (int64_t c = lane; c < r.C; c += kWarp) {
-    float y = (x[c] - mean) * rstd * r.scale[c] + (r.has_bias ? r.bias[c] : 0.f);
+    float y = (ldf(x, c) - mean) * rstd * r.scale[c] + (r.has_bias ? r.bias[c] : 0.f);
     o0 += y * r.w_readout[c * 3 + 0];
     o1 += y * r.w_readout[c * 3 + 1];
     o2 += y * r.w_readout[c * 3 + 2];

@@ -38,16 +38,16 @@ struct TransArgs {
   int HD, M;                   // C is 128
   const void *O;               // [R, HD] gated attention output (float32, or bf16 when
                                // the attention wrote bf16 rows)
-  const float *x;              // [R, 128] residual state start
-  const float *g0, *g1;        // attention / transition residual gates (row stride g_ld)
+  // x, the gates and the transition norm vectors are in the output's storage type
+  const void *x;               // [R, 128] residual state start
+  const void *g0, *g1;         // attention / transition residual gates (row stride g_ld)
   int64_t g_ld;
-  const float *sc, *sh;        // transition norm scale / shift (row stride cond_ld)
+  const void *sc, *sh;         // transition norm scale / shift (row stride cond_ld)
   int64_t cond_ld;
   int rms, plus1;
   float eps;
   const uint8_t *usable;
   const uint8_t *w_out, *w_ff1, *w_ff2;   // packed tensor-core images
-  float *hid32;                // [R, 128] float32 copy of hidden (null: not needed)
   void *hidden;                // [R, 128] output
   unsigned *status;
   // PAIR mode: two CTAs per row block, each on half of the SwiGLU width; w_ff_out partials
@@ -85,7 +85,8 @@ __device__ __forceinline__ void put8(uint8_t *blk, int r, int k, const float (&v
     *reinterpret_cast<uint4 *>(blk + kUmmaBlockBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
 }
 
-// 32 consecutive floats of row r from global memory (zeros when r is out of range)
+// 32 consecutive values of row r from global memory as floats (zeros when r is out of
+// range): float32 rows by 16-byte loads, bf16 rows by 16-byte loads of 8 values
 __device__ __forceinline__ void row32(const float *p, int64_t ld, int64_t r, bool ok, int c0,
                                       float (&v)[32]) {
 #pragma unroll
@@ -96,6 +97,20 @@ __device__ __forceinline__ void row32(const float *p, int64_t ld, int64_t r, boo
     v[i + 1] = x.y;
     v[i + 2] = x.z;
     v[i + 3] = x.w;
+  }
+}
+__device__ __forceinline__ void row32(const __nv_bfloat16 *p, int64_t ld, int64_t r, bool ok, int c0,
+                                      float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 8) {
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (ok) x = *reinterpret_cast<const uint4 *>(p + r * ld + c0 + i);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[i + 2 * e] = __uint_as_float(w[e] << 16);
+      v[i + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+    }
   }
 }
 
@@ -143,6 +158,9 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const TOut *tx = static_cast<const TOut *>(t.x);
+  const TOut *tg0 = static_cast<const TOut *>(t.g0), *tg1 = static_cast<const TOut *>(t.g1);
+  const TOut *tsc = static_cast<const TOut *>(t.sc), *tsh = static_cast<const TOut *>(t.sh);
   // PAIR: CTAs 2p and 2p+1 share row block p; rank k runs SwiGLU chunks [k nL, (k+1) nL)
   // and finishes output columns [64k, 64k + 64)
   const int pb = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x, rank = PAIR ? (int)(blockIdx.x & 1) : 0;
@@ -205,8 +223,8 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
     // partial statistics (shifted by the half's first x'), combined with the other half
     // through shared memory; then z -> operand
     float xv[32], gv[32];                       // chunk 0 fetched before the wait
-    row32(t.x, C, r, rok, cb, xv);
-    row32(t.g0, t.g_ld, r, rok, cb, gv);
+    row32(tx, C, r, rok, cb, xv);
+    row32(tg0, t.g_ld, r, rok, cb, gv);
     if (ok) ok = umma::mbar_wait_warp(acc0_done, 0, abort_flag, lane);
     umma::tc_fence_after();
     float shift = 0.f, s1 = 0.f, s2 = 0.f;
@@ -214,8 +232,8 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
     for (int c0 = cb; c0 < cb + 64; c0 += 32) {
       float a[32];
       if (c0 > cb) {
-        row32(t.x, C, r, rok, c0, xv);
-        row32(t.g0, t.g_ld, r, rok, c0, gv);
+        row32(tx, C, r, rok, c0, xv);
+        row32(tg0, t.g_ld, r, rok, c0, gv);
       }
       umma::tmem_ld32(tl + c0, a);
 #pragma unroll
@@ -251,8 +269,8 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
 #pragma unroll 1
     for (int c0 = cb; c0 < cb + 64; c0 += 32) {
       float a[32], sv[32], hv[32];
-      row32(t.sc, t.cond_ld, r, rok, c0, sv);
-      row32(t.sh, t.cond_ld, r, rok, c0, hv);
+      row32(tsc, t.cond_ld, r, rok, c0, sv);
+      row32(tsh, t.cond_ld, r, rok, c0, hv);
       umma::tmem_ld32(tl + c0, a);
 #pragma unroll
       for (int s8 = 0; s8 < 4; ++s8) {
@@ -307,7 +325,7 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
     const int64_t xrow = ((int64_t)pb * 2 + rank) * 128 + rl;        // this CTA's scratch row
     const int64_t prow = ((int64_t)pb * 2 + (1 - rank)) * 128 + rl;  // the peer's
     float g1v[32];                              // chunk 0 fetched before the wait
-    if (!sender) row32(t.g1, t.g_ld, r, rok, cb, g1v);
+    if (!sender) row32(tg1, t.g_ld, r, rok, cb, g1v);
     const bool use_row = rok && t.usable[r] != 0;
     if (ok) ok = umma::mbar_wait_warp(acc2_done, 0, abort_flag, lane);
     umma::tc_fence_after();
@@ -345,7 +363,7 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
 #pragma unroll 1
       for (int c0 = cb; c0 < cb + 64; c0 += 32) {
         float a[32], f[32];
-        if (c0 > cb) row32(t.g1, t.g_ld, r, rok, c0, g1v);
+        if (c0 > cb) row32(tg1, t.g_ld, r, rok, c0, g1v);
         umma::tmem_ld32(tl + c0, a);
         umma::tmem_ld32(tl + 384 + c0, f);
         if (PAIR) {
@@ -363,7 +381,6 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) o[e] = use ? fmaf(g1v[i + e], f[i + e], a[i + e]) : 0.f;
             const float4 o4 = make_float4(o[0], o[1], o[2], o[3]);
-            if (t.hid32) *reinterpret_cast<float4 *>(t.hid32 + r * C + c0 + i) = o4;
             store4<TOut>((TOut *)t.hidden, r * C + c0 + i, o4);
           }
         }
