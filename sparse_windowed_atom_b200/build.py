@@ -21,9 +21,10 @@ FLAGS = [
     "-O3", "-lineinfo", "-std=c++17",
     # IEEE float32: no fast-math, subnormals kept (the pages keep subnormal tails)
     "-ftz=false", "-prec-div=true", "-prec-sqrt=true", "-fmad=true",
-    "-Xcompiler", "-fPIC", "-shared",
+    "-Xcompiler", "-fPIC",
     "-I", os.path.join(ROOT, "include"),
 ]
+OBJ_DIR = os.path.join(HERE, "_build")
 
 
 def sources():
@@ -43,15 +44,28 @@ def stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every translation unit of csrc/ (in parallel) and link libatomenc.so."""
     if not force and not stale():
         return LIB
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    srcs = sources()
+    objs = [os.path.join(OBJ_DIR, os.path.basename(f)[:-3] + f".{os.getpid()}.o") for f in srcs]
+    extra = ["-Xptxas=-v"] if verbose else []
+    procs = []
+    for src, obj in zip(srcs, objs):
+        cmd = [NVCC, *FLAGS, *extra, "-c", "-o", obj, src]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        procs.append((src, subprocess.Popen(cmd)))
+    failed = [src for src, pr in procs if pr.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, f"nvcc ({', '.join(map(os.path.basename, failed))})")
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *FLAGS, "-o", tmp, *sources()]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.check_call(cmd)
+    subprocess.check_call([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
+                           "-Xcompiler", "-fPIC", "-o", tmp, *objs])
     os.replace(tmp, LIB)
+    for o in objs:
+        os.remove(o)
     return LIB
 
 

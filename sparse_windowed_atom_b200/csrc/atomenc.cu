@@ -15,28 +15,67 @@
 #include <type_traits>
 #include <utility>
 
-#include "../../include/atomenc.h"
-#include "attention.cuh"
-#include "attn_rows.cuh"
-#include "common.cuh"
-#include "epilogues.cuh"
-#include "gemm_umma.cuh"
-#include "rows.cuh"
-#include "transition.cuh"
-#include "weights.cuh"
+#include "host.cuh"
 
 using namespace atomenc;
+using namespace atomenc::host;
+
+namespace atomenc {
+namespace host {
+
+std::atomic<uint32_t> g_peer_spin_limit{kPeerSpinLimit};
+std::atomic<int> g_peer_withhold{0};
+
+struct SmemLimit {
+  const void *fn;
+  int dev, bytes;
+};
+constexpr int kMaxSmemLimits = 512;
+SmemLimit g_smem_limits[kMaxSmemLimits];
+int g_num_smem_limits = 0;
+std::mutex g_smem_limits_mutex;
+
+cudaError_t smem_limit_fn(const void *fn, size_t bytes) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  std::lock_guard<std::mutex> lock(g_smem_limits_mutex);
+  int slot = -1;
+  for (int i = 0; i < g_num_smem_limits; ++i)
+    if (g_smem_limits[i].fn == fn && g_smem_limits[i].dev == dev) slot = i;
+  if (slot >= 0 && (int)bytes <= g_smem_limits[slot].bytes) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess || dev < 0) return e;
+  if (slot < 0 && g_num_smem_limits < kMaxSmemLimits) {
+    slot = g_num_smem_limits++;
+    g_smem_limits[slot].fn = fn;
+    g_smem_limits[slot].dev = dev;
+  }
+  if (slot >= 0) g_smem_limits[slot].bytes = (int)bytes;
+  return e;
+}
+
+}  // namespace host
+}  // namespace atomenc
 
 namespace {
 
 constexpr int kVersion = 1;
-constexpr int kMaxD = 64;
-constexpr size_t kAttnSmemBudget = 210 * 1024;  // dynamic part: one CTA per SM, or per two (AF3) / 2 - 1 KB
-constexpr size_t kRowAttnSmemBudget = 220 * 1024;  // dynamic part of the row-gather attention
 
-struct Dims {
-  int64_t B = 0, A = 0, T = 0, K = 0, C = 0, S = 0, H = 0, D = 0, P = 0, M = 0, U = 0, V = 0;
-};
+// Multiprocessors of the current device, looked up once per device.
+int g_sm_count[kMaxDevices];
+std::mutex g_sm_mutex;
+int sm_count() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lock(g_sm_mutex);
+  if (g_sm_count[dev] <= 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_sm_count[dev] = n;
+  }
+  return g_sm_count[dev];
+}
 
 bool present(const atomenc_tensor &t) { return t.data != nullptr && t.ndim > 0; }
 
@@ -67,47 +106,6 @@ float bf16_round_host(float f) {
   std::memcpy(&f, &u, 4);
   return f;
 }
-
-constexpr int kMaxDevices = 64;
-
-// Multiprocessors of the current device, looked up once per device.
-int g_sm_count[kMaxDevices];
-std::mutex g_sm_mutex;
-int sm_count() {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-  std::lock_guard<std::mutex> lock(g_sm_mutex);
-  if (g_sm_count[dev] <= 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-    g_sm_count[dev] = n;
-  }
-  return g_sm_count[dev];
-}
-
-struct Plan {
-  int style = 0, stage = 0, fdt = 0;
-  bool af3 = false, enc = false, fuse_tail = false, tail_pair = false;
-  Dims d;
-  // workspace layout (byte offsets)
-  size_t o_status, o_usable, o_xstats, o_cstats, o_first, o_last, o_tp, o_x, o_cond, o_gate, o_feat,
-      o_q, o_k, o_v, o_g, o_o, o_xp, o_z, o_h, o_pool, o_xfer, o_xflag;
-  size_t o_wread, o_bscale, o_brg, o_bq, o_wpair, o_rscale, o_rbias;
-  // tensor-core images of the weight panels (bf16, hi[/lo])
-  size_t k_cond, k_gate, k_qkv0, k_qkv1, k_out, k_ff1, k_ff2, k_pool, k_tok;
-  size_t bytes = 0;
-  // attention launch
-  int QT = 0, DP = 0, kv_floats = 0;
-  size_t attn_smem = 0;
-  int sms = 148;                    // multiprocessors of the device the pass runs on
-  // row-gather attention (k_attn_rows): H*D in {64, 128} ... see attn_rows.cuh; Q, K, V,
-  // value-gate logits and the gated output are then kept in the storage type
-  bool rg = false;
-  int rg_qt = 0, rg_stage_rows = 0;
-  size_t rg_smem = 0;
-  bool ws_bf16 = false;             // Q/K/V/G/O intermediates in bf16
-};
 
 size_t take(size_t &cur, size_t bytes) {
   size_t o = cur;
@@ -346,476 +344,6 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
     pl.rg_smem = rowattn_fixed_smem(q, (int)K, (int)H, es, pl.af3) + 2 * (size_t)pl.rg_stage_rows * rb;
   }
   return ATOMENC_OK;
-}
-
-// Raise a kernel's dynamic shared-memory limit once per (kernel, device), and again only
-// if a larger size is asked for: the attribute outlives the call, so repeating it on
-// every forward would only add host time.
-struct SmemLimit {
-  const void *fn;
-  int dev, bytes;
-};
-constexpr int kMaxSmemLimits = 512;
-SmemLimit g_smem_limits[kMaxSmemLimits];
-int g_num_smem_limits = 0;
-std::mutex g_smem_limits_mutex;
-
-template <typename... KP>
-cudaError_t smem_limit(void (*kern)(KP...), size_t bytes) {
-  const void *fn = reinterpret_cast<const void *>(kern);
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
-  std::lock_guard<std::mutex> lock(g_smem_limits_mutex);
-  int slot = -1;
-  for (int i = 0; i < g_num_smem_limits; ++i)
-    if (g_smem_limits[i].fn == fn && g_smem_limits[i].dev == dev) slot = i;
-  if (slot >= 0 && (int)bytes <= g_smem_limits[slot].bytes) return cudaSuccess;
-  const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e != cudaSuccess || dev < 0) return e;
-  if (slot < 0 && g_num_smem_limits < kMaxSmemLimits) {
-    slot = g_num_smem_limits++;
-    g_smem_limits[slot].fn = fn;
-    g_smem_limits[slot].dev = dev;
-  }
-  if (slot >= 0) g_smem_limits[slot].bytes = (int)bytes;
-  return e;
-}
-
-struct Hooks {
-  cudaEvent_t const *ev = nullptr;  // ATOMENC_NUM_PHASES + 1 events, or null
-  cudaEvent_t const *kev = nullptr; // traced: one event before the pass and one per launch
-  int n_kev = 0;
-  int *kinds = nullptr;             // traced: enum atomenc_kernel_kind per launch
-  int launches = 0;
-  cudaError_t err = cudaSuccess;    // first launch failure
-  bool overflow = false;            // traced: more launches than events
-  void mark(int i, cudaStream_t st) const {
-    if (ev) cudaEventRecord(ev[i], st);
-  }
-  void begin(cudaStream_t st) {
-    if (kev && n_kev > 0) cudaEventRecord(kev[0], st);
-  }
-  // Every kernel is launched here, with programmatic stream serialization: it may be
-  // scheduled while its predecessor finishes and waits for it in pdl_enter(). A
-  // cluster size of 2 launches the grid as CTA pairs that the hardware schedules
-  // together.
-  template <typename... KP, typename... Args>
-  void launch(int kind, void (*kern)(KP...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-              Args &&...args) {
-    launch_cluster(kind, 1, kern, grid, block, smem, st, std::forward<Args>(args)...);
-  }
-  template <typename... KP, typename... Args>
-  void launch_cluster(int kind, int cluster, void (*kern)(KP...), dim3 grid, dim3 block,
-                      size_t smem, cudaStream_t st, Args &&...args) {
-    cudaLaunchAttribute at[2];
-    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[0].val.programmaticStreamSerializationAllowed = 1;
-    int nat = 1;
-    if (cluster > 1) {
-      at[1].id = cudaLaunchAttributeClusterDimension;
-      at[1].val.clusterDim.x = (unsigned)cluster;
-      at[1].val.clusterDim.y = 1;
-      at[1].val.clusterDim.z = 1;
-      nat = 2;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cfg.attrs = at;
-    cfg.numAttrs = nat;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
-    if (e != cudaSuccess && err == cudaSuccess) err = e;
-    if (kev) {
-      if (launches + 1 < n_kev) {
-        cudaEventRecord(kev[launches + 1], st);
-        if (kinds) kinds[launches] = kind;
-      } else {
-        overflow = true;
-      }
-    }
-    ++launches;
-  }
-};
-
-// Test hook for the bounded wait of the paired transition CTAs (see
-// atomenc_debug_peer_wait): poll limit, and whether the partials' flags are withheld.
-std::atomic<uint32_t> g_peer_spin_limit{kPeerSpinLimit};
-std::atomic<int> g_peer_withhold{0};
-
-template <typename Elt>
-int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p,
-               float eps, int64_t radius, const atomenc_outputs *out, unsigned char *ws,
-               cudaStream_t st, Hooks &hk) {
-  const Dims &d = pl.d;
-  const int64_t B = d.B, A = d.A, T = d.T, K = d.K, C = d.C, S = d.S, H = d.H, D = d.D,
-                P = d.P, M = d.M, U = d.U, V = d.V, HD = H * D, R = B * A;
-  auto F = [&](size_t off) { return reinterpret_cast<float *>(ws + off); };
-  unsigned *status = reinterpret_cast<unsigned *>(ws + pl.o_status);
-  uint8_t *usable = ws + pl.o_usable;
-  int *first = reinterpret_cast<int *>(ws + pl.o_first);
-  int *last = reinterpret_cast<int *>(ws + pl.o_last);
-
-  hk.mark(0, st);
-
-  // ---- one launch: tensor-core images of the projection weights (built from the
-  // caller's tensors), small float32 panels, status and token-range resets
-  WeightJobs wj;
-  std::memset(&wj, 0, sizeof(wj));
-  const size_t es = sizeof(Elt);
-  auto elt = [&](const atomenc_tensor &t, size_t off) -> const void * {
-    return t.data ? static_cast<const unsigned char *>(t.data) + off * es : nullptr;
-  };
-  auto copy = [&](const atomenc_tensor &src, size_t src_off, int64_t rows, int64_t cols, size_t dst_off,
-                  int64_t dst_ld, int64_t col0, const atomenc_tensor *rowscale, size_t rs_off) {
-    CopyJob &j = wj.copy[wj.ncopy++];
-    j.src = elt(src, src_off);
-    j.rowscale = rowscale ? elt(*rowscale, rs_off) : nullptr;
-    j.dst = F(dst_off);
-    j.rows = (int32_t)rows;
-    j.cols = (int32_t)cols;
-    j.dst_ld = (int32_t)dst_ld;
-    j.dst_col0 = (int32_t)col0;
-    j.dst_cstride = 1;
-  };
-  const bool split = pl.fdt == ATOMENC_F32;
-  auto pack = [&](size_t dst, int64_t Kd, int64_t N) -> PackJob & {
-    PackJob &j = wj.pack[wj.npack++];
-    j.dst = ws + dst;
-    j.K = (int32_t)Kd;
-    j.N = (int32_t)N;
-    j.split = split ? 1 : 0;
-    return j;
-  };
-  auto seg = [&](PackJob &j, const atomenc_tensor &src, size_t src_off, int64_t cols, int64_t col0,
-                 int cshift, const atomenc_tensor *rowscale, size_t rs_off) {
-    PackSeg &g = j.seg[j.nseg++];
-    g.src = elt(src, src_off);
-    g.rowscale = rowscale ? elt(*rowscale, rs_off) : nullptr;
-    g.cols = (int32_t)cols;
-    g.col0 = (int32_t)col0;
-    g.cshift = cshift;
-  };
-  if (pl.af3) {
-    PackJob &jc = pack(pl.k_cond, S, 6 * C);
-    for (int jj = 0; jj < 3; ++jj) {
-      seg(jc, p->w_scale, (size_t)jj * S * C, C, 2 * jj * C, 0, &p->cond_scale, (size_t)jj * S);
-      seg(jc, p->w_shift, (size_t)jj * S * C, C, 2 * jj * C + C, 0, &p->cond_scale, (size_t)jj * S);
-    }
-    PackJob &jg = pack(pl.k_gate, S, 2 * C);
-    seg(jg, p->w_residual_gate, 0, C, 0, 0, nullptr, 0);
-    seg(jg, p->w_residual_gate, (size_t)S * C, C, C, 0, nullptr, 0);
-    PackJob &j0 = pack(pl.k_qkv0, C, 2 * HD);
-    seg(j0, p->w_q, 0, HD, 0, 0, nullptr, 0);
-    seg(j0, p->w_value_gate, 0, HD, HD, 0, nullptr, 0);
-    PackJob &j1 = pack(pl.k_qkv1, C, 2 * HD);
-    seg(j1, p->w_k, 0, HD, 0, 0, nullptr, 0);
-    seg(j1, p->w_v, 0, HD, HD, 0, nullptr, 0);
-    copy(p->b_scale, 0, 1, 3 * C, pl.o_bscale, 3 * C, 0, nullptr, 0);
-    copy(p->b_residual_gate, 0, 1, 2 * C, pl.o_brg, 2 * C, 0, nullptr, 0);
-    copy(p->b_q, 0, 1, HD, pl.o_bq, HD, 0, nullptr, 0);
-    copy(p->w_pair, 0, P, H, pl.o_wpair, H, 0, &p->pair_scale, 0);
-  } else {
-    seg(pack(pl.k_cond, S, 6 * C), p->w_mod, 0, 6 * C, 0, 0, nullptr, 0);
-    PackJob &j0 = pack(pl.k_qkv0, C, 4 * HD);
-    seg(j0, p->w_q, 0, HD, 0, 0, nullptr, 0);
-    seg(j0, p->w_k, 0, HD, HD, 0, nullptr, 0);
-    seg(j0, p->w_v, 0, HD, 2 * HD, 0, nullptr, 0);
-    seg(j0, p->w_value_gate, 0, HD, 3 * HD, 0, nullptr, 0);
-  }
-  seg(pack(pl.k_out, HD, C), p->w_attention_out, 0, C, 0, 0, nullptr, 0);
-  PackJob &jf = pack(pl.k_ff1, C, 2 * M);
-  seg(jf, p->w_ff_gate, 0, M, 0, 1, nullptr, 0);
-  seg(jf, p->w_ff_up, 0, M, 1, 1, nullptr, 0);
-  seg(pack(pl.k_ff2, M, C), p->w_ff_out, 0, C, 0, 0, nullptr, 0);
-  if (pl.enc) {
-    seg(pack(pl.k_pool, C, U), p->w_pool, 0, U, 0, 0, nullptr, 0);
-  } else {
-    seg(pack(pl.k_tok, V, C), p->w_token, 0, C, 0, 0, nullptr, 0);
-    copy(p->readout_scale, 0, 1, C, pl.o_rscale, C, 0, nullptr, 0);
-    if (!pl.af3) copy(p->readout_bias, 0, 1, C, pl.o_rbias, C, 0, nullptr, 0);
-    copy(p->w_readout, 0, C, 3, pl.o_wread, 3, 0, nullptr, 0);
-  }
-  wj.fill[wj.nfill++] = FillJob{reinterpret_cast<int *>(status), 1, 0, 0};
-  if (pl.tail_pair)
-    wj.fill[wj.nfill++] = FillJob{reinterpret_cast<int *>(ws + pl.o_xflag), 2 * ((R + kUmmaBM - 1) / kUmmaBM), 0, 0};
-  if (pl.enc) {
-    wj.fill[wj.nfill++] = FillJob{first, B * T, INT_MAX, 0};
-    wj.fill[wj.nfill++] = FillJob{last, B * T, -1, 0};
-  }
-  hk.launch(ATOMENC_KERNEL_PREP, (k_prep_weights<Elt>), dim3(64, wj.ncopy + wj.npack + wj.nfill), 256, 0, st, wj);
-
-  // out = epi(A' @ W) on the tensor cores, W given by its packed image and A' produced by
-  // `prod` (A itself, or a row normalisation fused into the operand); K <= 256
-  auto gemm_rows = [&](auto prod, size_t wpk, int64_t Mr, int64_t N, int64_t Kd, auto epi) {
-    using P = decltype(prod);
-    using E = decltype(epi);
-    const int64_t mt = (Mr + kUmmaBM - 1) / kUmmaBM, nt = (N + kUmmaBN - 1) / kUmmaBN;
-    const int64_t want = (pl.sms + mt - 1) / mt;          // CTAs per row block to fill the GPU
-    const int64_t sp = want < nt ? want : nt;
-    const int per = (int)((nt + sp - 1) / sp);
-    dim3 grid((unsigned)((nt + per - 1) / per), (unsigned)mt);
-    const size_t smem = rows_smem_bytes(Kd, split);
-    if (split) {
-      smem_limit(k_gemm_rows<P, true, E>, smem);
-      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_rows<P, true, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, epi, status);
-    } else {
-      smem_limit(k_gemm_rows<P, false, E>, smem);
-      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_rows<P, false, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, epi, status);
-    }
-  };
-  // out = epi(A @ W): the row-block kernel for K <= 256, else the streaming kernel
-  auto gemm = [&](auto *A_, int64_t lda, size_t wpk, int64_t Mr, int64_t N, int64_t Kd, auto epi) {
-    using TA = std::remove_cv_t<std::remove_pointer_t<decltype(A_)>>;
-    using E = decltype(epi);
-    if (Kd <= kRowsKMax) {
-      gemm_rows(ProdPlain<TA>{A_, lda, Mr, Kd}, wpk, Mr, N, Kd, epi);
-      return;
-    }
-    dim3 grid((unsigned)((N + kUmmaBN - 1) / kUmmaBN), (unsigned)((Mr + kUmmaBM - 1) / kUmmaBM));
-    const size_t smem = umma_smem_bytes(split);
-    if (split) {
-      smem_limit(k_gemm_umma<TA, true, E>, smem);
-      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_umma<TA, true, E>), grid, kUmmaThreads, smem, st, A_, lda, ws + wpk, Mr, N, Kd, epi, status);
-    } else {
-      smem_limit(k_gemm_umma<TA, false, E>, smem);
-      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_umma<TA, false, E>), grid, kUmmaThreads, smem, st, A_, lda, ws + wpk, Mr, N, Kd, epi, status);
-    }
-  };
-  // the conditioning-modulated row norm of x (or x') fused into a projection's operand
-  const bool fuse_norm = C <= kRowsKMax;
-  Elt *xb = reinterpret_cast<Elt *>(ws + pl.o_x), *condb = reinterpret_cast<Elt *>(ws + pl.o_cond),
-      *gateb = reinterpret_cast<Elt *>(ws + pl.o_gate), *poolb = reinterpret_cast<Elt *>(ws + pl.o_pool);
-  auto norm_prod = [&](int64_t sc_off, int64_t sh_off, bool plus1) {
-    return ProdNormT<Elt>{xb, F(pl.o_xstats), condb, R, C, 6 * C, sc_off, sh_off, plus1 ? 1 : 0};
-  };
-  const int rows_per_block = 8;  // warps per 256-thread block for warp-per-row kernels
-  const unsigned row_blocks = (unsigned)((R + rows_per_block - 1) / rows_per_block);
-
-  // ---- decoder: token @ w_token, gathered per atom in the row pass
-  if (!pl.enc)
-    gemm(static_cast<const Elt *>(in->token.data), V, pl.k_tok, B * T, C, V,
-         Quad<EpiStore>{{F(pl.o_tp), C}});
-
-  // ---- usable, sanitised residual start, normalised condition
-  RowsArgs ra;
-  ra.B = B; ra.A = A; ra.T = T; ra.C = C; ra.S = S; ra.eps = eps;
-  ra.af3 = pl.af3; ra.decoder = !pl.enc; ra.encoder = pl.enc;
-  ra.atom = in->atom.data; ra.condition = in->condition.data;
-  ra.valid = static_cast<const uint8_t *>(in->valid.data);
-  ra.token_valid = static_cast<const uint8_t *>(in->token_valid.data);
-  ra.att = static_cast<const int64_t *>(in->atom_to_token.data);
-  ra.token_proj = F(pl.o_tp);
-  ra.usable = usable; ra.x = xb; ra.xstats = F(pl.o_xstats); ra.cstats = F(pl.o_cstats);
-  ra.tok_first = first; ra.tok_last = last;
-  {
-    const uintptr_t al = sizeof(Elt) == 4 ? 15 : 7;   // 4-element loads of atom / condition rows
-    const bool reg = C % 4 == 0 && S % 4 == 0 && C <= 256 && S <= 256 &&
-                     ((reinterpret_cast<uintptr_t>(in->atom.data) | reinterpret_cast<uintptr_t>(in->condition.data)) & al) == 0;
-    if (reg)
-      hk.launch(ATOMENC_KERNEL_ROWS, (k_rows_prep_reg<Elt>), row_blocks, 256, 0, st, ra);
-    else
-      hk.launch(ATOMENC_KERNEL_ROWS, (k_rows_prep<Elt>), row_blocks, 256, 0, st, ra);
-  }
-  hk.mark(1, st);
-
-  // ---- conditioning: the operand (LN(c), raw c or SiLU(c) of the sanitised condition)
-  // is formed from the caller's condition rows inside the product
-  const Elt *cin = static_cast<const Elt *>(in->condition.data);
-  if (pl.af3) {
-    gemm_rows(ProdCond<Elt, 2>{cin, usable, F(pl.o_cstats), R, S}, pl.k_cond, R, 6 * C, S,
-              EpiCondAF3<Elt>{condb, F(pl.o_bscale), C});
-    gemm_rows(ProdCond<Elt, 0>{cin, usable, nullptr, R, S}, pl.k_gate, R, 2 * C, S,
-              EpiGateAF3<Elt>{gateb, F(pl.o_brg), C});
-  } else {
-    gemm_rows(ProdCond<Elt, 1>{cin, usable, nullptr, R, S}, pl.k_cond, R, 6 * C, S,
-              Quad<EpiStoreT<Elt>>{{condb, 6 * C}});
-  }
-  hk.mark(2, st);
-  if (!fuse_norm) {
-    FeatArgs fa{R, C, eps, pl.af3 ? 1 : 0, xb, condb, F(pl.o_feat)};
-    hk.launch(ATOMENC_KERNEL_ROWS, (k_features<Elt>), row_blocks, 256, 0, st, fa);
-  }
-
-  // ---- projections .. transition; WT is the type of the Q/K/V/G/O intermediates
-  // (bf16 for bf16 workloads on the row-gather attention, float32 otherwise)
-  auto middle = [&](auto wt_tag) {
-    using WT = decltype(wt_tag);
-    WT *wq = reinterpret_cast<WT *>(ws + pl.o_q), *wk = reinterpret_cast<WT *>(ws + pl.o_k),
-       *wv = reinterpret_cast<WT *>(ws + pl.o_v), *wg = reinterpret_cast<WT *>(ws + pl.o_g),
-       *wo = reinterpret_cast<WT *>(ws + pl.o_o);
-    // ---- projections (attention inputs fused into the operand when C <= 256)
-    if (pl.af3) {
-      EpiSplitT<WT> e0{{wq, wg, nullptr, nullptr}, {F(pl.o_bq), nullptr, nullptr, nullptr}, HD};
-      EpiSplitT<WT> e1{{wk, wv, nullptr, nullptr}, {nullptr, nullptr, nullptr, nullptr}, HD};
-      if (fuse_norm) {
-        gemm_rows(norm_prod(0, C, false), pl.k_qkv0, R, 2 * HD, C, e0);
-        gemm_rows(norm_prod(2 * C, 3 * C, false), pl.k_qkv1, R, 2 * HD, C, e1);
-      } else {
-        gemm(F(pl.o_feat), 2 * C, pl.k_qkv0, R, 2 * HD, C, e0);
-        gemm(F(pl.o_feat) + C, 2 * C, pl.k_qkv1, R, 2 * HD, C, e1);
-      }
-    } else {
-      EpiSplitT<WT> e{{wq, wk, wv, wg}, {nullptr, nullptr, nullptr, nullptr}, HD};
-      if (fuse_norm)
-        gemm_rows(norm_prod(C, 0, true), pl.k_qkv0, R, 4 * HD, C, e);
-      else
-        gemm(F(pl.o_feat), C, pl.k_qkv0, R, 4 * HD, C, e);
-      RopeArgs rp{R, H, D, eps, usable, in->rope_cos.data, in->rope_sin.data, wq, wk};
-      if (D >= 8 && D <= 128 && (D & (D - 1)) == 0) {
-        const int64_t warps = R * 2;
-        hk.launch(ATOMENC_KERNEL_ROWS, (k_qk_rope_warp<Elt, WT>), (unsigned)((warps + 7) / 8), 256, 0, st, rp);
-      } else {
-        const int64_t n = R * H * 2;
-        hk.launch(ATOMENC_KERNEL_ROWS, (k_qk_rope<Elt>), (unsigned)((n + 255) / 256), 256, 0, st, rp);
-      }
-    }
-    hk.mark(3, st);
-
-    // ---- slot-gathered attention
-    const int rad = radius < 0 ? -1 : (radius > INT_MAX ? INT_MAX : (int)radius);
-    if (pl.rg) {
-      RowAttnArgs ra2;
-      ra2.B = (int)B; ra2.A = (int)A; ra2.K = (int)K; ra2.H = (int)H; ra2.D = (int)D; ra2.P = (int)P;
-      ra2.radius = rad;
-      ra2.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-      ra2.eps = eps;
-      ra2.QT = pl.rg_qt;
-      ra2.stage_rows = pl.rg_stage_rows;
-      ra2.Q = wq; ra2.Kf = wk; ra2.Vf = wv; ra2.G = wg;
-      ra2.key_index = static_cast<const int64_t *>(in->key_index.data);
-      ra2.window = static_cast<const uint8_t *>(in->window_mask.data);
-      ra2.usable = usable;
-      ra2.pair = pl.af3 ? in->pair.data : nullptr;
-      ra2.w_pair = F(pl.o_wpair);
-      ra2.attention = out->attention.data;
-      ra2.O = wo;
-      ra2.status = status;
-      ra2.pair_vec = pl.af3 && P == 16 && (reinterpret_cast<uintptr_t>(in->pair.data) & 15) == 0;
-      ra2.att_vec = (reinterpret_cast<uintptr_t>(out->attention.data) & 15) == 0;
-      dim3 grid((unsigned)((A + pl.rg_qt - 1) / pl.rg_qt), (unsigned)B);
-      auto go = [&](auto kern) {
-        smem_limit(kern, pl.rg_smem);
-        hk.launch(ATOMENC_KERNEL_ATTENTION, kern, grid, kRowAttnThreads, pl.rg_smem, st, ra2);
-      };
-      // the attention weights are written in the storage type: WT == Elt here
-      if constexpr (std::is_same<WT, Elt>::value) {
-#define ROWATTN(DH)                                                 \
-  if (D == DH) {                                                    \
-    if (pl.af3) go(k_attn_rows<WT, 128, DH, true>);                 \
-    else go(k_attn_rows<WT, 128, DH, false>);                       \
-  }
-        ROWATTN(16) ROWATTN(32) ROWATTN(64)
-#undef ROWATTN
-      }
-    } else {
-      AttnArgs ag;
-      ag.B = (int)B; ag.A = (int)A; ag.K = (int)K; ag.H = (int)H; ag.D = (int)D; ag.P = (int)P;
-      ag.radius = rad;
-      ag.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-      ag.eps = eps;
-      ag.QT = pl.QT; ag.DP = pl.DP; ag.kv_floats = pl.kv_floats;
-      ag.kmagic = K > 1 ? (uint32_t)(((uint64_t)1 << 32) / (uint64_t)K + (((uint64_t)1 << 32) % (uint64_t)K != 0)) : 0u;
-      ag.Q = F(pl.o_q); ag.Kf = F(pl.o_k); ag.Vf = F(pl.o_v); ag.G = F(pl.o_g);
-      ag.key_index = static_cast<const int64_t *>(in->key_index.data);
-      ag.window = static_cast<const uint8_t *>(in->window_mask.data);
-      ag.usable = usable;
-      ag.pair = pl.af3 ? in->pair.data : nullptr;
-      ag.w_pair = F(pl.o_wpair);
-      ag.attention = out->attention.data;
-      ag.O = F(pl.o_o);
-      ag.status = status;
-      dim3 grid((unsigned)((A + pl.QT - 1) / pl.QT), (unsigned)B);
-      auto go = [&](auto kern) {
-        smem_limit(kern, pl.attn_smem);
-        hk.launch(ATOMENC_KERNEL_ATTENTION, kern, grid, attn_threads(pl.af3), pl.attn_smem, st, ag);
-      };
-      const int dm = D <= 8 ? 8 : D <= 16 ? 16 : D <= 32 ? 32 : 64;
-      const bool multi = K > kChunk;
-#define ATTN_D(DM)                                                          \
-  if (dm == DM) {                                                           \
-    if (pl.af3)                                                             \
-      multi ? go(k_slot_attention<Elt, DM, true, true>)                     \
-            : go(k_slot_attention<Elt, DM, true, false>);                   \
-    else                                                                    \
-      multi ? go(k_slot_attention<Elt, DM, false, true>)                    \
-            : go(k_slot_attention<Elt, DM, false, false>);                  \
-  }
-      ATTN_D(8) ATTN_D(16) ATTN_D(32) ATTN_D(64)
-#undef ATTN_D
-    }
-
-    hk.mark(4, st);
-
-    // ---- out-projection + gated residual, transition norm, SwiGLU, gated residual + mask
-    const Elt *gbuf = pl.af3 ? gateb : condb;
-    const int64_t gld = pl.af3 ? 2 * C : 6 * C;
-    const int64_t g0off = pl.af3 ? 0 : 2 * C, g1off = pl.af3 ? C : 5 * C;
-    if (pl.fuse_tail) {
-      TransArgs ta;
-      ta.R = R; ta.HD = (int)HD; ta.M = (int)M;
-      ta.O = wo; ta.x = xb;
-      ta.g0 = gbuf + g0off; ta.g1 = gbuf + g1off; ta.g_ld = gld;
-      ta.sc = condb + 4 * C; ta.sh = condb + (pl.af3 ? 5 : 3) * C; ta.cond_ld = 6 * C;
-      ta.rms = pl.af3 ? 0 : 1; ta.plus1 = pl.af3 ? 0 : 1; ta.eps = eps;
-      ta.usable = usable;
-      ta.w_out = ws + pl.k_out; ta.w_ff1 = ws + pl.k_ff1; ta.w_ff2 = ws + pl.k_ff2;
-      ta.hidden = out->hidden.data; ta.status = status;
-      ta.xfer = F(pl.o_xfer); ta.xflag = reinterpret_cast<int *>(ws + pl.o_xflag);
-      ta.peer_spin_limit = g_peer_spin_limit.load();
-      ta.withhold_flag = g_peer_withhold.load();
-      const size_t smem = trans_smem_bytes(split);
-      const dim3 grid((unsigned)(((R + kUmmaBM - 1) / kUmmaBM) * (pl.tail_pair ? 2 : 1)));
-      // the two CTAs of a row block exchange partials: launched as a 2-CTA cluster, so
-      // that they are always resident at the same time
-      auto go = [&](auto kern) {
-        smem_limit(kern, smem);
-        hk.launch_cluster(ATOMENC_KERNEL_TRANSITION, pl.tail_pair ? 2 : 1, kern, grid, kTransThreads,
-                          smem, st, ta);
-      };
-      if constexpr (std::is_same<Elt, float>::value) {
-        pl.tail_pair ? go(k_transition<true, Elt, true, WT>) : go(k_transition<true, Elt, false, WT>);
-      } else {
-        pl.tail_pair ? go(k_transition<false, Elt, true, WT>) : go(k_transition<false, Elt, false, WT>);
-      }
-    } else {
-      gemm(static_cast<const WT *>(wo), HD, pl.k_out, R, C, HD,
-           Quad<EpiResidual<Elt>>{{xb, gbuf, gld, g0off, C, F(pl.o_xp)}});
-      TNormArgs tn{R, C, eps, pl.af3 ? 1 : 0, F(pl.o_xp), condb, F(pl.o_z)};
-      hk.launch(ATOMENC_KERNEL_ROWS, (k_transition_norm<Elt>), row_blocks, 256, 0, st, tn);
-      gemm(F(pl.o_z), C, pl.k_ff1, R, 2 * M, C, EpiSwiGLU{F(pl.o_h), M});
-      gemm(F(pl.o_h), M, pl.k_ff2, R, C, M,
-           Quad<EpiHidden<Elt>>{{F(pl.o_xp), gbuf, gld, g1off, C, usable,
-                                 static_cast<Elt *>(out->hidden.data)}});
-    }
-  };
-  if constexpr (std::is_same<Elt, __nv_bfloat16>::value) {
-    if (pl.ws_bf16)
-      middle(__nv_bfloat16{});
-    else
-      middle(float{});
-  } else {
-    middle(float{});
-  }
-
-  hk.mark(5, st);
-
-  // ---- boundary, read from the hidden output itself
-  const Elt *hid = static_cast<const Elt *>(out->hidden.data);
-  if (pl.enc) {
-    gemm(hid, C, pl.k_pool, R, U, C, Quad<EpiRelu<Elt>>{{poolb, U}});
-    PoolArgs pa{B, A, T, U, usable, static_cast<const int64_t *>(in->atom_to_token.data), first,
-                last, poolb, out->token_output.data};
-    hk.launch(ATOMENC_KERNEL_POOL, (k_token_mean<Elt>), (unsigned)(B * T), kPoolThreads, 0, st, pa);
-  } else {
-    ReadoutArgs rd{R, C, eps, pl.af3 ? 0 : 1, usable, hid, F(pl.o_rscale), F(pl.o_rbias),
-                   F(pl.o_wread), out->position_update.data};
-    hk.launch(ATOMENC_KERNEL_ROWS, (k_readout<Elt>), row_blocks, 256, 0, st, rd);
-  }
-  hk.mark(6, st);
-  if (hk.err != cudaSuccess) return ATOMENC_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? ATOMENC_OK : ATOMENC_ERR_CUDA;
 }
 
 }  // namespace
