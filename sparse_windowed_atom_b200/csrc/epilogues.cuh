@@ -37,6 +37,41 @@ __device__ __forceinline__ void st4i(__nv_bfloat16 *d, float4 o) {
   *reinterpret_cast<uint2 *>(d) = make_uint2(a, b);
 }
 
+// Plain store of four consecutive columns (one 16-byte / 8-byte store when the row
+// stride and the column keep them aligned).
+template <typename IT>
+struct QuadStore {
+  IT *out;
+  int64_t ld;
+  __device__ void quad(int64_t r, int64_t c0, const float (&v)[4], int64_t N) const {
+    if (c0 + 4 <= N && ((ld | c0) & 3) == 0) {
+      st4i(out + r * ld + c0, make_float4(v[0], v[1], v[2], v[3]));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (c0 + j < N) stf(out, r * ld + c0 + j, v[j]);
+    }
+  }
+};
+
+// ReLU(hidden @ w_pool) before the per-token mean (bullet 19), four columns at a time
+template <typename IT>
+struct QuadRelu {
+  IT *out;
+  int64_t ld;
+  __device__ void quad(int64_t r, int64_t c0, const float (&v)[4], int64_t N) const {
+    const float4 o = make_float4(fmaxf(v[0], 0.f), fmaxf(v[1], 0.f), fmaxf(v[2], 0.f), fmaxf(v[3], 0.f));
+    if (c0 + 4 <= N && ((ld | c0) & 3) == 0) {
+      st4i(out + r * ld + c0, o);
+    } else {
+      const float w[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (c0 + j < N) stf(out, r * ld + c0 + j, w[j]);
+    }
+  }
+};
+
 // AF3 conditioning: columns (scale_0, shift_0, scale_1, shift_1, scale_2, shift_2), C each;
 // scale columns become sigmoid(c_j @ w_scale[j] + b_scale[j])  (bullet 7)
 // Index math is done once per four columns, in 32 bits (C is a multiple of 4).

@@ -44,7 +44,8 @@ __device__ __forceinline__ void load8_t(const TA *A, int64_t lda, int64_t M, int
 template <>
 __device__ __forceinline__ void load8_t<float>(const float *A, int64_t lda, int64_t M, int64_t K,
                                              int64_t r, int64_t k, float (&v)[8]) {
-  if (r < M && k + 8 <= K && ((lda | k) & 3) == 0) {
+  // 16-byte loads only at 16-byte aligned addresses (callers' tensors may start anywhere)
+  if (r < M && k + 8 <= K && (reinterpret_cast<uintptr_t>(A + r * lda + k) & 15) == 0) {
     const float4 x = *reinterpret_cast<const float4 *>(A + r * lda + k);
     const float4 y = *reinterpret_cast<const float4 *>(A + r * lda + k + 4);
     v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
@@ -59,7 +60,7 @@ template <>
 __device__ __forceinline__ void load8_t<__nv_bfloat16>(const __nv_bfloat16 *A, int64_t lda,
                                                      int64_t M, int64_t K, int64_t r, int64_t k,
                                                      float (&v)[8]) {
-  if (r < M && k + 8 <= K && ((lda | k) & 7) == 0) {
+  if (r < M && k + 8 <= K && (reinterpret_cast<uintptr_t>(A + r * lda + k) & 15) == 0) {
     const uint4 x = *reinterpret_cast<const uint4 *>(A + r * lda + k);
     const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll

@@ -124,7 +124,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   // ---- decoder: token @ w_token, gathered per atom in the row pass
   if (!pl.enc)
     c.gemm(static_cast<const Elt *>(in->token.data), V, pl.k_tok, B * T, C, V,
-         Quad<EpiStore>{{F(pl.o_tp), C}});
+         QuadStore<float>{F(pl.o_tp), C});
 
   // ---- usable, sanitised residual start, normalised condition
   RowsArgs ra;
@@ -158,7 +158,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
               EpiGateAF3<Elt>{gateb, F(pl.o_brg), C});
   } else {
     c.gemm_rows(ProdCond<Elt, 1>{cin, usable, nullptr, R, S}, pl.k_cond, R, 6 * C, S,
-              Quad<EpiStoreT<Elt>>{{condb, 6 * C}});
+              QuadStore<Elt>{condb, 6 * C});
   }
   hk.mark(2, st);
   if (!fuse_norm) {
@@ -181,7 +181,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   // ---- boundary, read from the hidden output itself
   const Elt *hid = static_cast<const Elt *>(out->hidden.data);
   if (pl.enc) {
-    c.gemm(hid, C, pl.k_pool, R, U, C, Quad<EpiRelu<Elt>>{{poolb, U}});
+    c.gemm(hid, C, pl.k_pool, R, U, C, QuadRelu<Elt>{poolb, U});
     PoolArgs pa{B, A, T, U, usable, static_cast<const int64_t *>(in->atom_to_token.data), first,
                 last, poolb, out->token_output.data};
     hk.launch(ATOMENC_KERNEL_POOL, (k_token_mean<Elt>), (unsigned)(B * T), kPoolThreads, 0, st, pa);

@@ -116,15 +116,27 @@ __device__ __forceinline__ void row32(const __nv_bfloat16 *p, int64_t ld, int64_
 
 template <typename T>
 __device__ __forceinline__ void store4(T *p, int64_t i, float4 v);
+// (the output is the caller's tensor: vector stores only at aligned addresses)
 template <>
 __device__ __forceinline__ void store4<float>(float *p, int64_t i, float4 v) {
-  *reinterpret_cast<float4 *>(p + i) = v;
+  if ((reinterpret_cast<uintptr_t>(p + i) & 15) == 0) {
+    *reinterpret_cast<float4 *>(p + i) = v;
+  } else {
+    p[i] = v.x; p[i + 1] = v.y; p[i + 2] = v.z; p[i + 3] = v.w;
+  }
 }
 template <>
 __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *p, int64_t i, float4 v) {
-  const uint32_t lo = (uint32_t)umma::bf16_bits(v.x) | ((uint32_t)umma::bf16_bits(v.y) << 16);
-  const uint32_t hi = (uint32_t)umma::bf16_bits(v.z) | ((uint32_t)umma::bf16_bits(v.w) << 16);
-  *reinterpret_cast<uint2 *>(p + i) = make_uint2(lo, hi);
+  const uint16_t b[4] = {umma::bf16_bits(v.x), umma::bf16_bits(v.y), umma::bf16_bits(v.z),
+                         umma::bf16_bits(v.w)};
+  if ((reinterpret_cast<uintptr_t>(p + i) & 7) == 0) {
+    const uint32_t lo = (uint32_t)b[0] | ((uint32_t)b[1] << 16);
+    const uint32_t hi = (uint32_t)b[2] | ((uint32_t)b[3] << 16);
+    *reinterpret_cast<uint2 *>(p + i) = make_uint2(lo, hi);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) reinterpret_cast<uint16_t *>(p)[i + e] = b[e];
+  }
 }
 
 // the CTA pair's flags (global memory, GPU scope); the pair is launched as a 2-CTA
