@@ -72,23 +72,6 @@ __host__ __device__ inline size_t attn_fixed_smem(int QT, int K, int H, int HD, 
   return 4 * (ru4(slots) + (af3 ? ru4((size_t)H * slots) : 0) + ru4((size_t)QT * HD));
 }
 
-// Two floats packed in one 64-bit register, and the sm_100 packed FMA on them.
-typedef unsigned long long f32x2;
-__device__ __forceinline__ f32x2 ffma2(f32x2 a, f32x2 b, f32x2 c) {
-  f32x2 d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ f32x2 pack2(float x, float y) {
-  f32x2 d;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(x), "f"(y));
-  return d;
-}
-__device__ __forceinline__ float2 unpack2(f32x2 v) {
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-  return r;
-}
 
 // 16-byte / 4-byte shared-memory loads by 32-bit shared address
 __device__ __forceinline__ ulonglong2 lds128(uint32_t addr) {

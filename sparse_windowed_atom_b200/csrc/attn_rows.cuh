@@ -34,6 +34,7 @@
 #pragma once
 
 #include <climits>
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -399,52 +400,100 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
   uint8_t *wbuf = wbuf_all + (size_t)warp * H * WB;
   const int hd_lane = (li * LC) / DH;                 // this lane's head
   const bool head_writer = (li % LPH) == 0;
+  T *wrow = reinterpret_cast<T *>(wbuf + hd_lane * WB);
   const uint32_t kbase = (uint32_t)__cvta_generic_to_shared(kstage) + (uint32_t)li * 16u;
   const uint32_t vbase = (uint32_t)__cvta_generic_to_shared(vstage) + (uint32_t)li * 16u;
   const int oc0 = li * LC + OC * g4;                  // first output channel of this lane
+  // the per-warp weight rows are zeroed and written out in 16-byte chunks: lane l takes
+  // chunk l % cpr of rows l / cpr, l / cpr + 32 / cpr, ... (a row has cpr <= 32 chunks)
+  const int cpr = (K * ES + 15) / 16;
+  const int rpp = 32 / cpr, wr_row = lane / cpr, wr_chunk = lane - wr_row * cpr;
   const bool vecw = ((K * ES) & 15) == 0 && g.att_vec;
+  constexpr float kLog2e = 1.4426950408889634f;
 
-  for (int q = warp; q < nq; q += kRowAttnWarps) {
+  // One query: NIT list iterations at most (4 entries each), the K/V rows staged in
+  // shared memory or read from global memory.
+  auto run_query = [&](auto nit_c, auto staged_c, int q) {
+    constexpr int NI = decltype(nit_c)::value;
+    constexpr bool ST = decltype(staged_c)::value;
     const int a = a0 + q;
     const int64_t arow = rbase + a;
     const int n = cnt[q];
     const int niter = (n + 3) >> 2;
-    // the query's channels and the value-gate logits of this lane's output channels
-    float qv[LC], gv[OC];
-    rowattn::ldn<LC>(Qg + arow * HD + li * LC, qv);
+    const int *ck = ckey + q * K;
+    const uint8_t *cs = cks + q * K;
+    // the query's channels of this lane (bf16 pairs, or float32 pairs) and the value-gate
+    // logits of its output channels
+    uint32_t qb[LC / 2];
+    f32x2 qf[LC / 2];
+    if constexpr (ES == 2) {
+#pragma unroll
+      for (int c = 0; c < LC; c += 8) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(Qg + arow * HD + li * LC + c);
+        qb[c / 2] = v.x; qb[c / 2 + 1] = v.y; qb[c / 2 + 2] = v.z; qb[c / 2 + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < LC; c += 4) {
+        const ulonglong2 v = *reinterpret_cast<const ulonglong2 *>(Qg + arow * HD + li * LC + c);
+        qf[c / 2] = v.x;
+        qf[c / 2 + 1] = v.y;
+      }
+    }
+    float gv[OC];
     rowattn::ldn<OC>(Gg + arow * HD + oc0, gv);
     // zero this warp's weight rows
-    for (int c = lane; c < H * WB / 16; c += 32)
-      *reinterpret_cast<uint4 *>(wbuf + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+    if (wr_row < rpp)
+      for (int h = wr_row; h < H; h += rpp)
+        *reinterpret_cast<uint4 *>(wbuf + h * WB + wr_chunk * 16) = make_uint4(0u, 0u, 0u, 0u);
+
+    // the row of list entry e (a readable row with weight 0 past the list's end)
+    auto row_of = [&](int e) -> int { return e < n ? ck[e] : (ST ? klo : 0); };
+    // 16-byte chunk s of the K or V row of key j for this lane
+    auto chunk = [&](uint32_t sbase, const uint8_t *gbase, int j, int s) -> uint4 {
+      if constexpr (ST)
+        return rowattn::lds128(sbase + (uint32_t)((j - klo) * RB + s * 128));
+      else
+        return *reinterpret_cast<const uint4 *>(gbase + (size_t)(rbase + j) * RB + (size_t)(NSEG * li + s) * 16);
+    };
 
     // ---- logits of the listed slots (log2 units)
-    float lt[NIT];
+    float lt[NI];
     float mx = -INFINITY;
 #pragma unroll
-    for (int t = 0; t < NIT; ++t) {
+    for (int t = 0; t < NI; ++t) {
       lt[t] = -INFINITY;
       if (t < niter) {
         const int e = 4 * t + g4;
-        const bool live = e < n;
-        const int j = live ? ckey[q * K + e] : (staged ? klo : 0);
-        float part = 0.f;
+        const int j = row_of(e);
+        float part;
+        if constexpr (ES == 2) {
+          float p0 = 0.f, p1 = 0.f;
 #pragma unroll
-        for (int s = 0; s < NSEG; ++s) {
-          uint4 raw;
-          if (staged)
-            raw = rowattn::lds128(kbase + (uint32_t)((j - klo) * RB + s * 128));
-          else
-            raw = *reinterpret_cast<const uint4 *>(Kg + (size_t)(rbase + j) * RB + (size_t)(NSEG * li + s) * 16);
-          float f[CH];
-          rowattn::unpack(raw, f);
+          for (int s = 0; s < NSEG; ++s) {
+            const uint4 raw = chunk(kbase, Kg, j, s);
+            p0 = fma_bf16x2(qb[4 * s], raw.x, p0);
+            p1 = fma_bf16x2(qb[4 * s + 1], raw.y, p1);
+            p0 = fma_bf16x2(qb[4 * s + 2], raw.z, p0);
+            p1 = fma_bf16x2(qb[4 * s + 3], raw.w, p1);
+          }
+          part = p0 + p1;
+        } else {
+          f32x2 s0 = 0ull, s1 = 0ull;
 #pragma unroll
-          for (int c = 0; c < CH; ++c) part = fmaf(qv[s * CH + c], f[c], part);
+          for (int s = 0; s < NSEG; ++s) {
+            const uint4 raw = chunk(kbase, Kg, j, s);
+            s0 = ffma2(qf[2 * s], ((f32x2)raw.y << 32) | raw.x, s0);
+            s1 = ffma2(qf[2 * s + 1], ((f32x2)raw.w << 32) | raw.z, s1);
+          }
+          const float2 x = unpack2(s0), y = unpack2(s1);
+          part = (x.x + x.y) + (y.x + y.y);
         }
 #pragma unroll
         for (int w = 1; w < LPH; w <<= 1) part += __shfl_xor_sync(0xffffffffu, part, w);
         float l = part * g.scale_log2;
-        if (AF3 && live) l = fmaf(beta[((size_t)q * K + e) * H + hd_lane], 1.4426950408889634f, l);
-        lt[t] = live ? l : -INFINITY;
+        if (AF3 && e < n) l = fmaf(beta[((size_t)q * K + e) * H + hd_lane], kLog2e, l);
+        lt[t] = e < n ? l : -INFINITY;
         mx = fmaxf(mx, lt[t]);
       }
     }
@@ -452,7 +501,7 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
     float sum = 0.f;
 #pragma unroll
-    for (int t = 0; t < NIT; ++t) {
+    for (int t = 0; t < NI; ++t) {
       if (t < niter) {
         lt[t] = lt[t] > -INFINITY ? rowattn::ex2(lt[t] - mx) : 0.f;
         sum += lt[t];
@@ -466,29 +515,45 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
 
     // ---- weights out (per-warp rows), weighted values
     float acc[LC];
+    f32x2 acc2[LC / 2];
 #pragma unroll
     for (int c = 0; c < LC; ++c) acc[c] = 0.f;
 #pragma unroll
-    for (int t = 0; t < NIT; ++t) {
+    for (int c = 0; c < LC / 2; ++c) acc2[c] = 0ull;
+#pragma unroll
+    for (int t = 0; t < NI; ++t) {
       if (t < niter) {
         const int e = 4 * t + g4;
-        const bool live = e < n;
         const float w = lt[t] * inv;
-        if (live && head_writer)
-          rowattn::store_w<T>(reinterpret_cast<T *>(wbuf + hd_lane * WB) + cks[q * K + e], w);
-        const int j = live ? ckey[q * K + e] : (staged ? klo : 0);
+        if (e < n && head_writer) rowattn::store_w<T>(wrow + cs[e], w);
+        const int j = row_of(e);
+        if constexpr (ES == 2) {
+          const uint16_t wb = __bfloat16_as_ushort(__float2bfloat16_rn(w));
 #pragma unroll
-        for (int s = 0; s < NSEG; ++s) {
-          uint4 raw;
-          if (staged)
-            raw = rowattn::lds128(vbase + (uint32_t)((j - klo) * RB + s * 128));
-          else
-            raw = *reinterpret_cast<const uint4 *>(Vg + (size_t)(rbase + j) * RB + (size_t)(NSEG * li + s) * 16);
-          float f[CH];
-          rowattn::unpack(raw, f);
+          for (int s = 0; s < NSEG; ++s) {
+            const uint4 raw = chunk(vbase, Vg, j, s);
+            axpy_bf16x2(wb, raw.x, acc[8 * s], acc[8 * s + 1]);
+            axpy_bf16x2(wb, raw.y, acc[8 * s + 2], acc[8 * s + 3]);
+            axpy_bf16x2(wb, raw.z, acc[8 * s + 4], acc[8 * s + 5]);
+            axpy_bf16x2(wb, raw.w, acc[8 * s + 6], acc[8 * s + 7]);
+          }
+        } else {
+          const f32x2 w2 = pack2(w, w);
 #pragma unroll
-          for (int c = 0; c < CH; ++c) acc[s * CH + c] = fmaf(w, f[c], acc[s * CH + c]);
+          for (int s = 0; s < NSEG; ++s) {
+            const uint4 raw = chunk(vbase, Vg, j, s);
+            acc2[2 * s] = ffma2(w2, ((f32x2)raw.y << 32) | raw.x, acc2[2 * s]);
+            acc2[2 * s + 1] = ffma2(w2, ((f32x2)raw.w << 32) | raw.z, acc2[2 * s + 1]);
+          }
         }
+      }
+    }
+    if constexpr (ES == 4) {
+#pragma unroll
+      for (int c = 0; c < LC / 2; ++c) {
+        const float2 v = unpack2(acc2[c]);
+        acc[2 * c] = v.x;
+        acc[2 * c + 1] = v.y;
       }
     }
     // fold the four quarter-warps: lane (g4, li) ends with channels oc0 .. oc0 + OC
@@ -512,23 +577,32 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
     // ---- the query's weight rows to attention[b, h, a, :]
     __syncwarp();
     if (vecw) {
-      const int cpr = K * ES / 16;
-      for (int c = lane; c < H * cpr; c += 32) {
-        const int h = c / cpr, cc = c - h * cpr;
-        const uint4 v = *reinterpret_cast<const uint4 *>(wbuf + h * WB + cc * 16);
-        *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(Wg + (((int64_t)b * H + h) * A + a) * K) + cc * 16) = v;
-      }
+      if (wr_row < rpp)
+        for (int h = wr_row; h < H; h += rpp) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(wbuf + h * WB + wr_chunk * 16);
+          *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(Wg + (((int64_t)b * H + h) * A + a) * K) + wr_chunk * 16) = v;
+        }
     } else {
-      for (int c = lane; c < H * K; c += 32) {
-        const int h = c / K, k = c - h * K;
-        Wg[(((int64_t)b * H + h) * A + a) * K + k] = reinterpret_cast<const T *>(wbuf + h * WB)[k];
-      }
+      for (int h = 0; h < H; ++h)
+        for (int k = lane; k < K; k += 32)
+          Wg[(((int64_t)b * H + h) * A + a) * K + k] = reinterpret_cast<const T *>(wbuf + h * WB)[k];
     }
     __syncwarp();
-  }
+  };
 
-  // queries of the tile past A: nothing; queries with no permitted slot were written
-  // as zero rows above (their list is empty)
+  using I8 = std::integral_constant<int, 8>;
+  using I16 = std::integral_constant<int, 16>;
+  using I32 = std::integral_constant<int, 32>;
+  for (int q = warp; q < nq; q += kRowAttnWarps) {
+    const int niter = (cnt[q] + 3) >> 2;
+    if (staged) {
+      if (niter <= 8) run_query(I8{}, std::true_type{}, q);
+      else if (niter <= 16) run_query(I16{}, std::true_type{}, q);
+      else run_query(I32{}, std::true_type{}, q);
+    } else {
+      run_query(I32{}, std::false_type{}, q);
+    }
+  }
 }
 
 }  // namespace atomenc

@@ -61,6 +61,42 @@ __device__ __forceinline__ float sigmoid_fast(float z) {
 }
 __device__ __forceinline__ float silu_fast(float z) { return z * sigmoid_fast(z); }
 
+// Two floats packed in one 64-bit register, and the sm_100 packed FMA on them.
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 ffma2(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f32x2 pack2(float x, float y) {
+  f32x2 d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(x), "f"(y));
+  return d;
+}
+__device__ __forceinline__ float2 unpack2(f32x2 v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+
+// c + a.lo * b.lo + a.hi * b.hi for two pairs of bf16 values (each product is exact in
+// float32; two float32-accumulating fused multiply-adds with bf16 sources)
+__device__ __forceinline__ float fma_bf16x2(uint32_t a, uint32_t b, float c) {
+  float d;
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, al, bl, %3;\n\tfma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+      : "=f"(d)
+      : "r"(a), "r"(b), "f"(c));
+  return d;
+}
+// a0 += w * v.lo, a1 += w * v.hi with w and v bf16 (float32 accumulation)
+__device__ __forceinline__ void axpy_bf16x2(uint16_t w, uint32_t v, float &a0, float &a1) {
+  asm("{\n\t.reg .b16 vl, vh;\n\tmov.b32 {vl, vh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, %3, vl, %0;\n\tfma.rn.f32.bf16 %1, %3, vh, %1;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(v), "h"(w));
+}
+
 // ---- warp reductions
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

@@ -124,11 +124,13 @@ struct ProdCond {
   const float *stats;    // [M, 2] (MODE 2)
   int64_t M, K;
   __device__ void load8(int64_t r, int64_t k, float (&v)[8]) const {
-    const bool use = r < M && usable[r] != 0;
+    // the loads do not wait for the usable flag (every row in range is readable memory;
+    // what an unusable row holds is dropped by the select below)
     float cv[8];
-    load8_t(c, K, use ? M : 0, K, r, k, cv);   // rows of unusable atoms are not read
+    load8_t(c, K, M, K, r, k, cv);
     float2 ms = make_float2(0.f, 1.f);
-    if (MODE == 2 && use) ms = *reinterpret_cast<const float2 *>(stats + 2 * r);
+    if (MODE == 2 && r < M) ms = *reinterpret_cast<const float2 *>(stats + 2 * r);
+    const bool use = r < M && usable[r] != 0;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       float y = cv[e];
