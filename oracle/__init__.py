@@ -77,6 +77,12 @@ class _Params(ctypes.Structure):
     _fields_ = [(n, _pd) for n in _PARAM_NAMES] + [("value_gate_per_head", ctypes.c_int32)]
 
 
+class _CoreInputs(ctypes.Structure):
+    _fields_ = [("q", _pd), ("k", _pd), ("v", _pd), ("g", _pd), ("pair", _pd),
+                ("pair_scale", _pd), ("w_pair", _pd), ("key_index", _pi64),
+                ("window_mask", _pu8), ("usable", _pu8)]
+
+
 class _Outputs(ctypes.Structure):
     _fields_ = [("hidden", _pd), ("attention", _pd), ("token_output", _pd),
                 ("position_update", _pd)]
@@ -113,6 +119,12 @@ def _load(threads: str = "one"):
         lib.orc_single_to_pair.restype = ctypes.c_int
         lib.orc_single_to_pair.argtypes = [_i64, _i64, _i64, _i64, _i64, _pd, _pu8] + [_pd] * 8 + [
             ctypes.c_double, ctypes.c_int, _pd, _pd]
+        lib.orc_attention_core.restype = ctypes.c_int
+        lib.orc_attention_core.argtypes = [ctypes.c_int] + [_i64] * 6 + [
+            ctypes.POINTER(_CoreInputs), ctypes.c_double, _i64, _pd, _pd]
+        lib.orc_attention_core_backward.restype = ctypes.c_int
+        lib.orc_attention_core_backward.argtypes = [ctypes.c_int] + [_i64] * 6 + [
+            ctypes.POINTER(_CoreInputs), ctypes.c_double, _i64, _pd, _pd] + [_pd] * 7
         lib.orc_threads.restype = ctypes.c_int
         lib.orc_threads.argtypes = []
         _libs[threads] = lib
@@ -329,3 +341,65 @@ def single_to_pair(activations, parameters, masks, eps=1e-5, output_norm=False):
     if rc != 0:
         raise OracleError(rc, "orc_single_to_pair")
     return pf, out
+
+
+# ---------------------------------------------------------------- attention core
+
+def _core_struct(core, style):
+    keep = {}
+    for n in ("q", "k", "v", "g"):
+        keep[n] = _f64(core[n])
+    for n in ("pair", "pair_scale", "w_pair"):
+        keep[n] = _f64(core[n]) if style == "af3" else None
+    keep["key_index"] = _i64a(core["key_index"])
+    keep["window_mask"] = _u8(core["window_mask"])
+    keep["usable"] = _u8(core["usable"])
+    st = _CoreInputs(q=_ptr(keep["q"], _pd), k=_ptr(keep["k"], _pd), v=_ptr(keep["v"], _pd),
+                     g=_ptr(keep["g"], _pd), pair=_ptr(keep["pair"], _pd),
+                     pair_scale=_ptr(keep["pair_scale"], _pd), w_pair=_ptr(keep["w_pair"], _pd),
+                     key_index=_ptr(keep["key_index"], _pi64),
+                     window_mask=_ptr(keep["window_mask"], _pu8),
+                     usable=_ptr(keep["usable"], _pu8))
+    return st, keep
+
+
+def _core_dims(core, style, H):
+    B, A, HD = np.asarray(core["q"]).shape
+    K = np.asarray(core["key_index"]).shape[-1]
+    P = np.asarray(core["pair"]).shape[-1] if style == "af3" else 0
+    return B, A, K, H, HD // H, P
+
+
+def attention_core(core, H, eps=1e-5, style="af3", radius=-1):
+    """The attention core alone (float64): core = dict of q, k, v, g [B,A,H*D],
+    key_index [B,A,K], window_mask [B,A,K], usable [B,A] and, for AF3, pair [B,A,K,P],
+    pair_scale [P], w_pair [P,H]. Returns (attention [B,H,A,K], out [B,A,H*D])."""
+    st, keep = _core_struct(core, style)
+    B, A, K, H, D, P = _core_dims(core, style, H)
+    att = np.zeros((B, H, A, K))
+    out = np.zeros((B, A, H * D))
+    rc = _load().orc_attention_core(STYLES[style], B, A, K, H, D, P, ctypes.byref(st), float(eps),
+                                    int(radius), _ptr(att, _pd), _ptr(out, _pd))
+    if rc != 0:
+        raise OracleError(f"orc_attention_core failed with code {rc}")
+    return att, out
+
+
+def attention_core_backward(core, H, d_out, d_attention=None, eps=1e-5, style="af3", radius=-1):
+    """Gradient of attention_core: returns a dict d_q, d_k, d_v, d_g [B,A,H*D] and for AF3
+    d_pair [B,A,K,P], d_pair_scale [P], d_w_pair [P,H]."""
+    st, keep = _core_struct(core, style)
+    B, A, K, H, D, P = _core_dims(core, style, H)
+    dO = _f64(d_out)
+    dA = None if d_attention is None else _f64(d_attention)
+    res = {n: np.zeros((B, A, H * D)) for n in ("d_q", "d_k", "d_v", "d_g")}
+    if style == "af3":
+        res.update(d_pair=np.zeros((B, A, K, P)), d_pair_scale=np.zeros(P), d_w_pair=np.zeros((P, H)))
+    rc = _load().orc_attention_core_backward(
+        STYLES[style], B, A, K, H, D, P, ctypes.byref(st), float(eps), int(radius),
+        _ptr(dO, _pd), _ptr(dA, _pd), _ptr(res["d_q"], _pd), _ptr(res["d_k"], _pd),
+        _ptr(res["d_v"], _pd), _ptr(res["d_g"], _pd), _ptr(res.get("d_pair"), _pd),
+        _ptr(res.get("d_pair_scale"), _pd), _ptr(res.get("d_w_pair"), _pd))
+    if rc != 0:
+        raise OracleError(f"orc_attention_core_backward failed with code {rc}")
+    return res

@@ -460,6 +460,213 @@ int orc_forward(int style, int stage, const orc_dims *d, const orc_inputs *in,
   return ORC_OK;
 }
 
+/* ------------------------------------------------------------------ attention core */
+
+/* permitted(a, k) of one batch element  [WAA 4, WAA 5] */
+static int core_permitted(const orc_core_inputs *in, int64_t b, int64_t A, int64_t K,
+                          int64_t a, int64_t k, int64_t radius, int64_t *j_out) {
+  const int64_t s = (b * A + a) * K + k;
+  const int64_t j = in->key_index[s];
+  int ok = j >= 0 && j < A && in->usable[b * A + a] && in->usable[b * A + j] &&
+           in->window_mask[s];
+  if (ok && radius >= 0) ok = (j > a ? j - a : a - j) <= radius;
+  *j_out = j;
+  return ok;
+}
+
+/* the AF3 pair bias of slot row pr for every head: beta[h] = (LN(pr) * pair_scale)
+ * @ w_pair[:, h]; y receives LN(pr)  [WAA 8] */
+static void core_pair_bias(const double *pr, int64_t P, int64_t H, const double *ps,
+                           const double *wp, double eps, double *y, double *beta) {
+  orc_layer_norm(pr, P, eps, y);
+  for (int64_t h = 0; h < H; ++h) {
+    beta[h] = 0.0;
+    for (int64_t p = 0; p < P; ++p) beta[h] += y[p] * ps[p] * wp[p * H + h];
+  }
+}
+
+int orc_attention_core(int style, int64_t B, int64_t A, int64_t K, int64_t H, int64_t D,
+                       int64_t P, const orc_core_inputs *in, double eps, int64_t radius,
+                       double *attention, double *out) {
+  const int af3 = style == ORC_STYLE_AF3;
+  if (B < 1 || A < 1 || K < 1 || H < 1 || D < 1 || (af3 && P < 1)) return ORC_ERR_DIM;
+  if (!(eps > 0.0) || !isfinite(eps)) return ORC_ERR_EPS;
+  if (radius < -1) return ORC_ERR_RADIUS;
+  const int64_t HD = H * D;
+  const double inv_sqrt_d = 1.0 / sqrt((double)D);
+  double *lg = (double *)malloc(sizeof(double) * (size_t)(K * H + K + P + H + 1));
+  uint8_t *pm = (uint8_t *)malloc((size_t)K);
+  if (!lg || !pm) { free(lg); free(pm); return ORC_ERR_NOMEM; }
+  double *bias = lg + K, *y = bias + K * H, *beta = y + P;
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t a = 0; a < A; ++a) {
+      const int64_t ia = b * A + a;
+      for (int64_t k = 0; k < K; ++k) {
+        int64_t j;
+        pm[k] = (uint8_t)core_permitted(in, b, A, K, a, k, radius, &j);
+        for (int64_t h = 0; h < H; ++h) bias[k * H + h] = 0.0;
+        if (af3 && pm[k]) {
+          core_pair_bias(in->pair + (ia * K + k) * P, P, H, in->pair_scale, in->w_pair, eps, y, beta);
+          for (int64_t h = 0; h < H; ++h) bias[k * H + h] = beta[h];
+        }
+      }
+      for (int64_t h = 0; h < H; ++h) {
+        double *arow = attention + ((b * H + h) * A + a) * K;
+        for (int64_t k = 0; k < K; ++k) {
+          lg[k] = 0.0;
+          if (!pm[k]) continue;
+          const int64_t j = in->key_index[ia * K + k];
+          double dot = 0.0;
+          for (int64_t e = 0; e < D; ++e) dot += in->q[ia * HD + h * D + e] * in->k[(b * A + j) * HD + h * D + e];
+          lg[k] = dot * inv_sqrt_d + bias[k * H + h];
+        }
+        orc_masked_softmax(lg, pm, K, arow);
+        for (int64_t e = 0; e < D; ++e) {
+          double o = 0.0;
+          for (int64_t k = 0; k < K; ++k) {
+            if (!pm[k]) continue;
+            const int64_t j = in->key_index[ia * K + k];
+            o += arow[k] * in->v[(b * A + j) * HD + h * D + e];
+          }
+          out[ia * HD + h * D + e] = o * orc_sigmoid(in->g[ia * HD + h * D + e]);
+        }
+      }
+    }
+  free(lg);
+  free(pm);
+  return ORC_OK;
+}
+
+/* Reverse-mode derivative of orc_attention_core, step by step in reverse order of the
+ * forward above (chain rule of the same definitions). */
+int orc_attention_core_backward(int style, int64_t B, int64_t A, int64_t K, int64_t H,
+                                int64_t D, int64_t P, const orc_core_inputs *in, double eps,
+                                int64_t radius, const double *d_out,
+                                const double *d_attention, double *d_q, double *d_k,
+                                double *d_v, double *d_g, double *d_pair,
+                                double *d_pair_scale, double *d_w_pair) {
+  const int af3 = style == ORC_STYLE_AF3;
+  if (B < 1 || A < 1 || K < 1 || H < 1 || D < 1 || (af3 && P < 1)) return ORC_ERR_DIM;
+  if (!(eps > 0.0) || !isfinite(eps)) return ORC_ERR_EPS;
+  if (radius < -1) return ORC_ERR_RADIUS;
+  const int64_t HD = H * D;
+  const double inv_sqrt_d = 1.0 / sqrt((double)D);
+  for (int64_t i = 0; i < B * A * HD; ++i) d_q[i] = d_k[i] = d_v[i] = d_g[i] = 0.0;
+  if (af3) {
+    for (int64_t i = 0; i < B * A * K * P; ++i) d_pair[i] = 0.0;
+    for (int64_t p = 0; p < P; ++p) d_pair_scale[p] = 0.0;
+    for (int64_t i = 0; i < P * H; ++i) d_w_pair[i] = 0.0;
+  }
+  double *buf = (double *)malloc(sizeof(double) * (size_t)(3 * K + K * H + 2 * K * H + 3 * P + H + D + 1));
+  uint8_t *pm = (uint8_t *)malloc((size_t)K);
+  if (!buf || !pm) { free(buf); free(pm); return ORC_ERR_NOMEM; }
+  double *lg = buf, *w = lg + K, *dw = w + K, *bias = dw + K, *dbeta = bias + K * H,
+         *y = dbeta + K * H, *dy = y + P, *dx = dy + P, *beta = dx + P, *o = beta + H;
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t a = 0; a < A; ++a) {
+      const int64_t ia = b * A + a;
+      for (int64_t k = 0; k < K; ++k) {
+        int64_t j;
+        pm[k] = (uint8_t)core_permitted(in, b, A, K, a, k, radius, &j);
+        for (int64_t h = 0; h < H; ++h) {
+          bias[k * H + h] = 0.0;
+          dbeta[k * H + h] = 0.0;
+        }
+        if (af3 && pm[k]) {
+          core_pair_bias(in->pair + (ia * K + k) * P, P, H, in->pair_scale, in->w_pair, eps, y, beta);
+          for (int64_t h = 0; h < H; ++h) bias[k * H + h] = beta[h];
+        }
+      }
+      for (int64_t h = 0; h < H; ++h) {
+        /* forward of this row again: logits, weights, o */
+        for (int64_t k = 0; k < K; ++k) {
+          lg[k] = 0.0;
+          if (!pm[k]) continue;
+          const int64_t j = in->key_index[ia * K + k];
+          double dot = 0.0;
+          for (int64_t e = 0; e < D; ++e) dot += in->q[ia * HD + h * D + e] * in->k[(b * A + j) * HD + h * D + e];
+          lg[k] = dot * inv_sqrt_d + bias[k * H + h];
+        }
+        orc_masked_softmax(lg, pm, K, w);
+        for (int64_t e = 0; e < D; ++e) {
+          o[e] = 0.0;
+          for (int64_t k = 0; k < K; ++k) {
+            if (!pm[k]) continue;
+            o[e] += w[k] * in->v[(b * A + in->key_index[ia * K + k]) * HD + h * D + e];
+          }
+        }
+        /* out = o * sigmoid(g): d_g = d_out * o * s (1 - s), d_o = d_out * s */
+        for (int64_t e = 0; e < D; ++e) {
+          const int64_t c = ia * HD + h * D + e;
+          const double sg = orc_sigmoid(in->g[c]);
+          d_g[c] = d_out[c] * o[e] * sg * (1.0 - sg);
+          o[e] = d_out[c] * sg;   /* o now holds d_o */
+        }
+        /* o = sum_k w_k v_j: d_w_k = d_o . v_j (+ the weights' own gradient),
+         * d_v_j += w_k d_o (each slot separately: repeated keys add up) */
+        double sdw = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+          dw[k] = 0.0;
+          if (!pm[k]) continue;
+          const int64_t j = in->key_index[ia * K + k];
+          for (int64_t e = 0; e < D; ++e) {
+            dw[k] += o[e] * in->v[(b * A + j) * HD + h * D + e];
+            d_v[(b * A + j) * HD + h * D + e] += w[k] * o[e];
+          }
+          if (d_attention) dw[k] += d_attention[((b * H + h) * A + a) * K + k];
+          sdw += w[k] * dw[k];
+        }
+        /* softmax over the permitted slots: d_logit_k = w_k (d_w_k - sum_k' w_k' d_w_k');
+         * logit = q . k_j / sqrt(D) + beta */
+        for (int64_t k = 0; k < K; ++k) {
+          if (!pm[k]) continue;
+          const int64_t j = in->key_index[ia * K + k];
+          const double dl = w[k] * (dw[k] - sdw);
+          for (int64_t e = 0; e < D; ++e) {
+            d_q[ia * HD + h * D + e] += dl * in->k[(b * A + j) * HD + h * D + e] * inv_sqrt_d;
+            d_k[(b * A + j) * HD + h * D + e] += dl * in->q[ia * HD + h * D + e] * inv_sqrt_d;
+          }
+          dbeta[k * H + h] = dl;
+        }
+      }
+      if (!af3) continue;
+      /* beta_h = sum_p y_p pair_scale_p w_pair[p,h], y = LN(pair row) */
+      for (int64_t k = 0; k < K; ++k) {
+        if (!pm[k]) continue;
+        const double *pr = in->pair + (ia * K + k) * P;
+        orc_layer_norm(pr, P, eps, y);
+        for (int64_t p = 0; p < P; ++p) {
+          dy[p] = 0.0;
+          for (int64_t h = 0; h < H; ++h) {
+            const double db = dbeta[k * H + h];
+            d_w_pair[p * H + h] += db * y[p] * in->pair_scale[p];
+            d_pair_scale[p] += db * y[p] * in->w_pair[p * H + h];
+            dy[p] += db * in->pair_scale[p] * in->w_pair[p * H + h];
+          }
+        }
+        /* y = (x - mean) / sqrt(var + eps) (population variance):
+         * d_x = (d_y - mean(d_y) - y mean(d_y y)) / sqrt(var + eps) */
+        double mean = 0.0, var = 0.0, mdy = 0.0, mdyy = 0.0;
+        for (int64_t p = 0; p < P; ++p) mean += pr[p];
+        mean /= (double)P;
+        for (int64_t p = 0; p < P; ++p) var += (pr[p] - mean) * (pr[p] - mean);
+        var /= (double)P;
+        for (int64_t p = 0; p < P; ++p) {
+          mdy += dy[p];
+          mdyy += dy[p] * y[p];
+        }
+        mdy /= (double)P;
+        mdyy /= (double)P;
+        const double rstd = 1.0 / sqrt(var + eps);
+        for (int64_t p = 0; p < P; ++p) dx[p] = (dy[p] - mdy - y[p] * mdyy) * rstd;
+        for (int64_t p = 0; p < P; ++p) d_pair[(ia * K + k) * P + p] = dx[p];
+      }
+    }
+  free(buf);
+  free(pm);
+  return ORC_OK;
+}
+
 /* ------------------------------------------------------------------ single to pair */
 
 /* [S2P] one call: every step in the order the Required behavior lists it. */

@@ -134,6 +134,51 @@ int orc_forward(int style, int stage, const orc_dims *d, const orc_inputs *in,
                 const uint8_t *query_select, orc_outputs *out);
 
 /*
+ * The attention core of the block on its own, given the projections (the gradient
+ * check of the core runs through these two functions).
+ *   [WAA 4, 5]   slot (a, k) of batch element b is permitted iff its key id j is in
+ *                [0, A), usable[a] and usable[j], window_mask, and |j - a| <= radius
+ *                when radius >= 0;
+ *   [WAA 8, 15]  logit = q_a,h . k_j,h / sqrt(D) (+ AF3 pair bias
+ *                (LN(pair[a,k]) * pair_scale) @ w_pair[:, h]); masked stable softmax
+ *                over the permitted slots, a row without any is all zero; repeated
+ *                slots are separate terms;
+ *   [WAA 16]     o_a,h = sum_k w_k v_j,h, then out = o * sigmoid(g) per channel.
+ * q, k, v, g [B,A,H*D] (head-major channels h*D + e; ESMFold2 q and k are the rows
+ * after the per-head RMS and the rotary); pair [B,A,K,P], pair_scale [P], w_pair [P,H]
+ * only for AF3 (style 0). Writes attention [B,H,A,K] and out [B,A,H*D].
+ */
+typedef struct {
+  const double *q, *k, *v, *g;  /* [B,A,H*D] */
+  const double *pair;           /* [B,A,K,P] AF3 */
+  const double *pair_scale;     /* [P] AF3 */
+  const double *w_pair;         /* [P,H] AF3 */
+  const int64_t *key_index;     /* [B,A,K] */
+  const uint8_t *window_mask;   /* [B,A,K] */
+  const uint8_t *usable;        /* [B,A] */
+} orc_core_inputs;
+
+int orc_attention_core(int style, int64_t B, int64_t A, int64_t K, int64_t H, int64_t D,
+                       int64_t P, const orc_core_inputs *in, double eps, int64_t radius,
+                       double *attention, double *out);
+
+/*
+ * Gradient of the attention core: given d_out [B,A,H*D] (and, when not NULL,
+ * d_attention [B,H,A,K], the gradient reaching the attention weights output), writes
+ * d_q, d_k, d_v, d_g [B,A,H*D] and for AF3 d_pair [B,A,K,P], d_pair_scale [P],
+ * d_w_pair [P,H] (all overwritten). A key selected by several slots, of one query or
+ * of many, receives the sum of their contributions ([WAA 5]: repeated selection
+ * accumulates gradients); slots that are not permitted contribute nothing and their
+ * pair rows get zero gradient.
+ */
+int orc_attention_core_backward(int style, int64_t B, int64_t A, int64_t K, int64_t H,
+                                int64_t D, int64_t P, const orc_core_inputs *in, double eps,
+                                int64_t radius, const double *d_out,
+                                const double *d_attention, double *d_q, double *d_k,
+                                double *d_v, double *d_g, double *d_pair,
+                                double *d_pair_scale, double *d_w_pair);
+
+/*
  * Single-to-pair features [S2P 1-6]. x [B,N,C], mask [B,N] (1 = present);
  * norm_scale, norm_bias [C]; weight [C,2H], bias [2H] (columns 0..H-1 give q, H..2H-1
  * give k); out_weight [2H,Dp], out_bias [Dp]; output_scale, output_bias [Dp] (read only
