@@ -579,6 +579,7 @@ def run_atomenc(args):
             "cpu_baseline": cpu, "e2e": e2e,
             "kernel_ms": {k: v for k, v in sorted(by_kind.items())},
             "kernel_launches": kinds,
+            "launch_ms": kernel_ms,
             "gpu_launches": launches,
             "clocks": sampler.summary(),
             "phase_ms": dict(zip(atomenc.PHASES, phase_ms)),

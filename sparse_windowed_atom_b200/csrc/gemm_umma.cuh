@@ -265,28 +265,39 @@ __global__ void __launch_bounds__(kUmmaThreads)
 //              global reads and writes);
 //   warp 8     lane 0 issues the MMAs: two 128-column TMEM accumulators, so the MMAs of
 //              tile t+1 run while the epilogue drains tile t;
-//   warp 9     lane 0 streams the packed weight blocks through a ring of NSLOT shared
-//              buffers with bulk async copies.
+//   warp 9     lane 0 streams the packed weight blocks through a ring of nslot shared
+//              buffers with bulk async copies (nslot is sized on the host to what shared
+//              memory holds, up to every block the CTA needs, so the copies of all of a
+//              CTA's weight blocks can be in flight at once).
 // Requires K <= kRowsKMax; every wait is bounded (status bit 4 on timeout).
 constexpr int kRowsEpiWarps = 8;                        // two per TMEM lane quadrant
 constexpr int kRowsThreads = (kRowsEpiWarps + 2) * 32;  // + MMA issuer + weight loader
 constexpr int kRowsKMax = 256;
+constexpr int kRowsMaxSlots = 24;
+constexpr size_t kRowsSmemBudget = 225 * 1024;
 
-__host__ __device__ constexpr int rows_slots(bool) { return 2; }   // keeps two bf16 CTAs per SM
-__host__ __device__ inline size_t rows_smem_bytes(int64_t K, bool split) {
+// shared bytes of the row-block GEMM with nslot weight slots
+__host__ __device__ inline size_t rows_smem_bytes(int64_t K, bool split, int nslot) {
   const int parts = split ? 2 : 1;
   const size_t nkc = (size_t)((K + kUmmaBK - 1) / kUmmaBK);
-  return 1024 + (nkc + rows_slots(split)) * parts * kUmmaBlockBytes +
-         (size_t)kRowsEpiWarps * 32 * 33 * 4 + 256;
+  return 1024 + (nkc + (size_t)nslot) * parts * kUmmaBlockBytes +
+         (size_t)kRowsEpiWarps * 32 * 33 * 4 + 512;
+}
+// weight slots: every block one CTA consumes (blocks_per_cta) if they fit, else as many
+// as shared memory holds, at least 2
+__host__ __device__ inline int rows_slots(int64_t K, bool split, int blocks_per_cta) {
+  int n = blocks_per_cta < kRowsMaxSlots ? blocks_per_cta : kRowsMaxSlots;
+  while (n > 2 && rows_smem_bytes(K, split, n) > kRowsSmemBudget) --n;
+  return n < 2 ? 2 : n;
 }
 
 template <class Prod, bool SPLIT, class Epi>
 __global__ void __launch_bounds__(kRowsThreads, 1)
     k_gemm_rows(Prod prod, const uint8_t *__restrict__ Wpk, int64_t M, int64_t N, int64_t K,
-                int tiles_per_cta, Epi epi, unsigned *status) {
+                int tiles_per_cta, int NSLOT, Epi epi, unsigned *status) {
   pdl_enter();
   extern __shared__ __align__(1024) uint8_t smem_dyn[];
-  constexpr int PARTS = SPLIT ? 2 : 1, NSLOT = rows_slots(SPLIT);
+  constexpr int PARTS = SPLIT ? 2 : 1;
   constexpr uint32_t BLK = kUmmaBlockBytes;
   constexpr uint32_t idesc = umma::idesc_bf16(kUmmaBM, kUmmaBN);
   uint8_t *sm = reinterpret_cast<uint8_t *>(
@@ -329,15 +340,17 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
 
   if (warp < kRowsEpiWarps) {
     // ---- A: rows 16w..16w+15 of the tile, every k chunk, bf16 (hi[, lo]) swizzled;
-    // the 4 row-segments of a chunk are loaded before any is converted
-    for (int c = 0; c < nkc; ++c) {
-      uint8_t *a_c = sA + (size_t)c * PARTS * BLK;
-      float v[4][8];
+    // the loads of chunk c + 1 are issued before chunk c is converted
+    float vb[2][4][8];
+    auto load_chunk = [&](int c, float (&v)[4][8]) {
 #pragma unroll
       for (int it = 0; it < 4; ++it) {
         const int rl = warp * 16 + it * 4 + (lane >> 3);
         prod.load8(m0 + rl, (int64_t)c * kUmmaBK + (lane & 7) * 8, v[it]);
       }
+    };
+    auto store_chunk = [&](int c, float (&v)[4][8]) {
+      uint8_t *a_c = sA + (size_t)c * PARTS * BLK;
 #pragma unroll
       for (int it = 0; it < 4; ++it) {
         const int r = warp * 16 + it * 4 + (lane >> 3), seg = lane & 7;
@@ -356,6 +369,15 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         *reinterpret_cast<uint4 *>(a_c + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         if (SPLIT)
           *reinterpret_cast<uint4 *>(a_c + BLK + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+    };
+    load_chunk(0, vb[0]);
+    for (int c = 0; c < nkc; c += 2) {
+      if (c + 1 < nkc) load_chunk(c + 1, vb[1]);
+      store_chunk(c, vb[0]);
+      if (c + 1 < nkc) {
+        if (c + 2 < nkc) load_chunk(c + 2, vb[0]);
+        store_chunk(c + 1, vb[1]);
       }
     }
     umma::fence_async_smem();

@@ -159,13 +159,15 @@ struct PassCtx {
     const int64_t sp = want < nt ? want : nt;
     const int per = (int)((nt + sp - 1) / sp);
     dim3 grid((unsigned)((nt + per - 1) / per), (unsigned)mt);
-    const size_t smem = rows_smem_bytes(Kd, split);
+    const int nkc = (int)((Kd + kUmmaBK - 1) / kUmmaBK);
+    const int nslot = rows_slots(Kd, split, per * nkc);
+    const size_t smem = rows_smem_bytes(Kd, split, nslot);
     if (split) {
       smem_limit(k_gemm_rows<P, true, E>, smem);
-      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_rows<P, true, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, epi, status);
+      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_rows<P, true, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, nslot, epi, status);
     } else {
       smem_limit(k_gemm_rows<P, false, E>, smem);
-      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_rows<P, false, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, epi, status);
+      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_rows<P, false, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, nslot, epi, status);
     }
   }
   // out = epi(A @ W): the row-block kernel for K <= 256, else the streaming kernel
