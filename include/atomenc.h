@@ -266,6 +266,59 @@ int atomenc_forward_noalloc(int style, int stage, const atomenc_inputs *in,
  */
 int atomenc_noalloc_get_status(int *device_status, atomenc_stream_t stream);
 
+/* ---------------------------------------------------------------------------------
+ * Gradient of the attention core: the slot-gathered attention of the page "Local atom
+ * attention, encoder pooling and decoder skip/readout", Required behavior (slot
+ * permission and radius, bullets 4-5; logits q . k / sqrt(D) plus, in AF3 style, the
+ * pair bias (LN(pair) * pair_scale) @ w_pair, bullets 8 and 15; masked stable softmax
+ * over the permitted slots with repeated slots as separate entries, bullets 5, 6, 15;
+ * out = (sum_k w_k v_key) * sigmoid(g), bullet 16), taken from its projections q, k,
+ * v and the value-gate logits g. Given d_out (the gradient of out) and optionally
+ * d_attention (the gradient of the attention weights), it writes d_q, d_k, d_v, d_g
+ * and, in AF3 style, d_pair, d_pair_scale and d_w_pair. A key selected by several
+ * slots, of one query or of many, receives the sum of their contributions (the slot
+ * bullet: repeated selection accumulates gradients); the sums are formed in 64-bit
+ * fixed point (2^-32 resolution, |sum| < 2^31), so the results do not depend on the
+ * order of the GPU's work (deterministic).
+ * Shapes: q, k, v, g, d_out, d_q, d_k, d_v, d_g [B,A,H*D] (heads = H given; channel
+ * h*D + e, as the forward's Q/K/V/value-gate rows; ESMFold2 q and k after the per-head
+ * RMS and the rotary); key_index [B,A,K] int64; window_mask [B,A,K] bool; usable [B,A]
+ * bool (valid, mapped to a valid token); d_attention [B,H,A,K] (optional); AF3: pair
+ * [B,A,K,P], pair_scale [P], w_pair [P,H] and d_pair, d_pair_scale, d_w_pair alike.
+ * Float tensors share one type (F32 or BF16; arithmetic float32). Limits: K <= 128,
+ * D <= 64, AF3 P <= 32 and H <= 32 (ATOMENC_ERR_UNSUPPORTED beyond). Errors are decided
+ * on the host before anything is enqueued.
+ */
+typedef struct {
+  atomenc_tensor q, k, v, g;        /* [B,A,H*D] */
+  atomenc_tensor key_index;         /* [B,A,K] int64 */
+  atomenc_tensor window_mask;       /* [B,A,K] bool */
+  atomenc_tensor usable;            /* [B,A] bool */
+  atomenc_tensor pair;              /* [B,A,K,P] AF3 */
+  atomenc_tensor pair_scale;        /* [P] AF3 */
+  atomenc_tensor w_pair;            /* [P,H] AF3 */
+  atomenc_tensor d_out;             /* [B,A,H*D] */
+  atomenc_tensor d_attention;       /* [B,H,A,K], optional (empty: zero) */
+} atomenc_core_bwd_inputs;
+
+typedef struct {
+  atomenc_tensor d_q, d_k, d_v, d_g;              /* [B,A,H*D] */
+  atomenc_tensor d_pair;                          /* [B,A,K,P] AF3 */
+  atomenc_tensor d_pair_scale, d_w_pair;          /* [P], [P,H] AF3 */
+} atomenc_core_bwd_outputs;
+
+/* Workspace bytes (256-byte aligned buffer) for atomenc_attention_backward; 0 if the
+ * arguments do not validate. */
+size_t atomenc_attention_backward_workspace_size(int style, const atomenc_core_bwd_inputs *in,
+                                                 int64_t heads,
+                                                 const atomenc_core_bwd_outputs *out);
+
+/* Enqueue the gradient on `stream` (eps and radius as for atomenc_forward); returns
+ * ATOMENC_OK or an error code. */
+int atomenc_attention_backward(int style, const atomenc_core_bwd_inputs *in, int64_t heads,
+                               double eps, int64_t radius, const atomenc_core_bwd_outputs *out,
+                               void *workspace, size_t workspace_bytes, atomenc_stream_t stream);
+
 /* Static English text for an atomenc_status code. */
 const char *atomenc_strerror(int code);
 

@@ -65,6 +65,19 @@ class AtomencS2POutputs(ctypes.Structure):
     _fields_ = [(n, AtomencTensor) for n in S2P_OUTPUT_FIELDS]
 
 
+CORE_BWD_INPUT_FIELDS = ["q", "k", "v", "g", "key_index", "window_mask", "usable", "pair",
+                         "pair_scale", "w_pair", "d_out", "d_attention"]
+CORE_BWD_OUTPUT_FIELDS = ["d_q", "d_k", "d_v", "d_g", "d_pair", "d_pair_scale", "d_w_pair"]
+
+
+class AtomencCoreBwdInputs(ctypes.Structure):
+    _fields_ = [(n, AtomencTensor) for n in CORE_BWD_INPUT_FIELDS]
+
+
+class AtomencCoreBwdOutputs(ctypes.Structure):
+    _fields_ = [(n, AtomencTensor) for n in CORE_BWD_OUTPUT_FIELDS]
+
+
 class AtomencError(RuntimeError):
     def __init__(self, code: int, what: str):
         super().__init__(f"{what}: atomenc error {code}: {atomenc_strerror(code)}")
@@ -111,6 +124,13 @@ def load_library() -> ctypes.CDLL:
         lib.atomenc_strerror.argtypes = [ctypes.c_int]
         lib.atomenc_version.restype = ctypes.c_int
         lib.atomenc_version.argtypes = []
+        lib.atomenc_attention_backward_workspace_size.restype = ctypes.c_size_t
+        lib.atomenc_attention_backward_workspace_size.argtypes = [
+            ctypes.c_int, P(AtomencCoreBwdInputs), ctypes.c_int64, P(AtomencCoreBwdOutputs)]
+        lib.atomenc_attention_backward.restype = ctypes.c_int
+        lib.atomenc_attention_backward.argtypes = [
+            ctypes.c_int, P(AtomencCoreBwdInputs), ctypes.c_int64, ctypes.c_double, ctypes.c_int64,
+            P(AtomencCoreBwdOutputs), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
         lib.atomenc_s2p_workspace_size.restype = ctypes.c_size_t
         lib.atomenc_s2p_workspace_size.argtypes = [P(AtomencS2PInputs), P(AtomencS2PParams),
                                                    ctypes.c_int, P(AtomencS2POutputs)]
@@ -385,3 +405,37 @@ def single_to_pair(activations: dict, parameters: dict, masks: dict, eps: float 
     if rc != 0:
         raise AtomencError(rc, "atomenc_single_to_pair")
     return outputs["pair_features"], outputs["output"]
+
+
+# ---------------------------------------------------------------- attention core gradient
+
+def attention_backward(core: dict, heads: int, d_out: torch.Tensor, d_attention=None,
+                       eps: float = 1e-5, style: str = "af3", radius: int = -1,
+                       workspace: torch.Tensor | None = None, stream=None) -> dict:
+    """Gradient of the slot-gathered attention core on the GPU. core holds CUDA tensors
+    q, k, v, g [B,A,H*D], key_index [B,A,K] int64, window_mask [B,A,K] bool, usable [B,A]
+    bool and, for AF3, pair [B,A,K,P], pair_scale [P], w_pair [P,H]. Returns d_q, d_k,
+    d_v, d_g (and d_pair, d_pair_scale, d_w_pair for AF3), allocated with torch."""
+    q = core["q"]
+    outs = {n: torch.empty_like(q) for n in ("d_q", "d_k", "d_v", "d_g")}
+    if style == "af3":
+        outs["d_pair"] = torch.empty_like(core["pair"])
+        outs["d_pair_scale"] = torch.empty_like(core["pair_scale"])
+        outs["d_w_pair"] = torch.empty_like(core["w_pair"])
+    src = {**core, "d_out": d_out, "d_attention": d_attention}
+    ins = AtomencCoreBwdInputs(**{n: describe(src.get(n)) for n in CORE_BWD_INPUT_FIELDS})
+    out = AtomencCoreBwdOutputs(**{n: describe(outs.get(n)) for n in CORE_BWD_OUTPUT_FIELDS})
+    lib = load_library()
+    need = lib.atomenc_attention_backward_workspace_size(STYLES[style], ctypes.byref(ins), int(heads),
+                                                         ctypes.byref(out))
+    if need == 0:
+        raise ValueError("atomenc_attention_backward_workspace_size: the arguments do not validate")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    rc = lib.atomenc_attention_backward(STYLES[style], ctypes.byref(ins), int(heads), float(eps),
+                                        int(radius), ctypes.byref(out), workspace.data_ptr(),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream_ptr(stream))
+    if rc != 0:
+        raise AtomencError(rc, "atomenc_attention_backward")
+    return outs
