@@ -125,21 +125,37 @@ def load_peaks():
                 "fallback (6.65 TB/s and 1.4 PFLOP/s sustained, earlier measurements on this pool)")
 
 
-def kernel_source_sha() -> str:
+def attention_kernel(spec) -> str:
+    """The attention kernel the library launches for this shape: the row-gather kernel
+    when H*D = 128, a head spans a whole number of 16-channel lane groups (D a multiple
+    of 16, at most 8 heads), K <= 128 and (AF3) P <= 32; the per-(query, head) kernel
+    otherwise (the same rule as the workspace plan of the C library)."""
+    hd = spec.H * spec.D
+    lc = hd // 8
+    rg = (hd == 128 and spec.D >= lc and spec.D % lc == 0 and hd // spec.D <= 8
+          and spec.K <= 128 and (spec.style != "af3" or spec.P <= 32))
+    return "k_attn_rows" if rg else "k_slot_attention"
+
+
+KERNEL_SOURCES = {"k_attn_rows": ("attn_rows.cuh", "common.cuh"),
+                  "k_slot_attention": ("attention.cuh", "common.cuh")}
+
+
+def kernel_source_sha(kernel: str = "k_attn_rows") -> str:
     h = hashlib.sha256()
-    for name in ("attention.cuh", "common.cuh"):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "sparse_windowed_atom_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(workload: str, kernel: str = "k_attn_rows"):
     """DRAM bytes per attention launch from a committed ncu summary, if it was taken on
-    the current kernel source for this workload; else None."""
-    path = os.path.join(ROOT, "profiles", "traffic_k_slot_attention.txt")
+    the current source of that kernel for this workload; else None."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{kernel}.txt")
     if not os.path.exists(path):
         return None
-    sha = kernel_source_sha()
+    sha = kernel_source_sha(kernel)
     with open(path) as f:
         for line in f:
             if line.startswith("#") or "=" not in line:
@@ -457,15 +473,16 @@ def run_atomenc(args):
     atoms = spec.atoms * world
     value = ranks.job_rate(spec.atoms, ms_per_step)
 
-    # ---- roofline of the slot-attention kernel (its own device time, traced pass)
+    # ---- roofline of the attention kernel (its own device time, traced pass)
     attn_ms = max_over_ranks(by_kind.get("attention", phase_ms[3]))
     hbm_peak, tc_peak, peak_src = load_peaks()
     abytes = attention_bytes(spec)
     achieved = abytes / (attn_ms / 1e3) / 1e9
     dominant = max(range(atomenc.NUM_PHASES), key=lambda p: phase_ms[p])
+    akernel = attention_kernel(spec)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": recorded_traffic(spec.name),
-                "kernel": "k_slot_attention", "bytes_per_launch": abytes,
+                "frac": achieved / hbm_peak, "traffic": recorded_traffic(spec.name, akernel),
+                "kernel": akernel, "bytes_per_launch": abytes,
                 "avg_launch_ms": attn_ms, "peak_source": peak_src,
                 "frac_of_8TBs": achieved / 8000.0}
     # ---- the dense projections on the tensor cores: algorithmic flops over the summed

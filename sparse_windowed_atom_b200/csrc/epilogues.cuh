@@ -92,7 +92,9 @@ struct EpiCondAF3 {
       }
       return;
     }
-    const int blk = c / Ci, ch = c - blk * Ci;
+    // blk = c / C without a division (six blocks)
+    const int blk = (c >= Ci) + (c >= 2 * Ci) + (c >= 3 * Ci) + (c >= 4 * Ci) + (c >= 5 * Ci);
+    const int ch = c - blk * Ci;
     float4 o = make_float4(v[0], v[1], v[2], v[3]);
     if ((blk & 1) == 0) {  // scale block j = blk / 2
       const float *bs = b_scale + (blk >> 1) * Ci + ch;
@@ -146,7 +148,9 @@ struct EpiSplitT {
   const float *bias[4];
   int64_t HD;
   __device__ void quad(int64_t r, int64_t c0, const float (&v)[4], int64_t N) const {
-    const int HDi = (int)HD, c = (int)c0, part = c / HDi, ch = c - part * HDi;
+    // part = c / HD without a division (at most four parts)
+    const int HDi = (int)HD, c = (int)c0;
+    const int part = (c >= HDi) + (c >= 2 * HDi) + (c >= 3 * HDi), ch = c - part * HDi;
     float o[4] = {v[0], v[1], v[2], v[3]};
     const float *b = bias[part];
     if (b) {

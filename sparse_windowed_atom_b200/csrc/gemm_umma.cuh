@@ -273,7 +273,8 @@ __global__ void __launch_bounds__(kUmmaThreads)
 constexpr int kRowsEpiWarps = 8;                        // two per TMEM lane quadrant
 constexpr int kRowsThreads = (kRowsEpiWarps + 2) * 32;  // + MMA issuer + weight loader
 constexpr int kRowsKMax = 256;
-constexpr int kRowsMaxSlots = 24;
+constexpr int kRowsMaxSlots = 4;   // deeper rings were measured slower (every CTA fetches
+                                   // the same weight blocks)
 constexpr size_t kRowsSmemBudget = 225 * 1024;
 
 // shared bytes of the row-block GEMM with nslot weight slots

@@ -59,7 +59,7 @@ struct TransArgs {
                                // then runs out); 0 in normal use
 };
 
-constexpr int kTransSlotsSplit = 3, kTransSlotsPlain = 10;   // weight ring depth (fills shared memory)
+constexpr int kTransSlotsSplit = 3, kTransSlotsPlain = 6;   // weight ring depth
 __host__ __device__ inline size_t trans_smem_bytes(bool split) {
   const size_t parts = split ? 2 : 1, slots = split ? kTransSlotsSplit : kTransSlotsPlain;
   return 1024 + (2 + 2 + slots) * parts * kUmmaBlockBytes + 256;

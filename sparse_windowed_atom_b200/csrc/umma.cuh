@@ -15,7 +15,8 @@
 namespace atomenc {
 namespace umma {
 
-// every wait in this library gives up after this many polls and reports an error
+// every wait in this library gives up after this many polls (about two seconds with the
+// back-off between polls) and reports an error
 constexpr uint32_t kSpinLimit = 1u << 26;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -58,6 +59,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
         : "r"(a), "r"(parity)
         : "memory");
     if (done) return true;
+    // after a few quick polls, back off for a few tens of nanoseconds per poll, so that
+    // waiting warps leave the issue slots to the warps doing the work
+    if (i >= 8) __nanosleep(32);
   }
   return false;
 }

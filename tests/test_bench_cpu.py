@@ -57,11 +57,22 @@ def test_default_workload_is_the_largest():
 
 
 def test_recorded_traffic_is_keyed_by_workload_and_source():
-    v = bench.recorded_traffic("esm_encoder_fp32_a4096")
+    v = bench.recorded_traffic(bench.DEFAULT_WORKLOAD, "k_attn_rows")
     # the committed record is taken on the current kernel source; it may only be absent
     # while a kernel change awaits its capture
     assert v is None or v > 0
     assert bench.recorded_traffic("no_such_workload") is None
+
+
+def test_attention_kernel_choice():
+    # every workload of the benchmark list has H*D = 128 and K <= 128: the row-gather kernel
+    for w in workloads.WORKLOADS.values():
+        assert bench.attention_kernel(w) == "k_attn_rows", w.name
+    import dataclasses
+    w = workloads.WORKLOADS["esm_encoder_fp32_a4096"]
+    assert bench.attention_kernel(dataclasses.replace(w, K=160)) == "k_slot_attention"
+    assert bench.attention_kernel(dataclasses.replace(w, H=2, D=32)) == "k_slot_attention"
+    assert bench.attention_kernel(dataclasses.replace(w, H=16, D=8)) == "k_slot_attention"
 
 
 def test_reference_arm_prints_one_json_line():
