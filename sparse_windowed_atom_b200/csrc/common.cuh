@@ -36,6 +36,14 @@ __device__ __forceinline__ float ldf(const __nv_bfloat16 *p, int64_t i) {
   return __bfloat162float(p[i]);
 }
 __device__ __forceinline__ void stf(float *p, int64_t i, float v) { p[i] = v; }
+// two floats rounded to nearest-even bf16 by one packed conversion; lo in bits 0-15
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  uint32_t u;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(hi), "f"(lo));
+  return u;
+}
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 __device__ __forceinline__ void stf(__nv_bfloat16 *p, int64_t i, float v) {
   p[i] = __float2bfloat16_rn(v);
 }

@@ -30,11 +30,7 @@ using EpiStore = EpiStoreT<float>;
 // four consecutive values in the intermediate type (16-byte float32 / 8-byte bf16)
 __device__ __forceinline__ void st4i(float *d, float4 o) { *reinterpret_cast<float4 *>(d) = o; }
 __device__ __forceinline__ void st4i(__nv_bfloat16 *d, float4 o) {
-  const uint32_t a = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o.x)) |
-                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o.y)) << 16);
-  const uint32_t b = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o.z)) |
-                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o.w)) << 16);
-  *reinterpret_cast<uint2 *>(d) = make_uint2(a, b);
+  *reinterpret_cast<uint2 *>(d) = make_uint2(bf16x2_bits(o.x, o.y), bf16x2_bits(o.z, o.w));
 }
 
 // Plain store of four consecutive columns (one 16-byte / 8-byte store when the row
@@ -132,11 +128,7 @@ __device__ __forceinline__ void st4w(float *d, const float (&o)[4]) {
   *reinterpret_cast<float4 *>(d) = make_float4(o[0], o[1], o[2], o[3]);
 }
 __device__ __forceinline__ void st4w(__nv_bfloat16 *d, const float (&o)[4]) {
-  const uint32_t a = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o[0])) |
-                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o[1])) << 16);
-  const uint32_t b = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o[2])) |
-                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o[3])) << 16);
-  *reinterpret_cast<uint2 *>(d) = make_uint2(a, b);
+  *reinterpret_cast<uint2 *>(d) = make_uint2(bf16x2_bits(o[0], o[1]), bf16x2_bits(o[2], o[3]));
 }
 
 // Q/K/V/value-gate projections: the N columns are `nparts` blocks of HD written to
@@ -152,23 +144,25 @@ struct EpiSplitT {
     const int HDi = (int)HD, c = (int)c0;
     const int part = (c >= HDi) + (c >= 2 * HDi) + (c >= 3 * HDi), ch = c - part * HDi;
     float o[4] = {v[0], v[1], v[2], v[3]};
-    const float *b = bias[part];
-    if (b) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[e] += b[ch + e];
-    }
-    WT *d = dst[part] + r * HD + ch;
+    // selects, not an indexed read: an indexed read of the functor's arrays would copy
+    // the functor to local memory
+    auto bias_of = [&](int p) { return p == 0 ? bias[0] : p == 1 ? bias[1] : p == 2 ? bias[2] : bias[3]; };
+    auto dst_of = [&](int p) { return p == 0 ? dst[0] : p == 1 ? dst[1] : p == 2 ? dst[2] : dst[3]; };
     if ((HDi & 3) == 0) {
-      st4w(d, o);
+      const float *b = bias_of(part);
+      if (b) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[e] += b[ch + e];
+      }
+      st4w(dst_of(part) + r * HD + ch, o);
     } else {  // a quad may straddle two parts when HD is not a multiple of 4
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int ce = c + e;
         if (ce >= N) break;
-        const int pe = ce / HDi, he = ce - pe * HDi;
-        float x = v[e];
-        if (bias[pe]) x += bias[pe][he];
-        stf(dst[pe], r * HD + he, x);
+        const int pe = (ce >= HDi) + (ce >= 2 * HDi) + (ce >= 3 * HDi), he = ce - pe * HDi;
+        const float *b = bias_of(pe);
+        stf(dst_of(pe), r * HD + he, b ? v[e] + b[he] : v[e]);
       }
     }
   }

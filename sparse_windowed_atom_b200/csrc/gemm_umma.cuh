@@ -195,16 +195,7 @@ __global__ void __launch_bounds__(kUmmaThreads)
       float v[8];
       load8_t<TA>(A, lda, M, K, m0 + r, (int64_t)c * kUmmaBK + seg * 8, v);
       uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint16_t h0 = umma::bf16_bits(v[2 * e]), h1 = umma::bf16_bits(v[2 * e + 1]);
-        hi[e] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-        if (SPLIT) {
-          const uint16_t l0 = umma::bf16_bits(v[2 * e] - umma::bf16_val(h0));
-          const uint16_t l1 = umma::bf16_bits(v[2 * e + 1] - umma::bf16_val(h1));
-          lo[e] = (uint32_t)l0 | ((uint32_t)l1 << 16);
-        }
-      }
+      umma::split8<SPLIT>(v, hi, lo);
       const uint32_t off = umma::swz_offset(r, seg * 8, kUmmaBM);
       *reinterpret_cast<uint4 *>(a_s + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
       if (SPLIT)
@@ -271,6 +262,7 @@ __global__ void __launch_bounds__(kUmmaThreads)
 //              CTA's weight blocks can be in flight at once).
 // Requires K <= kRowsKMax; every wait is bounded (status bit 4 on timeout).
 constexpr int kRowsEpiWarps = 8;                        // two per TMEM lane quadrant
+constexpr int kRowsTPitch = 32;                         // floats per row of a transpose tile
 constexpr int kRowsThreads = (kRowsEpiWarps + 2) * 32;  // + MMA issuer + weight loader
 constexpr int kRowsKMax = 256;
 constexpr int kRowsMaxSlots = 4;   // deeper rings were measured slower (every CTA fetches
@@ -282,7 +274,7 @@ __host__ __device__ inline size_t rows_smem_bytes(int64_t K, bool split, int nsl
   const int parts = split ? 2 : 1;
   const size_t nkc = (size_t)((K + kUmmaBK - 1) / kUmmaBK);
   return 1024 + (nkc + (size_t)nslot) * parts * kUmmaBlockBytes +
-         (size_t)kRowsEpiWarps * 32 * 33 * 4 + 512;
+         (size_t)kRowsEpiWarps * 32 * kRowsTPitch * 4 + 512;
 }
 // weight slots: every block one CTA consumes (blocks_per_cta) if they fit, else as many
 // as shared memory holds, at least 2
@@ -306,8 +298,8 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
   const int nkc = (int)((K + kUmmaBK - 1) / kUmmaBK);
   uint8_t *sA = sm;                                       // [nkc][PARTS] blocks
   uint8_t *sR = sA + (size_t)nkc * PARTS * BLK;           // [NSLOT][PARTS] blocks
-  float *sT = reinterpret_cast<float *>(sR + (size_t)NSLOT * PARTS * BLK);   // [warps][32][33]
-  uint64_t *full = reinterpret_cast<uint64_t *>(sT + kRowsEpiWarps * 32 * 33);
+  float *sT = reinterpret_cast<float *>(sR + (size_t)NSLOT * PARTS * BLK);   // [warps][32][pitch]
+  uint64_t *full = reinterpret_cast<uint64_t *>(sT + kRowsEpiWarps * 32 * kRowsTPitch);
   uint64_t *empty = full + NSLOT, *accf = empty + NSLOT, *acce = accf + 2, *aready = acce + 2;
   uint32_t *tslot = reinterpret_cast<uint32_t *>(aready + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
@@ -356,16 +348,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
       for (int it = 0; it < 4; ++it) {
         const int r = warp * 16 + it * 4 + (lane >> 3), seg = lane & 7;
         uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint16_t h0 = umma::bf16_bits(v[it][2 * e]), h1 = umma::bf16_bits(v[it][2 * e + 1]);
-          hi[e] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-          if (SPLIT) {
-            const uint16_t l0 = umma::bf16_bits(v[it][2 * e] - umma::bf16_val(h0));
-            const uint16_t l1 = umma::bf16_bits(v[it][2 * e + 1] - umma::bf16_val(h1));
-            lo[e] = (uint32_t)l0 | ((uint32_t)l1 << 16);
-          }
-        }
+        umma::split8<SPLIT>(v[it], hi, lo);
         const uint32_t off = umma::swz_offset(r, seg * 8, kUmmaBM);
         *reinterpret_cast<uint4 *>(a_c + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         if (SPLIT)
@@ -388,7 +371,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
     // ---- epilogue of each output tile: warp w reads TMEM lane quadrant w % 4 and the
     // column half w / 4 of the tile
     const int qd = warp & 3, cb = (warp >> 2) * (kUmmaBN / 2);
-    float *T = sT + warp * 32 * 33;
+    float *T = sT + warp * 32 * kRowsTPitch;
     const uint32_t tlane = tmem + ((uint32_t)(qd * 32) << 16);
     for (int tl = 0; tl < ntl; ++tl) {
       const int buf = tl & 1;
@@ -400,16 +383,21 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         if (n0 + c0 >= N) break;
         float v[32];
         umma::tmem_ld32(tlane + buf * kUmmaBN + c0, v);
+        // 16-byte shared stores and loads; 16-byte chunk j of row r sits at chunk
+        // j ^ (r & 7), so the eight lanes of a store phase (eight rows, one chunk) and of
+        // a load phase (one row, eight chunks) each cover all 32 banks once
 #pragma unroll
-        for (int j = 0; j < 32; ++j) T[lane * 33 + j] = v[j];
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<float4 *>(T + lane * kRowsTPitch + 4 * (j ^ (lane & 7))) =
+              make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
         __syncwarp();
 #pragma unroll 2
         for (int i = 0; i < 8; ++i) {
           const int rl = i * 4 + (lane >> 3), q = lane & 7;
           const int64_t row = m0 + qd * 32 + rl, col = n0 + c0 + 4 * q;
           if (ok && row < M && col < N) {
-            const float x[4] = {T[rl * 33 + 4 * q], T[rl * 33 + 4 * q + 1], T[rl * 33 + 4 * q + 2],
-                                T[rl * 33 + 4 * q + 3]};
+            const float4 t4 = *reinterpret_cast<const float4 *>(T + rl * kRowsTPitch + 4 * (q ^ (rl & 7)));
+            const float x[4] = {t4.x, t4.y, t4.z, t4.w};
             epi.quad(row, col, x, N);
           }
         }

@@ -105,10 +105,9 @@ __device__ __forceinline__ void st4(__nv_bfloat16 *p, float *v) {
   uint32_t u[2];
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const __nv_bfloat16 a = __float2bfloat16_rn(v[2 * i]), b = __float2bfloat16_rn(v[2 * i + 1]);
-    v[2 * i] = __bfloat162float(a);
-    v[2 * i + 1] = __bfloat162float(b);
-    u[i] = (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
+    u[i] = bf16x2_bits(v[2 * i], v[2 * i + 1]);
+    v[2 * i] = bf16_lo(u[i]);
+    v[2 * i + 1] = bf16_hi(u[i]);
   }
   *reinterpret_cast<uint2 *>(p) = make_uint2(u[0], u[1]);
 }
@@ -292,11 +291,7 @@ __device__ __forceinline__ float4 ld4w(const __nv_bfloat16 *p) {
 }
 __device__ __forceinline__ void st4w(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
 __device__ __forceinline__ void st4w(__nv_bfloat16 *p, float4 v) {
-  const uint32_t a = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.x)) |
-                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.y)) << 16);
-  const uint32_t b = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.z)) |
-                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.w)) << 16);
-  *reinterpret_cast<uint2 *>(p) = make_uint2(a, b);
+  *reinterpret_cast<uint2 *>(p) = make_uint2(bf16x2_bits(v.x, v.y), bf16x2_bits(v.z, v.w));
 }
 
 // Warp per (atom, Q-or-K) for head widths D in {8, 16, 32, 64, 128}: lane l holds four

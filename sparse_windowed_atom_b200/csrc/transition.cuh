@@ -69,16 +69,7 @@ __host__ __device__ inline size_t trans_smem_bytes(bool split) {
 template <bool SPLIT>
 __device__ __forceinline__ void put8(uint8_t *blk, int r, int k, const float (&v)[8]) {
   uint32_t hi[4], lo[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const uint16_t h0 = umma::bf16_bits(v[2 * e]), h1 = umma::bf16_bits(v[2 * e + 1]);
-    hi[e] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-    if (SPLIT) {
-      const uint16_t l0 = umma::bf16_bits(v[2 * e] - umma::bf16_val(h0));
-      const uint16_t l1 = umma::bf16_bits(v[2 * e + 1] - umma::bf16_val(h1));
-      lo[e] = (uint32_t)l0 | ((uint32_t)l1 << 16);
-    }
-  }
+  umma::split8<SPLIT>(v, hi, lo);
   const uint32_t off = umma::swz_offset(r, k, kUmmaBM);
   *reinterpret_cast<uint4 *>(blk + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
   if (SPLIT)
@@ -127,13 +118,11 @@ __device__ __forceinline__ void store4<float>(float *p, int64_t i, float4 v) {
 }
 template <>
 __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *p, int64_t i, float4 v) {
-  const uint16_t b[4] = {umma::bf16_bits(v.x), umma::bf16_bits(v.y), umma::bf16_bits(v.z),
-                         umma::bf16_bits(v.w)};
+  const uint32_t lo = bf16x2_bits(v.x, v.y), hi = bf16x2_bits(v.z, v.w);
   if ((reinterpret_cast<uintptr_t>(p + i) & 7) == 0) {
-    const uint32_t lo = (uint32_t)b[0] | ((uint32_t)b[1] << 16);
-    const uint32_t hi = (uint32_t)b[2] | ((uint32_t)b[3] << 16);
     *reinterpret_cast<uint2 *>(p + i) = make_uint2(lo, hi);
   } else {
+    const uint16_t b[4] = {(uint16_t)lo, (uint16_t)(lo >> 16), (uint16_t)hi, (uint16_t)(hi >> 16)};
 #pragma unroll
     for (int e = 0; e < 4; ++e) reinterpret_cast<uint16_t *>(p)[i + e] = b[e];
   }

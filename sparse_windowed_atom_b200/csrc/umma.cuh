@@ -10,6 +10,8 @@
 // address by 32 bytes.
 #pragma once
 
+#include "common.cuh"
+
 #include <stdint.h>
 
 namespace atomenc {
@@ -200,6 +202,15 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
 }
 __device__ __forceinline__ float bf16_val(uint16_t b) {
   return __uint_as_float((uint32_t)b << 16);
+}
+// hi/lo split of eight floats (lo = the bf16 rounding of what hi leaves)
+template <bool SPLIT>
+__device__ __forceinline__ void split8(const float (&v)[8], uint32_t (&hi)[4], uint32_t (&lo)[4]) {
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    hi[e] = bf16x2_bits(v[2 * e], v[2 * e + 1]);
+    if (SPLIT) lo[e] = bf16x2_bits(v[2 * e] - bf16_lo(hi[e]), v[2 * e + 1] - bf16_hi(hi[e]));
+  }
 }
 
 }  // namespace umma
