@@ -252,7 +252,7 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   {
     const int64_t lc = HD / 8;
     pl.rg = HD == 128 && D >= lc && D % lc == 0 && HD / D <= kRowAttnHeadsMax &&
-            K <= kRowAttnKMax && (!pl.af3 || P <= kRowAttnPairMax);
+            K <= kRowAttnKMax && (!pl.af3 || P <= kRowAttnPairMax) && B * A < INT_MAX;
     pl.ws_bf16 = pl.rg && fdt == ATOMENC_BF16;
   }
   const int64_t wsz = pl.ws_bf16 ? 2 : 4;   // bytes per Q/K/V/G/O element
@@ -323,25 +323,34 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   pl.attn_smem = fixed + (size_t)pl.kv_floats * 4;
 
   if (pl.rg) {
-    // queries per CTA: the largest power of two (<= 64, and small enough that the grid
-    // covers the SMs) whose shared K/V stage holds the expected key span: the tile plus
-    // 2 radius + 1 rows with an index window, the tile plus K otherwise
+    // queries per tile: the largest power of two (<= 64, and small enough that there are
+    // at least as many tiles as SMs) whose shared K/V ring holds the expected key span:
+    // the tile plus 2 radius + 1 rows with an index window, the tile plus K otherwise
     const int es = (int)wsz, rb = (int)(HD * es);
     const int64_t fill = (B * A + pl.sms - 1) / pl.sms;
-    int q = 64;
-    while (q > 1 && q > fill) q /= 2;
-    auto rows_cap = [&](int qq) -> int64_t {
-      const size_t fx = rowattn_fixed_smem(qq, (int)K, (int)H, es, pl.af3);
+    auto rows_cap = [&](int qq, bool qg) -> int64_t {
+      const size_t fx = rowattn_fixed_smem(qq, (int)K, (int)H, es, pl.af3, qg);
       return fx >= kRowAttnSmemBudget ? 0 : (int64_t)((kRowAttnSmemBudget - fx) / (2 * (size_t)rb));
     };
     auto need = [&](int qq) -> int64_t {
       return radius_hint >= 0 ? qq + 2 * radius_hint + 1 : qq + K;
     };
-    while (q > 1 && rows_cap(q) < need(q)) q /= 2;
-    if (rows_cap(q) < 1) return ATOMENC_ERR_UNSUPPORTED;
+    auto pick = [&](bool qg) {
+      int q = 64;
+      while (q > 1 && q > fill) q /= 2;
+      while (q > 1 && rows_cap(q, qg) < need(q)) q /= 2;
+      return q;
+    };
+    // the tile's Q and value-gate rows go to shared memory too unless that would leave
+    // fewer queries per tile than the CTA has warps
+    const int q_qg = pick(true), q_plain = pick(false);
+    const bool qg = q_qg >= std::min(q_plain, kRowAttnWarps);
+    const int q = qg ? q_qg : q_plain;
+    if (rows_cap(q, qg) < 1) return ATOMENC_ERR_UNSUPPORTED;
     pl.rg_qt = q;
-    pl.rg_stage_rows = (int)rows_cap(q);
-    pl.rg_smem = rowattn_fixed_smem(q, (int)K, (int)H, es, pl.af3) + 2 * (size_t)pl.rg_stage_rows * rb;
+    pl.rg_qg = qg;
+    pl.rg_stage_rows = (int)rows_cap(q, qg);
+    pl.rg_smem = rowattn_fixed_smem(q, (int)K, (int)H, es, pl.af3, qg) + 2 * (size_t)pl.rg_stage_rows * rb;
   }
   return ATOMENC_OK;
 }

@@ -10,18 +10,22 @@
 // gate logits and stored head-major (bullet 16).
 //
 // Layout and work split (H*D = HD in {64, 128}, D a multiple of HD / 8, K <= 128):
-//  * One CTA (512 threads, one per SM) owns QT consecutive queries of one batch element.
-//  * Before the wait for the projections (the inputs and the usable flags come from
-//    kernels at least two places earlier): warp w builds, for each of its queries, the
-//    compacted list of permitted slots (key id, slot index) with ballots, and the CTA's
-//    key span [klo, khi]; AF3: the pair bias of every listed slot for every head
-//    (LayerNorm over P in one shifted pass, folded pair_scale * w_pair) into a float32
-//    table in list order.
-//  * After the wait: the K and V rows of the span are staged in shared memory in the
-//    storage type, whole rows (all heads), each 16-byte chunk placed so that the eight
-//    lanes of a quarter-warp read one 128-byte segment of a row per load: lane i of
-//    every quarter-warp owns channels [HD/8 i, HD/8 (i + 1)) of the row (the same head
-//    for HD/8 / D of the lanes), so a gathered row never meets a bank conflict.
+//  * Persistent CTAs (512 threads, one per SM): CTA c walks a contiguous range of query
+//    tiles (QT consecutive queries of one batch element each), in order.
+//  * Per tile, warp w builds, for each of its queries, the compacted list of permitted
+//    slots (key id, slot index) with ballots, and the tile's key span [klo, khi]; AF3:
+//    the pair bias of every listed slot for every head (LayerNorm over P in one shifted
+//    pass, folded pair_scale * w_pair) into a float32 table in list order. The first
+//    tile's lists are built before the wait for the projections (the inputs and the
+//    usable flags come from kernels at least two places earlier).
+//  * The K and V rows live in a shared ring of R rows: key j sits in row j mod R. A tile
+//    copies in only the rows of its span that the previous tile's span did not hold
+//    (consecutive tiles of a batch element share most of their span), together with its
+//    own Q and value-gate rows. Rows are whole (all heads, storage type), each 16-byte
+//    chunk placed so that the eight lanes of a quarter-warp read one 128-byte segment
+//    of a row per load: lane i of every quarter-warp owns channels [HD/8 i, HD/8 (i+1))
+//    of the row (the same head for HD/8 / D of the lanes), so a gathered row never
+//    meets a bank conflict.
 //  * A warp takes one query: quarter-warp g takes list entries g, g + 4, ...; lane i
 //    forms the partial dot product of its channels, the lanes of a head combine theirs
 //    with xor-shuffles; logits stay in registers (log2 units), max and sum across the
@@ -52,8 +56,11 @@ struct RowAttnArgs {
   int radius;                     // -1 = no index window
   float scale_log2;               // log2(e) / sqrt(D)
   float eps;
-  int QT;                         // queries per CTA
-  int stage_rows;                 // rows of K (and of V) the shared stage holds
+  int QT;                         // queries per tile
+  int tiles_per_b;                // ceil(A / QT)
+  int ntiles;                     // B * tiles_per_b
+  int stage_rows;                 // R: rows of K (and of V) the shared ring holds
+  int qg_staged;                  // the tile's Q and value-gate rows are copied to shared memory
   const void *Q, *Kf, *Vf, *G;    // [B*A, HD] storage type
   const int64_t *key_index;       // [B, A, K]
   const uint8_t *window;          // [B, A, K]
@@ -71,13 +78,14 @@ struct RowAttnArgs {
 __host__ __device__ inline int rowattn_wrow_bytes(int K, int es) {
   return ((K * es + 15) & ~15) + 16;
 }
-// shared bytes before the K/V stage: list keys, list slots, counts, (AF3) bias table,
-// per-warp weight rows; each region 128-byte aligned
-__host__ __device__ inline size_t rowattn_fixed_smem(int QT, int K, int H, int es, bool af3) {
+// shared bytes before the K/V ring: list keys, list slots, counts, (AF3) bias table,
+// per-warp weight rows, the tile's Q and value-gate rows; each region 128-byte aligned
+__host__ __device__ inline size_t rowattn_fixed_smem(int QT, int K, int H, int es, bool af3, bool qg) {
   auto r128 = [](size_t n) { return (n + 127) & ~size_t(127); };
   size_t b = r128((size_t)QT * K * 4) + r128((size_t)QT * K) + r128((size_t)QT * 4);
   if (af3) b += r128((size_t)QT * K * H * 4);
   b += r128((size_t)kRowAttnWarps * H * rowattn_wrow_bytes(K, es));
+  if (qg) b += 2 * (size_t)QT * 128 * es;   // the tile's Q and value-gate rows (H*D = 128)
   return b;
 }
 
@@ -279,9 +287,7 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g4 = lane >> 3, li = lane & 7;            // quarter-warp, lane in it
-  const int b = blockIdx.y, a0 = blockIdx.x * g.QT;
-  const int QT = g.QT, K = g.K, A = g.A, P = g.P;
-  const int nq = min(QT, A - a0);
+  const int QT = g.QT, K = g.K, A = g.A, P = g.P, R = g.stage_rows;
 
   auto r128 = [](size_t n) { return (n + 127) & ~size_t(127); };
   uint8_t *cur = smem_dyn;
@@ -291,8 +297,11 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
   float *beta = reinterpret_cast<float *>(cur);       if (AF3) cur += r128((size_t)QT * K * H * 4);
   const int WB = rowattn_wrow_bytes(K, ES);
   uint8_t *wbuf_all = cur;                             cur += r128((size_t)kRowAttnWarps * H * WB);
+  const bool qg_st = g.qg_staged != 0;
+  uint8_t *sQ = cur;                                   if (qg_st) cur += (size_t)QT * RB;
+  uint8_t *sG = cur;                                   if (qg_st) cur += (size_t)QT * RB;
   uint8_t *kstage = cur;
-  uint8_t *vstage = cur + (size_t)g.stage_rows * RB;
+  uint8_t *vstage = cur + (size_t)R * RB;
 
   if (tid == 0) {
     s_lo = INT_MAX;
@@ -308,7 +317,37 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
   }
   __syncthreads();
 
-  // ---------------- list of permitted slots per query (before the wait)
+  // per-thread constants of the query phase
+  const T *Qg = static_cast<const T *>(g.Q);
+  const T *Gg = static_cast<const T *>(g.G);
+  T *Og = static_cast<T *>(g.O);
+  T *Wg = static_cast<T *>(g.attention);
+  const uint8_t *Kg = static_cast<const uint8_t *>(g.Kf);
+  const uint8_t *Vg = static_cast<const uint8_t *>(g.Vf);
+  uint8_t *wbuf = wbuf_all + (size_t)warp * H * WB;
+  const int hd_lane = (li * LC) / DH;                 // this lane's head
+  const bool head_writer = (li % LPH) == 0;
+  T *wrow = reinterpret_cast<T *>(wbuf + hd_lane * WB);
+  const uint32_t kbase = (uint32_t)__cvta_generic_to_shared(kstage) + (uint32_t)li * 16u;
+  const uint32_t vbase = (uint32_t)__cvta_generic_to_shared(vstage) + (uint32_t)li * 16u;
+  const int oc0 = li * LC + OC * g4;                  // first output channel of this lane
+  // the per-warp weight rows are zeroed and written out in 16-byte chunks: lane l takes
+  // chunk l % cpr of rows l / cpr, l / cpr + 32 / cpr, ... (a row has cpr <= 32 chunks)
+  const int cpr = (K * ES + 15) / 16;
+  const int rpp = 32 / cpr, wr_row = lane / cpr, wr_chunk = lane - wr_row * cpr;
+  const bool vecw = ((K * ES) & 15) == 0 && g.att_vec;
+  constexpr float kLog2e = 1.4426950408889634f;
+  constexpr int CPR = RB / 16;                        // 16-byte chunks per row (a power of two)
+
+  // the ring holds the rows [ring_lo, ring_hi] of batch element ring_b (uniform over the CTA)
+  int ring_b = -1, ring_lo = 0, ring_hi = -1;
+  const int t_begin = (int)((int64_t)blockIdx.x * g.ntiles / gridDim.x);
+  const int t_end = (int)((int64_t)(blockIdx.x + 1) * g.ntiles / gridDim.x);
+  for (int tile = t_begin; tile < t_end; ++tile) {
+  const int b = tile / g.tiles_per_b, a0 = (tile - b * g.tiles_per_b) * QT;
+  const int nq = min(QT, A - a0);
+
+  // ---------------- list of permitted slots per query
   const int64_t rbase = (int64_t)b * A;
   int lo = INT_MAX, hi = -1;
   for (int q = warp; q < QT; q += kRowAttnWarps) {
@@ -365,51 +404,69 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
     atomicMax(&s_hi, hi);
   }
 
-  // ---------------- K/V stage (after the wait for the projections)
-  pdl_wait();
+  // ---------------- the ring: rows of the span the ring does not hold yet, and the
+  // tile's Q and value-gate rows (the first tile waits for the projections here)
+  if (tile == t_begin) pdl_wait();
   __syncthreads();
   const int klo = s_lo, khi = s_hi;
   const int span = khi >= klo ? khi - klo + 1 : 0;
-  const bool staged = span > 0 && span <= g.stage_rows;
+  const bool staged = span > 0 && span <= R;
   if (span > 0 && !staged && tid == 0) atomicOr(g.status, 1u);
-  const uint8_t *Kg = static_cast<const uint8_t *>(g.Kf);
-  const uint8_t *Vg = static_cast<const uint8_t *>(g.Vf);
-  if (staged) {
-    // logical 16-byte chunk c of a row goes to position (c % NSEG) * 8 + c / NSEG
-    constexpr int CPR = RB / 16;                        // chunks per row
-    const int total = span * CPR;
+  {
     const uint32_t ks = (uint32_t)__cvta_generic_to_shared(kstage);
     const uint32_t vs = (uint32_t)__cvta_generic_to_shared(vstage);
-    for (int i = tid; i < total; i += kRowAttnThreads) {
-      const int r = i / CPR, c = i - r * CPR;
-      const int p = (c % NSEG) * 8 + c / NSEG;
-      const size_t src = (size_t)(rbase + klo + r) * RB + (size_t)c * 16;
-      const uint32_t dst = (uint32_t)(r * RB + p * 16);
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ks + dst), "l"(Kg + src) : "memory");
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(vs + dst), "l"(Vg + src) : "memory");
+    if (staged) {
+      // key j lives in ring row j mod R = (j - klo + ph) mod R
+      const int ph = klo % R;
+      // rows to copy: [klo, khi] less what the ring holds (one or two intervals)
+      int l0 = klo, l1 = khi, m0 = 1, m1 = 0;
+      if (ring_b == b) {
+        const int i0 = max(klo, ring_lo), i1 = min(khi, ring_hi);
+        if (i0 <= i1) {
+          l1 = i0 - 1;
+          m0 = i1 + 1;
+          m1 = khi;
+        }
+      }
+      const int n1 = max(l1 - l0 + 1, 0), n2 = max(m1 - m0 + 1, 0);
+      const int total = (n1 + n2) * CPR;
+      for (int i = tid; i < total; i += kRowAttnThreads) {
+        const int rr = i / CPR, c = i - rr * CPR;
+        const int j = rr < n1 ? l0 + rr : m0 + (rr - n1);
+        int pr = j - klo + ph;
+        pr -= pr >= R ? R : 0;
+        // logical 16-byte chunk c of a row goes to position (c % NSEG) * 8 + c / NSEG
+        const int p = (c % NSEG) * 8 + c / NSEG;
+        const size_t src = (size_t)(rbase + j) * RB + (size_t)c * 16;
+        const uint32_t dst = (uint32_t)(pr * RB + p * 16);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ks + dst), "l"(Kg + src) : "memory");
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(vs + dst), "l"(Vg + src) : "memory");
+      }
+      ring_b = b;
+      ring_lo = klo;
+      ring_hi = khi;
+      // list entries name ring rows from here on
+      for (int q = warp; q < nq; q += kRowAttnWarps) {
+        const int n = cnt[q];
+        for (int e = lane; e < n; e += 32) {
+          int pr = ckey[q * K + e] - klo + ph;
+          pr -= pr >= R ? R : 0;
+          ckey[q * K + e] = pr;
+        }
+      }
+    }
+    // the tile's Q and value-gate rows (contiguous in global memory), when they fit
+    const uint32_t qs = (uint32_t)__cvta_generic_to_shared(sQ);
+    const uint32_t gs = (uint32_t)__cvta_generic_to_shared(sG);
+    const uint8_t *Qb = reinterpret_cast<const uint8_t *>(Qg) + (size_t)(rbase + a0) * RB;
+    const uint8_t *Gb = reinterpret_cast<const uint8_t *>(Gg) + (size_t)(rbase + a0) * RB;
+    for (int i = tid; qg_st && i < nq * CPR; i += kRowAttnThreads) {
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(qs + 16u * i), "l"(Qb + 16 * (size_t)i) : "memory");
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(gs + 16u * i), "l"(Gb + 16 * (size_t)i) : "memory");
     }
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
   }
   __syncthreads();
-
-  // ---------------- one warp per query
-  const T *Qg = static_cast<const T *>(g.Q);
-  const T *Gg = static_cast<const T *>(g.G);
-  T *Og = static_cast<T *>(g.O);
-  T *Wg = static_cast<T *>(g.attention);
-  uint8_t *wbuf = wbuf_all + (size_t)warp * H * WB;
-  const int hd_lane = (li * LC) / DH;                 // this lane's head
-  const bool head_writer = (li % LPH) == 0;
-  T *wrow = reinterpret_cast<T *>(wbuf + hd_lane * WB);
-  const uint32_t kbase = (uint32_t)__cvta_generic_to_shared(kstage) + (uint32_t)li * 16u;
-  const uint32_t vbase = (uint32_t)__cvta_generic_to_shared(vstage) + (uint32_t)li * 16u;
-  const int oc0 = li * LC + OC * g4;                  // first output channel of this lane
-  // the per-warp weight rows are zeroed and written out in 16-byte chunks: lane l takes
-  // chunk l % cpr of rows l / cpr, l / cpr + 32 / cpr, ... (a row has cpr <= 32 chunks)
-  const int cpr = (K * ES + 15) / 16;
-  const int rpp = 32 / cpr, wr_row = lane / cpr, wr_chunk = lane - wr_row * cpr;
-  const bool vecw = ((K * ES) & 15) == 0 && g.att_vec;
-  constexpr float kLog2e = 1.4426950408889634f;
 
   // One query: NIT list iterations at most (4 entries each), the K/V rows staged in
   // shared memory or read from global memory.
@@ -426,33 +483,36 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
     // logits of its output channels
     uint32_t qb[LC / 2];
     f32x2 qf[LC / 2];
+    const T *qrow = qg_st ? reinterpret_cast<const T *>(sQ + (size_t)q * RB) : Qg + arow * HD;
+    const T *grow = qg_st ? reinterpret_cast<const T *>(sG + (size_t)q * RB) : Gg + arow * HD;
     if constexpr (ES == 2) {
 #pragma unroll
       for (int c = 0; c < LC; c += 8) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(Qg + arow * HD + li * LC + c);
+        const uint4 v = *reinterpret_cast<const uint4 *>(qrow + li * LC + c);
         qb[c / 2] = v.x; qb[c / 2 + 1] = v.y; qb[c / 2 + 2] = v.z; qb[c / 2 + 3] = v.w;
       }
     } else {
 #pragma unroll
       for (int c = 0; c < LC; c += 4) {
-        const ulonglong2 v = *reinterpret_cast<const ulonglong2 *>(Qg + arow * HD + li * LC + c);
+        const ulonglong2 v = *reinterpret_cast<const ulonglong2 *>(qrow + li * LC + c);
         qf[c / 2] = v.x;
         qf[c / 2 + 1] = v.y;
       }
     }
     float gv[OC];
-    rowattn::ldn<OC>(Gg + arow * HD + oc0, gv);
+    rowattn::ldn<OC>(grow + oc0, gv);
     // zero this warp's weight rows
     if (wr_row < rpp)
       for (int h = wr_row; h < H; h += rpp)
         *reinterpret_cast<uint4 *>(wbuf + h * WB + wr_chunk * 16) = make_uint4(0u, 0u, 0u, 0u);
 
-    // the row of list entry e (a readable row with weight 0 past the list's end)
-    auto row_of = [&](int e) -> int { return e < n ? ck[e] : (ST ? klo : 0); };
-    // 16-byte chunk s of the K or V row of key j for this lane
+    // the row of list entry e (a readable row with weight 0 past the list's end): a ring
+    // row when staged, a key id otherwise
+    auto row_of = [&](int e) -> int { return e < n ? ck[e] : ck[0]; };
+    // 16-byte chunk s of the K or V row j for this lane
     auto chunk = [&](uint32_t sbase, const uint8_t *gbase, int j, int s) -> uint4 {
       if constexpr (ST)
-        return rowattn::lds128(sbase + (uint32_t)((j - klo) * RB + s * 128));
+        return rowattn::lds128(sbase + (uint32_t)(j * RB + s * 128));
       else
         return *reinterpret_cast<const uint4 *>(gbase + (size_t)(rbase + j) * RB + (size_t)(NSEG * li + s) * 16);
     };
@@ -603,6 +663,12 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
       run_query(I32{}, std::false_type{}, q);
     }
   }
+  if (tid == 0) {
+    s_lo = INT_MAX;
+    s_hi = -1;
+  }
+  __syncthreads();
+  }  // tiles
 }
 
 }  // namespace atomenc

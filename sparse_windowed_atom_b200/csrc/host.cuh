@@ -54,6 +54,7 @@ struct Plan {
   // value-gate logits and the gated output are then kept in the storage type
   bool rg = false;
   int rg_qt = 0, rg_stage_rows = 0;
+  bool rg_qg = false;               // row-gather attention stages the tile's Q and gate rows
   size_t rg_smem = 0;
   bool ws_bf16 = false;             // Q/K/V/G/O intermediates in bf16
 };

@@ -78,7 +78,10 @@ void launch_middle(PassCtx<Elt> &c) {
     ra2.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
     ra2.eps = eps;
     ra2.QT = pl.rg_qt;
+    ra2.tiles_per_b = (int)((A + pl.rg_qt - 1) / pl.rg_qt);
+    ra2.ntiles = (int)B * ra2.tiles_per_b;
     ra2.stage_rows = pl.rg_stage_rows;
+    ra2.qg_staged = pl.rg_qg ? 1 : 0;
     ra2.Q = wq; ra2.Kf = wk; ra2.Vf = wv; ra2.G = wg;
     ra2.key_index = static_cast<const int64_t *>(in->key_index.data);
     ra2.window = static_cast<const uint8_t *>(in->window_mask.data);
@@ -90,7 +93,8 @@ void launch_middle(PassCtx<Elt> &c) {
     ra2.status = status;
     ra2.pair_vec = pl.af3 && P == 16 && (reinterpret_cast<uintptr_t>(in->pair.data) & 15) == 0;
     ra2.att_vec = (reinterpret_cast<uintptr_t>(out->attention.data) & 15) == 0;
-    dim3 grid((unsigned)((A + pl.rg_qt - 1) / pl.rg_qt), (unsigned)B);
+    // persistent: one CTA per SM, each walking a contiguous range of tiles
+    dim3 grid((unsigned)std::min<int64_t>(ra2.ntiles, pl.sms));
     auto go = [&](auto kern) {
       smem_limit(kern, pl.rg_smem);
       hk.launch(ATOMENC_KERNEL_ATTENTION, kern, grid, kRowAttnThreads, pl.rg_smem, st, ra2);
