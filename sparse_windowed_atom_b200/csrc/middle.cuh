@@ -58,9 +58,12 @@ void launch_middle(PassCtx<Elt> &c) {
       gemm_rows(norm_prod(C, 0, true), pl.k_qkv0, R, 4 * HD, C, e);
     else
       gemm(F(pl.o_feat), C, pl.k_qkv0, R, 4 * HD, C, e);
-    RopeArgs rp{R, H, D, eps, usable, in->rope_cos.data, in->rope_sin.data, wq, wk};
+    const uintptr_t rope_al = 4 * sizeof(Elt) - 1;
+    const int rope_vec = ((reinterpret_cast<uintptr_t>(in->rope_cos.data) |
+                           reinterpret_cast<uintptr_t>(in->rope_sin.data)) & rope_al) == 0;
+    RopeArgs rp{R, H, D, eps, usable, in->rope_cos.data, in->rope_sin.data, wq, wk, rope_vec};
     if (D >= 8 && D <= 128 && (D & (D - 1)) == 0) {
-      const int64_t warps = R * 2;
+      const int64_t warps = R;   // one per atom: its Q and K rows
       hk.launch(ATOMENC_KERNEL_ROWS, (k_qk_rope_warp<Elt, WT>), (unsigned)((warps + 7) / 8), 256, 0, st, rp);
     } else {
       const int64_t n = R * H * 2;

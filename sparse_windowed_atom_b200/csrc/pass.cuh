@@ -184,7 +184,18 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     c.gemm(hid, C, pl.k_pool, R, U, C, QuadRelu<Elt>{poolb, U});
     PoolArgs pa{B, A, T, U, usable, static_cast<const int64_t *>(in->atom_to_token.data), first,
                 last, poolb, out->token_output.data};
-    hk.launch(ATOMENC_KERNEL_POOL, (k_token_mean<Elt>), (unsigned)(B * T), kPoolThreads, 0, st, pa);
+    const int vec_out = (reinterpret_cast<uintptr_t>(out->token_output.data) & (4 * sizeof(Elt) - 1)) == 0;
+    const unsigned tok_blocks = (unsigned)((B * T + 7) / 8);
+    if (U % 4 == 0 && U <= 128)
+      hk.launch(ATOMENC_KERNEL_POOL, (k_token_mean_warp<Elt, 1>), tok_blocks, 256, 0, st, pa, vec_out);
+    else if (U % 4 == 0 && U <= 256)
+      hk.launch(ATOMENC_KERNEL_POOL, (k_token_mean_warp<Elt, 2>), tok_blocks, 256, 0, st, pa, vec_out);
+    else if (U % 4 == 0 && U <= 384)
+      hk.launch(ATOMENC_KERNEL_POOL, (k_token_mean_warp<Elt, 3>), tok_blocks, 256, 0, st, pa, vec_out);
+    else if (U % 4 == 0 && U <= 512)
+      hk.launch(ATOMENC_KERNEL_POOL, (k_token_mean_warp<Elt, 4>), tok_blocks, 256, 0, st, pa, vec_out);
+    else
+      hk.launch(ATOMENC_KERNEL_POOL, (k_token_mean<Elt>), (unsigned)(B * T), kPoolThreads, 0, st, pa);
   } else {
     ReadoutArgs rd{R, C, eps, pl.af3 ? 0 : 1, usable, hid, F(pl.o_rscale), F(pl.o_rbias),
                    F(pl.o_wread), out->position_update.data};

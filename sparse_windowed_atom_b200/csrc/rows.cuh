@@ -123,16 +123,24 @@ __global__ void k_rows_prep_reg(RowsArgs r) {
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const bool live = row < r.B * r.A;
   const int64_t b = live ? row / r.A : 0, a = live ? row % r.A : 0;
-  const bool use = live && atom_usable(r.valid, r.att, r.token_valid, b, a, r.A, r.T);
-  const int64_t t = use ? r.att[row] : 0;
   const int C = (int)r.C, S = (int)r.S;
-  float xv[8], cv[8];
+  // the payload rows are loaded whatever the flags say (they are readable memory) and
+  // replaced by zero with a select below, so their loads overlap the flag loads
+  float4 xl[2], cl[2];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int c = h * 128 + 4 * lane;
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
-    if (use && c < C) x = ld4((const T *)r.atom + row * C + c);
-    if (r.af3 && use && c < S) y = ld4((const T *)r.condition + row * S + c);
+    xl[h] = cl[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (live && c < C) xl[h] = ld4((const T *)r.atom + row * C + c);
+    if (r.af3 && live && c < S) cl[h] = ld4((const T *)r.condition + row * S + c);
+  }
+  const bool use = live && atom_usable(r.valid, r.att, r.token_valid, b, a, r.A, r.T);
+  const int64_t t = use ? r.att[row] : 0;
+  float xv[8], cv[8];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const float4 x = use ? xl[h] : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 y = use ? cl[h] : make_float4(0.f, 0.f, 0.f, 0.f);
     xv[4 * h] = x.x; xv[4 * h + 1] = x.y; xv[4 * h + 2] = x.z; xv[4 * h + 3] = x.w;
     cv[4 * h] = y.x; cv[4 * h + 1] = y.y; cv[4 * h + 2] = y.z; cv[4 * h + 3] = y.w;
   }
@@ -249,6 +257,7 @@ struct RopeArgs {
   const void *cos, *sin;  // [rows, D]
   void *Q, *K;            // [rows, H*D], rewritten in place (float32; k_qk_rope_warp:
                           // its workspace type)
+  int vec;                // k_qk_rope_warp: cos/sin rows are aligned for 4-value loads
 };
 
 // Per-head RMS of Q and K over D, then q * cos + rotate_half(q) * sin with
@@ -294,48 +303,65 @@ __device__ __forceinline__ void st4w(__nv_bfloat16 *p, float4 v) {
   *reinterpret_cast<uint2 *>(p) = make_uint2(bf16x2_bits(v.x, v.y), bf16x2_bits(v.z, v.w));
 }
 
-// Warp per (atom, Q-or-K) for head widths D in {8, 16, 32, 64, 128}: lane l holds four
-// consecutive channels of each 128-channel chunk, the D/4 lanes of one head reduce the
-// sum of squares with xor-shuffles, and the half-split partner of channel d (d +- D/2)
-// sits D/8 lanes away in the same head group. Q and K are of type WT (float32, or bf16
-// when the attention reads bf16 rows); the arithmetic is float32.
+// Warp per atom for head widths D in {8, 16, 32, 64, 128}: lane l holds four consecutive
+// channels of each 128-channel chunk of the Q row and of the K row, the D/4 lanes of one
+// head reduce the sum of squares with xor-shuffles, and the half-split partner of
+// channel d (d +- D/2) sits D/8 lanes away in the same head group. Every load (Q, K,
+// cos, sin, the usable flag) is issued before any of them is used; an unusable atom's
+// rows become zero by a select. Q and K are of type WT (float32, or bf16 when the
+// attention reads bf16 rows); the arithmetic is float32. vec: cos/sin rows may be read
+// four values at a time.
 template <typename T, typename WT>
 __global__ void k_qk_rope_warp(RopeArgs r) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
-  const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (wid >= r.rows * 2) return;
-  const int64_t row = wid >> 1;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= r.rows) return;
   const int D = (int)r.D, HD = (int)(r.H * r.D), glanes = D / 4, half = D / 2;
-  WT *v = static_cast<WT *>((wid & 1) ? r.K : r.Q) + row * HD;
-  const bool use = r.usable[row] != 0;
+  WT *qv = static_cast<WT *>(r.Q) + row * HD;
+  WT *kv = static_cast<WT *>(r.K) + row * HD;
   const T *cs = (const T *)r.cos + row * D;
   const T *sn = (const T *)r.sin + row * D;
   for (int c0 = 0; c0 < HD; c0 += 128) {
     const int c = c0 + lane * 4;
     const bool in = c < HD;
-    float4 x = in ? ld4w(v + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-    float ss = x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
-    for (int o = 1; o < glanes; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float rstd = 1.f / sqrtf(ss / (float)D + r.eps);
-    x.x *= rstd; x.y *= rstd; x.z *= rstd; x.w *= rstd;
-    const int po = D / 8;  // lanes between channel d and d +- D/2
-    float4 p;
-    p.x = __shfl_xor_sync(0xffffffffu, x.x, po);
-    p.y = __shfl_xor_sync(0xffffffffu, x.y, po);
-    p.z = __shfl_xor_sync(0xffffffffu, x.z, po);
-    p.w = __shfl_xor_sync(0xffffffffu, x.w, po);
     const int d = c % D;
-    const float sg = d < half ? -1.f : 1.f;   // rotate_half: [-q2, q1]
+    const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 xq = in ? ld4w(qv + c) : z4, xk = in ? ld4w(kv + c) : z4, co = z4, si = z4;
     if (in) {
-      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (use) {
-        o.x = x.x * ldf(cs, d) + sg * p.x * ldf(sn, d);
-        o.y = x.y * ldf(cs, d + 1) + sg * p.y * ldf(sn, d + 1);
-        o.z = x.z * ldf(cs, d + 2) + sg * p.z * ldf(sn, d + 2);
-        o.w = x.w * ldf(cs, d + 3) + sg * p.w * ldf(sn, d + 3);
+      if (r.vec) {
+        co = ld4(cs + d);
+        si = ld4(sn + d);
+      } else {
+        co = make_float4(ldf(cs, d), ldf(cs, d + 1), ldf(cs, d + 2), ldf(cs, d + 3));
+        si = make_float4(ldf(sn, d), ldf(sn, d + 1), ldf(sn, d + 2), ldf(sn, d + 3));
       }
-      st4w(v + c, o);
+    }
+    const bool use = r.usable[row] != 0;
+    const int po = D / 8;  // lanes between channel d and d +- D/2
+    const float sg = d < half ? -1.f : 1.f;   // rotate_half: [-q2, q1]
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      float4 x = w ? xk : xq;
+      float ss = x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+      for (int o = 1; o < glanes; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float rstd = 1.f / sqrtf(ss / (float)D + r.eps);
+      x.x *= rstd; x.y *= rstd; x.z *= rstd; x.w *= rstd;
+      float4 p;
+      p.x = __shfl_xor_sync(0xffffffffu, x.x, po);
+      p.y = __shfl_xor_sync(0xffffffffu, x.y, po);
+      p.z = __shfl_xor_sync(0xffffffffu, x.z, po);
+      p.w = __shfl_xor_sync(0xffffffffu, x.w, po);
+      if (in) {
+        float4 o = z4;
+        if (use) {
+          o.x = x.x * co.x + sg * p.x * si.x;
+          o.y = x.y * co.y + sg * p.y * si.y;
+          o.z = x.z * co.z + sg * p.z * si.z;
+          o.w = x.w * co.w + sg * p.w * si.w;
+        }
+        st4w((w ? kv : qv) + c, o);
+      }
     }
   }
 }
@@ -438,6 +464,76 @@ __global__ void __launch_bounds__(kPoolThreads) k_token_mean(PoolArgs p) {
     for (int c = 0; c < 3; ++c) {
       const int64_t u = u0 + tid + c * kPoolThreads;
       if (u < U) stf((T *)p.out, bt * U + u, n > 0 ? acc[c] / (float)n : 0.f);
+    }
+  }
+}
+
+// The same mean with one warp per token, for U a multiple of 4 up to 512 (NCH chunks of
+// 128 channels): lane l sums channels 4l..4l+3 of each chunk over the token's range in
+// ascending atom order, four rows' loads in flight; the rows are loaded whatever the
+// flags say (they lie inside the pooled buffer) and the flags (usable and mapped to
+// this token, one per lane for 32 rows, by ballot) select what is added, so the sums
+// are those of k_token_mean. vec_out: token_output rows may be written four values at
+// a time.
+template <typename T, int NCH>
+__global__ void __launch_bounds__(256) k_token_mean_warp(PoolArgs p, int vec_out) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int64_t bt = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (bt >= p.B * p.T) return;
+  const int64_t b = bt / p.T, t = bt % p.T;
+  const int first = p.tok_first[bt], last = p.tok_last[bt];
+  const int U = (int)p.U;
+  const T *base = static_cast<const T *>(p.pooled) + b * p.A * (int64_t)U;
+  float acc[NCH][4];
+#pragma unroll
+  for (int k = 0; k < NCH; ++k) acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.f;
+  int n = 0;
+  for (int a0 = first; a0 <= last; a0 += 32) {
+    const int cnt = min(32, last - a0 + 1);
+    bool f = false;
+    if (lane < cnt) {
+      const int64_t row = b * p.A + a0 + lane;
+      f = p.usable[row] != 0 && p.att[row] == t;
+    }
+    for (int i = 0; i < cnt; i += 4) {
+      float4 x[4][NCH];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+#pragma unroll
+        for (int k = 0; k < NCH; ++k) {
+          const int c = 128 * k + 4 * lane;
+          x[e][k] = (i + e < cnt && c < U) ? ld4(base + (int64_t)(a0 + i + e) * U + c)
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      const unsigned m = __ballot_sync(0xffffffffu, f);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool on = (m >> (i + e)) & 1u;
+#pragma unroll
+        for (int k = 0; k < NCH; ++k) {
+          acc[k][0] += on ? x[e][k].x : 0.f;
+          acc[k][1] += on ? x[e][k].y : 0.f;
+          acc[k][2] += on ? x[e][k].z : 0.f;
+          acc[k][3] += on ? x[e][k].w : 0.f;
+        }
+      }
+    }
+    n += __popc(__ballot_sync(0xffffffffu, f));
+  }
+#pragma unroll
+  for (int k = 0; k < NCH; ++k) {
+    const int c = 128 * k + 4 * lane;
+    if (c >= U) continue;
+    float o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] = n > 0 ? acc[k][e] / (float)n : 0.f;
+    T *dst = static_cast<T *>(p.out) + bt * U + c;
+    if (vec_out) {
+      st4(dst, o);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) stf(dst, e, o[e]);
     }
   }
 }
