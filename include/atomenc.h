@@ -157,6 +157,40 @@ int atomenc_forward(int style, int stage, const atomenc_inputs *in,
                     const atomenc_outputs *out, void *workspace, size_t workspace_bytes,
                     atomenc_stream_t stream);
 
+/*
+ * Prepared weights. A forward pass first converts the caller's weight tensors into the
+ * layouts its kernels read (bf16 tensor-core images of every projection, hi and lo
+ * parts for float32 storage; float32 panels of the small vectors); with weights that
+ * stay fixed across calls that step can be done once:
+ *   atomenc_weight_image_size        bytes of an image for these shapes (0 on a
+ *                                    validation error)
+ *   atomenc_prepare_weights          enqueue the conversion into `image` (device buffer
+ *                                    of at least that many bytes, 256-byte aligned)
+ *   atomenc_prepared_workspace_size  bytes of workspace atomenc_forward_prepared needs
+ *                                    (the weight region lives in the image instead)
+ *   atomenc_forward_prepared         atomenc_forward reading the weights from `image`;
+ *                                    params still describe the weights (shapes are
+ *                                    validated) but their data is not read.
+ * The arguments are those of atomenc_forward; the image depends on style, stage, the
+ * storage type and the weight shapes only, and starts with a key naming them: a pass
+ * given an image built for anything else sets status bit 8 (outputs invalid) instead
+ * of reading it. Results are bit-identical to atomenc_forward. Returns enum
+ * atomenc_status; ATOMENC_ERR_WORKSPACE for a missing, short or unaligned image or
+ * workspace.
+ */
+size_t atomenc_weight_image_size(int style, int stage, const atomenc_inputs *in,
+                                 const atomenc_params *params, const atomenc_outputs *out);
+size_t atomenc_prepared_workspace_size(int style, int stage, const atomenc_inputs *in,
+                                       const atomenc_params *params, const atomenc_outputs *out);
+int atomenc_prepare_weights(int style, int stage, const atomenc_inputs *in,
+                            const atomenc_params *params, const atomenc_outputs *out,
+                            void *image, size_t image_bytes, atomenc_stream_t stream);
+int atomenc_forward_prepared(int style, int stage, const atomenc_inputs *in,
+                             const atomenc_params *params, const void *image,
+                             size_t image_bytes, double eps, int64_t radius,
+                             const atomenc_outputs *out, void *workspace, size_t workspace_bytes,
+                             atomenc_stream_t stream);
+
 /* Phases of one forward pass, in launch order (for atomenc_forward_profiled). */
 enum atomenc_phase {
   ATOMENC_PHASE_INPUTS = 0,        /* weight panels, usability, sanitisation, residual start */
@@ -216,6 +250,8 @@ int atomenc_forward_traced(int style, int stage, const atomenc_inputs *in,
  *       partner CTA of the paired transition) reached its poll limit and gave up. AN
  *       ERROR: the kernel returned without finishing, and hidden, attention and the
  *       pooled / readout outputs of this pass are invalid.
+ *   8 = (atomenc_forward_prepared) the weight image was built for another style, stage,
+ *       storage type or weight shapes. AN ERROR: the outputs of this pass are invalid.
  * Returns enum atomenc_status (of the read, not of the pass).
  */
 int atomenc_get_status(const void *workspace, int *device_status, atomenc_stream_t stream);

@@ -104,6 +104,18 @@ def load_library() -> ctypes.CDLL:
                                         P(AtomencParams), ctypes.c_double, ctypes.c_int64,
                                         P(AtomencOutputs), ctypes.c_void_p, ctypes.c_size_t,
                                         ctypes.c_void_p]
+        for fn in ("atomenc_weight_image_size", "atomenc_prepared_workspace_size"):
+            getattr(lib, fn).restype = ctypes.c_size_t
+            getattr(lib, fn).argtypes = lib.atomenc_workspace_size.argtypes
+        lib.atomenc_prepare_weights.restype = ctypes.c_int
+        lib.atomenc_prepare_weights.argtypes = [ctypes.c_int, ctypes.c_int, P(AtomencInputs),
+                                                P(AtomencParams), P(AtomencOutputs),
+                                                ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+        lib.atomenc_forward_prepared.restype = ctypes.c_int
+        lib.atomenc_forward_prepared.argtypes = [ctypes.c_int, ctypes.c_int, P(AtomencInputs),
+                                                 P(AtomencParams), ctypes.c_void_p, ctypes.c_size_t,
+                                                 ctypes.c_double, ctypes.c_int64, P(AtomencOutputs),
+                                                 ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
         lib.atomenc_forward_profiled.restype = ctypes.c_int
         lib.atomenc_forward_profiled.argtypes = lib.atomenc_forward.argtypes + [
             P(ctypes.c_void_p), ctypes.c_int, P(ctypes.c_int)]
@@ -202,19 +214,76 @@ def atomenc_forward(style: str, stage: str, inputs: dict, params: dict, eps: flo
         raise AtomencError(rc, "atomenc_forward")
 
 
+def _size(fn: str, style, stage, inputs, params, outputs) -> int:
+    ins, prm, outs = _structs(inputs, params, outputs)
+    n = getattr(load_library(), fn)(STYLES[style], STAGES[stage], ctypes.byref(ins),
+                                    ctypes.byref(prm), ctypes.byref(outs))
+    if n == 0:
+        raise ValueError(f"{fn}: the arguments do not validate")
+    return int(n)
+
+
+def atomenc_weight_image_size(style: str, stage: str, inputs: dict, params: dict, outputs: dict) -> int:
+    return _size("atomenc_weight_image_size", style, stage, inputs, params, outputs)
+
+
+def atomenc_prepared_workspace_size(style: str, stage: str, inputs: dict, params: dict,
+                                    outputs: dict) -> int:
+    return _size("atomenc_prepared_workspace_size", style, stage, inputs, params, outputs)
+
+
+def atomenc_prepare_weights(style: str, stage: str, inputs: dict, params: dict, outputs: dict,
+                            image: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Build the weight image for these weights (allocated with torch unless given)."""
+    need = atomenc_weight_image_size(style, stage, inputs, params, outputs)
+    if image is None:
+        image = torch.empty(need, dtype=torch.uint8, device=inputs["atom"].device)
+    ins, prm, outs = _structs(inputs, params, outputs)
+    rc = load_library().atomenc_prepare_weights(STYLES[style], STAGES[stage], ctypes.byref(ins),
+                                                ctypes.byref(prm), ctypes.byref(outs),
+                                                image.data_ptr(), image.numel() * image.element_size(),
+                                                _stream_ptr(stream))
+    if rc != 0:
+        raise AtomencError(rc, "atomenc_prepare_weights")
+    return image
+
+
+def atomenc_forward_prepared(style: str, stage: str, inputs: dict, params: dict,
+                             image: torch.Tensor, eps: float, radius: int, outputs: dict,
+                             workspace: torch.Tensor, stream=None) -> None:
+    ins, prm, outs = _structs(inputs, params, outputs)
+    rc = load_library().atomenc_forward_prepared(
+        STYLES[style], STAGES[stage], ctypes.byref(ins), ctypes.byref(prm), image.data_ptr(),
+        image.numel() * image.element_size(), float(eps), int(radius), ctypes.byref(outs),
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if rc != 0:
+        raise AtomencError(rc, "atomenc_forward_prepared")
+
+
 class Forward:
     """atomenc_forward prepared once for a fixed set of tensors: the descriptors are
     built at construction, so each call is a single C call (no per-call marshalling).
-    The tensors must stay alive, in place and unchanged in shape while it is used."""
+    The tensors must stay alive, in place and unchanged in shape while it is used.
+    With `image` (from atomenc_prepare_weights) each call is atomenc_forward_prepared:
+    the weight conversion is not repeated."""
 
     def __init__(self, style: str, stage: str, inputs: dict, params: dict, eps: float,
-                 radius: int, outputs: dict, workspace: torch.Tensor, stream=None):
+                 radius: int, outputs: dict, workspace: torch.Tensor, stream=None,
+                 image: torch.Tensor | None = None):
         self._ins, self._prm, self._outs = _structs(inputs, params, outputs)
-        self._keep = (inputs, params, outputs, workspace)
-        self._fn = load_library().atomenc_forward
-        self._args = (STYLES[style], STAGES[stage], ctypes.byref(self._ins),
-                      ctypes.byref(self._prm), float(eps), int(radius), ctypes.byref(self._outs),
-                      workspace.data_ptr(), workspace.numel() * workspace.element_size())
+        self._keep = (inputs, params, outputs, workspace, image)
+        if image is None:
+            self._fn = load_library().atomenc_forward
+            self._args = (STYLES[style], STAGES[stage], ctypes.byref(self._ins),
+                          ctypes.byref(self._prm), float(eps), int(radius), ctypes.byref(self._outs),
+                          workspace.data_ptr(), workspace.numel() * workspace.element_size())
+        else:
+            self._fn = load_library().atomenc_forward_prepared
+            self._args = (STYLES[style], STAGES[stage], ctypes.byref(self._ins),
+                          ctypes.byref(self._prm), image.data_ptr(),
+                          image.numel() * image.element_size(), float(eps), int(radius),
+                          ctypes.byref(self._outs), workspace.data_ptr(),
+                          workspace.numel() * workspace.element_size())
         self._stream = None if stream is None else _stream_ptr(stream)
 
     def __call__(self, stream=None) -> None:
@@ -294,6 +363,7 @@ def atomenc_forward_traced(style: str, stage: str, inputs: dict, params: dict, e
 
 STATUS_L2_FALLBACK = 1     # keys gathered from L2 (same results)
 STATUS_WAIT_TIMEOUT = 4    # a bounded wait gave up: the pass's outputs are invalid
+STATUS_IMAGE_MISMATCH = 8  # a prepared weight image built for other shapes: outputs invalid
 
 
 class AtomencStatusError(RuntimeError):

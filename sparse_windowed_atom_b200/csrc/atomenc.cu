@@ -275,6 +275,7 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   pl.o_z = take(cur, pl.fuse_tail ? 0 : R * C * 4);
   pl.o_h = take(cur, pl.fuse_tail ? 0 : R * M * 4);
   pl.o_pool = take(cur, pl.enc ? R * U * its : 0);
+  pl.o_wbase = cur;   // from here on: the weight region (panels and images)
   pl.o_wread = take(cur, pl.enc ? 0 : C * 3 * 4);
   pl.o_bscale = take(cur, pl.af3 ? 3 * C * 4 : 0);
   pl.o_brg = take(cur, pl.af3 ? 2 * C * 4 : 0);
@@ -366,10 +367,10 @@ size_t atomenc_workspace_size(int style, int stage, const atomenc_inputs *in,
   return pl.bytes;
 }
 
-static int forward_impl(int style, int stage, const atomenc_inputs *in,
-                        const atomenc_params *params, double eps, int64_t radius,
-                        const atomenc_outputs *out, void *workspace, size_t workspace_bytes,
-                        atomenc_stream_t stream, Hooks &hk) {
+static int run_impl(int mode, int style, int stage, const atomenc_inputs *in,
+                    const atomenc_params *params, double eps, int64_t radius,
+                    const atomenc_outputs *out, void *workspace, size_t workspace_bytes,
+                    void *image, size_t image_bytes, atomenc_stream_t stream, Hooks &hk) {
   Plan pl;
   CHECK(validate(style, stage, in, params, out, pl, radius));
   if (!std::isfinite(eps) || !(eps > 0.0)) return ATOMENC_ERR_EPS;
@@ -377,13 +378,63 @@ static int forward_impl(int style, int stage, const atomenc_inputs *in,
   if (!(feps > 0.f) || !std::isfinite(feps)) return ATOMENC_ERR_EPS;
   if (pl.fdt == ATOMENC_BF16 && !(bf16_round_host(feps) > 0.f)) return ATOMENC_ERR_EPS;
   if (radius < -1) return ATOMENC_ERR_RADIUS;
-  if (!workspace || workspace_bytes < pl.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255))
-    return ATOMENC_ERR_WORKSPACE;
+  if (mode != kPassPrepare) {
+    const size_t need = mode == kPassFull ? pl.bytes : pl.o_wbase;
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+      return ATOMENC_ERR_WORKSPACE;
+  }
+  if (mode != kPassFull) {
+    if (!image || image_bytes < kImageHeader + (pl.bytes - pl.o_wbase) ||
+        (reinterpret_cast<uintptr_t>(image) & 255))
+      return ATOMENC_ERR_WORKSPACE;
+  }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  unsigned char *ws = static_cast<unsigned char *>(workspace);
+  unsigned char *ws = static_cast<unsigned char *>(mode == kPassPrepare ? image : workspace);
+  unsigned char *img = static_cast<unsigned char *>(image);
   hk.begin(st);
-  if (pl.fdt == ATOMENC_F32) return launch_all<float>(pl, in, params, feps, radius, out, ws, st, hk);
-  return launch_all<__nv_bfloat16>(pl, in, params, feps, radius, out, ws, st, hk);
+  if (pl.fdt == ATOMENC_F32)
+    return launch_all<float>(pl, in, params, feps, radius, out, ws, st, hk, mode, img);
+  return launch_all<__nv_bfloat16>(pl, in, params, feps, radius, out, ws, st, hk, mode, img);
+}
+
+static int forward_impl(int style, int stage, const atomenc_inputs *in,
+                        const atomenc_params *params, double eps, int64_t radius,
+                        const atomenc_outputs *out, void *workspace, size_t workspace_bytes,
+                        atomenc_stream_t stream, Hooks &hk) {
+  return run_impl(kPassFull, style, stage, in, params, eps, radius, out, workspace,
+                  workspace_bytes, nullptr, 0, stream, hk);
+}
+
+size_t atomenc_weight_image_size(int style, int stage, const atomenc_inputs *in,
+                                 const atomenc_params *params, const atomenc_outputs *out) {
+  Plan pl;
+  if (validate(style, stage, in, params, out, pl, -1) != ATOMENC_OK) return 0;
+  return kImageHeader + (pl.bytes - pl.o_wbase);
+}
+
+size_t atomenc_prepared_workspace_size(int style, int stage, const atomenc_inputs *in,
+                                       const atomenc_params *params, const atomenc_outputs *out) {
+  Plan pl;
+  if (validate(style, stage, in, params, out, pl, -1) != ATOMENC_OK) return 0;
+  return pl.o_wbase;
+}
+
+int atomenc_prepare_weights(int style, int stage, const atomenc_inputs *in,
+                            const atomenc_params *params, const atomenc_outputs *out,
+                            void *image, size_t image_bytes, atomenc_stream_t stream) {
+  Hooks hk;
+  return run_impl(kPassPrepare, style, stage, in, params, 1.0, -1, out, nullptr, 0, image,
+                  image_bytes, stream, hk);
+}
+
+int atomenc_forward_prepared(int style, int stage, const atomenc_inputs *in,
+                             const atomenc_params *params, const void *image,
+                             size_t image_bytes, double eps, int64_t radius,
+                             const atomenc_outputs *out, void *workspace, size_t workspace_bytes,
+                             atomenc_stream_t stream) {
+  Hooks hk;
+  return run_impl(kPassPrepared, style, stage, in, params, eps, radius, out, workspace,
+                  workspace_bytes, const_cast<void *>(image), image_bytes, stream, hk);
 }
 
 int atomenc_forward(int style, int stage, const atomenc_inputs *in, const atomenc_params *params,

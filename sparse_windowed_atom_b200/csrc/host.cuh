@@ -8,6 +8,7 @@
 #include <climits>
 #include <cmath>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <type_traits>
@@ -35,6 +36,11 @@ struct Dims {
   int64_t B = 0, A = 0, T = 0, K = 0, C = 0, S = 0, H = 0, D = 0, P = 0, M = 0, U = 0, V = 0;
 };
 
+constexpr size_t kImageHeader = 256;
+// Modes of a pass: build the weight images in the workspace and run (the plain forward);
+// build them into a prepared image only; run from a prepared image.
+enum PassMode { kPassFull = 0, kPassPrepare = 1, kPassPrepared = 2 };
+
 struct Plan {
   int style = 0, stage = 0, fdt = 0;
   bool af3 = false, enc = false, fuse_tail = false, tail_pair = false;
@@ -43,6 +49,9 @@ struct Plan {
   size_t o_status, o_usable, o_xstats, o_cstats, o_first, o_last, o_tp, o_x, o_cond, o_gate, o_feat,
       o_q, o_k, o_v, o_g, o_o, o_xp, o_z, o_h, o_pool, o_xfer, o_xflag;
   size_t o_wread, o_bscale, o_brg, o_bq, o_wpair, o_rscale, o_rbias;
+  // the weight region [o_wbase, bytes): panels and images built from the weights; a
+  // prepared image holds it after a header of kImageHeader bytes
+  size_t o_wbase = 0;
   // tensor-core images of the weight panels (bf16, hi[/lo])
   size_t k_cond, k_gate, k_qkv0, k_qkv1, k_out, k_ff1, k_ff2, k_pool, k_tok;
   size_t bytes = 0;
@@ -58,6 +67,22 @@ struct Plan {
   size_t rg_smem = 0;
   bool ws_bf16 = false;             // Q/K/V/G/O intermediates in bf16
 };
+
+// The key a prepared image carries: style, stage, storage type, the dimensions the images
+// depend on (an FNV-1a hash of C, S, H, D, P, M, U, V) and the weight region's size.
+inline void image_key(const Plan &pl, int (&key)[kImageKeyWords]) {
+  const Dims &d = pl.d;
+  key[0] = 0x61656e63;
+  key[1] = pl.style | (pl.stage << 4) | (pl.fdt << 8);
+  uint32_t h = 2166136261u;
+  const int64_t dims[8] = {d.C, d.S, d.H, d.D, d.P, d.M, d.U, d.V};
+  for (int64_t v : dims) {
+    h = (h ^ (uint32_t)v) * 16777619u;
+    h = (h ^ (uint32_t)(v >> 32)) * 16777619u;
+  }
+  key[2] = (int)h;
+  key[3] = (int)(pl.bytes - pl.o_wbase);
+}
 
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device), and again only
 // if a larger size is asked for: the attribute outlives the call, so repeating it on
@@ -149,7 +174,9 @@ struct PassCtx {
   bool fuse_norm;       // the row norm of x is formed inside the projection operand
   unsigned row_blocks;  // 256-thread blocks of the warp-per-row kernels
   Elt *xb, *condb, *gateb, *poolb;   // intermediates in the storage type
+  unsigned char *wb;    // base of the weight-region offsets (the workspace, or a prepared image)
   float *F(size_t off) const { return reinterpret_cast<float *>(ws + off); }
+  float *WF(size_t off) const { return reinterpret_cast<float *>(wb + off); }
 
   // out = epi(A' @ W) on the tensor cores, W given by its packed image and A' produced by
   // `prod` (A itself, or a row normalisation fused into the operand); K <= 256
@@ -165,10 +192,10 @@ struct PassCtx {
     const size_t smem = rows_smem_bytes(Kd, split, nslot);
     if (split) {
       smem_limit(k_gemm_rows<P, true, E>, smem);
-      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_rows<P, true, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, nslot, epi, status);
+      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_rows<P, true, E>), grid, kRowsThreads, smem, st, prod, wb + wpk, Mr, N, Kd, per, nslot, epi, status);
     } else {
       smem_limit(k_gemm_rows<P, false, E>, smem);
-      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_rows<P, false, E>), grid, kRowsThreads, smem, st, prod, ws + wpk, Mr, N, Kd, per, nslot, epi, status);
+      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_rows<P, false, E>), grid, kRowsThreads, smem, st, prod, wb + wpk, Mr, N, Kd, per, nslot, epi, status);
     }
   }
   // out = epi(A @ W): the row-block kernel for K <= 256, else the streaming kernel
@@ -182,10 +209,10 @@ struct PassCtx {
     const size_t smem = umma_smem_bytes(split);
     if (split) {
       smem_limit(k_gemm_umma<TA, true, E>, smem);
-      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_umma<TA, true, E>), grid, kUmmaThreads, smem, st, A_, lda, ws + wpk, Mr, N, Kd, epi, status);
+      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_umma<TA, true, E>), grid, kUmmaThreads, smem, st, A_, lda, wb + wpk, Mr, N, Kd, epi, status);
     } else {
       smem_limit(k_gemm_umma<TA, false, E>, smem);
-      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_umma<TA, false, E>), grid, kUmmaThreads, smem, st, A_, lda, ws + wpk, Mr, N, Kd, epi, status);
+      hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_umma<TA, false, E>), grid, kUmmaThreads, smem, st, A_, lda, wb + wpk, Mr, N, Kd, epi, status);
     }
   }
   // the conditioning-modulated row norm of x fused into a projection's operand
@@ -200,7 +227,7 @@ struct PassCtx {
 template <typename Elt>
 int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p, float eps,
                int64_t radius, const atomenc_outputs *out, unsigned char *ws, cudaStream_t st,
-               Hooks &hk);
+               Hooks &hk, int mode = kPassFull, unsigned char *image = nullptr);
 template <typename Elt, typename WT>
 void launch_middle(PassCtx<Elt> &c);
 

@@ -43,7 +43,7 @@ void launch_middle(PassCtx<Elt> &c) {
      *wo = reinterpret_cast<WT *>(ws + pl.o_o);
   // ---- projections (attention inputs fused into the operand when C <= 256)
   if (pl.af3) {
-    EpiSplitT<WT> e0{{wq, wg, nullptr, nullptr}, {F(pl.o_bq), nullptr, nullptr, nullptr}, HD};
+    EpiSplitT<WT> e0{{wq, wg, nullptr, nullptr}, {c.WF(pl.o_bq), nullptr, nullptr, nullptr}, HD};
     EpiSplitT<WT> e1{{wk, wv, nullptr, nullptr}, {nullptr, nullptr, nullptr, nullptr}, HD};
     if (fuse_norm) {
       gemm_rows(norm_prod(0, C, false), pl.k_qkv0, R, 2 * HD, C, e0);
@@ -90,7 +90,7 @@ void launch_middle(PassCtx<Elt> &c) {
     ra2.window = static_cast<const uint8_t *>(in->window_mask.data);
     ra2.usable = usable;
     ra2.pair = pl.af3 ? in->pair.data : nullptr;
-    ra2.w_pair = F(pl.o_wpair);
+    ra2.w_pair = c.WF(pl.o_wpair);
     ra2.attention = out->attention.data;
     ra2.O = wo;
     ra2.status = status;
@@ -125,7 +125,7 @@ if (D == DH) {                                                    \
     ag.window = static_cast<const uint8_t *>(in->window_mask.data);
     ag.usable = usable;
     ag.pair = pl.af3 ? in->pair.data : nullptr;
-    ag.w_pair = F(pl.o_wpair);
+    ag.w_pair = c.WF(pl.o_wpair);
     ag.attention = out->attention.data;
     ag.O = F(pl.o_o);
     ag.status = status;
@@ -163,7 +163,7 @@ if (dm == DM) {                                                           \
     ta.sc = condb + 4 * C; ta.sh = condb + (pl.af3 ? 5 : 3) * C; ta.cond_ld = 6 * C;
     ta.rms = pl.af3 ? 0 : 1; ta.plus1 = pl.af3 ? 0 : 1; ta.eps = eps;
     ta.usable = usable;
-    ta.w_out = ws + pl.k_out; ta.w_ff1 = ws + pl.k_ff1; ta.w_ff2 = ws + pl.k_ff2;
+    ta.w_out = c.wb + pl.k_out; ta.w_ff1 = c.wb + pl.k_ff1; ta.w_ff2 = c.wb + pl.k_ff2;
     ta.hidden = out->hidden.data; ta.status = status;
     ta.xfer = F(pl.o_xfer); ta.xflag = reinterpret_cast<int *>(ws + pl.o_xflag);
     ta.peer_spin_limit = g_peer_spin_limit.load();

@@ -14,12 +14,18 @@ namespace host {
 template <typename Elt>
 int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p,
                float eps, int64_t radius, const atomenc_outputs *out, unsigned char *ws,
-               cudaStream_t st, Hooks &hk) {
+               cudaStream_t st, Hooks &hk, int mode, unsigned char *image) {
   const Dims &d = pl.d;
   const int64_t B = d.B, A = d.A, T = d.T, K = d.K, C = d.C, S = d.S, H = d.H, D = d.D,
                 P = d.P, M = d.M, U = d.U, V = d.V, HD = H * D, R = B * A;
   auto F = [&](size_t off) { return reinterpret_cast<float *>(ws + off); };
-  unsigned *status = reinterpret_cast<unsigned *>(ws + pl.o_status);
+  // weight-region offsets resolve against the workspace, or against a prepared image
+  // (whose region starts after its header)
+  unsigned char *wb = mode == kPassFull ? ws
+                                        : reinterpret_cast<unsigned char *>(
+                                              reinterpret_cast<uintptr_t>(image) + kImageHeader - pl.o_wbase);
+  auto WF = [&](size_t off) { return reinterpret_cast<float *>(wb + off); };
+  unsigned *status = mode == kPassPrepare ? nullptr : reinterpret_cast<unsigned *>(ws + pl.o_status);
   uint8_t *usable = ws + pl.o_usable;
   int *first = reinterpret_cast<int *>(ws + pl.o_first);
   int *last = reinterpret_cast<int *>(ws + pl.o_last);
@@ -39,7 +45,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     CopyJob &j = wj.copy[wj.ncopy++];
     j.src = elt(src, src_off);
     j.rowscale = rowscale ? elt(*rowscale, rs_off) : nullptr;
-    j.dst = F(dst_off);
+    j.dst = WF(dst_off);
     j.rows = (int32_t)rows;
     j.cols = (int32_t)cols;
     j.dst_ld = (int32_t)dst_ld;
@@ -49,7 +55,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   const bool split = pl.fdt == ATOMENC_F32;
   auto pack = [&](size_t dst, int64_t Kd, int64_t N) -> PackJob & {
     PackJob &j = wj.pack[wj.npack++];
-    j.dst = ws + dst;
+    j.dst = wb + dst;
     j.K = (int32_t)Kd;
     j.N = (int32_t)N;
     j.split = split ? 1 : 0;
@@ -64,6 +70,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     g.col0 = (int32_t)col0;
     g.cshift = cshift;
   };
+  if (mode != kPassPrepared) {   // the images and panels (a prepared image has them)
   if (pl.af3) {
     PackJob &jc = pack(pl.k_cond, S, 6 * C);
     for (int jj = 0; jj < 3; ++jj) {
@@ -104,14 +111,24 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     if (!pl.af3) copy(p->readout_bias, 0, 1, C, pl.o_rbias, C, 0, nullptr, 0);
     copy(p->w_readout, 0, C, 3, pl.o_wread, 3, 0, nullptr, 0);
   }
-  wj.fill[wj.nfill++] = FillJob{reinterpret_cast<int *>(status), 1, 0, 0};
+  }
+  // the image key: style, stage, storage type and every dimension the images depend on
+  image_key(pl, wj.key);
+  if (mode == kPassPrepare) {
+    wj.key_out = reinterpret_cast<int *>(image);
+    hk.launch(ATOMENC_KERNEL_PREP, (k_prep_weights<Elt>), dim3(64, wj.ncopy + wj.npack), 256, 0, st, wj);
+    if (hk.err != cudaSuccess) return ATOMENC_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? ATOMENC_OK : ATOMENC_ERR_CUDA;
+  }
+  if (mode == kPassPrepared) wj.key_in = reinterpret_cast<const int *>(image);
+  wj.status = status;   // reset (bit 8 when a prepared image does not match)
   if (pl.tail_pair)
     wj.fill[wj.nfill++] = FillJob{reinterpret_cast<int *>(ws + pl.o_xflag), 2 * ((R + kUmmaBM - 1) / kUmmaBM), 0, 0};
   if (pl.enc) {
     wj.fill[wj.nfill++] = FillJob{first, B * T, INT_MAX, 0};
     wj.fill[wj.nfill++] = FillJob{last, B * T, -1, 0};
   }
-  hk.launch(ATOMENC_KERNEL_PREP, (k_prep_weights<Elt>), dim3(64, wj.ncopy + wj.npack + wj.nfill), 256, 0, st, wj);
+  hk.launch(ATOMENC_KERNEL_PREP, (k_prep_weights<Elt>), dim3(64, std::max(wj.ncopy + wj.npack + wj.nfill, 1)), 256, 0, st, wj);
 
   const bool fuse_norm = C <= kRowsKMax;
   const int rows_per_block = 8;  // warps per 256-thread block for warp-per-row kernels
@@ -119,7 +136,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   Elt *xb = reinterpret_cast<Elt *>(ws + pl.o_x), *condb = reinterpret_cast<Elt *>(ws + pl.o_cond),
       *gateb = reinterpret_cast<Elt *>(ws + pl.o_gate), *poolb = reinterpret_cast<Elt *>(ws + pl.o_pool);
   PassCtx<Elt> c{pl, in, p, out, eps, radius, ws, st, hk, status, usable, split, fuse_norm,
-                 row_blocks, xb, condb, gateb, poolb};
+                 row_blocks, xb, condb, gateb, poolb, wb};
 
   // ---- decoder: token @ w_token, gathered per atom in the row pass
   if (!pl.enc)
@@ -153,9 +170,9 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   const Elt *cin = static_cast<const Elt *>(in->condition.data);
   if (pl.af3) {
     c.gemm_rows(ProdCond<Elt, 2>{cin, usable, F(pl.o_cstats), R, S}, pl.k_cond, R, 6 * C, S,
-              EpiCondAF3<Elt>{condb, F(pl.o_bscale), C});
+              EpiCondAF3<Elt>{condb, WF(pl.o_bscale), C});
     c.gemm_rows(ProdCond<Elt, 0>{cin, usable, nullptr, R, S}, pl.k_gate, R, 2 * C, S,
-              EpiGateAF3<Elt>{gateb, F(pl.o_brg), C});
+              EpiGateAF3<Elt>{gateb, WF(pl.o_brg), C});
   } else {
     c.gemm_rows(ProdCond<Elt, 1>{cin, usable, nullptr, R, S}, pl.k_cond, R, 6 * C, S,
               QuadStore<Elt>{condb, 6 * C});
@@ -197,8 +214,8 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     else
       hk.launch(ATOMENC_KERNEL_POOL, (k_token_mean<Elt>), (unsigned)(B * T), kPoolThreads, 0, st, pa);
   } else {
-    ReadoutArgs rd{R, C, eps, pl.af3 ? 0 : 1, usable, hid, F(pl.o_rscale), F(pl.o_rbias),
-                   F(pl.o_wread), out->position_update.data};
+    ReadoutArgs rd{R, C, eps, pl.af3 ? 0 : 1, usable, hid, WF(pl.o_rscale), WF(pl.o_rbias),
+                   WF(pl.o_wread), out->position_update.data};
     hk.launch(ATOMENC_KERNEL_ROWS, (k_readout<Elt>), row_blocks, 256, 0, st, rd);
   }
   hk.mark(6, st);

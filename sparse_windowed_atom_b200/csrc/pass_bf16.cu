@@ -3,6 +3,6 @@
 
 namespace atomenc {
 namespace host {
-template int launch_all<__nv_bfloat16>(const Plan &, const atomenc_inputs *, const atomenc_params *, float, int64_t, const atomenc_outputs *, unsigned char *, cudaStream_t, Hooks &);
+template int launch_all<__nv_bfloat16>(const Plan &, const atomenc_inputs *, const atomenc_params *, float, int64_t, const atomenc_outputs *, unsigned char *, cudaStream_t, Hooks &, int, unsigned char *);
 }  // namespace host
 }  // namespace atomenc

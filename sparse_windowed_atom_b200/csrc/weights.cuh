@@ -49,11 +49,21 @@ struct FillJob {
 };
 
 constexpr int kMaxCopyJobs = 12, kMaxPackJobs = 10, kMaxFillJobs = 4;
+// Prepared weight images start with kImageKeyWords words that name what they were built
+// for (style, stage, storage type, weight shapes): atomenc_prepare_weights writes them
+// (key_out), atomenc_forward_prepared checks them (key_in) and sets status bit 8 when they
+// differ.
+constexpr int kImageKeyWords = 4;
+constexpr unsigned kStatusImageMismatch = 8u;
 struct WeightJobs {
   CopyJob copy[kMaxCopyJobs];
   PackJob pack[kMaxPackJobs];
   FillJob fill[kMaxFillJobs];
   int ncopy, npack, nfill, pad;
+  int key[kImageKeyWords];
+  int *key_out;            // write the key here (preparation)
+  const int *key_in;       // compare the key found here (prepared forward)
+  unsigned *status;        // the pass's status word: reset here (bit 8 if key_in differs)
 };
 
 // One 16-byte chunk of the image per thread: output column n, eight consecutive k
@@ -107,6 +117,14 @@ __device__ __forceinline__ void pack_chunk(const PackJob &j, int64_t i, int64_t 
 template <typename T>
 __global__ void k_prep_weights(WeightJobs w) {
   pdl_enter();
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    bool same = true;
+    for (int i = 0; i < kImageKeyWords; ++i) {
+      if (w.key_out) w.key_out[i] = w.key[i];
+      if (w.key_in) same = same && w.key_in[i] == w.key[i];
+    }
+    if (w.status) *w.status = same ? 0u : kStatusImageMismatch;
+  }
   int y = blockIdx.y;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
