@@ -83,6 +83,7 @@ __device__ __forceinline__ void load8_t<__nv_bfloat16>(const __nv_bfloat16 *A, i
 // conditioning rows.
 template <typename TA>
 struct ProdPlain {
+  static constexpr bool kLight = true;   // a copy: four warps keep up with the epilogues
   const TA *A;
   int64_t lda, M, K;
   __device__ void load8(int64_t r, int64_t k, float (&v)[8]) const {
@@ -92,6 +93,7 @@ struct ProdPlain {
 
 template <typename IT>
 struct ProdNormT {
+  static constexpr bool kLight = false;
   const IT *x;           // [M, K] residual state, storage type
   const float *stats;    // [M, 2]: mean (0 for RMS) and rstd of each row of x
   const IT *cond;        // rows of cond_ld values, storage type
@@ -119,6 +121,7 @@ using ProdNorm = ProdNormT<float>;
 // LayerNorm statistics (AF3 c_j, bullet 7; cond_scale[j] is folded into the weights).
 template <typename T, int MODE>
 struct ProdCond {
+  static constexpr bool kLight = false;
   const T *c;            // [M, K] condition rows
   const uint8_t *usable; // [M]
   const float *stats;    // [M, 2] (MODE 2)
@@ -451,6 +454,233 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         umma::bulk_g2s(sR + (size_t)slot * PARTS * BLK,
                        Wpk + ((size_t)(t_begin + tl) * nkc + c) * PARTS * BLK, PARTS * BLK,
                        full + slot);
+      }
+    }
+  }
+  if (!ok) {
+    *abort_flag = 1;
+    atomicOr(status, kStatusMmaTimeout);
+  }
+  umma::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) umma::tmem_dealloc(tmem, 2 * kUmmaBN);
+}
+
+// ----------------------------------------------------------------------------------
+// Persistent row-block GEMM (bf16 operands, no hi/lo split): one CTA per SM walks the
+// row blocks blockIdx.x, blockIdx.x + gridDim.x, ... and all output tiles of each, with
+// the A operand double-buffered so that the operand of the next row block is formed
+// while the current one's MMAs and epilogues run. Fourteen warps (four per SM
+// sub-partition at most, so 128 registers a thread); roles:
+//   warps 0..EW-1      epilogue of each tile (TMEM lane quadrant w % 4, a 512/EW-column
+//                      share of the tile, transposed through a per-warp shared tile);
+//   warps EW..11       form the A operand (128/(12-EW) rows each) into the free buffer,
+//                      then arrive on its "full" barrier;
+//   warp 12            lane 0 issues the MMAs: two 128-column TMEM accumulators alternate
+//                      over the CTA's tiles; after a block's last tile a commit frees its A
+//                      buffer;
+//   warp 13            lane 0 streams the weight blocks through the ring (every block of
+//                      every tile, in the MMA's order).
+// EW = 8 for a light producer (a plain copy of bf16 rows), EW = 4 when the operand has a
+// normalisation or SiLU to form (eight producer warps keep up with four epilogue warps).
+// Every wait is bounded (status bit 4 on timeout; the other roles then stop too).
+constexpr int kRowsPThreads = 14 * 32;
+
+__host__ __device__ inline size_t rows_p_smem_bytes(int64_t K, int nslot, int ew) {
+  const size_t nkc = (size_t)((K + kUmmaBK - 1) / kUmmaBK);
+  return 1024 + (2 * nkc + (size_t)nslot) * kUmmaBlockBytes + (size_t)ew * 32 * kRowsTPitch * 4 + 512;
+}
+// weight slots of the persistent kernel: up to kRowsMaxSlots, at least 2, within the budget
+__host__ __device__ inline int rows_p_slots(int64_t K, int ew) {
+  int n = kRowsMaxSlots;
+  while (n > 2 && rows_p_smem_bytes(K, n, ew) > kRowsSmemBudget) --n;
+  return n;
+}
+
+template <class Prod, class Epi, int EW>
+__global__ void __launch_bounds__(kRowsPThreads, 1)
+    k_gemm_rows_p(Prod prod, const uint8_t *__restrict__ Wpk, int64_t M, int64_t N, int64_t K,
+                  int NSLOT, Epi epi, unsigned *status) {
+  constexpr int PW = 12 - EW;               // producer warps
+  constexpr int RPW = kUmmaBM / PW;         // operand rows per producer warp
+  constexpr int CPW = kUmmaBN * 4 / EW;     // tile columns per epilogue warp
+  static_assert(EW == 4 || EW == 8, "epilogue warps");
+  pdl_enter();
+  extern __shared__ __align__(1024) uint8_t smem_dyn[];
+  constexpr uint32_t BLK = kUmmaBlockBytes;
+  constexpr uint32_t idesc = umma::idesc_bf16(kUmmaBM, kUmmaBN);
+  uint8_t *sm = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  const int nkc = (int)((K + kUmmaBK - 1) / kUmmaBK);
+  uint8_t *sA = sm;                                       // [2][nkc] blocks
+  uint8_t *sR = sA + (size_t)2 * nkc * BLK;               // [NSLOT] blocks
+  float *sT = reinterpret_cast<float *>(sR + (size_t)NSLOT * BLK);   // [warps][32][pitch]
+  uint64_t *full = reinterpret_cast<uint64_t *>(sT + EW * 32 * kRowsTPitch);
+  uint64_t *empty = full + NSLOT, *accf = empty + NSLOT, *acce = accf + 2;
+  uint64_t *afull = acce + 2, *aempty = afull + 2;
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(aempty + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nt = (int)((N + kUmmaBN - 1) / kUmmaBN);
+  const int64_t mb = (M + kUmmaBM - 1) / kUmmaBM;
+  const int nblk = (int)((mb - blockIdx.x + gridDim.x - 1) / gridDim.x);   // my row blocks
+  if (nblk <= 0) return;  // uniform over the CTA
+
+  if (tid == 0) {
+    for (int s = 0; s < NSLOT; ++s) {
+      umma::mbar_init(full + s, 1);
+      umma::mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      umma::mbar_init(accf + b, 1);
+      umma::mbar_init(acce + b, EW);
+      umma::mbar_init(afull + b, PW);
+      umma::mbar_init(aempty + b, 1);
+    }
+    *abort_flag = 0;
+    umma::fence_mbar_init();
+  }
+  if (warp == 0) umma::tmem_alloc(tslot, 2 * kUmmaBN);
+  umma::tc_fence_before();
+  __syncthreads();
+  umma::tc_fence_after();
+  const uint32_t tmem = *tslot;
+  bool ok = true;
+
+  if (warp < EW) {
+    // ---- epilogues: tile g of the CTA (block bi, tile tl) reads accumulator g % 2
+    const int qd = warp & 3, cb = (warp >> 2) * CPW;
+    float *T = sT + warp * 32 * kRowsTPitch;
+    const uint32_t tlane = tmem + ((uint32_t)(qd * 32) << 16);
+    int g = 0;
+    for (int bi = 0; bi < nblk && ok; ++bi) {
+      const int64_t m0 = ((int64_t)blockIdx.x + (int64_t)bi * gridDim.x) * kUmmaBM;
+      for (int tl = 0; tl < nt && ok; ++tl, ++g) {
+        const int buf = g & 1;
+        ok = umma::mbar_wait_warp(accf + buf, (g >> 1) & 1, abort_flag, lane);
+        umma::tc_fence_after();
+        const int64_t n0 = (int64_t)tl * kUmmaBN;
+#pragma unroll 1
+        for (int c0 = cb; c0 < cb + CPW; c0 += 32) {
+          if (n0 + c0 >= N) break;
+          float v[32];
+          umma::tmem_ld32(tlane + buf * kUmmaBN + c0, v);
+          // 16-byte chunk j of row r at j ^ (r & 7): conflict-free stores and loads
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4 *>(T + lane * kRowsTPitch + 4 * (j ^ (lane & 7))) =
+                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+          __syncwarp();
+#pragma unroll 2
+          for (int i = 0; i < 8; ++i) {
+            const int rl = i * 4 + (lane >> 3), q = lane & 7;
+            const int64_t row = m0 + qd * 32 + rl, col = n0 + c0 + 4 * q;
+            if (ok && row < M && col < N) {
+              const float4 t4 = *reinterpret_cast<const float4 *>(T + rl * kRowsTPitch + 4 * (q ^ (rl & 7)));
+              const float x[4] = {t4.x, t4.y, t4.z, t4.w};
+              epi.quad(row, col, x, N);
+            }
+          }
+          __syncwarp();
+        }
+        umma::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) umma::mbar_arrive(acce + buf);
+      }
+    }
+  } else if (warp < EW + PW) {
+    // ---- A operand of each of the CTA's row blocks into buffer bi % 2: producer warp p
+    // forms rows RPW p .. RPW (p + 1) - 1 in groups of 16, the loads of chunk c + 1 in
+    // flight while chunk c is converted
+    const int pw = warp - EW;
+    for (int bi = 0; bi < nblk && ok; ++bi) {
+      const int buf = bi & 1;
+      if (bi >= 2) {
+        ok = umma::mbar_wait_warp(aempty + buf, ((bi - 2) >> 1) & 1, abort_flag, lane);
+        umma::tc_fence_after();
+        if (!ok) break;
+      }
+      const int64_t m0 = ((int64_t)blockIdx.x + (int64_t)bi * gridDim.x) * kUmmaBM;
+      uint8_t *aB = sA + (size_t)buf * nkc * BLK;
+      for (int half = 0; half < RPW / 16; ++half) {
+        const int r0 = pw * RPW + half * 16;
+        float vb[2][4][8];
+        auto load_chunk = [&](int c, float (&v)[4][8]) {
+#pragma unroll
+          for (int it = 0; it < 4; ++it)
+            prod.load8(m0 + r0 + it * 4 + (lane >> 3), (int64_t)c * kUmmaBK + (lane & 7) * 8, v[it]);
+        };
+        auto store_chunk = [&](int c, float (&v)[4][8]) {
+          uint8_t *a_c = aB + (size_t)c * BLK;
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int r = r0 + it * 4 + (lane >> 3), seg = lane & 7;
+            uint32_t hi[4], lo[4];
+            umma::split8<false>(v[it], hi, lo);
+            *reinterpret_cast<uint4 *>(a_c + umma::swz_offset(r, seg * 8, kUmmaBM)) =
+                make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          }
+        };
+        load_chunk(0, vb[0]);
+        for (int c = 0; c < nkc; c += 2) {
+          if (c + 1 < nkc) load_chunk(c + 1, vb[1]);
+          store_chunk(c, vb[0]);
+          if (c + 1 < nkc) {
+            if (c + 2 < nkc) load_chunk(c + 2, vb[0]);
+            store_chunk(c + 1, vb[1]);
+          }
+        }
+      }
+      umma::fence_async_smem();
+      __syncwarp();
+      if (lane == 0) umma::mbar_arrive(afull + buf);
+    }
+  } else if (warp == EW + PW) {
+    if (lane == 0) {
+      // ---- MMA issue
+      int g = 0;
+      for (int bi = 0; bi < nblk && ok; ++bi) {
+        const int ab = bi & 1;
+        ok = umma::mbar_wait(afull + ab, (bi >> 1) & 1, abort_flag);
+        umma::tc_fence_after();
+        for (int tl = 0; tl < nt && ok; ++tl, ++g) {
+          const int buf = g & 1;
+          if (g >= 2) {
+            ok = umma::mbar_wait(acce + buf, ((g - 2) >> 1) & 1, abort_flag);
+            umma::tc_fence_after();
+          }
+          const uint32_t dtm = tmem + buf * kUmmaBN;
+          for (int c = 0; c < nkc && ok; ++c) {
+            const int i = g * nkc + c, slot = i % NSLOT;
+            ok = umma::mbar_wait(full + slot, (i / NSLOT) & 1, abort_flag);
+            umma::tc_fence_after();
+            const uint32_t a0 = umma::smem_u32(sA + ((size_t)ab * nkc + c) * BLK);
+            const uint32_t b0 = umma::smem_u32(sR + (size_t)slot * BLK);
+#pragma unroll
+            for (int kk = 0; kk < kUmmaBK / 16; ++kk)
+              umma::mma_bf16(dtm, umma::sw128_desc(a0 + kk * 32), umma::sw128_desc(b0 + kk * 32), idesc,
+                             (c | kk) != 0);
+            umma::mma_commit(empty + slot);
+          }
+          umma::mma_commit(accf + buf);
+        }
+        umma::mma_commit(aempty + ab);   // the block's A buffer is free once these MMAs are done
+      }
+      // the last blocks' "A free" arrivals land before the CTA leaves
+      for (int bi = (nblk > 2 ? nblk - 2 : 0); bi < nblk && ok; ++bi)
+        ok = umma::mbar_wait(aempty + (bi & 1), (bi >> 1) & 1, abort_flag);
+    }
+  } else {
+    if (lane == 0) {
+      // ---- weight blocks of every tile of every block, ring of NSLOT buffers
+      const int total = nblk * nt * nkc;
+      for (int i = 0; i < total && ok; ++i) {
+        const int slot = i % NSLOT;
+        if (i >= NSLOT) ok = umma::mbar_wait(empty + slot, ((i - NSLOT) / NSLOT) & 1, abort_flag);
+        const int c = i % nkc, tl = (i / nkc) % nt;
+        umma::mbar_arrive_expect_tx(full + slot, BLK);
+        umma::bulk_g2s(sR + (size_t)slot * BLK, Wpk + ((size_t)tl * nkc + c) * BLK, BLK, full + slot);
       }
     }
   }

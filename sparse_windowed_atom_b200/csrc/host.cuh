@@ -183,6 +183,20 @@ struct PassCtx {
   template <class P, class E>
   void gemm_rows(P prod, size_t wpk, int64_t Mr, int64_t N, int64_t Kd, E epi) {
     const int64_t mt = (Mr + kUmmaBM - 1) / kUmmaBM, nt = (N + kUmmaBN - 1) / kUmmaBN;
+    // enough row blocks for every SM (a formed operand: three per SM, so that forming the
+    // next block's operand overlaps enough tiles): the persistent kernel (one CTA per SM,
+    // the next block's operand formed while the current one's tiles run)
+    if (!split && mt >= (P::kLight ? 1 : 3) * (int64_t)pl.sms) {
+      constexpr int EW = P::kLight ? 8 : 4;
+      const int nslot = rows_p_slots(Kd, EW);
+      const size_t smem = rows_p_smem_bytes(Kd, nslot, EW);
+      if (smem <= kRowsSmemBudget) {
+        smem_limit(k_gemm_rows_p<P, E, EW>, smem);
+        hk.launch(ATOMENC_KERNEL_GEMM, (k_gemm_rows_p<P, E, EW>), dim3((unsigned)pl.sms), kRowsPThreads,
+                  smem, st, prod, wb + wpk, Mr, N, Kd, nslot, epi, status);
+        return;
+      }
+    }
     const int64_t want = (pl.sms + mt - 1) / mt;          // CTAs per row block to fill the GPU
     const int64_t sp = want < nt ? want : nt;
     const int per = (int)((nt + sp - 1) / sp);
