@@ -211,6 +211,30 @@ __device__ __forceinline__ void ldpair16(const __nv_bfloat16 *pr, float (&x)[16]
 }
 __device__ __forceinline__ void ldpair16(const float *pr, float (&x)[16]) { ldn<16>(pr, x); }
 
+// Pair bias of one slot for heads 0..H-1 from its 16 pair channels x (in registers):
+// one shifted pass for the LayerNorm statistics, then the folded head sums
+template <int H>
+__device__ __forceinline__ void pair_bias16(float (&x)[16], float eps, const float *wp,
+                                            const float *wsum, float *out) {
+  const float x0 = x[0];
+  float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+  for (int p = 0; p < 16; ++p) {
+    x[p] -= x0;
+    s1 += x[p];
+    s2 = fmaf(x[p], x[p], s2);
+  }
+  const float m = s1 * (1.f / 16.f);
+  const float rstd = rsqrtf(fmaxf(s2 * (1.f / 16.f) - m * m, 0.f) + eps);
+#pragma unroll
+  for (int h = 0; h < H; ++h) {
+    float d = 0.f;
+#pragma unroll
+    for (int p = 0; p < 16; ++p) d = fmaf(x[p], wp[p * H + h], d);
+    out[h] = rstd * (d - m * wsum[h]);
+  }
+}
+
 // Pair bias of one slot for heads 0..H-1 (H <= 8):
 //   beta_h = sum_p LN(pair)_p * pair_scale_p * w_pair[p, h]
 //          = rstd * (sum_p y_p W'[p, h] - m * sum_p W'[p, h]),
@@ -392,6 +416,38 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
       // pair bias of every listed slot for every head, in list order
       __syncwarp();
       const T *prow = static_cast<const T *>(g.pair) + sb * P;
+      if constexpr (ES == 2) {
+        if (g.pair_vec) {
+          // 16 bf16 channels a slot: the rows of all of this lane's slots (at most 4) are
+          // loaded before any is used
+          uint4 raw[4][2];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int e = lane + 32 * u;
+            if (e < base) {
+              const uint4 *pr = reinterpret_cast<const uint4 *>(prow + (int64_t)cks[q * K + e] * P);
+              raw[u][0] = pr[0];
+              raw[u][1] = pr[1];
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int e = lane + 32 * u;
+            if (e < base) {
+              float x[16], lo8[8], hi8[8];
+              rowattn::unpack(raw[u][0], lo8);
+              rowattn::unpack(raw[u][1], hi8);
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                x[c] = lo8[c];
+                x[8 + c] = hi8[c];
+              }
+              rowattn::pair_bias16<H>(x, g.eps, s_wp, s_wsum, beta + ((size_t)q * K + e) * H);
+            }
+          }
+          continue;
+        }
+      }
       for (int e = lane; e < base; e += 32)
         rowattn::pair_bias<T, H>(prow + (int64_t)cks[q * K + e] * P, P, g.pair_vec != 0, g.eps,
                                  s_wp, s_wsum, beta + ((size_t)q * K + e) * H);

@@ -116,7 +116,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
   image_key(pl, wj.key);
   if (mode == kPassPrepare) {
     wj.key_out = reinterpret_cast<int *>(image);
-    hk.launch(ATOMENC_KERNEL_PREP, (k_prep_weights<Elt>), dim3(64, wj.ncopy + wj.npack), 256, 0, st, wj);
+    hk.launch(ATOMENC_KERNEL_PREP, (k_prep_weights<Elt>), dim3(kPrepBlocksPerJob, wj.ncopy + wj.npack), 256, 0, st, wj);
     if (hk.err != cudaSuccess) return ATOMENC_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? ATOMENC_OK : ATOMENC_ERR_CUDA;
   }
@@ -128,7 +128,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     wj.fill[wj.nfill++] = FillJob{first, B * T, INT_MAX, 0};
     wj.fill[wj.nfill++] = FillJob{last, B * T, -1, 0};
   }
-  hk.launch(ATOMENC_KERNEL_PREP, (k_prep_weights<Elt>), dim3(64, std::max(wj.ncopy + wj.npack + wj.nfill, 1)), 256, 0, st, wj);
+  hk.launch(ATOMENC_KERNEL_PREP, (k_prep_weights<Elt>), dim3(kPrepBlocksPerJob, std::max(wj.ncopy + wj.npack + wj.nfill, 1)), 256, 0, st, wj);
 
   const bool fuse_norm = C <= kRowsKMax;
   const int rows_per_block = 8;  // warps per 256-thread block for warp-per-row kernels

@@ -49,6 +49,7 @@ struct FillJob {
 };
 
 constexpr int kMaxCopyJobs = 12, kMaxPackJobs = 10, kMaxFillJobs = 4;
+constexpr int kPrepBlocksPerJob = 128;   // grid.x of k_prep_weights
 // Prepared weight images start with kImageKeyWords words that name what they were built
 // for (style, stage, storage type, weight shapes): atomenc_prepare_weights writes them
 // (key_out), atomenc_forward_prepared checks them (key_in) and sets status bit 8 when they
