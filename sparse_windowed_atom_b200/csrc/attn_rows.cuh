@@ -524,6 +524,41 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
   }
   __syncthreads();
 
+  // ---------------- while this tile computes: bring the next tile's inputs into L2 (its
+  // slot rows and AF3 pair rows, the Q and value-gate rows, and the rows its key span
+  // most likely adds, the QT after the ring's last), so that its lists and copies find
+  // them there
+  if (tile + 1 < t_end) {
+    const int nb = (tile + 1) / g.tiles_per_b, na0 = (tile + 1 - nb * g.tiles_per_b) * QT;
+    const int nnq = min(QT, A - na0);
+    const int64_t nrow = (int64_t)nb * A + na0;
+    const char *kb = reinterpret_cast<const char *>(g.key_index + nrow * K);
+    const char *wbp = reinterpret_cast<const char *>(g.window + nrow * K);
+    const int64_t kbytes = (int64_t)nnq * K * 8, wbytes = (int64_t)nnq * K, qbytes = (int64_t)nnq * RB;
+    const int nk = (int)((kbytes + 127) >> 7), nw = (int)((wbytes + 127) >> 7), nqr = (int)((qbytes + 127) >> 7);
+    int s0 = 0, ns = 0;
+    if (ring_b == nb && ring_lo <= ring_hi) {
+      s0 = ring_hi + 1;
+      ns = max(0, min(QT, A - s0));
+    }
+    const int nkv = (int)(((int64_t)ns * RB + 127) >> 7);
+    const int np = AF3 ? (int)(((int64_t)nnq * K * P * ES + 127) >> 7) : 0;
+    const char *pb = AF3 ? static_cast<const char *>(g.pair) + nrow * K * P * ES : nullptr;
+    const int total = nk + nw + 2 * nqr + 2 * nkv + np;
+    for (int i = tid; i < total; i += kRowAttnThreads) {
+      const char *ptr;
+      int j = i;
+      if (j < nk) ptr = kb + ((int64_t)j << 7);
+      else if ((j -= nk) < nw) ptr = wbp + ((int64_t)j << 7);
+      else if ((j -= nw) < nqr) ptr = reinterpret_cast<const char *>(Qg) + nrow * RB + ((int64_t)j << 7);
+      else if ((j -= nqr) < nqr) ptr = reinterpret_cast<const char *>(Gg) + nrow * RB + ((int64_t)j << 7);
+      else if ((j -= nqr) < nkv) ptr = reinterpret_cast<const char *>(Kg) + ((int64_t)nb * A + s0) * RB + ((int64_t)j << 7);
+      else if ((j -= nkv) < nkv) ptr = reinterpret_cast<const char *>(Vg) + ((int64_t)nb * A + s0) * RB + ((int64_t)j << 7);
+      else ptr = pb + ((int64_t)(j - nkv) << 7);
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+    }
+  }
+
   // One query: NIT list iterations at most (4 entries each), the K/V rows staged in
   // shared memory or read from global memory.
   auto run_query = [&](auto nit_c, auto staged_c, int q) {
