@@ -609,12 +609,16 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
     };
 
     // ---- logits of the listed slots (log2 units)
+    // (the loops over list iterations leave at the query's own count: no predicated
+    // iterations past it)
     float lt[NI];
     float mx = -INFINITY;
 #pragma unroll
+    for (int t = 0; t < NI; ++t) lt[t] = -INFINITY;
+#pragma unroll
     for (int t = 0; t < NI; ++t) {
-      lt[t] = -INFINITY;
-      if (t < niter) {
+      if (t >= niter) break;
+      {
         const int e = 4 * t + g4;
         const int j = row_of(e);
         float part;
@@ -653,10 +657,9 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
     float sum = 0.f;
 #pragma unroll
     for (int t = 0; t < NI; ++t) {
-      if (t < niter) {
-        lt[t] = lt[t] > -INFINITY ? rowattn::ex2(lt[t] - mx) : 0.f;
-        sum += lt[t];
-      }
+      if (t >= niter) break;
+      lt[t] = lt[t] > -INFINITY ? rowattn::ex2(lt[t] - mx) : 0.f;
+      sum += lt[t];
     }
     sum += __shfl_xor_sync(0xffffffffu, sum, 8);
     sum += __shfl_xor_sync(0xffffffffu, sum, 16);
@@ -673,7 +676,8 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
     for (int c = 0; c < LC / 2; ++c) acc2[c] = 0ull;
 #pragma unroll
     for (int t = 0; t < NI; ++t) {
-      if (t < niter) {
+      if (t >= niter) break;
+      {
         const int e = 4 * t + g4;
         const float w = lt[t] * inv;
         if (e < n && head_writer) rowattn::store_w<T>(wrow + cs[e], w);
