@@ -680,10 +680,11 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
       {
         const int e = 4 * t + g4;
         const float w = lt[t] * inv;
-        if (e < n && head_writer) rowattn::store_w<T>(wrow + cs[e], w);
         const int j = row_of(e);
         if constexpr (ES == 2) {
+          // the weight rounded to bf16 once: the stored weight and the one that scales V
           const uint16_t wb = __bfloat16_as_ushort(__float2bfloat16_rn(w));
+          if (e < n && head_writer) *reinterpret_cast<uint16_t *>(wrow + cs[e]) = wb;
 #pragma unroll
           for (int s = 0; s < NSEG; ++s) {
             const uint4 raw = chunk(vbase, Vg, j, s);
@@ -693,6 +694,7 @@ __global__ void __launch_bounds__(kRowAttnThreads, 1) k_attn_rows(RowAttnArgs g)
             axpy_bf16x2(wb, raw.w, acc[8 * s + 6], acc[8 * s + 7]);
           }
         } else {
+          if (e < n && head_writer) rowattn::store_w<T>(wrow + cs[e], w);
           const f32x2 w2 = pack2(w, w);
 #pragma unroll
           for (int s = 0; s < NSEG; ++s) {
