@@ -127,13 +127,14 @@ def load_peaks():
 
 def attention_kernel(spec) -> str:
     """The attention kernel the library launches for this shape: the row-gather kernel
-    when H*D = 128, a head spans a whole number of 16-channel lane groups (D a multiple
-    of 16, at most 8 heads), K <= 128 and (AF3) P <= 32; the per-(query, head) kernel
-    otherwise (the same rule as the workspace plan of the C library)."""
+    for bf16 storage (float32: problems of at most 1024 atoms) when H*D = 128, a head
+    spans a whole number of 16-channel lane groups (D a multiple of 16, at most 8
+    heads), K <= 128 and (AF3) P <= 32; the per-(query, head) kernel otherwise (the same
+    rule as the workspace plan of the C library)."""
     hd = spec.H * spec.D
     lc = hd // 8
-    rg = (hd == 128 and spec.D >= lc and spec.D % lc == 0 and hd // spec.D <= 8
-          and spec.K <= 128 and (spec.style != "af3" or spec.P <= 32))
+    rg = ((spec.dtype == "bfloat16" or spec.B * spec.A <= 1024) and hd == 128 and spec.D >= lc and spec.D % lc == 0
+          and hd // spec.D <= 8 and spec.K <= 128 and (spec.style != "af3" or spec.P <= 32))
     return "k_attn_rows" if rg else "k_slot_attention"
 
 

@@ -248,11 +248,14 @@ int validate(int style, int stage, const atomenc_inputs *in, const atomenc_param
   const bool fused = C <= kRowsKMax;
   pl.o_feat = take(cur, fused ? 0 : R * (pl.af3 ? 2 : 1) * C * 4);
   // row-gather attention: whole rows of all heads per quarter-warp (H*D == 128, a head
-  // spans a whole number of lanes, at most 8 heads, K <= 128)
+  // spans a whole number of lanes, at most 8 heads, K <= 128), for bf16 storage, and for
+  // float32 storage only on small problems (above a few thousand atoms the per-(query,
+  // head) kernel measured faster with float32 rows)
   {
     const int64_t lc = HD / 8;
-    pl.rg = HD == 128 && D >= lc && D % lc == 0 && HD / D <= kRowAttnHeadsMax &&
-            K <= kRowAttnKMax && (!pl.af3 || P <= kRowAttnPairMax) && B * A < INT_MAX;
+    pl.rg = (fdt == ATOMENC_BF16 || B * A <= kRowAttnF32MaxAtoms) && HD == 128 && D >= lc && D % lc == 0 &&
+            HD / D <= kRowAttnHeadsMax && K <= kRowAttnKMax && (!pl.af3 || P <= kRowAttnPairMax) &&
+            B * A < INT_MAX;
     pl.ws_bf16 = pl.rg && fdt == ATOMENC_BF16;
   }
   const int64_t wsz = pl.ws_bf16 ? 2 : 4;   // bytes per Q/K/V/G/O element

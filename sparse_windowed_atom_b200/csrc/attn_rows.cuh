@@ -50,6 +50,7 @@ constexpr int kRowAttnKMax = 128;                  // slots per query (list entr
 constexpr int kRowAttnIters = kRowAttnKMax / 4;     // list entries per quarter-warp
 constexpr int kRowAttnPairMax = 32;
 constexpr int kRowAttnHeadsMax = 8;
+constexpr int kRowAttnF32MaxAtoms = 1024;   // float32 storage: problems up to this many atoms
 
 struct RowAttnArgs {
   int B, A, K, H, D, P;

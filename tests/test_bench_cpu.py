@@ -65,11 +65,14 @@ def test_recorded_traffic_is_keyed_by_workload_and_source():
 
 
 def test_attention_kernel_choice():
-    # every workload of the benchmark list has H*D = 128 and K <= 128: the row-gather kernel
+    # every workload of the benchmark list has H*D = 128 and K <= 128: the row-gather
+    # kernel for bf16 storage and small float32 problems, the per-(query, head) kernel
+    # for larger float32 ones
     for w in workloads.WORKLOADS.values():
-        assert bench.attention_kernel(w) == "k_attn_rows", w.name
+        want = "k_attn_rows" if w.dtype == "bfloat16" or w.B * w.A <= 1024 else "k_slot_attention"
+        assert bench.attention_kernel(w) == want, w.name
     import dataclasses
-    w = workloads.WORKLOADS["esm_encoder_fp32_a4096"]
+    w = workloads.WORKLOADS["esm_encoder_bf16_b2_a32768"]
     assert bench.attention_kernel(dataclasses.replace(w, K=160)) == "k_slot_attention"
     assert bench.attention_kernel(dataclasses.replace(w, H=2, D=32)) == "k_slot_attention"
     assert bench.attention_kernel(dataclasses.replace(w, H=16, D=8)) == "k_slot_attention"
