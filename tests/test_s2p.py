@@ -93,6 +93,18 @@ def test_parity(dtype, output_norm):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("output_norm", [False, True])
+@pytest.mark.parametrize("kw", [dict(B=2, N=150, C=64, H=32, Dp=128), dict(B=1, N=130, C=96, H=64, Dp=96),
+                                dict(B=1, N=40, C=32, H=16, Dp=256)])
+def test_parity_tensor_core_readout(dtype, output_norm, kw):
+    """2H and D multiples of 32 (2H <= 128, D <= 256): the tensor-core readout, with a
+    ragged last tile of pairs, two k chunks (2H = 128), a padded output tile (D = 96) and
+    two output tiles (D = 256)."""
+    _check(17, dtype, output_norm, **kw)
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("kw", [dict(B=1, N=1, C=5, H=1, Dp=3), dict(B=3, N=33, C=130, H=128, Dp=64),
                                 dict(B=1, N=65, C=96, H=32, Dp=256), dict(B=2, N=20, p_present=0.0)])
 def test_shapes_and_edges(kw):
