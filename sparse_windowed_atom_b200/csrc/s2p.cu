@@ -42,7 +42,7 @@ struct QKArgs {
 };
 
 // rows per CTA of the projection pass; its weight [C, 2H] is staged once per CTA
-constexpr int kQKRows = 16, kQKThreads = kQKRows * 32;
+constexpr int kQKRows = 4, kQKThreads = kQKRows * 32;
 
 template <typename T>
 __global__ void __launch_bounds__(kQKThreads) k_s2p_qk(QKArgs a) {
