@@ -74,7 +74,47 @@ __device__ __forceinline__ void load8_t<__nv_bfloat16>(const __nv_bfloat16 *A, i
   }
 }
 
+// Eight consecutive elements of a row as loaded (one 16-byte load for bf16, two for
+// float32), and their values.
+template <typename T> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> { uint4 u; };
+template <> struct Raw8<float> { float4 a, b; };
+__device__ __forceinline__ void raw8_load(const __nv_bfloat16 *p, Raw8<__nv_bfloat16> &w) {
+  w.u = *reinterpret_cast<const uint4 *>(p);
+}
+__device__ __forceinline__ void raw8_load(const float *p, Raw8<float> &w) {
+  w.a = *reinterpret_cast<const float4 *>(p);
+  w.b = *reinterpret_cast<const float4 *>(p + 4);
+}
+__device__ __forceinline__ void raw8_get(const Raw8<__nv_bfloat16> &w, float (&v)[8]) {
+  const uint32_t u[4] = {w.u.x, w.u.y, w.u.z, w.u.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    v[2 * e] = __uint_as_float(u[e] << 16);
+    v[2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void raw8_get(const Raw8<float> &w, float (&v)[8]) {
+  v[0] = w.a.x; v[1] = w.a.y; v[2] = w.a.z; v[3] = w.a.w;
+  v[4] = w.b.x; v[5] = w.b.y; v[6] = w.b.z; v[7] = w.b.w;
+}
+// rows of a [*, ld] tensor can be read as aligned groups of eight from column 8j
+template <typename T>
+__device__ __forceinline__ bool rows_vec_ok(const T *p, int64_t ld) {
+  return (reinterpret_cast<uintptr_t>(p) & 15) == 0 && (ld & 7) == 0;
+}
+
 // ---- A producers of the row-block GEMM: what the CTA converts into its A operand.
+// Each has two ways of delivering eight consecutive k of one row:
+//   load8(r, k, v)        loads and converts at once, any shape or alignment;
+//   issue(r, k, w) and finish(w, r, k, v)
+//                         the loads alone (no branch: the row and k are clamped into the
+//                         tensor, so every address is readable) and, later, the
+//                         conversion, with rows >= M and k >= K set to zero. The operand
+//                         loops keep kPipe chunks of these loads in flight. Usable when
+//                         vec_ok() (K a multiple of 8, rows 16-byte aligned); kPipe = 0
+//                         keeps a producer on load8 (its raw loads would not fit in
+//                         registers).
 // ProdPlain: A itself. ProdNorm: a row normalisation fused into the operand,
 //   (x - mean) * rstd * scale + shift      (AF3 adaptive LN; the scale column already
 //                                           holds sigmoid(...))
@@ -84,32 +124,72 @@ __device__ __forceinline__ void load8_t<__nv_bfloat16>(const __nv_bfloat16 *A, i
 template <typename TA>
 struct ProdPlain {
   static constexpr bool kLight = true;   // a copy: four warps keep up with the epilogues
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kPipe = 1;
   const TA *A;
   int64_t lda, M, K;
   __device__ void load8(int64_t r, int64_t k, float (&v)[8]) const {
     load8_t(A, lda, M, K, r, k, v);
+  }
+  struct Raw { Raw8<TA> a; };
+  __device__ bool vec_ok() const { return M > 0 && K > 0 && (K & 7) == 0 && rows_vec_ok(A, lda); }
+  __device__ void issue(int64_t r, int64_t k, Raw &w) const {
+    raw8_load(A + (r < M ? r : M - 1) * lda + (k < K ? k : K - 8), w.a);
+  }
+  __device__ void finish(const Raw &w, int64_t r, int64_t k, float (&v)[8]) const {
+    float a[8];
+    raw8_get(w.a, a);
+    const bool in = r < M && k < K;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = in ? a[e] : 0.f;
   }
 };
 
 template <typename IT>
 struct ProdNormT {
   static constexpr bool kLight = false;
+  // bf16: the pipelined loads let four producer warps keep up with eight epilogue warps
+  static constexpr int kEpiWarps = sizeof(IT) == 2 ? 8 : 4;
   const IT *x;           // [M, K] residual state, storage type
   const float *stats;    // [M, 2]: mean (0 for RMS) and rstd of each row of x
   const IT *cond;        // rows of cond_ld values, storage type
   int64_t M, K, cond_ld, sc_off, sh_off;
   int plus1;
+  static constexpr int kPipe = sizeof(IT) == 2 ? 1 : 0;
   __device__ void load8(int64_t r, int64_t k, float (&v)[8]) const {
     float xv[8], sc[8], sh[8];
     load8_t(x, K, M, K, r, k, xv);
     load8_t(cond + sc_off, cond_ld, M, K, r, k, sc);
     load8_t(cond + sh_off, cond_ld, M, K, r, k, sh);
     const float2 ms = r < M ? *reinterpret_cast<const float2 *>(stats + 2 * r) : make_float2(0.f, 0.f);
+    combine(xv, sc, sh, ms, r < M, k, v);
+  }
+  __device__ void combine(const float (&xv)[8], const float (&sc)[8], const float (&sh)[8], float2 ms,
+                          bool row_in, int64_t k, float (&v)[8]) const {
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const float s = plus1 ? 1.f + sc[e] : sc[e];
-      v[e] = (r < M && k + e < K) ? fmaf((xv[e] - ms.x) * ms.y, s, sh[e]) : 0.f;
+      v[e] = (row_in && k + e < K) ? fmaf((xv[e] - ms.x) * ms.y, s, sh[e]) : 0.f;
     }
+  }
+  struct Raw { Raw8<IT> x, sc, sh; float2 ms; };
+  __device__ bool vec_ok() const {
+    return M > 0 && K > 0 && (K & 7) == 0 && rows_vec_ok(x, K) && rows_vec_ok(cond + sc_off, cond_ld) &&
+           rows_vec_ok(cond + sh_off, cond_ld) && (reinterpret_cast<uintptr_t>(stats) & 7) == 0;
+  }
+  __device__ void issue(int64_t r, int64_t k, Raw &w) const {
+    const int64_t rc = r < M ? r : M - 1, kc = k < K ? k : K - 8;
+    raw8_load(x + rc * K + kc, w.x);
+    raw8_load(cond + sc_off + rc * cond_ld + kc, w.sc);
+    raw8_load(cond + sh_off + rc * cond_ld + kc, w.sh);
+    w.ms = *reinterpret_cast<const float2 *>(stats + 2 * rc);
+  }
+  __device__ void finish(const Raw &w, int64_t r, int64_t k, float (&v)[8]) const {
+    float xv[8], sc[8], sh[8];
+    raw8_get(w.x, xv);
+    raw8_get(w.sc, sc);
+    raw8_get(w.sh, sh);
+    combine(xv, sc, sh, w.ms, r < M, k, v);
   }
 };
 using ProdNorm = ProdNormT<float>;
@@ -122,10 +202,12 @@ using ProdNorm = ProdNormT<float>;
 template <typename T, int MODE>
 struct ProdCond {
   static constexpr bool kLight = false;
+  static constexpr int kEpiWarps = 4;   // SiLU / LayerNorm operands over K up to 256
   const T *c;            // [M, K] condition rows
   const uint8_t *usable; // [M]
   const float *stats;    // [M, 2] (MODE 2)
   int64_t M, K;
+  static constexpr int kPipe = 1;
   __device__ void load8(int64_t r, int64_t k, float (&v)[8]) const {
     // the loads do not wait for the usable flag (every row in range is readable memory;
     // what an unusable row holds is dropped by the select below)
@@ -133,7 +215,9 @@ struct ProdCond {
     load8_t(c, K, M, K, r, k, cv);
     float2 ms = make_float2(0.f, 1.f);
     if (MODE == 2 && r < M) ms = *reinterpret_cast<const float2 *>(stats + 2 * r);
-    const bool use = r < M && usable[r] != 0;
+    combine(cv, ms, r < M && usable[r] != 0, k, v);
+  }
+  __device__ void combine(const float (&cv)[8], float2 ms, bool use, int64_t k, float (&v)[8]) const {
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       float y = cv[e];
@@ -141,6 +225,23 @@ struct ProdCond {
       if (MODE == 2) y = (y - ms.x) * ms.y;
       v[e] = (use && k + e < K) ? y : 0.f;
     }
+  }
+  struct Raw { Raw8<T> c; float2 ms; uint32_t use; };
+  __device__ bool vec_ok() const {
+    return M > 0 && K > 0 && (K & 7) == 0 && rows_vec_ok(c, K) &&
+           (MODE != 2 || (reinterpret_cast<uintptr_t>(stats) & 7) == 0);
+  }
+  __device__ void issue(int64_t r, int64_t k, Raw &w) const {
+    const int64_t rc = r < M ? r : M - 1;
+    raw8_load(c + rc * K + (k < K ? k : K - 8), w.c);
+    w.use = usable[rc];
+    w.ms = make_float2(0.f, 1.f);
+    if (MODE == 2) w.ms = *reinterpret_cast<const float2 *>(stats + 2 * rc);
+  }
+  __device__ void finish(const Raw &w, int64_t r, int64_t k, float (&v)[8]) const {
+    float cv[8];
+    raw8_get(w.c, cv);
+    combine(cv, w.ms, r < M && w.use != 0, k, v);
   }
 };
 
@@ -287,6 +388,86 @@ __host__ __device__ inline int rows_slots(int64_t K, bool split, int blocks_per_
   return n < 2 ? 2 : n;
 }
 
+// The epilogue of one 32 x 32 chunk of accumulator rows: v holds this lane's row (TMEM
+// lane = row) at 32 consecutive columns. The chunk is transposed through the warp's shared
+// tile T so that each store instruction covers 64 contiguous bytes of four rows: lane
+// (rr = lane / 8, q = lane % 8) hands columns col0 + 4q .. + 3 of rows row0 + rr, + 4, ...
+// to the epilogue functor. 16-byte chunk j of tile row r sits at chunk j ^ (r & 7), so the
+// eight lanes of a store phase (eight rows, one chunk) and of a load phase (one row, eight
+// chunks) each cover all 32 banks once. The shared loads are issued in batches of
+// epi_batch<Epi> and a whole in-range chunk takes one bounds check, so the stores of a
+// batch do not wait on one another.
+template <class Epi>
+__device__ __forceinline__ void epi_chunk(const Epi &epi, float *T, const float (&v)[32], int lane,
+                                          int64_t row0, int64_t col0, int64_t M, int64_t N, bool ok) {
+  constexpr int NB = EpiBatch<Epi>::value;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<float4 *>(T + lane * kRowsTPitch + 4 * (j ^ (lane & 7))) =
+        make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  __syncwarp();
+  const int q = lane & 7, rr = lane >> 3;
+  const int64_t col = col0 + 4 * q;
+  const bool whole = row0 + 32 <= M && col0 + 32 <= N;
+#pragma unroll
+  for (int i0 = 0; i0 < 8; i0 += NB) {
+    float4 t[NB];
+#pragma unroll
+    for (int i = 0; i < NB; ++i) {
+      const int rl = (i0 + i) * 4 + rr;
+      t[i] = *reinterpret_cast<const float4 *>(T + rl * kRowsTPitch + 4 * (q ^ (rl & 7)));
+    }
+    if (ok) {
+#pragma unroll
+      for (int i = 0; i < NB; ++i) {
+        const int64_t row = row0 + (i0 + i) * 4 + rr;
+        const float x[4] = {t[i].x, t[i].y, t[i].z, t[i].w};
+        if (whole || (row < M && col < N)) epi.quad(row, col, x, N);
+      }
+    }
+  }
+  __syncwarp();   // T is free for the next chunk
+}
+
+template <bool SPLIT, int P, class Prod>
+__device__ __forceinline__ void form_rows_pipelined(const Prod &prod, uint8_t *aB, int64_t m0, int row_first,
+                                                    int halves, int nkc, int lane) {
+  constexpr int PARTS = SPLIT ? 2 : 1;
+  constexpr uint32_t BLK = kUmmaBlockBytes;
+  const int nst = halves * nkc, seg = lane & 7;
+  auto row_of = [&](int st, int it) { return row_first + (st / nkc) * 16 + it * 4 + (lane >> 3); };
+  auto k_of = [&](int st) { return (int64_t)(st % nkc) * kUmmaBK + seg * 8; };
+  typename Prod::Raw w[P][4];
+#pragma unroll
+  for (int p = 0; p < P; ++p)
+    if (p < nst) {
+#pragma unroll
+      for (int it = 0; it < 4; ++it) prod.issue(m0 + row_of(p, it), k_of(p), w[p][it]);
+    }
+  for (int s0 = 0; s0 < nst; s0 += P) {
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+      const int st = s0 + p;
+      if (st < nst) {
+        uint8_t *a_c = aB + (size_t)(st % nkc) * PARTS * BLK;
+        const int64_t k = k_of(st);
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          const int r = row_of(st, it);
+          float v[8];
+          prod.finish(w[p][it], m0 + r, k, v);
+          if (st + P < nst) prod.issue(m0 + row_of(st + P, it), k_of(st + P), w[p][it]);
+          uint32_t hi[4], lo[4];
+          umma::split8<SPLIT>(v, hi, lo);
+          const uint32_t off = umma::swz_offset(r, seg * 8, kUmmaBM);
+          *reinterpret_cast<uint4 *>(a_c + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          if (SPLIT) *reinterpret_cast<uint4 *>(a_c + BLK + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+      }
+    }
+  }
+}
+
 template <class Prod, bool SPLIT, class Epi>
 __global__ void __launch_bounds__(kRowsThreads, 1)
     k_gemm_rows(Prod prod, const uint8_t *__restrict__ Wpk, int64_t M, int64_t N, int64_t K,
@@ -337,6 +518,14 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
   if (warp < kRowsEpiWarps) {
     // ---- A: rows 16w..16w+15 of the tile, every k chunk, bf16 (hi[, lo]) swizzled;
     // the loads of chunk c + 1 are issued before chunk c is converted
+    bool piped = false;
+    if constexpr (Prod::kPipe > 0) {
+      if (prod.vec_ok()) {
+        form_rows_pipelined<SPLIT, Prod::kPipe>(prod, sA, m0, warp * 16, 1, nkc, lane);
+        piped = true;
+      }
+    }
+    if (!piped) {
     float vb[2][4][8];
     auto load_chunk = [&](int c, float (&v)[4][8]) {
 #pragma unroll
@@ -367,6 +556,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         store_chunk(c + 1, vb[1]);
       }
     }
+    }
     umma::fence_async_smem();
     __syncwarp();
     if (lane == 0) umma::mbar_arrive(aready);
@@ -386,25 +576,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         if (n0 + c0 >= N) break;
         float v[32];
         umma::tmem_ld32(tlane + buf * kUmmaBN + c0, v);
-        // 16-byte shared stores and loads; 16-byte chunk j of row r sits at chunk
-        // j ^ (r & 7), so the eight lanes of a store phase (eight rows, one chunk) and of
-        // a load phase (one row, eight chunks) each cover all 32 banks once
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<float4 *>(T + lane * kRowsTPitch + 4 * (j ^ (lane & 7))) =
-              make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-        __syncwarp();
-#pragma unroll 2
-        for (int i = 0; i < 8; ++i) {
-          const int rl = i * 4 + (lane >> 3), q = lane & 7;
-          const int64_t row = m0 + qd * 32 + rl, col = n0 + c0 + 4 * q;
-          if (ok && row < M && col < N) {
-            const float4 t4 = *reinterpret_cast<const float4 *>(T + rl * kRowsTPitch + 4 * (q ^ (rl & 7)));
-            const float x[4] = {t4.x, t4.y, t4.z, t4.w};
-            epi.quad(row, col, x, N);
-          }
-        }
-        __syncwarp();
+        epi_chunk(epi, T, v, lane, m0 + qd * 32, n0 + c0, M, N, ok);
       }
       umma::tc_fence_before();
       __syncwarp();
@@ -481,8 +653,9 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
 //                      buffer;
 //   warp 13            lane 0 streams the weight blocks through the ring (every block of
 //                      every tile, in the MMA's order).
-// EW = 8 for a light producer (a plain copy of bf16 rows), EW = 4 when the operand has a
-// normalisation or SiLU to form (eight producer warps keep up with four epilogue warps).
+// EW is the producer's kEpiWarps: 8 for a plain copy and for the bf16 modulated norm of
+// the projections (four producer warps with pipelined loads keep up), 4 for the condition
+// operands (SiLU / LayerNorm over K up to 256 need eight producer warps).
 // Every wait is bounded (status bit 4 on timeout; the other roles then stop too).
 constexpr int kRowsPThreads = 14 * 32;
 
@@ -566,23 +739,7 @@ __global__ void __launch_bounds__(kRowsPThreads, 1)
           if (n0 + c0 >= N) break;
           float v[32];
           umma::tmem_ld32(tlane + buf * kUmmaBN + c0, v);
-          // 16-byte chunk j of row r at j ^ (r & 7): conflict-free stores and loads
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<float4 *>(T + lane * kRowsTPitch + 4 * (j ^ (lane & 7))) =
-                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-          __syncwarp();
-#pragma unroll 2
-          for (int i = 0; i < 8; ++i) {
-            const int rl = i * 4 + (lane >> 3), q = lane & 7;
-            const int64_t row = m0 + qd * 32 + rl, col = n0 + c0 + 4 * q;
-            if (ok && row < M && col < N) {
-              const float4 t4 = *reinterpret_cast<const float4 *>(T + rl * kRowsTPitch + 4 * (q ^ (rl & 7)));
-              const float x[4] = {t4.x, t4.y, t4.z, t4.w};
-              epi.quad(row, col, x, N);
-            }
-          }
-          __syncwarp();
+          epi_chunk(epi, T, v, lane, m0 + qd * 32, n0 + c0, M, N, ok);
         }
         umma::tc_fence_before();
         __syncwarp();
@@ -594,6 +751,8 @@ __global__ void __launch_bounds__(kRowsPThreads, 1)
     // forms rows RPW p .. RPW (p + 1) - 1 in groups of 16, the loads of chunk c + 1 in
     // flight while chunk c is converted
     const int pw = warp - EW;
+    bool pipe_ok = false;
+    if constexpr (Prod::kPipe > 0) pipe_ok = prod.vec_ok();
     for (int bi = 0; bi < nblk && ok; ++bi) {
       const int buf = bi & 1;
       if (bi >= 2) {
@@ -603,6 +762,15 @@ __global__ void __launch_bounds__(kRowsPThreads, 1)
       }
       const int64_t m0 = ((int64_t)blockIdx.x + (int64_t)bi * gridDim.x) * kUmmaBM;
       uint8_t *aB = sA + (size_t)buf * nkc * BLK;
+      if constexpr (Prod::kPipe > 0) {
+        if (pipe_ok) {
+          form_rows_pipelined<false, Prod::kPipe>(prod, aB, m0, pw * RPW, RPW / 16, nkc, lane);
+          umma::fence_async_smem();
+          __syncwarp();
+          if (lane == 0) umma::mbar_arrive(afull + buf);
+          continue;
+        }
+      }
       for (int half = 0; half < RPW / 16; ++half) {
         const int r0 = pw * RPW + half * 16;
         float vb[2][4][8];

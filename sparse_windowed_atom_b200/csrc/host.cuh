@@ -187,7 +187,7 @@ struct PassCtx {
     // next block's operand overlaps enough tiles): the persistent kernel (one CTA per SM,
     // the next block's operand formed while the current one's tiles run)
     if (!split && mt >= (P::kLight ? 1 : 3) * (int64_t)pl.sms) {
-      constexpr int EW = P::kLight ? 8 : 4;
+      constexpr int EW = P::kEpiWarps;
       const int nslot = rows_p_slots(Kd, EW);
       const size_t smem = rows_p_smem_bytes(Kd, nslot, EW);
       if (smem <= kRowsSmemBudget) {

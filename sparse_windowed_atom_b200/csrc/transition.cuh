@@ -205,16 +205,22 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
     auto epi_sync = []() { asm volatile("bar.sync 1, %0;" ::"n"(kTransEpiWarps * 32) : "memory"); };
 
     // ---- o rows -> first operand (warp w converts rows 16w..16w+15; 8 lanes per row
-    // segment, coalesced)
-    for (int kc = 0; kc < nkc_out; ++kc) {
-      float v[4][8];
+    // segment, coalesced; the next chunk's loads in flight while one is converted)
+    {
+      const ProdPlain<TO> po{static_cast<const TO *>(t.O), (int64_t)t.HD, t.R, (int64_t)t.HD};
+      if (po.vec_ok()) {
+        form_rows_pipelined<SPLIT, 1>(po, sA, m0, warp * 16, 1, nkc_out, lane);
+      } else {
+        for (int kc = 0; kc < nkc_out; ++kc) {
+          float v[4][8];
 #pragma unroll
-      for (int it = 0; it < 4; ++it)
-        load8_t(static_cast<const TO *>(t.O), t.HD, t.R, t.HD, m0 + warp * 16 + it * 4 + (lane >> 3),
-                (int64_t)kc * kUmmaBK + (lane & 7) * 8, v[it]);
+          for (int it = 0; it < 4; ++it)
+            po.load8(m0 + warp * 16 + it * 4 + (lane >> 3), (int64_t)kc * kUmmaBK + (lane & 7) * 8, v[it]);
 #pragma unroll
-      for (int it = 0; it < 4; ++it)
-        put8<SPLIT>(sA + kc * P * BLK, warp * 16 + it * 4 + (lane >> 3), (lane & 7) * 8, v[it]);
+          for (int it = 0; it < 4; ++it)
+            put8<SPLIT>(sA + kc * P * BLK, warp * 16 + it * 4 + (lane >> 3), (lane & 7) * 8, v[it]);
+        }
+      }
     }
     umma::fence_async_smem();
     __syncwarp();
