@@ -159,7 +159,8 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     const bool reg = C % 4 == 0 && S % 4 == 0 && C <= 256 && S <= 256 &&
                      ((reinterpret_cast<uintptr_t>(in->atom.data) | reinterpret_cast<uintptr_t>(in->condition.data)) & al) == 0;
     if (reg)
-      hk.launch(ATOMENC_KERNEL_ROWS, (k_rows_prep_reg<Elt>), row_blocks, 256, 0, st, ra);
+      hk.launch(ATOMENC_KERNEL_ROWS, (k_rows_prep_reg<Elt>), dim3((unsigned)((A + 7) / 8), (unsigned)B), 256, 0,
+                st, ra);
     else
       hk.launch(ATOMENC_KERNEL_ROWS, (k_rows_prep<Elt>), row_blocks, 256, 0, st, ra);
   }

@@ -25,6 +25,12 @@ struct RowsArgs {
 // The conditioning products read the condition itself (sanitised, and SiLU'd or
 // normalised with cstats, while their operand is formed); no copy of it is written.
 
+// x / n, as a multiply by 1/n when n is a power of two (1/n is then exact, so the product
+// is the same correctly rounded value as the quotient), else the IEEE division
+__device__ __forceinline__ float div_n(float x, int n) {
+  return (n & (n - 1)) == 0 ? x * __int_as_float((127 - (31 - __clz(n))) << 23) : x / (float)n;
+}
+
 // One warp per atom. usable = valid & 0 <= atom_to_token < T & token_valid  (bullet 2);
 // payloads of unusable atoms are replaced by zero with a select before any arithmetic
 // (bullet 3); encoder x = atom, decoder x = skip + gather(token @ w_token) (bullet 3).
@@ -116,13 +122,14 @@ __device__ __forceinline__ void st4(__nv_bfloat16 *p, float *v) {
 // the row held in registers (lane l owns channels 4l..4l+3 and 128+4l..128+4l+3). Every
 // load of the caller's inputs is issued before the wait for the previous kernel, whose
 // results (the reset token ranges; the token projection in the decoder) are used after.
+// Grid: (ceil(A / 8), B), a warp per atom a of batch element b = blockIdx.y.
 template <typename T>
 __global__ void k_rows_prep_reg(RowsArgs r) {
   pdl_launch_next();
   const int lane = threadIdx.x & 31;
-  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const bool live = row < r.B * r.A;
-  const int64_t b = live ? row / r.A : 0, a = live ? row % r.A : 0;
+  const int64_t b = blockIdx.y, a = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const bool live = a < r.A;
+  const int64_t row = b * r.A + a;
   const int C = (int)r.C, S = (int)r.S;
   // the payload rows are loaded whatever the flags say (they are readable memory) and
   // replaced by zero with a select below, so their loads overlap the flag loads
@@ -169,7 +176,7 @@ __global__ void k_rows_prep_reg(RowsArgs r) {
       s1 += (xv[4 * h] + xv[4 * h + 1]) + (xv[4 * h + 2] + xv[4 * h + 3]);
     }
   }
-  const float mean = r.af3 ? warp_sum(s1) / (float)C : 0.f;
+  const float mean = r.af3 ? div_n(warp_sum(s1), C) : 0.f;
   float s2 = 0.f;
 #pragma unroll
   for (int h = 0; h < 2; ++h)
@@ -182,7 +189,7 @@ __global__ void k_rows_prep_reg(RowsArgs r) {
   s2 = warp_sum(s2);
   if (lane == 0) {
     r.xstats[2 * row] = mean;
-    r.xstats[2 * row + 1] = 1.f / sqrtf(s2 / (float)C + r.eps);
+    r.xstats[2 * row + 1] = 1.f / sqrtf(div_n(s2, C) + r.eps);
   }
   if (r.af3) {
     // population LayerNorm statistics of the condition, eps inside the root (bullet 7)
@@ -190,7 +197,7 @@ __global__ void k_rows_prep_reg(RowsArgs r) {
 #pragma unroll
     for (int h = 0; h < 2; ++h)
       if (h * 128 + 4 * lane < S) sc += (cv[4 * h] + cv[4 * h + 1]) + (cv[4 * h + 2] + cv[4 * h + 3]);
-    const float cm = warp_sum(sc) / (float)S;
+    const float cm = div_n(warp_sum(sc), S);
     float q = 0.f;
 #pragma unroll
     for (int h = 0; h < 2; ++h)
@@ -200,7 +207,7 @@ __global__ void k_rows_prep_reg(RowsArgs r) {
           const float d = cv[4 * h + e] - cm;
           q = fmaf(d, d, q);
         }
-    const float rstd = 1.f / sqrtf(warp_sum(q) / (float)S + r.eps);
+    const float rstd = 1.f / sqrtf(div_n(warp_sum(q), S) + r.eps);
     if (lane == 0) {
       r.cstats[2 * row] = cm;
       r.cstats[2 * row + 1] = rstd;
@@ -325,7 +332,7 @@ __global__ void k_qk_rope_warp(RopeArgs r) {
   for (int c0 = 0; c0 < HD; c0 += 128) {
     const int c = c0 + lane * 4;
     const bool in = c < HD;
-    const int d = c % D;
+    const int d = c & (D - 1);   // D is a power of two
     const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
     float4 xq = in ? ld4w(qv + c) : z4, xk = in ? ld4w(kv + c) : z4, co = z4, si = z4;
     if (in) {
@@ -345,7 +352,7 @@ __global__ void k_qk_rope_warp(RopeArgs r) {
       float4 x = w ? xk : xq;
       float ss = x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
       for (int o = 1; o < glanes; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      const float rstd = 1.f / sqrtf(ss / (float)D + r.eps);
+      const float rstd = 1.f / sqrtf(div_n(ss, D) + r.eps);
       x.x *= rstd; x.y *= rstd; x.z *= rstd; x.w *= rstd;
       float4 p;
       p.x = __shfl_xor_sync(0xffffffffu, x.x, po);
