@@ -107,14 +107,15 @@ __device__ __forceinline__ bool rows_vec_ok(const T *p, int64_t ld) {
 // ---- A producers of the row-block GEMM: what the CTA converts into its A operand.
 // Each has two ways of delivering eight consecutive k of one row:
 //   load8(r, k, v)        loads and converts at once, any shape or alignment;
-//   issue(r, k, w) and finish(w, r, k, v)
+//   row(r, rw), issue(r, k, w) and finish(rw, w, r, k, v)
 //                         the loads alone (no branch: the row and k are clamped into the
-//                         tensor, so every address is readable) and, later, the
-//                         conversion, with rows >= M and k >= K set to zero. The operand
-//                         loops keep kPipe chunks of these loads in flight. Usable when
-//                         vec_ok() (K a multiple of 8, rows 16-byte aligned); kPipe = 0
-//                         keeps a producer on load8 (its raw loads would not fit in
-//                         registers).
+//                         tensor, so every address is readable): the row's own values
+//                         (flag, statistics) once per row, the eight payload values per k
+//                         chunk; later the conversion, with rows >= M and k >= K set to
+//                         zero. The operand loops keep kPipe chunks of payload loads in
+//                         flight. Usable when vec_ok() (K a multiple of 8, rows 16-byte
+//                         aligned); kPipe = 0 keeps a producer on load8 (its raw loads
+//                         would not fit in registers).
 // ProdPlain: A itself. ProdNorm: a row normalisation fused into the operand,
 //   (x - mean) * rstd * scale + shift      (AF3 adaptive LN; the scale column already
 //                                           holds sigmoid(...))
@@ -132,11 +133,13 @@ struct ProdPlain {
     load8_t(A, lda, M, K, r, k, v);
   }
   struct Raw { Raw8<TA> a; };
+  struct RowRaw {};
   __device__ bool vec_ok() const { return M > 0 && K > 0 && (K & 7) == 0 && rows_vec_ok(A, lda); }
+  __device__ void row(int64_t, RowRaw &) const {}
   __device__ void issue(int64_t r, int64_t k, Raw &w) const {
     raw8_load(A + (r < M ? r : M - 1) * lda + (k < K ? k : K - 8), w.a);
   }
-  __device__ void finish(const Raw &w, int64_t r, int64_t k, float (&v)[8]) const {
+  __device__ void finish(const RowRaw &, const Raw &w, int64_t r, int64_t k, float (&v)[8]) const {
     float a[8];
     raw8_get(w.a, a);
     const bool in = r < M && k < K;
@@ -172,24 +175,27 @@ struct ProdNormT {
       v[e] = (row_in && k + e < K) ? fmaf((xv[e] - ms.x) * ms.y, s, sh[e]) : 0.f;
     }
   }
-  struct Raw { Raw8<IT> x, sc, sh; float2 ms; };
+  struct Raw { Raw8<IT> x, sc, sh; };
+  struct RowRaw { float2 ms; };
   __device__ bool vec_ok() const {
     return M > 0 && K > 0 && (K & 7) == 0 && rows_vec_ok(x, K) && rows_vec_ok(cond + sc_off, cond_ld) &&
            rows_vec_ok(cond + sh_off, cond_ld) && (reinterpret_cast<uintptr_t>(stats) & 7) == 0;
+  }
+  __device__ void row(int64_t r, RowRaw &rw) const {
+    rw.ms = *reinterpret_cast<const float2 *>(stats + 2 * (r < M ? r : M - 1));
   }
   __device__ void issue(int64_t r, int64_t k, Raw &w) const {
     const int64_t rc = r < M ? r : M - 1, kc = k < K ? k : K - 8;
     raw8_load(x + rc * K + kc, w.x);
     raw8_load(cond + sc_off + rc * cond_ld + kc, w.sc);
     raw8_load(cond + sh_off + rc * cond_ld + kc, w.sh);
-    w.ms = *reinterpret_cast<const float2 *>(stats + 2 * rc);
   }
-  __device__ void finish(const Raw &w, int64_t r, int64_t k, float (&v)[8]) const {
+  __device__ void finish(const RowRaw &rw, const Raw &w, int64_t r, int64_t k, float (&v)[8]) const {
     float xv[8], sc[8], sh[8];
     raw8_get(w.x, xv);
     raw8_get(w.sc, sc);
     raw8_get(w.sh, sh);
-    combine(xv, sc, sh, w.ms, r < M, k, v);
+    combine(xv, sc, sh, rw.ms, r < M, k, v);
   }
 };
 using ProdNorm = ProdNormT<float>;
@@ -202,7 +208,9 @@ using ProdNorm = ProdNormT<float>;
 template <typename T, int MODE>
 struct ProdCond {
   static constexpr bool kLight = false;
-  static constexpr int kEpiWarps = 4;   // SiLU / LayerNorm operands over K up to 256
+  // SiLU / LayerNorm operands over K up to 256: eight producer warps (four, even with
+  // two chunks of loads in flight, fell behind eight epilogue warps)
+  static constexpr int kEpiWarps = 4;
   const T *c;            // [M, K] condition rows
   const uint8_t *usable; // [M]
   const float *stats;    // [M, 2] (MODE 2)
@@ -226,22 +234,25 @@ struct ProdCond {
       v[e] = (use && k + e < K) ? y : 0.f;
     }
   }
-  struct Raw { Raw8<T> c; float2 ms; uint32_t use; };
+  struct Raw { Raw8<T> c; };
+  struct RowRaw { float2 ms; uint32_t use; };
   __device__ bool vec_ok() const {
     return M > 0 && K > 0 && (K & 7) == 0 && rows_vec_ok(c, K) &&
            (MODE != 2 || (reinterpret_cast<uintptr_t>(stats) & 7) == 0);
   }
-  __device__ void issue(int64_t r, int64_t k, Raw &w) const {
+  __device__ void row(int64_t r, RowRaw &rw) const {
     const int64_t rc = r < M ? r : M - 1;
-    raw8_load(c + rc * K + (k < K ? k : K - 8), w.c);
-    w.use = usable[rc];
-    w.ms = make_float2(0.f, 1.f);
-    if (MODE == 2) w.ms = *reinterpret_cast<const float2 *>(stats + 2 * rc);
+    rw.use = usable[rc];
+    rw.ms = make_float2(0.f, 1.f);
+    if (MODE == 2) rw.ms = *reinterpret_cast<const float2 *>(stats + 2 * rc);
   }
-  __device__ void finish(const Raw &w, int64_t r, int64_t k, float (&v)[8]) const {
+  __device__ void issue(int64_t r, int64_t k, Raw &w) const {
+    raw8_load(c + (r < M ? r : M - 1) * K + (k < K ? k : K - 8), w.c);
+  }
+  __device__ void finish(const RowRaw &rw, const Raw &w, int64_t r, int64_t k, float (&v)[8]) const {
     float cv[8];
     raw8_get(w.c, cv);
-    combine(cv, w.ms, r < M && w.use != 0, k, v);
+    combine(cv, rw.ms, r < M && rw.use != 0, k, v);
   }
 };
 
@@ -429,14 +440,19 @@ __device__ __forceinline__ void epi_chunk(const Epi &epi, float *T, const float 
   __syncwarp();   // T is free for the next chunk
 }
 
-template <bool SPLIT, int P, class Prod>
+template <bool SPLIT, int P, int HALVES, class Prod>
 __device__ __forceinline__ void form_rows_pipelined(const Prod &prod, uint8_t *aB, int64_t m0, int row_first,
-                                                    int halves, int nkc, int lane) {
+                                                    int nkc, int lane) {
   constexpr int PARTS = SPLIT ? 2 : 1;
   constexpr uint32_t BLK = kUmmaBlockBytes;
-  const int nst = halves * nkc, seg = lane & 7;
+  const int nst = HALVES * nkc, seg = lane & 7;
   auto row_of = [&](int st, int it) { return row_first + (st / nkc) * 16 + it * 4 + (lane >> 3); };
   auto k_of = [&](int st) { return (int64_t)(st % nkc) * kUmmaBK + seg * 8; };
+  typename Prod::RowRaw rw[HALVES][4];
+#pragma unroll
+  for (int h = 0; h < HALVES; ++h)
+#pragma unroll
+    for (int it = 0; it < 4; ++it) prod.row(m0 + row_first + h * 16 + it * 4 + (lane >> 3), rw[h][it]);
   typename Prod::Raw w[P][4];
 #pragma unroll
   for (int p = 0; p < P; ++p)
@@ -452,10 +468,13 @@ __device__ __forceinline__ void form_rows_pipelined(const Prod &prod, uint8_t *a
         uint8_t *a_c = aB + (size_t)(st % nkc) * PARTS * BLK;
         const int64_t k = k_of(st);
 #pragma unroll
+        const int h = st / nkc;
+#pragma unroll
         for (int it = 0; it < 4; ++it) {
           const int r = row_of(st, it);
           float v[8];
-          prod.finish(w[p][it], m0 + r, k, v);
+          // rw is indexed by the half through a select (HALVES <= 2), not a dynamic index
+          prod.finish(HALVES == 1 || h == 0 ? rw[0][it] : rw[HALVES - 1][it], w[p][it], m0 + r, k, v);
           if (st + P < nst) prod.issue(m0 + row_of(st + P, it), k_of(st + P), w[p][it]);
           uint32_t hi[4], lo[4];
           umma::split8<SPLIT>(v, hi, lo);
@@ -521,7 +540,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
     bool piped = false;
     if constexpr (Prod::kPipe > 0) {
       if (prod.vec_ok()) {
-        form_rows_pipelined<SPLIT, Prod::kPipe>(prod, sA, m0, warp * 16, 1, nkc, lane);
+        form_rows_pipelined<SPLIT, Prod::kPipe, 1>(prod, sA, m0, warp * 16, nkc, lane);
         piped = true;
       }
     }
@@ -764,7 +783,7 @@ __global__ void __launch_bounds__(kRowsPThreads, 1)
       uint8_t *aB = sA + (size_t)buf * nkc * BLK;
       if constexpr (Prod::kPipe > 0) {
         if (pipe_ok) {
-          form_rows_pipelined<false, Prod::kPipe>(prod, aB, m0, pw * RPW, RPW / 16, nkc, lane);
+          form_rows_pipelined<false, Prod::kPipe, RPW / 16>(prod, aB, m0, pw * RPW, nkc, lane);
           umma::fence_async_smem();
           __syncwarp();
           if (lane == 0) umma::mbar_arrive(afull + buf);

@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
     {
       const ProdPlain<TO> po{static_cast<const TO *>(t.O), (int64_t)t.HD, t.R, (int64_t)t.HD};
       if (po.vec_ok()) {
-        form_rows_pipelined<SPLIT, 1>(po, sA, m0, warp * 16, 1, nkc_out, lane);
+        form_rows_pipelined<SPLIT, 1, 1>(po, sA, m0, warp * 16, nkc_out, lane);
       } else {
         for (int kc = 0; kc < nkc_out; ++kc) {
           float v[4][8];
