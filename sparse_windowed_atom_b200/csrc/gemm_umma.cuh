@@ -378,6 +378,9 @@ __global__ void __launch_bounds__(kUmmaThreads)
 // Requires K <= kRowsKMax; every wait is bounded (status bit 4 on timeout).
 constexpr int kRowsEpiWarps = 8;                        // two per TMEM lane quadrant
 constexpr int kRowsTPitch = 32;                         // floats per row of a transpose tile
+// shared loads per batch in this kernel's epilogue chunks (its eight warps also form the
+// operand; measured: 2 beats 1 and 8 on the AF3 conditioning and float32 products)
+constexpr int kRowsEpiBatch = 2;
 constexpr int kRowsThreads = (kRowsEpiWarps + 2) * 32;  // + MMA issuer + weight loader
 constexpr int kRowsKMax = 256;
 constexpr int kRowsMaxSlots = 4;   // deeper rings were measured slower (every CTA fetches
@@ -408,10 +411,9 @@ __host__ __device__ inline int rows_slots(int64_t K, bool split, int blocks_per_
 // chunks) each cover all 32 banks once. The shared loads are issued in batches of
 // epi_batch<Epi> and a whole in-range chunk takes one bounds check, so the stores of a
 // batch do not wait on one another.
-template <class Epi>
+template <int NB, class Epi>
 __device__ __forceinline__ void epi_chunk(const Epi &epi, float *T, const float (&v)[32], int lane,
                                           int64_t row0, int64_t col0, int64_t M, int64_t N, bool ok) {
-  constexpr int NB = EpiBatch<Epi>::value;
 #pragma unroll
   for (int j = 0; j < 8; ++j)
     *reinterpret_cast<float4 *>(T + lane * kRowsTPitch + 4 * (j ^ (lane & 7))) =
@@ -595,7 +597,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         if (n0 + c0 >= N) break;
         float v[32];
         umma::tmem_ld32(tlane + buf * kUmmaBN + c0, v);
-        epi_chunk(epi, T, v, lane, m0 + qd * 32, n0 + c0, M, N, ok);
+        epi_chunk<kRowsEpiBatch>(epi, T, v, lane, m0 + qd * 32, n0 + c0, M, N, ok);
       }
       umma::tc_fence_before();
       __syncwarp();
@@ -758,7 +760,7 @@ __global__ void __launch_bounds__(kRowsPThreads, 1)
           if (n0 + c0 >= N) break;
           float v[32];
           umma::tmem_ld32(tlane + buf * kUmmaBN + c0, v);
-          epi_chunk(epi, T, v, lane, m0 + qd * 32, n0 + c0, M, N, ok);
+          epi_chunk<EpiBatch<Epi>::value>(epi, T, v, lane, m0 + qd * 32, n0 + c0, M, N, ok);
         }
         umma::tc_fence_before();
         __syncwarp();
