@@ -37,10 +37,6 @@ __device__ __forceinline__ float ldf(const __nv_bfloat16 *p, int64_t i) {
 }
 __device__ __forceinline__ void stf(float *p, int64_t i, float v) { p[i] = v; }
 // two floats rounded to nearest-even bf16 by one packed conversion; lo in bits 0-15
-// Shared-memory loads a row-block GEMM epilogue issues at once per batch (of the eight a
-// lane makes per 32 x 32 chunk); functors that hold many registers take fewer.
-template <class Epi> struct EpiBatch { static constexpr int value = 8; };
-
 __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
   uint32_t u;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(hi), "f"(lo));

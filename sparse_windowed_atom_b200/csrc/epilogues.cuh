@@ -168,9 +168,6 @@ struct EpiSplitT {
   }
 };
 using EpiSplit = EpiSplitT<float>;
-// four destination and four bias pointers stay live: half batches keep the epilogue
-// within the persistent kernel's 128 registers
-template <typename WT> struct EpiBatch<EpiSplitT<WT>> { static constexpr int value = 4; };
 
 // x' = x + g_attn * (o @ w_attention_out)  (bullet 16); x and the gates in the
 // intermediate type, x' in float32

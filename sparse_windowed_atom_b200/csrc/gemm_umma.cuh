@@ -378,8 +378,8 @@ __global__ void __launch_bounds__(kUmmaThreads)
 // Requires K <= kRowsKMax; every wait is bounded (status bit 4 on timeout).
 constexpr int kRowsEpiWarps = 8;                        // two per TMEM lane quadrant
 constexpr int kRowsTPitch = 32;                         // floats per row of a transpose tile
-// shared loads per batch in this kernel's epilogue chunks (its eight warps also form the
-// operand; measured: 2 beats 1 and 8 on the AF3 conditioning and float32 products)
+// shared loads per batch in the row-block GEMMs' epilogue chunks (measured: 2 beats 1, 4
+// and 8 in both the one-CTA-per-row-block and the persistent kernel)
 constexpr int kRowsEpiBatch = 2;
 constexpr int kRowsThreads = (kRowsEpiWarps + 2) * 32;  // + MMA issuer + weight loader
 constexpr int kRowsKMax = 256;
@@ -408,9 +408,8 @@ __host__ __device__ inline int rows_slots(int64_t K, bool split, int blocks_per_
 // (rr = lane / 8, q = lane % 8) hands columns col0 + 4q .. + 3 of rows row0 + rr, + 4, ...
 // to the epilogue functor. 16-byte chunk j of tile row r sits at chunk j ^ (r & 7), so the
 // eight lanes of a store phase (eight rows, one chunk) and of a load phase (one row, eight
-// chunks) each cover all 32 banks once. The shared loads are issued in batches of
-// epi_batch<Epi> and a whole in-range chunk takes one bounds check, so the stores of a
-// batch do not wait on one another.
+// chunks) each cover all 32 banks once. The shared loads are issued NB at a time and a
+// whole in-range chunk takes one bounds check.
 template <int NB, class Epi>
 __device__ __forceinline__ void epi_chunk(const Epi &epi, float *T, const float (&v)[32], int lane,
                                           int64_t row0, int64_t col0, int64_t M, int64_t N, bool ok) {
@@ -760,7 +759,7 @@ __global__ void __launch_bounds__(kRowsPThreads, 1)
           if (n0 + c0 >= N) break;
           float v[32];
           umma::tmem_ld32(tlane + buf * kUmmaBN + c0, v);
-          epi_chunk<EpiBatch<Epi>::value>(epi, T, v, lane, m0 + qd * 32, n0 + c0, M, N, ok);
+          epi_chunk<kRowsEpiBatch>(epi, T, v, lane, m0 + qd * 32, n0 + c0, M, N, ok);
         }
         umma::tc_fence_before();
         __syncwarp();
