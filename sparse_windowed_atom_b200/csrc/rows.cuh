@@ -124,7 +124,7 @@ __device__ __forceinline__ void st4(__nv_bfloat16 *p, float *v) {
 // results (the reset token ranges; the token projection in the decoder) are used after.
 // Grid: (ceil(A / 8), B), a warp per atom a of batch element b = blockIdx.y.
 template <typename T>
-__global__ void k_rows_prep_reg(RowsArgs r) {
+__global__ void __launch_bounds__(256, 8) k_rows_prep_reg(RowsArgs r) {
   pdl_launch_next();
   const int lane = threadIdx.x & 31;
   const int64_t b = blockIdx.y, a = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -319,7 +319,7 @@ __device__ __forceinline__ void st4w(__nv_bfloat16 *p, float4 v) {
 // attention reads bf16 rows); the arithmetic is float32. vec: cos/sin rows may be read
 // four values at a time.
 template <typename T, typename WT>
-__global__ void k_qk_rope_warp(RopeArgs r) {
+__global__ void __launch_bounds__(256, 8) k_qk_rope_warp(RopeArgs r) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
