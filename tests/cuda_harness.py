@@ -1,5 +1,7 @@
 """Helpers shared by the GPU parity tests: move a seeded workload to the device, run
 the CUDA library through its C ABI, run the oracle on the same values, compare."""
+import os
+
 import numpy as np
 import torch
 
@@ -54,6 +56,12 @@ def compare(got, ref, dtype, what=""):
         err = np.abs(g[m] - r[m])
         bound = tol * (1.0 + np.abs(r[m]))
         bad = err > bound
+        # ATOMENC_MARGIN_LOG=<file>: append the largest error and its share of the bound
+        log = os.environ.get("ATOMENC_MARGIN_LOG")
+        if log and err.size:
+            with open(log, "a") as f:
+                f.write(f"{what} {k} n={err.size} max_err={err.max():.3e} "
+                        f"max_err_over_bound={(err / bound).max():.4f}\n")
         if bad.any():
             i = np.argmax(err / bound)
             raise AssertionError(
