@@ -468,7 +468,6 @@ __device__ __forceinline__ void form_rows_pipelined(const Prod &prod, uint8_t *a
       if (st < nst) {
         uint8_t *a_c = aB + (size_t)(st % nkc) * PARTS * BLK;
         const int64_t k = k_of(st);
-#pragma unroll
         const int h = st / nkc;
 #pragma unroll
         for (int it = 0; it < 4; ++it) {

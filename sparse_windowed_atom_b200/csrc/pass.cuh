@@ -16,7 +16,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
                float eps, int64_t radius, const atomenc_outputs *out, unsigned char *ws,
                cudaStream_t st, Hooks &hk, int mode, unsigned char *image) {
   const Dims &d = pl.d;
-  const int64_t B = d.B, A = d.A, T = d.T, K = d.K, C = d.C, S = d.S, H = d.H, D = d.D,
+  const int64_t B = d.B, A = d.A, T = d.T, C = d.C, S = d.S, H = d.H, D = d.D,
                 P = d.P, M = d.M, U = d.U, V = d.V, HD = H * D, R = B * A;
   auto F = [&](size_t off) { return reinterpret_cast<float *>(ws + off); };
   // weight-region offsets resolve against the workspace, or against a prepared image
