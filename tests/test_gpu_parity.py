@@ -111,6 +111,33 @@ def test_blocked_windows_with_shared_rows(dtype, A, radius, valid_p):
 
 
 @pytest.mark.parametrize("style,stage", [("af3", "encoder"), ("esmfold2", "decoder")])
+@pytest.mark.parametrize("dtype", ["float32", "bfloat16"])
+@pytest.mark.parametrize("C,S", [(24, 40), (20, 36)])
+def test_operand_widths_off_the_vector_path(style, stage, dtype, C, S):
+    """Channel widths below one 64-wide k chunk: K a multiple of 8 takes the pipelined
+    operand loads with a partial chunk (k past K clamped and zeroed), K not a multiple of
+    8 the per-element loads; C != 128 also runs the tail unfused."""
+    spec = workloads.tiny_spec(style, stage, dtype, C=C, S=S, H=2, D=8, M=40, U=28, V=20)
+    _check(workloads.make_inputs(spec, seed=31), f"C={C} S={S}")
+
+
+@pytest.mark.parametrize("style,C,S", [("esmfold2", 24, 36), ("af3", 40, 24)])
+def test_persistent_products_with_odd_widths(style, C, S):
+    """448 row blocks of bf16 rows (every product on the persistent kernel, formed
+    operands included) with widths whose operands take the pipelined loads with a partial
+    k chunk and the per-element loads; a seeded sample of whole tokens checked against the
+    oracle."""
+    spec = workloads.tiny_spec(style, "encoder", "bfloat16", B=1, A=448 * 128, T=7000, K=24,
+                               C=C, S=S, H=2, D=8, M=40, U=28, keys=("random", 64),
+                               tokens=("ragged", 16), radius=-1)
+    w = workloads.make_inputs(spec, seed=37)
+    got = run_cuda(w)
+    ref = run_oracle(w, query_select=sample_queries(spec, w, frac=0.01))
+    compare(got, ref, spec.dtype, f"persistent {style} C={C} S={S}")
+    exact_zero_pattern(got, ref)
+
+
+@pytest.mark.parametrize("style,stage", [("af3", "encoder"), ("esmfold2", "decoder")])
 def test_unaligned_atom_and_condition_rows(style, stage):
     """atom and condition views that start one element into their storage (dense, but not
     16-byte aligned) take the general row-preparation kernel; same results."""
