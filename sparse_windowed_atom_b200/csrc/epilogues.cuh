@@ -33,10 +33,24 @@ __device__ __forceinline__ void st4i(__nv_bfloat16 *d, float4 o) {
   *reinterpret_cast<uint2 *>(d) = make_uint2(bf16x2_bits(o.x, o.y), bf16x2_bits(o.z, o.w));
 }
 
+// eight consecutive values in the intermediate type (two 16-byte float32 stores / one
+// 16-byte bf16 store); the caller checks 16-byte alignment
+__device__ __forceinline__ void st8i(float *d, const float (&v)[8]) {
+  *reinterpret_cast<float4 *>(d) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4 *>(d + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void st8i(__nv_bfloat16 *d, const float (&v)[8]) {
+  *reinterpret_cast<uint4 *>(d) = make_uint4(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3]),
+                                             bf16x2_bits(v[4], v[5]), bf16x2_bits(v[6], v[7]));
+}
+template <typename T>
+__device__ __forceinline__ bool aligned16(const T *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
 // Plain store of four consecutive columns (one 16-byte / 8-byte store when the row
-// stride and the column keep them aligned).
+// stride and the column keep them aligned); oct: eight columns, one 16-byte bf16 store.
 template <typename IT>
 struct QuadStore {
+  static constexpr bool kOct = true;   // takes eight columns per lane
   IT *out;
   int64_t ld;
   __device__ void quad(int64_t r, int64_t c0, const float (&v)[4], int64_t N) const {
@@ -48,11 +62,20 @@ struct QuadStore {
         if (c0 + j < N) stf(out, r * ld + c0 + j, v[j]);
     }
   }
+  __device__ void oct(int64_t r, int64_t c0, const float (&v)[8], int64_t N) const {
+    if (c0 + 8 <= N && ((ld | c0) & 7) == 0 && aligned16(out)) {
+      st8i(out + r * ld + c0, v);
+    } else {
+      quad(r, c0, {v[0], v[1], v[2], v[3]}, N);
+      if (c0 + 4 < N) quad(r, c0 + 4, {v[4], v[5], v[6], v[7]}, N);   // quads store unchecked
+    }
+  }
 };
 
 // ReLU(hidden @ w_pool) before the per-token mean (bullet 19), four columns at a time
 template <typename IT>
 struct QuadRelu {
+  static constexpr bool kOct = true;   // takes eight columns per lane
   IT *out;
   int64_t ld;
   __device__ void quad(int64_t r, int64_t c0, const float (&v)[4], int64_t N) const {
@@ -66,6 +89,17 @@ struct QuadRelu {
         if (c0 + j < N) stf(out, r * ld + c0 + j, w[j]);
     }
   }
+  __device__ void oct(int64_t r, int64_t c0, const float (&v)[8], int64_t N) const {
+    if (c0 + 8 <= N && ((ld | c0) & 7) == 0 && aligned16(out)) {
+      float o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = fmaxf(v[e], 0.f);
+      st8i(out + r * ld + c0, o);
+    } else {
+      quad(r, c0, {v[0], v[1], v[2], v[3]}, N);
+      if (c0 + 4 < N) quad(r, c0 + 4, {v[4], v[5], v[6], v[7]}, N);   // quads store unchecked
+    }
+  }
 };
 
 // AF3 conditioning: columns (scale_0, shift_0, scale_1, shift_1, scale_2, shift_2), C each;
@@ -73,6 +107,7 @@ struct QuadRelu {
 // Index math is done once per four columns, in 32 bits (C is a multiple of 4).
 template <typename IT>
 struct EpiCondAF3 {
+  static constexpr bool kOct = true;   // takes eight columns per lane
   IT *out;     // [M, 6C]
   const float *b_scale;  // [3, C]
   int64_t C;
@@ -101,11 +136,32 @@ struct EpiCondAF3 {
     }
     st4i(out + r * 6 * C + c0, o);
   }
+  // eight columns of one block when C is a multiple of 8 (one 16-byte bf16 store)
+  __device__ void oct(int64_t r, int64_t c0, const float (&v)[8], int64_t N) const {
+    const int c = (int)c0, Ci = (int)C;
+    if ((Ci & 7) == 0 && c0 + 8 <= N && aligned16(out)) {
+      const int blk = (c >= Ci) + (c >= 2 * Ci) + (c >= 3 * Ci) + (c >= 4 * Ci) + (c >= 5 * Ci);
+      const int ch = c - blk * Ci;
+      float o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = v[e];
+      if ((blk & 1) == 0) {
+        const float *bs = b_scale + (blk >> 1) * Ci + ch;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = sigmoid_fast(v[e] + bs[e]);
+      }
+      st8i(out + r * 6 * C + c0, o);
+    } else {
+      quad(r, c0, {v[0], v[1], v[2], v[3]}, N);
+      if (c0 + 4 < N) quad(r, c0 + 4, {v[4], v[5], v[6], v[7]}, N);   // quads store unchecked
+    }
+  }
 };
 
 // AF3 residual gates sigmoid(raw condition @ w_residual_gate[j] + b_residual_gate[j])  (bullet 9)
 template <typename IT>
 struct EpiGateAF3 {
+  static constexpr bool kOct = true;   // takes eight columns per lane
   IT *out;     // [M, 2C]
   const float *b_rg;  // [2, C]
   int64_t C;
@@ -120,6 +176,18 @@ struct EpiGateAF3 {
     st4i(out + r * 2 * C + c0,
          make_float4(sigmoid_fast(v[0] + b[0]), sigmoid_fast(v[1] + b[1]), sigmoid_fast(v[2] + b[2]),
                      sigmoid_fast(v[3] + b[3])));
+  }
+  __device__ void oct(int64_t r, int64_t c0, const float (&v)[8], int64_t N) const {
+    if ((C & 3) == 0 && c0 + 8 <= N && aligned16(out)) {
+      const float *b = b_rg + c0;
+      float o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = sigmoid_fast(v[e] + b[e]);
+      st8i(out + r * 2 * C + c0, o);
+    } else {
+      quad(r, c0, {v[0], v[1], v[2], v[3]}, N);
+      if (c0 + 4 < N) quad(r, c0 + 4, {v[4], v[5], v[6], v[7]}, N);   // quads store unchecked
+    }
   }
 };
 
@@ -136,6 +204,7 @@ __device__ __forceinline__ void st4w(__nv_bfloat16 *d, const float (&o)[4]) {
 // attention reads bf16 rows); only Q takes a bias (AF3 b_q, bullet 8)
 template <typename WT>
 struct EpiSplitT {
+  static constexpr bool kOct = true;   // takes eight columns per lane
   WT *dst[4];
   const float *bias[4];
   int64_t HD;
@@ -164,6 +233,22 @@ struct EpiSplitT {
         const float *b = bias_of(pe);
         stf(dst_of(pe), r * HD + he, b ? v[e] + b[he] : v[e]);
       }
+    }
+  }
+  // eight columns: one part when HD is a multiple of 8 (one 16-byte bf16 store)
+  __device__ void oct(int64_t r, int64_t c0, const float (&v)[8], int64_t N) const {
+    const int HDi = (int)HD, c = (int)c0;
+    const int part = (c >= HDi) + (c >= 2 * HDi) + (c >= 3 * HDi), ch = c - part * HDi;
+    WT *d = part == 0 ? dst[0] : part == 1 ? dst[1] : part == 2 ? dst[2] : dst[3];
+    const float *b = part == 0 ? bias[0] : part == 1 ? bias[1] : part == 2 ? bias[2] : bias[3];
+    if ((HDi & 7) == 0 && c0 + 8 <= N && aligned16(d)) {
+      float o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = b ? v[e] + b[ch + e] : v[e];
+      st8i(d + r * HD + ch, o);
+    } else {
+      quad(r, c0, {v[0], v[1], v[2], v[3]}, N);
+      if (c0 + 4 < N) quad(r, c0 + 4, {v[4], v[5], v[6], v[7]}, N);   // quads store unchecked
     }
   }
 };

@@ -17,6 +17,8 @@
 //    tcgen05.ld and hands four consecutive columns at a time to the epilogue functor.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "umma.cuh"
 
@@ -410,6 +412,13 @@ __host__ __device__ inline int rows_slots(int64_t K, bool split, int blocks_per_
 // eight lanes of a store phase (eight rows, one chunk) and of a load phase (one row, eight
 // chunks) each cover all 32 banks once. The shared loads are issued NB at a time and a
 // whole in-range chunk takes one bounds check.
+// Epilogue functors whose kOct is true (with an oct(row, col, v[8], N) member) take eight
+// consecutive columns per lane: one 16-byte store of bf16 (two of float32), eight rows
+// per store instruction instead of four; the others take quads.
+template <class E, class = void> struct EpiOct : std::false_type {};
+template <class E>
+struct EpiOct<E, std::void_t<decltype(E::kOct)>> : std::bool_constant<E::kOct> {};
+
 template <int NB, class Epi>
 __device__ __forceinline__ void epi_chunk(const Epi &epi, float *T, const float (&v)[32], int lane,
                                           int64_t row0, int64_t col0, int64_t M, int64_t N, bool ok) {
@@ -418,23 +427,53 @@ __device__ __forceinline__ void epi_chunk(const Epi &epi, float *T, const float 
     *reinterpret_cast<float4 *>(T + lane * kRowsTPitch + 4 * (j ^ (lane & 7))) =
         make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
   __syncwarp();
-  const int q = lane & 7, rr = lane >> 3;
-  const int64_t col = col0 + 4 * q;
   const bool whole = row0 + 32 <= M && col0 + 32 <= N;
+  if constexpr (EpiOct<Epi>::value) {
+    // lane (g = lane / 8, h = lane / 4 % 2, q = lane % 4) takes columns 8q .. 8q + 7 of row
+    // 8i + 2g + h: each store instruction covers eight rows, 64 contiguous bytes of bf16
+    // each; the eight lanes of a load phase read two rows of opposite parity, whose four
+    // chunks each land on distinct swizzled positions (all 32 banks once). An oct whose
+    // eight columns cannot go in one aligned store falls back to quads, the second only
+    // where it starts inside the row (quads store without a column check).
+    const int q = lane & 3, rr = 2 * (lane >> 3) + ((lane >> 2) & 1);
+    const int64_t col = col0 + 8 * q;
 #pragma unroll
-  for (int i0 = 0; i0 < 8; i0 += NB) {
-    float4 t[NB];
-#pragma unroll
-    for (int i = 0; i < NB; ++i) {
-      const int rl = (i0 + i) * 4 + rr;
-      t[i] = *reinterpret_cast<const float4 *>(T + rl * kRowsTPitch + 4 * (q ^ (rl & 7)));
-    }
-    if (ok) {
+    for (int i0 = 0; i0 < 4; i0 += NB) {
+      float4 t[NB][2];
 #pragma unroll
       for (int i = 0; i < NB; ++i) {
-        const int64_t row = row0 + (i0 + i) * 4 + rr;
-        const float x[4] = {t[i].x, t[i].y, t[i].z, t[i].w};
-        if (whole || (row < M && col < N)) epi.quad(row, col, x, N);
+        const int rl = (i0 + i) * 8 + rr;
+        t[i][0] = *reinterpret_cast<const float4 *>(T + rl * kRowsTPitch + 4 * ((2 * q) ^ (rl & 7)));
+        t[i][1] = *reinterpret_cast<const float4 *>(T + rl * kRowsTPitch + 4 * ((2 * q + 1) ^ (rl & 7)));
+      }
+      if (ok) {
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+          const int64_t row = row0 + (i0 + i) * 8 + rr;
+          const float x[8] = {t[i][0].x, t[i][0].y, t[i][0].z, t[i][0].w,
+                              t[i][1].x, t[i][1].y, t[i][1].z, t[i][1].w};
+          if (whole || (row < M && col < N)) epi.oct(row, col, x, N);
+        }
+      }
+    }
+  } else {
+    const int q = lane & 7, rr = lane >> 3;
+    const int64_t col = col0 + 4 * q;
+#pragma unroll
+    for (int i0 = 0; i0 < 8; i0 += NB) {
+      float4 t[NB];
+#pragma unroll
+      for (int i = 0; i < NB; ++i) {
+        const int rl = (i0 + i) * 4 + rr;
+        t[i] = *reinterpret_cast<const float4 *>(T + rl * kRowsTPitch + 4 * (q ^ (rl & 7)));
+      }
+      if (ok) {
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+          const int64_t row = row0 + (i0 + i) * 4 + rr;
+          const float x[4] = {t[i].x, t[i].y, t[i].z, t[i].w};
+          if (whole || (row < M && col < N)) epi.quad(row, col, x, N);
+        }
       }
     }
   }

@@ -112,11 +112,12 @@ def test_blocked_windows_with_shared_rows(dtype, A, radius, valid_p):
 
 @pytest.mark.parametrize("style,stage", [("af3", "encoder"), ("esmfold2", "decoder")])
 @pytest.mark.parametrize("dtype", ["float32", "bfloat16"])
-@pytest.mark.parametrize("C,S", [(24, 40), (20, 36)])
+@pytest.mark.parametrize("C,S", [(24, 40), (20, 36), (10, 8)])
 def test_operand_widths_off_the_vector_path(style, stage, dtype, C, S):
     """Channel widths below one 64-wide k chunk: K a multiple of 8 takes the pipelined
     operand loads with a partial chunk (k past K clamped and zeroed), K not a multiple of
-    8 the per-element loads; C != 128 also runs the tail unfused."""
+    8 the per-element loads; C != 128 also runs the tail unfused. C = 2 mod 4 puts the
+    last eight-column group of a 2C-wide gate row past the row's end."""
     spec = workloads.tiny_spec(style, stage, dtype, C=C, S=S, H=2, D=8, M=40, U=28, V=20)
     _check(workloads.make_inputs(spec, seed=31), f"C={C} S={S}")
 
