@@ -128,6 +128,24 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *p, int64_t 
   }
 }
 
+// eight consecutive values: one 16-byte store of bf16 (two of float32) where the address
+// allows it, else two four-value stores
+template <typename T>
+__device__ __forceinline__ void store8(T *p, int64_t i, const float (&v)[8]) {
+  if ((reinterpret_cast<uintptr_t>(p + i) & 15) == 0) {
+    if constexpr (sizeof(T) == 2) {
+      *reinterpret_cast<uint4 *>(p + i) = make_uint4(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3]),
+                                                     bf16x2_bits(v[4], v[5]), bf16x2_bits(v[6], v[7]));
+    } else {
+      *reinterpret_cast<float4 *>(p + i) = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4 *>(p + i + 4) = make_float4(v[4], v[5], v[6], v[7]);
+    }
+  } else {
+    store4<T>(p, i, make_float4(v[0], v[1], v[2], v[3]));
+    store4<T>(p, i + 4, make_float4(v[4], v[5], v[6], v[7]));
+  }
+}
+
 // the CTA pair's flags (global memory, GPU scope); the pair is launched as a 2-CTA
 // cluster, so both CTAs are resident together, and a poll still gives up after
 // peer_spin_limit reads (default kPeerSpinLimit; status bit 4), so a missing peer cannot
@@ -383,12 +401,11 @@ __global__ void __launch_bounds__(kTransThreads, 1) k_transition(TransArgs t) {
         }
         if (rok) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            float o[4];
+          for (int i = 0; i < 32; i += 8) {
+            float o[8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) o[e] = use ? fmaf(g1v[i + e], f[i + e], a[i + e]) : 0.f;
-            const float4 o4 = make_float4(o[0], o[1], o[2], o[3]);
-            store4<TOut>((TOut *)t.hidden, r * C + c0 + i, o4);
+            for (int e = 0; e < 8; ++e) o[e] = use ? fmaf(g1v[i + e], f[i + e], a[i + e]) : 0.f;
+            store8<TOut>((TOut *)t.hidden, r * C + c0 + i, o);
           }
         }
       }
