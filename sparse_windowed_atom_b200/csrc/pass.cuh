@@ -203,7 +203,7 @@ int launch_all(const Plan &pl, const atomenc_inputs *in, const atomenc_params *p
     PoolArgs pa{B, A, T, U, usable, static_cast<const int64_t *>(in->atom_to_token.data), first,
                 last, poolb, out->token_output.data};
     const int vec_out = (reinterpret_cast<uintptr_t>(out->token_output.data) & (4 * sizeof(Elt) - 1)) == 0;
-    const unsigned tok_blocks = (unsigned)((B * T + 7) / 8);
+    const dim3 tok_blocks((unsigned)((T + 7) / 8), (unsigned)B);   // k_token_mean_warp
     if (U % 4 == 0 && U <= 128)
       hk.launch(ATOMENC_KERNEL_POOL, (k_token_mean_warp<Elt, 1>), tok_blocks, 256, 0, st, pa, vec_out);
     else if (U % 4 == 0 && U <= 256)

@@ -482,13 +482,14 @@ __global__ void __launch_bounds__(kPoolThreads) k_token_mean(PoolArgs p) {
 // this token, one per lane for 32 rows, by ballot) select what is added, so the sums
 // are those of k_token_mean. vec_out: token_output rows may be written four values at
 // a time.
+// Grid: (ceil(T / 8), B), a warp per token t of batch element b = blockIdx.y.
 template <typename T, int NCH>
 __global__ void __launch_bounds__(256) k_token_mean_warp(PoolArgs p, int vec_out) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
-  const int64_t bt = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (bt >= p.B * p.T) return;
-  const int64_t b = bt / p.T, t = bt % p.T;
+  const int64_t b = blockIdx.y, t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= p.T) return;
+  const int64_t bt = b * p.T + t;
   const int first = p.tok_first[bt], last = p.tok_last[bt];
   const int U = (int)p.U;
   const T *base = static_cast<const T *>(p.pooled) + b * p.A * (int64_t)U;
