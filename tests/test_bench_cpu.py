@@ -37,9 +37,9 @@ def test_attention_bytes_match_the_tensors():
 
 
 def test_attention_bytes_of_the_headline_workload():
-    """The survey's per-launch figure for the ESMFold2 bf16 workload (B=2, A=32768, H=8,
-    K=128): 75.5 MB of key_index + window_mask, 134.2 MB of weights, 84.0 MB of Q/K/V/G/O
-    and usable flags."""
+    """The algorithmic bytes of one attention launch at the ESMFold2 bf16 workload (B=2,
+    A=32768, H=8, K=128), counted by hand: 75.5 MB of key_index + window_mask, 134.2 MB of
+    weights, 84.0 MB of Q/K/V/G/O and usable flags."""
     spec = workloads.WORKLOADS["esm_encoder_bf16_b2_a32768"]
     assert bench.attention_bytes(spec) == 75_497_472 + 134_217_728 + 83_951_616
 
